@@ -1,0 +1,131 @@
+"""Plain double-precision CPU oracle for the fused Gaussian kernel reductions.
+
+TEST INFRASTRUCTURE ONLY: the test-suite, the smoke check and the benchmark's
+CPU-baseline leg may import this package; the product library never does.
+It shares no code with the CUDA path.  The arithmetic lives in
+``gauss_oracle.c``; this module only loads it and marshals numpy arrays.
+
+Functions, each the plain definition ("Kernel matrix reduction", Implementation
+sketch, eq. 1 and eq. 2; "Fast Gauss Sums via Flash Attention", Algorithm 1,
+step 2):
+
+* ``gauss_sum(x, y, w, tau, rows=None)``  -> [B, R, C]
+* ``gauss_lse(x, y, w, tau, rows=None)``  -> [B, R, C]
+* ``gauss_sum_bwd(x, y, w, g, tau, rows=None, wrows=None)`` -> (grad_x, grad_w)
+
+Inputs are float64 arrays x [B,M,D], y [B,N,D], w [B,N,C], g [B,M,C] (2-D
+arrays are read as B = 1).  Values must already be the quantised values the
+device sees (fp16/bf16/fp32 widened to double).
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from .build import LIB, build_oracle
+
+_lib = None
+_i64 = ctypes.c_int64
+_dp = ctypes.POINTER(ctypes.c_double)
+_ip = ctypes.POINTER(ctypes.c_int64)
+
+
+def _load(path=None):
+    global _lib
+    if path is not None:
+        lib = ctypes.CDLL(path)
+    else:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build_oracle())
+    for name in ("oracle_gauss_sum", "oracle_gauss_lse"):
+        f = getattr(lib, name)
+        f.restype = ctypes.c_int
+        f.argtypes = [_dp, _dp, _dp, _dp, _i64, _i64, _i64, _i64, _i64,
+                      ctypes.c_double, _ip, _i64]
+    f = lib.oracle_gauss_sum_bwd
+    f.restype = ctypes.c_int
+    f.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _i64, _i64, _i64, _i64, _i64,
+                  ctypes.c_double, _ip, _i64, _ip, _i64]
+    lib.oracle_num_threads.restype = ctypes.c_int
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def num_threads():
+    """Threads the oracle's OpenMP loops use."""
+    return int(_load().oracle_num_threads())
+
+
+def _as3(a, name):
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+    if a.ndim == 2:
+        a = a[None]
+    if a.ndim != 3:
+        raise ValueError(f"{name}: expected a 2-D or 3-D array, got shape {a.shape}")
+    return a
+
+
+def _ptr(a):
+    return a.ctypes.data_as(_dp) if a is not None else None
+
+
+def _rows(rows):
+    if rows is None:
+        return None, 0, None
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    return r, int(r.size), r.ctypes.data_as(_ip)
+
+
+def _check(x, y, w):
+    B, M, D = x.shape
+    if y.shape[0] != B or y.shape[2] != D or w.shape[0] != B or w.shape[1] != y.shape[1]:
+        raise ValueError(f"shape mismatch x{x.shape} y{y.shape} w{w.shape}")
+    return B, M, y.shape[1], D, w.shape[2]
+
+
+def _reduce(fn_name, x, y, w, tau, rows, lib):
+    x, y, w = _as3(x, "x"), _as3(y, "y"), _as3(w, "w")
+    B, M, N, D, C = _check(x, y, w)
+    r, nr, rp = _rows(rows)
+    R = nr if r is not None else M
+    out = np.empty((B, R, C), dtype=np.float64)
+    rc = getattr(lib or _load(), fn_name)(_ptr(x), _ptr(y), _ptr(w), _ptr(out), B, M, N, D, C,
+                                          float(tau), rp, nr)
+    if rc != 0:
+        raise ValueError(f"{fn_name} rejected its arguments (code {rc})")
+    return out
+
+
+def gauss_sum(x, y, w, tau, rows=None, lib=None):
+    """out[b,i,c] = sum_j exp(-tau/2 |x_i - y_j|^2) w[b,j,c]."""
+    return _reduce("oracle_gauss_sum", x, y, w, tau, rows, lib)
+
+
+def gauss_lse(x, y, w, tau, rows=None, lib=None):
+    """out[b,i,c] = log sum_j w[b,j,c] exp(-tau/2 |x_i - y_j|^2), max-shifted."""
+    return _reduce("oracle_gauss_lse", x, y, w, tau, rows, lib)
+
+
+def gauss_sum_bwd(x, y, w, g, tau, rows=None, wrows=None, want_x=True, want_w=True, lib=None):
+    """Gradients of sum(g * gauss_sum(x, y, w)) with respect to x and w."""
+    x, y, w, g = _as3(x, "x"), _as3(y, "y"), _as3(w, "w"), _as3(g, "g")
+    B, M, N, D, C = _check(x, y, w)
+    if g.shape != (B, M, C):
+        raise ValueError(f"g must be {(B, M, C)}, got {g.shape}")
+    r, nr, rp = _rows(rows)
+    rw, nrw, rwp = _rows(wrows)
+    R = nr if r is not None else M
+    Rw = nrw if rw is not None else N
+    gx = np.empty((B, R, D), dtype=np.float64) if want_x else None
+    gw = np.empty((B, Rw, C), dtype=np.float64) if want_w else None
+    rc = (lib or _load()).oracle_gauss_sum_bwd(_ptr(x), _ptr(y), _ptr(w), _ptr(g), _ptr(gx),
+                                              _ptr(gw), B, M, N, D, C, float(tau), rp, nr,
+                                              rwp, nrw)
+    if rc != 0:
+        raise ValueError(f"oracle_gauss_sum_bwd rejected its arguments (code {rc})")
+    return gx, gw
+
+
+__all__ = ["gauss_sum", "gauss_lse", "gauss_sum_bwd", "num_threads", "build_oracle", "LIB"]

@@ -1,0 +1,286 @@
+/*
+ * gauss_oracle.c -- plain, slow, double-precision CPU oracle for the fused
+ * Gaussian kernel reductions.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file: only the test-suite, the smoke check and the CPU-baseline
+ * leg of the benchmark use it.  It shares no source, header, table or helper
+ * with the CUDA library; the two meet only through the seeded input arrays.
+ *
+ * What it computes is the plain definition, written as the double loop that
+ * defines a reduction over the column index j ("Kernel matrix reduction",
+ * Implementation sketch, eq. 2: row i reduces the formula over every column j)
+ * applied to the Gaussian kernel of the same page's eq. 1 sketch:
+ *
+ *   sum : out[b,i,c] = sum_j exp(-tau/2 * |x[b,i,:] - y[b,j,:]|^2) * w[b,j,c]
+ *   lse : out[b,i,c] = log sum_j w[b,j,c] * exp(-tau/2 * |x_i - y_j|^2)
+ *   bwd : the gradient of L = sum_{i,c} g[b,i,c] * sum_out[b,i,c] with respect
+ *         to x and to w (the weights are called b on the pages; here w, so as
+ *         not to clash with the batch index b).
+ *
+ * tau is the bandwidth parameter of "Fast Gauss Sums via Flash Attention",
+ * Algorithm 1 (input tau > 0); the same kernel is exp(-d^2 / (2 sigma^2)) with
+ * tau = 1/sigma^2 in the eq. 1 sketch of "Kernel matrix reduction".
+ *
+ * Every inner sum over j (or over i, for the weight gradient) is carried out
+ * with Neumaier's compensated summation in double, so the oracle's own error
+ * stays far below the 1e-5 relative bar it is used to check.  The squared
+ * distance is formed in the direct difference form sum_k (x_k - y_k)^2, never
+ * through the expanded |x|^2 + |y|^2 - 2 x.y.
+ *
+ * All arrays are row-major and contiguous:
+ *   x [B, M, D], y [B, N, D], w [B, N, C], g [B, M, C],
+ *   out [B, R, C] where R = M, or R = n_rows when a row subset is given.
+ * rows (optional, may be NULL): indices of the rows i to evaluate, the same
+ * subset in every batch.  Rows are evaluated independently in parallel
+ * (OpenMP); the arithmetic of one row never depends on the thread count.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Neumaier's improvement of Kahan summation: s carries the sum, c the
+ * running compensation; the value is s + c. */
+typedef struct {
+    double s;
+    double c;
+} comp_sum;
+
+static void cs_add(comp_sum *a, double v)
+{
+    double t = a->s + v;
+    if (fabs(a->s) >= fabs(v))
+        a->c += (a->s - t) + v;
+    else
+        a->c += (v - t) + a->s;
+    a->s = t;
+}
+
+static double cs_value(const comp_sum *a) { return a->s + a->c; }
+
+/* |p - q|^2 over D coordinates, direct difference form. */
+static double sq_dist(const double *p, const double *q, int64_t D)
+{
+    double acc = 0.0;
+    for (int64_t k = 0; k < D; ++k) {
+        double d = p[k] - q[k];
+        acc += d * d;
+    }
+    return acc;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Gaussian kernel sum ("Kernel matrix reduction", eq. 1 sketch; output s_m of
+ * "Fast Gauss Sums via Flash Attention", Algorithm 1, step 2). */
+int oracle_gauss_sum(const double *x, const double *y, const double *w,
+                     double *out, int64_t B, int64_t M, int64_t N, int64_t D,
+                     int64_t C, double tau, const int64_t *rows,
+                     int64_t n_rows)
+{
+    int64_t R = rows ? n_rows : M;
+    if (B < 0 || M < 0 || N < 0 || D < 1 || C < 1 || R < 0 || !(tau > 0.0))
+        return 1;
+    int bad = 0;
+#pragma omp parallel
+    {
+        comp_sum *acc = (comp_sum *)malloc((size_t)C * sizeof(comp_sum));
+        if (!acc) {
+#pragma omp atomic write
+            bad = 1;
+        }
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t t = 0; t < B * R; ++t) {
+            if (!acc)
+                continue;
+            int64_t bb = t / R;
+            int64_t r = t % R;
+            int64_t i = rows ? rows[r] : r;
+            const double *xi = x + (bb * M + i) * D;
+            for (int64_t c = 0; c < C; ++c) {
+                acc[c].s = 0.0;
+                acc[c].c = 0.0;
+            }
+            for (int64_t j = 0; j < N; ++j) {
+                const double *yj = y + (bb * N + j) * D;
+                double k = exp(-0.5 * tau * sq_dist(xi, yj, D));
+                const double *wj = w + (bb * N + j) * C;
+                for (int64_t c = 0; c < C; ++c)
+                    cs_add(&acc[c], k * wj[c]);
+            }
+            for (int64_t c = 0; c < C; ++c)
+                out[(bb * R + r) * C + c] = cs_value(&acc[c]);
+        }
+        free(acc);
+    }
+    return bad ? 2 : 0;
+}
+
+/* Log-sum-exp reduction ("Kernel matrix reduction", Overview: the reductions
+ * covered include log-sum-exp; the .logsumexp() reduction of the LazyTensor
+ * API).  The weights enter as log w, so the result is the logarithm of the
+ * Gauss sum: out = log sum_j w_j exp(F_ij), F_ij = -tau/2 |x_i - y_j|^2.
+ * It is evaluated in two passes, m = max_j F_ij first and then
+ * m + log sum_j w_j exp(F_ij - m), so that rows whose every kernel value
+ * underflows a double still get their finite logarithm.  N == 0 gives -inf;
+ * a non-positive weight sum gives what log gives (-inf or NaN). */
+int oracle_gauss_lse(const double *x, const double *y, const double *w,
+                     double *out, int64_t B, int64_t M, int64_t N, int64_t D,
+                     int64_t C, double tau, const int64_t *rows,
+                     int64_t n_rows)
+{
+    int64_t R = rows ? n_rows : M;
+    if (B < 0 || M < 0 || N < 0 || D < 1 || C < 1 || R < 0 || !(tau > 0.0))
+        return 1;
+    int bad = 0;
+#pragma omp parallel
+    {
+        comp_sum *acc = (comp_sum *)malloc((size_t)C * sizeof(comp_sum));
+        if (!acc) {
+#pragma omp atomic write
+            bad = 1;
+        }
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t t = 0; t < B * R; ++t) {
+            if (!acc)
+                continue;
+            int64_t bb = t / R;
+            int64_t r = t % R;
+            int64_t i = rows ? rows[r] : r;
+            const double *xi = x + (bb * M + i) * D;
+            if (N == 0) {
+                for (int64_t c = 0; c < C; ++c)
+                    out[(bb * R + r) * C + c] = -INFINITY;
+                continue;
+            }
+            double m = -INFINITY;
+            for (int64_t j = 0; j < N; ++j) {
+                double f = -0.5 * tau * sq_dist(xi, y + (bb * N + j) * D, D);
+                if (f > m)
+                    m = f;
+            }
+            for (int64_t c = 0; c < C; ++c) {
+                acc[c].s = 0.0;
+                acc[c].c = 0.0;
+            }
+            for (int64_t j = 0; j < N; ++j) {
+                double f = -0.5 * tau * sq_dist(xi, y + (bb * N + j) * D, D);
+                double e = exp(f - m);
+                const double *wj = w + (bb * N + j) * C;
+                for (int64_t c = 0; c < C; ++c)
+                    cs_add(&acc[c], wj[c] * e);
+            }
+            for (int64_t c = 0; c < C; ++c)
+                out[(bb * R + r) * C + c] = m + log(cs_value(&acc[c]));
+        }
+        free(acc);
+    }
+    return bad ? 2 : 0;
+}
+
+/* Gradient of L = sum_{i,c} g[i,c] * s[i,c] with s the Gauss sum ("Kernel
+ * matrix reduction", Variants: gradients through the same reduction; the
+ * torch.autograd.grad example of the LazyTensor API).  Differentiating
+ * exp(-tau/2 |x_i - y_j|^2) w_j by hand:
+ *
+ *   dL/dw[j,c] = sum_i K_ij g[i,c]
+ *   dL/dx[i,k] = -tau * sum_j K_ij (sum_c g[i,c] w[j,c]) (x[i,k] - y[j,k])
+ *
+ * grad_x is [B, R, D] (R = M or n_rows, rows as for the forward); grad_w is
+ * [B, Rw, C] over the weight rows wrows (NULL = all N).  Either output may be
+ * NULL to skip it. */
+int oracle_gauss_sum_bwd(const double *x, const double *y, const double *w,
+                         const double *g, double *grad_x, double *grad_w,
+                         int64_t B, int64_t M, int64_t N, int64_t D, int64_t C,
+                         double tau, const int64_t *rows, int64_t n_rows,
+                         const int64_t *wrows, int64_t n_wrows)
+{
+    int64_t R = rows ? n_rows : M;
+    int64_t Rw = wrows ? n_wrows : N;
+    if (B < 0 || M < 0 || N < 0 || D < 1 || C < 1 || R < 0 || Rw < 0 ||
+        !(tau > 0.0))
+        return 1;
+    int bad = 0;
+    if (grad_x) {
+#pragma omp parallel
+        {
+            comp_sum *acc = (comp_sum *)malloc((size_t)D * sizeof(comp_sum));
+            if (!acc) {
+#pragma omp atomic write
+                bad = 1;
+            }
+#pragma omp for schedule(dynamic, 4)
+            for (int64_t t = 0; t < B * R; ++t) {
+                if (!acc)
+                    continue;
+                int64_t bb = t / R;
+                int64_t r = t % R;
+                int64_t i = rows ? rows[r] : r;
+                const double *xi = x + (bb * M + i) * D;
+                const double *gi = g + (bb * M + i) * C;
+                for (int64_t k = 0; k < D; ++k) {
+                    acc[k].s = 0.0;
+                    acc[k].c = 0.0;
+                }
+                for (int64_t j = 0; j < N; ++j) {
+                    const double *yj = y + (bb * N + j) * D;
+                    const double *wj = w + (bb * N + j) * C;
+                    double kv = exp(-0.5 * tau * sq_dist(xi, yj, D));
+                    double gw = 0.0;
+                    for (int64_t c = 0; c < C; ++c)
+                        gw += gi[c] * wj[c];
+                    for (int64_t k = 0; k < D; ++k)
+                        cs_add(&acc[k], kv * gw * (xi[k] - yj[k]));
+                }
+                for (int64_t k = 0; k < D; ++k)
+                    grad_x[(bb * R + r) * D + k] = -tau * cs_value(&acc[k]);
+            }
+            free(acc);
+        }
+    }
+    if (grad_w) {
+#pragma omp parallel
+        {
+            comp_sum *acc = (comp_sum *)malloc((size_t)C * sizeof(comp_sum));
+            if (!acc) {
+#pragma omp atomic write
+                bad = 1;
+            }
+#pragma omp for schedule(dynamic, 4)
+            for (int64_t t = 0; t < B * Rw; ++t) {
+                if (!acc)
+                    continue;
+                int64_t bb = t / Rw;
+                int64_t r = t % Rw;
+                int64_t j = wrows ? wrows[r] : r;
+                const double *yj = y + (bb * N + j) * D;
+                for (int64_t c = 0; c < C; ++c) {
+                    acc[c].s = 0.0;
+                    acc[c].c = 0.0;
+                }
+                for (int64_t i = 0; i < M; ++i) {
+                    const double *xi = x + (bb * M + i) * D;
+                    const double *gi = g + (bb * M + i) * C;
+                    double kv = exp(-0.5 * tau * sq_dist(xi, yj, D));
+                    for (int64_t c = 0; c < C; ++c)
+                        cs_add(&acc[c], kv * gi[c]);
+                }
+                for (int64_t c = 0; c < C; ++c)
+                    grad_w[(bb * Rw + r) * C + c] = cs_value(&acc[c]);
+            }
+            free(acc);
+        }
+    }
+    return bad ? 2 : 0;
+}

@@ -1,0 +1,21 @@
+"""The oracle against facts fixed outside itself (closed forms, library
+routines, the flash-attention identities, invariants, finite differences)."""
+import pytest
+
+import oracle
+from pins import ALL_PINS
+
+
+class _Real:
+    gauss_sum = staticmethod(oracle.gauss_sum)
+    gauss_lse = staticmethod(oracle.gauss_lse)
+    gauss_sum_bwd = staticmethod(oracle.gauss_sum_bwd)
+
+
+@pytest.mark.parametrize("pin", ALL_PINS, ids=[p.__name__ for p in ALL_PINS])
+def test_pin(pin):
+    pin(_Real)
+
+
+def test_thread_count_is_reported():
+    assert oracle.num_threads() >= 1
