@@ -1,0 +1,373 @@
+"""Benchmark: Gaussian kernel-sum throughput (G pairs/s) on B200, with the
+roofline fraction of the dominant kernel and the CPU oracle as the baseline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one pass of the whole hot path of the workload over its seeded
+synthetic inputs (already resident in HBM).  Default workload: ``d3_100k``
+(B=1, M=N=100,000, D=3, C=1, fp32, tau=1, x,y ~ N(0,1)^3, w ~ N(0,1) signed),
+the Gaussian product at 100k points of "Kernel matrix reduction" (Variants).
+Under torchrun (N > 1) every rank runs its own independent problem of that
+size (rank-specific query points, same sources): rows are independent, so
+there is no data-path collective, and throughput scales weakly; the time is
+the maximum over ranks.
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on
+the launching stream, with a 256 MiB write between steps to flush the 126 MB L2
+(the inputs are smaller than L2); barrier + synchronize around the timed loop.
+SM clocks and throttle reasons are sampled with nvidia-smi during the loop.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+# MUFU ex2 throughput: 16 results / clock / SM (4 per SM sub-partition); every
+# pair of the small-D and tensor-core paths costs exactly one ex2 on the MUFU
+# pipe, so the ALU roofline in pairs/s is 16 * SMs * clock.
+EX2_PER_CLK_PER_SM = 16
+PUBLISHED = {  # context only: the pages' number for the same workload, another GPU
+    "d3_100k": {"value": 1e10 / 15.0e-3 / 1e9,
+                "source": "KeOps Gaussian product, 100k points, 15.0 ms on an RTX 2080 Ti"},
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="d3_100k", choices=sorted(synth.BY_NAME))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-launch-count", action="store_true",
+                    help="skip the profiler-based kernel count (use under ncu)")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_init(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local, pg
+
+
+def barrier(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+def max_over_ranks(value, pg, device):
+    if pg is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index, path):
+        self.index, self.path, self.proc = index, path, None
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", "--query-gpu=" + self.QUERY,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if getattr(self, "f", None):
+            self.f.close()
+
+    def summary(self):
+        try:
+            rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.strip()]
+        except OSError:
+            rows = []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons = [], None, set()
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workloads
+def step_fn(gs, w, d, ws, outs):
+    """Return a closure running one pass of the workload's hot path."""
+    tau = d["tau"]
+    ops = w.ops
+
+    def run():
+        if "sum" in ops:
+            gs.gauss_sum_fwd(d["x"], d["y"], d["w"], tau, out=outs["sum"], workspace=ws)
+        if "lse" in ops:
+            gs.gauss_lse_fwd(d["x"], d["y"], d["w"], tau, out=outs["lse"], workspace=ws)
+        if "bwd" in ops:
+            gs.gauss_sum_bwd(d["x"], d["y"], d["w"], d["g"], tau, workspace=ws)
+    return run
+
+
+def pair_evals(w):
+    """Kernel evaluations (pairs) one step performs: B*M*N per op, two passes for bwd."""
+    per = w.pairs
+    return per * (("sum" in w.ops) + ("lse" in w.ops) + 2 * ("bwd" in w.ops))
+
+
+def launches_per_step(gs, run):
+    """Kernels one step launches, counted by the CUDA profiler (names prove they are ours)."""
+    from torch.profiler import ProfilerActivity, profile
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        run()
+        torch.cuda.synchronize()
+    names = [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA
+             and ("gs::" in e.name or "gauss" in e.name or "kernel" in e.name)]
+    return len(names), sorted(set(names))
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+def oracle_sample(w, inp, seconds, seed=1234):
+    """Time the oracle as it stands on a bounded row sample of the workload."""
+    import oracle
+    import numpy as np
+    x, y, wt = (synth.as_f64(inp[k]) for k in ("x", "y", "w"))
+    g = synth.as_f64(inp["g"]) if "g" in inp else None
+
+    def run(rows):
+        t0 = time.perf_counter()
+        if "sum" in w.ops:
+            oracle.gauss_sum(x, y, wt, w.tau, rows=rows)
+        if "lse" in w.ops:
+            oracle.gauss_lse(x, y, wt, w.tau, rows=rows)
+        if "bwd" in w.ops:
+            oracle.gauss_sum_bwd(x, y, wt, g, w.tau, rows=rows, wrows=rows % w.N)
+        return time.perf_counter() - t0
+
+    probe = synth.sample_rows(w.M, 16, seed).numpy()
+    t = max(run(probe), 1e-3)
+    n = int(min(w.M, max(16, 16 * seconds / t)))
+    rows = synth.sample_rows(w.M, n, seed).numpy()
+    dt = run(rows)
+    pairs = w.B * n * w.N * (("sum" in w.ops) + ("lse" in w.ops) + 2 * ("bwd" in w.ops))
+    return {"value": pairs / dt / 1e9, "unit": "G pairs/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "seconds": round(dt, 3),
+            "sample": f"{n} of {w.M} query rows x all {w.N} sources, B={w.B}, same seeded inputs"}, rows
+
+
+def reference_arm(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = synth.make_inputs(w)
+    per_step = args.cpu_seconds / max(args.steps, 1)
+    import oracle
+    base, rows = oracle_sample(w, inp, max(per_step, 0.5))
+    x, y, wt = (synth.as_f64(inp[k]) for k in ("x", "y", "w"))
+    g = synth.as_f64(inp["g"]) if "g" in inp else None
+
+    def step():
+        if "sum" in w.ops:
+            oracle.gauss_sum(x, y, wt, w.tau, rows=rows)
+        if "lse" in w.ops:
+            oracle.gauss_lse(x, y, wt, w.tau, rows=rows)
+        if "bwd" in w.ops:
+            oracle.gauss_sum_bwd(x, y, wt, g, w.tau, rows=rows, wrows=rows % w.N)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    pairs = w.B * len(rows) * w.N * (("sum" in w.ops) + ("lse" in w.ops) + 2 * ("bwd" in w.ops))
+    value = pairs / dt / 1e9
+    line = {"impl": "reference", "metric": "Gaussian kernel-sum pairs/sec (G pairs/s)",
+            "value": value, "unit": "G pairs/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "M": w.M, "N": w.N, "D": w.D, "C": w.C,
+                       "tau": w.tau, "ops": list(w.ops)},
+            "cpu_baseline": {"kind": "oracle", "cores": base["cores"], "value": value,
+                             "unit": "G pairs/s", "sample": base["sample"] + " per step"},
+            "e2e": {"value": value, "unit": "G pairs/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+def main():
+    args = parse()
+    w = synth.BY_NAME[args.workload]
+    if args.impl == "reference":
+        return reference_arm(args, w)
+    rank, world, local, pg = dist_init(args.gpus)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    import pairwise_reductions_b200 as gs
+    dev = torch.device("cuda", local)
+    inp = synth.make_inputs(w, seed=(1000 + w.wid + 7919 * rank) if rank else None)
+    d = {k: inp[k].to(dev) for k in ("x", "y", "w", "g") if k in inp}
+    d["tau"] = inp["tau"]
+    outs = {"sum": torch.empty(w.B, w.M, w.C, device=dev), "lse": torch.empty(w.B, w.M, w.C, device=dev)}
+    ws_bytes = max(gs.workspace_bytes(op, w.B, w.M, w.N, w.D, w.C, d["x"].dtype)
+                   for op, name in ((gs.GS_OP_SUM, "sum"), (gs.GS_OP_LSE, "lse"), (gs.GS_OP_SUM_BWD, "bwd"))
+                   if name in w.ops)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    run = step_fn(gs, w, d, ws, outs)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(max(args.warmup, 3)):
+        run()
+    torch.cuda.synchronize()
+    n_launch, kernel_names = (None, []) if args.no_launch_count else launches_per_step(gs, run)
+    if gs.last_device_error() != 0:
+        raise SystemExit("device error word set during warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clk = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
+                       if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/gs_clocks_{rank}.csv")
+    barrier(pg)
+    torch.cuda.synchronize()
+    with clk:
+        time.sleep(0.3)
+        for k in range(args.steps):
+            flush.fill_(float(k))
+            starts[k].record(stream)
+            run()
+            ends[k].record(stream)
+        torch.cuda.synchronize()
+        time.sleep(0.2)
+    barrier(pg)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(step_ms), pg, dev)
+    ms_per_step = total_ms / args.steps
+    evals = pair_evals(w)
+    value = evals * world * args.steps / (total_ms * 1e-3) / 1e9
+    if gs.last_device_error() != 0:
+        raise SystemExit("device error word set during the timed loop")
+
+    # ---- end to end through the public API: pinned host inputs -> device -> result -> host
+    hx = {k: inp[k].pin_memory() for k in ("x", "y", "w", "g") if k in inp}
+    hout = torch.empty(w.B, w.M, w.C).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in hx.values())
+    d2h = hout.numel() * hout.element_size()
+    e_s = torch.cuda.Event(enable_timing=True)
+    e_e = torch.cuda.Event(enable_timing=True)
+
+    def e2e_step():
+        dd = {k: t.to(dev, non_blocking=True) for k, t in hx.items()}
+        dd["tau"] = inp["tau"]
+        step_fn(gs, w, dd, ws, outs)()
+        hout.copy_(outs["lse" if "lse" in w.ops and "sum" not in w.ops else "sum"], non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(pg)
+    e_s.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e_e.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e_s.elapsed_time(e_e), pg, dev) / args.e2e_steps
+    e2e_value = evals * world / (e2e_ms * 1e-3) / 1e9
+    clocks = clk.summary()
+
+    if rank == 0:
+        props = torch.cuda.get_device_properties(dev)
+        sms = props.multi_processor_count
+        peaks = {}
+        try:
+            peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        except (OSError, ValueError):
+            pass
+        sm_max = float(clocks.get("sm_max_mhz") or peaks.get("sm_max_mhz") or 1965.0)
+        peak = EX2_PER_CLK_PER_SM * sms * sm_max * 1e6 / 1e9
+        achieved = evals / (ms_per_step * 1e-3) / 1e9
+        roof = {"bound": "alu", "kernel": "MUFU ex2 (one per pair)", "achieved": achieved,
+                "peak": peak, "unit": "G pairs/s", "frac": achieved / peak, "traffic": None,
+                "peak_basis": f"16 ex2/clk/SM x {sms} SMs x {sm_max:.0f} MHz (max SM clock)"}
+        if clocks.get("sm_mhz"):
+            roof["frac_at_measured_clock"] = achieved / (EX2_PER_CLK_PER_SM * sms * clocks["sm_mhz"] * 1e-3)
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu, _ = oracle_sample(w, inp, args.cpu_seconds)
+        pub = PUBLISHED.get(w.name)
+        line = {"metric": "Gaussian kernel-sum pairs/sec (G pairs/s)", "value": value,
+                "unit": "G pairs/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": (value / pub["value"]) if pub else None,
+                "dtype": w.dtype, "data": "synthetic",
+                "config": {"workload": w.name, "B": w.B, "M": w.M, "N": w.N, "D": w.D, "C": w.C,
+                           "tau": w.tau, "ops": list(w.ops), "pairs_per_step_per_gpu": evals,
+                           "l2": "flushed by a 256 MiB write between timed steps",
+                           "parallelism": f"independent problems, {world} rank(s)"},
+                "roofline": roof, "cpu_baseline": cpu,
+                "e2e": {"value": e2e_value, "unit": "G pairs/s", "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "gpu_launches": (n_launch * args.steps) if n_launch is not None else None, "kernels": kernel_names,
+                "clocks": clocks}
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,141 @@
+/*
+ * gauss.h -- C ABI of the B200 (sm_100a) fused Gaussian kernel reduction library.
+ *
+ * The operation (Gaussian kernel sum with signed weights, "Kernel matrix
+ * reduction", Implementation sketch, eq. 1; output s_m of "Fast Gauss Sums via
+ * Flash Attention", Algorithm 1, step 2, with inputs q = x, k = y, v = w and
+ * tau > 0 as in its step 1):
+ *
+ *     out[b,i,c] = sum_j exp(-tau/2 * |x[b,i,:] - y[b,j,:]|^2) * w[b,j,c]
+ *
+ * is evaluated without ever forming the M x N kernel matrix: every kernel value
+ * is produced on chip and consumed at once.  The weights are called b on the
+ * pages; here they are w, to keep b for the batch index.
+ *
+ * Layouts (all row-major, contiguous, no strides):
+ *     x    [B, M, D]   query points, dtype dt
+ *     y    [B, N, D]   source points, dtype dt
+ *     w    [B, N, C]   weights, dtype dt
+ *     out  [B, M, C]   float32
+ *     g    [B, M, C]   float32 upstream gradient (backward only)
+ *
+ * Supported shapes and types:
+ *     GS_F32           : 1 <= D <= 8 (CUDA-core path), any C >= 1
+ *     GS_F16 / GS_BF16 : 1 <= D <= 126 (tensor-core path), any C >= 1.
+ *                        Arithmetic: x.y on the tensor cores with fp32
+ *                        accumulation, kernel values rounded to fp16 for the
+ *                        second product, weights converted to fp16 (for bf16
+ *                        weights this is exact for |w| in [2^-14, 65504]).
+ *   Anything else returns GS_ERR_UNSUPPORTED; there is no CPU fallback.
+ *
+ * Ownership and synchronisation: the caller owns every buffer, allocates the
+ * workspace (size from gs_workspace_bytes) and keeps all of them alive until
+ * the work queued on `stream` has finished.  The library allocates no device
+ * memory, never synchronises, and enqueues its kernels on `stream` (NULL = the
+ * legacy default stream).  All pointers are device pointers that must be
+ * 16-byte aligned (GS_ERR_ALIGNMENT otherwise); a pointer may be NULL only when
+ * the tensor it names is empty.  Results are deterministic: no floating-point
+ * atomics, and every partial sum is combined in a fixed order.
+ *
+ * Errors: arguments are validated on the host before anything is enqueued; a
+ * rejected call enqueues nothing.  Device-side faults the library can detect
+ * (a wait on an on-chip barrier that exceeds its time limit) set a device error
+ * word instead of trapping; gs_last_device_error() reads and clears it.
+ */
+#ifndef GAUSS_B200_H
+#define GAUSS_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st *gs_stream_t;
+
+typedef enum { GS_F32 = 0, GS_F16 = 1, GS_BF16 = 2 } gs_dtype;
+
+typedef enum { GS_OP_SUM = 0, GS_OP_LSE = 1, GS_OP_SUM_BWD = 2 } gs_op;
+
+typedef enum {
+    GS_OK = 0,
+    GS_ERR_INVALID_ARG = 1, /* NULL pointer for a non-empty tensor, negative size, tau not finite > 0 */
+    GS_ERR_UNSUPPORTED = 2, /* a (dtype, D) combination with no kernel */
+    GS_ERR_ALIGNMENT = 3,   /* a pointer not 16-byte aligned */
+    GS_ERR_WORKSPACE = 4,   /* workspace smaller than gs_workspace_bytes() */
+    GS_ERR_TIMEOUT = 5,     /* a device-side wait gave up (reported by gs_last_device_error) */
+    GS_ERR_CUDA = 6         /* a CUDA runtime call failed */
+} gs_status;
+
+/*
+ * Workspace, in bytes, that a call of `op` with these sizes needs on the
+ * current device (0 when none; the workspace pointer may then be NULL).  It
+ * holds packed operand copies, per-row norms and split-j partial results; the
+ * library never reads it before writing it, so it need not be initialised.
+ * Returns (size_t)-1 for arguments the corresponding call would reject.
+ */
+size_t gs_workspace_bytes(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, int64_t C,
+                          gs_dtype dt);
+
+/*
+ * Gaussian kernel sum (defined above; "Kernel matrix reduction", Implementation
+ * sketch, eq. 1 and eq. 2).  N == 0 writes zeros; M == 0 or B == 0 does nothing.
+ */
+gs_status gauss_sum_fwd(const void *x, const void *y, const void *w, float *out, int64_t B,
+                        int64_t M, int64_t N, int64_t D, int64_t C, float tau, gs_dtype dt,
+                        void *ws, size_t ws_bytes, gs_stream_t stream);
+
+/*
+ * Log-sum-exp reduction ("Kernel matrix reduction", Overview, the log-sum-exp
+ * reduction; the .logsumexp() reduction of the LazyTensor API in "KeOps: a
+ * symbolic tensor that never materialises the matrix it represents"), with the
+ * weights entering as their logarithm:
+ *
+ *     out[b,i,c] = log sum_j w[b,j,c] * exp(-tau/2 * |x_i - y_j|^2)
+ *
+ * computed with a shift so that rows whose every kernel value underflows fp32
+ * still get a finite result.  Requires w > 0 (not checked: a non-positive
+ * weight gives NaN or -inf, as log does).  N == 0 writes -inf.
+ * Supported for GS_F32 with 1 <= D <= 8.
+ */
+gs_status gauss_lse_fwd(const void *x, const void *y, const void *w, float *out, int64_t B,
+                        int64_t M, int64_t N, int64_t D, int64_t C, float tau, gs_dtype dt,
+                        void *ws, size_t ws_bytes, gs_stream_t stream);
+
+/*
+ * Gradient of L = sum_{b,i,c} g[b,i,c] * out[b,i,c] for the Gaussian kernel sum
+ * ("Kernel matrix reduction", Variants: gradients through the same fused
+ * reduction; the torch.autograd.grad example of the LazyTensor API):
+ *
+ *     grad_w[b,j,c] = sum_i K_ij g[b,i,c]                                 [B, N, C]
+ *     grad_x[b,i,k] = -tau * sum_j K_ij (sum_c g[b,i,c] w[b,j,c]) (x_ik - y_jk)   [B, M, D]
+ *
+ * with K_ij = exp(-tau/2 |x_i - y_j|^2), recomputed tile by tile, never stored.
+ * Either output may be NULL to skip it.  Both outputs are float32.
+ */
+gs_status gauss_sum_bwd(const void *x, const void *y, const void *w, const float *g,
+                        float *grad_x, float *grad_w, int64_t B, int64_t M, int64_t N, int64_t D,
+                        int64_t C, float tau, gs_dtype dt, void *ws, size_t ws_bytes,
+                        gs_stream_t stream);
+
+/* A static, human-readable name for a status code. */
+const char *gs_status_string(gs_status status);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word of the
+ * current device: GS_OK, GS_ERR_TIMEOUT (a kernel gave up on a wait and
+ * returned early; its outputs are not valid), or GS_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+gs_status gs_last_device_error(gs_stream_t stream);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int gs_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GAUSS_B200_H */

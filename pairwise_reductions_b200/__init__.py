@@ -1,0 +1,175 @@
+"""Python binding of the B200 fused Gaussian kernel reduction library.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libgauss_b200.so`` (declared in ``include/gauss.h``); PyTorch
+provides device memory and the current stream.  There is no CPU fallback: if
+the shared library is missing, importing this package raises.
+
+    gauss_sum_fwd(x, y, w, tau)           -> out [B, M, C] float32
+    gauss_lse_fwd(x, y, w, tau)           -> out [B, M, C] float32
+    gauss_sum_bwd(x, y, w, g, tau)        -> (grad_x [B, M, D], grad_w [B, N, C])
+
+x [B, M, D], y [B, N, D], w [B, N, C] share one dtype (float32, float16 or
+bfloat16) and must be contiguous CUDA tensors; 2-D inputs are read as B = 1.
+"""
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = _build.LIB
+
+GS_F32, GS_F16, GS_BF16 = 0, 1, 2
+GS_OP_SUM, GS_OP_LSE, GS_OP_SUM_BWD = 0, 1, 2
+STATUS = {0: "GS_OK", 1: "GS_ERR_INVALID_ARG", 2: "GS_ERR_UNSUPPORTED", 3: "GS_ERR_ALIGNMENT",
+          4: "GS_ERR_WORKSPACE", 5: "GS_ERR_TIMEOUT", 6: "GS_ERR_CUDA"}
+_DT = {torch.float32: GS_F32, torch.float16: GS_F16, torch.bfloat16: GS_BF16}
+
+# Every symbol include/gauss.h declares, with its ctypes signature.
+_i64, _f, _vp, _sz = ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+SIGNATURES = {
+    "gs_workspace_bytes": (_sz, [ctypes.c_int, _i64, _i64, _i64, _i64, _i64, ctypes.c_int]),
+    "gauss_sum_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _f,
+                                     ctypes.c_int, _vp, _sz, _vp]),
+    "gauss_lse_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _f,
+                                     ctypes.c_int, _vp, _sz, _vp]),
+    "gauss_sum_bwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64,
+                                     _f, ctypes.c_int, _vp, _sz, _vp]),
+    "gs_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "gs_last_device_error": (ctypes.c_int, [_vp]),
+    "gs_version": (ctypes.c_int, []),
+}
+
+
+class GaussError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn}: {STATUS.get(status, status)} ({_lib.gs_status_string(status).decode()})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m pairwise_reductions_b200.build` (needs nvcc)")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def library():
+    """The loaded ctypes handle of libgauss_b200.so."""
+    return _lib
+
+
+def status_string(code):
+    return _lib.gs_status_string(int(code)).decode()
+
+
+def workspace_bytes(op, B, M, N, D, C, dtype):
+    """Bytes of workspace a call needs (see gs_workspace_bytes)."""
+    v = _lib.gs_workspace_bytes(int(op), B, M, N, D, C, _DT[dtype] if isinstance(dtype, torch.dtype) else int(dtype))
+    if v == ctypes.c_size_t(-1).value:
+        raise ValueError("gs_workspace_bytes rejected the arguments")
+    return int(v)
+
+
+def _as3(t, name):
+    if t.dim() == 2:
+        t = t.unsqueeze(0)
+    if t.dim() != 3:
+        raise ValueError(f"{name}: expected a 2-D or 3-D tensor, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None and t.numel() > 0 else ctypes.c_void_p(0)
+
+
+def _workspace(nbytes, device, ws):
+    if nbytes == 0:
+        return None
+    if ws is not None and ws.numel() >= nbytes:
+        return ws
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def _check(fn, st):
+    if st != 0:
+        raise GaussError(fn, st)
+
+
+def _dims(x, y, w):
+    B, M, D = x.shape
+    if y.shape[0] != B or y.shape[2] != D or w.shape[0] != B or w.shape[1] != y.shape[1]:
+        raise ValueError(f"shape mismatch x{tuple(x.shape)} y{tuple(y.shape)} w{tuple(w.shape)}")
+    if not (x.dtype == y.dtype == w.dtype) or x.dtype not in _DT:
+        raise ValueError("x, y, w must share one dtype among float32, float16, bfloat16")
+    return B, M, y.shape[1], D, w.shape[2]
+
+
+def _reduce(name, op, x, y, w, tau, out, workspace, stream):
+    x, y, w = _as3(x, "x"), _as3(y, "y"), _as3(w, "w")
+    B, M, N, D, C = _dims(x, y, w)
+    if out is None:
+        out = torch.empty((B, M, C), dtype=torch.float32, device=x.device)
+    nbytes = workspace_bytes(op, B, M, N, D, C, x.dtype)
+    ws = _workspace(nbytes, x.device, workspace)
+    st = getattr(_lib, name)(_ptr(x), _ptr(y), _ptr(w), _ptr(out), B, M, N, D, C, float(tau),
+                             _DT[x.dtype], _ptr(ws), nbytes if ws is not None else 0,
+                             _stream(stream))
+    _check(name, st)
+    return out
+
+
+def gauss_sum_fwd(x, y, w, tau, out=None, workspace=None, stream=None):
+    """out[b,i,c] = sum_j exp(-tau/2 |x_i - y_j|^2) w[b,j,c]   (float32 result)."""
+    return _reduce("gauss_sum_fwd", GS_OP_SUM, x, y, w, tau, out, workspace, stream)
+
+
+def gauss_lse_fwd(x, y, w, tau, out=None, workspace=None, stream=None):
+    """out[b,i,c] = log sum_j w[b,j,c] exp(-tau/2 |x_i - y_j|^2)   (w > 0)."""
+    return _reduce("gauss_lse_fwd", GS_OP_LSE, x, y, w, tau, out, workspace, stream)
+
+
+def gauss_sum_bwd(x, y, w, g, tau, want_x=True, want_w=True, workspace=None, stream=None):
+    """Gradients of sum(g * gauss_sum_fwd(x, y, w)) with respect to x and w."""
+    x, y, w, g = _as3(x, "x"), _as3(y, "y"), _as3(w, "w"), _as3(g, "g")
+    B, M, N, D, C = _dims(x, y, w)
+    if g.shape != (B, M, C) or g.dtype != torch.float32:
+        raise ValueError(f"g must be float32 of shape {(B, M, C)}")
+    gx = torch.empty((B, M, D), dtype=torch.float32, device=x.device) if want_x else None
+    gw = torch.empty((B, N, C), dtype=torch.float32, device=x.device) if want_w else None
+    nbytes = workspace_bytes(GS_OP_SUM_BWD, B, M, N, D, C, x.dtype)
+    ws = _workspace(nbytes, x.device, workspace)
+    st = _lib.gauss_sum_bwd(_ptr(x), _ptr(y), _ptr(w), _ptr(g), _ptr(gx) if want_x else None,
+                            _ptr(gw) if want_w else None, B, M, N, D, C, float(tau), _DT[x.dtype],
+                            _ptr(ws), nbytes if ws is not None else 0, _stream(stream))
+    _check("gauss_sum_bwd", st)
+    return gx, gw
+
+
+def last_device_error(stream=None):
+    """Synchronise and read/clear the device error word (0 = none)."""
+    return int(_lib.gs_last_device_error(_stream(stream)))
+
+
+__all__ = ["gauss_sum_fwd", "gauss_lse_fwd", "gauss_sum_bwd", "workspace_bytes",
+           "last_device_error", "library", "status_string", "GaussError", "SIGNATURES",
+           "LIB_PATH"]

@@ -1,0 +1,428 @@
+// api.cpp -- the C ABI front end: argument validation, workspace sizing and
+// dispatch to the CUDA-core (fp32, small D) or tensor-core (fp16/bf16) path.
+// Nothing here synchronises or allocates; all work goes onto the caller's
+// stream.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "internal.h"
+
+using namespace gs;
+
+namespace {
+
+constexpr size_t kAlign = 1024;
+constexpr size_t kBad = static_cast<size_t>(-1);
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return kSmCountDefault;
+  }
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return kSmCountDefault;
+  }
+  return n;
+}
+
+size_t elem_size(gs_dtype dt) { return dt == GS_F32 ? 4 : 2; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape and type checks shared by every entry point (no pointers).
+gs_status check_dims(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, int64_t C, gs_dtype dt) {
+  if (B < 0 || M < 0 || N < 0 || D < 1 || C < 1) return GS_ERR_INVALID_ARG;
+  if (dt != GS_F32 && dt != GS_F16 && dt != GS_BF16) return GS_ERR_INVALID_ARG;
+  // index arithmetic stays in int64, grid.z holds B, TMA coordinates are int32
+  const int64_t lim = int64_t(1) << 31;
+  if (B >= 65536 || M >= lim || N >= lim || C >= lim || D >= lim) return GS_ERR_UNSUPPORTED;
+  const double big = 9.0e18;
+  if (double(B) * double(M > N ? M : N) * double((D > C ? D : C) + 1) * double(D + 2) > big)
+    return GS_ERR_UNSUPPORTED;
+  if (dt == GS_F32) {
+    if (D > kSdMaxD) return GS_ERR_UNSUPPORTED;
+  } else {
+    if (D > kTcMaxD) return GS_ERR_UNSUPPORTED;
+    if (op == GS_OP_LSE) return GS_ERR_UNSUPPORTED;
+  }
+  return GS_OK;
+}
+
+gs_status check_tau(float tau) {
+  return (std::isfinite(tau) && tau > 0.f) ? GS_OK : GS_ERR_INVALID_ARG;
+}
+
+gs_status check_ptr(const void* p, int64_t n_elems) {
+  if (n_elems == 0) return GS_OK;
+  if (p == nullptr) return GS_ERR_INVALID_ARG;
+  if (!aligned16(p)) return GS_ERR_ALIGNMENT;
+  return GS_OK;
+}
+
+#define GS_TRY(expr)                    \
+  do {                                  \
+    gs_status _st = (expr);             \
+    if (_st != GS_OK) return _st;       \
+  } while (0)
+
+#define GS_CUDA(expr)                   \
+  do {                                  \
+    cudaError_t _e = (expr);            \
+    if (_e != cudaSuccess) return GS_ERR_CUDA; \
+  } while (0)
+
+float coord_scale(float tau) {
+  return static_cast<float>(std::sqrt(0.5 * static_cast<double>(tau) * 1.4426950408889634074));
+}
+
+// ------------------------------------------------------------------ one Gauss-sum pass
+// out[B, rows, CV] = sum over cols of K(rows, cols) * values, where values are
+// w (CV = C) or the gradient values [w, w (x) col points] (CV = C (1 + D)).
+struct Pass {
+  const void* rows_pts;
+  const void* cols_pts;
+  const void* w;
+  bool w_is_f32;
+  bool bwd_values;
+  int64_t B, R, N;   // rows, columns
+  int D, C, CV;
+  gs_dtype dt;
+  float tau;
+};
+
+struct PassLayout {
+  bool tc;
+  SdPlan sd;
+  TcPlan tcp;
+  size_t off_part, off_vals, off_xpack, off_rnorm, off_ypack, off_vt;
+  size_t total;
+};
+
+PassLayout pass_layout(const Pass& p, int sm) {
+  PassLayout L{};
+  size_t off = 0;
+  L.tc = p.dt != GS_F32;
+  if (!L.tc) {
+    L.sd = sd_plan(p.B, p.R, p.N, p.D, p.CV, sm);
+    if (p.bwd_values) {
+      L.off_vals = off;
+      off = align_up(off + size_t(p.B) * p.N * p.CV * 4);
+    }
+    if (L.sd.splits > 1) {
+      L.off_part = off;
+      off = align_up(off + size_t(L.sd.splits) * p.B * p.R * p.CV * 4);
+    }
+  } else {
+    L.tcp = tc_plan(p.B, p.R, p.N, p.D, sm);
+    const size_t KP = static_cast<size_t>(L.tcp.KP);
+    const int chunk = p.CV < kTcMaxChunk ? p.CV : kTcMaxChunk;
+    const size_t CPmax = (chunk + 15) / 16 * 16 <= 64 ? (chunk + 15) / 16 * 16
+                                                      : ((chunk + 15) / 16 * 16 <= 96 ? 96 : 128);
+    const size_t Nst = (p.N + 7) / 8 * 8;
+    L.off_xpack = off;
+    off = align_up(off + size_t(p.B) * p.R * KP * 2);
+    L.off_rnorm = off;
+    off = align_up(off + size_t(p.B) * p.R * 4);
+    L.off_ypack = off;
+    off = align_up(off + size_t(p.B) * p.N * KP * 2);
+    L.off_vt = off;
+    off = align_up(off + size_t(p.B) * CPmax * Nst * 2);
+    if (L.tcp.splits > 1) {
+      L.off_part = off;
+      off = align_up(off + size_t(L.tcp.splits) * p.B * p.R * p.CV * 4);
+    }
+  }
+  L.total = off;
+  return L;
+}
+
+// Run one pass into `out` ([B, R, CV] float32) using workspace `ws`.
+gs_status run_pass(const Pass& p, const PassLayout& L, float* out, uint8_t* ws, cudaStream_t s) {
+  const int64_t total = p.B * p.R * p.CV;
+  if (total == 0) return GS_OK;
+  if (p.N == 0) {
+    GS_CUDA(cudaMemsetAsync(out, 0, size_t(total) * 4, s));
+    return GS_OK;
+  }
+  if (!L.tc) {
+    const float* values = static_cast<const float*>(p.w);
+    if (p.bwd_values) {
+      float* v = reinterpret_cast<float*>(ws + L.off_vals);
+      GS_CUDA(launch_pack_bwd_values_f32(static_cast<const float*>(p.cols_pts), values, v, p.B, p.N,
+                                         p.D, p.C, s));
+      values = v;
+    }
+    const int S = L.sd.splits;
+    float* dst = S > 1 ? reinterpret_cast<float*>(ws + L.off_part) : out;
+    for (int c0 = 0; c0 < p.CV; c0 += kSdMaxChunk) {
+      SdArgs a{};
+      a.x = static_cast<const float*>(p.rows_pts);
+      a.y = static_cast<const float*>(p.cols_pts);
+      a.w = values;
+      a.ldw = p.CV;
+      a.c0 = c0;
+      a.cw = (p.CV - c0) < kSdMaxChunk ? (p.CV - c0) : kSdMaxChunk;
+      a.out = dst;
+      a.out_l = nullptr;
+      a.ldo = p.CV;
+      a.split_stride = S > 1 ? total : 0;
+      a.B = p.B;
+      a.M = p.R;
+      a.N = p.N;
+      a.D = p.D;
+      a.scale = coord_scale(p.tau);
+      a.plan = L.sd;
+      GS_CUDA(launch_small_d_sum(a, s));
+    }
+    if (S > 1) GS_CUDA(launch_combine_sum(dst, S, total, out, s));
+    return GS_OK;
+  }
+  const int S = L.tcp.splits;
+  float* dst = S > 1 ? reinterpret_cast<float*>(ws + L.off_part) : out;
+  TcArgs a{};
+  a.x = p.rows_pts;
+  a.y = p.cols_pts;
+  a.w = p.w;
+  a.w_is_f32 = p.w_is_f32;
+  a.values = p.bwd_values ? kValuesBwd : kValuesW;
+  a.C = p.C;
+  a.CV = p.CV;
+  a.out = dst;
+  a.split_stride = S > 1 ? total : 0;
+  a.B = p.B;
+  a.M = p.R;
+  a.N = p.N;
+  a.D = p.D;
+  a.dt = p.dt;
+  a.tau = p.tau;
+  a.plan = L.tcp;
+  a.xpack = ws + L.off_xpack;
+  a.rnorm = reinterpret_cast<float*>(ws + L.off_rnorm);
+  a.ypack = ws + L.off_ypack;
+  a.vt = ws + L.off_vt;
+  GS_CUDA(launch_tc_sum(a, s));
+  if (S > 1) GS_CUDA(launch_combine_sum(dst, S, total, out, s));
+  return GS_OK;
+}
+
+Pass fwd_pass(const void* x, const void* y, const void* w, int64_t B, int64_t M, int64_t N,
+              int64_t D, int64_t C, float tau, gs_dtype dt) {
+  Pass p{};
+  p.rows_pts = x;
+  p.cols_pts = y;
+  p.w = w;
+  p.w_is_f32 = dt == GS_F32;
+  p.bwd_values = false;
+  p.B = B;
+  p.R = M;
+  p.N = N;
+  p.D = static_cast<int>(D);
+  p.C = static_cast<int>(C);
+  p.CV = static_cast<int>(C);
+  p.dt = dt;
+  p.tau = tau;
+  return p;
+}
+
+// Backward = two passes: grad_w from (rows = y, cols = x, values = g) and the
+// x-gradient values O = K [w, w (x) y] from (rows = x, cols = y), then an
+// elementwise epilogue.  They run one after the other and share the workspace;
+// O sits after the larger pass layout.
+struct BwdLayout {
+  Pass pw, px;
+  PassLayout lw, lx;
+  size_t off_o;
+  size_t total;
+};
+
+BwdLayout bwd_layout(const void* x, const void* y, const void* w, const float* g, int64_t B,
+                     int64_t M, int64_t N, int64_t D, int64_t C, float tau, gs_dtype dt, int sm,
+                     bool want_x, bool want_w) {
+  BwdLayout L{};
+  L.pw = fwd_pass(y, x, g, B, N, M, D, C, tau, dt);
+  L.pw.w_is_f32 = true;
+  L.px = fwd_pass(x, y, w, B, M, N, D, C, tau, dt);
+  L.px.bwd_values = true;
+  L.px.CV = static_cast<int>(C * (1 + D));
+  L.lw = pass_layout(L.pw, sm);
+  L.lx = pass_layout(L.px, sm);
+  size_t need = 0;
+  if (want_w) need = L.lw.total;
+  if (want_x) {
+    L.off_o = align_up(L.lx.total > need ? L.lx.total : need);
+    need = align_up(L.off_o + size_t(B) * M * C * (1 + D) * 4);
+  }
+  L.total = need;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gs_version(void) { return 100; }
+
+const char* gs_status_string(gs_status st) {
+  switch (st) {
+    case GS_OK: return "ok";
+    case GS_ERR_INVALID_ARG: return "invalid argument";
+    case GS_ERR_UNSUPPORTED: return "unsupported dtype/shape combination";
+    case GS_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case GS_ERR_WORKSPACE: return "workspace too small";
+    case GS_ERR_TIMEOUT: return "device-side wait timed out";
+    case GS_ERR_CUDA: return "CUDA runtime error";
+  }
+  return "unknown status";
+}
+
+size_t gs_workspace_bytes(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, int64_t C,
+                          gs_dtype dt) {
+  if (op != GS_OP_SUM && op != GS_OP_LSE && op != GS_OP_SUM_BWD) return kBad;
+  if (check_dims(op, B, M, N, D, C, dt) != GS_OK) return kBad;
+  if (B == 0) return 0;
+  const int sm = sm_count();
+  if (op == GS_OP_SUM) {
+    if (M == 0 || N == 0) return 0;
+    return pass_layout(fwd_pass(nullptr, nullptr, nullptr, B, M, N, D, C, 1.f, dt), sm).total;
+  }
+  if (op == GS_OP_LSE) {
+    if (M == 0 || N == 0) return 0;
+    const SdPlan sp = sd_plan(B, M, N, static_cast<int>(D), C, sm);
+    return align_up(size_t(2) * sp.splits * B * M * C * 4);
+  }
+  if (M == 0 || N == 0) return 0;
+  return bwd_layout(nullptr, nullptr, nullptr, nullptr, B, M, N, D, C, 1.f, dt, sm, true, true).total;
+}
+
+gs_status gauss_sum_fwd(const void* x, const void* y, const void* w, float* out, int64_t B,
+                        int64_t M, int64_t N, int64_t D, int64_t C, float tau, gs_dtype dt,
+                        void* ws, size_t ws_bytes, gs_stream_t stream) {
+  GS_TRY(check_dims(GS_OP_SUM, B, M, N, D, C, dt));
+  GS_TRY(check_tau(tau));
+  GS_TRY(check_ptr(x, B * M * D));
+  GS_TRY(check_ptr(y, B * N * D));
+  GS_TRY(check_ptr(w, B * N * C));
+  GS_TRY(check_ptr(out, B * M * C));
+  if (B == 0 || M == 0) return GS_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const Pass p = fwd_pass(x, y, w, B, M, N, D, C, tau, dt);
+  const PassLayout L = pass_layout(p, sm_count());
+  if (N > 0 && L.total > 0) {
+    if (ws_bytes < L.total) return GS_ERR_WORKSPACE;
+    GS_TRY(check_ptr(ws, 1));
+  }
+  return run_pass(p, L, out, static_cast<uint8_t*>(ws), s);
+}
+
+gs_status gauss_lse_fwd(const void* x, const void* y, const void* w, float* out, int64_t B,
+                        int64_t M, int64_t N, int64_t D, int64_t C, float tau, gs_dtype dt,
+                        void* ws, size_t ws_bytes, gs_stream_t stream) {
+  GS_TRY(check_dims(GS_OP_LSE, B, M, N, D, C, dt));
+  GS_TRY(check_tau(tau));
+  GS_TRY(check_ptr(x, B * M * D));
+  GS_TRY(check_ptr(y, B * N * D));
+  GS_TRY(check_ptr(w, B * N * C));
+  GS_TRY(check_ptr(out, B * M * C));
+  if (B == 0 || M == 0) return GS_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (N == 0) {
+    GS_CUDA(launch_fill(out, B * M * C, -INFINITY, s));
+    return GS_OK;
+  }
+  const int sm = sm_count();
+  const SdPlan sp = sd_plan(B, M, N, static_cast<int>(D), C, sm);
+  const size_t need = align_up(size_t(2) * sp.splits * B * M * C * 4);
+  if (ws_bytes < need) return GS_ERR_WORKSPACE;
+  GS_TRY(check_ptr(ws, 1));
+  const int64_t total = B * M * C;
+  float* part_m = static_cast<float*>(ws);
+  float* part_l = part_m + size_t(sp.splits) * total;
+  const float scale = coord_scale(tau);
+  for (int c0 = 0; c0 < C; c0 += kSdMaxChunk) {
+    SdArgs a{};
+    a.x = static_cast<const float*>(x);
+    a.y = static_cast<const float*>(y);
+    a.w = static_cast<const float*>(w);
+    a.ldw = static_cast<int>(C);
+    a.c0 = c0;
+    a.cw = static_cast<int>((C - c0) < kSdMaxChunk ? (C - c0) : kSdMaxChunk);
+    a.out = part_m;
+    a.out_l = part_l;
+    a.ldo = static_cast<int>(C);
+    a.split_stride = total;
+    a.B = B;
+    a.M = M;
+    a.N = N;
+    a.D = static_cast<int>(D);
+    a.scale = scale;
+    a.plan = sp;
+    GS_CUDA(launch_small_d_lse(a, s));
+  }
+  LseFinalizeArgs f{};
+  f.part_m = part_m;
+  f.part_l = part_l;
+  f.splits = sp.splits;
+  f.split_stride = total;
+  f.out = out;
+  f.x = static_cast<const float*>(x);
+  f.y = static_cast<const float*>(y);
+  f.w = static_cast<const float*>(w);
+  f.B = B;
+  f.M = M;
+  f.N = N;
+  f.D = static_cast<int>(D);
+  f.C = static_cast<int>(C);
+  f.scale = scale;
+  GS_CUDA(launch_lse_finalize(f, s));
+  return GS_OK;
+}
+
+gs_status gauss_sum_bwd(const void* x, const void* y, const void* w, const float* g,
+                        float* grad_x, float* grad_w, int64_t B, int64_t M, int64_t N, int64_t D,
+                        int64_t C, float tau, gs_dtype dt, void* ws, size_t ws_bytes,
+                        gs_stream_t stream) {
+  GS_TRY(check_dims(GS_OP_SUM_BWD, B, M, N, D, C, dt));
+  GS_TRY(check_tau(tau));
+  GS_TRY(check_ptr(x, B * M * D));
+  GS_TRY(check_ptr(y, B * N * D));
+  GS_TRY(check_ptr(w, B * N * C));
+  GS_TRY(check_ptr(g, B * M * C));
+  if (grad_x) GS_TRY(check_ptr(grad_x, B * M * D));
+  if (grad_w) GS_TRY(check_ptr(grad_w, B * N * C));
+  if (B == 0 || (!grad_x && !grad_w)) return GS_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool want_x = grad_x != nullptr && M > 0;
+  const bool want_w = grad_w != nullptr && N > 0;
+  if (grad_x && M > 0 && N == 0) GS_CUDA(cudaMemsetAsync(grad_x, 0, size_t(B) * M * D * 4, s));
+  if (grad_w && N > 0 && M == 0) GS_CUDA(cudaMemsetAsync(grad_w, 0, size_t(B) * N * C * 4, s));
+  if (M == 0 || N == 0) return GS_OK;
+  const BwdLayout L = bwd_layout(x, y, w, g, B, M, N, D, C, tau, dt, sm_count(), want_x, want_w);
+  if (L.total > 0) {
+    if (ws_bytes < L.total) return GS_ERR_WORKSPACE;
+    GS_TRY(check_ptr(ws, 1));
+  }
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  if (want_w) GS_TRY(run_pass(L.pw, L.lw, grad_w, wsb, s));
+  if (want_x) {
+    float* o = reinterpret_cast<float*>(wsb + L.off_o);
+    GS_TRY(run_pass(L.px, L.lx, o, wsb, s));
+    GS_CUDA(launch_bwd_grad_x_epilogue(x, dt, g, o, grad_x, B, M, static_cast<int>(D),
+                                       static_cast<int>(C), tau, s));
+  }
+  return GS_OK;
+}
+
+gs_status gs_last_device_error(gs_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return GS_ERR_CUDA;
+  int v = 0;
+  if (read_and_clear_device_error(&v) != cudaSuccess) return GS_ERR_CUDA;
+  return v ? GS_ERR_TIMEOUT : GS_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,132 @@
+// internal.h -- host-side interface between the C ABI front end (api.cpp)
+// and the kernel translation units.  Not part of the public ABI.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/gauss.h"
+
+namespace gs {
+
+constexpr int kSmCountDefault = 148;   // B200
+
+// ------------------------------------------------------------- small-D path
+// Rows per CTA of the CUDA-core kernel and its widest channel chunk.
+constexpr int kSdThreads = 128;
+constexpr int kSdMaxChunk = 8;
+constexpr int kSdMaxD = 8;
+
+// Rows each thread of the small-D kernel keeps in registers, by feature
+// width D and padded channel chunk CP (register budget ~ R * (D + 2 CP)).
+__host__ __device__ constexpr int sd_rows_per_thread(int D, int CP) {
+  return (D + 2 * CP <= 16) ? 4 : ((D + 2 * CP <= 40) ? 2 : 1);
+}
+// Channel chunk width the kernel is instantiated for (1, 2, 4 or 8).
+__host__ __device__ constexpr int sd_chunk_pad(int c) {
+  return c <= 1 ? 1 : (c <= 2 ? 2 : (c <= 4 ? 4 : 8));
+}
+
+struct SdPlan {
+  int rows_per_cta;    // kSdThreads * rows per thread
+  int splits;          // j-splits (partials combined afterwards when > 1)
+  int64_t cols_per_split;
+};
+
+// Choose rows per CTA and the j-split for the small-D kernel.
+SdPlan sd_plan(int64_t B, int64_t M, int64_t N, int D, int64_t C, int sm_count);
+
+struct SdArgs {
+  const float* x;
+  const float* y;
+  const float* w;      // [B, N, ldw]
+  int ldw;             // channels in w rows
+  int c0;              // first channel of this chunk
+  int cw;              // channels in this chunk (<= kSdMaxChunk)
+  float* out;          // sum: [S?][B][M][ldo]; lse: shift part
+  float* out_l;        // lse only: scaled sums, same layout as out
+  int ldo;
+  int64_t split_stride;  // elements between split slices (0 if one split)
+  int64_t B, M, N;
+  int D;
+  float scale;         // sqrt(tau / 2 * log2 e)
+  SdPlan plan;
+};
+
+cudaError_t launch_small_d_sum(const SdArgs& a, cudaStream_t s);
+cudaError_t launch_small_d_lse(const SdArgs& a, cudaStream_t s);
+
+// Combine `splits` partial sums [S][total] into out[total] in fixed order.
+cudaError_t launch_combine_sum(const float* part, int splits, int64_t total, float* out,
+                               cudaStream_t s);
+
+// Combine (shift, scaled sum) partials into the log-sum-exp and recompute
+// exactly any row whose scaled sum came out too small to trust.
+struct LseFinalizeArgs {
+  const float* part_m;
+  const float* part_l;
+  int splits;
+  int64_t split_stride;
+  float* out;          // [B, M, C]
+  const float* x;
+  const float* y;
+  const float* w;
+  int64_t B, M, N;
+  int D, C;
+  float scale;
+};
+cudaError_t launch_lse_finalize(const LseFinalizeArgs& a, cudaStream_t s);
+
+// Value matrix for the x-gradient on the fp32 path: v = [w, w (x) y], [B, N, C*(1+D)].
+cudaError_t launch_pack_bwd_values_f32(const float* y, const float* w, float* v, int64_t B,
+                                       int64_t N, int D, int C, cudaStream_t s);
+
+// grad_x[b,i,k] = -tau * sum_c g[b,i,c] (x[b,i,k] * o[b,i,c] - o[b,i,C + c*D + k])
+cudaError_t launch_bwd_grad_x_epilogue(const void* x, gs_dtype dt, const float* g,
+                                       const float* o, float* grad_x, int64_t B, int64_t M,
+                                       int D, int C, float tau, cudaStream_t s);
+
+// ------------------------------------------------------------- tensor-core path
+constexpr int kTcMaxD = 126;
+constexpr int kTcMaxChunk = 128;   // channels per tensor-core pass
+
+struct TcPlan {
+  int KP;              // padded feature width of the packed operands (64 or 128)
+  int splits;
+  int64_t cols_per_split;   // multiple of 128
+};
+TcPlan tc_plan(int64_t B, int64_t M, int64_t N, int64_t D, int sm_count);
+
+// Which values the tensor-core pass multiplies by the kernel.
+enum TcValues { kValuesW = 0, kValuesBwd = 1 };
+
+struct TcArgs {
+  const void* x;       // rows side [B, M, D]
+  const void* y;       // column side [B, N, D]
+  const void* w;       // values source [B, N, C] (dtype dt, or float32 if w_is_f32)
+  bool w_is_f32;
+  TcValues values;     // kValuesW: v = w; kValuesBwd: v = [w, w (x) y]
+  int C;               // channels of w
+  int CV;              // channels of the value matrix (C or C*(1+D))
+  float* out;          // [S?][B][M][CV]
+  int64_t split_stride;
+  int64_t B, M, N;
+  int D;
+  gs_dtype dt;
+  float tau;
+  TcPlan plan;
+  // workspace pieces
+  void* xpack;         // [B, M, KP]
+  float* rnorm;        // [B, M]
+  void* ypack;         // [B, N, KP]
+  void* vt;            // [B, CP, Nst] f16
+};
+cudaError_t launch_tc_sum(const TcArgs& a, cudaStream_t s);
+
+// out[0 .. n) = value
+cudaError_t launch_fill(float* out, int64_t n, float value, cudaStream_t s);
+
+// Device error word (set by kernels whose waits time out).
+cudaError_t read_and_clear_device_error(int* value);
+
+}  // namespace gs

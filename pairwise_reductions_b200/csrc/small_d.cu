@@ -1,0 +1,492 @@
+// small_d.cu -- CUDA-core kernels for the Gaussian kernel sum and its
+// log-sum-exp at small feature width (fp32, 1 <= D <= 8).
+//
+// Computes ("Kernel matrix reduction", Implementation sketch, eq. 1)
+//     a[b,i,c] = sum_j exp(-tau/2 |x_i - y_j|^2) w[b,j,c]
+// and the weighted log-sum-exp of the same page's Overview, without forming
+// the kernel matrix.  Design:
+//   * coordinates are pre-multiplied by s = sqrt(tau/2 * log2 e), so each
+//     kernel value is a single MUFU ex2 of -|x^ - y^|^2 (direct difference
+//     form: 3 FADD + 1 FMUL + 2 FFMA per pair at D = 3, one FFMA to
+//     accumulate);
+//   * a CTA keeps R rows per thread (x^ and accumulators in registers) and
+//     streams y/w through shared memory in tiles of 256 points, packed
+//     per point as {y^_0 .. y^_{D-1}, v_0 .. v_{CP-1}} so one broadcast
+//     LDS.128 feeds R * CP kernel evaluations;
+//   * each tile is summed into a tile accumulator before it joins the running
+//     total (two-level summation keeps fp32 rounding well below 1e-5 relative
+//     at 10^6 terms with signed weights);
+//   * the column range is split over CTAs when there are too few row tiles
+//     to fill 148 SMs; partials are combined in a fixed order afterwards.
+// Log-sum-exp: the weights enter as log2 w; every tile shifts them by the
+// running maximum of log2 w over the tiles seen so far (a uniform upper bound
+// of every exponent, since the kernel is at most 1), rescaling the
+// accumulator when the maximum grows -- the online normaliser of Milakov and
+// Gimelshein that the FlashDiffusion page cites, with the bound taken from
+// the weights.  Rows whose scaled sum comes out tiny are recomputed exactly
+// (per-row maximum) by the finalisation kernel.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cmath>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace gs {
+namespace {
+
+constexpr int kTileJ = 256;
+constexpr int kPer = kTileJ / kSdThreads;   // points each thread stages per tile
+constexpr float kLn2 = 0.69314718055994530942f;
+
+template <int D, int CP>
+struct PackShape {
+  static constexpr int PK = ((D + CP + 3) / 4) * 4;   // floats per staged point
+};
+
+template <int D, int CP, bool LSE>
+__global__ void __launch_bounds__(kSdThreads)
+    sd_kernel(const SdArgs a) {
+  constexpr int R = sd_rows_per_thread(D, CP);
+  constexpr int PK = PackShape<D, CP>::PK;
+  constexpr int NW = kSdThreads / 32;
+  __shared__ __align__(16) float tile[kTileJ * PK];
+  __shared__ float red[NW][CP];
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int64_t b = blockIdx.z;
+  const int split = blockIdx.y;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * (kSdThreads * R);
+  const int64_t jbeg = static_cast<int64_t>(split) * a.plan.cols_per_split;
+  const int64_t jend = min(a.N, jbeg + a.plan.cols_per_split);
+  const float* __restrict__ yb = a.y + b * a.N * D;
+  const float* __restrict__ wb = a.w + b * a.N * a.ldw + a.c0;
+
+  float xs[R][D];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int64_t i = row0 + tid + r * kSdThreads;
+#pragma unroll
+    for (int k = 0; k < D; ++k)
+      xs[r][k] = (i < a.M) ? a.x[(b * a.M + i) * D + k] * a.scale : 0.f;
+  }
+  float acc[R][CP];
+  float mrun[CP];
+#pragma unroll
+  for (int c = 0; c < CP; ++c) {
+    mrun[c] = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[r][c] = 0.f;
+  }
+
+  for (int64_t j0 = jbeg; j0 < jend; j0 += kTileJ) {
+    // ---- stage one tile of (scaled y, weight or shifted log2 weight)
+    float sy[kPer][D], sv[kPer][CP];
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int64_t j = j0 + tid + q * kSdThreads;
+      const bool ok = j < jend;
+#pragma unroll
+      for (int k = 0; k < D; ++k) sy[q][k] = ok ? yb[j * D + k] * a.scale : 0.f;
+#pragma unroll
+      for (int c = 0; c < CP; ++c) {
+        const bool okc = ok && c < a.cw;
+        const float wv = okc ? wb[j * a.ldw + c] : 0.f;
+        if constexpr (LSE)
+          sv[q][c] = okc ? lg2(wv) : -INFINITY;
+        else
+          sv[q][c] = wv;
+      }
+    }
+    if constexpr (LSE) {
+#pragma unroll
+      for (int c = 0; c < CP; ++c) {
+        float m = sv[0][c];
+#pragma unroll
+        for (int q = 1; q < kPer; ++q) m = fmaxf(m, sv[q][c]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) red[warp][c] = m;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int c = 0; c < CP; ++c) {
+        float mt = red[0][c];
+#pragma unroll
+        for (int v = 1; v < NW; ++v) mt = fmaxf(mt, red[v][c]);
+        const float mnew = fmaxf(mrun[c], mt);
+        const float fac = (mrun[c] == -INFINITY) ? 0.f : ex2(mrun[c] - mnew);
+#pragma unroll
+        for (int r = 0; r < R; ++r) acc[r][c] *= fac;
+        mrun[c] = mnew;
+        const float sh = (mnew == -INFINITY) ? 0.f : mnew;
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) sv[q][c] -= sh;
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      float* p = tile + (tid + q * kSdThreads) * PK;
+#pragma unroll
+      for (int k = 0; k < D; ++k) p[k] = sy[q][k];
+#pragma unroll
+      for (int c = 0; c < CP; ++c) p[D + c] = sv[q][c];
+#pragma unroll
+      for (int k = D + CP; k < PK; ++k) p[k] = 0.f;
+    }
+    __syncthreads();
+
+    // ---- all pairs (my R rows) x (256 staged points)
+    float tacc[R][CP];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int c = 0; c < CP; ++c) tacc[r][c] = 0.f;
+
+    const float4* t4 = reinterpret_cast<const float4*>(tile);
+#pragma unroll 4
+    for (int jj = 0; jj < kTileJ; ++jj) {
+      float pk[PK];
+#pragma unroll
+      for (int v = 0; v < PK / 4; ++v) {
+        const float4 q = t4[jj * (PK / 4) + v];
+        pk[4 * v + 0] = q.x;
+        pk[4 * v + 1] = q.y;
+        pk[4 * v + 2] = q.z;
+        pk[4 * v + 3] = q.w;
+      }
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        if constexpr (LSE && CP == 1) {
+          // exponent = log2 w - shift - |x^ - y^|^2, accumulated from the weight term
+          float t = pk[D];
+#pragma unroll
+          for (int k = 0; k < D; ++k) {
+            const float e = xs[r][k] - pk[k];
+            t = fmaf(-e, e, t);
+          }
+          tacc[r][0] += ex2(t);
+        } else {
+          const float e0 = xs[r][0] - pk[0];
+          float t = -e0 * e0;
+#pragma unroll
+          for (int k = 1; k < D; ++k) {
+            const float e = xs[r][k] - pk[k];
+            t = fmaf(-e, e, t);
+          }
+          if constexpr (LSE) {
+#pragma unroll
+            for (int c = 0; c < CP; ++c) tacc[r][c] += ex2(t + pk[D + c]);
+          } else {
+            const float kv = ex2(t);
+#pragma unroll
+            for (int c = 0; c < CP; ++c) tacc[r][c] = fmaf(kv, pk[D + c], tacc[r][c]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int c = 0; c < CP; ++c) acc[r][c] += tacc[r][c];
+    __syncthreads();
+  }
+
+  // ---- write this split's result (final sum, or shift + scaled sum)
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int64_t i = row0 + tid + r * kSdThreads;
+    if (i >= a.M) continue;
+    const int64_t base = split * a.split_stride + (b * a.M + i) * a.ldo + a.c0;
+#pragma unroll
+    for (int c = 0; c < CP; ++c) {
+      if (c >= a.cw) break;
+      if constexpr (LSE) {
+        a.out[base + c] = mrun[c];
+        a.out_l[base + c] = acc[r][c];
+      } else {
+        a.out[base + c] = acc[r][c];
+      }
+    }
+  }
+}
+
+template <int D, int CP, bool LSE>
+cudaError_t launch_t(const SdArgs& a, cudaStream_t s) {
+  constexpr int R = sd_rows_per_thread(D, CP);
+  const int64_t tiles = (a.M + kSdThreads * R - 1) / (kSdThreads * R);
+  dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(a.plan.splits),
+            static_cast<unsigned>(a.B));
+  sd_kernel<D, CP, LSE><<<grid, kSdThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D, bool LSE>
+cudaError_t launch_cp(const SdArgs& a, cudaStream_t s) {
+  switch (sd_chunk_pad(a.cw)) {
+    case 1: return launch_t<D, 1, LSE>(a, s);
+    case 2: return launch_t<D, 2, LSE>(a, s);
+    case 4: return launch_t<D, 4, LSE>(a, s);
+    default: return launch_t<D, 8, LSE>(a, s);
+  }
+}
+
+template <bool LSE>
+cudaError_t launch_d(const SdArgs& a, cudaStream_t s) {
+  switch (a.D) {
+    case 1: return launch_cp<1, LSE>(a, s);
+    case 2: return launch_cp<2, LSE>(a, s);
+    case 3: return launch_cp<3, LSE>(a, s);
+    case 4: return launch_cp<4, LSE>(a, s);
+    case 5: return launch_cp<5, LSE>(a, s);
+    case 6: return launch_cp<6, LSE>(a, s);
+    case 7: return launch_cp<7, LSE>(a, s);
+    case 8: return launch_cp<8, LSE>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// ------------------------------------------------------------------ combine
+__global__ void combine_sum_kernel(const float* __restrict__ part, int splits, int64_t total,
+                                   float* __restrict__ out) {
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float s = 0.f;
+    for (int k = 0; k < splits; ++k) s += part[k * total + e];
+    out[e] = s;
+  }
+}
+
+// ------------------------------------------------------------------ LSE finalisation
+// One warp per (batch, row).  Lane k holds split k's (shift, scaled sum); the
+// merge m = max m_k, l = sum_k l_k 2^(m_k - m) runs as a fixed xor-tree.
+// Rows whose merged l is below 2^-64 (terms may have been flushed to zero)
+// are recomputed from scratch with their own exact maximum.
+__device__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__global__ void lse_finalize_kernel(const LseFinalizeArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int64_t rows = a.B * a.M;
+  const float kTiny = 5.421010862427522e-20f;   // 2^-64
+  for (int64_t row = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
+       row < rows; row += warps_total) {
+    const int64_t b = row / a.M;
+    const int64_t i = row % a.M;
+    for (int c = 0; c < a.C; ++c) {
+      const int64_t e = row * a.C + c;
+      float mk = -INFINITY, lk = 0.f;
+      if (lane < a.splits) {
+        mk = a.part_m[lane * a.split_stride + e];
+        lk = a.part_l[lane * a.split_stride + e];
+      }
+      const float m = warp_max(mk);
+      const float contrib = (mk == -INFINITY) ? 0.f : lk * ex2(mk - m);
+      const float l = warp_sum(contrib);
+      float res;
+      if (!(l < kTiny)) {
+        res = (m + log2f(l)) * kLn2;
+      } else {
+        // exact per-row recompute: pass 1 maximum, pass 2 shifted sum
+        const float* xi = a.x + (b * a.M + i) * a.D;
+        float xs[kSdMaxD];
+        for (int k = 0; k < a.D; ++k) xs[k] = xi[k] * a.scale;
+        float mx = -INFINITY;
+        for (int64_t j = lane; j < a.N; j += 32) {
+          const float* yj = a.y + (b * a.N + j) * a.D;
+          float t = lg2(a.w[(b * a.N + j) * a.C + c]);
+          for (int k = 0; k < a.D; ++k) {
+            const float d = xs[k] - yj[k] * a.scale;
+            t = fmaf(-d, d, t);
+          }
+          mx = fmaxf(mx, t);
+        }
+        mx = warp_max(mx);
+        float outer = 0.f;
+        if (mx != -INFINITY) {
+          float inner = 0.f;
+          int n_in = 0;
+          for (int64_t j = lane; j < a.N; j += 32) {
+            const float* yj = a.y + (b * a.N + j) * a.D;
+            float t = lg2(a.w[(b * a.N + j) * a.C + c]);
+            for (int k = 0; k < a.D; ++k) {
+              const float d = xs[k] - yj[k] * a.scale;
+              t = fmaf(-d, d, t);
+            }
+            inner += ex2(t - mx);
+            if (++n_in == 64) {
+              outer += inner;
+              inner = 0.f;
+              n_in = 0;
+            }
+          }
+          outer += inner;
+        }
+        const float ls = warp_sum(outer);
+        res = (mx == -INFINITY) ? -INFINITY : (mx + log2f(ls)) * kLn2;
+      }
+      if (lane == 0) a.out[e] = res;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ backward helpers
+__global__ void pack_bwd_values_f32_kernel(const float* __restrict__ y,
+                                           const float* __restrict__ w, float* __restrict__ v,
+                                           int64_t rows, int D, int C) {
+  const int CV = C * (1 + D);
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+       e < rows * CV; e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t j = e / CV;
+    const int ch = static_cast<int>(e % CV);
+    float val;
+    if (ch < C) {
+      val = w[j * C + ch];
+    } else {
+      const int c = (ch - C) / D, k = (ch - C) % D;
+      val = w[j * C + c] * y[j * D + k];
+    }
+    v[e] = val;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
+  return __bfloat162float(v);
+}
+
+template <typename T>
+__global__ void grad_x_epilogue_kernel(const T* __restrict__ x, const float* __restrict__ g,
+                                       const float* __restrict__ o, float* __restrict__ gx,
+                                       int64_t rows, int D, int C, float tau) {
+  const int CV = C * (1 + D);
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < rows * D;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t i = e / D;
+    const int k = static_cast<int>(e % D);
+    const float xk = to_f32(x[e]);
+    const float* oi = o + i * CV;
+    const float* gi = g + i * C;
+    float s = 0.f;
+    for (int c = 0; c < C; ++c) s = fmaf(gi[c], fmaf(xk, oi[c], -oi[C + c * D + k]), s);
+    gx[e] = -tau * s;
+  }
+}
+
+__global__ void fill_kernel(float* __restrict__ out, int64_t n, float value) {
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    out[e] = value;
+}
+
+int grid_for(int64_t n, int threads) {
+  int64_t b = (n + threads - 1) / threads;
+  if (b < 1) b = 1;
+  if (b > 148 * 32) b = 148 * 32;
+  return static_cast<int>(b);
+}
+
+}  // namespace
+
+SdPlan sd_plan(int64_t B, int64_t M, int64_t N, int D, int64_t C, int sm_count) {
+  SdPlan p{};
+  const int cw = static_cast<int>(C < kSdMaxChunk ? C : kSdMaxChunk);
+  const int R = sd_rows_per_thread(D, sd_chunk_pad(cw));
+  p.rows_per_cta = kSdThreads * R;
+  const int64_t U = B * ((M + p.rows_per_cta - 1) / p.rows_per_cta);
+  int64_t smax = N / 256;
+  if (smax > 32) smax = 32;
+  if (smax < 1) smax = 1;
+  // cost ~ CTAs per SM (at least 4 to keep the MUFU pipe fed) x columns per CTA
+  const int64_t k_sat = 4;
+  int best = 1;
+  double best_cost = 1e300;
+  for (int64_t S = 1; S <= smax; ++S) {
+    int64_t per_sm = (U * S + sm_count - 1) / sm_count;
+    if (per_sm < k_sat) per_sm = k_sat;
+    const double cost = static_cast<double>(per_sm) * static_cast<double>((N + S - 1) / S + 64);
+    if (cost < best_cost * 0.999) {
+      best_cost = cost;
+      best = static_cast<int>(S);
+    }
+  }
+  p.splits = best;
+  p.cols_per_split = (N + best - 1) / best;
+  // keep every split non-empty
+  if (p.cols_per_split < 1) p.cols_per_split = 1;
+  p.splits = static_cast<int>((N + p.cols_per_split - 1) / p.cols_per_split);
+  if (p.splits < 1) p.splits = 1;
+  return p;
+}
+
+cudaError_t launch_small_d_sum(const SdArgs& a, cudaStream_t s) { return launch_d<false>(a, s); }
+cudaError_t launch_small_d_lse(const SdArgs& a, cudaStream_t s) { return launch_d<true>(a, s); }
+
+cudaError_t launch_combine_sum(const float* part, int splits, int64_t total, float* out,
+                               cudaStream_t s) {
+  combine_sum_kernel<<<grid_for(total, 256), 256, 0, s>>>(part, splits, total, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lse_finalize(const LseFinalizeArgs& a, cudaStream_t s) {
+  const int64_t rows = a.B * a.M;
+  int64_t blocks = (rows + 7) / 8;   // 8 warps per block
+  if (blocks > 148 * 64) blocks = 148 * 64;
+  if (blocks < 1) blocks = 1;
+  lse_finalize_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill(float* out, int64_t n, float value, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  fill_kernel<<<grid_for(n, 256), 256, 0, s>>>(out, n, value);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_bwd_values_f32(const float* y, const float* w, float* v, int64_t B,
+                                       int64_t N, int D, int C, cudaStream_t s) {
+  const int64_t n = B * N * C * (1 + D);
+  pack_bwd_values_f32_kernel<<<grid_for(n, 256), 256, 0, s>>>(y, w, v, B * N, D, C);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_grad_x_epilogue(const void* x, gs_dtype dt, const float* g,
+                                       const float* o, float* grad_x, int64_t B, int64_t M,
+                                       int D, int C, float tau, cudaStream_t s) {
+  const int64_t n = B * M * D;
+  const int blocks = grid_for(n, 256);
+  switch (dt) {
+    case GS_F32:
+      grad_x_epilogue_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(x), g, o,
+                                                           grad_x, B * M, D, C, tau);
+      break;
+    case GS_F16:
+      grad_x_epilogue_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<const __half*>(x), g, o,
+                                                            grad_x, B * M, D, C, tau);
+      break;
+    default:
+      grad_x_epilogue_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(x), g, o, grad_x, B * M, D, C, tau);
+      break;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace gs

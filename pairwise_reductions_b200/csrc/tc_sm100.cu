@@ -1,0 +1,618 @@
+// tc_sm100.cu -- tensor-core Gaussian kernel sum for fp16 / bf16 inputs
+// (1 <= D <= 126) on sm_100a: tcgen05 MMAs with TMEM accumulators, operands
+// staged by TMA, nothing of size M x N ever leaves the SM.
+//
+// The fold.  With c = tau/2 * log2 e,
+//     exp(-tau/2 |x_i - y_j|^2) = 2^(2c (x_i.y_j - |y_j|^2/2) - c |x_i|^2)
+// ("Fast Gauss Sums via Flash Attention", Algorithm 1: the two norm factors
+// exp(-tau/2 |q|^2) and exp(-tau/2 |k|^2) around a dot-product exponent).
+// The column norm is folded into the first MMA by augmenting the operands
+// (as Algorithm 2 of the same page augments q and k): x~ = [x, 1, 1, 0..],
+// y~ = [y, h, l, 0..] with h + l = -|y|^2/2 split over two fp16 (or bf16)
+// values so the augmented product keeps ~22 bits.  Then per pair
+//     P_ij = ex2(fma(S~_ij, 2c, r_i)),  S~ = x~ . y~,  r_i = -c |x_i|^2 + 14
+// is one FFMA and one MUFU ex2; the +14 (undone on output) keeps P in the
+// normal fp16 range down to kernel values of 2^-28.
+//
+// CTA = 256 rows (two 128-row MMA tiles) x one column split, 10 warps:
+//   warp 0      TMA producer: x~ tiles once, then a ring of (y~, v^T) stages
+//   warp 1      TMEM owner + single-thread MMA issuer
+//   warps 2-5   exp warpgroup of row tile 0 (TMEM lane quarters 2,3,0,1)
+//   warps 6-9   exp warpgroup of row tile 1
+// Per 128-column tile t and row tile h:
+//   S_h = x~_h . y~(t)^T        (tcgen05.mma, smem x smem -> TMEM fp32)
+//   P_h = ex2(fma(S_h, 2c, r))  (tcgen05.ld -> MUFU -> fp16 -> tcgen05.st)
+//   O_h += P_h . v(t)           (tcgen05.mma, A = P from TMEM, B = v^T smem)
+// The issue order S0(t+1) before O1(t) lets both exp warpgroups run at once.
+// Every mbarrier wait is bounded (2 s); on expiry the kernel raises the device
+// error word, lets the other warps leave, frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace gs {
+
+__device__ int g_device_error;
+
+namespace {
+
+constexpr int kBM = 128;   // rows per MMA tile
+constexpr int kBN = 128;   // columns per tile
+constexpr int kNT = 2;     // row tiles per CTA
+constexpr int kThreads = 320;
+constexpr float kPShift = 14.f;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct TcKParams {
+  const float* rnorm;   // [B, M]
+  float* out;
+  int64_t split_stride;
+  int64_t M, N;
+  int64_t ldo;          // row stride of out (floats)
+  int c0, cw;           // first output channel, channels written
+  int64_t cols_per_split;
+  float two_c;
+  float out_scale;
+};
+
+template <int KP, int CP>
+struct TcCfg {
+  static constexpr int KC = KP / 64;            // 128-byte swizzle atoms along K
+  static constexpr int ATOM = kBM * 128;        // one 128-row x 64-col block: 16 KB
+  static constexpr int X_BYTES = kNT * KC * ATOM;
+  static constexpr int Y_BYTES = KC * ATOM;
+  static constexpr int V_BYTES = 2 * CP * 128;  // two 64-column atoms of CP rows
+  static constexpr int STAGE = Y_BYTES + V_BYTES;
+  static constexpr int NST_FIT = (200 * 1024 - X_BYTES) / STAGE;
+  static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
+  static constexpr int NBARS = 2 * NST + 7;
+  static constexpr int SMEM_RAW = 1024 + X_BYTES + NST * STAGE + 8 * NBARS + 16;
+  // at least ~120 KB so that a second CTA never lands on the SM and blocks on
+  // the 512-column TMEM allocation
+  static constexpr int SMEM = SMEM_RAW < 122880 ? 122880 : SMEM_RAW;
+  // TMEM columns (512 allocated): S0 | S1 | O0 | O1 | P0 | P1.  When the value
+  // chunk is wider than 64 the fp16 P tiles overwrite the S tile they came
+  // from (the next S MMA is issued after the P MMA that reads it).
+  static constexpr bool P_SEPARATE = CP <= 64;
+  __host__ __device__ static constexpr uint32_t col_s(int h) { return 128u * h; }
+  __host__ __device__ static constexpr uint32_t col_o(int h) {
+    return 256u + (P_SEPARATE ? 64u : 128u) * h;
+  }
+  __host__ __device__ static constexpr uint32_t col_p(int h) {
+    return P_SEPARATE ? 384u + 64u * h : 128u * h;
+  }
+  static_assert(NST >= 2, "shared memory budget");
+  static_assert(CP % 16 == 0 && CP >= 16 && CP <= 128, "value chunk");
+};
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  uint32_t n = 0;
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((++n & 63u) == 0u) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        atomicOr(&g_device_error, 1);
+        return false;
+      }
+    }
+  }
+}
+
+template <int KP, int CP, int DTFMT>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_gauss_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+                    const __grid_constant__ CUtensorMap tmV, const TcKParams p) {
+  using Cfg = TcCfg<KP, CP>;
+  constexpr int NST = Cfg::NST;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sX = smem;
+  uint8_t* sStage = smem + Cfg::X_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + NST * Cfg::STAGE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NBARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const uint32_t bar0 = smem_u32(bars);
+  auto bar_full = [&](int s) { return bar0 + 8u * s; };
+  auto bar_empty = [&](int s) { return bar0 + 8u * (NST + s); };
+  const uint32_t bar_x = bar0 + 8u * (2 * NST);
+  auto bar_s = [&](int h) { return bar0 + 8u * (2 * NST + 1 + h); };   // S tile h ready
+  auto bar_p = [&](int h) { return bar0 + 8u * (2 * NST + 3 + h); };   // P tile h written
+  const uint32_t bar_o = bar0 + 8u * (2 * NST + 5);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t b = blockIdx.z;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * (kNT * kBM);
+  const int64_t jbeg = static_cast<int64_t>(blockIdx.y) * p.cols_per_split;
+  const int64_t jend = min(p.N, jbeg + p.cols_per_split);
+  const int T = (jend > jbeg) ? static_cast<int>((jend - jbeg + kBN - 1) / kBN) : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_empty(s), 1);
+    }
+    mbar_init(bar_x, 1);
+    mbar_init(bar_s(0), 1);
+    mbar_init(bar_s(1), 1);
+    mbar_init(bar_p(0), 4 * 32);
+    mbar_init(bar_p(1), 4 * 32);
+    mbar_init(bar_o, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmX);
+      tma_prefetch_desc(&tmY);
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(bar_x, Cfg::X_BYTES);
+      for (int h = 0; h < kNT; ++h)
+        for (int kc = 0; kc < Cfg::KC; ++kc)
+          tma_load_3d(smem_u32(sX + (h * Cfg::KC + kc) * Cfg::ATOM), &tmX, bar_x, kc * 64,
+                      static_cast<int>(row0 + h * kBM), static_cast<int>(b));
+      for (int t = 0; t < T; ++t) {
+        const int st = t % NST;
+        if (t >= NST && !wait_bar(bar_empty(st), ((t / NST) - 1) & 1, abort_flag)) break;
+        uint8_t* sy = sStage + st * Cfg::STAGE;
+        uint8_t* sv = sy + Cfg::Y_BYTES;
+        const int j0 = static_cast<int>(jbeg + static_cast<int64_t>(t) * kBN);
+        mbar_arrive_expect_tx(bar_full(st), Cfg::STAGE);
+        for (int kc = 0; kc < Cfg::KC; ++kc)
+          tma_load_3d(smem_u32(sy + kc * Cfg::ATOM), &tmY, bar_full(st), kc * 64, j0,
+                      static_cast<int>(b));
+        for (int hh = 0; hh < 2; ++hh)
+          tma_load_3d(smem_u32(sv + hh * CP * 128), &tmV, bar_full(st), j0 + hh * 64, 0,
+                      static_cast<int>(b));
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idS = idesc_f16(DTFMT, kBM, kBN);
+      const uint32_t idO = idesc_f16(0, kBM, CP);
+      auto issue_S = [&](int h, int st) {
+        const uint8_t* sy = sStage + st * Cfg::STAGE;
+#pragma unroll
+        for (int ks = 0; ks < KP / 16; ++ks) {
+          const int kc = ks >> 2, kw = ks & 3;
+          const uint64_t ad = desc_k_sw128(smem_u32(sX + (h * Cfg::KC + kc) * Cfg::ATOM) + kw * 32);
+          const uint64_t bd = desc_k_sw128(smem_u32(sy + kc * Cfg::ATOM) + kw * 32);
+          mma_ss(tmem + Cfg::col_s(h), ad, bd, idS, ks > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_O = [&](int h, int st, bool acc_prev) {
+        const uint8_t* sv = sStage + st * Cfg::STAGE + Cfg::Y_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < kBN / 16; ++ks) {
+          const int kc = ks >> 2, kw = ks & 3;
+          const uint64_t bd = desc_k_sw128(smem_u32(sv + kc * CP * 128) + kw * 32);
+          mma_ts(tmem + Cfg::col_o(h), tmem + Cfg::col_p(h) + ks * 8, bd, idO,
+                 (acc_prev || ks > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = wait_bar(bar_x, 0, abort_flag);
+      if (ok && T > 0) {
+        ok = wait_bar(bar_full(0), 0, abort_flag);
+        if (ok) {
+          tc_fence_after();
+          issue_S(0, 0);
+          mma_commit(bar_s(0));
+          issue_S(1, 0);
+          mma_commit(bar_s(1));
+        }
+      }
+      for (int t = 0; ok && t < T; ++t) {
+        const int st = t % NST;
+        const int st1 = (t + 1) % NST;
+        if (!(ok = wait_bar(bar_p(0), t & 1, abort_flag))) break;
+        tc_fence_after();
+        issue_O(0, st, t > 0);
+        if (t + 1 < T) {
+          if (!(ok = wait_bar(bar_full(st1), ((t + 1) / NST) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_S(0, st1);
+          mma_commit(bar_s(0));
+        }
+        if (!(ok = wait_bar(bar_p(1), t & 1, abort_flag))) break;
+        tc_fence_after();
+        issue_O(1, st, t > 0);
+        mma_commit(bar_empty(st));
+        if (t + 1 < T) {
+          issue_S(1, st1);
+          mma_commit(bar_s(1));
+        }
+      }
+      mma_commit(bar_o);   // also the drain point for whatever was issued
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ exp warpgroups
+    const int h = (warp - 2) >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int64_t i = row0 + h * kBM + row;
+    const bool valid = i < p.M;
+    const float r = valid ? p.rnorm[b * p.M + i] : 0.f;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_base + Cfg::col_s(h);
+    const uint32_t tP = tmem + lane_base + Cfg::col_p(h);
+    const uint32_t tO = tmem + lane_base + Cfg::col_o(h);
+    const float two_c = p.two_c;
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      ok = wait_bar(bar_s(h), t & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int ch = 0; ch < kBN / 32; ++ch) {
+        uint32_t v[32];
+        tmem_ld32(tS + ch * 32, v);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const float e0 = ex2(fmaf(__uint_as_float(v[2 * q]), two_c, r));
+          const float e1 = ex2(fmaf(__uint_as_float(v[2 * q + 1]), two_c, r));
+          pk[q] = pack_f16x2(e0, e1);
+        }
+        tmem_st16(tP + ch * 16, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_p(h));
+    }
+    if (ok) ok = wait_bar(bar_o, 0, abort_flag);
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+    if (ok) {
+      float* orow = p.out + static_cast<int64_t>(blockIdx.y) * p.split_stride +
+                    (b * p.M + i) * p.ldo + p.c0;
+#pragma unroll
+      for (int ch = 0; ch < CP / 16; ++ch) {
+        uint32_t v[16];
+        tmem_ld16(tO + ch * 16, v);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const int c = ch * 16 + q;
+            if (c < p.cw) orow[c] = (T > 0) ? __uint_as_float(v[q]) * p.out_scale : 0.f;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ packing prologue
+template <typename T>
+__device__ __forceinline__ float tof(T v);
+template <>
+__device__ __forceinline__ float tof<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float tof<__half>(__half v) { return __half2float(v); }
+template <>
+__device__ __forceinline__ float tof<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T>
+__device__ __forceinline__ T fromf(float v);
+template <>
+__device__ __forceinline__ __half fromf<__half>(float v) { return __float2half_rn(v); }
+template <>
+__device__ __forceinline__ __nv_bfloat16 fromf<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+__device__ __forceinline__ uint16_t bits16(__half v) { return __half_as_ushort(v); }
+__device__ __forceinline__ uint16_t bits16(__nv_bfloat16 v) { return __bfloat16_as_ushort(v); }
+
+// Packed operand rows.  Row side (is_x): [x, 1, 1, 0 ...] and
+// rnorm = -c |x|^2 + shift.  Column side: [y, h, l, 0 ...] with h + l = -|y|^2/2.
+// A group of KP/8 consecutive threads builds one row, 8 elements (16 bytes) each.
+template <typename T, int KP>
+__global__ void pack_rows_kernel(const T* __restrict__ src, T* __restrict__ dst,
+                                 float* __restrict__ rnorm, int64_t rows, int D, float c,
+                                 float shift, int is_x) {
+  constexpr int G = KP / 8;   // threads per row (8 or 16), a power of two dividing 32
+  const int64_t gt = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const int64_t row = gt / G;
+  const int part = static_cast<int>(gt % G);
+  const bool live = row < rows;
+  float vals[8];
+  float sq = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int k = part * 8 + e;
+    float v = 0.f;
+    if (live && k < D) v = tof(src[row * D + k]);
+    vals[e] = v;
+    sq = fmaf(v, v, sq);
+  }
+#pragma unroll
+  for (int o = G / 2; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o, G);
+  if (!live) return;
+  float aug0, aug1;
+  if (is_x) {
+    aug0 = 1.f;
+    aug1 = 1.f;
+  } else {
+    const float hn = -0.5f * sq;
+    aug0 = tof(fromf<T>(hn));
+    aug1 = hn - aug0;
+  }
+  uint32_t packed[4];
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    float v0 = vals[e], v1 = vals[e + 1];
+    const int k = part * 8 + e;
+    if (k == D) v0 = aug0;
+    if (k == D + 1) v0 = aug1;
+    if (k + 1 == D) v1 = aug0;
+    if (k + 1 == D + 1) v1 = aug1;
+    packed[e / 2] = static_cast<uint32_t>(bits16(fromf<T>(v0))) |
+                    (static_cast<uint32_t>(bits16(fromf<T>(v1))) << 16);
+  }
+  *reinterpret_cast<uint4*>(dst + row * KP + part * 8) =
+      make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  if (is_x && part == 0) rnorm[row] = fmaf(-c, sq, shift);
+}
+
+// Transposed fp16 value matrix v^T [B, CP, Nst] for channels [c0, c0 + CP) of
+// either v = w (kValuesW) or v = [w, w (x) y] (kValuesBwd).  Channels past CV
+// are written as zeros.
+template <typename TW, typename TY>
+__global__ void pack_values_kernel(const TW* __restrict__ w, const TY* __restrict__ y,
+                                   __half* __restrict__ vt, int64_t B, int64_t N, int64_t Nst,
+                                   int C, int D, int CV, int c0, int CP, int bwd) {
+  const int64_t total = B * CP * N;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t j = e % N;
+    const int64_t bc = e / N;
+    const int cc = static_cast<int>(bc % CP);
+    const int64_t b = bc / CP;
+    const int ch = c0 + cc;
+    float v = 0.f;
+    if (ch < CV) {
+      const int64_t bj = b * N + j;
+      if (!bwd || ch < C) {
+        v = tof(w[bj * C + ch]);
+      } else {
+        const int cw = (ch - C) / D, k = (ch - C) % D;
+        v = tof(w[bj * C + cw]) * tof(y[bj * D + k]);
+      }
+    }
+    vt[(b * CP + cc) * Nst + j] = __float2half_rn(v);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn get_encode() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(ptr);
+  });
+  return fn;
+}
+
+bool make_tmap_3d(CUtensorMap* m, CUtensorMapDataType dt, void* base, uint64_t d0, uint64_t d1,
+                  uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0,
+                  uint32_t box1) {
+  EncodeFn enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  const cuuint32_t box[3] = {box0, box1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, dt, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int grid_for(int64_t n, int threads) {
+  int64_t b = (n + threads - 1) / threads;
+  if (b < 1) b = 1;
+  if (b > 148 * 32) b = 148 * 32;
+  return static_cast<int>(b);
+}
+
+template <typename T>
+cudaError_t pack_operands(const TcArgs& a, cudaStream_t s) {
+  const float c = 0.5f * a.tau * kLog2e;
+  const int KP = a.plan.KP;
+  auto launch_rows = [&](const void* src, void* dst, float* rn, int64_t rows, int is_x) {
+    const int64_t threads_total = rows * (KP / 8);
+    const int blocks = static_cast<int>((threads_total + 255) / 256);
+    if (KP == 64)
+      pack_rows_kernel<T, 64><<<blocks, 256, 0, s>>>(static_cast<const T*>(src),
+                                                     static_cast<T*>(dst), rn, rows, a.D, c,
+                                                     kPShift, is_x);
+    else
+      pack_rows_kernel<T, 128><<<blocks, 256, 0, s>>>(static_cast<const T*>(src),
+                                                      static_cast<T*>(dst), rn, rows, a.D, c,
+                                                      kPShift, is_x);
+  };
+  launch_rows(a.x, a.xpack, a.rnorm, a.B * a.M, 1);
+  launch_rows(a.y, a.ypack, nullptr, a.B * a.N, 0);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t pack_values(const TcArgs& a, int c0, int CP, int64_t Nst, cudaStream_t s) {
+  const int64_t total = a.B * CP * a.N;
+  const int blocks = grid_for(total, 256);
+  const int bwd = a.values == kValuesBwd ? 1 : 0;
+  if (a.w_is_f32)
+    pack_values_kernel<float, T><<<blocks, 256, 0, s>>>(
+        static_cast<const float*>(a.w), static_cast<const T*>(a.y), static_cast<__half*>(a.vt),
+        a.B, a.N, Nst, a.C, a.D, a.CV, c0, CP, bwd);
+  else
+    pack_values_kernel<T, T><<<blocks, 256, 0, s>>>(
+        static_cast<const T*>(a.w), static_cast<const T*>(a.y), static_cast<__half*>(a.vt), a.B,
+        a.N, Nst, a.C, a.D, a.CV, c0, CP, bwd);
+  return cudaGetLastError();
+}
+
+template <int KP, int CP, int DTFMT>
+cudaError_t launch_kernel(const CUtensorMap& tx, const CUtensorMap& ty, const CUtensorMap& tv,
+                          const TcKParams& kp, dim3 grid, cudaStream_t s) {
+  using Cfg = TcCfg<KP, CP>;
+  auto fn = tc_gauss_kernel<KP, CP, DTFMT>;
+  static bool attr_done = false;   // idempotent; a benign race at worst repeats the call
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  fn<<<grid, kThreads, Cfg::SMEM, s>>>(tx, ty, tv, kp);
+  return cudaGetLastError();
+}
+
+template <int KP, int DTFMT>
+cudaError_t launch_cp(int CP, const CUtensorMap& tx, const CUtensorMap& ty, const CUtensorMap& tv,
+                      const TcKParams& kp, dim3 grid, cudaStream_t s) {
+  switch (CP) {
+    case 16: return launch_kernel<KP, 16, DTFMT>(tx, ty, tv, kp, grid, s);
+    case 32: return launch_kernel<KP, 32, DTFMT>(tx, ty, tv, kp, grid, s);
+    case 48: return launch_kernel<KP, 48, DTFMT>(tx, ty, tv, kp, grid, s);
+    case 64: return launch_kernel<KP, 64, DTFMT>(tx, ty, tv, kp, grid, s);
+    case 96: return launch_kernel<KP, 96, DTFMT>(tx, ty, tv, kp, grid, s);
+    default: return launch_kernel<KP, 128, DTFMT>(tx, ty, tv, kp, grid, s);
+  }
+}
+
+int cp_for(int cw) {
+  const int c16 = (cw + 15) / 16 * 16;
+  if (c16 <= 64) return c16 == 0 ? 16 : c16;
+  return c16 <= 96 ? 96 : 128;
+}
+
+}  // namespace
+
+TcPlan tc_plan(int64_t B, int64_t M, int64_t N, int64_t D, int sm_count) {
+  TcPlan p{};
+  p.KP = (D + 2 <= 64) ? 64 : 128;
+  const int64_t U = B * ((M + kNT * kBM - 1) / (kNT * kBM));
+  const int64_t ntj = (N + kBN - 1) / kBN;
+  int64_t smax = ntj / 4;
+  if (smax > 32) smax = 32;
+  if (smax < 1) smax = 1;
+  int best = 1;
+  double best_cost = 1e300;
+  for (int64_t S = 1; S <= smax; ++S) {
+    const int64_t waves = (U * S + sm_count - 1) / sm_count;
+    const double cost = static_cast<double>(waves) * static_cast<double>((ntj + S - 1) / S + 3);
+    if (cost < best_cost * 0.999) {
+      best_cost = cost;
+      best = static_cast<int>(S);
+    }
+  }
+  const int64_t tiles_per_split = (ntj + best - 1) / best;
+  p.cols_per_split = (tiles_per_split < 1 ? 1 : tiles_per_split) * kBN;
+  p.splits = static_cast<int>((N + p.cols_per_split - 1) / p.cols_per_split);
+  if (p.splits < 1) p.splits = 1;
+  return p;
+}
+
+cudaError_t launch_tc_sum(const TcArgs& a, cudaStream_t s) {
+  if (a.B == 0 || a.M == 0) return cudaSuccess;
+  const bool bf = a.dt == GS_BF16;
+  cudaError_t e = bf ? pack_operands<__nv_bfloat16>(a, s) : pack_operands<__half>(a, s);
+  if (e != cudaSuccess) return e;
+  const int KP = a.plan.KP;
+  const CUtensorMapDataType tdt = bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUtensorMap tx, ty;
+  if (!make_tmap_3d(&tx, tdt, a.xpack, KP, a.M, a.B, KP * 2ull, a.M * KP * 2ull, 64, kBM) ||
+      !make_tmap_3d(&ty, tdt, a.ypack, KP, a.N, a.B, KP * 2ull, a.N * KP * 2ull, 64, kBN))
+    return cudaErrorInvalidValue;
+  const int64_t Nst = (a.N + 7) / 8 * 8;
+  const dim3 grid(static_cast<unsigned>((a.M + kNT * kBM - 1) / (kNT * kBM)),
+                  static_cast<unsigned>(a.plan.splits), static_cast<unsigned>(a.B));
+  for (int c0 = 0; c0 < a.CV; c0 += kTcMaxChunk) {
+    const int cw = (a.CV - c0) < kTcMaxChunk ? (a.CV - c0) : kTcMaxChunk;
+    const int CP = cp_for(cw);
+    e = bf ? pack_values<__nv_bfloat16>(a, c0, CP, Nst, s) : pack_values<__half>(a, c0, CP, Nst, s);
+    if (e != cudaSuccess) return e;
+    CUtensorMap tv;
+    if (!make_tmap_3d(&tv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.vt, a.N, CP, a.B, Nst * 2ull,
+                      CP * Nst * 2ull, 64, CP))
+      return cudaErrorInvalidValue;
+    TcKParams kp{};
+    kp.rnorm = a.rnorm;
+    kp.out = a.out;
+    kp.split_stride = a.split_stride;
+    kp.M = a.M;
+    kp.N = a.N;
+    kp.ldo = a.CV;
+    kp.c0 = c0;
+    kp.cw = cw;
+    kp.cols_per_split = a.plan.cols_per_split;
+    kp.two_c = a.tau * kLog2e;
+    kp.out_scale = exp2f(-kPShift);
+    if (KP == 64)
+      e = bf ? launch_cp<64, 1>(CP, tx, ty, tv, kp, grid, s) : launch_cp<64, 0>(CP, tx, ty, tv, kp, grid, s);
+    else
+      e = bf ? launch_cp<128, 1>(CP, tx, ty, tv, kp, grid, s) : launch_cp<128, 0>(CP, tx, ty, tv, kp, grid, s);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t read_and_clear_device_error(int* value) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  *value = v;
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+  }
+  return e;
+}
+
+}  // namespace gs

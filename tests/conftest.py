@@ -27,3 +27,17 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(autouse=True)
+def _device_error_word_stays_clear(request):
+    """After every GPU test, the library's device error word must be clear
+    (a set word means a kernel gave up on a bounded wait)."""
+    yield
+    if "gpu" not in request.keywords:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    import pairwise_reductions_b200 as gs
+    assert gs.last_device_error() == 0, "device error word set (a bounded wait timed out)"

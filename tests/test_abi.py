@@ -1,0 +1,105 @@
+"""The C ABI library loads, exports every symbol include/gauss.h declares, and
+rejects bad arguments on the host -- all without a GPU (no compute call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import pairwise_reductions_b200 as gs
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "gauss.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", text)) - {"if", "sizeof"})
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for n in ("gauss_sum_fwd", "gauss_lse_fwd", "gauss_sum_bwd", "gs_workspace_bytes",
+              "gs_status_string", "gs_last_device_error", "gs_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(gs.LIB_PATH)
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, f"declared in gauss.h but not exported: {missing}"
+    # and the binding binds exactly those names
+    assert set(gs.SIGNATURES) == set(_declared_functions())
+
+
+def test_status_strings_and_version():
+    for code in range(7):
+        assert gs.status_string(code)
+    assert gs.library().gs_version() >= 100
+
+
+NULL = ctypes.c_void_p(0)
+FAKE = ctypes.c_void_p(0x100000)   # 16-byte aligned, never dereferenced on these paths
+ODD = ctypes.c_void_p(0x100004)
+
+
+def _fwd(fn="gauss_sum_fwd", x=FAKE, y=FAKE, w=FAKE, out=FAKE, B=1, M=10, N=10, D=3, C=1, tau=1.0,
+         dt=0, ws=NULL, wsb=0):
+    return getattr(gs.library(), fn)(x, y, w, out, B, M, N, D, C, tau, dt, ws, wsb, NULL)
+
+
+@pytest.mark.parametrize("fn", ["gauss_sum_fwd", "gauss_lse_fwd"])
+def test_invalid_arguments_are_rejected_before_any_launch(fn):
+    assert _fwd(fn, x=NULL) == 1
+    assert _fwd(fn, out=NULL) == 1
+    assert _fwd(fn, tau=0.0) == 1
+    assert _fwd(fn, tau=-1.0) == 1
+    assert _fwd(fn, tau=float("nan")) == 1
+    assert _fwd(fn, tau=float("inf")) == 1
+    assert _fwd(fn, M=-1) == 1
+    assert _fwd(fn, D=0) == 1
+    assert _fwd(fn, C=0) == 1
+    assert _fwd(fn, dt=7) == 1
+    assert _fwd(fn, x=ODD) == 3
+    assert _fwd(fn, D=9) == 2              # fp32 path covers D <= 8
+    assert _fwd(fn, dt=1, D=127) == 2      # tensor-core path covers D <= 126
+    assert _fwd(fn, B=70000) == 2
+
+
+def test_lse_has_no_half_precision_path():
+    assert _fwd("gauss_lse_fwd", dt=1, D=32) == 2
+
+
+def test_empty_problems_are_no_ops_without_pointers():
+    assert _fwd(x=NULL, y=NULL, w=NULL, out=NULL, B=0) == 0
+    assert _fwd(x=NULL, out=NULL, M=0) == 0
+
+
+def test_workspace_too_small_is_reported():
+    # tensor-core path always needs packed operands in the workspace
+    assert _fwd(dt=1, D=32, C=32, M=1000, N=1000) == 4
+
+
+def test_workspace_query():
+    ws = gs.workspace_bytes
+    assert ws(gs.GS_OP_SUM, 0, 10, 10, 3, 1, gs.GS_F32) == 0
+    assert ws(gs.GS_OP_SUM, 1, 10, 0, 3, 1, gs.GS_F32) == 0
+    big = ws(gs.GS_OP_SUM, 4, 65536, 65536, 32, 32, gs.GS_F16)
+    # packed x~ and y~ (2 x 4 x 65536 x 64 x 2 B) + v^T (4 x 32 x 65536 x 2 B) at least
+    assert big >= 2 * 4 * 65536 * 64 * 2 + 4 * 32 * 65536 * 2
+    assert ws(gs.GS_OP_LSE, 1, 1000, 1000, 3, 1, gs.GS_F32) >= 2 * 1000 * 4
+    assert ws(gs.GS_OP_SUM_BWD, 4, 16384, 16384, 32, 1, gs.GS_F16) >= 4 * 16384 * 33 * 4
+    with pytest.raises(ValueError):
+        ws(gs.GS_OP_SUM, 1, 10, 10, 9, 1, gs.GS_F32)
+    with pytest.raises(ValueError):
+        ws(7, 1, 10, 10, 3, 1, gs.GS_F32)
+
+
+def test_bwd_argument_checks():
+    lib = gs.library()
+    args = lambda **k: (k.get("x", FAKE), FAKE, FAKE, k.get("g", FAKE), k.get("gx", FAKE),
+                        k.get("gw", FAKE), 1, 10, 10, 3, 1, k.get("tau", 1.0), 0, NULL, 0, NULL)
+    assert lib.gauss_sum_bwd(*args(g=NULL)) == 1
+    assert lib.gauss_sum_bwd(*args(tau=0.0)) == 1
+    assert lib.gauss_sum_bwd(*args(gx=ODD)) == 3
+    assert lib.gauss_sum_bwd(*args(gx=NULL, gw=NULL)) == 0   # nothing requested

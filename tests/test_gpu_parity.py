@@ -1,0 +1,239 @@
+"""CUDA path against the CPU oracle, element by element, on the same seeded
+inputs, through the C ABI (via the ctypes binding).
+
+Tolerances (relative L2 over the compared outputs): 1e-5 for float32 inputs,
+3e-3 for float16 / bfloat16 inputs with float32 accumulation.  Full-size
+workloads run on the GPU in the launch configuration the benchmark times and
+are compared on seeded row samples the oracle evaluates one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-5, "f16": 3e-3, "bf16": 3e-3}
+
+
+def gs():
+    import pairwise_reductions_b200 as m
+    return m
+
+
+def rel_l2(a, b):
+    a = np.asarray(a, dtype=np.float64).ravel()
+    b = np.asarray(b, dtype=np.float64).ravel()
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def dev(inp):
+    return {k: inp[k].cuda() for k in ("x", "y", "w", "g") if k in inp}
+
+
+def f64(inp, k):
+    return synth.as_f64(inp[k])
+
+
+# ------------------------------------------------------------------ the five workloads
+def test_d3_10k_full():
+    inp = synth.make_inputs(1)
+    d = dev(inp)
+    out = gs().gauss_sum_fwd(d["x"], d["y"], d["w"], inp["tau"]).cpu().numpy()
+    ref = oracle.gauss_sum(f64(inp, "x"), f64(inp, "y"), f64(inp, "w"), inp["tau"])
+    assert rel_l2(out, ref) <= TOL["f32"], rel_l2(out, ref)
+
+
+def test_d3_100k_sampled_rows():
+    inp = synth.make_inputs(2)
+    d = dev(inp)
+    out = gs().gauss_sum_fwd(d["x"], d["y"], d["w"], inp["tau"]).cpu().numpy()
+    rows = synth.sample_rows(inp["M"], 3000, seed=7).numpy()
+    ref = oracle.gauss_sum(f64(inp, "x"), f64(inp, "y"), f64(inp, "w"), inp["tau"], rows=rows)
+    assert rel_l2(out[:, rows], ref) <= TOL["f32"], rel_l2(out[:, rows], ref)
+
+
+def test_d3_1m_sum_and_lse_sampled_rows():
+    inp = synth.make_inputs(3)
+    d = dev(inp)
+    rows = synth.sample_rows(inp["M"], 768, seed=8).numpy()
+    x, y, w = f64(inp, "x"), f64(inp, "y"), f64(inp, "w")
+    out = gs().gauss_sum_fwd(d["x"], d["y"], d["w"], inp["tau"]).cpu().numpy()
+    ref = oracle.gauss_sum(x, y, w, inp["tau"], rows=rows)
+    assert rel_l2(out[:, rows], ref) <= TOL["f32"], rel_l2(out[:, rows], ref)
+    lse = gs().gauss_lse_fwd(d["x"], d["y"], d["w"], inp["tau"]).cpu().numpy()
+    ref_l = oracle.gauss_lse(x, y, w, inp["tau"], rows=rows)
+    assert rel_l2(lse[:, rows], ref_l) <= TOL["f32"], rel_l2(lse[:, rows], ref_l)
+    # the stricter check: exp(lse) against exp(oracle lse) is a relative check of the sum
+    assert rel_l2(np.exp(lse[:, rows]), np.exp(ref_l)) <= TOL["f32"]
+
+
+def test_d32_c32_f16_sampled_rows():
+    inp = synth.make_inputs(4)
+    d = dev(inp)
+    out = gs().gauss_sum_fwd(d["x"], d["y"], d["w"], inp["tau"]).cpu().numpy()
+    rows = synth.sample_rows(inp["M"], 160, seed=9).numpy()
+    ref = oracle.gauss_sum(f64(inp, "x"), f64(inp, "y"), f64(inp, "w"), inp["tau"], rows=rows)
+    assert rel_l2(out[:, rows], ref) <= TOL["f16"], rel_l2(out[:, rows], ref)
+
+
+def test_d32_c1_f16_fwd_bwd_sampled():
+    inp = synth.make_inputs(5)
+    d = dev(inp)
+    x, y, w, g = (f64(inp, k) for k in "xywg")
+    out = gs().gauss_sum_fwd(d["x"], d["y"], d["w"], inp["tau"]).cpu().numpy()
+    gx, gw = gs().gauss_sum_bwd(d["x"], d["y"], d["w"], d["g"], inp["tau"])
+    gx, gw = gx.cpu().numpy(), gw.cpu().numpy()
+    rows = synth.sample_rows(inp["M"], 512, seed=10).numpy()
+    wrows = synth.sample_rows(inp["N"], 512, seed=11).numpy()
+    ref = oracle.gauss_sum(x, y, w, inp["tau"], rows=rows)
+    assert rel_l2(out[:, rows], ref) <= TOL["f16"], rel_l2(out[:, rows], ref)
+    rgx, rgw = oracle.gauss_sum_bwd(x, y, w, g, inp["tau"], rows=rows, wrows=wrows)
+    assert rel_l2(gx[:, rows], rgx) <= TOL["f16"], rel_l2(gx[:, rows], rgx)
+    assert rel_l2(gw[:, wrows], rgw) <= TOL["f16"], rel_l2(gw[:, wrows], rgw)
+
+
+# ------------------------------------------------------------------ odd shapes, both paths
+F32_SHAPES = [  # B, M, N, D, C
+    (1, 1, 1, 3, 1), (1, 1, 777, 3, 1), (1, 777, 1, 3, 1), (2, 777, 1301, 3, 1),
+    (1, 513, 257, 1, 2), (1, 1000, 999, 5, 3), (1, 300, 2000, 8, 9), (3, 129, 4097, 2, 4),
+    (1, 2049, 3000, 7, 8), (2, 100, 600, 4, 16),
+]
+HALF_SHAPES = [
+    (1, 1, 1, 32, 1), (1, 1, 300, 32, 1), (2, 300, 1000, 32, 32), (1, 257, 129, 16, 33),
+    (1, 200, 700, 5, 1), (1, 100, 300, 100, 16), (2, 130, 260, 48, 130), (1, 511, 640, 62, 64),
+    (1, 70, 1200, 63, 3), (1, 129, 257, 126, 96),
+]
+
+
+@pytest.mark.parametrize("shape", F32_SHAPES, ids=[str(s) for s in F32_SHAPES])
+def test_f32_odd_shapes(shape):
+    B, M, N, D, C = shape
+    inp = synth.make_inputs(1, seed=hash(shape) % 1000, B=B, M=M, N=N, D=D, C=C)
+    d = dev(inp)
+    out = gs().gauss_sum_fwd(d["x"], d["y"], d["w"], inp["tau"]).cpu().numpy()
+    ref = oracle.gauss_sum(f64(inp, "x"), f64(inp, "y"), f64(inp, "w"), inp["tau"])
+    assert rel_l2(out, ref) <= TOL["f32"], rel_l2(out, ref)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("shape", HALF_SHAPES, ids=[str(s) for s in HALF_SHAPES])
+def test_half_odd_shapes(shape, dtype):
+    B, M, N, D, C = shape
+    inp = synth.make_inputs(4, seed=hash(shape) % 1000, B=B, M=M, N=N, D=D, C=C, dtype=dtype)
+    d = dev(inp)
+    out = gs().gauss_sum_fwd(d["x"], d["y"], d["w"], inp["tau"]).cpu().numpy()
+    ref = oracle.gauss_sum(f64(inp, "x"), f64(inp, "y"), f64(inp, "w"), inp["tau"])
+    assert rel_l2(out, ref) <= TOL[dtype], rel_l2(out, ref)
+
+
+@pytest.mark.parametrize("shape", [(1, 700, 900, 3, 1), (2, 300, 1100, 2, 3), (1, 64, 5000, 8, 9)])
+def test_lse_f32_shapes(shape):
+    B, M, N, D, C = shape
+    inp = synth.make_inputs(3, seed=5, B=B, M=M, N=N, D=D, C=C)
+    d = dev(inp)
+    out = gs().gauss_lse_fwd(d["x"], d["y"], d["w"], inp["tau"]).cpu().numpy()
+    ref = oracle.gauss_lse(f64(inp, "x"), f64(inp, "y"), f64(inp, "w"), inp["tau"])
+    assert rel_l2(out, ref) <= TOL["f32"], rel_l2(out, ref)
+    assert rel_l2(np.exp(out), np.exp(ref)) <= TOL["f32"]
+
+
+def test_lse_rows_far_from_every_point():
+    """Rows whose every kernel value underflows fp32 take the exact per-row
+    recompute; the result must still match the oracle's shifted evaluation."""
+    inp = synth.make_inputs(3, seed=6, M=300, N=2000)
+    x = inp["x"].clone()
+    x[0, :50] += 5.0           # 5 units away from the unit cube, tau = 100: exp(-1250) ~ 0
+    inp["x"] = x
+    d = dev(inp)
+    out = gs().gauss_lse_fwd(d["x"], d["y"], d["w"], inp["tau"]).cpu().numpy()
+    ref = oracle.gauss_lse(f64(inp, "x"), f64(inp, "y"), f64(inp, "w"), inp["tau"])
+    assert np.isfinite(out).all()
+    assert rel_l2(out, ref) <= TOL["f32"], rel_l2(out, ref)
+
+
+@pytest.mark.parametrize("dtype,shape", [
+    ("f32", (1, 500, 700, 3, 1)), ("f32", (2, 300, 400, 2, 3)), ("f32", (1, 200, 300, 8, 2)),
+    ("f16", (1, 300, 500, 32, 1)), ("f16", (2, 257, 300, 16, 4)), ("bf16", (1, 200, 333, 32, 1)),
+])
+def test_bwd_shapes(dtype, shape):
+    B, M, N, D, C = shape
+    wid = 1 if dtype == "f32" else 5
+    inp = synth.make_inputs(wid, seed=12, B=B, M=M, N=N, D=D, C=C, dtype=dtype, with_g=True)
+    d = dev(inp)
+    gx, gw = gs().gauss_sum_bwd(d["x"], d["y"], d["w"], d["g"], inp["tau"])
+    rgx, rgw = oracle.gauss_sum_bwd(*(f64(inp, k) for k in "xywg"), inp["tau"])
+    assert rel_l2(gx.cpu().numpy(), rgx) <= TOL[dtype], rel_l2(gx.cpu().numpy(), rgx)
+    assert rel_l2(gw.cpu().numpy(), rgw) <= TOL[dtype], rel_l2(gw.cpu().numpy(), rgw)
+
+
+# ------------------------------------------------------------------ edge cases
+def test_empty_inputs():
+    m = gs()
+    x = torch.randn(1, 5, 3, device="cuda")
+    y = torch.empty(1, 0, 3, device="cuda")
+    w = torch.empty(1, 0, 2, device="cuda")
+    assert torch.equal(m.gauss_sum_fwd(x, y, w, 1.0), torch.zeros(1, 5, 2, device="cuda"))
+    lse = m.gauss_lse_fwd(x, y, w, 1.0)
+    assert torch.isneginf(lse).all()
+    x0 = torch.empty(1, 0, 3, device="cuda")
+    yy, ww = torch.randn(1, 4, 3, device="cuda"), torch.randn(1, 4, 2, device="cuda")
+    assert m.gauss_sum_fwd(x0, yy, ww, 1.0).shape == (1, 0, 2)
+    xh = torch.randn(2, 5, 32, device="cuda", dtype=torch.float16)
+    yh = torch.empty(2, 0, 32, device="cuda", dtype=torch.float16)
+    wh = torch.empty(2, 0, 4, device="cuda", dtype=torch.float16)
+    assert torch.equal(m.gauss_sum_fwd(xh, yh, wh, 1.0), torch.zeros(2, 5, 4, device="cuda"))
+    gx, gw = m.gauss_sum_bwd(xh, yh, wh, torch.randn(2, 5, 4, device="cuda"), 1.0)
+    assert torch.equal(gx, torch.zeros_like(gx)) and gw.shape == (2, 0, 4)
+
+
+def test_coincident_points_give_the_weight_sum():
+    m = gs()
+    x = torch.tensor([[[0.5, -1.0, 2.0]]], device="cuda")
+    y = x.repeat(1, 1000, 1)
+    w = torch.randn(1, 1000, 1, device="cuda", generator=torch.Generator("cuda").manual_seed(3))
+    out = m.gauss_sum_fwd(x, y, w, 2.0)
+    assert abs(out.item() - w.double().sum().item()) <= 1e-5 * w.abs().sum().item()
+
+
+def test_deterministic_and_no_writes_past_the_output():
+    m = gs()
+    inp = synth.make_inputs(1, seed=21, M=3001, N=5000)
+    d = dev(inp)
+    guard = 4096
+    buf = torch.full((inp["M"] + guard,), 12345.0, device="cuda")
+    out = buf[: inp["M"]].view(1, inp["M"], 1)
+    m.gauss_sum_fwd(d["x"], d["y"], d["w"], inp["tau"], out=out)
+    first = out.clone()
+    m.gauss_sum_fwd(d["x"], d["y"], d["w"], inp["tau"], out=out)
+    assert torch.equal(first, out), "two identical calls differ"
+    assert (buf[inp["M"]:] == 12345.0).all(), "canary after the output was overwritten"
+    h = synth.make_inputs(4, seed=22, B=1, M=300, N=2000, C=32)
+    dh = dev(h)
+    hb = torch.full((300 * 32 + guard,), -7.0, device="cuda")
+    ho = hb[: 300 * 32].view(1, 300, 32)
+    m.gauss_sum_fwd(dh["x"], dh["y"], dh["w"], 1.0, out=ho)
+    r1 = ho.clone()
+    m.gauss_sum_fwd(dh["x"], dh["y"], dh["w"], 1.0, out=ho)
+    assert torch.equal(r1, ho)
+    assert (hb[300 * 32:] == -7.0).all()
+    assert m.last_device_error() == 0
+
+
+def test_abi_rejects_bad_arguments_on_device():
+    import ctypes
+    m = gs()
+    lib = m.library()
+    x = torch.randn(1, 10, 3, device="cuda")
+    out = torch.empty(1, 10, 1, device="cuda")
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert lib.gauss_sum_fwd(p(x), p(x), p(out), p(out), 1, 10, 10, 3, 1, -1.0, 0, None, 0, s) == 1
+    odd = ctypes.c_void_p(x.data_ptr() + 4)
+    assert lib.gauss_sum_fwd(odd, p(x), p(out), p(out), 1, 10, 10, 3, 1, 1.0, 0, None, 0, s) == 3
+    h = torch.randn(1, 300, 32, device="cuda", dtype=torch.float16)
+    ho = torch.empty(1, 300, 32, device="cuda")
+    assert lib.gauss_sum_fwd(p(h), p(h), p(h), p(ho), 1, 300, 300, 32, 32, 1.0, 1, None, 0, s) == 4
+    assert m.last_device_error() == 0
