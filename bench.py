@@ -19,7 +19,6 @@ SM clocks and throttle reasons are sampled with nvidia-smi during the loop.
 """
 import argparse
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -317,17 +316,19 @@ def main():
         step_fn(gs, w, dd, ws, outs)()
         hout.copy_(outs["lse" if "lse" in w.ops and "sum" not in w.ops else "sum"], non_blocking=True)
 
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier(pg)
-    e_s.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
-    e_e.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e_s.elapsed_time(e_e), pg, dev) / args.e2e_steps
-    e2e_value = evals * world / (e2e_ms * 1e-3) / 1e9
+    e2e_ms, e2e_value = None, None
+    if args.e2e_steps > 0:
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(pg)
+        e_s.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e_e.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e_s.elapsed_time(e_e), pg, dev) / args.e2e_steps
+        e2e_value = evals * world / (e2e_ms * 1e-3) / 1e9
     clocks = clk.summary()
 
     if rank == 0:
