@@ -41,6 +41,7 @@ SIGNATURES = {
     "gs_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "gs_last_device_error": (ctypes.c_int, [_vp]),
     "gs_version": (ctypes.c_int, []),
+    "gs_test_exp2_poly": (ctypes.c_int, [_vp, _vp, _i64, ctypes.c_int, _vp]),
 }
 
 
@@ -163,6 +164,16 @@ def gauss_sum_bwd(x, y, w, g, tau, want_x=True, want_w=True, workspace=None, str
                             _ptr(ws), nbytes if ws is not None else 0, _stream(stream))
     _check("gauss_sum_bwd", st)
     return gx, gw
+
+
+def test_exp2_poly(x, degree, stream=None):
+    """Device evaluation of the FMA-pipe 2^x (test hook, see include/gauss_testing.h)."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 CUDA tensor")
+    out = torch.empty_like(x)
+    _check("gs_test_exp2_poly", _lib.gs_test_exp2_poly(_ptr(x), _ptr(out), x.numel(), int(degree),
+                                                       _stream(stream)))
+    return out
 
 
 def last_device_error(stream=None):

@@ -3,7 +3,8 @@
 Each translation unit under ``csrc/`` is compiled by nvcc in parallel into
 ``_build/`` and linked into a shared library next to this file, with the CUDA
 runtime linked statically so the library loads without a CUDA toolkit on the
-library path.  ``python -m pairwise_reductions_b200.build [--force] [-v]``.
+library path.  Run it as a script, ``python pairwise_reductions_b200/build.py
+[--force] [-v]`` (importing the package first would load the old library).
 """
 import concurrent.futures as cf
 import os
@@ -17,7 +18,7 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libgauss_b200.so")
 SOURCES = ["api.cpp", "small_d.cu", "tc_sm100.cu"]
-HEADERS = ["internal.h", "ptx.cuh"]
+HEADERS = ["internal.h", "ptx.cuh", "exp2_poly.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -47,7 +48,8 @@ def build(force=False, verbose=False):
     """Compile (if stale) and return the path of the shared library."""
     os.makedirs(BUILD, exist_ok=True)
     nvcc = _nvcc()
-    hdrs = [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(ROOT, "include", "gauss.h")]
+    hdrs = [os.path.join(CSRC, h) for h in HEADERS] + [
+        os.path.join(ROOT, "include", h) for h in ("gauss.h", "gauss_testing.h")]
     objs, jobs = [], []
     for src in SOURCES:
         sp = os.path.join(CSRC, src)

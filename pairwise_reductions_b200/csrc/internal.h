@@ -20,7 +20,7 @@ constexpr int kSdMaxD = 8;
 // Rows each thread of the small-D kernel keeps in registers, by feature
 // width D and padded channel chunk CP (register budget ~ R * (D + 2 CP)).
 __host__ __device__ constexpr int sd_rows_per_thread(int D, int CP) {
-  return (D + 2 * CP <= 16) ? 4 : ((D + 2 * CP <= 40) ? 2 : 1);
+  return (D + 2 * CP <= 8) ? 8 : ((D + 2 * CP <= 20) ? 4 : 2);
 }
 // Channel chunk width the kernel is instantiated for (1, 2, 4 or 8).
 __host__ __device__ constexpr int sd_chunk_pad(int c) {

@@ -6,6 +6,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "exp2_poly.cuh"
+
 namespace gs {
 
 // ---------------------------------------------------------------- arithmetic
@@ -28,6 +30,88 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// ---------------------------------------------------------------- packed fp32 pairs
+// sm_100 executes add/sub/mul/fma on two fp32 values per lane in one
+// instruction (.f32x2): twice the FP32 work per issue slot.  A pair lives in a
+// 64-bit register pair, low half first.
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// ---------------------------------------------------------------- exp2 on the FMA pipe
+// 2^x (NEG = false) or 2^-x (NEG = true) for a packed pair, by Cody-Waite
+// reduction for base 2 -- x = n + f with n = round(x) taken exactly from the
+// low mantissa bits of x + 1.5*2^23 and f in [-1/2, 1/2] -- followed by a
+// minimax polynomial for 2^f of degree DEG (coefficients from
+// gen_exp2_poly.py) and the addition of n to the exponent field.  Valid for
+// results in the normal range: the caller keeps the exponent >= -125.
+template <int DEG>
+__device__ __forceinline__ float exp2_coef(int k, bool neg) {
+  float c;
+  if constexpr (DEG == 3) {
+    c = k == 0 ? exp2poly::kD3C0 : k == 1 ? exp2poly::kD3C1 : k == 2 ? exp2poly::kD3C2 : exp2poly::kD3C3;
+  } else {
+    static_assert(DEG == 5, "degree 3 or 5");
+    c = k == 0 ? exp2poly::kD5C0 : k == 1 ? exp2poly::kD5C1 : k == 2 ? exp2poly::kD5C2
+      : k == 3 ? exp2poly::kD5C3 : k == 4 ? exp2poly::kD5C4 : exp2poly::kD5C5;
+  }
+  return (neg && (k & 1)) ? -c : c;
+}
+
+template <int DEG, bool NEG>
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+  const float kMagic = 12582912.f;   // 1.5 * 2^23: adding it rounds to an integer
+  const uint64_t magic = pk2(kMagic, kMagic);
+  // y = magic + n with n = round(+-x); r = n; g = x - n (or x + n for NEG), so
+  // that the polynomial argument is +-f
+  const uint64_t y = NEG ? sub2(magic, x) : add2(x, magic);
+  const uint64_t r = sub2(y, magic);
+  const uint64_t g = NEG ? add2(x, r) : sub2(x, r);
+  const float cd = exp2_coef<DEG>(DEG, NEG);
+  uint64_t p = pk2(cd, cd);
+#pragma unroll
+  for (int k = DEG - 1; k >= 0; --k) {
+    const float ck = exp2_coef<DEG>(k, NEG);
+    p = fma2(p, g, pk2(ck, ck));
+  }
+  // 2^n * p: add n << 23 to the bits of p.  (magic's own bits vanish when
+  // shifted by 23 modulo 2^32, so the bits of y can be used directly.)
+  uint32_t ylo, yhi, plo, phi;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(ylo), "=r"(yhi) : "l"(y));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(plo), "=r"(phi) : "l"(p));
+  uint32_t rlo, rhi;
+  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(rlo) : "r"(ylo), "r"(plo));
+  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(rhi) : "r"(yhi), "r"(phi));
+  uint64_t res;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(res) : "r"(rlo), "r"(rhi));
+  return res;
 }
 
 __device__ __forceinline__ uint64_t global_timer_ns() {

@@ -30,6 +30,7 @@
 
 #include <cmath>
 
+#include "../../include/gauss_testing.h"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -42,15 +43,34 @@ constexpr float kLn2 = 0.69314718055994530942f;
 
 template <int D, int CP>
 struct PackShape {
-  static constexpr int PK = ((D + CP + 3) / 4) * 4;   // floats per staged point
+  // floats per staged point: D duplicated negated coordinates and CP duplicated
+  // values, so every operand of the packed (two-row) arithmetic is one 64-bit load
+  static constexpr int PK = ((2 * (D + CP) + 3) / 4) * 4;
 };
+
+// Row pairs per thread that take the FMA-pipe exp2 instead of MUFU ex2.  At
+// D = 3 one of four row pairs balances the MUFU pipe (8 cycles per warp
+// instruction) against the issue slots of the packed arithmetic.
+template <int D, int CP, int R>
+__host__ __device__ constexpr int poly_pairs() {
+  return (R == 8 && D <= 4 && CP <= 2) ? 1 : 0;
+}
+
+// 2^e for an integer e (0 below 2^-126), built from its exponent bits: exact.
+__device__ __forceinline__ float pow2i(float e) {
+  if (!(e >= -126.f)) return 0.f;
+  return __int_as_float((static_cast<int>(e) + 127) << 23);
+}
 
 template <int D, int CP, bool LSE>
 __global__ void __launch_bounds__(kSdThreads)
     sd_kernel(const SdArgs a) {
   constexpr int R = sd_rows_per_thread(D, CP);
+  constexpr int RP = R / 2;                     // row pairs per thread
+  constexpr int NPOLY = poly_pairs<D, CP, R>();
   constexpr int PK = PackShape<D, CP>::PK;
   constexpr int NW = kSdThreads / 32;
+  static_assert(R % 2 == 0, "rows are processed in pairs");
   __shared__ __align__(16) float tile[kTileJ * PK];
   __shared__ float red[NW][CP];
 
@@ -64,43 +84,43 @@ __global__ void __launch_bounds__(kSdThreads)
   const float* __restrict__ yb = a.y + b * a.N * D;
   const float* __restrict__ wb = a.w + b * a.N * a.ldw + a.c0;
 
-  float xs[R][D];
+  // scaled coordinates of my rows, two rows per 64-bit pair
+  uint64_t xs[RP][D];
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const int64_t i = row0 + tid + r * kSdThreads;
+  for (int q = 0; q < RP; ++q) {
+    const int64_t i0 = row0 + tid + (2 * q) * kSdThreads;
+    const int64_t i1 = i0 + kSdThreads;
 #pragma unroll
-    for (int k = 0; k < D; ++k)
-      xs[r][k] = (i < a.M) ? a.x[(b * a.M + i) * D + k] * a.scale : 0.f;
+    for (int k = 0; k < D; ++k) {
+      const float v0 = (i0 < a.M) ? a.x[(b * a.M + i0) * D + k] * a.scale : 0.f;
+      const float v1 = (i1 < a.M) ? a.x[(b * a.M + i1) * D + k] * a.scale : 0.f;
+      xs[q][k] = pk2(v0, v1);
+    }
   }
-  float acc[R][CP];
-  float mrun[CP];
+  uint64_t acc[RP][CP];
+  float mrun[CP];   // LSE: integer log2 shift of the weights (-inf before any positive weight)
 #pragma unroll
   for (int c = 0; c < CP; ++c) {
     mrun[c] = -INFINITY;
 #pragma unroll
-    for (int r = 0; r < R; ++r) acc[r][c] = 0.f;
+    for (int q = 0; q < RP; ++q) acc[q][c] = 0ull;
   }
 
   for (int64_t j0 = jbeg; j0 < jend; j0 += kTileJ) {
-    // ---- stage one tile of (scaled y, weight or shifted log2 weight)
+    // ---- stage one tile: negated scaled y and the (shifted) weights
     float sy[kPer][D], sv[kPer][CP];
 #pragma unroll
     for (int q = 0; q < kPer; ++q) {
       const int64_t j = j0 + tid + q * kSdThreads;
       const bool ok = j < jend;
 #pragma unroll
-      for (int k = 0; k < D; ++k) sy[q][k] = ok ? yb[j * D + k] * a.scale : 0.f;
+      for (int k = 0; k < D; ++k) sy[q][k] = ok ? -(yb[j * D + k] * a.scale) : 0.f;
 #pragma unroll
-      for (int c = 0; c < CP; ++c) {
-        const bool okc = ok && c < a.cw;
-        const float wv = okc ? wb[j * a.ldw + c] : 0.f;
-        if constexpr (LSE)
-          sv[q][c] = okc ? lg2(wv) : -INFINITY;
-        else
-          sv[q][c] = wv;
-      }
+      for (int c = 0; c < CP; ++c) sv[q][c] = (ok && c < a.cw) ? wb[j * a.ldw + c] : 0.f;
     }
     if constexpr (LSE) {
+      // running power-of-two bound of the weights: w * 2^-m stays <= 1, so every
+      // term w K 2^-m <= 1 (K <= 1); accumulators follow the bound exactly
 #pragma unroll
       for (int c = 0; c < CP; ++c) {
         float m = sv[0][c];
@@ -116,98 +136,107 @@ __global__ void __launch_bounds__(kSdThreads)
         float mt = red[0][c];
 #pragma unroll
         for (int v = 1; v < NW; ++v) mt = fmaxf(mt, red[v][c]);
-        const float mnew = fmaxf(mrun[c], mt);
-        const float fac = (mrun[c] == -INFINITY) ? 0.f : ex2(mrun[c] - mnew);
+        // smallest integer e with max w < 2^e (from the exponent bits)
+        const float et = (mt > 0.f) ? static_cast<float>(((__float_as_int(mt) >> 23) & 0xff) - 126)
+                                    : -INFINITY;
+        const float mnew = fmaxf(mrun[c], et);
+        if (mnew > mrun[c]) {
+          const float fac = pow2i(mrun[c] - mnew);
 #pragma unroll
-        for (int r = 0; r < R; ++r) acc[r][c] *= fac;
-        mrun[c] = mnew;
-        const float sh = (mnew == -INFINITY) ? 0.f : mnew;
+          for (int q = 0; q < RP; ++q) {
+            acc[q][c] = mul2(acc[q][c], pk2(fac, fac));
+          }
+          mrun[c] = mnew;
+        }
+        const float sc = (mnew == -INFINITY) ? 1.f : pow2i(-mnew);
 #pragma unroll
-        for (int q = 0; q < kPer; ++q) sv[q][c] -= sh;
+        for (int q = 0; q < kPer; ++q) sv[q][c] *= sc;
       }
     }
 #pragma unroll
     for (int q = 0; q < kPer; ++q) {
       float* p = tile + (tid + q * kSdThreads) * PK;
 #pragma unroll
-      for (int k = 0; k < D; ++k) p[k] = sy[q][k];
+      for (int k = 0; k < D; ++k) {
+        p[2 * k] = sy[q][k];
+        p[2 * k + 1] = sy[q][k];
+      }
 #pragma unroll
-      for (int c = 0; c < CP; ++c) p[D + c] = sv[q][c];
+      for (int c = 0; c < CP; ++c) {
+        p[2 * (D + c)] = sv[q][c];
+        p[2 * (D + c) + 1] = sv[q][c];
+      }
 #pragma unroll
-      for (int k = D + CP; k < PK; ++k) p[k] = 0.f;
+      for (int k = 2 * (D + CP); k < PK; ++k) p[k] = 0.f;
     }
     __syncthreads();
 
     // ---- all pairs (my R rows) x (256 staged points)
-    float tacc[R][CP];
+    uint64_t tacc[RP][CP];
 #pragma unroll
-    for (int r = 0; r < R; ++r)
+    for (int q = 0; q < RP; ++q)
 #pragma unroll
-      for (int c = 0; c < CP; ++c) tacc[r][c] = 0.f;
+      for (int c = 0; c < CP; ++c) tacc[q][c] = 0ull;
 
-    const float4* t4 = reinterpret_cast<const float4*>(tile);
-#pragma unroll 4
+    const ulonglong2* t2 = reinterpret_cast<const ulonglong2*>(tile);
+#pragma unroll 2
     for (int jj = 0; jj < kTileJ; ++jj) {
-      float pk[PK];
+      uint64_t pk[PK / 2];
 #pragma unroll
       for (int v = 0; v < PK / 4; ++v) {
-        const float4 q = t4[jj * (PK / 4) + v];
-        pk[4 * v + 0] = q.x;
-        pk[4 * v + 1] = q.y;
-        pk[4 * v + 2] = q.z;
-        pk[4 * v + 3] = q.w;
+        const ulonglong2 u = t2[jj * (PK / 4) + v];
+        pk[2 * v] = u.x;
+        pk[2 * v + 1] = u.y;
       }
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        if constexpr (LSE && CP == 1) {
-          // exponent = log2 w - shift - |x^ - y^|^2, accumulated from the weight term
-          float t = pk[D];
+      for (int q = 0; q < RP; ++q) {
+        // d = |x^ - y^|^2 for two rows at once
+        uint64_t e = add2(xs[q][0], pk[0]);
+        uint64_t d = mul2(e, e);
 #pragma unroll
-          for (int k = 0; k < D; ++k) {
-            const float e = xs[r][k] - pk[k];
-            t = fmaf(-e, e, t);
-          }
-          tacc[r][0] += ex2(t);
-        } else {
-          const float e0 = xs[r][0] - pk[0];
-          float t = -e0 * e0;
-#pragma unroll
-          for (int k = 1; k < D; ++k) {
-            const float e = xs[r][k] - pk[k];
-            t = fmaf(-e, e, t);
-          }
-          if constexpr (LSE) {
-#pragma unroll
-            for (int c = 0; c < CP; ++c) tacc[r][c] += ex2(t + pk[D + c]);
-          } else {
-            const float kv = ex2(t);
-#pragma unroll
-            for (int c = 0; c < CP; ++c) tacc[r][c] = fmaf(kv, pk[D + c], tacc[r][c]);
-          }
+        for (int k = 1; k < D; ++k) {
+          e = add2(xs[q][k], pk[k]);
+          d = fma2(e, e, d);
         }
+        float d0, d1;
+        upk2(d, d0, d1);
+        uint64_t kv;
+        if (q >= RP - NPOLY) {
+          kv = exp2_poly2<5, true>(pk2(fminf(d0, 125.f), fminf(d1, 125.f)));
+        } else {
+          kv = pk2(ex2(-d0), ex2(-d1));
+        }
+#pragma unroll
+        for (int c = 0; c < CP; ++c) tacc[q][c] = fma2(kv, pk[D + c], tacc[q][c]);
       }
     }
 #pragma unroll
-    for (int r = 0; r < R; ++r)
+    for (int q = 0; q < RP; ++q)
 #pragma unroll
-      for (int c = 0; c < CP; ++c) acc[r][c] += tacc[r][c];
+      for (int c = 0; c < CP; ++c) acc[q][c] = add2(acc[q][c], tacc[q][c]);
     __syncthreads();
   }
 
   // ---- write this split's result (final sum, or shift + scaled sum)
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const int64_t i = row0 + tid + r * kSdThreads;
-    if (i >= a.M) continue;
-    const int64_t base = split * a.split_stride + (b * a.M + i) * a.ldo + a.c0;
+  for (int q = 0; q < RP; ++q) {
 #pragma unroll
-    for (int c = 0; c < CP; ++c) {
-      if (c >= a.cw) break;
-      if constexpr (LSE) {
-        a.out[base + c] = mrun[c];
-        a.out_l[base + c] = acc[r][c];
-      } else {
-        a.out[base + c] = acc[r][c];
+    for (int h = 0; h < 2; ++h) {
+      const int64_t i = row0 + tid + (2 * q + h) * kSdThreads;
+      if (i >= a.M) continue;
+      const int64_t base = split * a.split_stride + (b * a.M + i) * a.ldo + a.c0;
+#pragma unroll
+      for (int c = 0; c < CP; ++c) {
+        if (c >= a.cw) break;
+        float lo, hi;
+        upk2(acc[q][c], lo, hi);
+        const float v = h ? hi : lo;
+        if constexpr (LSE) {
+          a.out[base + c] = mrun[c];
+          a.out_l[base + c] = v;
+        } else {
+          a.out[base + c] = v;
+        }
       }
     }
   }
@@ -396,6 +425,22 @@ __global__ void fill_kernel(float* __restrict__ out, int64_t n, float value) {
     out[e] = value;
 }
 
+template <int DEG>
+__global__ void exp2_poly_eval_kernel(const float* __restrict__ x, float* __restrict__ out,
+                                      int64_t n) {
+  const int64_t pairs = (n + 1) / 2;
+  for (int64_t p = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; p < pairs;
+       p += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t i = 2 * p;
+    const float a = fmaxf(x[i], -125.f);
+    const float b = (i + 1 < n) ? fmaxf(x[i + 1], -125.f) : 0.f;
+    float ra, rb;
+    upk2(exp2_poly2<DEG, false>(pk2(a, b)), ra, rb);
+    out[i] = ra;
+    if (i + 1 < n) out[i + 1] = rb;
+  }
+}
+
 int grid_for(int64_t n, int threads) {
   int64_t b = (n + threads - 1) / threads;
   if (b < 1) b = 1;
@@ -490,3 +535,17 @@ cudaError_t launch_bwd_grad_x_epilogue(const void* x, gs_dtype dt, const float* 
 }
 
 }  // namespace gs
+
+extern "C" gs_status gs_test_exp2_poly(const float* x, float* out, int64_t n, int degree,
+                                       gs_stream_t stream) {
+  if (n < 0 || (degree != 3 && degree != 5)) return GS_ERR_INVALID_ARG;
+  if (n == 0) return GS_OK;
+  if (!x || !out) return GS_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int blocks = gs::grid_for((n + 1) / 2, 256);
+  if (degree == 3)
+    gs::exp2_poly_eval_kernel<3><<<blocks, 256, 0, s>>>(x, out, n);
+  else
+    gs::exp2_poly_eval_kernel<5><<<blocks, 256, 0, s>>>(x, out, n);
+  return cudaGetLastError() == cudaSuccess ? GS_OK : GS_ERR_CUDA;
+}

@@ -109,6 +109,50 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
+// Pairs of P columns (out of 16 per 32-column chunk) that take the FMA-pipe
+// exp2; the rest use MUFU ex2.  Half and half keeps both pipes busy.
+constexpr int kPolyPairs = 8;
+
+// Tie the registers of a TMEM load to the point after tcgen05.wait::ld, so
+// that no use of them is scheduled before the load has completed.
+__device__ __forceinline__ void reg_fence32(uint32_t (&v)[32]) {
+  asm volatile(""
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]), "+r"(v[16]), "+r"(v[17]),
+                 "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]), "+r"(v[22]), "+r"(v[23]),
+                 "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]), "+r"(v[29]),
+                 "+r"(v[30]), "+r"(v[31]));
+}
+__device__ __forceinline__ void reg_fence16(uint32_t (&v)[16]) {
+  asm volatile(""
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]));
+}
+
+// 32 S values of one row -> 16 packed fp16 pairs of P = 2^(2c S + r).
+__device__ __forceinline__ void exp_chunk(const uint32_t (&v)[32], uint64_t two_c2, uint64_t r2,
+                                          uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const uint64_t s2 = pk2(__uint_as_float(v[2 * q]), __uint_as_float(v[2 * q + 1]));
+    const uint64_t t2 = fma2(s2, two_c2, r2);
+    float t0, t1;
+    upk2(t2, t0, t1);
+    float e0, e1;
+    if ((q & 1) && (q >> 1) < kPolyPairs) {
+      // FMA pipe; exponents below -125 would leave the normal range (P is 0 in fp16 there)
+      const uint64_t e2 = exp2_poly2<3, false>(pk2(fmaxf(t0, -125.f), fmaxf(t1, -125.f)));
+      upk2(e2, e0, e1);
+    } else {
+      e0 = ex2(t0);
+      e1 = ex2(t1);
+    }
+    pk[q] = pack_f16x2(e0, e1);
+  }
+}
+
 template <int KP, int CP, int DTFMT>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gauss_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
@@ -263,6 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_base + Cfg::col_o(h);
     const float two_c = p.two_c;
     bool ok = true;
+    const uint64_t two_c2 = pk2(two_c, two_c);
+    const uint64_t r2 = pk2(r, r);
     for (int t = 0; t < T; ++t) {
       ok = wait_bar(bar_s(h), t & 1, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
@@ -270,19 +316,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
+      // double-buffered TMEM loads: chunk ch + 1 is in flight while chunk ch
+      // is exponentiated and its fp16 P written back
+      uint32_t va[32], vb[32];
+      tmem_ld32(tS, va);
+      tmem_wait_ld();
+      reg_fence32(va);
 #pragma unroll
       for (int ch = 0; ch < kBN / 32; ++ch) {
-        uint32_t v[32];
-        tmem_ld32(tS + ch * 32, v);
-        tmem_wait_ld();
+        uint32_t(&cur)[32] = (ch & 1) ? vb : va;
+        uint32_t(&nxt)[32] = (ch & 1) ? va : vb;
+        if (ch + 1 < kBN / 32) tmem_ld32(tS + (ch + 1) * 32, nxt);
         uint32_t pk[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const float e0 = ex2(fmaf(__uint_as_float(v[2 * q]), two_c, r));
-          const float e1 = ex2(fmaf(__uint_as_float(v[2 * q + 1]), two_c, r));
-          pk[q] = pack_f16x2(e0, e1);
-        }
+        exp_chunk(cur, two_c2, r2, pk);
         tmem_st16(tP + ch * 16, pk);
+        if (ch + 1 < kBN / 32) {
+          tmem_wait_ld();
+          reg_fence32(nxt);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
@@ -299,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t v[16];
         tmem_ld16(tO + ch * 16, v);
         tmem_wait_ld();
+        reg_fence16(v);
         if (valid) {
 #pragma unroll
           for (int q = 0; q < 16; ++q) {
