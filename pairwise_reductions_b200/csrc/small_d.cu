@@ -48,12 +48,13 @@ struct PackShape {
   static constexpr int PK = ((2 * (D + CP) + 3) / 4) * 4;
 };
 
-// Row pairs per thread that take the FMA-pipe exp2 instead of MUFU ex2.  At
-// D = 3 one of four row pairs balances the MUFU pipe (8 cycles per warp
-// instruction) against the issue slots of the packed arithmetic.
+// Row pairs per thread that take the FMA-pipe exp2 instead of MUFU ex2.  None:
+// measured on B200, the packed distance arithmetic already keeps the FMA pipe
+// about as busy as the exponentials keep MUFU, and the polynomial (about five
+// FMA-pipe instructions per value) costs more than the MUFU slot it frees.
 template <int D, int CP, int R>
 __host__ __device__ constexpr int poly_pairs() {
-  return (R == 8 && D <= 4 && CP <= 2) ? 1 : 0;
+  return 0;
 }
 
 // 2^e for an integer e (0 below 2^-126), built from its exponent bits: exact.

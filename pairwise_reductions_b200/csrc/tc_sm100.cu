@@ -72,7 +72,7 @@ struct TcCfg {
   static constexpr int STAGE = Y_BYTES + V_BYTES;
   static constexpr int NST_FIT = (200 * 1024 - X_BYTES) / STAGE;
   static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
-  static constexpr int NBARS = 2 * NST + 7;
+  static constexpr int NBARS = 2 * NST + 9;
   static constexpr int SMEM_RAW = 1024 + X_BYTES + NST * STAGE + 8 * NBARS + 16;
   // at least ~120 KB so that a second CTA never lands on the SM and blocks on
   // the 512-column TMEM allocation
@@ -141,7 +141,7 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&v)[32], uint64_t two_
     float t0, t1;
     upk2(t2, t0, t1);
     float e0, e1;
-    if ((q & 1) && (q >> 1) < kPolyPairs) {
+    if (((q * kPolyPairs) & 15) < kPolyPairs) {   // kPolyPairs of the 16 pairs, evenly spread
       // FMA pipe; exponents below -125 would leave the normal range (P is 0 in fp16 there)
       const uint64_t e2 = exp2_poly2<3, false>(pk2(fmaxf(t0, -125.f), fmaxf(t1, -125.f)));
       upk2(e2, e0, e1);
@@ -175,6 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_s = [&](int h) { return bar0 + 8u * (2 * NST + 1 + h); };   // S tile h ready
   auto bar_p = [&](int h) { return bar0 + 8u * (2 * NST + 3 + h); };   // P tile h written
   const uint32_t bar_o = bar0 + 8u * (2 * NST + 5);
+  auto bar_f = [&](int h) { return bar0 + 8u * (2 * NST + 7 + h); };   // S tile h read out
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t b = blockIdx.z;
@@ -194,6 +195,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_p(0), 4 * 32);
     mbar_init(bar_p(1), 4 * 32);
     mbar_init(bar_o, 1);
+    mbar_init(bar_f(0), 4 * 32);
+    mbar_init(bar_f(1), 4 * 32);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -272,22 +275,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; ok && t < T; ++t) {
         const int st = t % NST;
         const int st1 = (t + 1) % NST;
-        if (!(ok = wait_bar(bar_p(0), t & 1, abort_flag))) break;
-        tc_fence_after();
-        issue_O(0, st, t > 0);
-        if (t + 1 < T) {
-          if (!(ok = wait_bar(bar_full(st1), ((t + 1) / NST) & 1, abort_flag))) break;
+        if constexpr (Cfg::P_SEPARATE) {
+          // S_h(t+1) may overwrite S_h as soon as warpgroup h has read S_h(t)
+          // into registers: it then runs while the exponentials of tile t are
+          // still being computed.
+          if (t + 1 < T) {
+            if (!(ok = wait_bar(bar_f(0), t & 1, abort_flag))) break;
+            if (!(ok = wait_bar(bar_full(st1), ((t + 1) / NST) & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_S(0, st1);
+            mma_commit(bar_s(0));
+          }
+          if (!(ok = wait_bar(bar_p(0), t & 1, abort_flag))) break;
           tc_fence_after();
-          issue_S(0, st1);
-          mma_commit(bar_s(0));
-        }
-        if (!(ok = wait_bar(bar_p(1), t & 1, abort_flag))) break;
-        tc_fence_after();
-        issue_O(1, st, t > 0);
-        mma_commit(bar_empty(st));
-        if (t + 1 < T) {
-          issue_S(1, st1);
-          mma_commit(bar_s(1));
+          issue_O(0, st, t > 0);
+          if (t + 1 < T) {
+            if (!(ok = wait_bar(bar_f(1), t & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_S(1, st1);
+            mma_commit(bar_s(1));
+          }
+          if (!(ok = wait_bar(bar_p(1), t & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_O(1, st, t > 0);
+          mma_commit(bar_empty(st));
+        } else {
+          // P lives in the S columns: the next S MMA must follow the P MMA
+          if (!(ok = wait_bar(bar_p(0), t & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_O(0, st, t > 0);
+          if (t + 1 < T) {
+            if (!(ok = wait_bar(bar_full(st1), ((t + 1) / NST) & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_S(0, st1);
+            mma_commit(bar_s(0));
+          }
+          if (!(ok = wait_bar(bar_p(1), t & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_O(1, st, t > 0);
+          mma_commit(bar_empty(st));
+          if (t + 1 < T) {
+            issue_S(1, st1);
+            mma_commit(bar_s(1));
+          }
         }
       }
       mma_commit(bar_o);   // also the drain point for whatever was issued
@@ -333,6 +363,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ch + 1 < kBN / 32) {
           tmem_wait_ld();
           reg_fence32(nxt);
+          if (ch + 2 == kBN / 32) {
+            // the whole S tile is in registers: its TMEM columns may be reused
+            tc_fence_before();
+            mbar_arrive(bar_f(h));
+          }
         }
       }
       tmem_wait_st();
