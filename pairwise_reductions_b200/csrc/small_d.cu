@@ -460,8 +460,10 @@ SdPlan sd_plan(int64_t B, int64_t M, int64_t N, int D, int64_t C, int sm_count) 
   int64_t smax = N / 256;
   if (smax > 32) smax = 32;
   if (smax < 1) smax = 1;
-  // cost ~ CTAs per SM (at least 4 to keep the MUFU pipe fed) x columns per CTA
-  const int64_t k_sat = 4;
+  // cost ~ CTAs per SM (at least 12 resident-CTA equivalents, to keep the MUFU
+  // pipe fed: measured on B200 at 100k points, a floor of 4 left 10% and 8
+  // left 2.5% on the table) x columns per CTA
+  const int64_t k_sat = 12;
   int best = 1;
   double best_cost = 1e300;
   for (int64_t S = 1; S <= smax; ++S) {

@@ -110,8 +110,11 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
 }
 
 // Pairs of P columns (out of 16 per 32-column chunk) that take the FMA-pipe
-// exp2; the rest use MUFU ex2.  Half and half keeps both pipes busy.
-constexpr int kPolyPairs = 8;
+// exp2; the rest use MUFU ex2.  Measured on B200 (d32_c32, d32_c1): once the
+// next S tile overlaps the exponentials, 0 beats 2, 3, 4 and 5 -- the exp warps
+// are partly latency-bound and the polynomial's longer dependency chain costs
+// more than the MUFU slots it frees.  Kept as a tuning knob.
+constexpr int kPolyPairs = 0;
 
 // Tie the registers of a TMEM load to the point after tcgen05.wait::ld, so
 // that no use of them is scheduled before the load has completed.
