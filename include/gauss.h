@@ -120,6 +120,26 @@ gs_status gauss_sum_bwd(const void *x, const void *y, const void *w, const float
                         int64_t C, float tau, gs_dtype dt, void *ws, size_t ws_bytes,
                         gs_stream_t stream);
 
+/*
+ * Allocation-free variant of gauss_sum_fwd (no counterpart on the pages: it
+ * exists for callers of this library that cannot allocate device memory for a
+ * workspace -- a plugin whose host application owns the device-memory budget,
+ * a latency-critical loop that must not block in the CUDA allocator, a process
+ * under a hard memory cap).  Same arguments, results and kernels as
+ * gauss_sum_fwd, without ws / ws_bytes: the scratch comes from a fixed 32 MiB
+ * device array inside the library, held by every GPU on which it has been used
+ * until the process exits.  Calls whose scratch need (gs_workspace_bytes of
+ * GS_OP_SUM) exceeds 32 MiB return GS_ERR_WORKSPACE.  All calls on a device
+ * share the array: calls that overlap on the GPU race (order them on one
+ * stream).  The array keeps the last call's contents; nothing in it needs to
+ * start at zero.  The first call on a device looks up the array's device
+ * address with that device current; make that first call before any stream
+ * capture.  The library allocates nothing in this call.
+ */
+gs_status gauss_sum_fwd_noalloc(const void *x, const void *y, const void *w, float *out, int64_t B,
+                                int64_t M, int64_t N, int64_t D, int64_t C, float tau, gs_dtype dt,
+                                gs_stream_t stream);
+
 /* A static, human-readable name for a status code. */
 const char *gs_status_string(gs_status status);
 

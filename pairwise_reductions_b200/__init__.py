@@ -42,6 +42,8 @@ SIGNATURES = {
     "gs_last_device_error": (ctypes.c_int, [_vp]),
     "gs_version": (ctypes.c_int, []),
     "gs_test_exp2_poly": (ctypes.c_int, [_vp, _vp, _i64, ctypes.c_int, _vp]),
+    "gauss_sum_fwd_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _f,
+                                             ctypes.c_int, _vp]),
 }
 
 
@@ -144,6 +146,20 @@ def gauss_sum_fwd(x, y, w, tau, out=None, workspace=None, stream=None):
     return _reduce("gauss_sum_fwd", GS_OP_SUM, x, y, w, tau, out, workspace, stream)
 
 
+def gauss_sum_fwd_noalloc(x, y, w, tau, out=None, stream=None):
+    """gauss_sum_fwd without a workspace: for callers that cannot allocate device
+    memory; the library's fixed 32 MiB scratch array is used instead (see
+    include/gauss.h for its limits: calls that overlap on the GPU race on it)."""
+    x, y, w = _as3(x, "x"), _as3(y, "y"), _as3(w, "w")
+    B, M, N, D, C = _dims(x, y, w)
+    if out is None:
+        out = torch.empty((B, M, C), dtype=torch.float32, device=x.device)
+    st = _lib.gauss_sum_fwd_noalloc(_ptr(x), _ptr(y), _ptr(w), _ptr(out), B, M, N, D, C,
+                                    float(tau), _DT[x.dtype], _stream(stream))
+    _check("gauss_sum_fwd_noalloc", st)
+    return out
+
+
 def gauss_lse_fwd(x, y, w, tau, out=None, workspace=None, stream=None):
     """out[b,i,c] = log sum_j w[b,j,c] exp(-tau/2 |x_i - y_j|^2)   (w > 0)."""
     return _reduce("gauss_lse_fwd", GS_OP_LSE, x, y, w, tau, out, workspace, stream)
@@ -181,6 +197,6 @@ def last_device_error(stream=None):
     return int(_lib.gs_last_device_error(_stream(stream)))
 
 
-__all__ = ["gauss_sum_fwd", "gauss_lse_fwd", "gauss_sum_bwd", "workspace_bytes",
+__all__ = ["gauss_sum_fwd", "gauss_sum_fwd_noalloc", "gauss_lse_fwd", "gauss_sum_bwd", "workspace_bytes",
            "last_device_error", "library", "status_string", "GaussError", "SIGNATURES",
            "LIB_PATH"]
