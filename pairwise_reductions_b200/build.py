@@ -37,6 +37,28 @@ def _flags(verbose):
     return f
 
 
+# Kernels whose registers receive asynchronous tcgen05.ld results must not
+# spill: a spill store placed between the load and its tcgen05.wait::ld would
+# save a register before the load has written it.  The build refuses them.
+NO_SPILL_KERNELS = ("tc_gauss_kernel",)
+
+
+def _check_spills(ptxas_log):
+    import re
+    bad, current = [], None
+    for line in ptxas_log.splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            current = m.group(1)
+            continue
+        m = re.search(r"(\d+) bytes spill stores, (\d+) bytes spill loads", line)
+        if m and current and any(k in current for k in NO_SPILL_KERNELS):
+            if int(m.group(1)) or int(m.group(2)):
+                bad.append((current, m.group(0)))
+    if bad:
+        raise RuntimeError("register spills in kernels that hold tcgen05.ld results: " + repr(bad))
+
+
 def _stale(out, deps):
     if not os.path.exists(out):
         return True
@@ -56,7 +78,7 @@ def build(force=False, verbose=False):
         obj = os.path.join(BUILD, src + ".o")
         objs.append(obj)
         if force or _stale(obj, [sp] + hdrs):
-            cmd = [nvcc, *_flags(verbose), "-c", sp, "-o", obj]
+            cmd = [nvcc, *_flags(verbose or src == "tc_sm100.cu"), "-c", sp, "-o", obj]
             if src.endswith(".cpp"):
                 cmd[1:1] = ["-x", "cu"]
             jobs.append(cmd)
@@ -69,6 +91,12 @@ def build(force=False, verbose=False):
             if r.returncode != 0:
                 sys.stderr.write(r.stdout + r.stderr)
                 raise RuntimeError("nvcc failed: " + " ".join(cmd))
+            if "tc_sm100.cu" in cmd[-3]:
+                try:
+                    _check_spills(r.stderr)
+                except RuntimeError:
+                    os.remove(cmd[-1])
+                    raise
     if force or jobs or _stale(LIB, objs):
         cmd = [nvcc, *ARCH, "-shared", "-cudart", "static", "-o", LIB, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)

@@ -104,3 +104,16 @@ def test_bwd_argument_checks():
     assert lib.gauss_sum_bwd(*args(tau=0.0)) == 1
     assert lib.gauss_sum_bwd(*args(gx=ODD)) == 3
     assert lib.gauss_sum_bwd(*args(gx=NULL, gw=NULL)) == 0   # nothing requested
+
+
+def test_build_refuses_spills_in_tensor_core_kernels():
+    import importlib.util
+    path = os.path.join(os.path.dirname(INCLUDE), "pairwise_reductions_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_gs_build_for_test", path)
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    ok_log = ("ptxas info    : Compiling entry function '_Z15tc_gauss_kernelILi64E' for 'sm_100a'\n"
+              "    0 bytes stack frame, 0 bytes spill stores, 0 bytes spill loads\n")
+    b._check_spills(ok_log)
+    with pytest.raises(RuntimeError):
+        b._check_spills(ok_log.replace("0 bytes spill stores", "12 bytes spill stores"))
