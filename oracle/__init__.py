@@ -12,6 +12,8 @@ step 2):
 * ``gauss_sum(x, y, w, tau, rows=None)``  -> [B, R, C]
 * ``gauss_lse(x, y, w, tau, rows=None)``  -> [B, R, C]
 * ``gauss_sum_bwd(x, y, w, g, tau, rows=None, wrows=None)`` -> (grad_x, grad_w)
+* ``gauss_sum_vjp_y_tau(x, y, w, g, tau, yrows=None)`` -> (grad_y, grad_tau)
+* ``gauss_lse_bwd(x, y, w, g, tau)`` -> (grad_x, grad_y, grad_w, grad_tau)
 
 Inputs are float64 arrays x [B,M,D], y [B,N,D], w [B,N,C], g [B,M,C] (2-D
 arrays are read as B = 1).  Values must already be the quantised values the
@@ -47,6 +49,14 @@ def _load(path=None):
     f.restype = ctypes.c_int
     f.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _i64, _i64, _i64, _i64, _i64,
                   ctypes.c_double, _ip, _i64, _ip, _i64]
+    f = lib.oracle_gauss_sum_vjp_y_tau
+    f.restype = ctypes.c_int
+    f.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _i64, _i64, _i64, _i64, _i64, ctypes.c_double,
+                  _ip, _i64]
+    f = lib.oracle_gauss_lse_bwd
+    f.restype = ctypes.c_int
+    f.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _i64, _i64, _i64, _i64, _i64,
+                  ctypes.c_double]
     lib.oracle_num_threads.restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -128,4 +138,36 @@ def gauss_sum_bwd(x, y, w, g, tau, rows=None, wrows=None, want_x=True, want_w=Tr
     return gx, gw
 
 
-__all__ = ["gauss_sum", "gauss_lse", "gauss_sum_bwd", "num_threads", "build_oracle", "LIB"]
+def gauss_sum_vjp_y_tau(x, y, w, g, tau, yrows=None, want_y=True, want_tau=True, lib=None):
+    """Gradients of sum(g * gauss_sum(x, y, w)) with respect to y and tau."""
+    x, y, w, g = _as3(x, "x"), _as3(y, "y"), _as3(w, "w"), _as3(g, "g")
+    B, M, N, D, C = _check(x, y, w)
+    if g.shape != (B, M, C):
+        raise ValueError(f"g must be {(B, M, C)}, got {g.shape}")
+    r, nr, rp = _rows(yrows)
+    R = nr if r is not None else N
+    gy = np.empty((B, R, D), dtype=np.float64) if want_y else None
+    gt = np.zeros(1, dtype=np.float64) if want_tau else None
+    rc = (lib or _load()).oracle_gauss_sum_vjp_y_tau(_ptr(x), _ptr(y), _ptr(w), _ptr(g), _ptr(gy),
+                                                    _ptr(gt), B, M, N, D, C, float(tau), rp, nr)
+    if rc != 0:
+        raise ValueError(f"oracle_gauss_sum_vjp_y_tau rejected its arguments (code {rc})")
+    return gy, (float(gt[0]) if want_tau else None)
+
+
+def gauss_lse_bwd(x, y, w, g, tau, lib=None):
+    """Gradients of sum(g * gauss_lse(x, y, w)) w.r.t. x, y, w and tau (small sizes)."""
+    x, y, w, g = _as3(x, "x"), _as3(y, "y"), _as3(w, "w"), _as3(g, "g")
+    B, M, N, D, C = _check(x, y, w)
+    if g.shape != (B, M, C):
+        raise ValueError(f"g must be {(B, M, C)}, got {g.shape}")
+    gx = np.empty((B, M, D)); gy = np.empty((B, N, D)); gw = np.empty((B, N, C))
+    gt = np.zeros(1)
+    rc = (lib or _load()).oracle_gauss_lse_bwd(_ptr(x), _ptr(y), _ptr(w), _ptr(g), _ptr(gx), _ptr(gy),
+                                              _ptr(gw), _ptr(gt), B, M, N, D, C, float(tau))
+    if rc != 0:
+        raise ValueError(f"oracle_gauss_lse_bwd rejected its arguments (code {rc})")
+    return gx, gy, gw, float(gt[0])
+
+
+__all__ = ["gauss_sum_vjp_y_tau", "gauss_lse_bwd", "gauss_sum", "gauss_lse", "gauss_sum_bwd", "num_threads", "build_oracle", "LIB"]

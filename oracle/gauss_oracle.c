@@ -284,3 +284,148 @@ int oracle_gauss_sum_bwd(const double *x, const double *y, const double *w,
     }
     return bad ? 2 : 0;
 }
+
+/* Full vector-Jacobian product of L = sum_{i,c} g[i,c] * s[i,c], s the Gauss
+ * sum, extending oracle_gauss_sum_bwd with the source points and the bandwidth
+ * ("Kernel matrix reduction", Variants: derivatives of any order through the
+ * fused reduction; here the first order in every input):
+ *
+ *   dL/dy[j,k] = -tau * sum_i K_ij (sum_c g[i,c] w[j,c]) (y[j,k] - x[i,k])
+ *   dL/dtau    = -1/2 * sum_b sum_i sum_j K_ij |x_i - y_j|^2 (sum_c g[i,c] w[j,c])
+ *
+ * grad_y is [B, Rw, D] over the source rows yrows (NULL = all N); grad_tau is
+ * one double (NULL to skip).  Either may be NULL. */
+int oracle_gauss_sum_vjp_y_tau(const double *x, const double *y, const double *w,
+                               const double *g, double *grad_y, double *grad_tau, int64_t B,
+                               int64_t M, int64_t N, int64_t D, int64_t C, double tau,
+                               const int64_t *yrows, int64_t n_yrows)
+{
+    int64_t Rw = yrows ? n_yrows : N;
+    if (B < 0 || M < 0 || N < 0 || D < 1 || C < 1 || Rw < 0 || !(tau > 0.0))
+        return 1;
+    int bad = 0;
+    if (grad_y) {
+#pragma omp parallel
+        {
+            comp_sum *acc = (comp_sum *)malloc((size_t)D * sizeof(comp_sum));
+            if (!acc) {
+#pragma omp atomic write
+                bad = 1;
+            }
+#pragma omp for schedule(dynamic, 4)
+            for (int64_t t = 0; t < B * Rw; ++t) {
+                if (!acc)
+                    continue;
+                int64_t bb = t / Rw;
+                int64_t r = t % Rw;
+                int64_t j = yrows ? yrows[r] : r;
+                const double *yj = y + (bb * N + j) * D;
+                const double *wj = w + (bb * N + j) * C;
+                for (int64_t k = 0; k < D; ++k) {
+                    acc[k].s = 0.0;
+                    acc[k].c = 0.0;
+                }
+                for (int64_t i = 0; i < M; ++i) {
+                    const double *xi = x + (bb * M + i) * D;
+                    const double *gi = g + (bb * M + i) * C;
+                    double kv = exp(-0.5 * tau * sq_dist(xi, yj, D));
+                    double gw = 0.0;
+                    for (int64_t c = 0; c < C; ++c)
+                        gw += gi[c] * wj[c];
+                    for (int64_t k = 0; k < D; ++k)
+                        cs_add(&acc[k], kv * gw * (yj[k] - xi[k]));
+                }
+                for (int64_t k = 0; k < D; ++k)
+                    grad_y[(bb * Rw + r) * D + k] = -tau * cs_value(&acc[k]);
+            }
+            free(acc);
+        }
+    }
+    if (grad_tau) {
+        comp_sum total = {0.0, 0.0};
+        for (int64_t bb = 0; bb < B; ++bb) {
+            for (int64_t i = 0; i < M; ++i) {
+                const double *xi = x + (bb * M + i) * D;
+                const double *gi = g + (bb * M + i) * C;
+                comp_sum row = {0.0, 0.0};
+                for (int64_t j = 0; j < N; ++j) {
+                    const double *yj = y + (bb * N + j) * D;
+                    const double *wj = w + (bb * N + j) * C;
+                    double d2 = sq_dist(xi, yj, D);
+                    double gw = 0.0;
+                    for (int64_t c = 0; c < C; ++c)
+                        gw += gi[c] * wj[c];
+                    cs_add(&row, exp(-0.5 * tau * d2) * d2 * gw);
+                }
+                cs_add(&total, cs_value(&row));
+            }
+        }
+        *grad_tau = -0.5 * cs_value(&total);
+    }
+    return bad ? 2 : 0;
+}
+
+/* Gradient of L = sum_{i,c} g[i,c] * lse[i,c], lse the log-sum-exp of
+ * oracle_gauss_lse.  With the normalised weights
+ *   p_ijc = w[j,c] K_ij / sum_j' w[j',c] K_ij'   (computed max-shifted),
+ *   dL/dx[i,k] = -tau * sum_c g[i,c] sum_j p_ijc (x[i,k] - y[j,k])
+ *   dL/dy[j,k] = -tau * sum_i sum_c g[i,c] p_ijc (y[j,k] - x[i,k])
+ *   dL/dw[j,c] = sum_i g[i,c] p_ijc / w[j,c]  ( = sum_i g[i,c] K_ij / S_ic )
+ *   dL/dtau    = -1/2 * sum_i sum_c g[i,c] sum_j p_ijc |x_i - y_j|^2
+ * Outputs over all rows ([B,M,D], [B,N,D], [B,N,C], one double); any may be
+ * NULL.  Requires w > 0.  Plain triple loops, small sizes only. */
+int oracle_gauss_lse_bwd(const double *x, const double *y, const double *w, const double *g,
+                         double *grad_x, double *grad_y, double *grad_w, double *grad_tau,
+                         int64_t B, int64_t M, int64_t N, int64_t D, int64_t C, double tau)
+{
+    if (B < 0 || M < 0 || N < 0 || D < 1 || C < 1 || !(tau > 0.0))
+        return 1;
+    if (grad_x)
+        memset(grad_x, 0, (size_t)(B * M * D) * sizeof(double));
+    if (grad_y)
+        memset(grad_y, 0, (size_t)(B * N * D) * sizeof(double));
+    if (grad_w)
+        memset(grad_w, 0, (size_t)(B * N * C) * sizeof(double));
+    double tau_acc = 0.0;
+    double *f = (double *)malloc((size_t)(N > 0 ? N : 1) * sizeof(double));
+    if (!f)
+        return 2;
+    for (int64_t bb = 0; bb < B; ++bb) {
+        for (int64_t i = 0; i < M; ++i) {
+            const double *xi = x + (bb * M + i) * D;
+            double m = -INFINITY;
+            for (int64_t j = 0; j < N; ++j) {
+                f[j] = -0.5 * tau * sq_dist(xi, y + (bb * N + j) * D, D);
+                if (f[j] > m)
+                    m = f[j];
+            }
+            for (int64_t c = 0; c < C; ++c) {
+                double gic = g[(bb * M + i) * C + c];
+                comp_sum z = {0.0, 0.0};
+                for (int64_t j = 0; j < N; ++j)
+                    cs_add(&z, w[(bb * N + j) * C + c] * exp(f[j] - m));
+                double zs = cs_value(&z);
+                for (int64_t j = 0; j < N; ++j) {
+                    const double *yj = y + (bb * N + j) * D;
+                    double e = exp(f[j] - m);
+                    double p = w[(bb * N + j) * C + c] * e / zs;
+                    double d2 = sq_dist(xi, yj, D);
+                    for (int64_t k = 0; k < D; ++k) {
+                        double diff = xi[k] - yj[k];
+                        if (grad_x)
+                            grad_x[(bb * M + i) * D + k] += -tau * gic * p * diff;
+                        if (grad_y)
+                            grad_y[(bb * N + j) * D + k] += tau * gic * p * diff;
+                    }
+                    if (grad_w)
+                        grad_w[(bb * N + j) * C + c] += gic * e / zs;
+                    tau_acc += -0.5 * gic * p * d2;
+                }
+            }
+        }
+    }
+    free(f);
+    if (grad_tau)
+        *grad_tau = tau_acc;
+    return 0;
+}

@@ -309,9 +309,89 @@ def pin_large_n_expectation(O):
         assert abs(out[i] / N - mean1) <= 6 * se, f"row {i}: {out[i] / N} vs {mean1} (se {se})"
 
 
+# --------------------------------------------------------------------------- full gradient, LSE gradient
+def pin_golden_vjp_y_tau(O):
+    for case in golden()["vjp_y_tau"]:
+        gy, gt = O.gauss_sum_vjp_y_tau(case["x"], case["y"], case["w"], case["g"], case["tau"])
+        _close(gy, _eval_tree(case["expected_grad_y"]), 1e-14, 1e-15, case["name"] + " grad_y")
+        _close(gt, _eval_tree(case["expected_grad_tau"]), 1e-14, 1e-15, case["name"] + " grad_tau")
+
+
+def pin_golden_lse_bwd(O):
+    for case in golden()["lse_bwd"]:
+        gx, gy, gw, gt = O.gauss_lse_bwd(case["x"], case["y"], case["w"], case["g"], case["tau"])
+        e = case["expected"]
+        for name, got in (("grad_x", gx), ("grad_y", gy), ("grad_w", gw), ("grad_tau", gt)):
+            _close(got, _eval_tree(e[name]), 1e-14, 1e-15, case["name"] + " " + name)
+
+
+def _fd(f, a, h=1e-5):
+    out = np.zeros_like(a)
+    for idx in np.ndindex(a.shape):
+        ap, am = a.copy(), a.copy()
+        ap[idx] += h
+        am[idx] -= h
+        out[idx] = (f(ap) - f(am)) / (2 * h)
+    return out
+
+
+def pin_finite_differences_y_tau(O):
+    """Central differences for dL/dy and dL/dtau of L = sum g * S(x, y, w, tau)."""
+    r = _rng(15)
+    B, M, N, D, C, tau = 2, 4, 6, 3, 2, 0.8
+    x, y = r.normal(size=(B, M, D)), r.normal(size=(B, N, D))
+    w, g = r.normal(size=(B, N, C)), r.normal(size=(B, M, C))
+    gy, gt = O.gauss_sum_vjp_y_tau(x, y, w, g, tau)
+    fdy = _fd(lambda yy: float((g * O.gauss_sum(x, yy, w, tau)).sum()), y)
+    fdt = _fd(lambda tt: float((g * O.gauss_sum(x, y, w, float(tt))).sum()), np.array(tau))
+    assert _rel_l2(gy, fdy) < 1e-8, f"grad_y vs finite differences: {_rel_l2(gy, fdy):.2e}"
+    assert abs(gt - float(fdt)) <= 1e-8 * max(1.0, abs(gt)), f"grad_tau {gt} vs {float(fdt)}"
+    rows = np.array([5, 1])
+    sy, _ = O.gauss_sum_vjp_y_tau(x, y, w, g, tau, yrows=rows, want_tau=False)
+    _close(sy, gy[:, rows], 0, 0, "grad_y rows")
+
+
+def pin_finite_differences_lse(O):
+    """Central differences of L = sum g * LSE(x, y, w, tau) for every input."""
+    r = _rng(16)
+    B, M, N, D, C, tau = 1, 4, 5, 2, 2, 1.3
+    x, y = r.normal(size=(B, M, D)), r.normal(size=(B, N, D))
+    w, g = r.uniform(0.5, 1.5, size=(B, N, C)), r.normal(size=(B, M, C))
+    gx, gy, gw, gt = O.gauss_lse_bwd(x, y, w, g, tau)
+    L = lambda xx, yy, ww, tt: float((g * O.gauss_lse(xx, yy, ww, tt)).sum())
+    checks = [("grad_x", gx, _fd(lambda a: L(a, y, w, tau), x)),
+              ("grad_y", gy, _fd(lambda a: L(x, a, w, tau), y)),
+              ("grad_w", gw, _fd(lambda a: L(x, y, a, tau), w))]
+    for name, got, fd in checks:
+        assert _rel_l2(got, fd) < 1e-8, f"lse {name} vs finite differences: {_rel_l2(got, fd):.2e}"
+    fdt = float(_fd(lambda a: L(x, y, w, float(a)), np.array(tau)))
+    assert abs(gt - fdt) <= 1e-8 * max(1.0, abs(gt)), f"lse grad_tau {gt} vs {fdt}"
+
+
+def pin_gradient_symmetries(O):
+    """Translation: sum_i dL/dx_i + sum_j dL/dy_j = 0.  Scaling (K(a x, a y, tau) =
+    K(x, y, a^2 tau)): sum x.dL/dx + sum y.dL/dy = 2 tau dL/dtau.  For the sum and the LSE."""
+    r = _rng(17)
+    B, M, N, D, C, tau = 1, 7, 9, 3, 2, 0.6
+    x, y = r.normal(size=(B, M, D)), r.normal(size=(B, N, D))
+    w, g = r.uniform(0.5, 1.5, size=(B, N, C)), r.normal(size=(B, M, C))
+    gx, _ = O.gauss_sum_bwd(x, y, w, g, tau, want_w=False)
+    gy, gt = O.gauss_sum_vjp_y_tau(x, y, w, g, tau)
+    scale = float(np.abs(gx).sum() + np.abs(gy).sum())
+    assert abs(gx.sum(axis=(0, 1)) + gy.sum(axis=(0, 1))).max() <= 1e-12 * scale, "sum: translation"
+    lhs = float((x * gx).sum() + (y * gy).sum())
+    assert abs(lhs - 2 * tau * gt) <= 1e-11 * max(1.0, abs(lhs)), f"sum: scaling {lhs} vs {2 * tau * gt}"
+    lx, ly, _, lt = O.gauss_lse_bwd(x, y, w, g, tau)
+    scale = float(np.abs(lx).sum() + np.abs(ly).sum())
+    assert abs(lx.sum(axis=(0, 1)) + ly.sum(axis=(0, 1))).max() <= 1e-12 * scale, "lse: translation"
+    lhs = float((x * lx).sum() + (y * ly).sum())
+    assert abs(lhs - 2 * tau * lt) <= 1e-11 * max(1.0, abs(lhs)), f"lse: scaling {lhs} vs {2 * tau * lt}"
+
+
 ALL_PINS = [
     pin_golden_sum, pin_golden_lse, pin_golden_bwd, pin_dense_library, pin_flash_prescale,
     pin_flash_reweight, pin_coincident, pin_single_point, pin_separable_grid, pin_translation,
     pin_small_tau, pin_symmetry, pin_linearity, pin_lse_is_log_sum, pin_rows_subset,
-    pin_finite_differences, pin_large_n_expectation,
+    pin_finite_differences, pin_large_n_expectation, pin_golden_vjp_y_tau, pin_golden_lse_bwd,
+    pin_finite_differences_y_tau, pin_finite_differences_lse, pin_gradient_symmetries,
 ]

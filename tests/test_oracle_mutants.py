@@ -28,6 +28,12 @@ MUTANTS = [
     ("grad_x drops the g.w coupling", [("gw += gi[c] * wj[c];", "gw += gi[c];", 1)]),
     ("grad_x factor tau/2", [("-tau * cs_value(&acc[k])", "-0.5 * tau * cs_value(&acc[k])", 1)]),
     ("grad_w drops the upstream gradient", [("cs_add(&acc[c], kv * gi[c]);", "cs_add(&acc[c], kv);", 1)]),
+    ("grad_y sign of the difference", [("cs_add(&acc[k], kv * gw * (yj[k] - xi[k]));", "cs_add(&acc[k], kv * gw * (xi[k] - yj[k]));", 1)]),
+    ("grad_tau factor 1/2 dropped", [("*grad_tau = -0.5 * cs_value(&total);", "*grad_tau = -cs_value(&total);", 1)]),
+    ("grad_tau without the squared distance", [("cs_add(&row, exp(-0.5 * tau * d2) * d2 * gw);", "cs_add(&row, exp(-0.5 * tau * d2) * gw);", 1)]),
+    ("lse grad unnormalised weights", [("double p = w[(bb * N + j) * C + c] * e / zs;", "double p = w[(bb * N + j) * C + c] * e;", 1)]),
+    ("lse grad_w uses p instead of p / w", [("grad_w[(bb * N + j) * C + c] += gic * e / zs;", "grad_w[(bb * N + j) * C + c] += gic * p;", 1)]),
+    ("lse grad_y sign", [("grad_y[(bb * N + j) * D + k] += tau * gic * p * diff;", "grad_y[(bb * N + j) * D + k] += -tau * gic * p * diff;", 1)]),
     ("grad_w kernel against x_0 only", [("const double *xi = x + (bb * M + i) * D;\n                    const double *gi", "const double *xi = x + (bb * M) * D;\n                    const double *gi", 1)]),
 ]
 
@@ -50,6 +56,8 @@ class _Handle:
         self.gauss_sum = functools.partial(oracle.gauss_sum, lib=lib)
         self.gauss_lse = functools.partial(oracle.gauss_lse, lib=lib)
         self.gauss_sum_bwd = functools.partial(oracle.gauss_sum_bwd, lib=lib)
+        self.gauss_sum_vjp_y_tau = functools.partial(oracle.gauss_sum_vjp_y_tau, lib=lib)
+        self.gauss_lse_bwd = functools.partial(oracle.gauss_lse_bwd, lib=lib)
 
 
 @pytest.mark.parametrize("idx", range(len(MUTANTS)), ids=[m[0] for m in MUTANTS])
