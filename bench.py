@@ -179,6 +179,30 @@ def launches_per_step(gs, run):
     return len(names), sorted(set(names))
 
 
+# ------------------------------------------------------------------ ncu traffic of the dominant kernel
+DOMINANT = {"f32": ("sd_kernel", "small_d.cu"), "f16": ("tc_gauss_kernel", "tc_sm100.cu"),
+            "bf16": ("tc_gauss_kernel", "tc_sm100.cu")}
+
+
+def traffic_per_launch(w):
+    """DRAM bytes (read + write) per launch of the dominant kernel from the committed ncu
+    summary, or None when there is none for this workload or the kernel source changed since."""
+    import hashlib
+    kernel, src = DOMINANT[w.dtype]
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None, kernel
+    cur = hashlib.sha256(open(os.path.join(ROOT, "pairwise_reductions_b200", "csrc", src), "rb").read())
+    for line in lines:
+        f = line.split()
+        if len(f) == 6 and not line.startswith("#") and f[0] == kernel and f[1] == w.name:
+            if f[4] == src and cur.hexdigest().startswith(f[5]):
+                return int(f[2]) + int(f[3]), kernel
+    return None, kernel
+
+
 # ------------------------------------------------------------------ CPU oracle baseline
 def oracle_sample(w, inp, seconds, seed=1234):
     """Time the oracle as it stands on a bounded row sample of the workload."""
@@ -342,8 +366,9 @@ def main():
         sm_max = float(clocks.get("sm_max_mhz") or peaks.get("sm_max_mhz") or 1965.0)
         peak = EX2_PER_CLK_PER_SM * sms * sm_max * 1e6 / 1e9
         achieved = evals / (ms_per_step * 1e-3) / 1e9
-        roof = {"bound": "alu", "kernel": "MUFU ex2 (one per pair)", "achieved": achieved,
-                "peak": peak, "unit": "G pairs/s", "frac": achieved / peak, "traffic": None,
+        traffic, dom = traffic_per_launch(w)
+        roof = {"bound": "alu", "kernel": f"{dom}: one MUFU ex2 per pair", "achieved": achieved,
+                "peak": peak, "unit": "G pairs/s", "frac": achieved / peak, "traffic": traffic,
                 "peak_basis": f"16 ex2/clk/SM x {sms} SMs x {sm_max:.0f} MHz (max SM clock)"}
         if clocks.get("sm_mhz"):
             roof["frac_at_measured_clock"] = achieved / (EX2_PER_CLK_PER_SM * sms * clocks["sm_mhz"] * 1e-3)

@@ -113,12 +113,34 @@ gs_status gauss_lse_fwd(const void *x, const void *y, const void *w, float *out,
  *     grad_x[b,i,k] = -tau * sum_j K_ij (sum_c g[b,i,c] w[b,j,c]) (x_ik - y_jk)   [B, M, D]
  *
  * with K_ij = exp(-tau/2 |x_i - y_j|^2), recomputed tile by tile, never stored.
- * Either output may be NULL to skip it.  Both outputs are float32.
+ * Either output may be NULL to skip it.  Both outputs are float32.  Same as
+ * gauss_sum_vjp with grad_y = grad_tau = NULL.
  */
 gs_status gauss_sum_bwd(const void *x, const void *y, const void *w, const float *g,
                         float *grad_x, float *grad_w, int64_t B, int64_t M, int64_t N, int64_t D,
                         int64_t C, float tau, gs_dtype dt, void *ws, size_t ws_bytes,
                         gs_stream_t stream);
+
+/*
+ * Every first-order gradient of L = sum_{b,i,c} g[b,i,c] * out[b,i,c] for the
+ * Gaussian kernel sum ("Kernel matrix reduction", Variants: derivatives through
+ * the fused reduction, for every input):
+ *
+ *     grad_x[b,i,k] = -tau sum_j K_ij (g_i . w_j) (x_ik - y_jk)            [B, M, D]
+ *     grad_y[b,j,k] = -tau sum_i K_ij (g_i . w_j) (y_jk - x_ik)            [B, N, D]
+ *     grad_w[b,j,c] = sum_i K_ij g[b,i,c]                                  [B, N, C]
+ *     grad_tau[0]   = -1/2 sum_b sum_ij K_ij |x_i - y_j|^2 (g_i . w_j)     one float
+ *
+ * Any output may be NULL to skip it (grad_tau needs no alignment).  Two passes
+ * of the fused kernels at most (rows y for grad_w / grad_y, rows x for grad_x /
+ * grad_tau), tiles recomputed, never stored; coordinates in the augmented
+ * values are centred at the first row point of each batch.  Workspace:
+ * gs_workspace_bytes(GS_OP_SUM_BWD, ...).  grad_tau is a fixed-order reduction.
+ */
+gs_status gauss_sum_vjp(const void *x, const void *y, const void *w, const float *g,
+                        float *grad_x, float *grad_y, float *grad_w, float *grad_tau, int64_t B,
+                        int64_t M, int64_t N, int64_t D, int64_t C, float tau, gs_dtype dt,
+                        void *ws, size_t ws_bytes, gs_stream_t stream);
 
 /*
  * Allocation-free variant of gauss_sum_fwd (no counterpart on the pages: it

@@ -38,6 +38,8 @@ SIGNATURES = {
                                      ctypes.c_int, _vp, _sz, _vp]),
     "gauss_sum_bwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64,
                                      _f, ctypes.c_int, _vp, _sz, _vp]),
+    "gauss_sum_vjp": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                                     _i64, _f, ctypes.c_int, _vp, _sz, _vp]),
     "gs_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "gs_last_device_error": (ctypes.c_int, [_vp]),
     "gs_version": (ctypes.c_int, []),
@@ -182,6 +184,28 @@ def gauss_sum_bwd(x, y, w, g, tau, want_x=True, want_w=True, workspace=None, str
     return gx, gw
 
 
+def gauss_sum_vjp(x, y, w, g, tau, want=("x", "y", "w", "tau"), workspace=None, stream=None):
+    """Every first-order gradient of sum(g * gauss_sum_fwd(x, y, w, tau)):
+    returns a dict with the requested keys among x, y, w, tau."""
+    x, y, w, g = _as3(x, "x"), _as3(y, "y"), _as3(w, "w"), _as3(g, "g")
+    B, M, N, D, C = _dims(x, y, w)
+    if g.shape != (B, M, C) or g.dtype != torch.float32:
+        raise ValueError(f"g must be float32 of shape {(B, M, C)}")
+    dev = x.device
+    out = {"x": torch.empty((B, M, D), dtype=torch.float32, device=dev) if "x" in want else None,
+           "y": torch.empty((B, N, D), dtype=torch.float32, device=dev) if "y" in want else None,
+           "w": torch.empty((B, N, C), dtype=torch.float32, device=dev) if "w" in want else None,
+           "tau": torch.empty((1,), dtype=torch.float32, device=dev) if "tau" in want else None}
+    nbytes = workspace_bytes(GS_OP_SUM_BWD, B, M, N, D, C, x.dtype)
+    ws = _workspace(nbytes, dev, workspace)
+    p = lambda t: _ptr(t) if t is not None else None
+    st = _lib.gauss_sum_vjp(_ptr(x), _ptr(y), _ptr(w), _ptr(g), p(out["x"]), p(out["y"]),
+                            p(out["w"]), p(out["tau"]), B, M, N, D, C, float(tau), _DT[x.dtype],
+                            _ptr(ws), nbytes if ws is not None else 0, _stream(stream))
+    _check("gauss_sum_vjp", st)
+    return {k: v for k, v in out.items() if v is not None}
+
+
 def test_exp2_poly(x, degree, stream=None):
     """Device evaluation of the FMA-pipe 2^x (test hook, see include/gauss_testing.h)."""
     if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
@@ -197,6 +221,6 @@ def last_device_error(stream=None):
     return int(_lib.gs_last_device_error(_stream(stream)))
 
 
-__all__ = ["gauss_sum_fwd", "gauss_sum_fwd_noalloc", "gauss_lse_fwd", "gauss_sum_bwd", "workspace_bytes",
+__all__ = ["gauss_sum_fwd", "gauss_sum_fwd_noalloc", "gauss_lse_fwd", "gauss_sum_bwd", "gauss_sum_vjp", "workspace_bytes",
            "last_device_error", "library", "status_string", "GaussError", "SIGNATURES",
            "LIB_PATH"]

@@ -7,6 +7,7 @@
 #include <cstring>
 
 #include "internal.h"
+#include "values.cuh"
 
 using namespace gs;
 
@@ -86,10 +87,10 @@ float coord_scale(float tau) {
 struct Pass {
   const void* rows_pts;
   const void* cols_pts;
-  const void* w;
+  const void* w;       // value source [B, N, C] (values.cuh)
   bool w_is_f32;
-  bool bwd_values;
-  int64_t B, R, N;   // rows, columns
+  int vmode;           // values.cuh mode: 0 = w, 1 = [w, w (col - z)], 2 = + w |col - z|^2
+  int64_t B, R, N;     // rows, columns
   int D, C, CV;
   gs_dtype dt;
   float tau;
@@ -109,7 +110,7 @@ PassLayout pass_layout(const Pass& p, int sm) {
   L.tc = p.dt != GS_F32;
   if (!L.tc) {
     L.sd = sd_plan(p.B, p.R, p.N, p.D, p.CV, sm);
-    if (p.bwd_values) {
+    if (p.vmode != 0) {
       L.off_vals = off;
       off = align_up(off + size_t(p.B) * p.N * p.CV * 4);
     }
@@ -151,10 +152,10 @@ gs_status run_pass(const Pass& p, const PassLayout& L, float* out, uint8_t* ws, 
   }
   if (!L.tc) {
     const float* values = static_cast<const float*>(p.w);
-    if (p.bwd_values) {
+    if (p.vmode != 0) {
       float* v = reinterpret_cast<float*>(ws + L.off_vals);
-      GS_CUDA(launch_pack_bwd_values_f32(static_cast<const float*>(p.cols_pts), values, v, p.B, p.N,
-                                         p.D, p.C, s));
+      GS_CUDA(launch_pack_values_f32(p.w, true, p.cols_pts, p.rows_pts, p.dt, v, p.B, p.N, p.R,
+                                     p.D, p.C, p.vmode, s));
       values = v;
     }
     const int S = L.sd.splits;
@@ -189,7 +190,7 @@ gs_status run_pass(const Pass& p, const PassLayout& L, float* out, uint8_t* ws, 
   a.y = p.cols_pts;
   a.w = p.w;
   a.w_is_f32 = p.w_is_f32;
-  a.values = p.bwd_values ? kValuesBwd : kValuesW;
+  a.values = static_cast<TcValues>(p.vmode);
   a.C = p.C;
   a.CV = p.CV;
   a.out = dst;
@@ -217,7 +218,7 @@ Pass fwd_pass(const void* x, const void* y, const void* w, int64_t B, int64_t M,
   p.cols_pts = y;
   p.w = w;
   p.w_is_f32 = dt == GS_F32;
-  p.bwd_values = false;
+  p.vmode = 0;
   p.B = B;
   p.R = M;
   p.N = N;
@@ -229,35 +230,56 @@ Pass fwd_pass(const void* x, const void* y, const void* w, int64_t B, int64_t M,
   return p;
 }
 
-// Backward = two passes: grad_w from (rows = y, cols = x, values = g) and the
-// x-gradient values O = K [w, w (x) y] from (rows = x, cols = y), then an
-// elementwise epilogue.  They run one after the other and share the workspace;
-// O sits after the larger pass layout.
-struct BwdLayout {
-  Pass pw, px;
-  PassLayout lw, lx;
-  size_t off_o;
+// Gradients = up to two passes (grad.cu): rows y / columns x with values
+// [g, g (x - z)] for dL/dw and dL/dy, and rows x / columns y with values
+// [w, w (y - z) (, w |y - z|^2)] for dL/dx (and dL/dtau), each followed by an
+// epilogue.  They run one after the other and share the pass scratch; the
+// pass outputs o_y, o_x and the per-row dL/dtau terms sit after it.
+struct VjpLayout {
+  Pass py, px;
+  PassLayout ly, lx;
+  bool do_y, do_x, y_direct;   // y_direct: the y pass writes grad_w itself
+  size_t off_oy, off_ox, off_tau;
   size_t total;
 };
 
-BwdLayout bwd_layout(const void* x, const void* y, const void* w, const float* g, int64_t B,
+VjpLayout vjp_layout(const void* x, const void* y, const void* w, const float* g, int64_t B,
                      int64_t M, int64_t N, int64_t D, int64_t C, float tau, gs_dtype dt, int sm,
-                     bool want_x, bool want_w) {
-  BwdLayout L{};
-  L.pw = fwd_pass(y, x, g, B, N, M, D, C, tau, dt);
-  L.pw.w_is_f32 = true;
+                     bool want_x, bool want_y, bool want_w, bool want_tau) {
+  VjpLayout L{};
+  L.do_y = want_w || want_y;
+  L.do_x = want_x || want_tau;
+  L.py = fwd_pass(y, x, g, B, N, M, D, C, tau, dt);
+  L.py.w_is_f32 = true;
+  L.py.vmode = want_y ? 1 : 0;
+  L.py.CV = value_channels(L.py.vmode, static_cast<int>(C), static_cast<int>(D));
+  L.y_direct = !want_y;
   L.px = fwd_pass(x, y, w, B, M, N, D, C, tau, dt);
-  L.px.bwd_values = true;
-  L.px.CV = static_cast<int>(C * (1 + D));
-  L.lw = pass_layout(L.pw, sm);
-  L.lx = pass_layout(L.px, sm);
-  size_t need = 0;
-  if (want_w) need = L.lw.total;
-  if (want_x) {
-    L.off_o = align_up(L.lx.total > need ? L.lx.total : need);
-    need = align_up(L.off_o + size_t(B) * M * C * (1 + D) * 4);
+  L.px.vmode = want_tau ? 2 : 1;
+  L.px.CV = value_channels(L.px.vmode, static_cast<int>(C), static_cast<int>(D));
+  size_t scratch = 0;
+  if (L.do_y) {
+    L.ly = pass_layout(L.py, sm);
+    scratch = L.ly.total;
   }
-  L.total = need;
+  if (L.do_x) {
+    L.lx = pass_layout(L.px, sm);
+    if (L.lx.total > scratch) scratch = L.lx.total;
+  }
+  size_t off = align_up(scratch);
+  if (L.do_y && !L.y_direct) {
+    L.off_oy = off;
+    off = align_up(off + size_t(B) * N * L.py.CV * 4);
+  }
+  if (L.do_x) {
+    L.off_ox = off;
+    off = align_up(off + size_t(B) * M * L.px.CV * 4);
+  }
+  if (want_tau) {
+    L.off_tau = off;
+    off = align_up(off + size_t(B) * M * 4);
+  }
+  L.total = off;
   return L;
 }
 
@@ -296,7 +318,9 @@ size_t gs_workspace_bytes(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, 
     return align_up(size_t(2) * sp.splits * B * M * C * 4);
   }
   if (M == 0 || N == 0) return 0;
-  return bwd_layout(nullptr, nullptr, nullptr, nullptr, B, M, N, D, C, 1.f, dt, sm, true, true).total;
+  return vjp_layout(nullptr, nullptr, nullptr, nullptr, B, M, N, D, C, 1.f, dt, sm, true, true, true,
+                    true)
+      .total;
 }
 
 gs_status gauss_sum_fwd(const void* x, const void* y, const void* w, float* out, int64_t B,
@@ -382,10 +406,10 @@ gs_status gauss_lse_fwd(const void* x, const void* y, const void* w, float* out,
   return GS_OK;
 }
 
-gs_status gauss_sum_bwd(const void* x, const void* y, const void* w, const float* g,
-                        float* grad_x, float* grad_w, int64_t B, int64_t M, int64_t N, int64_t D,
-                        int64_t C, float tau, gs_dtype dt, void* ws, size_t ws_bytes,
-                        gs_stream_t stream) {
+gs_status gauss_sum_vjp(const void* x, const void* y, const void* w, const float* g,
+                        float* grad_x, float* grad_y, float* grad_w, float* grad_tau, int64_t B,
+                        int64_t M, int64_t N, int64_t D, int64_t C, float tau, gs_dtype dt,
+                        void* ws, size_t ws_bytes, gs_stream_t stream) {
   GS_TRY(check_dims(GS_OP_SUM_BWD, B, M, N, D, C, dt));
   GS_TRY(check_tau(tau));
   GS_TRY(check_ptr(x, B * M * D));
@@ -393,28 +417,52 @@ gs_status gauss_sum_bwd(const void* x, const void* y, const void* w, const float
   GS_TRY(check_ptr(w, B * N * C));
   GS_TRY(check_ptr(g, B * M * C));
   if (grad_x) GS_TRY(check_ptr(grad_x, B * M * D));
+  if (grad_y) GS_TRY(check_ptr(grad_y, B * N * D));
   if (grad_w) GS_TRY(check_ptr(grad_w, B * N * C));
-  if (B == 0 || (!grad_x && !grad_w)) return GS_OK;
+  if (!grad_x && !grad_y && !grad_w && !grad_tau) return GS_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const bool want_x = grad_x != nullptr && M > 0;
-  const bool want_w = grad_w != nullptr && N > 0;
-  if (grad_x && M > 0 && N == 0) GS_CUDA(cudaMemsetAsync(grad_x, 0, size_t(B) * M * D * 4, s));
-  if (grad_w && N > 0 && M == 0) GS_CUDA(cudaMemsetAsync(grad_w, 0, size_t(B) * N * C * 4, s));
-  if (M == 0 || N == 0) return GS_OK;
-  const BwdLayout L = bwd_layout(x, y, w, g, B, M, N, D, C, tau, dt, sm_count(), want_x, want_w);
+  if (grad_tau) GS_CUDA(cudaMemsetAsync(grad_tau, 0, sizeof(float), s));
+  if (B == 0) return GS_OK;
+  if (M == 0 || N == 0) {   // every kernel sum is empty: all gradients vanish
+    if (grad_x && M > 0) GS_CUDA(cudaMemsetAsync(grad_x, 0, size_t(B) * M * D * 4, s));
+    if (grad_y && N > 0) GS_CUDA(cudaMemsetAsync(grad_y, 0, size_t(B) * N * D * 4, s));
+    if (grad_w && N > 0) GS_CUDA(cudaMemsetAsync(grad_w, 0, size_t(B) * N * C * 4, s));
+    return GS_OK;
+  }
+  const VjpLayout L = vjp_layout(x, y, w, g, B, M, N, D, C, tau, dt, sm_count(), grad_x != nullptr,
+                                 grad_y != nullptr, grad_w != nullptr, grad_tau != nullptr);
   if (L.total > 0) {
     if (ws_bytes < L.total) return GS_ERR_WORKSPACE;
     GS_TRY(check_ptr(ws, 1));
   }
   uint8_t* wsb = static_cast<uint8_t*>(ws);
-  if (want_w) GS_TRY(run_pass(L.pw, L.lw, grad_w, wsb, s));
-  if (want_x) {
-    float* o = reinterpret_cast<float*>(wsb + L.off_o);
-    GS_TRY(run_pass(L.px, L.lx, o, wsb, s));
-    GS_CUDA(launch_bwd_grad_x_epilogue(x, dt, g, o, grad_x, B, M, static_cast<int>(D),
-                                       static_cast<int>(C), tau, s));
+  if (L.do_y) {
+    if (L.y_direct) {
+      GS_TRY(run_pass(L.py, L.ly, grad_w, wsb, s));
+    } else {
+      float* oy = reinterpret_cast<float*>(wsb + L.off_oy);
+      GS_TRY(run_pass(L.py, L.ly, oy, wsb, s));
+      GS_CUDA(launch_grad_y_epilogue(y, w, dt, oy, grad_y, grad_w, B, N, static_cast<int>(D),
+                                     static_cast<int>(C), L.py.CV, tau, s));
+    }
+  }
+  if (L.do_x) {
+    float* ox = reinterpret_cast<float*>(wsb + L.off_ox);
+    float* tau_rows = grad_tau ? reinterpret_cast<float*>(wsb + L.off_tau) : nullptr;
+    GS_TRY(run_pass(L.px, L.lx, ox, wsb, s));
+    GS_CUDA(launch_grad_x_epilogue(x, dt, g, ox, grad_x, tau_rows, B, M, static_cast<int>(D),
+                                   static_cast<int>(C), L.px.CV, tau, s));
+    if (grad_tau) GS_CUDA(launch_sum_rows(tau_rows, B * M, grad_tau, s));
   }
   return GS_OK;
+}
+
+gs_status gauss_sum_bwd(const void* x, const void* y, const void* w, const float* g,
+                        float* grad_x, float* grad_w, int64_t B, int64_t M, int64_t N, int64_t D,
+                        int64_t C, float tau, gs_dtype dt, void* ws, size_t ws_bytes,
+                        gs_stream_t stream) {
+  return gauss_sum_vjp(x, y, w, g, grad_x, nullptr, grad_w, nullptr, B, M, N, D, C, tau, dt, ws,
+                       ws_bytes, stream);
 }
 
 gs_status gs_last_device_error(gs_stream_t stream) {

@@ -1,0 +1,207 @@
+// grad.cu -- packing and epilogue kernels of the gradient passes.
+//
+// Every gradient of the Gauss sum is assembled from forward passes of the fused
+// kernels with augmented values ("Kernel matrix reduction", Variants: gradients
+// run through the same fused reduction; the kernel tile is recomputed, never
+// stored), followed by small per-point epilogues:
+//
+//   pass over rows x, columns y, values [w, w (y - z), w |y - z|^2]  ->  o_x
+//     dL/dx[i,k] = -tau sum_c g_ic ((x_ik - z_k) o_x[i,c] - o_x[i, C + cD + k])
+//     dL/dtau    = -1/2 sum_i sum_c g_ic (|x_i - z|^2 o_x[i,c]
+//                      - 2 (x_i - z) . o_x[i, C + cD + :] + o_x[i, C(1+D) + c])
+//   pass over rows y, columns x, values [g, g (x - z)]              ->  o_y
+//     dL/dw[j,c] = o_y[j,c]
+//     dL/dy[j,k] = -tau sum_c w_jc ((y_jk - z_k) o_y[j,c] - o_y[j, C + cD + k])
+//
+// z is the first row point of each batch: the identities hold for any z (the
+// kernel only depends on differences), and centring keeps the values, and the
+// cancellation between the two terms, at the scale of the point cloud's spread
+// rather than of its distance from the origin.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "internal.h"
+#include "values.cuh"
+
+namespace gs {
+namespace {
+
+template <typename T>
+__device__ __forceinline__ float tf(T v);
+template <>
+__device__ __forceinline__ float tf<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float tf<__half>(__half v) { return __half2float(v); }
+template <>
+__device__ __forceinline__ float tf<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+int grid_for(int64_t n, int threads) {
+  int64_t b = (n + threads - 1) / threads;
+  if (b < 1) b = 1;
+  if (b > 148 * 32) b = 148 * 32;
+  return static_cast<int>(b);
+}
+
+// Value matrix, float32 [B, N, CV] (CUDA-core path) -------------------------------
+template <typename TS, typename TP>
+__global__ void pack_values_f32_kernel(const TS* __restrict__ src, const TP* __restrict__ cols,
+                                       const TP* __restrict__ rows, float* __restrict__ v,
+                                       int64_t B, int64_t N, int64_t Mrows, int D, int C,
+                                       int mode) {
+  const int CV = value_channels(mode, C, D);
+  const int64_t total = B * N * CV;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t bj = e / CV;
+    const int ch = static_cast<int>(e % CV);
+    const int64_t b = bj / N;
+    v[e] = value_at(src, cols, rows, b, bj, Mrows, D, C, ch);
+  }
+}
+
+// dL/dx (optional) and the per-row dL/dtau terms (optional) from o_x -------------
+template <typename T>
+__global__ void grad_x_epilogue_kernel(const T* __restrict__ x, const float* __restrict__ g,
+                                       const float* __restrict__ o, float* __restrict__ gx,
+                                       float* __restrict__ tau_rows, int64_t B, int64_t M, int D,
+                                       int C, int CV, float tau) {
+  const int64_t rows = B * M;
+  for (int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; r < rows;
+       r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = r / M;
+    const T* xi = x + r * D;
+    const T* z = x + b * M * D;
+    const float* oi = o + r * CV;
+    const float* gi = g + r * C;
+    float tau_acc = 0.f;
+    float xx = 0.f;
+    for (int k = 0; k < D; ++k) {
+      const float xk = tf(xi[k]) - tf(z[k]);
+      xx = fmaf(xk, xk, xx);
+      float s = 0.f;
+      for (int c = 0; c < C; ++c) s = fmaf(gi[c], fmaf(xk, oi[c], -oi[C + c * D + k]), s);
+      if (gx) gx[r * D + k] = -tau * s;
+      if (tau_rows) {
+        float cross = 0.f;
+        for (int c = 0; c < C; ++c) cross = fmaf(gi[c], oi[C + c * D + k], cross);
+        tau_acc = fmaf(-2.f * xk, cross, tau_acc);
+      }
+    }
+    if (tau_rows) {
+      for (int c = 0; c < C; ++c)
+        tau_acc = fmaf(gi[c], fmaf(xx, oi[c], oi[C * (1 + D) + c]), tau_acc);
+      tau_rows[r] = -0.5f * tau_acc;
+    }
+  }
+}
+
+// dL/dy (optional) and dL/dw from o_y ---------------------------------------------
+template <typename T>
+__global__ void grad_y_epilogue_kernel(const T* __restrict__ y, const T* __restrict__ w,
+                                       const float* __restrict__ o, float* __restrict__ gy,
+                                       float* __restrict__ gw, int64_t B, int64_t N, int D, int C,
+                                       int CV, float tau) {
+  const int64_t rows = B * N;
+  for (int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; r < rows;
+       r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = r / N;
+    const T* yj = y + r * D;
+    const T* z = y + b * N * D;
+    const T* wj = w + r * C;
+    const float* oj = o + r * CV;
+    if (gw)
+      for (int c = 0; c < C; ++c) gw[r * C + c] = oj[c];
+    if (gy) {
+      for (int k = 0; k < D; ++k) {
+        const float yk = tf(yj[k]) - tf(z[k]);
+        float s = 0.f;
+        for (int c = 0; c < C; ++c) s = fmaf(tf(wj[c]), fmaf(yk, oj[c], -oj[C + c * D + k]), s);
+        gy[r * D + k] = -tau * s;
+      }
+    }
+  }
+}
+
+// Fixed-order reduction of the per-row dL/dtau terms: one block, each thread
+// sums a strided slice in order, then a fixed tree in shared memory.
+__global__ void sum_rows_kernel(const float* __restrict__ v, int64_t n, float* __restrict__ out) {
+  __shared__ double part[1024];
+  double s = 0.0;
+  for (int64_t e = threadIdx.x; e < n; e += blockDim.x) s += static_cast<double>(v[e]);
+  part[threadIdx.x] = s;
+  __syncthreads();
+  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
+    if (threadIdx.x < o) part[threadIdx.x] += part[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *out = static_cast<float>(part[0]);
+}
+
+template <typename T>
+const T* as(const void* p) {
+  return static_cast<const T*>(p);
+}
+
+}  // namespace
+
+cudaError_t launch_pack_values_f32(const void* src, bool src_is_f32, const void* cols,
+                                   const void* rows, gs_dtype pt, float* v, int64_t B, int64_t N,
+                                   int64_t Mrows, int D, int C, int mode, cudaStream_t s) {
+  const int64_t n = B * N * value_channels(mode, C, D);
+  const int blocks = grid_for(n, 256);
+  // the CUDA-core path only runs float32 points and values
+  (void)src_is_f32;
+  (void)pt;
+  pack_values_f32_kernel<float, float><<<blocks, 256, 0, s>>>(
+      as<float>(src), as<float>(cols), as<float>(rows), v, B, N, Mrows, D, C, mode);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_grad_x_epilogue(const void* x, gs_dtype dt, const float* g, const float* o,
+                                   float* grad_x, float* tau_rows, int64_t B, int64_t M, int D,
+                                   int C, int CV, float tau, cudaStream_t s) {
+  const int blocks = grid_for(B * M, 256);
+  switch (dt) {
+    case GS_F32:
+      grad_x_epilogue_kernel<float><<<blocks, 256, 0, s>>>(as<float>(x), g, o, grad_x, tau_rows, B,
+                                                           M, D, C, CV, tau);
+      break;
+    case GS_F16:
+      grad_x_epilogue_kernel<__half><<<blocks, 256, 0, s>>>(as<__half>(x), g, o, grad_x, tau_rows,
+                                                            B, M, D, C, CV, tau);
+      break;
+    default:
+      grad_x_epilogue_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+          as<__nv_bfloat16>(x), g, o, grad_x, tau_rows, B, M, D, C, CV, tau);
+      break;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_grad_y_epilogue(const void* y, const void* w, gs_dtype dt, const float* o,
+                                   float* grad_y, float* grad_w, int64_t B, int64_t N, int D,
+                                   int C, int CV, float tau, cudaStream_t s) {
+  const int blocks = grid_for(B * N, 256);
+  switch (dt) {
+    case GS_F32:
+      grad_y_epilogue_kernel<float><<<blocks, 256, 0, s>>>(as<float>(y), as<float>(w), o, grad_y,
+                                                           grad_w, B, N, D, C, CV, tau);
+      break;
+    case GS_F16:
+      grad_y_epilogue_kernel<__half><<<blocks, 256, 0, s>>>(as<__half>(y), as<__half>(w), o,
+                                                            grad_y, grad_w, B, N, D, C, CV, tau);
+      break;
+    default:
+      grad_y_epilogue_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+          as<__nv_bfloat16>(y), as<__nv_bfloat16>(w), o, grad_y, grad_w, B, N, D, C, CV, tau);
+      break;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sum_rows(const float* v, int64_t n, float* out, cudaStream_t s) {
+  sum_rows_kernel<<<1, 1024, 0, s>>>(v, n, out);
+  return cudaGetLastError();
+}
+
+}  // namespace gs

@@ -77,14 +77,21 @@ struct LseFinalizeArgs {
 };
 cudaError_t launch_lse_finalize(const LseFinalizeArgs& a, cudaStream_t s);
 
-// Value matrix for the x-gradient on the fp32 path: v = [w, w (x) y], [B, N, C*(1+D)].
-cudaError_t launch_pack_bwd_values_f32(const float* y, const float* w, float* v, int64_t B,
-                                       int64_t N, int D, int C, cudaStream_t s);
+// Value matrix of a pass on the CUDA-core path, float32 [B, N, CV] (values.cuh).
+cudaError_t launch_pack_values_f32(const void* src, bool src_is_f32, const void* cols,
+                                   const void* rows, gs_dtype pt, float* v, int64_t B, int64_t N,
+                                   int64_t Mrows, int D, int C, int mode, cudaStream_t s);
 
-// grad_x[b,i,k] = -tau * sum_c g[b,i,c] (x[b,i,k] * o[b,i,c] - o[b,i,C + c*D + k])
-cudaError_t launch_bwd_grad_x_epilogue(const void* x, gs_dtype dt, const float* g,
-                                       const float* o, float* grad_x, int64_t B, int64_t M,
-                                       int D, int C, float tau, cudaStream_t s);
+// Gradient epilogues (grad.cu).  grad_x and tau_rows may each be NULL; so may
+// grad_y and grad_w.
+cudaError_t launch_grad_x_epilogue(const void* x, gs_dtype dt, const float* g, const float* o,
+                                   float* grad_x, float* tau_rows, int64_t B, int64_t M, int D,
+                                   int C, int CV, float tau, cudaStream_t s);
+cudaError_t launch_grad_y_epilogue(const void* y, const void* w, gs_dtype dt, const float* o,
+                                   float* grad_y, float* grad_w, int64_t B, int64_t N, int D,
+                                   int C, int CV, float tau, cudaStream_t s);
+// out[0] = sum of v[0 .. n) in a fixed order (double accumulation).
+cudaError_t launch_sum_rows(const float* v, int64_t n, float* out, cudaStream_t s);
 
 // ------------------------------------------------------------- tensor-core path
 constexpr int kTcMaxD = 126;
@@ -97,17 +104,17 @@ struct TcPlan {
 };
 TcPlan tc_plan(int64_t B, int64_t M, int64_t N, int64_t D, int sm_count);
 
-// Which values the tensor-core pass multiplies by the kernel.
-enum TcValues { kValuesW = 0, kValuesBwd = 1 };
+// Which values the tensor-core pass multiplies by the kernel (values.cuh modes).
+enum TcValues { kValuesW = 0, kValuesBwd = 1, kValuesBwdTau = 2 };
 
 struct TcArgs {
   const void* x;       // rows side [B, M, D]
   const void* y;       // column side [B, N, D]
   const void* w;       // values source [B, N, C] (dtype dt, or float32 if w_is_f32)
   bool w_is_f32;
-  TcValues values;     // kValuesW: v = w; kValuesBwd: v = [w, w (x) y]
+  TcValues values;     // value mode (values.cuh), columns centred at x[b, 0]
   int C;               // channels of w
-  int CV;              // channels of the value matrix (C or C*(1+D))
+  int CV;              // channels of the value matrix
   float* out;          // [S?][B][M][CV]
   int64_t split_stride;
   int64_t B, M, N;

@@ -371,55 +371,6 @@ __global__ void lse_finalize_kernel(const LseFinalizeArgs a) {
   }
 }
 
-// ------------------------------------------------------------------ backward helpers
-__global__ void pack_bwd_values_f32_kernel(const float* __restrict__ y,
-                                           const float* __restrict__ w, float* __restrict__ v,
-                                           int64_t rows, int D, int C) {
-  const int CV = C * (1 + D);
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-       e < rows * CV; e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t j = e / CV;
-    const int ch = static_cast<int>(e % CV);
-    float val;
-    if (ch < C) {
-      val = w[j * C + ch];
-    } else {
-      const int c = (ch - C) / D, k = (ch - C) % D;
-      val = w[j * C + c] * y[j * D + k];
-    }
-    v[e] = val;
-  }
-}
-
-template <typename T>
-__device__ __forceinline__ float to_f32(T v);
-template <>
-__device__ __forceinline__ float to_f32<float>(float v) { return v; }
-template <>
-__device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
-template <>
-__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
-  return __bfloat162float(v);
-}
-
-template <typename T>
-__global__ void grad_x_epilogue_kernel(const T* __restrict__ x, const float* __restrict__ g,
-                                       const float* __restrict__ o, float* __restrict__ gx,
-                                       int64_t rows, int D, int C, float tau) {
-  const int CV = C * (1 + D);
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < rows * D;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t i = e / D;
-    const int k = static_cast<int>(e % D);
-    const float xk = to_f32(x[e]);
-    const float* oi = o + i * CV;
-    const float* gi = g + i * C;
-    float s = 0.f;
-    for (int c = 0; c < C; ++c) s = fmaf(gi[c], fmaf(xk, oi[c], -oi[C + c * D + k]), s);
-    gx[e] = -tau * s;
-  }
-}
-
 __global__ void fill_kernel(float* __restrict__ out, int64_t n, float value) {
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x)
@@ -505,35 +456,6 @@ cudaError_t launch_lse_finalize(const LseFinalizeArgs& a, cudaStream_t s) {
 cudaError_t launch_fill(float* out, int64_t n, float value, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
   fill_kernel<<<grid_for(n, 256), 256, 0, s>>>(out, n, value);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_pack_bwd_values_f32(const float* y, const float* w, float* v, int64_t B,
-                                       int64_t N, int D, int C, cudaStream_t s) {
-  const int64_t n = B * N * C * (1 + D);
-  pack_bwd_values_f32_kernel<<<grid_for(n, 256), 256, 0, s>>>(y, w, v, B * N, D, C);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_bwd_grad_x_epilogue(const void* x, gs_dtype dt, const float* g,
-                                       const float* o, float* grad_x, int64_t B, int64_t M,
-                                       int D, int C, float tau, cudaStream_t s) {
-  const int64_t n = B * M * D;
-  const int blocks = grid_for(n, 256);
-  switch (dt) {
-    case GS_F32:
-      grad_x_epilogue_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(x), g, o,
-                                                           grad_x, B * M, D, C, tau);
-      break;
-    case GS_F16:
-      grad_x_epilogue_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<const __half*>(x), g, o,
-                                                            grad_x, B * M, D, C, tau);
-      break;
-    default:
-      grad_x_epilogue_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
-          static_cast<const __nv_bfloat16*>(x), g, o, grad_x, B * M, D, C, tau);
-      break;
-  }
   return cudaGetLastError();
 }
 

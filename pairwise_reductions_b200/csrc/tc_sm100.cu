@@ -35,6 +35,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "values.cuh"
 
 namespace gs {
 
@@ -72,7 +73,7 @@ struct TcCfg {
   static constexpr int STAGE = Y_BYTES + V_BYTES;
   static constexpr int NST_FIT = (200 * 1024 - X_BYTES) / STAGE;
   static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
-  static constexpr int NBARS = 2 * NST + 9;
+  static constexpr int NBARS = 2 * NST + 11;
   static constexpr int SMEM_RAW = 1024 + X_BYTES + NST * STAGE + 8 * NBARS + 16;
   // at least ~120 KB so that a second CTA never lands on the SM and blocks on
   // the 512-column TMEM allocation
@@ -179,6 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_p = [&](int h) { return bar0 + 8u * (2 * NST + 3 + h); };   // P tile h written
   const uint32_t bar_o = bar0 + 8u * (2 * NST + 5);
   auto bar_f = [&](int h) { return bar0 + 8u * (2 * NST + 7 + h); };   // S tile h read out
+  auto bar_q = [&](int h) { return bar0 + 8u * (2 * NST + 9 + h); };   // P tile h consumed
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t b = blockIdx.z;
@@ -200,6 +202,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_o, 1);
     mbar_init(bar_f(0), 4 * 32);
     mbar_init(bar_f(1), 4 * 32);
+    mbar_init(bar_q(0), 1);
+    mbar_init(bar_q(1), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -292,6 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = wait_bar(bar_p(0), t & 1, abort_flag))) break;
           tc_fence_after();
           issue_O(0, st, t > 0);
+          mma_commit(bar_q(0));
           if (t + 1 < T) {
             if (!(ok = wait_bar(bar_f(1), t & 1, abort_flag))) break;
             tc_fence_after();
@@ -301,6 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = wait_bar(bar_p(1), t & 1, abort_flag))) break;
           tc_fence_after();
           issue_O(1, st, t > 0);
+          mma_commit(bar_q(1));
           mma_commit(bar_empty(st));
         } else {
           // P lives in the S columns: the next S MMA must follow the P MMA
@@ -362,6 +368,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ch + 1 < kBN / 32) tmem_ld32(tS + (ch + 1) * 32, nxt);
         uint32_t pk[16];
         exp_chunk(cur, two_c2, r2, pk);
+        if (Cfg::P_SEPARATE && ch == 0 && t > 0) {
+          // a warp that runs ahead must not overwrite its rows of P(t-1) before
+          // the P MMA of tile t-1 has read them (waited for as late as possible)
+          ok = __all_sync(0xffffffffu, wait_bar(bar_q(h), (t - 1) & 1, abort_flag));
+          if (!ok) {
+            tmem_wait_ld();   // the next chunk's load may still be in flight
+            break;
+          }
+          tc_fence_after();
+        }
         tmem_st16(tP + ch * 16, pk);
         if (ch + 1 < kBN / 32) {
           tmem_wait_ld();
@@ -373,6 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      if (!ok) break;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p(h));
@@ -482,12 +499,13 @@ __global__ void pack_rows_kernel(const T* __restrict__ src, T* __restrict__ dst,
 }
 
 // Transposed fp16 value matrix v^T [B, CP, Nst] for channels [c0, c0 + CP) of
-// either v = w (kValuesW) or v = [w, w (x) y] (kValuesBwd).  Channels past CV
-// are written as zeros.
+// the pass's value matrix (values.cuh; columns = the y side of this pass,
+// centre = its first row point).  Channels past CV are written as zeros.
 template <typename TW, typename TY>
 __global__ void pack_values_kernel(const TW* __restrict__ w, const TY* __restrict__ y,
-                                   __half* __restrict__ vt, int64_t B, int64_t N, int64_t Nst,
-                                   int C, int D, int CV, int c0, int CP, int bwd) {
+                                   const TY* __restrict__ rows, __half* __restrict__ vt, int64_t B,
+                                   int64_t N, int64_t Nst, int64_t Mrows, int C, int D, int CV,
+                                   int c0, int CP) {
   const int64_t total = B * CP * N;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -496,16 +514,7 @@ __global__ void pack_values_kernel(const TW* __restrict__ w, const TY* __restric
     const int cc = static_cast<int>(bc % CP);
     const int64_t b = bc / CP;
     const int ch = c0 + cc;
-    float v = 0.f;
-    if (ch < CV) {
-      const int64_t bj = b * N + j;
-      if (!bwd || ch < C) {
-        v = tof(w[bj * C + ch]);
-      } else {
-        const int cw = (ch - C) / D, k = (ch - C) % D;
-        v = tof(w[bj * C + cw]) * tof(y[bj * D + k]);
-      }
-    }
+    const float v = (ch < CV) ? value_at(w, y, rows, b, b * N + j, Mrows, D, C, ch) : 0.f;
     vt[(b * CP + cc) * Nst + j] = __float2half_rn(v);
   }
 }
@@ -576,15 +585,16 @@ template <typename T>
 cudaError_t pack_values(const TcArgs& a, int c0, int CP, int64_t Nst, cudaStream_t s) {
   const int64_t total = a.B * CP * a.N;
   const int blocks = grid_for(total, 256);
-  const int bwd = a.values == kValuesBwd ? 1 : 0;
+  const T* y = static_cast<const T*>(a.y);
+  const T* rows = static_cast<const T*>(a.x);
   if (a.w_is_f32)
-    pack_values_kernel<float, T><<<blocks, 256, 0, s>>>(
-        static_cast<const float*>(a.w), static_cast<const T*>(a.y), static_cast<__half*>(a.vt),
-        a.B, a.N, Nst, a.C, a.D, a.CV, c0, CP, bwd);
+    pack_values_kernel<float, T><<<blocks, 256, 0, s>>>(static_cast<const float*>(a.w), y, rows,
+                                                        static_cast<__half*>(a.vt), a.B, a.N, Nst,
+                                                        a.M, a.C, a.D, a.CV, c0, CP);
   else
-    pack_values_kernel<T, T><<<blocks, 256, 0, s>>>(
-        static_cast<const T*>(a.w), static_cast<const T*>(a.y), static_cast<__half*>(a.vt), a.B,
-        a.N, Nst, a.C, a.D, a.CV, c0, CP, bwd);
+    pack_values_kernel<T, T><<<blocks, 256, 0, s>>>(static_cast<const T*>(a.w), y, rows,
+                                                    static_cast<__half*>(a.vt), a.B, a.N, Nst, a.M,
+                                                    a.C, a.D, a.CV, c0, CP);
   return cudaGetLastError();
 }
 

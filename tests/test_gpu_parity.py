@@ -237,3 +237,65 @@ def test_abi_rejects_bad_arguments_on_device():
     ho = torch.empty(1, 300, 32, device="cuda")
     assert lib.gauss_sum_fwd(p(h), p(h), p(h), p(ho), 1, 300, 300, 32, 32, 1.0, 1, None, 0, s) == 4
     assert m.last_device_error() == 0
+
+
+@pytest.mark.parametrize("C", [1, 32, 96])
+def test_tensor_core_path_is_deterministic_under_repetition(C):
+    """Twenty identical calls give bit-identical results: a race between the
+    exp warps and the MMAs (a P tile overwritten before it is consumed, an S
+    tile before it is read) would show up as run-to-run differences."""
+    m = gs()
+    h = synth.make_inputs(4, seed=31, B=2, M=1000, N=3000, C=C)
+    d = dev(h)
+    ref = m.gauss_sum_fwd(d["x"], d["y"], d["w"], 1.0)
+    for _ in range(19):
+        assert torch.equal(m.gauss_sum_fwd(d["x"], d["y"], d["w"], 1.0), ref)
+    ro = oracle.gauss_sum(f64(h, "x"), f64(h, "y"), f64(h, "w"), 1.0, rows=np.arange(0, 1000, 7))
+    assert rel_l2(ref.cpu().numpy()[:, ::7], ro) <= TOL["f16"]
+
+
+# ------------------------------------------------------------------ full gradient
+@pytest.mark.parametrize("dtype,shape,shift", [
+    ("f32", (1, 400, 600, 3, 1), 0.0), ("f32", (2, 300, 500, 2, 3), 0.0), ("f32", (1, 250, 350, 8, 2), 0.0),
+    ("f32", (1, 300, 400, 3, 1), 40.0),
+    ("f16", (1, 300, 500, 32, 1), 0.0), ("f16", (2, 257, 300, 16, 4), 0.0), ("bf16", (1, 200, 333, 32, 1), 0.0),
+    ("f16", (1, 300, 500, 16, 2), 20.0),
+])
+def test_vjp_every_gradient(dtype, shape, shift):
+    """dL/dx, dL/dy, dL/dw and dL/dtau against the oracle; `shift` moves the
+    whole point cloud away from the origin (the gradients do not change, the
+    centred values keep the cancellation at the cloud's own scale)."""
+    B, M, N, D, C = shape
+    wid = 1 if dtype == "f32" else 5
+    inp = synth.make_inputs(wid, seed=13, B=B, M=M, N=N, D=D, C=C, dtype=dtype, with_g=True)
+    if shift:
+        for k in ("x", "y"):
+            inp[k] = (inp[k].double() + shift).to(inp[k].dtype)
+    d = dev(inp)
+    got = gs().gauss_sum_vjp(d["x"], d["y"], d["w"], d["g"], inp["tau"])
+    x, y, w, g = (f64(inp, k) for k in "xywg")
+    rgx, rgw = oracle.gauss_sum_bwd(x, y, w, g, inp["tau"])
+    rgy, rgt = oracle.gauss_sum_vjp_y_tau(x, y, w, g, inp["tau"])
+    tol = TOL[dtype]
+    for name, ref in (("x", rgx), ("y", rgy), ("w", rgw)):
+        e = rel_l2(got[name].cpu().numpy(), ref)
+        assert e <= tol, (name, e)
+    et = abs(float(got["tau"].item()) - rgt) / max(abs(rgt), 1e-30)
+    assert et <= tol, ("tau", et, float(got["tau"].item()), rgt)
+    # subsets of outputs give the same values
+    only = gs().gauss_sum_vjp(d["x"], d["y"], d["w"], d["g"], inp["tau"], want=("y", "tau"))
+    assert torch.equal(only["y"], got["y"]) and torch.equal(only["tau"], got["tau"])
+
+
+def test_vjp_d32_c1_full_size_sampled():
+    inp = synth.make_inputs(5)
+    d = dev(inp)
+    got = gs().gauss_sum_vjp(d["x"], d["y"], d["w"], d["g"], inp["tau"], want=("x", "y", "w"))
+    x, y, w, g = (f64(inp, k) for k in "xywg")
+    rows = synth.sample_rows(inp["M"], 256, seed=14).numpy()
+    yrows = synth.sample_rows(inp["N"], 256, seed=15).numpy()
+    rgx, rgw = oracle.gauss_sum_bwd(x, y, w, g, inp["tau"], rows=rows, wrows=yrows)
+    rgy, _ = oracle.gauss_sum_vjp_y_tau(x, y, w, g, inp["tau"], yrows=yrows, want_tau=False)
+    assert rel_l2(got["x"].cpu().numpy()[:, rows], rgx) <= TOL["f16"]
+    assert rel_l2(got["w"].cpu().numpy()[:, yrows], rgw) <= TOL["f16"]
+    assert rel_l2(got["y"].cpu().numpy()[:, yrows], rgy) <= TOL["f16"]
