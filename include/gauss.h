@@ -57,7 +57,7 @@ typedef struct CUstream_st *gs_stream_t;
 
 typedef enum { GS_F32 = 0, GS_F16 = 1, GS_BF16 = 2 } gs_dtype;
 
-typedef enum { GS_OP_SUM = 0, GS_OP_LSE = 1, GS_OP_SUM_BWD = 2 } gs_op;
+typedef enum { GS_OP_SUM = 0, GS_OP_LSE = 1, GS_OP_SUM_BWD = 2, GS_OP_LSE_BWD = 3 } gs_op;
 
 typedef enum {
     GS_OK = 0,
@@ -141,6 +141,27 @@ gs_status gauss_sum_vjp(const void *x, const void *y, const void *w, const float
                         float *grad_x, float *grad_y, float *grad_w, float *grad_tau, int64_t B,
                         int64_t M, int64_t N, int64_t D, int64_t C, float tau, gs_dtype dt,
                         void *ws, size_t ws_bytes, gs_stream_t stream);
+
+/*
+ * Every first-order gradient of L = sum_{b,i,c} g[b,i,c] * lse[b,i,c] for the
+ * log-sum-exp reduction of gauss_lse_fwd ("Kernel matrix reduction", Overview
+ * and Variants: the log-sum-exp reduction and gradients through it).  With the
+ * normalised weights p_ijc = w_jc K_ij exp(-lse_ic):
+ *
+ *     grad_x[b,i,k] = -tau sum_c g_ic sum_j p_ijc (x_ik - y_jk)            [B, M, D]
+ *     grad_y[b,j,k] = -tau sum_i sum_c g_ic p_ijc (y_jk - x_ik)            [B, N, D]
+ *     grad_w[b,j,c] = sum_i g_ic K_ij exp(-lse_ic)                          [B, N, C]
+ *     grad_tau[0]   = -1/2 sum_ic g_ic sum_j p_ijc |x_i - y_j|^2             one float
+ *
+ * lse [B, M, C] float32 is the forward's output for the same inputs.  The
+ * shift -lse is folded into every kernel exponent, so the passes sum p
+ * directly (no overflow, no separate normalisation).  GS_F32, 1 <= D <= 8,
+ * w > 0; any output may be NULL.  Workspace: gs_workspace_bytes(GS_OP_LSE_BWD, ...).
+ */
+gs_status gauss_lse_bwd(const void *x, const void *y, const void *w, const float *lse,
+                        const float *g, float *grad_x, float *grad_y, float *grad_w,
+                        float *grad_tau, int64_t B, int64_t M, int64_t N, int64_t D, int64_t C,
+                        float tau, gs_dtype dt, void *ws, size_t ws_bytes, gs_stream_t stream);
 
 /*
  * Allocation-free variant of gauss_sum_fwd (no counterpart on the pages: it

@@ -23,7 +23,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = _build.LIB
 
 GS_F32, GS_F16, GS_BF16 = 0, 1, 2
-GS_OP_SUM, GS_OP_LSE, GS_OP_SUM_BWD = 0, 1, 2
+GS_OP_SUM, GS_OP_LSE, GS_OP_SUM_BWD, GS_OP_LSE_BWD = 0, 1, 2, 3
 STATUS = {0: "GS_OK", 1: "GS_ERR_INVALID_ARG", 2: "GS_ERR_UNSUPPORTED", 3: "GS_ERR_ALIGNMENT",
           4: "GS_ERR_WORKSPACE", 5: "GS_ERR_TIMEOUT", 6: "GS_ERR_CUDA"}
 _DT = {torch.float32: GS_F32, torch.float16: GS_F16, torch.bfloat16: GS_BF16}
@@ -40,6 +40,8 @@ SIGNATURES = {
                                      _f, ctypes.c_int, _vp, _sz, _vp]),
     "gauss_sum_vjp": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                      _i64, _f, ctypes.c_int, _vp, _sz, _vp]),
+    "gauss_lse_bwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                     _i64, _i64, _f, ctypes.c_int, _vp, _sz, _vp]),
     "gs_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "gs_last_device_error": (ctypes.c_int, [_vp]),
     "gs_version": (ctypes.c_int, []),
@@ -206,6 +208,29 @@ def gauss_sum_vjp(x, y, w, g, tau, want=("x", "y", "w", "tau"), workspace=None, 
     return {k: v for k, v in out.items() if v is not None}
 
 
+def gauss_lse_bwd(x, y, w, lse, g, tau, want=("x", "y", "w", "tau"), workspace=None, stream=None):
+    """Every first-order gradient of sum(g * lse) with lse = gauss_lse_fwd(x, y, w, tau)
+    (float32 inputs); returns a dict with the requested keys among x, y, w, tau."""
+    x, y, w, lse, g = (_as3(t, n) for t, n in ((x, "x"), (y, "y"), (w, "w"), (lse, "lse"), (g, "g")))
+    B, M, N, D, C = _dims(x, y, w)
+    for t, n in ((lse, "lse"), (g, "g")):
+        if t.shape != (B, M, C) or t.dtype != torch.float32:
+            raise ValueError(f"{n} must be float32 of shape {(B, M, C)}")
+    dev = x.device
+    out = {"x": torch.empty((B, M, D), dtype=torch.float32, device=dev) if "x" in want else None,
+           "y": torch.empty((B, N, D), dtype=torch.float32, device=dev) if "y" in want else None,
+           "w": torch.empty((B, N, C), dtype=torch.float32, device=dev) if "w" in want else None,
+           "tau": torch.empty((1,), dtype=torch.float32, device=dev) if "tau" in want else None}
+    nbytes = workspace_bytes(GS_OP_LSE_BWD, B, M, N, D, C, x.dtype)
+    ws = _workspace(nbytes, dev, workspace)
+    p = lambda t: _ptr(t) if t is not None else None
+    st = _lib.gauss_lse_bwd(_ptr(x), _ptr(y), _ptr(w), _ptr(lse), _ptr(g), p(out["x"]), p(out["y"]),
+                            p(out["w"]), p(out["tau"]), B, M, N, D, C, float(tau), _DT[x.dtype],
+                            _ptr(ws), nbytes if ws is not None else 0, _stream(stream))
+    _check("gauss_lse_bwd", st)
+    return {k: v for k, v in out.items() if v is not None}
+
+
 def test_exp2_poly(x, degree, stream=None):
     """Device evaluation of the FMA-pipe 2^x (test hook, see include/gauss_testing.h)."""
     if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
@@ -221,6 +246,6 @@ def last_device_error(stream=None):
     return int(_lib.gs_last_device_error(_stream(stream)))
 
 
-__all__ = ["gauss_sum_fwd", "gauss_sum_fwd_noalloc", "gauss_lse_fwd", "gauss_sum_bwd", "gauss_sum_vjp", "workspace_bytes",
+__all__ = ["gauss_sum_fwd", "gauss_sum_fwd_noalloc", "gauss_lse_fwd", "gauss_sum_bwd", "gauss_sum_vjp", "gauss_lse_bwd", "workspace_bytes",
            "last_device_error", "library", "status_string", "GaussError", "SIGNATURES",
            "LIB_PATH"]

@@ -49,7 +49,7 @@ gs_status check_dims(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, int64
     if (D > kSdMaxD) return GS_ERR_UNSUPPORTED;
   } else {
     if (D > kTcMaxD) return GS_ERR_UNSUPPORTED;
-    if (op == GS_OP_LSE) return GS_ERR_UNSUPPORTED;
+    if (op == GS_OP_LSE || op == GS_OP_LSE_BWD) return GS_ERR_UNSUPPORTED;
   }
   return GS_OK;
 }
@@ -94,6 +94,13 @@ struct Pass {
   int D, C, CV;
   gs_dtype dt;
   float tau;
+  int64_t src_ld;      // row stride of the value source (0 = C)
+  // exponent shift (CUDA-core path only, see SdArgs)
+  int shift_mode;
+  const float* shift_src;
+  int64_t shift_ld;
+  int shift_c;
+  float shift_scale;
 };
 
 struct PassLayout {
@@ -154,8 +161,8 @@ gs_status run_pass(const Pass& p, const PassLayout& L, float* out, uint8_t* ws, 
     const float* values = static_cast<const float*>(p.w);
     if (p.vmode != 0) {
       float* v = reinterpret_cast<float*>(ws + L.off_vals);
-      GS_CUDA(launch_pack_values_f32(p.w, true, p.cols_pts, p.rows_pts, p.dt, v, p.B, p.N, p.R,
-                                     p.D, p.C, p.vmode, s));
+      GS_CUDA(launch_pack_values_f32(p.w, p.src_ld > 0 ? p.src_ld : p.C, p.cols_pts, p.rows_pts,
+                                     v, p.B, p.N, p.R, p.D, p.C, p.vmode, s));
       values = v;
     }
     const int S = L.sd.splits;
@@ -165,7 +172,7 @@ gs_status run_pass(const Pass& p, const PassLayout& L, float* out, uint8_t* ws, 
       a.x = static_cast<const float*>(p.rows_pts);
       a.y = static_cast<const float*>(p.cols_pts);
       a.w = values;
-      a.ldw = p.CV;
+      a.ldw = (p.vmode == 0 && p.src_ld > 0) ? static_cast<int>(p.src_ld) : p.CV;
       a.c0 = c0;
       a.cw = (p.CV - c0) < kSdMaxChunk ? (p.CV - c0) : kSdMaxChunk;
       a.out = dst;
@@ -178,6 +185,11 @@ gs_status run_pass(const Pass& p, const PassLayout& L, float* out, uint8_t* ws, 
       a.D = p.D;
       a.scale = coord_scale(p.tau);
       a.plan = L.sd;
+      a.shift_mode = p.shift_mode;
+      a.shift_src = p.shift_src;
+      a.shift_ld = p.shift_ld;
+      a.shift_c = p.shift_c;
+      a.shift_scale = p.shift_scale;
       GS_CUDA(launch_small_d_sum(a, s));
     }
     if (S > 1) GS_CUDA(launch_combine_sum(dst, S, total, out, s));
@@ -236,10 +248,10 @@ Pass fwd_pass(const void* x, const void* y, const void* w, int64_t B, int64_t M,
 // epilogue.  They run one after the other and share the pass scratch; the
 // pass outputs o_y, o_x and the per-row dL/dtau terms sit after it.
 struct VjpLayout {
-  Pass py, px;
-  PassLayout ly, lx;
-  bool do_y, do_x, y_direct;   // y_direct: the y pass writes grad_w itself
-  size_t off_oy, off_ox, off_tau;
+  Pass py, px, pt;
+  PassLayout ly, lx, lt;
+  bool do_y, do_x, do_t, y_direct;   // y_direct: the y pass writes grad_w itself
+  size_t off_oy, off_ox, off_ot, off_tau;
   size_t total;
 };
 
@@ -248,15 +260,21 @@ VjpLayout vjp_layout(const void* x, const void* y, const void* w, const float* g
                      bool want_x, bool want_y, bool want_w, bool want_tau) {
   VjpLayout L{};
   L.do_y = want_w || want_y;
-  L.do_x = want_x || want_tau;
   L.py = fwd_pass(y, x, g, B, N, M, D, C, tau, dt);
   L.py.w_is_f32 = true;
   L.py.vmode = want_y ? 1 : 0;
   L.py.CV = value_channels(L.py.vmode, static_cast<int>(C), static_cast<int>(D));
   L.y_direct = !want_y;
+  // dL/dtau: on the CUDA-core path a pass whose kernel values carry the scaled
+  // squared distance (no cancellation); on the tensor-core path the extra
+  // value channel w |y - z|^2 of the grad_x pass
+  L.do_t = want_tau && dt == GS_F32;
+  L.do_x = want_x || (want_tau && !L.do_t);
   L.px = fwd_pass(x, y, w, B, M, N, D, C, tau, dt);
-  L.px.vmode = want_tau ? 2 : 1;
+  L.px.vmode = (want_tau && !L.do_t) ? 2 : 1;
   L.px.CV = value_channels(L.px.vmode, static_cast<int>(C), static_cast<int>(D));
+  L.pt = fwd_pass(x, y, w, B, M, N, D, C, tau, dt);
+  L.pt.shift_mode = 3;
   size_t scratch = 0;
   if (L.do_y) {
     L.ly = pass_layout(L.py, sm);
@@ -265,6 +283,10 @@ VjpLayout vjp_layout(const void* x, const void* y, const void* w, const float* g
   if (L.do_x) {
     L.lx = pass_layout(L.px, sm);
     if (L.lx.total > scratch) scratch = L.lx.total;
+  }
+  if (L.do_t) {
+    L.lt = pass_layout(L.pt, sm);
+    if (L.lt.total > scratch) scratch = L.lt.total;
   }
   size_t off = align_up(scratch);
   if (L.do_y && !L.y_direct) {
@@ -275,10 +297,71 @@ VjpLayout vjp_layout(const void* x, const void* y, const void* w, const float* g
     L.off_ox = off;
     off = align_up(off + size_t(B) * M * L.px.CV * 4);
   }
+  if (L.do_t) {
+    L.off_ot = off;
+    off = align_up(off + size_t(B) * M * C * 4);
+  }
   if (want_tau) {
     L.off_tau = off;
     off = align_up(off + size_t(B) * M * 4);
   }
+  L.total = off;
+  return L;
+}
+
+// Log-sum-exp backward (CUDA-core path), per channel c with the shift
+// -lse_c log2 e folded into the exponent: rows x / columns y with values
+// [w_c, w_c (y - z)] and a per-row shift (dL/dx), the same rows with values w_c,
+// the per-row shift and the squared-distance factor (dL/dtau), and rows y /
+// columns x with values [g_c, g_c (x - z)] and a per-column shift (dL/dw, dL/dy).
+struct LseBwdLayout {
+  Pass px, pt, py;
+  PassLayout lx, lt, ly;
+  size_t off_ox, off_ot, off_oy, off_tau, total;
+};
+
+LseBwdLayout lse_bwd_layout(const void* x, const void* y, const void* w, const float* lse,
+                            const float* g, int64_t B, int64_t M, int64_t N, int64_t D, int64_t C,
+                            float tau, int sm) {
+  LseBwdLayout L{};
+  const float kNegLog2e = -1.4426950408889634f;
+  L.px = fwd_pass(x, y, w, B, M, N, D, 1, tau, GS_F32);
+  L.px.vmode = 1;
+  L.px.CV = value_channels(1, 1, static_cast<int>(D));
+  L.px.src_ld = C;
+  L.px.shift_mode = 1;
+  L.px.shift_src = lse;
+  L.px.shift_ld = C;
+  L.px.shift_scale = kNegLog2e;
+  L.pt = fwd_pass(x, y, w, B, M, N, D, 1, tau, GS_F32);
+  L.pt.src_ld = C;
+  L.pt.shift_mode = 4;
+  L.pt.shift_src = lse;
+  L.pt.shift_ld = C;
+  L.pt.shift_scale = kNegLog2e;
+  L.py = fwd_pass(y, x, g, B, N, M, D, 1, tau, GS_F32);
+  L.py.vmode = 1;
+  L.py.CV = value_channels(1, 1, static_cast<int>(D));
+  L.py.src_ld = C;
+  L.py.shift_mode = 2;
+  L.py.shift_src = lse;
+  L.py.shift_ld = C;
+  L.py.shift_scale = kNegLog2e;
+  L.lx = pass_layout(L.px, sm);
+  L.lt = pass_layout(L.pt, sm);
+  L.ly = pass_layout(L.py, sm);
+  size_t scratch = L.lx.total;
+  if (L.lt.total > scratch) scratch = L.lt.total;
+  if (L.ly.total > scratch) scratch = L.ly.total;
+  size_t off = align_up(scratch);
+  L.off_ox = off;
+  off = align_up(off + size_t(B) * M * L.px.CV * 4);
+  L.off_ot = off;
+  off = align_up(off + size_t(B) * M * 4);
+  L.off_oy = off;
+  off = align_up(off + size_t(B) * N * L.py.CV * 4);
+  L.off_tau = off;
+  off = align_up(off + size_t(B) * M * 4);
   L.total = off;
   return L;
 }
@@ -304,7 +387,7 @@ const char* gs_status_string(gs_status st) {
 
 size_t gs_workspace_bytes(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, int64_t C,
                           gs_dtype dt) {
-  if (op != GS_OP_SUM && op != GS_OP_LSE && op != GS_OP_SUM_BWD) return kBad;
+  if (op != GS_OP_SUM && op != GS_OP_LSE && op != GS_OP_SUM_BWD && op != GS_OP_LSE_BWD) return kBad;
   if (check_dims(op, B, M, N, D, C, dt) != GS_OK) return kBad;
   if (B == 0) return 0;
   const int sm = sm_count();
@@ -316,6 +399,11 @@ size_t gs_workspace_bytes(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, 
     if (M == 0 || N == 0) return 0;
     const SdPlan sp = sd_plan(B, M, N, static_cast<int>(D), C, sm);
     return align_up(size_t(2) * sp.splits * B * M * C * 4);
+  }
+  if (op == GS_OP_LSE_BWD) {
+    if (dt != GS_F32) return kBad;
+    if (M == 0 || N == 0) return 0;
+    return lse_bwd_layout(nullptr, nullptr, nullptr, nullptr, nullptr, B, M, N, D, C, 1.f, sm).total;
   }
   if (M == 0 || N == 0) return 0;
   return vjp_layout(nullptr, nullptr, nullptr, nullptr, B, M, N, D, C, 1.f, dt, sm, true, true, true,
@@ -446,14 +534,23 @@ gs_status gauss_sum_vjp(const void* x, const void* y, const void* w, const float
                                      static_cast<int>(C), L.py.CV, tau, s));
     }
   }
+  float* tau_rows = grad_tau ? reinterpret_cast<float*>(wsb + L.off_tau) : nullptr;
   if (L.do_x) {
     float* ox = reinterpret_cast<float*>(wsb + L.off_ox);
-    float* tau_rows = grad_tau ? reinterpret_cast<float*>(wsb + L.off_tau) : nullptr;
     GS_TRY(run_pass(L.px, L.lx, ox, wsb, s));
-    GS_CUDA(launch_grad_x_epilogue(x, dt, g, ox, grad_x, tau_rows, B, M, static_cast<int>(D),
-                                   static_cast<int>(C), L.px.CV, tau, s));
-    if (grad_tau) GS_CUDA(launch_sum_rows(tau_rows, B * M, grad_tau, s));
+    GS_CUDA(launch_grad_x_epilogue(x, dt, g, ox, grad_x, L.do_t ? nullptr : tau_rows, B, M,
+                                   static_cast<int>(D), static_cast<int>(C), L.px.CV, tau, s));
   }
+  if (L.do_t) {
+    // o[i,c] = sum_j K_ij w_jc (tau/2 log2 e) |x_i - y_j|^2, so
+    // dL/dtau(i) = -1/2 sum_c g_ic o[i,c] / (tau/2 log2 e)
+    float* ot = reinterpret_cast<float*>(wsb + L.off_ot);
+    GS_TRY(run_pass(L.pt, L.lt, ot, wsb, s));
+    const double cfac = 0.5 * static_cast<double>(tau) * 1.4426950408889634074;
+    GS_CUDA(launch_weighted_rows(g, ot, tau_rows, B * M, static_cast<int>(C), 0,
+                                 static_cast<int>(C), static_cast<float>(-0.5 / cfac), false, s));
+  }
+  if (grad_tau) GS_CUDA(launch_sum_rows(tau_rows, B * M, grad_tau, s));
   return GS_OK;
 }
 
@@ -463,6 +560,69 @@ gs_status gauss_sum_bwd(const void* x, const void* y, const void* w, const float
                         gs_stream_t stream) {
   return gauss_sum_vjp(x, y, w, g, grad_x, nullptr, grad_w, nullptr, B, M, N, D, C, tau, dt, ws,
                        ws_bytes, stream);
+}
+
+gs_status gauss_lse_bwd(const void* x, const void* y, const void* w, const float* lse,
+                        const float* g, float* grad_x, float* grad_y, float* grad_w,
+                        float* grad_tau, int64_t B, int64_t M, int64_t N, int64_t D, int64_t C,
+                        float tau, gs_dtype dt, void* ws, size_t ws_bytes, gs_stream_t stream) {
+  GS_TRY(check_dims(GS_OP_LSE_BWD, B, M, N, D, C, dt));
+  GS_TRY(check_tau(tau));
+  GS_TRY(check_ptr(x, B * M * D));
+  GS_TRY(check_ptr(y, B * N * D));
+  GS_TRY(check_ptr(w, B * N * C));
+  GS_TRY(check_ptr(lse, B * M * C));
+  GS_TRY(check_ptr(g, B * M * C));
+  if (grad_x) GS_TRY(check_ptr(grad_x, B * M * D));
+  if (grad_y) GS_TRY(check_ptr(grad_y, B * N * D));
+  if (grad_w) GS_TRY(check_ptr(grad_w, B * N * C));
+  if (!grad_x && !grad_y && !grad_w && !grad_tau) return GS_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (grad_tau) GS_CUDA(cudaMemsetAsync(grad_tau, 0, sizeof(float), s));
+  if (B == 0) return GS_OK;
+  if (M == 0 || N == 0) {   // no terms: every gradient vanishes
+    if (grad_x && M > 0) GS_CUDA(cudaMemsetAsync(grad_x, 0, size_t(B) * M * D * 4, s));
+    if (grad_y && N > 0) GS_CUDA(cudaMemsetAsync(grad_y, 0, size_t(B) * N * D * 4, s));
+    if (grad_w && N > 0) GS_CUDA(cudaMemsetAsync(grad_w, 0, size_t(B) * N * C * 4, s));
+    return GS_OK;
+  }
+  LseBwdLayout L = lse_bwd_layout(x, y, w, lse, g, B, M, N, D, C, tau, sm_count());
+  if (ws_bytes < L.total) return GS_ERR_WORKSPACE;
+  GS_TRY(check_ptr(ws, 1));
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  float* ox = reinterpret_cast<float*>(wsb + L.off_ox);
+  float* ot = reinterpret_cast<float*>(wsb + L.off_ot);
+  float* oy = reinterpret_cast<float*>(wsb + L.off_oy);
+  float* tau_rows = reinterpret_cast<float*>(wsb + L.off_tau);
+  const float* wf = static_cast<const float*>(w);
+  const double cfac = 0.5 * static_cast<double>(tau) * 1.4426950408889634074;
+  for (int c = 0; c < static_cast<int>(C); ++c) {
+    const bool acc = c > 0;
+    if (grad_x || grad_tau) {
+      L.px.w = wf + c;
+      L.px.shift_c = c;
+      GS_TRY(run_pass(L.px, L.lx, ox, wsb, s));
+      if (grad_tau) {
+        L.pt.w = wf + c;
+        L.pt.shift_c = c;
+        GS_TRY(run_pass(L.pt, L.lt, ot, wsb, s));
+      }
+      GS_CUDA(launch_lse_x_tau_epilogue(static_cast<const float*>(x), g, ox, grad_tau ? ot : nullptr,
+                                        grad_x, grad_tau ? tau_rows : nullptr, B, M,
+                                        static_cast<int>(D), static_cast<int>(C), c, tau,
+                                        static_cast<float>(1.0 / cfac), acc, s));
+    }
+    if (grad_y || grad_w) {
+      L.py.w = g + c;
+      L.py.shift_c = c;
+      GS_TRY(run_pass(L.py, L.ly, oy, wsb, s));
+      GS_CUDA(launch_lse_grad_y_epilogue(static_cast<const float*>(y), wf, oy, grad_y, grad_w, B,
+                                         N, static_cast<int>(D), static_cast<int>(C), c, tau, acc,
+                                         s));
+    }
+  }
+  if (grad_tau) GS_CUDA(launch_sum_rows(tau_rows, B * M, grad_tau, s));
+  return GS_OK;
 }
 
 gs_status gs_last_device_error(gs_stream_t stream) {

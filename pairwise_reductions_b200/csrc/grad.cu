@@ -44,10 +44,10 @@ int grid_for(int64_t n, int threads) {
 
 // Value matrix, float32 [B, N, CV] (CUDA-core path) -------------------------------
 template <typename TS, typename TP>
-__global__ void pack_values_f32_kernel(const TS* __restrict__ src, const TP* __restrict__ cols,
-                                       const TP* __restrict__ rows, float* __restrict__ v,
-                                       int64_t B, int64_t N, int64_t Mrows, int D, int C,
-                                       int mode) {
+__global__ void pack_values_f32_kernel(const TS* __restrict__ src, int64_t src_ld,
+                                       const TP* __restrict__ cols, const TP* __restrict__ rows,
+                                       float* __restrict__ v, int64_t B, int64_t N, int64_t Mrows,
+                                       int D, int C, int mode) {
   const int CV = value_channels(mode, C, D);
   const int64_t total = B * N * CV;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
@@ -55,7 +55,7 @@ __global__ void pack_values_f32_kernel(const TS* __restrict__ src, const TP* __r
     const int64_t bj = e / CV;
     const int ch = static_cast<int>(e % CV);
     const int64_t b = bj / N;
-    v[e] = value_at(src, cols, rows, b, bj, Mrows, D, C, ch);
+    v[e] = value_at(src, cols, rows, b, bj, Mrows, D, C, ch, src_ld);
   }
 }
 
@@ -122,6 +122,18 @@ __global__ void grad_y_epilogue_kernel(const T* __restrict__ y, const T* __restr
   }
 }
 
+// out[r] (+)= factor * sum_{c in [c0, c0 + nc)} g[r, c] * o[r, c - c0]  (o rows nc wide)
+__global__ void weighted_rows_kernel(const float* __restrict__ g, const float* __restrict__ o,
+                                     float* __restrict__ out, int64_t rows, int C, int c0, int nc,
+                                     float factor, int accumulate) {
+  for (int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; r < rows;
+       r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float s = 0.f;
+    for (int c = 0; c < nc; ++c) s = fmaf(g[r * C + c0 + c], o[r * nc + c], s);
+    out[r] = accumulate ? out[r] + factor * s : factor * s;
+  }
+}
+
 // Fixed-order reduction of the per-row dL/dtau terms: one block, each thread
 // sums a strided slice in order, then a fixed tree in shared memory.
 __global__ void sum_rows_kernel(const float* __restrict__ v, int64_t n, float* __restrict__ out) {
@@ -137,6 +149,67 @@ __global__ void sum_rows_kernel(const float* __restrict__ v, int64_t n, float* _
   if (threadIdx.x == 0) *out = static_cast<float>(part[0]);
 }
 
+// Log-sum-exp backward, channel c: o_x row = [A, B_k (D)] with A = sum_j p_ij and
+// B = sum_j p_ij (y_j - z), and o_t row = T = sum_j p_ij |x^_i - y^_j|^2 (scaled
+// squared distances).  A is 1 up to the rounding of lse, a factor common to
+// every p_ij of the row, so dividing by A cancels it:
+//   dL/dx_ik   += -tau g_ic ((x_ik - z_k) - B_k / A)
+//   dL/dtau(i) += -1/2 g_ic (T / A) / (tau/2 log2 e)
+__global__ void lse_x_tau_epilogue_kernel(const float* __restrict__ x, const float* __restrict__ g,
+                                          const float* __restrict__ o, const float* __restrict__ ot,
+                                          float* __restrict__ gx, float* __restrict__ tau_rows,
+                                          int64_t B, int64_t M, int D, int C, int c, float tau,
+                                          float inv_cfac, int accumulate) {
+  const int64_t rows = B * M;
+  const int CV = 1 + D;
+  for (int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; r < rows;
+       r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = r / M;
+    const float* xi = x + r * D;
+    const float* z = x + b * M * D;
+    const float* oi = o + r * CV;
+    const float gic = g[r * C + c];
+    const float inv_a = 1.f / oi[0];
+    if (gx) {
+      for (int k = 0; k < D; ++k) {
+        const float v = -tau * gic * ((xi[k] - z[k]) - oi[1 + k] * inv_a);
+        gx[r * D + k] = accumulate ? gx[r * D + k] + v : v;
+      }
+    }
+    if (tau_rows) {
+      const float v = -0.5f * gic * ot[r] * inv_a * inv_cfac;
+      tau_rows[r] = accumulate ? tau_rows[r] + v : v;
+    }
+  }
+}
+
+// Log-sum-exp backward, channel c: o_y row = [A', B'_k (D)] with
+// A' = sum_i g_ic K_ij e^-lse_ic, B' = sum_i g_ic K_ij e^-lse_ic (x_i - z).
+//   dL/dw_jc   = A'
+//   dL/dy_jk  += -tau w_jc ((y_jk - z_k) A' - B'_k)
+__global__ void lse_grad_y_epilogue_kernel(const float* __restrict__ y, const float* __restrict__ w,
+                                           const float* __restrict__ o, float* __restrict__ gy,
+                                           float* __restrict__ gw, int64_t B, int64_t N, int D,
+                                           int C, int c, float tau, int accumulate) {
+  const int64_t rows = B * N;
+  const int CV = 1 + D;
+  for (int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; r < rows;
+       r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = r / N;
+    const float* yj = y + r * D;
+    const float* z = y + b * N * D;
+    const float* oj = o + r * CV;
+    if (gw) gw[r * C + c] = oj[0];
+    if (gy) {
+      const float wjc = w[r * C + c];
+      for (int k = 0; k < D; ++k) {
+        const float v = -tau * wjc * fmaf(yj[k] - z[k], oj[0], -oj[1 + k]);
+        gy[r * D + k] = accumulate ? gy[r * D + k] + v : v;
+      }
+    }
+  }
+}
+
 template <typename T>
 const T* as(const void* p) {
   return static_cast<const T*>(p);
@@ -144,16 +217,13 @@ const T* as(const void* p) {
 
 }  // namespace
 
-cudaError_t launch_pack_values_f32(const void* src, bool src_is_f32, const void* cols,
-                                   const void* rows, gs_dtype pt, float* v, int64_t B, int64_t N,
-                                   int64_t Mrows, int D, int C, int mode, cudaStream_t s) {
+cudaError_t launch_pack_values_f32(const void* src, int64_t src_ld, const void* cols,
+                                   const void* rows, float* v, int64_t B, int64_t N, int64_t Mrows,
+                                   int D, int C, int mode, cudaStream_t s) {
   const int64_t n = B * N * value_channels(mode, C, D);
   const int blocks = grid_for(n, 256);
-  // the CUDA-core path only runs float32 points and values
-  (void)src_is_f32;
-  (void)pt;
   pack_values_f32_kernel<float, float><<<blocks, 256, 0, s>>>(
-      as<float>(src), as<float>(cols), as<float>(rows), v, B, N, Mrows, D, C, mode);
+      as<float>(src), src_ld, as<float>(cols), as<float>(rows), v, B, N, Mrows, D, C, mode);
   return cudaGetLastError();
 }
 
@@ -196,6 +266,31 @@ cudaError_t launch_grad_y_epilogue(const void* y, const void* w, gs_dtype dt, co
           as<__nv_bfloat16>(y), as<__nv_bfloat16>(w), o, grad_y, grad_w, B, N, D, C, CV, tau);
       break;
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lse_x_tau_epilogue(const float* x, const float* g, const float* o,
+                                      const float* ot, float* grad_x, float* tau_rows, int64_t B,
+                                      int64_t M, int D, int C, int c, float tau, float inv_cfac,
+                                      bool accumulate, cudaStream_t s) {
+  lse_x_tau_epilogue_kernel<<<grid_for(B * M, 256), 256, 0, s>>>(
+      x, g, o, ot, grad_x, tau_rows, B, M, D, C, c, tau, inv_cfac, accumulate ? 1 : 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lse_grad_y_epilogue(const float* y, const float* w, const float* o,
+                                       float* grad_y, float* grad_w, int64_t B, int64_t N, int D,
+                                       int C, int c, float tau, bool accumulate, cudaStream_t s) {
+  lse_grad_y_epilogue_kernel<<<grid_for(B * N, 256), 256, 0, s>>>(y, w, o, grad_y, grad_w, B, N, D,
+                                                                  C, c, tau, accumulate ? 1 : 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_weighted_rows(const float* g, const float* o, float* tau_rows, int64_t rows,
+                                 int C, int c0, int nc, float factor, bool accumulate,
+                                 cudaStream_t s) {
+  weighted_rows_kernel<<<grid_for(rows, 256), 256, 0, s>>>(g, o, tau_rows, rows, C, c0, nc, factor,
+                                                           accumulate ? 1 : 0);
   return cudaGetLastError();
 }
 

@@ -51,6 +51,14 @@ struct SdArgs {
   int D;
   float scale;         // sqrt(tau / 2 * log2 e)
   SdPlan plan;
+  // optional exponent shift (log2 units), sum kernel only: every kernel value
+  // becomes K_ij * 2^shift with shift = shift_scale * shift_src[(b * n + p) * shift_ld + shift_c],
+  // p the row i (shift_mode 1, n = M) or the column j (shift_mode 2, n = N)
+  int shift_mode;      // 0 none, 1 per row, 2 per column, 3 kernel x scaled |x - y|^2, 4 = 1 and 3
+  const float* shift_src;
+  int64_t shift_ld;
+  int shift_c;
+  float shift_scale;
 };
 
 cudaError_t launch_small_d_sum(const SdArgs& a, cudaStream_t s);
@@ -77,10 +85,24 @@ struct LseFinalizeArgs {
 };
 cudaError_t launch_lse_finalize(const LseFinalizeArgs& a, cudaStream_t s);
 
-// Value matrix of a pass on the CUDA-core path, float32 [B, N, CV] (values.cuh).
-cudaError_t launch_pack_values_f32(const void* src, bool src_is_f32, const void* cols,
-                                   const void* rows, gs_dtype pt, float* v, int64_t B, int64_t N,
-                                   int64_t Mrows, int D, int C, int mode, cudaStream_t s);
+// Value matrix of a pass on the CUDA-core path, float32 [B, N, CV] (values.cuh);
+// src rows are src_ld floats apart (src_ld >= C; a channel slice of a wider array).
+cudaError_t launch_pack_values_f32(const void* src, int64_t src_ld, const void* cols,
+                                   const void* rows, float* v, int64_t B, int64_t N, int64_t Mrows,
+                                   int D, int C, int mode, cudaStream_t s);
+
+// Log-sum-exp backward epilogues for channel c of C (grad.cu): o_x [B, M, 1 + D]
+// holds [sum_j p, sum_j p (y - z)] and o_y [B, N, 1 + D] holds
+// [sum_i g p / w, sum_i g p (x - z) / w]; with `accumulate` the results add to
+// the outputs of the previous channels.
+// ot [B, M] holds sum_j p |x^ - y^|^2 (NULL when tau_rows is NULL)
+cudaError_t launch_lse_x_tau_epilogue(const float* x, const float* g, const float* o,
+                                      const float* ot, float* grad_x, float* tau_rows, int64_t B,
+                                      int64_t M, int D, int C, int c, float tau, float inv_cfac,
+                                      bool accumulate, cudaStream_t s);
+cudaError_t launch_lse_grad_y_epilogue(const float* y, const float* w, const float* o,
+                                       float* grad_y, float* grad_w, int64_t B, int64_t N, int D,
+                                       int C, int c, float tau, bool accumulate, cudaStream_t s);
 
 // Gradient epilogues (grad.cu).  grad_x and tau_rows may each be NULL; so may
 // grad_y and grad_w.
@@ -90,6 +112,10 @@ cudaError_t launch_grad_x_epilogue(const void* x, gs_dtype dt, const float* g, c
 cudaError_t launch_grad_y_epilogue(const void* y, const void* w, gs_dtype dt, const float* o,
                                    float* grad_y, float* grad_w, int64_t B, int64_t N, int D,
                                    int C, int CV, float tau, cudaStream_t s);
+// tau_rows[r] (+)= factor * sum_{c in [c0, c0 + nc)} g[r, c] * o[r, c - c0]
+cudaError_t launch_weighted_rows(const float* g, const float* o, float* tau_rows, int64_t rows,
+                                 int C, int c0, int nc, float factor, bool accumulate,
+                                 cudaStream_t s);
 // out[0] = sum of v[0 .. n) in a fixed order (double accumulation).
 cudaError_t launch_sum_rows(const float* v, int64_t n, float* out, cudaStream_t s);
 

@@ -41,11 +41,13 @@ constexpr int kTileJ = 256;
 constexpr int kPer = kTileJ / kSdThreads;   // points each thread stages per tile
 constexpr float kLn2 = 0.69314718055994530942f;
 
-template <int D, int CP>
+template <int D, int CP, int SHIFT = 0>
 struct PackShape {
-  // floats per staged point: D duplicated negated coordinates and CP duplicated
-  // values, so every operand of the packed (two-row) arithmetic is one 64-bit load
-  static constexpr int PK = ((2 * (D + CP) + 3) / 4) * 4;
+  // floats per staged point: D duplicated negated coordinates, CP duplicated
+  // values (and, for a per-column exponent shift, the duplicated shift), so
+  // every operand of the packed (two-row) arithmetic is one 64-bit load
+  static constexpr int NPAIR = D + CP + (SHIFT == 2 ? 1 : 0);
+  static constexpr int PK = ((2 * NPAIR + 3) / 4) * 4;
 };
 
 // Row pairs per thread that take the FMA-pipe exp2 instead of MUFU ex2.  None:
@@ -63,13 +65,20 @@ __device__ __forceinline__ float pow2i(float e) {
   return __int_as_float((static_cast<int>(e) + 127) << 23);
 }
 
-template <int D, int CP, bool LSE>
+// SHIFT: 0 none; 1 per-row and 2 per-column exponent shift (SdArgs), so that
+// each kernel value is K_ij * 2^shift -- used by the log-sum-exp backward to
+// sum the normalised weights w K e^-lse directly; 3 multiplies each kernel
+// value by the scaled squared distance |x^ - y^|^2 = (tau/2 log2 e) |x - y|^2,
+// which gives the bandwidth gradient sum_j K w |x - y|^2 without cancellation;
+// 4 does both the per-row shift and the squared-distance factor.
+template <int D, int CP, bool LSE, int SHIFT>
 __global__ void __launch_bounds__(kSdThreads)
     sd_kernel(const SdArgs a) {
   constexpr int R = sd_rows_per_thread(D, CP);
   constexpr int RP = R / 2;                     // row pairs per thread
   constexpr int NPOLY = poly_pairs<D, CP, R>();
-  constexpr int PK = PackShape<D, CP>::PK;
+  constexpr int PK = PackShape<D, CP, SHIFT>::PK;
+  static_assert(!(LSE && SHIFT), "shifts apply to the sum kernel");
   constexpr int NW = kSdThreads / 32;
   static_assert(R % 2 == 0, "rows are processed in pairs");
   __shared__ __align__(16) float tile[kTileJ * PK];
@@ -98,6 +107,19 @@ __global__ void __launch_bounds__(kSdThreads)
       xs[q][k] = pk2(v0, v1);
     }
   }
+  uint64_t rho[RP];   // SHIFT == 1: per-row exponent shift of my row pairs
+#pragma unroll
+  for (int q = 0; q < RP; ++q) {
+    if constexpr (SHIFT == 1 || SHIFT == 4) {
+      const int64_t i0 = row0 + tid + (2 * q) * kSdThreads;
+      const int64_t i1 = i0 + kSdThreads;
+      const float s0 = (i0 < a.M) ? a.shift_scale * a.shift_src[(b * a.M + i0) * a.shift_ld + a.shift_c] : 0.f;
+      const float s1 = (i1 < a.M) ? a.shift_scale * a.shift_src[(b * a.M + i1) * a.shift_ld + a.shift_c] : 0.f;
+      rho[q] = pk2(s0, s1);
+    } else {
+      rho[q] = 0ull;
+    }
+  }
   uint64_t acc[RP][CP];
   float mrun[CP];   // LSE: integer log2 shift of the weights (-inf before any positive weight)
 #pragma unroll
@@ -109,11 +131,15 @@ __global__ void __launch_bounds__(kSdThreads)
 
   for (int64_t j0 = jbeg; j0 < jend; j0 += kTileJ) {
     // ---- stage one tile: negated scaled y and the (shifted) weights
-    float sy[kPer][D], sv[kPer][CP];
+    float sy[kPer][D], sv[kPer][CP], sk[kPer];
 #pragma unroll
     for (int q = 0; q < kPer; ++q) {
       const int64_t j = j0 + tid + q * kSdThreads;
       const bool ok = j < jend;
+      if constexpr (SHIFT == 2)
+        sk[q] = ok ? a.shift_scale * a.shift_src[(b * a.N + j) * a.shift_ld + a.shift_c] : 0.f;
+      else
+        sk[q] = 0.f;
 #pragma unroll
       for (int k = 0; k < D; ++k) sy[q][k] = ok ? -(yb[j * D + k] * a.scale) : 0.f;
 #pragma unroll
@@ -167,8 +193,12 @@ __global__ void __launch_bounds__(kSdThreads)
         p[2 * (D + c)] = sv[q][c];
         p[2 * (D + c) + 1] = sv[q][c];
       }
+      if constexpr (SHIFT == 2) {
+        p[2 * (D + CP)] = sk[q];
+        p[2 * (D + CP) + 1] = sk[q];
+      }
 #pragma unroll
-      for (int k = 2 * (D + CP); k < PK; ++k) p[k] = 0.f;
+      for (int k = 2 * PackShape<D, CP, SHIFT>::NPAIR; k < PK; ++k) p[k] = 0.f;
     }
     __syncthreads();
 
@@ -199,13 +229,28 @@ __global__ void __launch_bounds__(kSdThreads)
           e = add2(xs[q][k], pk[k]);
           d = fma2(e, e, d);
         }
-        float d0, d1;
-        upk2(d, d0, d1);
         uint64_t kv;
-        if (q >= RP - NPOLY) {
-          kv = exp2_poly2<5, true>(pk2(fminf(d0, 125.f), fminf(d1, 125.f)));
+        if constexpr (SHIFT == 3) {
+          float d0, d1;
+          upk2(d, d0, d1);
+          kv = mul2(pk2(ex2(-d0), ex2(-d1)), d);
+        } else if constexpr (SHIFT == 4) {
+          float t0, t1;
+          upk2(sub2(rho[q], d), t0, t1);
+          kv = mul2(pk2(ex2(t0), ex2(t1)), d);
+        } else if constexpr (SHIFT != 0) {
+          // exponent = shift - d (per row, or per column from the staged pair)
+          float t0, t1;
+          upk2(sub2(SHIFT == 1 ? rho[q] : pk[D + CP], d), t0, t1);
+          kv = pk2(ex2(t0), ex2(t1));
         } else {
-          kv = pk2(ex2(-d0), ex2(-d1));
+          float d0, d1;
+          upk2(d, d0, d1);
+          if (q >= RP - NPOLY) {
+            kv = exp2_poly2<5, true>(pk2(fminf(d0, 125.f), fminf(d1, 125.f)));
+          } else {
+            kv = pk2(ex2(-d0), ex2(-d1));
+          }
         }
 #pragma unroll
         for (int c = 0; c < CP; ++c) tacc[q][c] = fma2(kv, pk[D + c], tacc[q][c]);
@@ -249,7 +294,17 @@ cudaError_t launch_t(const SdArgs& a, cudaStream_t s) {
   const int64_t tiles = (a.M + kSdThreads * R - 1) / (kSdThreads * R);
   dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(a.plan.splits),
             static_cast<unsigned>(a.B));
-  sd_kernel<D, CP, LSE><<<grid, kSdThreads, 0, s>>>(a);
+  if constexpr (LSE) {
+    sd_kernel<D, CP, true, 0><<<grid, kSdThreads, 0, s>>>(a);
+  } else {
+    switch (a.shift_mode) {
+      case 1: sd_kernel<D, CP, false, 1><<<grid, kSdThreads, 0, s>>>(a); break;
+      case 2: sd_kernel<D, CP, false, 2><<<grid, kSdThreads, 0, s>>>(a); break;
+      case 3: sd_kernel<D, CP, false, 3><<<grid, kSdThreads, 0, s>>>(a); break;
+      case 4: sd_kernel<D, CP, false, 4><<<grid, kSdThreads, 0, s>>>(a); break;
+      default: sd_kernel<D, CP, false, 0><<<grid, kSdThreads, 0, s>>>(a); break;
+    }
+  }
   return cudaGetLastError();
 }
 

@@ -514,7 +514,7 @@ __global__ void pack_values_kernel(const TW* __restrict__ w, const TY* __restric
     const int cc = static_cast<int>(bc % CP);
     const int64_t b = bc / CP;
     const int ch = c0 + cc;
-    const float v = (ch < CV) ? value_at(w, y, rows, b, b * N + j, Mrows, D, C, ch) : 0.f;
+    const float v = (ch < CV) ? value_at(w, y, rows, b, b * N + j, Mrows, D, C, ch, C) : 0.f;
     vt[(b * CP + cc) * Nst + j] = __float2half_rn(v);
   }
 }

@@ -25,17 +25,17 @@ __device__ __forceinline__ float vf(float v) { return v; }
 __device__ __forceinline__ float vf(__half v) { return __half2float(v); }
 __device__ __forceinline__ float vf(__nv_bfloat16 v) { return __bfloat162float(v); }
 
-// Channel ch of the values of column bj = b * Ncols + j.
+// Channel ch of the values of column bj = b * Ncols + j; src rows are src_ld apart.
 template <typename TS, typename TP>
 __device__ __forceinline__ float value_at(const TS* __restrict__ src, const TP* __restrict__ cols,
                                           const TP* __restrict__ rows, int64_t b, int64_t bj,
-                                          int64_t Mrows, int D, int C, int ch) {
-  if (ch < C) return vf(src[bj * C + ch]);
+                                          int64_t Mrows, int D, int C, int ch, int64_t src_ld) {
+  if (ch < C) return vf(src[bj * src_ld + ch]);
   const TP* z = rows + b * Mrows * D;
   const TP* col = cols + bj * D;
   if (ch < C * (1 + D)) {
     const int c = (ch - C) / D, k = (ch - C) % D;
-    return vf(src[bj * C + c]) * (vf(col[k]) - vf(z[k]));
+    return vf(src[bj * src_ld + c]) * (vf(col[k]) - vf(z[k]));
   }
   const int c = ch - C * (1 + D);
   float q = 0.f;
@@ -43,7 +43,7 @@ __device__ __forceinline__ float value_at(const TS* __restrict__ src, const TP* 
     const float d = vf(col[k]) - vf(z[k]);
     q = fmaf(d, d, q);
   }
-  return vf(src[bj * C + c]) * q;
+  return vf(src[bj * src_ld + c]) * q;
 }
 
 }  // namespace gs

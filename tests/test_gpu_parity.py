@@ -299,3 +299,39 @@ def test_vjp_d32_c1_full_size_sampled():
     assert rel_l2(got["x"].cpu().numpy()[:, rows], rgx) <= TOL["f16"]
     assert rel_l2(got["w"].cpu().numpy()[:, yrows], rgw) <= TOL["f16"]
     assert rel_l2(got["y"].cpu().numpy()[:, yrows], rgy) <= TOL["f16"]
+
+
+# ------------------------------------------------------------------ log-sum-exp backward
+@pytest.mark.parametrize("shape,shift", [((1, 300, 500, 3, 1), 0.0), ((2, 200, 300, 2, 3), 0.0),
+                                         ((1, 150, 400, 8, 2), 0.0), ((1, 256, 700, 3, 1), 30.0)])
+def test_lse_bwd_every_gradient(shape, shift):
+    B, M, N, D, C = shape
+    inp = synth.make_inputs(3, seed=17, B=B, M=M, N=N, D=D, C=C, with_g=True, tau=20.0)
+    if shift:
+        for k in ("x", "y"):
+            inp[k] = inp[k] + shift
+    d = dev(inp)
+    lse = gs().gauss_lse_fwd(d["x"], d["y"], d["w"], inp["tau"])
+    got = gs().gauss_lse_bwd(d["x"], d["y"], d["w"], lse, d["g"], inp["tau"])
+    rgx, rgy, rgw, rgt = oracle.gauss_lse_bwd(*(f64(inp, k) for k in "xywg"), inp["tau"])
+    for name, ref in (("x", rgx), ("y", rgy), ("w", rgw)):
+        e = rel_l2(got[name].cpu().numpy(), ref)
+        assert e <= TOL["f32"], (name, e)
+    et = abs(float(got["tau"].item()) - rgt) / max(abs(rgt), 1e-30)
+    assert et <= TOL["f32"], ("tau", et, float(got["tau"].item()), rgt)
+
+
+def test_lse_bwd_rows_far_from_every_point():
+    """Rows whose kernel values all underflow fp32: the -lse shift in the
+    exponent keeps the normalised weights exact."""
+    inp = synth.make_inputs(3, seed=18, M=120, N=400, with_g=True)
+    x = inp["x"].clone()
+    x[0, :20] += 3.0
+    inp["x"] = x
+    d = dev(inp)
+    lse = gs().gauss_lse_fwd(d["x"], d["y"], d["w"], inp["tau"])
+    got = gs().gauss_lse_bwd(d["x"], d["y"], d["w"], lse, d["g"], inp["tau"], want=("x", "w"))
+    rgx, _, rgw, _ = oracle.gauss_lse_bwd(*(f64(inp, k) for k in "xywg"), inp["tau"])
+    assert np.isfinite(got["x"].cpu().numpy()).all()
+    assert rel_l2(got["x"].cpu().numpy(), rgx) <= TOL["f32"]
+    assert rel_l2(got["w"].cpu().numpy(), rgw) <= TOL["f32"]
