@@ -14,6 +14,7 @@ step 2):
 * ``gauss_sum_bwd(x, y, w, g, tau, rows=None, wrows=None)`` -> (grad_x, grad_w)
 * ``gauss_sum_vjp_y_tau(x, y, w, g, tau, yrows=None)`` -> (grad_y, grad_tau)
 * ``gauss_lse_bwd(x, y, w, g, tau)`` -> (grad_x, grad_y, grad_w, grad_tau)
+* ``knn(x, y, K, rows=None, f32=False)`` -> (sq_dist [B, R, K], index [B, R, K])
 
 Inputs are float64 arrays x [B,M,D], y [B,N,D], w [B,N,C], g [B,M,C] (2-D
 arrays are read as B = 1).  Values must already be the quantised values the
@@ -57,6 +58,13 @@ def _load(path=None):
     f.restype = ctypes.c_int
     f.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _i64, _i64, _i64, _i64, _i64,
                   ctypes.c_double]
+    _fp = ctypes.POINTER(ctypes.c_float)
+    f = lib.oracle_knn
+    f.restype = ctypes.c_int
+    f.argtypes = [_dp, _dp, _dp, _ip, _i64, _i64, _i64, _i64, _i64, _ip, _i64]
+    f = lib.oracle_knn_f32
+    f.restype = ctypes.c_int
+    f.argtypes = [_fp, _fp, _fp, _ip, _i64, _i64, _i64, _i64, _i64, _ip, _i64]
     lib.oracle_num_threads.restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -170,4 +178,34 @@ def gauss_lse_bwd(x, y, w, g, tau, lib=None):
     return gx, gy, gw, float(gt[0])
 
 
-__all__ = ["gauss_sum_vjp_y_tau", "gauss_lse_bwd", "gauss_sum", "gauss_lse", "gauss_sum_bwd", "num_threads", "build_oracle", "LIB"]
+def knn(x, y, K, rows=None, lib=None, f32=False):
+    """K smallest squared distances |x_i - y_j|^2 per row (ascending, ties by lower j)
+    and their indices; f32=True decides in float (fixed order of operations)."""
+    if f32:
+        x = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+        y = np.ascontiguousarray(np.asarray(y, dtype=np.float32))
+        if x.ndim == 2:
+            x, y = x[None], y[None]
+    else:
+        x, y = _as3(x, "x"), _as3(y, "y")
+    B, M, D = x.shape
+    N = y.shape[1]
+    if y.shape[0] != B or y.shape[2] != D:
+        raise ValueError(f"shape mismatch x{x.shape} y{y.shape}")
+    r, nr, rp = _rows(rows)
+    R = nr if r is not None else M
+    od = np.empty((B, R, K), dtype=np.float32 if f32 else np.float64)
+    oi = np.empty((B, R, K), dtype=np.int64)
+    L = lib or _load()
+    if f32:
+        fp = ctypes.POINTER(ctypes.c_float)
+        rc = L.oracle_knn_f32(x.ctypes.data_as(fp), y.ctypes.data_as(fp), od.ctypes.data_as(fp),
+                              oi.ctypes.data_as(_ip), B, M, N, D, int(K), rp, nr)
+    else:
+        rc = L.oracle_knn(_ptr(x), _ptr(y), _ptr(od), oi.ctypes.data_as(_ip), B, M, N, D, int(K), rp, nr)
+    if rc != 0:
+        raise ValueError(f"oracle knn rejected its arguments (code {rc})")
+    return od, oi
+
+
+__all__ = ["knn", "gauss_sum_vjp_y_tau", "gauss_lse_bwd", "gauss_sum", "gauss_lse", "gauss_sum_bwd", "num_threads", "build_oracle", "LIB"]

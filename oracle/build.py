@@ -19,8 +19,8 @@ def build_oracle(out=LIB, extra_flags=(), force=False):
             and os.path.getmtime(out) >= os.path.getmtime(SRC)
             and not extra_flags):
         return out
-    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
-           "-fno-fast-math", "-ffp-contract=off", *extra_flags, SRC, "-o", out, "-lm"]
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-fno-fast-math",
+           "-ffp-contract=off", "-fexcess-precision=standard", *extra_flags, SRC, "-o", out, "-lm"]
     subprocess.run(cmd, check=True)
     return out
 

@@ -429,3 +429,102 @@ int oracle_gauss_lse_bwd(const double *x, const double *y, const double *w, cons
         *grad_tau = tau_acc;
     return 0;
 }
+
+/* K-nearest reduction ("Kernel matrix reduction", Overview: the reductions
+ * covered include minima and the indices of the K smallest entries per row;
+ * the .argmin() reduction of the LazyTensor API).  For each row i the K
+ * smallest squared distances |x_i - y_j|^2 over j, ascending, with their
+ * indices j; equal distances are ordered by the lower j.  Rows with fewer than
+ * K columns get +inf and index -1 in the missing places.  The maximum of the
+ * Gaussian kernel over j is exp(-tau/2 * out_d[...,0]), at out_idx[...,0].
+ *
+ * Two precisions.  oracle_knn computes the distances in double (the plain
+ * definition).  oracle_knn_f32 takes float inputs and computes every distance
+ * in float with one fixed order of operations -- e_k = x_k - y_k, then
+ * d = e_0 * e_0, then d = fma(e_k, e_k, d) for k = 1 .. D-1, each rounded to
+ * nearest -- so that an integer result decided by floating point (which index
+ * is nearer) is decided in float, the precision of the device kernel.
+ * Selection is a plain insertion into a sorted list of K. */
+static void knn_insert(double d, int64_t j, double *bd, int64_t *bj, int64_t K)
+{
+    if (!(d < bd[K - 1] || (d == bd[K - 1] && j < bj[K - 1])))
+        return;
+    int64_t p = K - 1;
+    while (p > 0 && (d < bd[p - 1] || (d == bd[p - 1] && j < bj[p - 1]))) {
+        bd[p] = bd[p - 1];
+        bj[p] = bj[p - 1];
+        --p;
+    }
+    bd[p] = d;
+    bj[p] = j;
+}
+
+int oracle_knn(const double *x, const double *y, double *out_d, int64_t *out_idx, int64_t B,
+               int64_t M, int64_t N, int64_t D, int64_t K, const int64_t *rows, int64_t n_rows)
+{
+    int64_t R = rows ? n_rows : M;
+    if (B < 0 || M < 0 || N < 0 || D < 1 || K < 1 || R < 0)
+        return 1;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t t = 0; t < B * R; ++t) {
+        int64_t bb = t / R;
+        int64_t r = t % R;
+        int64_t i = rows ? rows[r] : r;
+        const double *xi = x + (bb * M + i) * D;
+        double *bd = out_d + (bb * R + r) * K;
+        int64_t *bj = out_idx + (bb * R + r) * K;
+        for (int64_t k = 0; k < K; ++k) {
+            bd[k] = INFINITY;
+            bj[k] = -1;
+        }
+        for (int64_t j = 0; j < N; ++j)
+            knn_insert(sq_dist(xi, y + (bb * N + j) * D, D), j, bd, bj, K);
+    }
+    return 0;
+}
+
+int oracle_knn_f32(const float *x, const float *y, float *out_d, int64_t *out_idx, int64_t B,
+                   int64_t M, int64_t N, int64_t D, int64_t K, const int64_t *rows,
+                   int64_t n_rows)
+{
+    int64_t R = rows ? n_rows : M;
+    if (B < 0 || M < 0 || N < 0 || D < 1 || K < 1 || R < 0)
+        return 1;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *bd = (double *)malloc((size_t)K * sizeof(double));
+        if (!bd) {
+#pragma omp atomic write
+            bad = 1;
+        }
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t t = 0; t < B * R; ++t) {
+            if (!bd)
+                continue;
+            int64_t bb = t / R;
+            int64_t r = t % R;
+            int64_t i = rows ? rows[r] : r;
+            const float *xi = x + (bb * M + i) * D;
+            int64_t *bj = out_idx + (bb * R + r) * K;
+            for (int64_t k = 0; k < K; ++k) {
+                bd[k] = INFINITY;
+                bj[k] = -1;
+            }
+            for (int64_t j = 0; j < N; ++j) {
+                const float *yj = y + (bb * N + j) * D;
+                float e = xi[0] - yj[0];
+                float d = e * e;
+                for (int64_t k = 1; k < D; ++k) {
+                    e = xi[k] - yj[k];
+                    d = fmaf(e, e, d);
+                }
+                knn_insert((double)d, j, bd, bj, K);
+            }
+            for (int64_t k = 0; k < K; ++k)
+                out_d[(bb * R + r) * K + k] = (float)bd[k];
+        }
+        free(bd);
+    }
+    return bad ? 2 : 0;
+}

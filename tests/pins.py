@@ -388,10 +388,65 @@ def pin_gradient_symmetries(O):
     assert abs(lhs - 2 * tau * lt) <= 1e-11 * max(1.0, abs(lhs)), f"lse: scaling {lhs} vs {2 * tau * lt}"
 
 
+# --------------------------------------------------------------------------- k-nearest reduction
+def pin_knn_against_library_sort(O):
+    """torch.cdist (float64) then a stable sort: ascending distances, equal
+    distances in index order."""
+    r = _rng(20)
+    for (B, M, N, D, K) in [(1, 9, 40, 3, 5), (2, 7, 13, 2, 13), (1, 5, 30, 8, 1)]:
+        x, y = r.normal(size=(B, M, D)), r.normal(size=(B, N, D))
+        d, i = O.knn(x, y, K)
+        dd = torch.cdist(torch.from_numpy(x), torch.from_numpy(y),
+                         compute_mode="donot_use_mm_for_euclid_dist") ** 2
+        sd, si = torch.sort(dd, dim=-1, stable=True)
+        _close(d, sd[..., :K].numpy(), 1e-12, 1e-14, f"knn dist B{B}M{M}N{N}K{K}")
+        assert np.array_equal(i, si[..., :K].numpy()), "knn indices"
+
+
+def pin_knn_ties_padding_and_grid(O):
+    """Duplicated sources come out lowest index first; rows with fewer than K
+    sources are padded with +inf / -1; on an integer lattice the distances and
+    neighbours are known exactly."""
+    y = np.array([[[0.0, 0.0], [1.0, 0.0], [0.0, 0.0], [0.0, 1.0], [1.0, 0.0]]])
+    x = np.array([[[0.0, 0.0], [0.25, 0.0]]])
+    d, i = O.knn(x, y, 4)
+    assert i[0, 0].tolist() == [0, 2, 1, 3], i[0, 0]
+    _close(d[0, 0], [0, 0, 1, 1], 0, 0, "ties distances")
+    assert i[0, 1].tolist() == [0, 2, 1, 4], i[0, 1]
+    _close(d[0, 1], [0.0625, 0.0625, 0.5625, 0.5625], 0, 0, "near-tie distances")
+    d, i = O.knn(x, y[:, :2], 3)
+    assert i[0, 0].tolist() == [0, 1, -1] and np.isinf(d[0, 0, 2])
+    g = np.array([[[a, b] for a in range(4) for b in range(4)]], dtype=np.float64)  # 4x4 lattice
+    q = np.array([[[1.0, 2.0], [3.0, 0.0]]])
+    d, i = O.knn(q, g, 5)
+    assert i[0, 0].tolist() == [6, 2, 5, 7, 10], i[0, 0]     # itself, then the 4 axis neighbours
+    _close(d[0, 0], [0, 1, 1, 1, 1], 0, 0, "lattice")
+    assert i[0, 1].tolist() == [12, 8, 13, 9, 4], i[0, 1]    # corner: 2 at 1, then diagonal, then 4
+    _close(d[0, 1], [0, 1, 1, 2, 4], 0, 0, "lattice corner")
+
+
+def pin_knn_permutation_and_f32(O):
+    """Permuting the sources permutes the indices; the float decision agrees
+    with the double one away from near-ties."""
+    r = _rng(21)
+    x, y = r.normal(size=(1, 12, 3)), r.normal(size=(1, 50, 3))
+    perm = r.permutation(50)
+    d, i = O.knn(x, y, 6)
+    d2, i2 = O.knn(x, y[:, perm], 6)
+    _close(d2, d, 0, 0, "permuted distances")
+    assert np.array_equal(perm[i2], i), "permuted indices"
+    df, i_f = O.knn(x.astype(np.float32), y.astype(np.float32), 6, f32=True)
+    xd, yd = x.astype(np.float32).astype(np.float64), y.astype(np.float32).astype(np.float64)
+    dd, idd = O.knn(xd, yd, 6)
+    assert np.array_equal(i_f, idd), "float and double decisions differ on separated data"
+    _close(df, dd, 1e-6, 1e-7, "float distances")
+
+
 ALL_PINS = [
     pin_golden_sum, pin_golden_lse, pin_golden_bwd, pin_dense_library, pin_flash_prescale,
     pin_flash_reweight, pin_coincident, pin_single_point, pin_separable_grid, pin_translation,
     pin_small_tau, pin_symmetry, pin_linearity, pin_lse_is_log_sum, pin_rows_subset,
     pin_finite_differences, pin_large_n_expectation, pin_golden_vjp_y_tau, pin_golden_lse_bwd,
     pin_finite_differences_y_tau, pin_finite_differences_lse, pin_gradient_symmetries,
+    pin_knn_against_library_sort, pin_knn_ties_padding_and_grid, pin_knn_permutation_and_f32,
 ]

@@ -34,6 +34,9 @@ MUTANTS = [
     ("lse grad unnormalised weights", [("double p = w[(bb * N + j) * C + c] * e / zs;", "double p = w[(bb * N + j) * C + c] * e;", 1)]),
     ("lse grad_w uses p instead of p / w", [("grad_w[(bb * N + j) * C + c] += gic * e / zs;", "grad_w[(bb * N + j) * C + c] += gic * p;", 1)]),
     ("lse grad_y sign", [("grad_y[(bb * N + j) * D + k] += tau * gic * p * diff;", "grad_y[(bb * N + j) * D + k] += -tau * gic * p * diff;", 1)]),
+    ("knn keeps the largest", [("if (!(d < bd[K - 1] || (d == bd[K - 1] && j < bj[K - 1])))", "if (!(d > bd[K - 1] || (d == bd[K - 1] && j < bj[K - 1])))", 1)]),
+    ("knn ties by the higher index", [("while (p > 0 && (d < bd[p - 1] || (d == bd[p - 1] && j < bj[p - 1]))) {", "while (p > 0 && (d < bd[p - 1] || (d == bd[p - 1] && j > bj[p - 1]))) {", 1)]),
+    ("knn float distance drops a coordinate", [("for (int64_t k = 1; k < D; ++k) {\n                    e = xi[k] - yj[k];", "for (int64_t k = 2; k < D; ++k) {\n                    e = xi[k] - yj[k];", 1)]),
     ("grad_w kernel against x_0 only", [("const double *xi = x + (bb * M + i) * D;\n                    const double *gi", "const double *xi = x + (bb * M) * D;\n                    const double *gi", 1)]),
 ]
 
@@ -58,6 +61,7 @@ class _Handle:
         self.gauss_sum_bwd = functools.partial(oracle.gauss_sum_bwd, lib=lib)
         self.gauss_sum_vjp_y_tau = functools.partial(oracle.gauss_sum_vjp_y_tau, lib=lib)
         self.gauss_lse_bwd = functools.partial(oracle.gauss_lse_bwd, lib=lib)
+        self.knn = functools.partial(oracle.knn, lib=lib)
 
 
 @pytest.mark.parametrize("idx", range(len(MUTANTS)), ids=[m[0] for m in MUTANTS])

@@ -12,6 +12,7 @@ class _Real:
     gauss_sum_bwd = staticmethod(oracle.gauss_sum_bwd)
     gauss_sum_vjp_y_tau = staticmethod(oracle.gauss_sum_vjp_y_tau)
     gauss_lse_bwd = staticmethod(oracle.gauss_lse_bwd)
+    knn = staticmethod(oracle.knn)
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=[p.__name__ for p in ALL_PINS])
