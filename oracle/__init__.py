@@ -15,6 +15,7 @@ step 2):
 * ``gauss_sum_vjp_y_tau(x, y, w, g, tau, yrows=None)`` -> (grad_y, grad_tau)
 * ``gauss_lse_bwd(x, y, w, g, tau)`` -> (grad_x, grad_y, grad_w, grad_tau)
 * ``knn(x, y, K, rows=None, f32=False)`` -> (sq_dist [B, R, K], index [B, R, K])
+* ``diffusion_scales(x, tau, alpha)`` -> (q, d, s) and ``diffusion_apply(x, s, v, tau)``
 
 Inputs are float64 arrays x [B,M,D], y [B,N,D], w [B,N,C], g [B,M,C] (2-D
 arrays are read as B = 1).  Values must already be the quantised values the
@@ -65,6 +66,12 @@ def _load(path=None):
     f = lib.oracle_knn_f32
     f.restype = ctypes.c_int
     f.argtypes = [_fp, _fp, _fp, _ip, _i64, _i64, _i64, _i64, _i64, _ip, _i64]
+    f = lib.oracle_diffusion_scales
+    f.restype = ctypes.c_int
+    f.argtypes = [_dp, _dp, _dp, _dp, _i64, _i64, _i64, ctypes.c_double, ctypes.c_double]
+    f = lib.oracle_diffusion_apply
+    f.restype = ctypes.c_int
+    f.argtypes = [_dp, _dp, _dp, _dp, _i64, _i64, _i64, _i64, ctypes.c_double]
     lib.oracle_num_threads.restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -208,4 +215,30 @@ def knn(x, y, K, rows=None, lib=None, f32=False):
     return od, oi
 
 
-__all__ = ["knn", "gauss_sum_vjp_y_tau", "gauss_lse_bwd", "gauss_sum", "gauss_lse", "gauss_sum_bwd", "num_threads", "build_oracle", "LIB"]
+def diffusion_scales(x, tau, alpha, lib=None):
+    """(q, d, s) of the alpha-normalised diffusion operator over the point set x."""
+    x = _as3(x, "x")
+    B, N, D = x.shape
+    q, d, s = (np.empty((B, N)) for _ in range(3))
+    rc = (lib or _load()).oracle_diffusion_scales(_ptr(x), _ptr(q), _ptr(d), _ptr(s), B, N, D,
+                                                 float(tau), float(alpha))
+    if rc != 0:
+        raise ValueError(f"oracle_diffusion_scales rejected its arguments (code {rc})")
+    return q, d, s
+
+
+def diffusion_apply(x, s, v, tau, lib=None):
+    """diag(s) K diag(s) v over the point set x."""
+    x, v = _as3(x, "x"), _as3(v, "v")
+    B, N, D = x.shape
+    C = v.shape[2]
+    s = np.ascontiguousarray(np.asarray(s, dtype=np.float64).reshape(B, N))
+    out = np.empty((B, N, C))
+    rc = (lib or _load()).oracle_diffusion_apply(_ptr(x), _ptr(s), _ptr(v), _ptr(out), B, N, D, C,
+                                                float(tau))
+    if rc != 0:
+        raise ValueError(f"oracle_diffusion_apply rejected its arguments (code {rc})")
+    return out
+
+
+__all__ = ["diffusion_scales", "diffusion_apply", "knn", "gauss_sum_vjp_y_tau", "gauss_lse_bwd", "gauss_sum", "gauss_lse", "gauss_sum_bwd", "num_threads", "build_oracle", "LIB"]

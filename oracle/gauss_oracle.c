@@ -528,3 +528,91 @@ int oracle_knn_f32(const float *x, const float *y, float *out_d, int64_t *out_id
     }
     return bad ? 2 : 0;
 }
+
+/* Diffusion operator of "FlashDiffusion: Fused Tiled Kernel Spectral
+ * Decomposition" (section 2.2, XGEMM: the operator diag(s) K diag(s) applied
+ * to a block V; the q and d normalisation passes are kernel applications with
+ * V replaced by 1 and by q^-alpha).  The page's section 2.1, which defines s,
+ * is missing from the extracted text; the reading taken is the alpha-
+ * normalised diffusion map those two passes compute:
+ *
+ *   q_i = sum_j K_ij                              (pass with V = 1)
+ *   d_i = q_i^-alpha * sum_j K_ij q_j^-alpha      (pass with V = q^-alpha)
+ *   s_i = q_i^-alpha * d_i^-1/2
+ *   A   = diag(s) K diag(s)  (the symmetric form of the Markov matrix of
+ *         K_ij / (q_i q_j)^alpha)
+ *
+ * with K_ij = exp(-tau/2 |x_i - x_j|^2) over one point set x [B, N, D].
+ * oracle_diffusion_scales writes q, d and s ([B, N] each, any may be NULL);
+ * oracle_diffusion_apply writes out = A V for V [B, N, C]. */
+int oracle_diffusion_scales(const double *x, double *q, double *d, double *s, int64_t B,
+                            int64_t N, int64_t D, double tau, double alpha)
+{
+    if (B < 0 || N < 0 || D < 1 || !(tau > 0.0))
+        return 1;
+    double *qq = (double *)malloc((size_t)((B * N) > 0 ? B * N : 1) * sizeof(double));
+    if (!qq)
+        return 2;
+#pragma omp parallel for schedule(dynamic, 8)
+    for (int64_t t = 0; t < B * N; ++t) {
+        int64_t bb = t / N, i = t % N;
+        comp_sum acc = {0.0, 0.0};
+        for (int64_t j = 0; j < N; ++j)
+            cs_add(&acc, exp(-0.5 * tau * sq_dist(x + (bb * N + i) * D, x + (bb * N + j) * D, D)));
+        qq[t] = cs_value(&acc);
+    }
+#pragma omp parallel for schedule(dynamic, 8)
+    for (int64_t t = 0; t < B * N; ++t) {
+        int64_t bb = t / N, i = t % N;
+        comp_sum acc = {0.0, 0.0};
+        for (int64_t j = 0; j < N; ++j) {
+            double k = exp(-0.5 * tau * sq_dist(x + (bb * N + i) * D, x + (bb * N + j) * D, D));
+            cs_add(&acc, k * pow(qq[bb * N + j], -alpha));
+        }
+        double di = pow(qq[t], -alpha) * cs_value(&acc);
+        if (q)
+            q[t] = qq[t];
+        if (d)
+            d[t] = di;
+        if (s)
+            s[t] = pow(qq[t], -alpha) / sqrt(di);
+    }
+    free(qq);
+    return 0;
+}
+
+int oracle_diffusion_apply(const double *x, const double *s, const double *v, double *out,
+                           int64_t B, int64_t N, int64_t D, int64_t C, double tau)
+{
+    if (B < 0 || N < 0 || D < 1 || C < 1 || !(tau > 0.0))
+        return 1;
+    int bad = 0;
+#pragma omp parallel
+    {
+        comp_sum *acc = (comp_sum *)malloc((size_t)C * sizeof(comp_sum));
+        if (!acc) {
+#pragma omp atomic write
+            bad = 1;
+        }
+#pragma omp for schedule(dynamic, 8)
+        for (int64_t t = 0; t < B * N; ++t) {
+            if (!acc)
+                continue;
+            int64_t bb = t / N, i = t % N;
+            for (int64_t c = 0; c < C; ++c) {
+                acc[c].s = 0.0;
+                acc[c].c = 0.0;
+            }
+            for (int64_t j = 0; j < N; ++j) {
+                double k = exp(-0.5 * tau * sq_dist(x + (bb * N + i) * D, x + (bb * N + j) * D, D));
+                double ksj = k * s[bb * N + j];
+                for (int64_t c = 0; c < C; ++c)
+                    cs_add(&acc[c], ksj * v[(bb * N + j) * C + c]);
+            }
+            for (int64_t c = 0; c < C; ++c)
+                out[t * C + c] = s[t] * cs_value(&acc[c]);
+        }
+        free(acc);
+    }
+    return bad ? 2 : 0;
+}

@@ -442,6 +442,42 @@ def pin_knn_permutation_and_f32(O):
     _close(df, dd, 1e-6, 1e-7, "float distances")
 
 
+# --------------------------------------------------------------------------- diffusion operator
+def pin_diffusion_operator(O):
+    """A = diag(s) K diag(s): sqrt(d) is its fixed point (the Markov matrix
+    D^-1 K_alpha is row-stochastic), A is symmetric with spectrum in [0, 1]
+    (a Gaussian kernel is positive semi-definite), q and d are the kernel
+    applications to 1 and q^-alpha, and two points give a closed form."""
+    r = _rng(22)
+    B, N, D, tau = 2, 40, 3, 1.7
+    x = r.normal(size=(B, N, D))
+    for alpha in (0.0, 0.5, 1.0):
+        q, d, s = O.diffusion_scales(x, tau, alpha)
+        _close(q[..., None], O.gauss_sum(x, x, np.ones((B, N, 1)), tau), 1e-13, 0, "q = K 1")
+        _close(d[..., None], q[..., None] ** -alpha * O.gauss_sum(x, x, q[..., None] ** -alpha, tau),
+               1e-13, 0, "d = q^-a K q^-a")
+        _close(s, q ** -alpha / np.sqrt(d), 1e-14, 0, "s")
+        _close(O.diffusion_apply(x, s, np.sqrt(d)[..., None], tau), np.sqrt(d)[..., None], 1e-12, 0,
+               "sqrt(d) is a fixed point")
+        xt = torch.from_numpy(x[0])
+        K = torch.exp(-0.5 * tau * torch.cdist(xt, xt, compute_mode="donot_use_mm_for_euclid_dist") ** 2)
+        A = (torch.from_numpy(s[0])[:, None] * K * torch.from_numpy(s[0])[None, :]).numpy()
+        ev = np.linalg.eigvalsh(A)
+        assert ev.max() <= 1 + 1e-10 and ev.min() >= -1e-10 and abs(ev.max() - 1) <= 1e-10
+        u, v = r.normal(size=(1, N, 1)), r.normal(size=(1, N, 1))
+        lhs = float((u * O.diffusion_apply(x[:1], s[:1], v, tau)).sum())
+        rhs = float((v * O.diffusion_apply(x[:1], s[:1], u, tau)).sum())
+        assert abs(lhs - rhs) <= 1e-12 * max(1.0, abs(lhs)), "symmetric"
+    # two points at distance^2 = 2: K = [[1, e], [e, 1]], e = exp(-tau); q = 1 + e, A = K / (1 + e)
+    x2 = np.array([[[0.0, 0.0], [1.0, 1.0]]])
+    e = math.exp(-tau)
+    q, d, s = O.diffusion_scales(x2, tau, 0.5)
+    _close(q, [[1 + e, 1 + e]], 1e-15, 0, "two-point q")
+    _close(s, [[(1 + e) ** -0.5, (1 + e) ** -0.5]], 1e-15, 0, "two-point s")
+    _close(O.diffusion_apply(x2, s, np.array([[[1.0], [0.0]]]), tau), [[[1 / (1 + e)], [e / (1 + e)]]],
+           1e-15, 0, "two-point A")
+
+
 ALL_PINS = [
     pin_golden_sum, pin_golden_lse, pin_golden_bwd, pin_dense_library, pin_flash_prescale,
     pin_flash_reweight, pin_coincident, pin_single_point, pin_separable_grid, pin_translation,
@@ -449,4 +485,5 @@ ALL_PINS = [
     pin_finite_differences, pin_large_n_expectation, pin_golden_vjp_y_tau, pin_golden_lse_bwd,
     pin_finite_differences_y_tau, pin_finite_differences_lse, pin_gradient_symmetries,
     pin_knn_against_library_sort, pin_knn_ties_padding_and_grid, pin_knn_permutation_and_f32,
+    pin_diffusion_operator,
 ]

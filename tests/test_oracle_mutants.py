@@ -37,6 +37,9 @@ MUTANTS = [
     ("knn keeps the largest", [("if (!(d < bd[K - 1] || (d == bd[K - 1] && j < bj[K - 1])))", "if (!(d > bd[K - 1] || (d == bd[K - 1] && j < bj[K - 1])))", 1)]),
     ("knn ties by the higher index", [("while (p > 0 && (d < bd[p - 1] || (d == bd[p - 1] && j < bj[p - 1]))) {", "while (p > 0 && (d < bd[p - 1] || (d == bd[p - 1] && j > bj[p - 1]))) {", 1)]),
     ("knn float distance drops a coordinate", [("for (int64_t k = 1; k < D; ++k) {\n                    e = xi[k] - yj[k];", "for (int64_t k = 2; k < D; ++k) {\n                    e = xi[k] - yj[k];", 1)]),
+    ("diffusion d without the left q^-alpha", [("double di = pow(qq[t], -alpha) * cs_value(&acc);", "double di = cs_value(&acc);", 1)]),
+    ("diffusion s with d^-1 instead of d^-1/2", [("s[t] = pow(qq[t], -alpha) / sqrt(di);", "s[t] = pow(qq[t], -alpha) / di;", 1)]),
+    ("diffusion apply without the right scaling", [("double ksj = k * s[bb * N + j];", "double ksj = k;", 1)]),
     ("grad_w kernel against x_0 only", [("const double *xi = x + (bb * M + i) * D;\n                    const double *gi", "const double *xi = x + (bb * M) * D;\n                    const double *gi", 1)]),
 ]
 
@@ -62,6 +65,8 @@ class _Handle:
         self.gauss_sum_vjp_y_tau = functools.partial(oracle.gauss_sum_vjp_y_tau, lib=lib)
         self.gauss_lse_bwd = functools.partial(oracle.gauss_lse_bwd, lib=lib)
         self.knn = functools.partial(oracle.knn, lib=lib)
+        self.diffusion_scales = functools.partial(oracle.diffusion_scales, lib=lib)
+        self.diffusion_apply = functools.partial(oracle.diffusion_apply, lib=lib)
 
 
 @pytest.mark.parametrize("idx", range(len(MUTANTS)), ids=[m[0] for m in MUTANTS])

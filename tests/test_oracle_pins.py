@@ -13,6 +13,8 @@ class _Real:
     gauss_sum_vjp_y_tau = staticmethod(oracle.gauss_sum_vjp_y_tau)
     gauss_lse_bwd = staticmethod(oracle.gauss_lse_bwd)
     knn = staticmethod(oracle.knn)
+    diffusion_scales = staticmethod(oracle.diffusion_scales)
+    diffusion_apply = staticmethod(oracle.diffusion_apply)
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=[p.__name__ for p in ALL_PINS])
