@@ -57,7 +57,14 @@ typedef struct CUstream_st *gs_stream_t;
 
 typedef enum { GS_F32 = 0, GS_F16 = 1, GS_BF16 = 2 } gs_dtype;
 
-typedef enum { GS_OP_SUM = 0, GS_OP_LSE = 1, GS_OP_SUM_BWD = 2, GS_OP_LSE_BWD = 3 } gs_op;
+typedef enum {
+    GS_OP_SUM = 0,
+    GS_OP_LSE = 1,
+    GS_OP_SUM_BWD = 2,
+    GS_OP_LSE_BWD = 3,
+    GS_OP_KNN = 4,      /* gs_workspace_bytes: pass K as C */
+    GS_OP_DIFFUSION = 5 /* gs_workspace_bytes: M = N, C = columns of V (1 for the scales) */
+} gs_op;
 
 typedef enum {
     GS_OK = 0,
@@ -162,6 +169,50 @@ gs_status gauss_lse_bwd(const void *x, const void *y, const void *w, const float
                         const float *g, float *grad_x, float *grad_y, float *grad_w,
                         float *grad_tau, int64_t B, int64_t M, int64_t N, int64_t D, int64_t C,
                         float tau, gs_dtype dt, void *ws, size_t ws_bytes, gs_stream_t stream);
+
+/*
+ * k-nearest reduction ("Kernel matrix reduction", Overview: minima and the
+ * indices of the K smallest entries per row; the .argmin() reduction of the
+ * LazyTensor API): for every row i, the K smallest squared distances
+ * |x[b,i] - y[b,j]|^2 over j, ascending, and their indices j; equal distances
+ * are ordered by the lower j.  Rows with fewer than K sources get +inf and
+ * index -1 in the missing places.  The row maximum of the Gaussian kernel is
+ * exp(-tau/2 * out_sqdist[b,i,0]), attained at out_index[b,i,0].
+ * Distances are computed in fp32 as e_k = x_k - y_k, d = e_0^2, then
+ * d = fma(e_k, e_k, d) for k = 1 .. D-1 (round to nearest), and every
+ * comparison is made on those fp32 values.
+ *     out_sqdist [B, M, K] float32, out_index [B, M, K] int64.
+ * GS_F32, 1 <= D <= 8, 1 <= K <= 32.  Workspace:
+ * gs_workspace_bytes(GS_OP_KNN, B, M, N, D, K, GS_F32).
+ */
+gs_status gauss_knn(const void *x, const void *y, float *out_sqdist, int64_t *out_index, int64_t B,
+                    int64_t M, int64_t N, int64_t D, int64_t K, gs_dtype dt, void *ws,
+                    size_t ws_bytes, gs_stream_t stream);
+
+/*
+ * Diffusion operator of "FlashDiffusion: Fused Tiled Kernel Spectral
+ * Decomposition" (section 2.2, XGEMM: diag(s) K diag(s) applied to a block V;
+ * the q and d normalisation passes are kernel applications with V replaced by
+ * 1 and by q^-alpha; the right scaling is applied to V, the left one to the
+ * rows of the result).  Over one point set x [B, N, D], K_ij =
+ * exp(-tau/2 |x_i - x_j|^2).  The page's section 2.1, defining s, did not
+ * survive extraction; the reading implemented is the alpha-normalised diffusion
+ * map those passes compute:
+ *     q = K 1,  d = q^-alpha (K q^-alpha),  s = q^-alpha d^-1/2,
+ * so that diag(s) K diag(s) is the symmetric form of the Markov matrix of
+ * K_ij / (q_i q_j)^alpha (eigenvalues in [0, 1], sqrt(d) its fixed point).
+ *   gauss_diffusion_scales: s_out [B, N] (q_out, d_out optional, may be NULL)
+ *   gauss_diffusion_apply:  out [B, N, C] = diag(s) K diag(s) v, v [B, N, C]
+ * All of s, q, d, v, out are float32; x has dtype dt (the paths of
+ * gauss_sum_fwd).  Workspace: gs_workspace_bytes(GS_OP_DIFFUSION, B, N, N, D, C, dt)
+ * with C = 1 for the scales.
+ */
+gs_status gauss_diffusion_scales(const void *x, float *q_out, float *d_out, float *s_out,
+                                 int64_t B, int64_t N, int64_t D, float tau, float alpha,
+                                 gs_dtype dt, void *ws, size_t ws_bytes, gs_stream_t stream);
+gs_status gauss_diffusion_apply(const void *x, const float *s, const float *v, float *out,
+                                int64_t B, int64_t N, int64_t D, int64_t C, float tau, gs_dtype dt,
+                                void *ws, size_t ws_bytes, gs_stream_t stream);
 
 /*
  * Allocation-free variant of gauss_sum_fwd (no counterpart on the pages: it

@@ -23,7 +23,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = _build.LIB
 
 GS_F32, GS_F16, GS_BF16 = 0, 1, 2
-GS_OP_SUM, GS_OP_LSE, GS_OP_SUM_BWD, GS_OP_LSE_BWD = 0, 1, 2, 3
+GS_OP_SUM, GS_OP_LSE, GS_OP_SUM_BWD, GS_OP_LSE_BWD, GS_OP_KNN, GS_OP_DIFFUSION = 0, 1, 2, 3, 4, 5
 STATUS = {0: "GS_OK", 1: "GS_ERR_INVALID_ARG", 2: "GS_ERR_UNSUPPORTED", 3: "GS_ERR_ALIGNMENT",
           4: "GS_ERR_WORKSPACE", 5: "GS_ERR_TIMEOUT", 6: "GS_ERR_CUDA"}
 _DT = {torch.float32: GS_F32, torch.float16: GS_F16, torch.bfloat16: GS_BF16}
@@ -42,6 +42,12 @@ SIGNATURES = {
                                      _i64, _f, ctypes.c_int, _vp, _sz, _vp]),
     "gauss_lse_bwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
                                      _i64, _i64, _f, ctypes.c_int, _vp, _sz, _vp]),
+    "gauss_knn": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, ctypes.c_int, _vp,
+                                 _sz, _vp]),
+    "gauss_diffusion_scales": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _f, _f,
+                                              ctypes.c_int, _vp, _sz, _vp]),
+    "gauss_diffusion_apply": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _f,
+                                             ctypes.c_int, _vp, _sz, _vp]),
     "gs_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "gs_last_device_error": (ctypes.c_int, [_vp]),
     "gs_version": (ctypes.c_int, []),
@@ -231,6 +237,54 @@ def gauss_lse_bwd(x, y, w, lse, g, tau, want=("x", "y", "w", "tau"), workspace=N
     return {k: v for k, v in out.items() if v is not None}
 
 
+def gauss_knn(x, y, K, workspace=None, stream=None):
+    """K smallest squared distances per row (ascending, ties by the lower index)
+    and their int64 indices; float32 inputs."""
+    x, y = _as3(x, "x"), _as3(y, "y")
+    B, M, D = x.shape
+    N = y.shape[1]
+    if y.shape[0] != B or y.shape[2] != D or x.dtype != y.dtype or x.dtype not in _DT:
+        raise ValueError(f"shape/dtype mismatch x{tuple(x.shape)} y{tuple(y.shape)}")
+    od = torch.empty((B, M, K), dtype=torch.float32, device=x.device)
+    oi = torch.empty((B, M, K), dtype=torch.int64, device=x.device)
+    nbytes = workspace_bytes(GS_OP_KNN, B, M, N, D, K, x.dtype)
+    ws = _workspace(nbytes, x.device, workspace)
+    st = _lib.gauss_knn(_ptr(x), _ptr(y), _ptr(od), _ptr(oi), B, M, N, D, int(K), _DT[x.dtype],
+                        _ptr(ws), nbytes if ws is not None else 0, _stream(stream))
+    _check("gauss_knn", "gauss_diffusion_scales", "gauss_diffusion_apply", st)
+    return od, oi
+
+
+def gauss_diffusion_scales(x, tau, alpha, workspace=None, stream=None):
+    """(q, d, s) of the alpha-normalised diffusion operator over the point set x."""
+    x = _as3(x, "x")
+    B, N, D = x.shape
+    q, d, s = (torch.empty((B, N), dtype=torch.float32, device=x.device) for _ in range(3))
+    nbytes = workspace_bytes(GS_OP_DIFFUSION, B, N, N, D, 1, x.dtype)
+    ws = _workspace(nbytes, x.device, workspace)
+    st = _lib.gauss_diffusion_scales(_ptr(x), _ptr(q), _ptr(d), _ptr(s), B, N, D, float(tau),
+                                     float(alpha), _DT[x.dtype], _ptr(ws),
+                                     nbytes if ws is not None else 0, _stream(stream))
+    _check("gauss_diffusion_scales", st)
+    return q, d, s
+
+
+def gauss_diffusion_apply(x, s, v, tau, out=None, workspace=None, stream=None):
+    """diag(s) K diag(s) v over the point set x (float32 s, v)."""
+    x, v = _as3(x, "x"), _as3(v, "v")
+    B, N, D = x.shape
+    C = v.shape[2]
+    if out is None:
+        out = torch.empty((B, N, C), dtype=torch.float32, device=x.device)
+    nbytes = workspace_bytes(GS_OP_DIFFUSION, B, N, N, D, C, x.dtype)
+    ws = _workspace(nbytes, x.device, workspace)
+    st = _lib.gauss_diffusion_apply(_ptr(x), _ptr(s.contiguous()), _ptr(v), _ptr(out), B, N, D, C,
+                                    float(tau), _DT[x.dtype], _ptr(ws),
+                                    nbytes if ws is not None else 0, _stream(stream))
+    _check("gauss_diffusion_apply", st)
+    return out
+
+
 def test_exp2_poly(x, degree, stream=None):
     """Device evaluation of the FMA-pipe 2^x (test hook, see include/gauss_testing.h)."""
     if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
@@ -246,6 +300,6 @@ def last_device_error(stream=None):
     return int(_lib.gs_last_device_error(_stream(stream)))
 
 
-__all__ = ["gauss_sum_fwd", "gauss_sum_fwd_noalloc", "gauss_lse_fwd", "gauss_sum_bwd", "gauss_sum_vjp", "gauss_lse_bwd", "workspace_bytes",
+__all__ = ["gauss_sum_fwd", "gauss_sum_fwd_noalloc", "gauss_lse_fwd", "gauss_sum_bwd", "gauss_sum_vjp", "gauss_lse_bwd", "gauss_knn", "gauss_diffusion_scales", "gauss_diffusion_apply", "workspace_bytes",
            "last_device_error", "library", "status_string", "GaussError", "SIGNATURES",
            "LIB_PATH"]

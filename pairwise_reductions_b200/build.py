@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libgauss_b200.so")
-SOURCES = ["api.cpp", "small_d.cu", "tc_sm100.cu", "grad.cu", "noalloc.cu"]
+SOURCES = ["api.cpp", "small_d.cu", "tc_sm100.cu", "grad.cu", "knn.cu", "noalloc.cu"]
 HEADERS = ["internal.h", "ptx.cuh", "exp2_poly.cuh", "values.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

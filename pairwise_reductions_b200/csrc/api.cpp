@@ -366,6 +366,29 @@ LseBwdLayout lse_bwd_layout(const void* x, const void* y, const void* w, const f
   return L;
 }
 
+// Diffusion operator: q = K 1 and u = K q^-alpha (scales), and K (s V) (apply),
+// each one forward pass over a single point set, with f32 value blocks.
+struct DiffusionLayout {
+  PassLayout lp;
+  size_t off_vals, off_a, off_b, total;
+};
+
+DiffusionLayout diffusion_layout(int64_t B, int64_t N, int64_t D, int64_t C, gs_dtype dt, int sm) {
+  DiffusionLayout L{};
+  Pass p = fwd_pass(nullptr, nullptr, nullptr, B, N, N, D, C, 1.f, dt);
+  p.w_is_f32 = true;
+  L.lp = pass_layout(p, sm);
+  size_t off = align_up(L.lp.total);
+  L.off_vals = off;
+  off = align_up(off + size_t(B) * N * C * 4);
+  L.off_a = off;
+  off = align_up(off + size_t(B) * N * 4);
+  L.off_b = off;
+  off = align_up(off + size_t(B) * N * 4);
+  L.total = off;
+  return L;
+}
+
 }  // namespace
 
 extern "C" {
@@ -387,7 +410,23 @@ const char* gs_status_string(gs_status st) {
 
 size_t gs_workspace_bytes(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, int64_t C,
                           gs_dtype dt) {
-  if (op != GS_OP_SUM && op != GS_OP_LSE && op != GS_OP_SUM_BWD && op != GS_OP_LSE_BWD) return kBad;
+  if (op != GS_OP_SUM && op != GS_OP_LSE && op != GS_OP_SUM_BWD && op != GS_OP_LSE_BWD &&
+      op != GS_OP_KNN && op != GS_OP_DIFFUSION)
+    return kBad;
+  if (op == GS_OP_DIFFUSION) {
+    // one point set: M = N; C = columns of the block V (1 for the scales)
+    if (check_dims(GS_OP_SUM, B, N, N, D, C, dt) != GS_OK || M != N) return kBad;
+    if (B == 0 || N == 0) return 0;
+    return diffusion_layout(B, N, D, C, dt, sm_count()).total;
+  }
+  if (op == GS_OP_KNN) {
+    // C carries K for this op
+    if (dt != GS_F32 || C < 1 || C > kKnnMaxK || check_dims(GS_OP_SUM, B, M, N, D, 1, dt) != GS_OK)
+      return kBad;
+    if (B == 0 || M == 0 || N == 0) return 0;
+    const KnnPlan kp = knn_plan(B, M, N, static_cast<int>(C), sm_count());
+    return align_up(size_t(kp.splits) * B * M * C * 8);
+  }
   if (check_dims(op, B, M, N, D, C, dt) != GS_OK) return kBad;
   if (B == 0) return 0;
   const int sm = sm_count();
@@ -622,6 +661,101 @@ gs_status gauss_lse_bwd(const void* x, const void* y, const void* w, const float
     }
   }
   if (grad_tau) GS_CUDA(launch_sum_rows(tau_rows, B * M, grad_tau, s));
+  return GS_OK;
+}
+
+gs_status gauss_knn(const void* x, const void* y, float* out_sqdist, int64_t* out_index, int64_t B,
+                    int64_t M, int64_t N, int64_t D, int64_t K, gs_dtype dt, void* ws,
+                    size_t ws_bytes, gs_stream_t stream) {
+  GS_TRY(check_dims(GS_OP_SUM, B, M, N, D, 1, dt));
+  if (K < 1) return GS_ERR_INVALID_ARG;
+  if (dt != GS_F32 || K > kKnnMaxK) return GS_ERR_UNSUPPORTED;
+  GS_TRY(check_ptr(x, B * M * D));
+  GS_TRY(check_ptr(y, B * N * D));
+  GS_TRY(check_ptr(out_sqdist, B * M * K));
+  GS_TRY(check_ptr(out_index, B * M * K));
+  if (B == 0 || M == 0) return GS_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (N == 0) {   // no source: +inf distances, index -1 (all bytes 0xff)
+    GS_CUDA(launch_fill(out_sqdist, B * M * K, INFINITY, s));
+    GS_CUDA(cudaMemsetAsync(out_index, 0xff, size_t(B) * M * K * sizeof(int64_t), s));
+    return GS_OK;
+  }
+  const KnnPlan kp = knn_plan(B, M, N, static_cast<int>(K), sm_count());
+  const size_t need = align_up(size_t(kp.splits) * B * M * K * 8);
+  if (ws_bytes < need) return GS_ERR_WORKSPACE;
+  GS_TRY(check_ptr(ws, 1));
+  KnnArgs a{};
+  a.x = static_cast<const float*>(x);
+  a.y = static_cast<const float*>(y);
+  a.part_d = static_cast<float*>(ws);
+  a.part_i = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + size_t(kp.splits) * B * M * K * 4);
+  a.out_d = out_sqdist;
+  a.out_i = out_index;
+  a.B = B;
+  a.M = M;
+  a.N = N;
+  a.D = static_cast<int>(D);
+  a.K = static_cast<int>(K);
+  a.splits = kp.splits;
+  a.cols_per_split = kp.cols_per_split;
+  a.split_stride = B * M * K;
+  GS_CUDA(launch_knn(a, s));
+  return GS_OK;
+}
+
+gs_status gauss_diffusion_scales(const void* x, float* q_out, float* d_out, float* s_out,
+                                 int64_t B, int64_t N, int64_t D, float tau, float alpha,
+                                 gs_dtype dt, void* ws, size_t ws_bytes, gs_stream_t stream) {
+  GS_TRY(check_dims(GS_OP_SUM, B, N, N, D, 1, dt));
+  GS_TRY(check_tau(tau));
+  if (!std::isfinite(alpha)) return GS_ERR_INVALID_ARG;
+  GS_TRY(check_ptr(x, B * N * D));
+  GS_TRY(check_ptr(s_out, B * N));
+  if (q_out) GS_TRY(check_ptr(q_out, B * N));
+  if (d_out) GS_TRY(check_ptr(d_out, B * N));
+  if (B == 0 || N == 0) return GS_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const DiffusionLayout L = diffusion_layout(B, N, D, 1, dt, sm_count());
+  if (ws_bytes < L.total) return GS_ERR_WORKSPACE;
+  GS_TRY(check_ptr(ws, 1));
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  float* vals = reinterpret_cast<float*>(wsb + L.off_vals);
+  float* q = q_out ? q_out : reinterpret_cast<float*>(wsb + L.off_a);
+  float* u = reinterpret_cast<float*>(wsb + L.off_b);
+  Pass p = fwd_pass(x, x, vals, B, N, N, D, 1, tau, dt);
+  p.w_is_f32 = true;
+  GS_CUDA(launch_diffusion_elementwise(0, nullptr, nullptr, vals, nullptr, B * N, 1, alpha, s));
+  GS_TRY(run_pass(p, L.lp, q, wsb, s));                       // q = K 1
+  GS_CUDA(launch_diffusion_elementwise(1, q, nullptr, vals, nullptr, B * N, 1, alpha, s));
+  GS_TRY(run_pass(p, L.lp, u, wsb, s));                       // u = K q^-alpha
+  GS_CUDA(launch_diffusion_elementwise(2, q, u, d_out, s_out, B * N, 1, alpha, s));
+  return GS_OK;
+}
+
+gs_status gauss_diffusion_apply(const void* x, const float* s_scale, const float* v, float* out,
+                                int64_t B, int64_t N, int64_t D, int64_t C, float tau, gs_dtype dt,
+                                void* ws, size_t ws_bytes, gs_stream_t stream) {
+  GS_TRY(check_dims(GS_OP_SUM, B, N, N, D, C, dt));
+  GS_TRY(check_tau(tau));
+  GS_TRY(check_ptr(x, B * N * D));
+  GS_TRY(check_ptr(s_scale, B * N));
+  GS_TRY(check_ptr(v, B * N * C));
+  GS_TRY(check_ptr(out, B * N * C));
+  if (B == 0 || N == 0) return GS_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const DiffusionLayout L = diffusion_layout(B, N, D, C, dt, sm_count());
+  if (ws_bytes < L.total) return GS_ERR_WORKSPACE;
+  GS_TRY(check_ptr(ws, 1));
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  float* sv = reinterpret_cast<float*>(wsb + L.off_vals);
+  const int64_t n = B * N * C;
+  GS_CUDA(launch_diffusion_elementwise(3, s_scale, v, sv, nullptr, n, static_cast<int>(C), 0.f, s));
+  Pass p = fwd_pass(x, x, sv, B, N, N, D, C, tau, dt);
+  p.w_is_f32 = true;
+  GS_TRY(run_pass(p, L.lp, out, wsb, s));                     // K (s V)
+  GS_CUDA(launch_diffusion_elementwise(3, s_scale, out, out, nullptr, n, static_cast<int>(C), 0.f,
+                                       s));                    // left scaling
   return GS_OK;
 }
 

@@ -210,6 +210,36 @@ __global__ void lse_grad_y_epilogue_kernel(const float* __restrict__ y, const fl
   }
 }
 
+// Elementwise steps of the diffusion operator (FlashDiffusion XGEMM section).
+__global__ void diffusion_elementwise_kernel(int op, const float* __restrict__ a,
+                                             const float* __restrict__ b2, float* __restrict__ o1,
+                                             float* __restrict__ o2, int64_t n, int C,
+                                             float alpha) {
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    switch (op) {
+      case 0:   // o1 = 1
+        o1[e] = 1.f;
+        break;
+      case 1:   // o1 = a^-alpha
+        o1[e] = powf(a[e], -alpha);
+        break;
+      case 2: {   // a = q, b2 = K q^-alpha  ->  o1 = d = q^-alpha b2, o2 = s = q^-alpha d^-1/2
+        const float qa = powf(a[e], -alpha);
+        const float d = qa * b2[e];
+        if (o1) o1[e] = d;
+        o2[e] = qa * rsqrtf(d);
+        break;
+      }
+      case 3:   // o1[e] = a[e / C] * b2[e]   (row scale of a [rows, C] block)
+        o1[e] = a[e / C] * b2[e];
+        break;
+      default:
+        break;
+    }
+  }
+}
+
 template <typename T>
 const T* as(const void* p) {
   return static_cast<const T*>(p);
@@ -291,6 +321,13 @@ cudaError_t launch_weighted_rows(const float* g, const float* o, float* tau_rows
                                  cudaStream_t s) {
   weighted_rows_kernel<<<grid_for(rows, 256), 256, 0, s>>>(g, o, tau_rows, rows, C, c0, nc, factor,
                                                            accumulate ? 1 : 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_diffusion_elementwise(int op, const float* a, const float* b, float* o1,
+                                         float* o2, int64_t n, int C, float alpha,
+                                         cudaStream_t s) {
+  diffusion_elementwise_kernel<<<grid_for(n, 256), 256, 0, s>>>(op, a, b, o1, o2, n, C, alpha);
   return cudaGetLastError();
 }
 

@@ -116,6 +116,11 @@ cudaError_t launch_grad_y_epilogue(const void* y, const void* w, gs_dtype dt, co
 cudaError_t launch_weighted_rows(const float* g, const float* o, float* tau_rows, int64_t rows,
                                  int C, int c0, int nc, float factor, bool accumulate,
                                  cudaStream_t s);
+// Diffusion operator elementwise steps (grad.cu): op 0 o1 = 1; op 1 o1 = a^-alpha;
+// op 2 (a = q, b = K q^-alpha) o1 = d = q^-alpha b, o2 = s = q^-alpha d^-1/2;
+// op 3 o1[e] = a[e / C] * b[e].
+cudaError_t launch_diffusion_elementwise(int op, const float* a, const float* b, float* o1,
+                                         float* o2, int64_t n, int C, float alpha, cudaStream_t s);
 // out[0] = sum of v[0 .. n) in a fixed order (double accumulation).
 cudaError_t launch_sum_rows(const float* v, int64_t n, float* out, cudaStream_t s);
 
@@ -158,6 +163,28 @@ cudaError_t launch_tc_sum(const TcArgs& a, cudaStream_t s);
 
 // out[0 .. n) = value
 cudaError_t launch_fill(float* out, int64_t n, float value, cudaStream_t s);
+
+// ------------------------------------------------------------- k-nearest reduction
+constexpr int kKnnMaxK = 32;
+struct KnnPlan {
+  int splits;
+  int64_t cols_per_split;
+};
+KnnPlan knn_plan(int64_t B, int64_t M, int64_t N, int K, int sm_count);
+struct KnnArgs {
+  const float* x;
+  const float* y;
+  float* part_d;       // [splits][B][M][K] per-split sorted lists
+  int* part_i;
+  float* out_d;        // [B, M, K]
+  int64_t* out_i;
+  int64_t B, M, N;
+  int D, K;
+  int splits;
+  int64_t cols_per_split;
+  int64_t split_stride;   // B * M * K
+};
+cudaError_t launch_knn(const KnnArgs& a, cudaStream_t s);
 
 // Device error word (set by kernels whose waits time out).
 cudaError_t read_and_clear_device_error(int* value);

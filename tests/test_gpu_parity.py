@@ -335,3 +335,53 @@ def test_lse_bwd_rows_far_from_every_point():
     assert np.isfinite(got["x"].cpu().numpy()).all()
     assert rel_l2(got["x"].cpu().numpy(), rgx) <= TOL["f32"]
     assert rel_l2(got["w"].cpu().numpy(), rgw) <= TOL["f32"]
+
+
+# ------------------------------------------------------------------ k-nearest reduction
+@pytest.mark.parametrize("shape", [(1, 1000, 3000, 3, 1), (2, 777, 1301, 3, 5), (1, 300, 5000, 8, 32),
+                                   (1, 513, 257, 2, 16), (1, 50, 10, 3, 16), (3, 129, 4097, 1, 8),
+                                   (1, 2049, 20000, 3, 4)])
+def test_knn_bit_exact(shape):
+    """Indices bit-exact, distances bit-exact: both sides decide in fp32 with the
+    same order of operations, ties by the lower index."""
+    B, M, N, D, K = shape
+    inp = synth.make_inputs(1, seed=19, B=B, M=M, N=N, D=D, C=1)
+    d = dev(inp)
+    od, oi = gs().gauss_knn(d["x"], d["y"], K)
+    rd, ri = oracle.knn(inp["x"].numpy(), inp["y"].numpy(), K, f32=True)
+    assert np.array_equal(oi.cpu().numpy(), ri), "indices differ"
+    assert np.array_equal(od.cpu().numpy(), rd), "distances differ"
+
+
+def test_knn_duplicates_and_quantised_grid():
+    """Many exact ties: duplicated sources and points on a coarse grid."""
+    g = torch.Generator().manual_seed(20)
+    y = torch.randint(0, 4, (1, 3000, 3), generator=g).float() * 0.5
+    y = torch.cat([y, y[:, :500]], dim=1)                 # exact duplicates at higher indices
+    x = torch.randint(0, 4, (1, 700, 3), generator=g).float() * 0.5 + 0.25
+    od, oi = gs().gauss_knn(x.cuda(), y.cuda(), 12)
+    rd, ri = oracle.knn(x.numpy(), y.numpy(), 12, f32=True)
+    assert np.array_equal(oi.cpu().numpy(), ri)
+    assert np.array_equal(od.cpu().numpy(), rd)
+
+
+# ------------------------------------------------------------------ diffusion operator
+@pytest.mark.parametrize("dtype,shape,alpha", [("f32", (1, 3000, 3, 4), 0.5), ("f32", (2, 1500, 6, 1), 1.0),
+                                               ("f32", (1, 2000, 2, 3), 0.0), ("f16", (1, 2500, 32, 8), 0.5),
+                                               ("bf16", (2, 1000, 16, 2), 0.5)])
+def test_diffusion_scales_and_apply(dtype, shape, alpha):
+    B, N, D, C = shape
+    inp = synth.make_inputs(1 if dtype == "f32" else 4, seed=23, B=B, M=N, N=N, D=D, C=C, dtype=dtype)
+    tau = 2.0 if dtype == "f32" else 8.0
+    x = inp["x"].cuda()
+    q, dd, s = gs().gauss_diffusion_scales(x, tau, alpha)
+    rq, rd, rs = oracle.diffusion_scales(f64(inp, "x"), tau, alpha)
+    for name, got, ref in (("q", q, rq), ("d", dd, rd), ("s", s, rs)):
+        assert rel_l2(got.cpu().numpy(), ref) <= TOL[dtype], (name, rel_l2(got.cpu().numpy(), ref))
+    v = torch.randn(B, N, C, generator=torch.Generator().manual_seed(24))
+    out = gs().gauss_diffusion_apply(x, s, v.cuda(), tau)
+    ref = oracle.diffusion_apply(f64(inp, "x"), s.cpu().double().numpy(), v.double().numpy(), tau)
+    assert rel_l2(out.cpu().numpy(), ref) <= TOL[dtype], rel_l2(out.cpu().numpy(), ref)
+    # sqrt(d) is the operator's fixed point
+    fp = gs().gauss_diffusion_apply(x, s, dd.sqrt()[..., None].contiguous(), tau)
+    assert rel_l2(fp.cpu().numpy(), dd.sqrt()[..., None].cpu().numpy()) <= TOL[dtype]
