@@ -251,7 +251,7 @@ def gauss_knn(x, y, K, workspace=None, stream=None):
     ws = _workspace(nbytes, x.device, workspace)
     st = _lib.gauss_knn(_ptr(x), _ptr(y), _ptr(od), _ptr(oi), B, M, N, D, int(K), _DT[x.dtype],
                         _ptr(ws), nbytes if ws is not None else 0, _stream(stream))
-    _check("gauss_knn", "gauss_diffusion_scales", "gauss_diffusion_apply", st)
+    _check("gauss_knn", st)
     return od, oi
 
 

@@ -117,3 +117,20 @@ def test_build_refuses_spills_in_tensor_core_kernels():
     b._check_spills(ok_log)
     with pytest.raises(RuntimeError):
         b._check_spills(ok_log.replace("0 bytes spill stores", "12 bytes spill stores"))
+
+
+def test_binding_status_checks_are_well_formed():
+    """Every _check(name, status) call in the binding names a declared entry
+    point and passes exactly two arguments (a static check: the GPU-only paths
+    that reach these calls cannot run here)."""
+    import ast
+    src = open(os.path.join(os.path.dirname(INCLUDE), "pairwise_reductions_b200", "__init__.py")).read()
+    calls = [n for n in ast.walk(ast.parse(src)) if isinstance(n, ast.Call)
+             and getattr(n.func, "id", None) == "_check"]
+    assert calls
+    declared = set(_declared_functions())
+    for c in calls:
+        assert len(c.args) == 2 and not c.keywords, ast.unparse(c)
+        first = c.args[0]
+        if isinstance(first, ast.Constant):
+            assert first.value in declared, first.value
