@@ -21,7 +21,7 @@
  *
  * Supported shapes and types:
  *     GS_F32           : 1 <= D <= 8 (CUDA-core path), any C >= 1
- *     GS_F16 / GS_BF16 : 1 <= D <= 126 (tensor-core path), any C >= 1.
+ *     GS_F16 / GS_BF16 : 1 <= D <= 128 (tensor-core path), any C >= 1.
  *                        Arithmetic: x.y on the tensor cores with fp32
  *                        accumulation, kernel values rounded to fp16 for the
  *                        second product, weights converted to fp16 (for bf16

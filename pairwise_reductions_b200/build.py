@@ -17,7 +17,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libgauss_b200.so")
-SOURCES = ["api.cpp", "small_d.cu", "tc_sm100.cu", "grad.cu", "knn.cu", "noalloc.cu"]
+SOURCES = ["api.cpp", "small_d.cu", "tc_sm100.cu", "tc_f32_sm100.cu", "grad.cu", "knn.cu",
+           "noalloc.cu"]
 HEADERS = ["internal.h", "ptx.cuh", "exp2_poly.cuh", "values.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -39,8 +40,11 @@ def _flags(verbose):
 
 # Kernels whose registers receive asynchronous tcgen05.ld results must not
 # spill: a spill store placed between the load and its tcgen05.wait::ld would
-# save a register before the load has written it.  The build refuses them.
-NO_SPILL_KERNELS = ("tc_gauss_kernel",)
+# save a register before the load has written it.  The pair loops of the
+# small-D kernel must not spill either: a local-memory round trip per point
+# would cost more than the exponential it serves.  The build refuses both.
+NO_SPILL_KERNELS = ("tc_gauss_kernel", "tc_f32_kernel", "sd_kernel")
+SPILL_CHECKED = ("tc_sm100.cu", "tc_f32_sm100.cu", "small_d.cu")
 
 
 def _check_spills(ptxas_log):
@@ -56,7 +60,7 @@ def _check_spills(ptxas_log):
             if int(m.group(1)) or int(m.group(2)):
                 bad.append((current, m.group(0)))
     if bad:
-        raise RuntimeError("register spills in kernels that hold tcgen05.ld results: " + repr(bad))
+        raise RuntimeError("register spills in kernels that must not spill: " + repr(bad))
 
 
 def _stale(out, deps):
@@ -78,7 +82,7 @@ def build(force=False, verbose=False):
         obj = os.path.join(BUILD, src + ".o")
         objs.append(obj)
         if force or _stale(obj, [sp] + hdrs):
-            cmd = [nvcc, *_flags(verbose or src == "tc_sm100.cu"), "-c", sp, "-o", obj]
+            cmd = [nvcc, *_flags(verbose or src in SPILL_CHECKED), "-c", sp, "-o", obj]
             if src.endswith(".cpp"):
                 cmd[1:1] = ["-x", "cu"]
             jobs.append(cmd)
@@ -91,7 +95,7 @@ def build(force=False, verbose=False):
             if r.returncode != 0:
                 sys.stderr.write(r.stdout + r.stderr)
                 raise RuntimeError("nvcc failed: " + " ".join(cmd))
-            if "tc_sm100.cu" in cmd[-3]:
+            if os.path.basename(cmd[-3]) in SPILL_CHECKED:
                 try:
                     _check_spills(r.stderr)
                 except RuntimeError:

@@ -46,7 +46,10 @@ gs_status check_dims(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, int64
   if (double(B) * double(M > N ? M : N) * double((D > C ? D : C) + 1) * double(D + 2) > big)
     return GS_ERR_UNSUPPORTED;
   if (dt == GS_F32) {
-    if (D > kSdMaxD) return GS_ERR_UNSUPPORTED;
+    // D > 8: the split-tf32 tensor-core path, for the Gauss-sum passes only
+    if (D > kTcMaxD) return GS_ERR_UNSUPPORTED;
+    if (D > kSdMaxD && (op == GS_OP_LSE || op == GS_OP_LSE_BWD || op == GS_OP_KNN))
+      return GS_ERR_UNSUPPORTED;
   } else {
     if (D > kTcMaxD) return GS_ERR_UNSUPPORTED;
     if (op == GS_OP_LSE || op == GS_OP_LSE_BWD) return GS_ERR_UNSUPPORTED;
@@ -103,19 +106,53 @@ struct Pass {
   float shift_scale;
 };
 
+// Which kernel family runs a pass: the CUDA-core small-D kernel (fp32, D <= 8),
+// the fp16/bf16 tensor-core kernel, or the split-tf32 tensor-core kernel
+// (fp32, D > 8).
+enum PassPath { kPathSmallD = 0, kPathTcHalf = 1, kPathTcF32 = 2 };
+
+PassPath pass_path(gs_dtype dt, int D) {
+  if (dt != GS_F32) return kPathTcHalf;
+  return D <= kSdMaxD ? kPathSmallD : kPathTcF32;
+}
+
 struct PassLayout {
   bool tc;
+  PassPath path;
   SdPlan sd;
   TcPlan tcp;
-  size_t off_part, off_vals, off_xpack, off_rnorm, off_ypack, off_vt;
+  F32Plan f32;
+  size_t off_part, off_vals, off_xpack, off_rnorm, off_ypack, off_vt, off_qw;
   size_t total;
 };
 
 PassLayout pass_layout(const Pass& p, int sm) {
   PassLayout L{};
   size_t off = 0;
-  L.tc = p.dt != GS_F32;
-  if (!L.tc) {
+  L.path = pass_path(p.dt, p.D);
+  L.tc = L.path != kPathSmallD;
+  if (L.path == kPathTcF32) {
+    L.f32 = f32_plan(p.B, p.R, p.N, p.D, sm);
+    const size_t rowb = size_t(2) * L.f32.Kp * 4;
+    const size_t CPmax = static_cast<size_t>(
+        f32_chunk_pad(p.CV < L.f32.max_chunk ? p.CV : L.f32.max_chunk));
+    const size_t Nst = (p.N + 3) / 4 * 4;
+    const size_t Nq = (p.N + 63) / 64 * 64;
+    L.off_xpack = off;
+    off = align_up(off + size_t(p.B) * p.R * rowb);
+    L.off_rnorm = off;
+    off = align_up(off + size_t(p.B) * p.R * 4);
+    L.off_ypack = off;
+    off = align_up(off + size_t(p.B) * p.N * rowb);
+    L.off_qw = off;
+    off = align_up(off + size_t(p.B) * Nq * 16);
+    L.off_vt = off;
+    off = align_up(off + size_t(2) * p.B * CPmax * Nst * 4);
+    if (L.f32.splits > 1) {
+      L.off_part = off;
+      off = align_up(off + size_t(L.f32.splits) * p.B * p.R * p.CV * 4);
+    }
+  } else if (!L.tc) {
     L.sd = sd_plan(p.B, p.R, p.N, p.D, p.CV, sm);
     if (p.vmode != 0) {
       L.off_vals = off;
@@ -128,9 +165,8 @@ PassLayout pass_layout(const Pass& p, int sm) {
   } else {
     L.tcp = tc_plan(p.B, p.R, p.N, p.D, sm);
     const size_t KP = static_cast<size_t>(L.tcp.KP);
-    const int chunk = p.CV < kTcMaxChunk ? p.CV : kTcMaxChunk;
-    const size_t CPmax = (chunk + 15) / 16 * 16 <= 64 ? (chunk + 15) / 16 * 16
-                                                      : ((chunk + 15) / 16 * 16 <= 96 ? 96 : 128);
+    const int maxc = tc_max_chunk(L.tcp.KP);
+    const size_t CPmax = static_cast<size_t>(tc_chunk_pad(p.CV < maxc ? p.CV : maxc));
     const size_t Nst = (p.N + 7) / 8 * 8;
     L.off_xpack = off;
     off = align_up(off + size_t(p.B) * p.R * KP * 2);
@@ -192,6 +228,33 @@ gs_status run_pass(const Pass& p, const PassLayout& L, float* out, uint8_t* ws, 
       a.shift_scale = p.shift_scale;
       GS_CUDA(launch_small_d_sum(a, s));
     }
+    if (S > 1) GS_CUDA(launch_combine_sum(dst, S, total, out, s));
+    return GS_OK;
+  }
+  if (L.path == kPathTcF32) {
+    const int S = L.f32.splits;
+    float* dst = S > 1 ? reinterpret_cast<float*>(ws + L.off_part) : out;
+    F32Args a{};
+    a.x = p.rows_pts;
+    a.y = p.cols_pts;
+    a.w = static_cast<const float*>(p.w);
+    a.values = static_cast<TcValues>(p.vmode);
+    a.C = p.C;
+    a.CV = p.CV;
+    a.out = dst;
+    a.split_stride = S > 1 ? total : 0;
+    a.B = p.B;
+    a.M = p.R;
+    a.N = p.N;
+    a.D = p.D;
+    a.tau = p.tau;
+    a.plan = L.f32;
+    a.xpack = reinterpret_cast<float*>(ws + L.off_xpack);
+    a.rnorm = reinterpret_cast<float*>(ws + L.off_rnorm);
+    a.ypack = reinterpret_cast<float*>(ws + L.off_ypack);
+    a.qw = reinterpret_cast<float*>(ws + L.off_qw);
+    a.vt = reinterpret_cast<float*>(ws + L.off_vt);
+    GS_CUDA(launch_tc_f32_sum(a, s));
     if (S > 1) GS_CUDA(launch_combine_sum(dst, S, total, out, s));
     return GS_OK;
   }
@@ -268,7 +331,7 @@ VjpLayout vjp_layout(const void* x, const void* y, const void* w, const float* g
   // dL/dtau: on the CUDA-core path a pass whose kernel values carry the scaled
   // squared distance (no cancellation); on the tensor-core path the extra
   // value channel w |y - z|^2 of the grad_x pass
-  L.do_t = want_tau && dt == GS_F32;
+  L.do_t = want_tau && pass_path(dt, static_cast<int>(D)) == kPathSmallD;
   L.do_x = want_x || (want_tau && !L.do_t);
   L.px = fwd_pass(x, y, w, B, M, N, D, C, tau, dt);
   L.px.vmode = (want_tau && !L.do_t) ? 2 : 1;
@@ -421,7 +484,7 @@ size_t gs_workspace_bytes(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, 
   }
   if (op == GS_OP_KNN) {
     // C carries K for this op
-    if (dt != GS_F32 || C < 1 || C > kKnnMaxK || check_dims(GS_OP_SUM, B, M, N, D, 1, dt) != GS_OK)
+    if (dt != GS_F32 || C < 1 || C > kKnnMaxK || check_dims(GS_OP_KNN, B, M, N, D, 1, dt) != GS_OK)
       return kBad;
     if (B == 0 || M == 0 || N == 0) return 0;
     const KnnPlan kp = knn_plan(B, M, N, static_cast<int>(C), sm_count());
@@ -667,7 +730,7 @@ gs_status gauss_lse_bwd(const void* x, const void* y, const void* w, const float
 gs_status gauss_knn(const void* x, const void* y, float* out_sqdist, int64_t* out_index, int64_t B,
                     int64_t M, int64_t N, int64_t D, int64_t K, gs_dtype dt, void* ws,
                     size_t ws_bytes, gs_stream_t stream) {
-  GS_TRY(check_dims(GS_OP_SUM, B, M, N, D, 1, dt));
+  GS_TRY(check_dims(GS_OP_KNN, B, M, N, D, 1, dt));
   if (K < 1) return GS_ERR_INVALID_ARG;
   if (dt != GS_F32 || K > kKnnMaxK) return GS_ERR_UNSUPPORTED;
   GS_TRY(check_ptr(x, B * M * D));
@@ -762,9 +825,10 @@ gs_status gauss_diffusion_apply(const void* x, const float* s_scale, const float
 gs_status gs_last_device_error(gs_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return GS_ERR_CUDA;
-  int v = 0;
+  int v = 0, v32 = 0;
   if (read_and_clear_device_error(&v) != cudaSuccess) return GS_ERR_CUDA;
-  return v ? GS_ERR_TIMEOUT : GS_OK;
+  if (read_and_clear_device_error_f32(&v32) != cudaSuccess) return GS_ERR_CUDA;
+  return (v || v32) ? GS_ERR_TIMEOUT : GS_OK;
 }
 
 }  // extern "C"

@@ -3,6 +3,7 @@
 #pragma once
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/gauss.h"
@@ -125,15 +126,19 @@ cudaError_t launch_diffusion_elementwise(int op, const float* a, const float* b,
 cudaError_t launch_sum_rows(const float* v, int64_t n, float* out, cudaStream_t s);
 
 // ------------------------------------------------------------- tensor-core path
-constexpr int kTcMaxD = 126;
+constexpr int kTcMaxD = 128;
 constexpr int kTcMaxChunk = 128;   // channels per tensor-core pass
 
 struct TcPlan {
-  int KP;              // padded feature width of the packed operands (64 or 128)
+  int KP;              // padded feature width of the packed operands (64, 128 or 192)
   int splits;
   int64_t cols_per_split;   // multiple of 128
 };
 TcPlan tc_plan(int64_t B, int64_t M, int64_t N, int64_t D, int sm_count);
+// Channels per tensor-core pass for a packed width KP, and the padded value
+// chunk (16, 32, 48, 64, 96 or 128) a pass of cw channels is compiled for.
+int tc_max_chunk(int KP);
+int tc_chunk_pad(int cw);
 
 // Which values the tensor-core pass multiplies by the kernel (values.cuh modes).
 enum TcValues { kValuesW = 0, kValuesBwd = 1, kValuesBwdTau = 2 };
@@ -160,6 +165,47 @@ struct TcArgs {
   void* vt;            // [B, CP, Nst] f16
 };
 cudaError_t launch_tc_sum(const TcArgs& a, cudaStream_t s);
+
+// 3-D tiled TMA descriptor: dims {d0, d1, d2} (d0 innermost, in elements),
+// strides of dims 1 and 2 in bytes, box {box0, box1, 1}, 128-byte swizzle or none.
+bool make_tmap_3d(CUtensorMap* m, CUtensorMapDataType dt, void* base, uint64_t d0, uint64_t d1,
+                  uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0,
+                  uint32_t box1, bool swizzle128 = true);
+
+// ------------------------------------------------------------- fp32 tensor-core path
+// fp32 inputs with kSdMaxD < D <= kTcMaxD: split-tf32 MMAs (tc_f32_sm100.cu).
+struct F32Plan {
+  int Kp;              // D rounded up to 8: floats per half of a packed row [hi | lo]
+  int atoms;           // 128-byte atoms per packed row (2 Kp floats)
+  int max_chunk;       // channels per pass (64, or 32 for the widest rows)
+  int splits;
+  int64_t cols_per_split;   // multiple of 64
+};
+F32Plan f32_plan(int64_t B, int64_t M, int64_t N, int64_t D, int sm_count);
+int f32_chunk_pad(int cw);            // 16, 32 or 64
+int f32_tile_cols(int KA, int mode);  // columns per tile of an instantiation
+
+struct F32Args {
+  const void* x;       // rows side [B, M, D] float32
+  const void* y;       // column side [B, N, D] float32
+  const float* w;      // values source [B, N, C] float32
+  TcValues values;     // value mode (values.cuh), columns centred at x[b, 0]
+  int C, CV;
+  float* out;          // [S?][B][M][CV]
+  int64_t split_stride;
+  int64_t B, M, N;
+  int D;
+  float tau;
+  F32Plan plan;
+  // workspace pieces
+  float* xpack;        // [B, M, 2 Kp]
+  float* rnorm;        // [B, M]
+  float* ypack;        // [B, N, 2 Kp]
+  float* qw;           // [B, Nq, 4]: -c |y'|^2 (-inf past N) and up to 3 value channels
+  float* vt;           // [2 B, CP, Nst] (hi, lo), Nst = N rounded up to 4
+};
+cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s);
+cudaError_t read_and_clear_device_error_f32(int* value);
 
 // out[0 .. n) = value
 cudaError_t launch_fill(float* out, int64_t n, float value, cudaStream_t s);

@@ -216,6 +216,26 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
 
 // Arrive once on `bar` when every tcgen05 async op issued so far by this
 // thread has completed.
+// kind::tf32: 32-bit operands of which the tensor core reads the tf32 part
+// (sign, exponent, 10 mantissa bits); fp32 accumulator.
+__device__ __forceinline__ void mma_ss_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_tf32(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -279,14 +299,32 @@ __device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor, kind::f16 with fp32 accumulation, both operands
-// K-major.  fmt: 0 = f16, 1 = bf16.
+// Instruction descriptor with fp32 accumulation, both operands K-major.
+// fmt: 0 = f16, 1 = bf16 (kind::f16), 2 = tf32 (kind::tf32).
 __host__ __device__ constexpr uint32_t idesc_f16(uint32_t fmt_ab, uint32_t m, uint32_t n) {
   return (1u << 4)                 // accumulator format: f32
          | (fmt_ab << 7)           // A format
          | (fmt_ab << 10)          // B format
          | ((n >> 3) << 17)        // N / 8
          | ((m >> 4) << 24);       // M / 16
+}
+
+// Tie the registers of a TMEM load to the point after tcgen05.wait::ld, so
+// that no use of them is scheduled before the load has completed.
+__device__ __forceinline__ void reg_fence32(uint32_t (&v)[32]) {
+  asm volatile(""
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]), "+r"(v[16]), "+r"(v[17]),
+                 "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]), "+r"(v[22]), "+r"(v[23]),
+                 "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]), "+r"(v[29]),
+                 "+r"(v[30]), "+r"(v[31]));
+}
+__device__ __forceinline__ void reg_fence16(uint32_t (&v)[16]) {
+  asm volatile(""
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]));
 }
 
 }  // namespace gs

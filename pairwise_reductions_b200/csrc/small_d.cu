@@ -71,8 +71,16 @@ __device__ __forceinline__ float pow2i(float e) {
 // value by the scaled squared distance |x^ - y^|^2 = (tau/2 log2 e) |x - y|^2,
 // which gives the bandwidth gradient sum_j K w |x - y|^2 without cancellation;
 // 4 does both the per-row shift and the squared-distance factor.
+// Resident CTAs per SM asked of the register allocator.  Eight (at most 64
+// registers a thread) is worth 1-4 % on the single-channel D <= 3 kernels and
+// costs them no spill; the other instantiations keep the default, where the
+// same bound would spill.
+__host__ __device__ constexpr int sd_min_blocks(int D, int CP, int SHIFT) {
+  return (CP == 1 && D <= 3 && SHIFT != 1 && SHIFT != 4) ? 8 : 1;
+}
+
 template <int D, int CP, bool LSE, int SHIFT>
-__global__ void __launch_bounds__(kSdThreads)
+__global__ void __launch_bounds__(kSdThreads, sd_min_blocks(D, CP, SHIFT))
     sd_kernel(const SdArgs a) {
   constexpr int R = sd_rows_per_thread(D, CP);
   constexpr int RP = R / 2;                     // row pairs per thread

@@ -1,0 +1,723 @@
+// tc_f32_sm100.cu -- tensor-core Gaussian kernel sum for fp32 inputs with
+// 9 <= D <= 128 on sm_100a, at fp32 accuracy: split-tf32 products on tcgen05.
+//
+// Each fp32 operand v is split into v = hi + lo with hi = v rounded to tf32
+// (the 19 bits the kind::tf32 MMA reads) and lo = v - hi, itself rounded to
+// tf32.  A product a b is then taken as a_lo b_hi + a_hi b_lo + a_hi b_hi: the
+// dropped a_lo b_lo is ~2^-22 of a b, so three tf32 MMAs give close to fp32
+// products with fp32 accumulation.  This is the "memory-efficient" fp32 runs'
+// arithmetic of "Fast Gauss Sums via Flash Attention" (Figures 4 and 5), done
+// with B200's tensor cores: both products of the method -- the similarity
+// tile x.y^T and the value product P.v -- are split this way.
+//
+// The exponent.  With c = tau/2 * log2 e and the points centred at z = x[b, 0]
+// (x' = x - z, y' = y - z, which leaves every |x - y| unchanged and keeps the
+// norms small for clouds far from the origin),
+//     exp(-tau/2 |x_i - y_j|^2) = 2^(2c x'_i.y'_j + r_i + q_j),
+//     r_i = -c |x'_i|^2,  q_j = -c |y'_j|^2
+// (the norm factors of Algorithm 1 on the same page).  P_ij = ex2(fma(S, 2c, r_i) + q_j)
+// with S from the split MMAs; P is split into tf32 hi/lo again for P.v.
+//
+// CTA = one 128-row tile, 10 warps:
+//   warp 0      TMA producer: x' tile once, then a ring of (y' tile, v tile) stages
+//   warp 1      TMEM owner + single-thread MMA issuer
+//   warps 2-5   exp warpgroup 0: column tiles 0, 2, 4, ...
+//   warps 6-9   exp warpgroup 1: column tiles 1, 3, 5, ...
+// Both warpgroups hold the same rows (TMEM lanes), so each keeps its own
+// accumulator O_h and warpgroup 0 adds O_0 + O_1 at the end.  Per column tile
+// t of warpgroup h:
+//   S_h  = x'.y'(t)^T                 3 tf32 MMAs per K step (smem x smem -> TMEM)
+//   P_h  = ex2(fma(S_h, 2c, r) + q)   tcgen05.ld -> MUFU -> hi/lo -> tcgen05.st
+//   O_h += P_h . v(t)                 3 tf32 MMAs per K step (A = P from TMEM)
+// Every mbarrier wait is bounded (2 s); on expiry the kernel raises its device
+// error word, lets the other warps leave, frees TMEM and returns.
+#include <cuda.h>
+
+#include <cmath>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "values.cuh"
+
+namespace gs {
+
+__device__ int g_device_error_f32;
+
+namespace {
+
+constexpr int kBM = 128;        // rows per CTA (one MMA tile)
+constexpr int kThreads = 320;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kAtom = kBM * 128;   // one 128-row x 32-float (128-byte) swizzle atom
+
+struct F32KParams {
+  const float* rnorm;   // [B, M]
+  float* out;
+  int64_t split_stride;
+  int64_t M, N;
+  int64_t ldo;
+  int c0, cw;
+  int64_t cols_per_split;
+  int ksteps;           // K' / 8: tf32 K steps of the hi (and of the lo) half
+  int atoms;            // 128-byte atoms of a packed row actually loaded (<= KA)
+  int Bsz;              // batch count (the lo half of v sits at batch index B + b)
+  float two_c;
+};
+
+// KA: 128-byte atoms per packed row [hi K' | lo K'] the shared memory holds.
+// MODE 1 or 3: the values (at most MODE channels) ride with the column norms
+// and P.v is summed in registers (exact fp32 products); MODE 16, 32 or 64:
+// P.v on the tensor cores for a chunk of MODE channels.
+template <int KA, int MODE>
+struct F32Cfg {
+  static constexpr bool REG = MODE <= 3;
+  static constexpr int CP = REG ? 16 : MODE;
+  static constexpr int X_BYTES = KA * kAtom;
+  static constexpr int QW_BYTES = 1024;                 // up to 64 columns x 16 bytes
+  static constexpr int v_bytes(int bn) { return REG ? 0 : 2 * (bn / 32) * CP * 128; }
+  static constexpr int stage_bytes(int bn) { return KA * bn * 128 + QW_BYTES + v_bytes(bn); }
+  static constexpr int BUDGET = 214 * 1024;
+  // register path, one channel: 64-column tiles where two stages fit (three
+  // channels: 32, for registers); tensor-core P.v: 32-column tiles (TMEM holds
+  // S, P hi/lo and O for both warpgroups)
+  static constexpr int BN = (MODE == 1 && (BUDGET - X_BYTES) / stage_bytes(64) >= 2) ? 64 : 32;
+  static constexpr int Y_BYTES = KA * BN * 128;
+  static constexpr int V_ATOM = CP * 128;               // CP rows x 32 columns
+  static constexpr int V_BYTES = v_bytes(BN);
+  static constexpr int STAGE = stage_bytes(BN);
+  static constexpr int NST_FIT = (BUDGET - X_BYTES) / STAGE;
+  static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
+  static constexpr int NBARS = 2 * NST + 10;
+  static constexpr int RED_BYTES = kBM * 16;            // warpgroup 1 partial sums
+  static constexpr int SMEM_RAW = 1024 + X_BYTES + NST * STAGE + 8 * NBARS + 16 + RED_BYTES;
+  // at least ~120 KB: one CTA per SM, so the 512-column TMEM allocation never waits
+  static constexpr int SMEM = SMEM_RAW < 122880 ? 122880 : SMEM_RAW;
+  // TMEM columns: Sbig0 | Sbig1 | Ssmall0 | Ssmall1 [| Phi0 | Phi1 | Plo0 | Plo1 | O0 | O1]
+  static constexpr int CPA = (CP + 31) / 32 * 32;
+  __host__ __device__ static constexpr uint32_t col_sb(int h) { return BN * h; }
+  __host__ __device__ static constexpr uint32_t col_ss(int h) { return 2 * BN + BN * h; }
+  __host__ __device__ static constexpr uint32_t col_phi(int h) { return 4 * BN + BN * h; }
+  __host__ __device__ static constexpr uint32_t col_plo(int h) { return 6 * BN + BN * h; }
+  __host__ __device__ static constexpr uint32_t col_o(int h) { return 8 * BN + CPA * h; }
+  static_assert(NST >= 2, "shared memory budget");
+  static_assert(REG ? 4 * BN <= 512 : 8 * BN + 2 * CPA <= 512, "TMEM budget");
+  static_assert(REG || (CP % 16 == 0 && CP >= 16 && CP <= 64), "value chunk");
+  static_assert(SMEM_RAW <= 227 * 1024, "shared memory per CTA");
+};
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  uint32_t n = 0;
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((++n & 63u) == 0u) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        atomicOr(&g_device_error_f32, 1);
+        return false;
+      }
+    }
+  }
+}
+
+// v -> its tf32 part by truncation (the bits a kind::tf32 MMA reads); v - hi
+// is then exact in fp32.
+__device__ __forceinline__ float tf32_trunc(float v) {
+  return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
+}
+// Round to the nearest tf32 value, ties away from zero (finite inputs).
+__device__ __forceinline__ float tf32_round(float v) {
+  return __uint_as_float((__float_as_uint(v) + 0x1000u) & 0xFFFFE000u);
+}
+
+// Named barrier of the two exp warpgroups (warps 2-9).
+__device__ __forceinline__ void exp_warps_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+template <int KA, int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_f32_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+                  const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmV,
+                  const F32KParams p) {
+  using Cfg = F32Cfg<KA, MODE>;
+  constexpr bool REG = Cfg::REG;
+  constexpr int CP = Cfg::CP;
+  constexpr int NST = Cfg::NST;
+  constexpr int BN = Cfg::BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sX = smem;
+  uint8_t* sStage = smem + Cfg::X_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + NST * Cfg::STAGE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NBARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float4* red = reinterpret_cast<float4*>(tmem_slot + 4);   // 16-byte aligned
+
+  const uint32_t bar0 = smem_u32(bars);
+  auto bar_full = [&](int s) { return bar0 + 8u * s; };
+  auto bar_empty = [&](int s) { return bar0 + 8u * (NST + s); };
+  const uint32_t bar_x = bar0 + 8u * (2 * NST);
+  auto bar_s = [&](int h) { return bar0 + 8u * (2 * NST + 1 + h); };   // S_h ready
+  auto bar_p = [&](int h) { return bar0 + 8u * (2 * NST + 3 + h); };   // P_h written
+  auto bar_f = [&](int h) { return bar0 + 8u * (2 * NST + 5 + h); };   // S_h read out
+  auto bar_q = [&](int h) { return bar0 + 8u * (2 * NST + 7 + h); };   // P_h consumed
+  const uint32_t bar_o = bar0 + 8u * (2 * NST + 9);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t b = blockIdx.z;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kBM;
+  const int64_t jbeg = static_cast<int64_t>(blockIdx.y) * p.cols_per_split;
+  const int64_t jend = min(p.N, jbeg + p.cols_per_split);
+  const int T = (jend > jbeg) ? static_cast<int>((jend - jbeg + BN - 1) / BN) : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bar_full(s), 1);
+      // a stage is released by the P.v MMAs (tensor-core values) or by the
+      // 128 exp threads that read its norms and values (register values)
+      mbar_init(bar_empty(s), REG ? 4 * 32 : 1);
+    }
+    mbar_init(bar_x, 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(bar_s(h), 1);
+      mbar_init(bar_p(h), 4 * 32);
+      mbar_init(bar_f(h), 4 * 32);
+      mbar_init(bar_q(h), 1);
+    }
+    mbar_init(bar_o, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmX);
+      tma_prefetch_desc(&tmY);
+      tma_prefetch_desc(&tmQ);
+      if constexpr (!REG) tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(bar_x, p.atoms * kAtom);
+      for (int a = 0; a < p.atoms; ++a)
+        tma_load_3d(smem_u32(sX + a * kAtom), &tmX, bar_x, a * 32, static_cast<int>(row0),
+                    static_cast<int>(b));
+      const uint32_t stage_tx = p.atoms * BN * 128 + BN * 16 + Cfg::V_BYTES;
+      for (int t = 0; t < T; ++t) {
+        const int st = t % NST;
+        if (t >= NST && !wait_bar(bar_empty(st), ((t / NST) - 1) & 1, abort_flag)) break;
+        uint8_t* sy = sStage + st * Cfg::STAGE;
+        uint8_t* sq = sy + Cfg::Y_BYTES;
+        uint8_t* sv = sq + Cfg::QW_BYTES;
+        const int j0 = static_cast<int>(jbeg + static_cast<int64_t>(t) * BN);
+        mbar_arrive_expect_tx(bar_full(st), stage_tx);
+        for (int a = 0; a < p.atoms; ++a)
+          tma_load_3d(smem_u32(sy + a * BN * 128), &tmY, bar_full(st), a * 32, j0,
+                      static_cast<int>(b));
+        tma_load_3d(smem_u32(sq), &tmQ, bar_full(st), 0, j0, static_cast<int>(b));
+        if constexpr (!REG) {
+          for (int hl = 0; hl < 2; ++hl)
+            for (int a = 0; a < BN / 32; ++a)
+              tma_load_3d(smem_u32(sv + (hl * (BN / 32) + a) * Cfg::V_ATOM), &tmV, bar_full(st),
+                          j0 + a * 32, 0, static_cast<int>(hl * p.Bsz + b));
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idS = idesc_f16(2, kBM, BN);
+      const uint32_t idO = idesc_f16(2, kBM, CP);
+      const int ks_lo = p.ksteps;
+      // K step ks (8 floats = 32 bytes) of a packed row block whose atoms are
+      // atom_bytes apart
+      auto kdesc = [](const uint8_t* base, int atom_bytes, int ks) {
+        const int off = ks * 32;
+        return desc_k_sw128(smem_u32(base + (off >> 7) * atom_bytes) + (off & 127));
+      };
+      // S = x'.y'^T: the two small products accumulate apart from the large
+      // one, so that each of them is rounded against its own magnitude
+      auto issue_S = [&](int h, int st) {
+        const uint8_t* sy = sStage + st * Cfg::STAGE;
+        const uint32_t db = tmem + Cfg::col_sb(h), ds = tmem + Cfg::col_ss(h);
+        for (int ks = 0; ks < p.ksteps; ++ks) {
+          const uint64_t ah = kdesc(sX, kAtom, ks), al = kdesc(sX, kAtom, ks + ks_lo);
+          const uint64_t bh = kdesc(sy, BN * 128, ks), bl = kdesc(sy, BN * 128, ks + ks_lo);
+          mma_ss_tf32(ds, al, bh, idS, ks > 0 ? 1u : 0u);
+          mma_ss_tf32(ds, ah, bl, idS, 1u);
+          mma_ss_tf32(db, ah, bh, idS, ks > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_O = [&](int h, int st, bool acc_prev) {
+        const uint8_t* sv = sStage + st * Cfg::STAGE + Cfg::Y_BYTES + Cfg::QW_BYTES;
+        const uint32_t d = tmem + Cfg::col_o(h);
+#pragma unroll
+        for (int ks = 0; ks < BN / 8; ++ks) {
+          const int a = ks >> 2, within = (ks & 3) * 32;
+          const uint64_t bh = desc_k_sw128(smem_u32(sv + a * Cfg::V_ATOM) + within);
+          const uint64_t bl = desc_k_sw128(smem_u32(sv + ((BN / 32) + a) * Cfg::V_ATOM) + within);
+          const uint32_t phi = tmem + Cfg::col_phi(h) + ks * 8;
+          const uint32_t plo = tmem + Cfg::col_plo(h) + ks * 8;
+          mma_ts_tf32(d, plo, bh, idO, (acc_prev || ks > 0) ? 1u : 0u);
+          mma_ts_tf32(d, phi, bl, idO, 1u);
+          mma_ts_tf32(d, phi, bh, idO, 1u);
+        }
+      };
+      bool ok = wait_bar(bar_x, 0, abort_flag);
+      for (int h = 0; ok && h < 2 && h < T; ++h) {
+        ok = wait_bar(bar_full(h), 0, abort_flag);
+        if (ok) {
+          tc_fence_after();
+          issue_S(h, h);
+          mma_commit(bar_s(h));
+        }
+      }
+      // S_h(t + 2) may overwrite S_h once warpgroup h has read S_h(t).  With
+      // tensor-core values it goes ahead of O_h(t) when tile t + 2 does not
+      // need the stage of tile t (three or more stages), else after it.
+      constexpr bool kSFirst = REG || NST >= 3;
+      auto next_S = [&](int h, int k, int t2) {
+        if (!wait_bar(bar_f(h), k & 1, abort_flag)) return false;
+        if (!wait_bar(bar_full(t2 % NST), (t2 / NST) & 1, abort_flag)) return false;
+        tc_fence_after();
+        issue_S(h, t2 % NST);
+        mma_commit(bar_s(h));
+        return true;
+      };
+      for (int k = 0; ok && 2 * k < T; ++k) {
+        for (int h = 0; h < 2; ++h) {
+          const int t = 2 * k + h;
+          if (t >= T) break;
+          const int t2 = t + 2;
+          if (kSFirst && t2 < T && !(ok = next_S(h, k, t2))) break;
+          if constexpr (!REG) {
+            if (!(ok = wait_bar(bar_p(h), k & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_O(h, t % NST, k > 0);
+            mma_commit(bar_q(h));
+            mma_commit(bar_empty(t % NST));
+            if (!kSFirst && t2 < T && !(ok = next_S(h, k, t2))) break;
+          }
+        }
+      }
+      mma_commit(bar_o);   // also the drain point for whatever was issued
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ exp warpgroups
+    const int h = (warp - 2) >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int64_t i = row0 + row;
+    const bool valid = i < p.M;
+    const float r = valid ? p.rnorm[b * p.M + i] : 0.f;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tSb = tmem + lane_base + Cfg::col_sb(h);
+    const uint32_t tSs = tmem + lane_base + Cfg::col_ss(h);
+    const uint32_t tPh = tmem + lane_base + Cfg::col_phi(h);
+    const uint32_t tPl = tmem + lane_base + Cfg::col_plo(h);
+    const float two_c = p.two_c;
+    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f;   // register values: running row sums
+    bool ok = true;
+    int k = 0;
+    for (int t = h; t < T; t += 2, ++k) {
+      const int st = t % NST;
+      ok = wait_bar(bar_s(h), k & 1, abort_flag) &&
+           wait_bar(bar_full(st), (t / NST) & 1, abort_flag);   // norms and values landed
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // S = Sbig + Ssmall, the whole tile into registers; then its TMEM
+      // columns may be reused
+      uint32_t sv[BN / 32][32];
+#pragma unroll
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        uint32_t ss[32];
+        tmem_ld32(tSb + ch * 32, sv[ch]);
+        tmem_ld32(tSs + ch * 32, ss);
+        tmem_wait_ld();
+        reg_fence32(sv[ch]);
+        reg_fence32(ss);
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          sv[ch][e] = __float_as_uint(__uint_as_float(sv[ch][e]) + __uint_as_float(ss[e]));
+      }
+      tc_fence_before();
+      mbar_arrive(bar_f(h));
+      const float4* qw = reinterpret_cast<const float4*>(sStage + st * Cfg::STAGE + Cfg::Y_BYTES);
+      if constexpr (REG) {
+        // P.v in registers, a partial sum per tile (two-level accumulation)
+        float p0 = 0.f, p1 = 0.f, p2 = 0.f;
+#pragma unroll
+        for (int ch = 0; ch < BN / 32; ++ch) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float4 q = qw[ch * 32 + e];
+            const float pe = ex2(fmaf(__uint_as_float(sv[ch][e]), two_c, r) + q.x);
+            p0 = fmaf(pe, q.y, p0);
+            if constexpr (MODE > 1) {
+              p1 = fmaf(pe, q.z, p1);
+              p2 = fmaf(pe, q.w, p2);
+            }
+          }
+        }
+        acc0 += p0;
+        acc1 += p1;
+        acc2 += p2;
+        mbar_arrive(bar_empty(st));
+      } else {
+#pragma unroll
+        for (int ch = 0; ch < BN / 32; ++ch) {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t hi[16], lo[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int c = half * 16 + e;
+              const float pe = ex2(fmaf(__uint_as_float(sv[ch][c]), two_c, r) + qw[ch * 32 + c].x);
+              const float ph = tf32_trunc(pe);
+              hi[e] = __float_as_uint(ph);
+              lo[e] = __float_as_uint(pe - ph);
+            }
+            if (ch == 0 && half == 0 && k > 0) {
+              // P_h(previous tile) must have been read by its P.v MMAs
+              // (waited for as late as possible)
+              ok = __all_sync(0xffffffffu, wait_bar(bar_q(h), (k - 1) & 1, abort_flag));
+              if (!ok) break;
+              tc_fence_after();
+            }
+            tmem_st16(tPh + ch * 32 + half * 16, hi);
+            tmem_st16(tPl + ch * 32 + half * 16, lo);
+          }
+          if (!ok) break;
+        }
+        if (!ok) break;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_p(h));
+      }
+    }
+    if constexpr (REG) {
+      // warpgroup 1 hands its row sums to warpgroup 0 (both reach this barrier)
+      if (h == 1) red[row] = make_float4(acc0, acc1, acc2, 0.f);
+      exp_warps_sync();
+      if (h == 0 && valid && ok && !*abort_flag) {
+        const float4 o = red[row];
+        float* orow = p.out + static_cast<int64_t>(blockIdx.y) * p.split_stride +
+                      (b * p.M + i) * p.ldo + p.c0;
+        orow[0] = acc0 + o.x;
+        if (p.cw > 1) orow[1] = acc1 + o.y;
+        if (p.cw > 2) orow[2] = acc2 + o.z;
+      }
+    } else {
+      if (ok) ok = wait_bar(bar_o, 0, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+      if (ok && h == 0) {
+        const uint32_t tO0 = tmem + lane_base + Cfg::col_o(0);
+        const uint32_t tO1 = tmem + lane_base + Cfg::col_o(1);
+        float* orow = p.out + static_cast<int64_t>(blockIdx.y) * p.split_stride +
+                      (b * p.M + i) * p.ldo + p.c0;
+#pragma unroll
+        for (int ch = 0; ch < CP / 16; ++ch) {
+          uint32_t v0[16], v1[16];
+          tmem_ld16(tO0 + ch * 16, v0);
+          tmem_ld16(tO1 + ch * 16, v1);
+          tmem_wait_ld();
+          reg_fence16(v0);
+          reg_fence16(v1);
+          if (valid) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const int c = ch * 16 + q;
+              float o = 0.f;
+              if (T > 0) o = __uint_as_float(v0[q]);
+              if (T > 1) o += __uint_as_float(v1[q]);   // O_1 holds tiles only when T > 1
+              if (c < p.cw) orow[c] = o;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ packing prologue
+// Packed operand rows [hi (K') | lo (K')] of the centred points v' = v - z,
+// z = rows[b, 0, :], and the norm term -c |v'|^2: for the row side into
+// norm[b * R + r]; for the column side into norm[(b * Rpad + r) * 4] (lanes
+// 1-3 zeroed) with -inf for the padding columns r >= R.  One thread per row.
+__global__ void pack_rows_f32_kernel(const float* __restrict__ src, const float* __restrict__ rows,
+                                     float* __restrict__ dst, float* __restrict__ norm, int64_t B,
+                                     int64_t R, int64_t Rpad, int64_t Mrows, int D, int Kp,
+                                     float c, int norm_stride) {
+  const int64_t total = B * Rpad;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = e / Rpad, rr = e % Rpad;
+    float* nrm = norm + e * norm_stride;
+    if (norm_stride == 4) nrm[1] = nrm[2] = nrm[3] = 0.f;
+    if (rr >= R) {
+      nrm[0] = -INFINITY;   // padding columns: kernel value 0
+      continue;
+    }
+    const float* v = src + (b * R + rr) * D;
+    const float* z = rows + b * Mrows * D;
+    float* out = dst + (b * R + rr) * (2 * static_cast<int64_t>(Kp));
+    float sq = 0.f;
+    for (int k = 0; k < Kp; ++k) {
+      float d = 0.f;
+      if (k < D) d = v[k] - z[k];
+      sq = fmaf(d, d, sq);
+      const float hi = tf32_round(d);
+      out[k] = hi;
+      out[Kp + k] = tf32_round(d - hi);
+    }
+    nrm[0] = -c * sq;
+  }
+}
+
+// Register-path values: channels [0, CV) (CV <= 3) of the pass's values
+// (values.cuh) into lanes 1.. of qw[b, j, :].
+__global__ void pack_values_qw_kernel(const float* __restrict__ w, const float* __restrict__ y,
+                                      const float* __restrict__ rows, float* __restrict__ qw,
+                                      int64_t B, int64_t N, int64_t Nq, int64_t Mrows, int C, int D,
+                                      int CV) {
+  const int64_t total = B * N;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = e / N, j = e % N;
+    for (int ch = 0; ch < CV; ++ch)
+      qw[(b * Nq + j) * 4 + 1 + ch] = value_at(w, y, rows, b, e, Mrows, D, C, ch, C);
+  }
+}
+
+// Split fp32 value matrix v^T: hi at [b][CP][Nst], lo at [B + b][CP][Nst], for
+// channels [c0, c0 + CP) of the pass's values (values.cuh); zeros past CV.
+__global__ void pack_values_f32_split_kernel(const float* __restrict__ w,
+                                             const float* __restrict__ y,
+                                             const float* __restrict__ rows,
+                                             float* __restrict__ vt, int64_t B, int64_t N,
+                                             int64_t Nst, int64_t Mrows, int C, int D, int CV,
+                                             int c0, int CP) {
+  const int64_t total = B * CP * N;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t j = e % N;
+    const int64_t bc = e / N;
+    const int cc = static_cast<int>(bc % CP);
+    const int64_t b = bc / CP;
+    const int ch = c0 + cc;
+    const float v = (ch < CV) ? value_at(w, y, rows, b, b * N + j, Mrows, D, C, ch, C) : 0.f;
+    const float hi = tf32_round(v);
+    vt[(b * CP + cc) * Nst + j] = hi;
+    vt[((B + b) * CP + cc) * Nst + j] = tf32_round(v - hi);
+  }
+}
+
+int grid_for(int64_t n, int threads) {
+  int64_t b = (n + threads - 1) / threads;
+  if (b < 1) b = 1;
+  if (b > 148 * 32) b = 148 * 32;
+  return static_cast<int>(b);
+}
+
+struct TileMaps {
+  CUtensorMap x, y, q, v;
+};
+
+template <int KA, int MODE>
+cudaError_t launch_kernel(const TileMaps& m, const F32KParams& kp, dim3 grid, cudaStream_t s) {
+  using Cfg = F32Cfg<KA, MODE>;
+  auto fn = tc_f32_kernel<KA, MODE>;
+  static bool attr_done = false;   // idempotent; a benign race at worst repeats the call
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  fn<<<grid, kThreads, Cfg::SMEM, s>>>(m.x, m.y, m.q, m.v, kp);
+  return cudaGetLastError();
+}
+
+template <int KA>
+cudaError_t launch_mode(int mode, const TileMaps& m, const F32KParams& kp, dim3 grid,
+                        cudaStream_t s) {
+  switch (mode) {
+    case 1: return launch_kernel<KA, 1>(m, kp, grid, s);
+    case 3: return launch_kernel<KA, 3>(m, kp, grid, s);
+    case 16: return launch_kernel<KA, 16>(m, kp, grid, s);
+    case 32: return launch_kernel<KA, 32>(m, kp, grid, s);
+    default:
+      if constexpr (KA < 8) return launch_kernel<KA, 64>(m, kp, grid, s);
+      return cudaErrorInvalidValue;
+  }
+}
+
+// Shared-memory atoms the kernel is compiled for, covering `atoms`.
+int ka_for(int atoms) { return atoms <= 1 ? 1 : (atoms <= 2 ? 2 : (atoms <= 4 ? 4 : (atoms <= 6 ? 6 : 8))); }
+
+template <int KA>
+int tile_cols_ka(int mode) {
+  switch (mode) {
+    case 1: return F32Cfg<KA, 1>::BN;
+    case 3: return F32Cfg<KA, 3>::BN;
+    default: return F32Cfg<KA, 16>::BN;   // every tensor-core value chunk: 32
+  }
+}
+
+// Register values for at most 3 channels, else tensor-core chunks.
+int mode_for(int CV, int cw) { return CV <= 3 ? (CV == 1 ? 1 : 3) : f32_chunk_pad(cw); }
+
+}  // namespace
+
+F32Plan f32_plan(int64_t B, int64_t M, int64_t N, int64_t D, int sm_count) {
+  F32Plan p{};
+  p.Kp = static_cast<int>((D + 7) / 8 * 8);
+  p.atoms = (2 * p.Kp + 31) / 32;
+  p.max_chunk = ka_for(p.atoms) >= 8 ? 32 : 64;
+  // a split is a whole number of 64-column blocks (either tile width divides it)
+  const int64_t U = B * ((M + kBM - 1) / kBM);
+  const int64_t ntj = (N + 63) / 64;
+  int64_t smax = ntj / 4;
+  if (smax > 32) smax = 32;
+  if (smax < 1) smax = 1;
+  int best = 1;
+  double best_cost = 1e300;
+  for (int64_t S = 1; S <= smax; ++S) {
+    const int64_t waves = (U * S + sm_count - 1) / sm_count;
+    const double cost = static_cast<double>(waves) * static_cast<double>((ntj + S - 1) / S + 3);
+    if (cost < best_cost * 0.999) {
+      best_cost = cost;
+      best = static_cast<int>(S);
+    }
+  }
+  const int64_t per = (ntj + best - 1) / best;
+  p.cols_per_split = (per < 1 ? 1 : per) * 64;
+  p.splits = static_cast<int>((N + p.cols_per_split - 1) / p.cols_per_split);
+  if (p.splits < 1) p.splits = 1;
+  return p;
+}
+
+int f32_chunk_pad(int cw) { return cw <= 16 ? 16 : (cw <= 32 ? 32 : 64); }
+
+int f32_tile_cols(int KA, int mode) {
+  switch (KA) {
+    case 1: return tile_cols_ka<1>(mode);
+    case 2: return tile_cols_ka<2>(mode);
+    case 4: return tile_cols_ka<4>(mode);
+    case 6: return tile_cols_ka<6>(mode);
+    default: return tile_cols_ka<8>(mode);
+  }
+}
+
+cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
+  if (a.B == 0 || a.M == 0) return cudaSuccess;
+  const int Kp = a.plan.Kp;
+  const float c = 0.5f * a.tau * kLog2e;
+  const int64_t Nq = (a.N + 63) / 64 * 64;
+  const float* x = static_cast<const float*>(a.x);
+  const float* y = static_cast<const float*>(a.y);
+  pack_rows_f32_kernel<<<grid_for(a.B * a.M, 128), 128, 0, s>>>(x, x, a.xpack, a.rnorm, a.B, a.M,
+                                                               a.M, a.M, a.D, Kp, c, 1);
+  pack_rows_f32_kernel<<<grid_for(a.B * Nq, 128), 128, 0, s>>>(y, x, a.ypack, a.qw, a.B, a.N, Nq,
+                                                              a.M, a.D, Kp, c, 4);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const bool reg = a.CV <= 3;
+  if (reg) {
+    pack_values_qw_kernel<<<grid_for(a.B * a.N, 256), 256, 0, s>>>(a.w, y, x, a.qw, a.B, a.N, Nq,
+                                                                   a.M, a.C, a.D, a.CV);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  TileMaps m;
+  const uint64_t rowf = 2ull * Kp;
+  if (!make_tmap_3d(&m.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.xpack, rowf, a.M, a.B, rowf * 4,
+                    a.M * rowf * 4, 32, kBM))
+    return cudaErrorInvalidValue;
+  const int KA = ka_for(a.plan.atoms);
+  const int64_t Nst = (a.N + 3) / 4 * 4;
+  const dim3 grid(static_cast<unsigned>((a.M + kBM - 1) / kBM), static_cast<unsigned>(a.plan.splits),
+                  static_cast<unsigned>(a.B));
+  const int chunk = reg ? a.CV : a.plan.max_chunk;
+  for (int c0 = 0; c0 < a.CV; c0 += chunk) {
+    const int cw = (a.CV - c0) < chunk ? (a.CV - c0) : chunk;
+    const int mode = mode_for(a.CV, cw);
+    const int BN = f32_tile_cols(KA, mode);
+    if (!make_tmap_3d(&m.y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.ypack, rowf, a.N, a.B, rowf * 4,
+                      a.N * rowf * 4, 32, BN) ||
+        !make_tmap_3d(&m.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.qw, 4, Nq, a.B, 16, Nq * 16ull, 4,
+                      BN, false))
+      return cudaErrorInvalidValue;
+    if (reg) {
+      m.v = m.q;   // unused
+    } else {
+      const int CP = mode;
+      const int64_t total = a.B * CP * a.N;
+      pack_values_f32_split_kernel<<<grid_for(total, 256), 256, 0, s>>>(
+          a.w, y, x, a.vt, a.B, a.N, Nst, a.M, a.C, a.D, a.CV, c0, CP);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+      if (!make_tmap_3d(&m.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.vt, a.N, CP, 2 * a.B, Nst * 4ull,
+                        CP * Nst * 4ull, 32, CP))
+        return cudaErrorInvalidValue;
+    }
+    F32KParams kp{};
+    kp.rnorm = a.rnorm;
+    kp.out = a.out;
+    kp.split_stride = a.split_stride;
+    kp.M = a.M;
+    kp.N = a.N;
+    kp.ldo = a.CV;
+    kp.c0 = c0;
+    kp.cw = cw;
+    kp.cols_per_split = a.plan.cols_per_split;
+    kp.ksteps = Kp / 8;
+    kp.atoms = a.plan.atoms;
+    kp.Bsz = static_cast<int>(a.B);
+    kp.two_c = a.tau * kLog2e;
+    switch (KA) {
+      case 1: e = launch_mode<1>(mode, m, kp, grid, s); break;
+      case 2: e = launch_mode<2>(mode, m, kp, grid, s); break;
+      case 4: e = launch_mode<4>(mode, m, kp, grid, s); break;
+      case 6: e = launch_mode<6>(mode, m, kp, grid, s); break;
+      default: e = launch_mode<8>(mode, m, kp, grid, s); break;
+    }
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t read_and_clear_device_error_f32(int* value) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_error_f32, sizeof(int));
+  if (e != cudaSuccess) return e;
+  *value = v;
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error_f32, &zero, sizeof(int));
+  }
+  return e;
+}
+
+}  // namespace gs

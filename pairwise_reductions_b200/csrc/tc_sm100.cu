@@ -1,5 +1,5 @@
 // tc_sm100.cu -- tensor-core Gaussian kernel sum for fp16 / bf16 inputs
-// (1 <= D <= 126) on sm_100a: tcgen05 MMAs with TMEM accumulators, operands
+// (1 <= D <= 128) on sm_100a: tcgen05 MMAs with TMEM accumulators, operands
 // staged by TMA, nothing of size M x N ever leaves the SM.
 //
 // The fold.  With c = tau/2 * log2 e,
@@ -71,7 +71,9 @@ struct TcCfg {
   static constexpr int Y_BYTES = KC * ATOM;
   static constexpr int V_BYTES = 2 * CP * 128;  // two 64-column atoms of CP rows
   static constexpr int STAGE = Y_BYTES + V_BYTES;
-  static constexpr int NST_FIT = (200 * 1024 - X_BYTES) / STAGE;
+  // 200 KB of operand stages; the three-atom rows (D > 126) may take 220 KB
+  static constexpr int BUDGET = (KC > 2 ? 220 : 200) * 1024;
+  static constexpr int NST_FIT = (BUDGET - X_BYTES) / STAGE;
   static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
   static constexpr int NBARS = 2 * NST + 11;
   static constexpr int SMEM_RAW = 1024 + X_BYTES + NST * STAGE + 8 * NBARS + 16;
@@ -116,24 +118,6 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
 // are partly latency-bound and the polynomial's longer dependency chain costs
 // more than the MUFU slots it frees.  Kept as a tuning knob.
 constexpr int kPolyPairs = 0;
-
-// Tie the registers of a TMEM load to the point after tcgen05.wait::ld, so
-// that no use of them is scheduled before the load has completed.
-__device__ __forceinline__ void reg_fence32(uint32_t (&v)[32]) {
-  asm volatile(""
-               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
-                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
-                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]), "+r"(v[16]), "+r"(v[17]),
-                 "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]), "+r"(v[22]), "+r"(v[23]),
-                 "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]), "+r"(v[29]),
-                 "+r"(v[30]), "+r"(v[31]));
-}
-__device__ __forceinline__ void reg_fence16(uint32_t (&v)[16]) {
-  asm volatile(""
-               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
-                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
-                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]));
-}
 
 // 32 S values of one row -> 16 packed fp16 pairs of P = 2^(2c S + r).
 __device__ __forceinline__ void exp_chunk(const uint32_t (&v)[32], uint64_t two_c2, uint64_t r2,
@@ -449,26 +433,30 @@ __device__ __forceinline__ uint16_t bits16(__nv_bfloat16 v) { return __bfloat16_
 
 // Packed operand rows.  Row side (is_x): [x, 1, 1, 0 ...] and
 // rnorm = -c |x|^2 + shift.  Column side: [y, h, l, 0 ...] with h + l = -|y|^2/2.
-// A group of KP/8 consecutive threads builds one row, 8 elements (16 bytes) each.
+// A group of 8 consecutive threads builds one row, KP/8 elements each, written
+// as 8-element (16-byte) pieces: thread `part` owns pieces part, part + 8, ...
 template <typename T, int KP>
 __global__ void pack_rows_kernel(const T* __restrict__ src, T* __restrict__ dst,
                                  float* __restrict__ rnorm, int64_t rows, int D, float c,
                                  float shift, int is_x) {
-  constexpr int G = KP / 8;   // threads per row (8 or 16), a power of two dividing 32
+  constexpr int G = 8;          // threads per row
+  constexpr int NPC = KP / 64;  // pieces per thread (1, 2 or 3)
   const int64_t gt = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   const int64_t row = gt / G;
   const int part = static_cast<int>(gt % G);
   const bool live = row < rows;
-  float vals[8];
+  float vals[NPC][8];
   float sq = 0.f;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const int k = part * 8 + e;
-    float v = 0.f;
-    if (live && k < D) v = tof(src[row * D + k]);
-    vals[e] = v;
-    sq = fmaf(v, v, sq);
-  }
+  for (int pc = 0; pc < NPC; ++pc)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int k = (part + pc * G) * 8 + e;
+      float v = 0.f;
+      if (live && k < D) v = tof(src[row * D + k]);
+      vals[pc][e] = v;
+      sq = fmaf(v, v, sq);
+    }
 #pragma unroll
   for (int o = G / 2; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o, G);
   if (!live) return;
@@ -481,20 +469,23 @@ __global__ void pack_rows_kernel(const T* __restrict__ src, T* __restrict__ dst,
     aug0 = tof(fromf<T>(hn));
     aug1 = hn - aug0;
   }
-  uint32_t packed[4];
 #pragma unroll
-  for (int e = 0; e < 8; e += 2) {
-    float v0 = vals[e], v1 = vals[e + 1];
-    const int k = part * 8 + e;
-    if (k == D) v0 = aug0;
-    if (k == D + 1) v0 = aug1;
-    if (k + 1 == D) v1 = aug0;
-    if (k + 1 == D + 1) v1 = aug1;
-    packed[e / 2] = static_cast<uint32_t>(bits16(fromf<T>(v0))) |
-                    (static_cast<uint32_t>(bits16(fromf<T>(v1))) << 16);
+  for (int pc = 0; pc < NPC; ++pc) {
+    uint32_t packed[4];
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      float v0 = vals[pc][e], v1 = vals[pc][e + 1];
+      const int k = (part + pc * G) * 8 + e;
+      if (k == D) v0 = aug0;
+      if (k == D + 1) v0 = aug1;
+      if (k + 1 == D) v1 = aug0;
+      if (k + 1 == D + 1) v1 = aug1;
+      packed[e / 2] = static_cast<uint32_t>(bits16(fromf<T>(v0))) |
+                      (static_cast<uint32_t>(bits16(fromf<T>(v1))) << 16);
+    }
+    *reinterpret_cast<uint4*>(dst + row * KP + (part + pc * G) * 8) =
+        make_uint4(packed[0], packed[1], packed[2], packed[3]);
   }
-  *reinterpret_cast<uint4*>(dst + row * KP + part * 8) =
-      make_uint4(packed[0], packed[1], packed[2], packed[3]);
   if (is_x && part == 0) rnorm[row] = fmaf(-c, sq, shift);
 }
 
@@ -520,39 +511,6 @@ __global__ void pack_values_kernel(const TW* __restrict__ w, const TY* __restric
 }
 
 // ------------------------------------------------------------------ host side
-using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeFn get_encode() {
-  static EncodeFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeFn>(ptr);
-  });
-  return fn;
-}
-
-bool make_tmap_3d(CUtensorMap* m, CUtensorMapDataType dt, void* base, uint64_t d0, uint64_t d1,
-                  uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0,
-                  uint32_t box1) {
-  EncodeFn enc = get_encode();
-  if (!enc) return false;
-  const cuuint64_t dims[3] = {d0, d1, d2};
-  const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
-  const cuuint32_t box[3] = {box0, box1, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, dt, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 int grid_for(int64_t n, int threads) {
   int64_t b = (n + threads - 1) / threads;
   if (b < 1) b = 1;
@@ -565,16 +523,16 @@ cudaError_t pack_operands(const TcArgs& a, cudaStream_t s) {
   const float c = 0.5f * a.tau * kLog2e;
   const int KP = a.plan.KP;
   auto launch_rows = [&](const void* src, void* dst, float* rn, int64_t rows, int is_x) {
-    const int64_t threads_total = rows * (KP / 8);
+    const int64_t threads_total = rows * 8;
     const int blocks = static_cast<int>((threads_total + 255) / 256);
+    const T* sp = static_cast<const T*>(src);
+    T* dp = static_cast<T*>(dst);
     if (KP == 64)
-      pack_rows_kernel<T, 64><<<blocks, 256, 0, s>>>(static_cast<const T*>(src),
-                                                     static_cast<T*>(dst), rn, rows, a.D, c,
-                                                     kPShift, is_x);
+      pack_rows_kernel<T, 64><<<blocks, 256, 0, s>>>(sp, dp, rn, rows, a.D, c, kPShift, is_x);
+    else if (KP == 128)
+      pack_rows_kernel<T, 128><<<blocks, 256, 0, s>>>(sp, dp, rn, rows, a.D, c, kPShift, is_x);
     else
-      pack_rows_kernel<T, 128><<<blocks, 256, 0, s>>>(static_cast<const T*>(src),
-                                                      static_cast<T*>(dst), rn, rows, a.D, c,
-                                                      kPShift, is_x);
+      pack_rows_kernel<T, 192><<<blocks, 256, 0, s>>>(sp, dp, rn, rows, a.D, c, kPShift, is_x);
   };
   launch_rows(a.x, a.xpack, a.rnorm, a.B * a.M, 1);
   launch_rows(a.y, a.ypack, nullptr, a.B * a.N, 0);
@@ -616,27 +574,72 @@ cudaError_t launch_kernel(const CUtensorMap& tx, const CUtensorMap& ty, const CU
 template <int KP, int DTFMT>
 cudaError_t launch_cp(int CP, const CUtensorMap& tx, const CUtensorMap& ty, const CUtensorMap& tv,
                       const TcKParams& kp, dim3 grid, cudaStream_t s) {
-  switch (CP) {
-    case 16: return launch_kernel<KP, 16, DTFMT>(tx, ty, tv, kp, grid, s);
-    case 32: return launch_kernel<KP, 32, DTFMT>(tx, ty, tv, kp, grid, s);
-    case 48: return launch_kernel<KP, 48, DTFMT>(tx, ty, tv, kp, grid, s);
-    case 64: return launch_kernel<KP, 64, DTFMT>(tx, ty, tv, kp, grid, s);
-    case 96: return launch_kernel<KP, 96, DTFMT>(tx, ty, tv, kp, grid, s);
-    default: return launch_kernel<KP, 128, DTFMT>(tx, ty, tv, kp, grid, s);
+  if constexpr (KP > 128) {
+    // three-atom rows: value chunks of at most 48 channels fit two stages
+    switch (CP) {
+      case 16: return launch_kernel<KP, 16, DTFMT>(tx, ty, tv, kp, grid, s);
+      case 32: return launch_kernel<KP, 32, DTFMT>(tx, ty, tv, kp, grid, s);
+      default: return launch_kernel<KP, 48, DTFMT>(tx, ty, tv, kp, grid, s);
+    }
+  } else {
+    switch (CP) {
+      case 16: return launch_kernel<KP, 16, DTFMT>(tx, ty, tv, kp, grid, s);
+      case 32: return launch_kernel<KP, 32, DTFMT>(tx, ty, tv, kp, grid, s);
+      case 48: return launch_kernel<KP, 48, DTFMT>(tx, ty, tv, kp, grid, s);
+      case 64: return launch_kernel<KP, 64, DTFMT>(tx, ty, tv, kp, grid, s);
+      case 96: return launch_kernel<KP, 96, DTFMT>(tx, ty, tv, kp, grid, s);
+      default: return launch_kernel<KP, 128, DTFMT>(tx, ty, tv, kp, grid, s);
+    }
   }
 }
 
-int cp_for(int cw) {
+}  // namespace
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeFn get_encode() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(ptr);
+  });
+  return fn;
+}
+
+bool make_tmap_3d(CUtensorMap* m, CUtensorMapDataType dt, void* base, uint64_t d0, uint64_t d1,
+                  uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0,
+                  uint32_t box1, bool swizzle128) {
+  EncodeFn enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  const cuuint32_t box[3] = {box0, box1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, dt, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int tc_max_chunk(int KP) { return KP > 128 ? 48 : kTcMaxChunk; }
+
+int tc_chunk_pad(int cw) {
   const int c16 = (cw + 15) / 16 * 16;
   if (c16 <= 64) return c16 == 0 ? 16 : c16;
   return c16 <= 96 ? 96 : 128;
 }
 
-}  // namespace
-
 TcPlan tc_plan(int64_t B, int64_t M, int64_t N, int64_t D, int sm_count) {
   TcPlan p{};
-  p.KP = (D + 2 <= 64) ? 64 : 128;
+  p.KP = (D + 2 <= 64) ? 64 : ((D + 2 <= 128) ? 128 : 192);
   const int64_t U = B * ((M + kNT * kBM - 1) / (kNT * kBM));
   const int64_t ntj = (N + kBN - 1) / kBN;
   int64_t smax = ntj / 4;
@@ -673,9 +676,10 @@ cudaError_t launch_tc_sum(const TcArgs& a, cudaStream_t s) {
   const int64_t Nst = (a.N + 7) / 8 * 8;
   const dim3 grid(static_cast<unsigned>((a.M + kNT * kBM - 1) / (kNT * kBM)),
                   static_cast<unsigned>(a.plan.splits), static_cast<unsigned>(a.B));
-  for (int c0 = 0; c0 < a.CV; c0 += kTcMaxChunk) {
-    const int cw = (a.CV - c0) < kTcMaxChunk ? (a.CV - c0) : kTcMaxChunk;
-    const int CP = cp_for(cw);
+  const int chunk = tc_max_chunk(KP);
+  for (int c0 = 0; c0 < a.CV; c0 += chunk) {
+    const int cw = (a.CV - c0) < chunk ? (a.CV - c0) : chunk;
+    const int CP = tc_chunk_pad(cw);
     e = bf ? pack_values<__nv_bfloat16>(a, c0, CP, Nst, s) : pack_values<__half>(a, c0, CP, Nst, s);
     if (e != cudaSuccess) return e;
     CUtensorMap tv;
@@ -696,8 +700,10 @@ cudaError_t launch_tc_sum(const TcArgs& a, cudaStream_t s) {
     kp.out_scale = exp2f(-kPShift);
     if (KP == 64)
       e = bf ? launch_cp<64, 1>(CP, tx, ty, tv, kp, grid, s) : launch_cp<64, 0>(CP, tx, ty, tv, kp, grid, s);
-    else
+    else if (KP == 128)
       e = bf ? launch_cp<128, 1>(CP, tx, ty, tv, kp, grid, s) : launch_cp<128, 0>(CP, tx, ty, tv, kp, grid, s);
+    else
+      e = bf ? launch_cp<192, 1>(CP, tx, ty, tv, kp, grid, s) : launch_cp<192, 0>(CP, tx, ty, tv, kp, grid, s);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

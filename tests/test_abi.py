@@ -62,13 +62,22 @@ def test_invalid_arguments_are_rejected_before_any_launch(fn):
     assert _fwd(fn, C=0) == 1
     assert _fwd(fn, dt=7) == 1
     assert _fwd(fn, x=ODD) == 3
-    assert _fwd(fn, D=9) == 2              # fp32 path covers D <= 8
-    assert _fwd(fn, dt=1, D=127) == 2      # tensor-core path covers D <= 126
+    assert _fwd(fn, D=129) == 2            # fp32 covers D <= 128 (sums), D <= 8 (LSE)
+    assert _fwd(fn, dt=1, D=129) == 2      # tensor-core path covers D <= 128
     assert _fwd(fn, B=70000) == 2
 
 
 def test_lse_has_no_half_precision_path():
     assert _fwd("gauss_lse_fwd", dt=1, D=32) == 2
+
+
+def test_lse_and_knn_stay_on_the_small_d_path():
+    # the split-tf32 path (fp32, D > 8) serves the Gauss-sum passes only
+    assert _fwd("gauss_lse_fwd", D=9) == 2
+    assert _fwd("gauss_sum_fwd", D=9) == 4        # supported: asks for its workspace
+    lib = gs.library()
+    i64 = ctypes.c_void_p(0x100000)
+    assert lib.gauss_knn(FAKE, FAKE, FAKE, i64, 1, 10, 10, 9, 1, 0, NULL, 0, NULL) == 2
 
 
 def test_empty_problems_are_no_ops_without_pointers():
@@ -90,8 +99,12 @@ def test_workspace_query():
     assert big >= 2 * 4 * 65536 * 64 * 2 + 4 * 32 * 65536 * 2
     assert ws(gs.GS_OP_LSE, 1, 1000, 1000, 3, 1, gs.GS_F32) >= 2 * 1000 * 4
     assert ws(gs.GS_OP_SUM_BWD, 4, 16384, 16384, 32, 1, gs.GS_F16) >= 4 * 16384 * 33 * 4
+    # fp32 D > 8: packed split rows [hi | lo] of x and y at least
+    assert ws(gs.GS_OP_SUM, 1, 1000, 1000, 9, 1, gs.GS_F32) >= 2 * 1000 * 2 * 16 * 4
     with pytest.raises(ValueError):
-        ws(gs.GS_OP_SUM, 1, 10, 10, 9, 1, gs.GS_F32)
+        ws(gs.GS_OP_SUM, 1, 10, 10, 129, 1, gs.GS_F32)
+    with pytest.raises(ValueError):
+        ws(gs.GS_OP_LSE, 1, 10, 10, 9, 1, gs.GS_F32)
     with pytest.raises(ValueError):
         ws(7, 1, 10, 10, 3, 1, gs.GS_F32)
 

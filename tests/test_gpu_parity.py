@@ -104,7 +104,14 @@ F32_SHAPES = [  # B, M, N, D, C
 HALF_SHAPES = [
     (1, 1, 1, 32, 1), (1, 1, 300, 32, 1), (2, 300, 1000, 32, 32), (1, 257, 129, 16, 33),
     (1, 200, 700, 5, 1), (1, 100, 300, 100, 16), (2, 130, 260, 48, 130), (1, 511, 640, 62, 64),
-    (1, 70, 1200, 63, 3), (1, 129, 257, 126, 96),
+    (1, 70, 1200, 63, 3), (1, 129, 257, 126, 96), (1, 300, 700, 127, 1), (2, 257, 390, 128, 50),
+]
+# fp32 with D > 8: the split-tf32 tensor-core path (every packed-row width, one
+# and two value passes, single and several column tiles per warpgroup)
+F32_TC_SHAPES = [
+    (1, 1, 1, 9, 1), (1, 1, 300, 12, 1), (1, 300, 700, 9, 1), (1, 257, 1000, 16, 3),
+    (2, 300, 1100, 32, 32), (1, 129, 513, 33, 17), (1, 200, 333, 64, 64), (1, 130, 260, 65, 70),
+    (1, 100, 300, 96, 5), (1, 150, 450, 100, 40), (1, 128, 400, 128, 33), (3, 64, 2000, 24, 1),
 ]
 
 
@@ -127,6 +134,29 @@ def test_half_odd_shapes(shape, dtype):
     out = gs().gauss_sum_fwd(d["x"], d["y"], d["w"], inp["tau"]).cpu().numpy()
     ref = oracle.gauss_sum(f64(inp, "x"), f64(inp, "y"), f64(inp, "w"), inp["tau"])
     assert rel_l2(out, ref) <= TOL[dtype], rel_l2(out, ref)
+
+
+@pytest.mark.parametrize("shape", F32_TC_SHAPES, ids=[str(s) for s in F32_TC_SHAPES])
+def test_f32_tensor_core_shapes(shape):
+    B, M, N, D, C = shape
+    inp = synth.make_inputs(4, seed=hash(shape) % 1000, B=B, M=M, N=N, D=D, C=C, dtype="f32")
+    d = dev(inp)
+    out = gs().gauss_sum_fwd(d["x"], d["y"], d["w"], inp["tau"]).cpu().numpy()
+    ref = oracle.gauss_sum(f64(inp, "x"), f64(inp, "y"), f64(inp, "w"), inp["tau"])
+    assert rel_l2(out, ref) <= TOL["f32"], rel_l2(out, ref)
+
+
+@pytest.mark.parametrize("shift,tau", [(0.0, 4.0), (30.0, 1.0), (300.0, 1.0)])
+def test_f32_tensor_core_shifted_clouds_and_sharp_kernels(shift, tau):
+    """Clouds far from the origin (the operands are centred on a point of the
+    cloud, so the norms stay at the cloud's own scale) and a sharper kernel."""
+    inp = synth.make_inputs(4, seed=31, B=2, M=300, N=900, D=32, C=3, dtype="f32")
+    for k in ("x", "y"):
+        inp[k] = (inp[k].double() + shift).float()
+    d = dev(inp)
+    out = gs().gauss_sum_fwd(d["x"], d["y"], d["w"], tau).cpu().numpy()
+    ref = oracle.gauss_sum(f64(inp, "x"), f64(inp, "y"), f64(inp, "w"), tau)
+    assert rel_l2(out, ref) <= TOL["f32"], rel_l2(out, ref)
 
 
 @pytest.mark.parametrize("shape", [(1, 700, 900, 3, 1), (2, 300, 1100, 2, 3), (1, 64, 5000, 8, 9)])
@@ -157,10 +187,11 @@ def test_lse_rows_far_from_every_point():
 @pytest.mark.parametrize("dtype,shape", [
     ("f32", (1, 500, 700, 3, 1)), ("f32", (2, 300, 400, 2, 3)), ("f32", (1, 200, 300, 8, 2)),
     ("f16", (1, 300, 500, 32, 1)), ("f16", (2, 257, 300, 16, 4)), ("bf16", (1, 200, 333, 32, 1)),
+    ("f32", (1, 300, 500, 32, 1)), ("f32", (2, 257, 300, 20, 4)),
 ])
 def test_bwd_shapes(dtype, shape):
     B, M, N, D, C = shape
-    wid = 1 if dtype == "f32" else 5
+    wid = 1 if (dtype == "f32" and D <= 8) else 5
     inp = synth.make_inputs(wid, seed=12, B=B, M=M, N=N, D=D, C=C, dtype=dtype, with_g=True)
     d = dev(inp)
     gx, gw = gs().gauss_sum_bwd(d["x"], d["y"], d["w"], d["g"], inp["tau"])
@@ -260,13 +291,14 @@ def test_tensor_core_path_is_deterministic_under_repetition(C):
     ("f32", (1, 300, 400, 3, 1), 40.0),
     ("f16", (1, 300, 500, 32, 1), 0.0), ("f16", (2, 257, 300, 16, 4), 0.0), ("bf16", (1, 200, 333, 32, 1), 0.0),
     ("f16", (1, 300, 500, 16, 2), 20.0),
+    ("f32", (1, 300, 500, 32, 1), 0.0), ("f32", (2, 200, 300, 12, 3), 0.0), ("f32", (1, 250, 400, 32, 2), 25.0),
 ])
 def test_vjp_every_gradient(dtype, shape, shift):
     """dL/dx, dL/dy, dL/dw and dL/dtau against the oracle; `shift` moves the
     whole point cloud away from the origin (the gradients do not change, the
     centred values keep the cancellation at the cloud's own scale)."""
     B, M, N, D, C = shape
-    wid = 1 if dtype == "f32" else 5
+    wid = 1 if (dtype == "f32" and D <= 8) else 5
     inp = synth.make_inputs(wid, seed=13, B=B, M=M, N=N, D=D, C=C, dtype=dtype, with_g=True)
     if shift:
         for k in ("x", "y"):
@@ -368,11 +400,12 @@ def test_knn_duplicates_and_quantised_grid():
 # ------------------------------------------------------------------ diffusion operator
 @pytest.mark.parametrize("dtype,shape,alpha", [("f32", (1, 3000, 3, 4), 0.5), ("f32", (2, 1500, 6, 1), 1.0),
                                                ("f32", (1, 2000, 2, 3), 0.0), ("f16", (1, 2500, 32, 8), 0.5),
-                                               ("bf16", (2, 1000, 16, 2), 0.5)])
+                                               ("bf16", (2, 1000, 16, 2), 0.5), ("f32", (1, 2000, 80, 4), 0.5)])
 def test_diffusion_scales_and_apply(dtype, shape, alpha):
     B, N, D, C = shape
-    inp = synth.make_inputs(1 if dtype == "f32" else 4, seed=23, B=B, M=N, N=N, D=D, C=C, dtype=dtype)
-    tau = 2.0 if dtype == "f32" else 8.0
+    small = dtype == "f32" and D <= 8
+    inp = synth.make_inputs(1 if small else 4, seed=23, B=B, M=N, N=N, D=D, C=C, dtype=dtype)
+    tau = 2.0 if small else 8.0
     x = inp["x"].cuda()
     q, dd, s = gs().gauss_diffusion_scales(x, tau, alpha)
     rq, rd, rs = oracle.diffusion_scales(f64(inp, "x"), tau, alpha)
