@@ -137,7 +137,7 @@ PassLayout pass_layout(const Pass& p, int sm) {
     const size_t CPmax = static_cast<size_t>(
         f32_chunk_pad(p.CV < L.f32.max_chunk ? p.CV : L.f32.max_chunk));
     const size_t Nst = (p.N + 3) / 4 * 4;
-    const size_t Nq = (p.N + 63) / 64 * 64;
+    const size_t Nq = (p.N + 127) / 128 * 128;
     L.off_xpack = off;
     off = align_up(off + size_t(p.B) * p.R * rowb);
     L.off_rnorm = off;

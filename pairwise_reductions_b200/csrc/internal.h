@@ -179,7 +179,7 @@ struct F32Plan {
   int atoms;           // 128-byte atoms per packed row (2 Kp floats)
   int max_chunk;       // channels per pass (64, or 32 for the widest rows)
   int splits;
-  int64_t cols_per_split;   // multiple of 64
+  int64_t cols_per_split;   // multiple of 128
 };
 F32Plan f32_plan(int64_t B, int64_t M, int64_t N, int64_t D, int sm_count);
 int f32_chunk_pad(int cw);            // 16, 32 or 64
@@ -201,7 +201,8 @@ struct F32Args {
   float* xpack;        // [B, M, 2 Kp]
   float* rnorm;        // [B, M]
   float* ypack;        // [B, N, 2 Kp]
-  float* qw;           // [B, Nq, 4]: -c |y'|^2 (-inf past N) and up to 3 value channels
+  float* qw;           // [B, Nq, 4], Nq = N rounded up to 128: -c |y'|^2 (-inf past N)
+                       // and up to 3 value channels
   float* vt;           // [2 B, CP, Nst] (hi, lo), Nst = N rounded up to 4
 };
 cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s);

@@ -52,6 +52,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kAtom = kBM * 128;   // one 128-row x 32-float (128-byte) swizzle atom
 
 struct F32KParams {
+  const float* xpack;   // [B, M, 2 K'] packed rows (copied into TMEM when it has room)
   const float* rnorm;   // [B, M]
   float* out;
   int64_t split_stride;
@@ -62,10 +63,11 @@ struct F32KParams {
   int ksteps;           // K' / 8: tf32 K steps of the hi (and of the lo) half
   int atoms;            // 128-byte atoms of a packed row actually loaded (<= KA)
   int Bsz;              // batch count (the lo half of v sits at batch index B + b)
+  int bn;               // tile width the TMA boxes were made for
   float two_c;
 };
 
-// KA: 128-byte atoms per packed row [hi K' | lo K'] the shared memory holds.
+// KA: 128-byte atoms per packed row [hi K' | lo K'] the operands may hold.
 // MODE 1 or 3: the values (at most MODE channels) ride with the column norms
 // and P.v is summed in registers (exact fp32 products); MODE 16, 32 or 64:
 // P.v on the tensor cores for a chunk of MODE channels.
@@ -73,15 +75,33 @@ template <int KA, int MODE>
 struct F32Cfg {
   static constexpr bool REG = MODE <= 3;
   static constexpr int CP = REG ? 16 : MODE;
-  static constexpr int X_BYTES = KA * kAtom;
-  static constexpr int QW_BYTES = 1024;                 // up to 64 columns x 16 bytes
+  static constexpr int CPA = (CP + 31) / 32 * 32;
+  static constexpr int qw_bytes(int bn) { return bn * 16 <= 1024 ? 1024 : bn * 16; }
   static constexpr int v_bytes(int bn) { return REG ? 0 : 2 * (bn / 32) * CP * 128; }
-  static constexpr int stage_bytes(int bn) { return KA * bn * 128 + QW_BYTES + v_bytes(bn); }
+  static constexpr int stage_bytes(int bn) { return KA * bn * 128 + qw_bytes(bn) + v_bytes(bn); }
   static constexpr int BUDGET = 214 * 1024;
-  // register path, one channel: 64-column tiles where two stages fit (three
-  // channels: 32, for registers); tensor-core P.v: 32-column tiles (TMEM holds
-  // S, P hi/lo and O for both warpgroups)
-  static constexpr int BN = (MODE == 1 && (BUDGET - X_BYTES) / stage_bytes(64) >= 2) ? 64 : 32;
+  // TMEM columns of the accumulators.  Register values: the large and the
+  // small products of S in separate accumulators for each warpgroup (two
+  // independent MMA chains; the small ones never round against the large
+  // sum).  Tensor-core values: one S (small products first, then the large
+  // ones), P hi/lo and O per warpgroup.
+  static constexpr int tmem_acc(int bn) { return REG ? 4 * bn : 6 * bn + 2 * CPA; }
+  // The x' rows (2 K' <= 32 KA columns) sit in TMEM as the A operand of the
+  // similarity MMAs when the accumulators leave room, else in shared memory.
+  static constexpr bool xt(int bn) { return tmem_acc(bn) + 32 * KA <= 512; }
+  static constexpr int x_bytes(int bn) { return xt(bn) ? 0 : KA * kAtom; }
+  static constexpr bool fits(int bn) {
+    return tmem_acc(bn) <= 512 && (BUDGET - x_bytes(bn)) / stage_bytes(bn) >= 2;
+  }
+  // Column tile.  An M = 128 tf32 MMA takes about the same time for any N up
+  // to 128 (measured on B200: ~78 cycles at N = 32 .. 128), so the widest
+  // tile that fits is the cheapest per pair; three register channels use 32
+  // columns (registers).
+  static constexpr int BN =
+      MODE == 3 ? 32 : ((MODE == 1 && fits(128)) ? 128 : (fits(64) ? 64 : 32));
+  static constexpr bool XT = xt(BN);
+  static constexpr int X_BYTES = x_bytes(BN);
+  static constexpr int QW_BYTES = qw_bytes(BN);
   static constexpr int Y_BYTES = KA * BN * 128;
   static constexpr int V_ATOM = CP * 128;               // CP rows x 32 columns
   static constexpr int V_BYTES = v_bytes(BN);
@@ -93,15 +113,16 @@ struct F32Cfg {
   static constexpr int SMEM_RAW = 1024 + X_BYTES + NST * STAGE + 8 * NBARS + 16 + RED_BYTES;
   // at least ~120 KB: one CTA per SM, so the 512-column TMEM allocation never waits
   static constexpr int SMEM = SMEM_RAW < 122880 ? 122880 : SMEM_RAW;
-  // TMEM columns: Sbig0 | Sbig1 | Ssmall0 | Ssmall1 [| Phi0 | Phi1 | Plo0 | Plo1 | O0 | O1]
-  static constexpr int CPA = (CP + 31) / 32 * 32;
-  __host__ __device__ static constexpr uint32_t col_sb(int h) { return BN * h; }
-  __host__ __device__ static constexpr uint32_t col_ss(int h) { return 2 * BN + BN * h; }
-  __host__ __device__ static constexpr uint32_t col_phi(int h) { return 4 * BN + BN * h; }
-  __host__ __device__ static constexpr uint32_t col_plo(int h) { return 6 * BN + BN * h; }
-  __host__ __device__ static constexpr uint32_t col_o(int h) { return 8 * BN + CPA * h; }
+  // TMEM columns.  Register values: Sbig0 | Sbig1 | Ssmall0 | Ssmall1 | x'.
+  // Tensor-core values: S0 | S1 | Phi0 | Phi1 | Plo0 | Plo1 | O0 | O1 | x'.
+  __host__ __device__ static constexpr uint32_t col_s(int h) { return h * BN; }
+  __host__ __device__ static constexpr uint32_t col_ss(int h) { return 2 * BN + h * BN; }
+  __host__ __device__ static constexpr uint32_t col_phi(int h) { return 2 * BN + BN * h; }
+  __host__ __device__ static constexpr uint32_t col_plo(int h) { return 4 * BN + BN * h; }
+  __host__ __device__ static constexpr uint32_t col_o(int h) { return 6 * BN + CPA * h; }
+  static constexpr uint32_t COL_X = tmem_acc(BN);
   static_assert(NST >= 2, "shared memory budget");
-  static_assert(REG ? 4 * BN <= 512 : 8 * BN + 2 * CPA <= 512, "TMEM budget");
+  static_assert(tmem_acc(BN) + (XT ? 32 * KA : 0) <= 512, "TMEM budget");
   static_assert(REG || (CP % 16 == 0 && CP >= 16 && CP <= 64), "value chunk");
   static_assert(SMEM_RAW <= 227 * 1024, "shared memory per CTA");
 };
@@ -146,6 +167,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int CP = Cfg::CP;
   constexpr int NST = Cfg::NST;
   constexpr int BN = Cfg::BN;
+  if (p.bn != BN) {   // boxes sized for another tile: touch nothing, report
+    if (threadIdx.x == 0) atomicOr(&g_device_error_f32, 2);
+    return;
+  }
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -161,8 +186,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_empty = [&](int s) { return bar0 + 8u * (NST + s); };
   const uint32_t bar_x = bar0 + 8u * (2 * NST);
   auto bar_s = [&](int h) { return bar0 + 8u * (2 * NST + 1 + h); };   // S_h ready
-  auto bar_p = [&](int h) { return bar0 + 8u * (2 * NST + 3 + h); };   // P_h written
-  auto bar_f = [&](int h) { return bar0 + 8u * (2 * NST + 5 + h); };   // S_h read out
+  auto bar_f = [&](int h) { return bar0 + 8u * (2 * NST + 3 + h); };   // S_h read out
+  auto bar_p = [&](int h) { return bar0 + 8u * (2 * NST + 5 + h); };   // P_h written
   auto bar_q = [&](int h) { return bar0 + 8u * (2 * NST + 7 + h); };   // P_h consumed
   const uint32_t bar_o = bar0 + 8u * (2 * NST + 9);
 
@@ -180,11 +205,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // 128 exp threads that read its norms and values (register values)
       mbar_init(bar_empty(s), REG ? 4 * 32 : 1);
     }
-    mbar_init(bar_x, 1);
+    // x' ready: the TMA load (shared memory), or the 128 threads of exp
+    // warpgroup 0 that copy the rows into TMEM
+    mbar_init(bar_x, Cfg::XT ? 4 * 32 : 1);
     for (int h = 0; h < 2; ++h) {
       mbar_init(bar_s(h), 1);
-      mbar_init(bar_p(h), 4 * 32);
       mbar_init(bar_f(h), 4 * 32);
+      mbar_init(bar_p(h), 4 * 32);
       mbar_init(bar_q(h), 1);
     }
     mbar_init(bar_o, 1);
@@ -203,14 +230,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      tma_prefetch_desc(&tmX);
       tma_prefetch_desc(&tmY);
       tma_prefetch_desc(&tmQ);
       if constexpr (!REG) tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(bar_x, p.atoms * kAtom);
-      for (int a = 0; a < p.atoms; ++a)
-        tma_load_3d(smem_u32(sX + a * kAtom), &tmX, bar_x, a * 32, static_cast<int>(row0),
-                    static_cast<int>(b));
+      if constexpr (!Cfg::XT) {
+        tma_prefetch_desc(&tmX);
+        mbar_arrive_expect_tx(bar_x, p.atoms * kAtom);
+        for (int a = 0; a < p.atoms; ++a)
+          tma_load_3d(smem_u32(sX + a * kAtom), &tmX, bar_x, a * 32, static_cast<int>(row0),
+                      static_cast<int>(b));
+      }
       const uint32_t stage_tx = p.atoms * BN * 128 + BN * 16 + Cfg::V_BYTES;
       for (int t = 0; t < T; ++t) {
         const int st = t % NST;
@@ -245,17 +274,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int off = ks * 32;
         return desc_k_sw128(smem_u32(base + (off >> 7) * atom_bytes) + (off & 127));
       };
-      // S = x'.y'^T: the two small products accumulate apart from the large
-      // one, so that each of them is rounded against its own magnitude
+      // S = x'.y'^T for warpgroup h.  Register values: the small products
+      // (lo.hi, hi.lo) into Ssmall_h and the large ones into Sbig_h, K step
+      // by K step (two independent chains).  Tensor-core values: one
+      // accumulator, every small product of every K step first, while it is
+      // small, then the large ones -- each addition is rounded against the
+      // magnitude of what it adds to.
       auto issue_S = [&](int h, int st) {
         const uint8_t* sy = sStage + st * Cfg::STAGE;
-        const uint32_t db = tmem + Cfg::col_sb(h), ds = tmem + Cfg::col_ss(h);
-        for (int ks = 0; ks < p.ksteps; ++ks) {
-          const uint64_t ah = kdesc(sX, kAtom, ks), al = kdesc(sX, kAtom, ks + ks_lo);
-          const uint64_t bh = kdesc(sy, BN * 128, ks), bl = kdesc(sy, BN * 128, ks + ks_lo);
-          mma_ss_tf32(ds, al, bh, idS, ks > 0 ? 1u : 0u);
-          mma_ss_tf32(ds, ah, bl, idS, 1u);
-          mma_ss_tf32(db, ah, bh, idS, ks > 0 ? 1u : 0u);
+        const uint32_t db = tmem + Cfg::col_s(h);
+        const uint32_t ds = REG ? tmem + Cfg::col_ss(h) : db;
+        auto mma = [&](uint32_t d, int ka, uint64_t bdesc, uint32_t acc) {
+          if constexpr (Cfg::XT) {
+            mma_ts_tf32(d, tmem + Cfg::COL_X + ka * 8, bdesc, idS, acc);
+          } else {
+            mma_ss_tf32(d, kdesc(sX, kAtom, ka), bdesc, idS, acc);
+          }
+        };
+        if constexpr (REG) {
+          for (int ks = 0; ks < p.ksteps; ++ks) {
+            const uint64_t bh = kdesc(sy, BN * 128, ks), bl = kdesc(sy, BN * 128, ks + ks_lo);
+            mma(ds, ks + ks_lo, bh, ks > 0 ? 1u : 0u);
+            mma(ds, ks, bl, 1u);
+            mma(db, ks, bh, ks > 0 ? 1u : 0u);
+          }
+        } else {
+          for (int ks = 0; ks < p.ksteps; ++ks) {
+            mma(db, ks + ks_lo, kdesc(sy, BN * 128, ks), ks > 0 ? 1u : 0u);
+            mma(db, ks, kdesc(sy, BN * 128, ks + ks_lo), 1u);
+          }
+          for (int ks = 0; ks < p.ksteps; ++ks) mma(db, ks, kdesc(sy, BN * 128, ks), 1u);
         }
       };
       auto issue_O = [&](int h, int st, bool acc_prev) {
@@ -274,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       bool ok = wait_bar(bar_x, 0, abort_flag);
+      tc_fence_after();
       for (int h = 0; ok && h < 2 && h < T; ++h) {
         ok = wait_bar(bar_full(h), 0, abort_flag);
         if (ok) {
@@ -322,12 +371,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool valid = i < p.M;
     const float r = valid ? p.rnorm[b * p.M + i] : 0.f;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tSb = tmem + lane_base + Cfg::col_sb(h);
-    const uint32_t tSs = tmem + lane_base + Cfg::col_ss(h);
     const uint32_t tPh = tmem + lane_base + Cfg::col_phi(h);
     const uint32_t tPl = tmem + lane_base + Cfg::col_plo(h);
     const float two_c = p.two_c;
     float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f;   // register values: running row sums
+    if constexpr (Cfg::XT) {
+      if (h == 0) {
+        // this thread's packed row (zeros past M) into its TMEM lane
+        const int rowf = 2 * p.ksteps * 8;
+        const float4* src = reinterpret_cast<const float4*>(p.xpack + (b * p.M + i) * rowf);
+        for (int c = 0; c < rowf / 16; ++c) {
+          uint32_t v[16];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float4 f = valid ? src[c * 4 + u] : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[4 * u + 0] = __float_as_uint(f.x);
+            v[4 * u + 1] = __float_as_uint(f.y);
+            v[4 * u + 2] = __float_as_uint(f.z);
+            v[4 * u + 3] = __float_as_uint(f.w);
+          }
+          tmem_st16(tmem + lane_base + Cfg::COL_X + c * 16, v);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_x);
+      }
+    }
     bool ok = true;
     int k = 0;
     for (int t = h; t < T; t += 2, ++k) {
@@ -339,38 +408,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      // S = Sbig + Ssmall, the whole tile into registers; then its TMEM
-      // columns may be reused
-      uint32_t sv[BN / 32][32];
-#pragma unroll
-      for (int ch = 0; ch < BN / 32; ++ch) {
-        uint32_t ss[32];
-        tmem_ld32(tSb + ch * 32, sv[ch]);
-        tmem_ld32(tSs + ch * 32, ss);
-        tmem_wait_ld();
-        reg_fence32(sv[ch]);
-        reg_fence32(ss);
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          sv[ch][e] = __float_as_uint(__uint_as_float(sv[ch][e]) + __uint_as_float(ss[e]));
-      }
-      tc_fence_before();
-      mbar_arrive(bar_f(h));
+      const uint32_t tS = tmem + lane_base + Cfg::col_s(h);
       const float4* qw = reinterpret_cast<const float4*>(sStage + st * Cfg::STAGE + Cfg::Y_BYTES);
       if constexpr (REG) {
-        // P.v in registers, a partial sum per tile (two-level accumulation)
+        // S = Sbig + Ssmall, 32 columns at a time: the loads of chunk ch + 1
+        // are in flight while chunk ch is exponentiated; once the last chunk
+        // is in registers the TMEM columns may be reused.  P.v in registers,
+        // a partial sum per tile (two-level accumulation).
+        constexpr int NCH = BN / 32;
+        const uint32_t tSs = tmem + lane_base + Cfg::col_ss(h);
+        uint32_t cb[32], cs[32];
+        tmem_ld32(tS, cb);
+        tmem_ld32(tSs, cs);
+        tmem_wait_ld();
+        reg_fence32(cb);
+        reg_fence32(cs);
         float p0 = 0.f, p1 = 0.f, p2 = 0.f;
 #pragma unroll
-        for (int ch = 0; ch < BN / 32; ++ch) {
+        for (int ch = 0; ch < NCH; ++ch) {
+          float cur[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            cur[e] = fmaf(__uint_as_float(cb[e]) + __uint_as_float(cs[e]), two_c, r);
+          if (ch + 1 < NCH) {
+            tmem_ld32(tS + (ch + 1) * 32, cb);
+            tmem_ld32(tSs + (ch + 1) * 32, cs);
+          } else {
+            tc_fence_before();
+            mbar_arrive(bar_f(h));
+          }
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const float4 q = qw[ch * 32 + e];
-            const float pe = ex2(fmaf(__uint_as_float(sv[ch][e]), two_c, r) + q.x);
-            p0 = fmaf(pe, q.y, p0);
-            if constexpr (MODE > 1) {
+            const int j = ch * 32 + e;
+            if constexpr (MODE == 1) {
+              // (norm, value): the first half of the column's 16 bytes
+              const float2 q = reinterpret_cast<const float2*>(qw)[2 * j];
+              p0 = fmaf(ex2(cur[e] + q.x), q.y, p0);
+            } else {
+              const float4 q = qw[j];
+              const float pe = ex2(cur[e] + q.x);
+              p0 = fmaf(pe, q.y, p0);
               p1 = fmaf(pe, q.z, p1);
               p2 = fmaf(pe, q.w, p2);
             }
+          }
+          if (ch + 1 < NCH) {
+            tmem_wait_ld();
+            reg_fence32(cb);
+            reg_fence32(cs);
           }
         }
         acc0 += p0;
@@ -378,6 +463,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc2 += p2;
         mbar_arrive(bar_empty(st));
       } else {
+        // the whole S tile into registers; then its TMEM columns may be reused
+        uint32_t sv[BN / 32][32];
+#pragma unroll
+        for (int ch = 0; ch < BN / 32; ++ch) tmem_ld32(tS + ch * 32, sv[ch]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int ch = 0; ch < BN / 32; ++ch) reg_fence32(sv[ch]);
+        tc_fence_before();
+        mbar_arrive(bar_f(h));
 #pragma unroll
         for (int ch = 0; ch < BN / 32; ++ch) {
 #pragma unroll
@@ -576,12 +670,17 @@ cudaError_t launch_mode(int mode, const TileMaps& m, const F32KParams& kp, dim3 
 // Shared-memory atoms the kernel is compiled for, covering `atoms`.
 int ka_for(int atoms) { return atoms <= 1 ? 1 : (atoms <= 2 ? 2 : (atoms <= 4 ? 4 : (atoms <= 6 ? 6 : 8))); }
 
+// Tile width of instantiation (KA, mode): the host sizes the TMA boxes with it.
 template <int KA>
 int tile_cols_ka(int mode) {
   switch (mode) {
     case 1: return F32Cfg<KA, 1>::BN;
     case 3: return F32Cfg<KA, 3>::BN;
-    default: return F32Cfg<KA, 16>::BN;   // every tensor-core value chunk: 32
+    case 16: return F32Cfg<KA, 16>::BN;
+    case 32: return F32Cfg<KA, 32>::BN;
+    default:
+      if constexpr (KA < 8) return F32Cfg<KA, 64>::BN;
+      return 0;
   }
 }
 
@@ -595,9 +694,10 @@ F32Plan f32_plan(int64_t B, int64_t M, int64_t N, int64_t D, int sm_count) {
   p.Kp = static_cast<int>((D + 7) / 8 * 8);
   p.atoms = (2 * p.Kp + 31) / 32;
   p.max_chunk = ka_for(p.atoms) >= 8 ? 32 : 64;
-  // a split is a whole number of 64-column blocks (either tile width divides it)
+  // a split is a whole number of 128-column blocks (every tile width divides
+  // it, so no tile straddles two splits)
   const int64_t U = B * ((M + kBM - 1) / kBM);
-  const int64_t ntj = (N + 63) / 64;
+  const int64_t ntj = (N + 127) / 128;
   int64_t smax = ntj / 4;
   if (smax > 32) smax = 32;
   if (smax < 1) smax = 1;
@@ -612,7 +712,7 @@ F32Plan f32_plan(int64_t B, int64_t M, int64_t N, int64_t D, int sm_count) {
     }
   }
   const int64_t per = (ntj + best - 1) / best;
-  p.cols_per_split = (per < 1 ? 1 : per) * 64;
+  p.cols_per_split = (per < 1 ? 1 : per) * 128;
   p.splits = static_cast<int>((N + p.cols_per_split - 1) / p.cols_per_split);
   if (p.splits < 1) p.splits = 1;
   return p;
@@ -634,7 +734,7 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
   if (a.B == 0 || a.M == 0) return cudaSuccess;
   const int Kp = a.plan.Kp;
   const float c = 0.5f * a.tau * kLog2e;
-  const int64_t Nq = (a.N + 63) / 64 * 64;
+  const int64_t Nq = (a.N + 127) / 128 * 128;
   const float* x = static_cast<const float*>(a.x);
   const float* y = static_cast<const float*>(a.y);
   pack_rows_f32_kernel<<<grid_for(a.B * a.M, 128), 128, 0, s>>>(x, x, a.xpack, a.rnorm, a.B, a.M,
@@ -664,6 +764,7 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
     const int cw = (a.CV - c0) < chunk ? (a.CV - c0) : chunk;
     const int mode = mode_for(a.CV, cw);
     const int BN = f32_tile_cols(KA, mode);
+    if (BN != 32 && BN != 64 && BN != 128) return cudaErrorInvalidValue;
     if (!make_tmap_3d(&m.y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.ypack, rowf, a.N, a.B, rowf * 4,
                       a.N * rowf * 4, 32, BN) ||
         !make_tmap_3d(&m.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.qw, 4, Nq, a.B, 16, Nq * 16ull, 4,
@@ -683,6 +784,7 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
         return cudaErrorInvalidValue;
     }
     F32KParams kp{};
+    kp.xpack = a.xpack;
     kp.rnorm = a.rnorm;
     kp.out = a.out;
     kp.split_stride = a.split_stride;
@@ -695,6 +797,7 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
     kp.ksteps = Kp / 8;
     kp.atoms = a.plan.atoms;
     kp.Bsz = static_cast<int>(a.B);
+    kp.bn = BN;
     kp.two_c = a.tau * kLog2e;
     switch (KA) {
       case 1: e = launch_mode<1>(mode, m, kp, grid, s); break;
