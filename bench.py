@@ -180,15 +180,18 @@ def launches_per_step(gs, run):
 
 
 # ------------------------------------------------------------------ ncu traffic of the dominant kernel
-DOMINANT = {"f32": ("sd_kernel", "small_d.cu"), "f16": ("tc_gauss_kernel", "tc_sm100.cu"),
-            "bf16": ("tc_gauss_kernel", "tc_sm100.cu")}
+def dominant(w):
+    """(kernel, source file) that does the pair work of a workload."""
+    if w.dtype != "f32":
+        return "tc_gauss_kernel", "tc_sm100.cu"
+    return ("sd_kernel", "small_d.cu") if w.D <= 8 else ("tc_f32_kernel", "tc_f32_sm100.cu")
 
 
 def traffic_per_launch(w):
     """DRAM bytes (read + write) per launch of the dominant kernel from the committed ncu
     summary, or None when there is none for this workload or the kernel source changed since."""
     import hashlib
-    kernel, src = DOMINANT[w.dtype]
+    kernel, src = dominant(w)
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     try:
         lines = open(path).read().splitlines()

@@ -48,8 +48,7 @@ gs_status check_dims(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, int64
   if (dt == GS_F32) {
     // D > 8: the split-tf32 tensor-core path, for the Gauss-sum passes only
     if (D > kTcMaxD) return GS_ERR_UNSUPPORTED;
-    if (D > kSdMaxD && (op == GS_OP_LSE || op == GS_OP_LSE_BWD || op == GS_OP_KNN))
-      return GS_ERR_UNSUPPORTED;
+    if (D > kSdMaxD && (op == GS_OP_LSE_BWD || op == GS_OP_KNN)) return GS_ERR_UNSUPPORTED;
   } else {
     if (D > kTcMaxD) return GS_ERR_UNSUPPORTED;
     if (op == GS_OP_LSE || op == GS_OP_LSE_BWD) return GS_ERR_UNSUPPORTED;
@@ -122,7 +121,7 @@ struct PassLayout {
   SdPlan sd;
   TcPlan tcp;
   F32Plan f32;
-  size_t off_part, off_vals, off_xpack, off_rnorm, off_ypack, off_vt, off_qw;
+  size_t off_part, off_vals, off_xpack, off_rnorm, off_ypack, off_vt, off_qw, off_zc;
   size_t total;
 };
 
@@ -138,6 +137,8 @@ PassLayout pass_layout(const Pass& p, int sm) {
         f32_chunk_pad(p.CV < L.f32.max_chunk ? p.CV : L.f32.max_chunk));
     const size_t Nst = (p.N + 3) / 4 * 4;
     const size_t Nq = (p.N + 127) / 128 * 128;
+    L.off_zc = off;
+    off = align_up(off + size_t(p.B) * p.D * 4);
     L.off_xpack = off;
     off = align_up(off + size_t(p.B) * p.R * rowb);
     L.off_rnorm = off;
@@ -249,6 +250,7 @@ gs_status run_pass(const Pass& p, const PassLayout& L, float* out, uint8_t* ws, 
     a.D = p.D;
     a.tau = p.tau;
     a.plan = L.f32;
+    a.zc = reinterpret_cast<float*>(ws + L.off_zc);
     a.xpack = reinterpret_cast<float*>(ws + L.off_xpack);
     a.rnorm = reinterpret_cast<float*>(ws + L.off_rnorm);
     a.ypack = reinterpret_cast<float*>(ws + L.off_ypack);
@@ -368,6 +370,37 @@ VjpLayout vjp_layout(const void* x, const void* y, const void* w, const float* g
     L.off_tau = off;
     off = align_up(off + size_t(B) * M * 4);
   }
+  L.total = off;
+  return L;
+}
+
+// Log-sum-exp forward on the fp32 tensor-core path (D > 8): packed operands,
+// the column norms / log-weights, and the per-split (m, l) partials.
+struct LseF32Layout {
+  F32Plan plan;
+  size_t off_zc, off_xpack, off_rnorm, off_ypack, off_qw, off_m, off_l, total;
+};
+
+LseF32Layout lse_f32_layout(int64_t B, int64_t M, int64_t N, int64_t D, int64_t C, int sm) {
+  LseF32Layout L{};
+  L.plan = f32_plan(B, M, N, D, sm);
+  const size_t rowb = size_t(2) * L.plan.Kp * 4;
+  const size_t Nq = (N + 127) / 128 * 128;
+  size_t off = 0;
+  L.off_zc = off;
+  off = align_up(off + size_t(B) * D * 4);
+  L.off_xpack = off;
+  off = align_up(off + size_t(B) * M * rowb);
+  L.off_rnorm = off;
+  off = align_up(off + size_t(B) * M * 4);
+  L.off_ypack = off;
+  off = align_up(off + size_t(B) * N * rowb);
+  L.off_qw = off;
+  off = align_up(off + size_t(B) * Nq * 16);
+  L.off_m = off;
+  off = align_up(off + size_t(L.plan.splits) * B * M * C * 4);
+  L.off_l = off;
+  off = align_up(off + size_t(L.plan.splits) * B * M * C * 4);
   L.total = off;
   return L;
 }
@@ -499,6 +532,7 @@ size_t gs_workspace_bytes(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, 
   }
   if (op == GS_OP_LSE) {
     if (M == 0 || N == 0) return 0;
+    if (D > kSdMaxD) return lse_f32_layout(B, M, N, D, C, sm).total;
     const SdPlan sp = sd_plan(B, M, N, static_cast<int>(D), C, sm);
     return align_up(size_t(2) * sp.splits * B * M * C * 4);
   }
@@ -549,6 +583,55 @@ gs_status gauss_lse_fwd(const void* x, const void* y, const void* w, float* out,
     return GS_OK;
   }
   const int sm = sm_count();
+  if (D > kSdMaxD) {
+    // fp32 tensor-core path: running-maximum (m, l) per split, then the finalize
+    const LseF32Layout L = lse_f32_layout(B, M, N, D, C, sm);
+    if (ws_bytes < L.total) return GS_ERR_WORKSPACE;
+    GS_TRY(check_ptr(ws, 1));
+    uint8_t* w8 = static_cast<uint8_t*>(ws);
+    const int64_t tot = B * M * C;
+    F32Args a{};
+    a.x = x;
+    a.y = y;
+    a.w = static_cast<const float*>(w);
+    a.values = kValuesW;
+    a.C = static_cast<int>(C);
+    a.CV = static_cast<int>(C);
+    a.out = reinterpret_cast<float*>(w8 + L.off_m);
+    a.out_l = reinterpret_cast<float*>(w8 + L.off_l);
+    a.lse = true;
+    a.split_stride = tot;
+    a.B = B;
+    a.M = M;
+    a.N = N;
+    a.D = static_cast<int>(D);
+    a.tau = tau;
+    a.plan = L.plan;
+    a.zc = reinterpret_cast<float*>(w8 + L.off_zc);
+    a.xpack = reinterpret_cast<float*>(w8 + L.off_xpack);
+    a.rnorm = reinterpret_cast<float*>(w8 + L.off_rnorm);
+    a.ypack = reinterpret_cast<float*>(w8 + L.off_ypack);
+    a.qw = reinterpret_cast<float*>(w8 + L.off_qw);
+    a.vt = nullptr;
+    GS_CUDA(launch_tc_f32_sum(a, s));
+    LseFinalizeArgs f{};
+    f.part_m = a.out;
+    f.part_l = a.out_l;
+    f.splits = L.plan.splits;
+    f.split_stride = tot;
+    f.out = out;
+    f.x = static_cast<const float*>(x);
+    f.y = static_cast<const float*>(y);
+    f.w = static_cast<const float*>(w);
+    f.B = B;
+    f.M = M;
+    f.N = N;
+    f.D = static_cast<int>(D);
+    f.C = static_cast<int>(C);
+    f.scale = coord_scale(tau);
+    GS_CUDA(launch_lse_finalize(f, s));
+    return GS_OK;
+  }
   const SdPlan sp = sd_plan(B, M, N, static_cast<int>(D), C, sm);
   const size_t need = align_up(size_t(2) * sp.splits * B * M * C * 4);
   if (ws_bytes < need) return GS_ERR_WORKSPACE;

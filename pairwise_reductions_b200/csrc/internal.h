@@ -189,15 +189,18 @@ struct F32Args {
   const void* x;       // rows side [B, M, D] float32
   const void* y;       // column side [B, N, D] float32
   const float* w;      // values source [B, N, C] float32
-  TcValues values;     // value mode (values.cuh), columns centred at x[b, 0]
+  TcValues values;     // value mode (values.cuh; its own centre x[b, 0])
   int C, CV;
-  float* out;          // [S?][B][M][CV]
+  float* out;          // [S?][B][M][CV]; log-sum-exp: the shifts m (log2 units)
+  float* out_l;        // log-sum-exp only: the scaled sums l, same layout
+  bool lse;            // log-sum-exp of w K per channel (w > 0) instead of the sum
   int64_t split_stride;
   int64_t B, M, N;
   int D;
   float tau;
   F32Plan plan;
   // workspace pieces
+  float* zc;           // [B, D] centre of each batch (the mean of its column points)
   float* xpack;        // [B, M, 2 Kp]
   float* rnorm;        // [B, M]
   float* ypack;        // [B, N, 2 Kp]

@@ -10,9 +10,10 @@
 // with B200's tensor cores: both products of the method -- the similarity
 // tile x.y^T and the value product P.v -- are split this way.
 //
-// The exponent.  With c = tau/2 * log2 e and the points centred at z = x[b, 0]
-// (x' = x - z, y' = y - z, which leaves every |x - y| unchanged and keeps the
-// norms small for clouds far from the origin),
+// The exponent.  With c = tau/2 * log2 e and the points centred at z, the mean
+// of the batch's column points (x' = x - z, y' = y - z: every |x - y| is
+// unchanged, and the norms stay at the scale of the cloud of columns, so the
+// expanded form below loses little to cancellation for the rows near them),
 //     exp(-tau/2 |x_i - y_j|^2) = 2^(2c x'_i.y'_j + r_i + q_j),
 //     r_i = -c |x'_i|^2,  q_j = -c |y'_j|^2
 // (the norm factors of Algorithm 1 on the same page).  P_ij = ex2(fma(S, 2c, r_i) + q_j)
@@ -54,7 +55,8 @@ constexpr int kAtom = kBM * 128;   // one 128-row x 32-float (128-byte) swizzle 
 struct F32KParams {
   const float* xpack;   // [B, M, 2 K'] packed rows (copied into TMEM when it has room)
   const float* rnorm;   // [B, M]
-  float* out;
+  float* out;           // sums; log-sum-exp: the shifts m (log2 units)
+  float* out_l;         // log-sum-exp: the scaled sums l (sum = 2^m l)
   int64_t split_stride;
   int64_t M, N;
   int64_t ldo;
@@ -109,7 +111,7 @@ struct F32Cfg {
   static constexpr int NST_FIT = (BUDGET - X_BYTES) / STAGE;
   static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
   static constexpr int NBARS = 2 * NST + 10;
-  static constexpr int RED_BYTES = kBM * 16;            // warpgroup 1 partial sums
+  static constexpr int RED_BYTES = kBM * 32;            // warpgroup 1 partial sums (m, l)
   static constexpr int SMEM_RAW = 1024 + X_BYTES + NST * STAGE + 8 * NBARS + 16 + RED_BYTES;
   // at least ~120 KB: one CTA per SM, so the 512-column TMEM allocation never waits
   static constexpr int SMEM = SMEM_RAW < 122880 ? 122880 : SMEM_RAW;
@@ -157,13 +159,18 @@ __device__ __forceinline__ float tf32_round(float v) {
 // Named barrier of the two exp warpgroups (warps 2-9).
 __device__ __forceinline__ void exp_warps_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
-template <int KA, int MODE>
+// LSE (register values, one channel): per row, the log-sum-exp of
+// t_ij + log2 w_j as a running maximum m and a sum l of 2^(t - m), updated per
+// 32-column chunk (the maximum of the chunk first, then its shifted sum), so
+// that no value under- or overflows.
+template <int KA, int MODE, bool LSE>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_f32_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                   const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmV,
                   const F32KParams p) {
   using Cfg = F32Cfg<KA, MODE>;
   constexpr bool REG = Cfg::REG;
+  static_assert(REG || !LSE, "log-sum-exp runs on the register path");
   constexpr int CP = Cfg::CP;
   constexpr int NST = Cfg::NST;
   constexpr int BN = Cfg::BN;
@@ -374,7 +381,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tPh = tmem + lane_base + Cfg::col_phi(h);
     const uint32_t tPl = tmem + lane_base + Cfg::col_plo(h);
     const float two_c = p.two_c;
-    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f;   // register values: running row sums
+    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f;   // register values: running row sums (l for LSE)
+    float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY;   // LSE: running maxima
     if constexpr (Cfg::XT) {
       if (h == 0) {
         // this thread's packed row (zeros past M) into its TMEM lane
@@ -437,19 +445,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             mbar_arrive(bar_f(h));
           }
+          if constexpr (!LSE) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int j = ch * 32 + e;
-            if constexpr (MODE == 1) {
-              // (norm, value): the first half of the column's 16 bytes
-              const float2 q = reinterpret_cast<const float2*>(qw)[2 * j];
-              p0 = fmaf(ex2(cur[e] + q.x), q.y, p0);
-            } else {
-              const float4 q = qw[j];
-              const float pe = ex2(cur[e] + q.x);
-              p0 = fmaf(pe, q.y, p0);
-              p1 = fmaf(pe, q.z, p1);
-              p2 = fmaf(pe, q.w, p2);
+            for (int e = 0; e < 32; ++e) {
+              const int j = ch * 32 + e;
+              if constexpr (MODE == 1) {
+                // (norm, value): the first half of the column's 16 bytes
+                const float2 q = reinterpret_cast<const float2*>(qw)[2 * j];
+                p0 = fmaf(ex2(cur[e] + q.x), q.y, p0);
+              } else {
+                const float4 q = qw[j];
+                const float pe = ex2(cur[e] + q.x);
+                p0 = fmaf(pe, q.y, p0);
+                p1 = fmaf(pe, q.z, p1);
+                p2 = fmaf(pe, q.w, p2);
+              }
+            }
+          } else {
+            // lanes 1.. of qw hold log2 w: u = t + log2 w per channel
+            auto lse_channel = [&](int lanec, float& m, float& l) {
+              float cm = -INFINITY;
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                cm = fmaxf(cm, cur[e] + reinterpret_cast<const float*>(qw + ch * 32 + e)[lanec]);
+              const float mn = fmaxf(m, cm);
+              if (mn != -INFINITY) {
+                float cs = 0.f;
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                  cs += ex2(cur[e] + reinterpret_cast<const float*>(qw + ch * 32 + e)[lanec] - mn);
+                l = fmaf(l, ex2(m - mn), cs);   // m = -inf: l = 0 and ex2(-inf) = 0
+                m = mn;
+              }
+            };
+#pragma unroll
+            for (int e = 0; e < 32; ++e) cur[e] += qw[ch * 32 + e].x;
+            lse_channel(1, mx0, acc0);
+            if constexpr (MODE > 1) {
+              lse_channel(2, mx1, acc1);
+              lse_channel(3, mx2, acc2);
             }
           }
           if (ch + 1 < NCH) {
@@ -458,9 +492,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             reg_fence32(cs);
           }
         }
-        acc0 += p0;
-        acc1 += p1;
-        acc2 += p2;
+        if constexpr (!LSE) {   // (log-sum-exp: the running (m, l) are mx*, acc*)
+          acc0 += p0;
+          acc1 += p1;
+          acc2 += p2;
+        }
         mbar_arrive(bar_empty(st));
       } else {
         // the whole S tile into registers; then its TMEM columns may be reused
@@ -504,16 +540,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if constexpr (REG) {
-      // warpgroup 1 hands its row sums to warpgroup 0 (both reach this barrier)
-      if (h == 1) red[row] = make_float4(acc0, acc1, acc2, 0.f);
+      // warpgroup 1 hands its row sums (or its (m, l)) to warpgroup 0; both
+      // reach this barrier
+      if (h == 1) {
+        red[2 * row] = make_float4(acc0, acc1, acc2, 0.f);
+        red[2 * row + 1] = make_float4(mx0, mx1, mx2, 0.f);
+      }
       exp_warps_sync();
       if (h == 0 && valid && ok && !*abort_flag) {
-        const float4 o = red[row];
-        float* orow = p.out + static_cast<int64_t>(blockIdx.y) * p.split_stride +
-                      (b * p.M + i) * p.ldo + p.c0;
-        orow[0] = acc0 + o.x;
-        if (p.cw > 1) orow[1] = acc1 + o.y;
-        if (p.cw > 2) orow[2] = acc2 + o.z;
+        const float4 o = red[2 * row];
+        const int64_t at = static_cast<int64_t>(blockIdx.y) * p.split_stride +
+                           (b * p.M + i) * p.ldo + p.c0;
+        if constexpr (!LSE) {
+          float* orow = p.out + at;
+          orow[0] = acc0 + o.x;
+          if (p.cw > 1) orow[1] = acc1 + o.y;
+          if (p.cw > 2) orow[2] = acc2 + o.z;
+        } else {
+          const float4 om = red[2 * row + 1];
+          auto merge = [&](int c, float m0, float l0, float m1, float l1) {
+            const float m = fmaxf(m0, m1);
+            float l = 0.f;
+            if (m != -INFINITY) l = l0 * ex2(m0 - m) + l1 * ex2(m1 - m);
+            p.out[at + c] = m;
+            p.out_l[at + c] = l;
+          };
+          merge(0, mx0, acc0, om.x, o.x);
+          if (p.cw > 1) merge(1, mx1, acc1, om.y, o.y);
+          if (p.cw > 2) merge(2, mx2, acc2, om.z, o.z);
+        }
       }
     } else {
       if (ok) ok = wait_bar(bar_o, 0, abort_flag);
@@ -556,52 +611,84 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ packing prologue
+// z[b, :] = the mean of y[b, :, :] over its N points (fixed summation order:
+// warp w of a block takes points w, w + 8, ...; lanes take features).
+__global__ void column_mean_kernel(const float* __restrict__ y, float* __restrict__ z, int64_t N,
+                                   int D) {
+  __shared__ float part[8][32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t b = blockIdx.x;
+  const int k = blockIdx.y * 32 + lane;
+  float acc = 0.f;
+  if (k < D)
+    for (int64_t j = w; j < N; j += 8) acc += y[(b * N + j) * D + k];
+  part[w][lane] = acc;
+  __syncthreads();
+  if (w == 0 && k < D) {
+    float t = 0.f;
+    for (int q = 0; q < 8; ++q) t += part[q][lane];
+    z[b * D + k] = N > 0 ? t / static_cast<float>(N) : 0.f;
+  }
+}
+
 // Packed operand rows [hi (K') | lo (K')] of the centred points v' = v - z,
-// z = rows[b, 0, :], and the norm term -c |v'|^2: for the row side into
+// z = zc[b, :], and the norm term -c |v'|^2: for the row side into
 // norm[b * R + r]; for the column side into norm[(b * Rpad + r) * 4] (lanes
-// 1-3 zeroed) with -inf for the padding columns r >= R.  One thread per row.
-__global__ void pack_rows_f32_kernel(const float* __restrict__ src, const float* __restrict__ rows,
+// 1-3 zeroed) with -inf for the padding columns r >= R.  One warp per row,
+// lanes along the features (coalesced reads and writes).
+__global__ void pack_rows_f32_kernel(const float* __restrict__ src, const float* __restrict__ zc,
                                      float* __restrict__ dst, float* __restrict__ norm, int64_t B,
-                                     int64_t R, int64_t Rpad, int64_t Mrows, int D, int Kp,
-                                     float c, int norm_stride) {
+                                     int64_t R, int64_t Rpad, int D, int Kp, float c,
+                                     int norm_stride) {
+  const int lane = threadIdx.x & 31;
   const int64_t total = B * Rpad;
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+  const int64_t wstride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
+       e < total; e += wstride) {
     const int64_t b = e / Rpad, rr = e % Rpad;
     float* nrm = norm + e * norm_stride;
-    if (norm_stride == 4) nrm[1] = nrm[2] = nrm[3] = 0.f;
     if (rr >= R) {
-      nrm[0] = -INFINITY;   // padding columns: kernel value 0
+      if (lane == 0) {
+        nrm[0] = -INFINITY;   // padding columns: kernel value 0
+        if (norm_stride == 4) nrm[1] = nrm[2] = nrm[3] = 0.f;
+      }
       continue;
     }
     const float* v = src + (b * R + rr) * D;
-    const float* z = rows + b * Mrows * D;
+    const float* z = zc + b * D;
     float* out = dst + (b * R + rr) * (2 * static_cast<int64_t>(Kp));
     float sq = 0.f;
-    for (int k = 0; k < Kp; ++k) {
-      float d = 0.f;
-      if (k < D) d = v[k] - z[k];
+    for (int k = lane; k < Kp; k += 32) {
+      const float d = (k < D) ? v[k] - z[k] : 0.f;
       sq = fmaf(d, d, sq);
       const float hi = tf32_round(d);
       out[k] = hi;
       out[Kp + k] = tf32_round(d - hi);
     }
-    nrm[0] = -c * sq;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    if (lane == 0) {
+      nrm[0] = -c * sq;
+      if (norm_stride == 4) nrm[1] = nrm[2] = nrm[3] = 0.f;
+    }
   }
 }
 
-// Register-path values: channels [0, CV) (CV <= 3) of the pass's values
-// (values.cuh) into lanes 1.. of qw[b, j, :].
+// Register-path values: channels [c0, c0 + cw) (cw <= 3) of the pass's values
+// (values.cuh) into lanes 1.. of qw[b, j, :]; for the log-sum-exp, their
+// base-2 logarithms.
 __global__ void pack_values_qw_kernel(const float* __restrict__ w, const float* __restrict__ y,
                                       const float* __restrict__ rows, float* __restrict__ qw,
                                       int64_t B, int64_t N, int64_t Nq, int64_t Mrows, int C, int D,
-                                      int CV) {
+                                      int c0, int cw, int log2_values) {
   const int64_t total = B * N;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t b = e / N, j = e % N;
-    for (int ch = 0; ch < CV; ++ch)
-      qw[(b * Nq + j) * 4 + 1 + ch] = value_at(w, y, rows, b, e, Mrows, D, C, ch, C);
+    for (int ch = 0; ch < cw; ++ch) {
+      const float v = value_at(w, y, rows, b, e, Mrows, D, C, c0 + ch, C);
+      qw[(b * Nq + j) * 4 + 1 + ch] = log2_values ? lg2(v) : v;
+    }
   }
 }
 
@@ -639,10 +726,10 @@ struct TileMaps {
   CUtensorMap x, y, q, v;
 };
 
-template <int KA, int MODE>
+template <int KA, int MODE, bool LSE = false>
 cudaError_t launch_kernel(const TileMaps& m, const F32KParams& kp, dim3 grid, cudaStream_t s) {
   using Cfg = F32Cfg<KA, MODE>;
-  auto fn = tc_f32_kernel<KA, MODE>;
+  auto fn = tc_f32_kernel<KA, MODE, LSE>;
   static bool attr_done = false;   // idempotent; a benign race at worst repeats the call
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
@@ -654,8 +741,9 @@ cudaError_t launch_kernel(const TileMaps& m, const F32KParams& kp, dim3 grid, cu
 }
 
 template <int KA>
-cudaError_t launch_mode(int mode, const TileMaps& m, const F32KParams& kp, dim3 grid,
+cudaError_t launch_mode(int mode, bool lse, const TileMaps& m, const F32KParams& kp, dim3 grid,
                         cudaStream_t s) {
+  if (lse) return launch_kernel<KA, 1, true>(m, kp, grid, s);   // one channel per pass
   switch (mode) {
     case 1: return launch_kernel<KA, 1>(m, kp, grid, s);
     case 3: return launch_kernel<KA, 3>(m, kp, grid, s);
@@ -684,8 +772,6 @@ int tile_cols_ka(int mode) {
   }
 }
 
-// Register values for at most 3 channels, else tensor-core chunks.
-int mode_for(int CV, int cw) { return CV <= 3 ? (CV == 1 ? 1 : 3) : f32_chunk_pad(cw); }
 
 }  // namespace
 
@@ -737,19 +823,18 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
   const int64_t Nq = (a.N + 127) / 128 * 128;
   const float* x = static_cast<const float*>(a.x);
   const float* y = static_cast<const float*>(a.y);
-  pack_rows_f32_kernel<<<grid_for(a.B * a.M, 128), 128, 0, s>>>(x, x, a.xpack, a.rnorm, a.B, a.M,
-                                                               a.M, a.M, a.D, Kp, c, 1);
-  pack_rows_f32_kernel<<<grid_for(a.B * Nq, 128), 128, 0, s>>>(y, x, a.ypack, a.qw, a.B, a.N, Nq,
-                                                              a.M, a.D, Kp, c, 4);
+  column_mean_kernel<<<dim3(static_cast<unsigned>(a.B), static_cast<unsigned>((a.D + 31) / 32)),
+                       256, 0, s>>>(y, a.zc, a.N, a.D);
+  // one warp per row, 8 rows per 256-thread block
+  pack_rows_f32_kernel<<<grid_for(a.B * a.M, 8), 256, 0, s>>>(x, a.zc, a.xpack, a.rnorm, a.B, a.M,
+                                                             a.M, a.D, Kp, c, 1);
+  pack_rows_f32_kernel<<<grid_for(a.B * Nq, 8), 256, 0, s>>>(y, a.zc, a.ypack, a.qw, a.B, a.N, Nq,
+                                                            a.D, Kp, c, 4);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const bool reg = a.CV <= 3;
-  if (reg) {
-    pack_values_qw_kernel<<<grid_for(a.B * a.N, 256), 256, 0, s>>>(a.w, y, x, a.qw, a.B, a.N, Nq,
-                                                                   a.M, a.C, a.D, a.CV);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
+  // register values for at most 3 channels per pass; the log-sum-exp one
+  // channel per pass
+  const bool reg = a.lse || a.CV <= 3;
   TileMaps m;
   const uint64_t rowf = 2ull * Kp;
   if (!make_tmap_3d(&m.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.xpack, rowf, a.M, a.B, rowf * 4,
@@ -759,10 +844,16 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
   const int64_t Nst = (a.N + 3) / 4 * 4;
   const dim3 grid(static_cast<unsigned>((a.M + kBM - 1) / kBM), static_cast<unsigned>(a.plan.splits),
                   static_cast<unsigned>(a.B));
-  const int chunk = reg ? a.CV : a.plan.max_chunk;
+  const int chunk = a.lse ? 1 : (reg ? 3 : a.plan.max_chunk);
   for (int c0 = 0; c0 < a.CV; c0 += chunk) {
     const int cw = (a.CV - c0) < chunk ? (a.CV - c0) : chunk;
-    const int mode = mode_for(a.CV, cw);
+    const int mode = reg ? (cw == 1 ? 1 : 3) : f32_chunk_pad(cw);
+    if (reg) {
+      pack_values_qw_kernel<<<grid_for(a.B * a.N, 256), 256, 0, s>>>(
+          a.w, y, x, a.qw, a.B, a.N, Nq, a.M, a.C, a.D, c0, cw, a.lse ? 1 : 0);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
     const int BN = f32_tile_cols(KA, mode);
     if (BN != 32 && BN != 64 && BN != 128) return cudaErrorInvalidValue;
     if (!make_tmap_3d(&m.y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.ypack, rowf, a.N, a.B, rowf * 4,
@@ -787,6 +878,7 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
     kp.xpack = a.xpack;
     kp.rnorm = a.rnorm;
     kp.out = a.out;
+    kp.out_l = a.out_l;
     kp.split_stride = a.split_stride;
     kp.M = a.M;
     kp.N = a.N;
@@ -800,11 +892,11 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
     kp.bn = BN;
     kp.two_c = a.tau * kLog2e;
     switch (KA) {
-      case 1: e = launch_mode<1>(mode, m, kp, grid, s); break;
-      case 2: e = launch_mode<2>(mode, m, kp, grid, s); break;
-      case 4: e = launch_mode<4>(mode, m, kp, grid, s); break;
-      case 6: e = launch_mode<6>(mode, m, kp, grid, s); break;
-      default: e = launch_mode<8>(mode, m, kp, grid, s); break;
+      case 1: e = launch_mode<1>(mode, a.lse, m, kp, grid, s); break;
+      case 2: e = launch_mode<2>(mode, a.lse, m, kp, grid, s); break;
+      case 4: e = launch_mode<4>(mode, a.lse, m, kp, grid, s); break;
+      case 6: e = launch_mode<6>(mode, a.lse, m, kp, grid, s); break;
+      default: e = launch_mode<8>(mode, a.lse, m, kp, grid, s); break;
     }
     if (e != cudaSuccess) return e;
   }

@@ -12,11 +12,16 @@ round-to-nearest-even cast to the workload's dtype):
 * ``d3_1m_lse``: x, y ~ U[0, 1)^3, w ~ U(0.5, 1.5), tau = 100
 * ``d32_c32``: x, y ~ N(0, 1/D)^D (coordinate variance 1/D), w ~ N(0, 1), tau = 1
 * ``d32_c1_bwd``: as ``d32_c32`` with C = 1, plus an upstream gradient g ~ N(0, 1)
+* ``b64_d32_f16`` / ``b64_d32_f32`` / ``b64_d128_f32``: B = 64, M = N = 16384, C = 1,
+  x, y ~ N(0, 1/D)^D, w ~ N(0, 1), tau = 1 -- points of the D sweeps (fp16 and fp32)
+* ``d32_c32_f32``: ``d32_c32`` in fp32 -- a point of the fp32 N sweep
 
 The shapes are those of the Gaussian-product runs of "Kernel matrix reduction"
 (Variants: D = 3, float32, 10k / 100k / 1M points) and of the sweeps in the
-figures of "Fast Gauss Sums via Flash Attention" (B = 4, D = 32, C = 32 or 1,
-fp16).  No dataset is involved.
+figures of "Fast Gauss Sums via Flash Attention" (Figures 1-2: B = 4, D = 32,
+C = 32 or 1, fp16; Figures 3-4: D sweeps at B = 64, C = 1, N = 16384 in fp16 and
+fp32; Figure 5: an N sweep at B = 4, D = 32, C = 32 in fp32).  No dataset is
+involved.
 """
 from dataclasses import dataclass
 
@@ -59,6 +64,14 @@ WORKLOADS = {
                 "normal1"),
     5: Workload(5, "d32_c1_bwd", ("sum", "bwd"), 4, 16_384, 16_384, 32, 1, "f16", 1.0,
                 "normal_invD", "normal1", with_g=True),
+    6: Workload(6, "b64_d32_f16", ("sum",), 64, 16_384, 16_384, 32, 1, "f16", 1.0,
+                "normal_invD", "normal1"),
+    7: Workload(7, "b64_d32_f32", ("sum",), 64, 16_384, 16_384, 32, 1, "f32", 1.0,
+                "normal_invD", "normal1"),
+    8: Workload(8, "b64_d128_f32", ("sum",), 64, 16_384, 16_384, 128, 1, "f32", 1.0,
+                "normal_invD", "normal1"),
+    9: Workload(9, "d32_c32_f32", ("sum",), 4, 65_536, 65_536, 32, 32, "f32", 1.0,
+                "normal_invD", "normal1"),
 }
 BY_NAME = {w.name: w for w in WORKLOADS.values()}
 

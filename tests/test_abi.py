@@ -71,10 +71,12 @@ def test_lse_has_no_half_precision_path():
     assert _fwd("gauss_lse_fwd", dt=1, D=32) == 2
 
 
-def test_lse_and_knn_stay_on_the_small_d_path():
-    # the split-tf32 path (fp32, D > 8) serves the Gauss-sum passes only
-    assert _fwd("gauss_lse_fwd", D=9) == 2
-    assert _fwd("gauss_sum_fwd", D=9) == 4        # supported: asks for its workspace
+def test_fp32_wide_features_route_to_the_tensor_core_path():
+    # fp32 with D > 8 (split-tf32 tensor cores): sums and the log-sum-exp are
+    # supported (they ask for their workspace); the log-sum-exp backward and
+    # kNN stay on the small-D path
+    assert _fwd("gauss_lse_fwd", D=9) == 4
+    assert _fwd("gauss_sum_fwd", D=9) == 4
     lib = gs.library()
     i64 = ctypes.c_void_p(0x100000)
     assert lib.gauss_knn(FAKE, FAKE, FAKE, i64, 1, 10, 10, 9, 1, 0, NULL, 0, NULL) == 2
@@ -103,8 +105,9 @@ def test_workspace_query():
     assert ws(gs.GS_OP_SUM, 1, 1000, 1000, 9, 1, gs.GS_F32) >= 2 * 1000 * 2 * 16 * 4
     with pytest.raises(ValueError):
         ws(gs.GS_OP_SUM, 1, 10, 10, 129, 1, gs.GS_F32)
+    assert ws(gs.GS_OP_LSE, 1, 1000, 1000, 9, 1, gs.GS_F32) >= 2 * 1000 * 2 * 16 * 4
     with pytest.raises(ValueError):
-        ws(gs.GS_OP_LSE, 1, 10, 10, 9, 1, gs.GS_F32)
+        ws(gs.GS_OP_LSE_BWD, 1, 10, 10, 9, 1, gs.GS_F32)
     with pytest.raises(ValueError):
         ws(7, 1, 10, 10, 3, 1, gs.GS_F32)
 

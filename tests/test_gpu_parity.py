@@ -170,6 +170,37 @@ def test_lse_f32_shapes(shape):
     assert rel_l2(np.exp(out), np.exp(ref)) <= TOL["f32"]
 
 
+@pytest.mark.parametrize("shape,tau", [((1, 300, 700, 16, 1), 1.0), ((2, 200, 500, 32, 2), 1.0),
+                                       ((1, 130, 1000, 100, 1), 1.0), ((1, 257, 900, 24, 3), 30.0)])
+def test_lse_f32_tensor_core_shapes(shape, tau):
+    """fp32 with D > 8: the log-sum-exp on the split-tf32 path (running maximum)."""
+    B, M, N, D, C = shape
+    inp = synth.make_inputs(3, seed=41, B=B, M=M, N=N, D=D, C=C)
+    inp["x"] = (inp["x"].double() / D ** 0.5).float()   # unit-scale clouds in D dimensions
+    inp["y"] = (inp["y"].double() / D ** 0.5).float()
+    d = dev(inp)
+    out = gs().gauss_lse_fwd(d["x"], d["y"], d["w"], tau).cpu().numpy()
+    ref = oracle.gauss_lse(f64(inp, "x"), f64(inp, "y"), f64(inp, "w"), tau)
+    assert rel_l2(out, ref) <= TOL["f32"], rel_l2(out, ref)
+    assert rel_l2(np.exp(out), np.exp(ref)) <= TOL["f32"]
+
+
+def test_lse_f32_tensor_core_rows_far_from_every_point():
+    """Rows whose every kernel value underflows fp32 (exp(-tau/2 d^2) ~ e^-5000):
+    the running maximum keeps the log-sum-exp finite and exact."""
+    inp = synth.make_inputs(3, seed=42, B=1, M=64, N=600, D=20, C=1)
+    x = inp["x"].double()
+    x[0, :32] += 100.0
+    inp["x"] = x.float()
+    d = dev(inp)
+    out = gs().gauss_lse_fwd(d["x"], d["y"], d["w"], 1.0).cpu().numpy()
+    ref = oracle.gauss_lse(f64(inp, "x"), f64(inp, "y"), f64(inp, "w"), 1.0)
+    assert np.isfinite(out).all()
+    assert rel_l2(out, ref) <= TOL["f32"], rel_l2(out, ref)
+    # the rows near the cloud, on the stricter exp scale
+    assert rel_l2(np.exp(out[:, 32:]), np.exp(ref[:, 32:])) <= TOL["f32"]
+
+
 def test_lse_rows_far_from_every_point():
     """Rows whose every kernel value underflows fp32 take the exact per-row
     recompute; the result must still match the oracle's shifted evaluation."""
