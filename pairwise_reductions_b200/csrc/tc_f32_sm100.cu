@@ -11,9 +11,10 @@
 // tile x.y^T and the value product P.v -- are split this way.
 //
 // The exponent.  With c = tau/2 * log2 e and the points centred at z, the mean
-// of the batch's column points (x' = x - z, y' = y - z: every |x - y| is
-// unchanged, and the norms stay at the scale of the cloud of columns, so the
-// expanded form below loses little to cancellation for the rows near them),
+// of a strided sample of the batch's column points (x' = x - z, y' = y - z:
+// every |x - y| is unchanged, and the norms stay at the scale of the cloud of
+// columns, so the expanded form below loses little to cancellation for the
+// rows near them),
 //     exp(-tau/2 |x_i - y_j|^2) = 2^(2c x'_i.y'_j + r_i + q_j),
 //     r_i = -c |x'_i|^2,  q_j = -c |y'_j|^2
 // (the norm factors of Algorithm 1 on the same page).  P_ij = ex2(fma(S, 2c, r_i) + q_j)
@@ -611,23 +612,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ packing prologue
-// z[b, :] = the mean of y[b, :, :] over its N points (fixed summation order:
-// warp w of a block takes points w, w + 8, ...; lanes take features).
+// z[b, :] = the mean of the column points y[b, s * stride, :], s < S, with
+// S = min(N, 1024) and stride = N / S (any centre is exact; a sample mean
+// costs little and is not thrown off by one outlying point).  Fixed summation
+// order: warp w of the block takes samples w, w + 8, ...; lanes take features.
 __global__ void column_mean_kernel(const float* __restrict__ y, float* __restrict__ z, int64_t N,
                                    int D) {
   __shared__ float part[8][32];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int64_t b = blockIdx.x;
   const int k = blockIdx.y * 32 + lane;
+  const int64_t S = N < 1024 ? N : 1024;
+  const int64_t stride = S > 0 ? N / S : 1;
   float acc = 0.f;
   if (k < D)
-    for (int64_t j = w; j < N; j += 8) acc += y[(b * N + j) * D + k];
+    for (int64_t q = w; q < S; q += 8) acc += y[(b * N + q * stride) * D + k];
   part[w][lane] = acc;
   __syncthreads();
   if (w == 0 && k < D) {
     float t = 0.f;
     for (int q = 0; q < 8; ++q) t += part[q][lane];
-    z[b * D + k] = N > 0 ? t / static_cast<float>(N) : 0.f;
+    z[b * D + k] = S > 0 ? t / static_cast<float>(S) : 0.f;
   }
 }
 
