@@ -56,18 +56,30 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-launch-count", action="store_true",
                     help="skip the profiler-based kernel count (use under ncu)")
+    ap.add_argument("--sharded", action="store_true",
+                    help="one problem of the workload's size split over the ranks by rows and "
+                         "sources (strong scaling; the sources are all-gathered every step)")
     return ap.parse_args()
 
 
 # ------------------------------------------------------------------ distributed plumbing
-def dist_init(n_gpus):
+def dist_init(n_gpus, need_group=False):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world != n_gpus:
         raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
     pg = None
-    if world > 1:
+    if world > 1 or need_group:
+        if world == 1:   # a one-rank group, for the collectives of the sharded mode
+            import socket
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            if "MASTER_PORT" not in os.environ:
+                with socket.socket() as sk:
+                    sk.bind(("127.0.0.1", 0))
+                    os.environ["MASTER_PORT"] = str(sk.getsockname()[1])
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
         import datetime
         import torch.distributed as dist
         backend = "nccl" if torch.cuda.is_available() else "gloo"
@@ -147,6 +159,36 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ workloads
+def sharded_step_fn(w, d):
+    """One pass of the hot path for this rank's shard of one problem."""
+    from pairwise_reductions_b200 import sharded
+    tau = d["tau"]
+
+    def run():
+        if "sum" in w.ops:
+            d["out_sum"] = sharded.sharded_sum_fwd(d["x"], d["y"], d["w"], tau)
+        if "lse" in w.ops:
+            d["out_lse"] = sharded.sharded_lse_fwd(d["x"], d["y"], d["w"], tau)
+        if "bwd" in w.ops:
+            sharded.sharded_sum_bwd(d["x"], d["y"], d["w"], d["g"], tau)
+    return run
+
+
+def shard_of(inp, rank, world):
+    """Contiguous row and source slices of the whole problem for this rank."""
+    def sl(n):
+        lo = n * rank // world
+        return slice(lo, n * (rank + 1) // world)
+    rows, srcs = sl(inp["x"].shape[1]), sl(inp["y"].shape[1])
+    out = dict(inp)
+    out["x"] = inp["x"][:, rows].contiguous()
+    out["y"] = inp["y"][:, srcs].contiguous()
+    out["w"] = inp["w"][:, srcs].contiguous()
+    if "g" in inp:
+        out["g"] = inp["g"][:, rows].contiguous()
+    return out
+
+
 def step_fn(gs, w, d, ws, outs):
     """Return a closure running one pass of the workload's hot path."""
     tau = d["tau"]
@@ -281,12 +323,15 @@ def main():
     w = synth.BY_NAME[args.workload]
     if args.impl == "reference":
         return reference_arm(args, w)
-    rank, world, local, pg = dist_init(args.gpus)
+    rank, world, local, pg = dist_init(args.gpus, need_group=args.sharded)
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
     import pairwise_reductions_b200 as gs
     dev = torch.device("cuda", local)
-    inp = synth.make_inputs(w, seed=(1000 + w.wid + 7919 * rank) if rank else None)
+    if args.sharded:   # one problem: the workload's own seed on every rank, then this rank's slice
+        inp = shard_of(synth.make_inputs(w), rank, world)
+    else:              # independent problems: a seed per rank
+        inp = synth.make_inputs(w, seed=(1000 + w.wid + 7919 * rank) if rank else None)
     d = {k: inp[k].to(dev) for k in ("x", "y", "w", "g") if k in inp}
     d["tau"] = inp["tau"]
     outs = {"sum": torch.empty(w.B, w.M, w.C, device=dev), "lse": torch.empty(w.B, w.M, w.C, device=dev)}
@@ -294,7 +339,7 @@ def main():
                    for op, name in ((gs.GS_OP_SUM, "sum"), (gs.GS_OP_LSE, "lse"), (gs.GS_OP_SUM_BWD, "bwd"))
                    if name in w.ops)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    run = step_fn(gs, w, d, ws, outs)
+    run = sharded_step_fn(w, d) if args.sharded else step_fn(gs, w, d, ws, outs)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -324,14 +369,15 @@ def main():
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(sum(step_ms), pg, dev)
     ms_per_step = total_ms / args.steps
-    evals = pair_evals(w)
-    value = evals * world * args.steps / (total_ms * 1e-3) / 1e9
+    evals = pair_evals(w)   # one problem's pairs per step
+    jobs = 1 if args.sharded else world   # problems the whole job solves per step
+    value = evals * jobs * args.steps / (total_ms * 1e-3) / 1e9
     if gs.last_device_error() != 0:
         raise SystemExit("device error word set during the timed loop")
 
     # ---- end to end through the public API: pinned host inputs -> device -> result -> host
     hx = {k: inp[k].pin_memory() for k in ("x", "y", "w", "g") if k in inp}
-    hout = torch.empty(w.B, w.M, w.C).pin_memory()
+    hout = torch.empty(w.B, inp["x"].shape[1], w.C).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in hx.values())
     d2h = hout.numel() * hout.element_size()
     e_s = torch.cuda.Event(enable_timing=True)
@@ -340,8 +386,13 @@ def main():
     def e2e_step():
         dd = {k: t.to(dev, non_blocking=True) for k, t in hx.items()}
         dd["tau"] = inp["tau"]
-        step_fn(gs, w, dd, ws, outs)()
-        hout.copy_(outs["lse" if "lse" in w.ops and "sum" not in w.ops else "sum"], non_blocking=True)
+        if args.sharded:
+            sharded_step_fn(w, dd)()
+            hout.copy_(dd["out_lse" if "lse" in w.ops and "sum" not in w.ops else "out_sum"],
+                       non_blocking=True)
+        else:
+            step_fn(gs, w, dd, ws, outs)()
+            hout.copy_(outs["lse" if "lse" in w.ops and "sum" not in w.ops else "sum"], non_blocking=True)
 
     e2e_ms, e2e_value = None, None
     if args.e2e_steps > 0:
@@ -355,7 +406,7 @@ def main():
         e_e.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e_s.elapsed_time(e_e), pg, dev) / args.e2e_steps
-        e2e_value = evals * world / (e2e_ms * 1e-3) / 1e9
+        e2e_value = evals * jobs / (e2e_ms * 1e-3) / 1e9
     clocks = clk.summary()
 
     if rank == 0:
@@ -368,7 +419,7 @@ def main():
             pass
         sm_max = float(clocks.get("sm_max_mhz") or peaks.get("sm_max_mhz") or 1965.0)
         peak = EX2_PER_CLK_PER_SM * sms * sm_max * 1e6 / 1e9
-        achieved = evals / (ms_per_step * 1e-3) / 1e9
+        achieved = evals * jobs / world / (ms_per_step * 1e-3) / 1e9   # pairs per GPU
         traffic, dom = traffic_per_launch(w)
         roof = {"bound": "alu", "kernel": f"{dom}: one MUFU ex2 per pair", "achieved": achieved,
                 "peak": peak, "unit": "G pairs/s", "frac": achieved / peak, "traffic": traffic,
@@ -381,13 +432,16 @@ def main():
         pub = PUBLISHED.get(w.name)
         line = {"metric": "Gaussian kernel-sum pairs/sec (G pairs/s)", "value": value,
                 "unit": "G pairs/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                "ms_per_step": ms_per_step, "higher_is_better": True,
+                "scaling": "strong" if args.sharded else "weak",
                 "vs_baseline": (value / pub["value"]) if pub else None,
                 "dtype": w.dtype, "data": "synthetic",
                 "config": {"workload": w.name, "B": w.B, "M": w.M, "N": w.N, "D": w.D, "C": w.C,
                            "tau": w.tau, "ops": list(w.ops), "pairs_per_step_per_gpu": evals,
                            "l2": "flushed by a 256 MiB write between timed steps",
-                           "parallelism": f"independent problems, {world} rank(s)"},
+                           "parallelism": (f"one problem sharded over {world} rank(s): rows and "
+                                           f"sources split, sources all-gathered each step")
+                           if args.sharded else f"independent problems, {world} rank(s)"},
                 "roofline": roof, "cpu_baseline": cpu,
                 "e2e": {"value": e2e_value, "unit": "G pairs/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
