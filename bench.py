@@ -159,18 +159,21 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ workloads
-def sharded_step_fn(w, d):
-    """One pass of the hot path for this rank's shard of one problem."""
+def sharded_step_fn(w, d, counts):
+    """One pass of the hot path for this rank's shard of one problem (counts: the
+    ranks' row and source counts, exchanged once before timing)."""
     from pairwise_reductions_b200 import sharded
     tau = d["tau"]
+    rc, sc = counts
 
     def run():
         if "sum" in w.ops:
-            d["out_sum"] = sharded.sharded_sum_fwd(d["x"], d["y"], d["w"], tau)
+            d["out_sum"] = sharded.sharded_sum_fwd(d["x"], d["y"], d["w"], tau, src_counts=sc)
         if "lse" in w.ops:
-            d["out_lse"] = sharded.sharded_lse_fwd(d["x"], d["y"], d["w"], tau)
+            d["out_lse"] = sharded.sharded_lse_fwd(d["x"], d["y"], d["w"], tau, src_counts=sc)
         if "bwd" in w.ops:
-            sharded.sharded_sum_bwd(d["x"], d["y"], d["w"], d["g"], tau)
+            sharded.sharded_sum_bwd(d["x"], d["y"], d["w"], d["g"], tau, row_counts=rc,
+                                    src_counts=sc)
     return run
 
 
@@ -339,7 +342,11 @@ def main():
                    for op, name in ((gs.GS_OP_SUM, "sum"), (gs.GS_OP_LSE, "lse"), (gs.GS_OP_SUM_BWD, "bwd"))
                    if name in w.ops)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    run = sharded_step_fn(w, d) if args.sharded else step_fn(gs, w, d, ws, outs)
+    counts = None
+    if args.sharded:
+        from pairwise_reductions_b200 import sharded
+        counts = (sharded.shard_counts(d["x"].shape[1], dev), sharded.shard_counts(d["y"].shape[1], dev))
+    run = sharded_step_fn(w, d, counts) if args.sharded else step_fn(gs, w, d, ws, outs)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -387,7 +394,7 @@ def main():
         dd = {k: t.to(dev, non_blocking=True) for k, t in hx.items()}
         dd["tau"] = inp["tau"]
         if args.sharded:
-            sharded_step_fn(w, dd)()
+            sharded_step_fn(w, dd, counts)()
             hout.copy_(dd["out_lse" if "lse" in w.ops and "sum" not in w.ops else "out_sum"],
                        non_blocking=True)
         else:

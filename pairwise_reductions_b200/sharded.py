@@ -15,7 +15,9 @@ over NVLink for CUDA tensors); the pair work runs in this library's kernels
 size; they are concatenated in rank order.
 
 `kernels` replaces the three compute calls (same signatures); the default is
-the CUDA library.
+the CUDA library.  `row_counts` / `src_counts` (every rank's number of rows /
+sources, from `shard_counts`) spare each gather the exchange of the counts and
+its host synchronisation; without them the counts are exchanged every call.
 """
 import torch
 import torch.distributed as dist
@@ -26,17 +28,26 @@ def _default_kernels():
     return {"sum": gauss_sum_fwd, "lse": gauss_lse_fwd, "bwd": gauss_sum_bwd}
 
 
-def all_gather_rows(t, group=None):
-    """Concatenate every rank's t [B, n_r, ...] along dim 1, in rank order.
-
-    Shards may have different n_r: the counts are exchanged first, every shard
-    is padded to the largest, gathered, and trimmed.
-    """
+def shard_counts(n_local, device, group=None):
+    """Every rank's n_local, in rank order (one small all-gather and a host sync)."""
     world = dist.get_world_size(group)
-    n = torch.tensor([t.shape[1]], dtype=torch.int64, device=t.device)
+    n = torch.tensor([n_local], dtype=torch.int64, device=device)
     counts = [torch.zeros_like(n) for _ in range(world)]
     dist.all_gather(counts, n, group=group)
-    counts = [int(c.item()) for c in counts]
+    return [int(c.item()) for c in counts]
+
+
+def all_gather_rows(t, group=None, counts=None):
+    """Concatenate every rank's t [B, n_r, ...] along dim 1, in rank order.
+
+    Shards may have different n_r (`counts`, exchanged here when not given):
+    every shard is padded to the largest, gathered, and trimmed.
+    """
+    world = dist.get_world_size(group)
+    if counts is None:
+        counts = shard_counts(t.shape[1], t.device, group)
+    if len(counts) != world or counts[dist.get_rank(group)] != t.shape[1]:
+        raise ValueError("counts do not match the group or this rank's shard")
     nmax = max(counts)
     pad = t
     if t.shape[1] < nmax:
@@ -48,30 +59,41 @@ def all_gather_rows(t, group=None):
     return torch.cat([p[:, :c] for p, c in zip(parts, counts)], dim=1).contiguous()
 
 
-def sharded_sum_fwd(x, y, w, tau, group=None, kernels=None):
+def sharded_sum_fwd(x, y, w, tau, group=None, kernels=None, src_counts=None):
     """Rows x of this rank against the sources of every rank: [B, M_r, C] float32."""
     k = kernels or _default_kernels()
-    return k["sum"](x, all_gather_rows(y, group), all_gather_rows(w, group), tau)
+    if src_counts is None:
+        src_counts = shard_counts(y.shape[1], y.device, group)
+    return k["sum"](x, all_gather_rows(y, group, src_counts), all_gather_rows(w, group, src_counts),
+                    tau)
 
 
-def sharded_lse_fwd(x, y, w, tau, group=None, kernels=None):
+def sharded_lse_fwd(x, y, w, tau, group=None, kernels=None, src_counts=None):
     """Log-sum-exp of this rank's rows against the sources of every rank."""
     k = kernels or _default_kernels()
-    return k["lse"](x, all_gather_rows(y, group), all_gather_rows(w, group), tau)
+    if src_counts is None:
+        src_counts = shard_counts(y.shape[1], y.device, group)
+    return k["lse"](x, all_gather_rows(y, group, src_counts), all_gather_rows(w, group, src_counts),
+                    tau)
 
 
-def sharded_sum_bwd(x, y, w, g, tau, group=None, kernels=None):
+def sharded_sum_bwd(x, y, w, g, tau, group=None, kernels=None, row_counts=None, src_counts=None):
     """(dL/dx for this rank's rows, dL/dw for this rank's sources) of L = <g, sum>.
 
     dL/dx_i sums over every source (all-gathered y, w); dL/dw_j sums over every
     row (all-gathered x, g).
     """
     k = kernels or _default_kernels()
-    gx, _ = k["bwd"](x, all_gather_rows(y, group), all_gather_rows(w, group), g, tau,
-                     want_x=True, want_w=False)
-    _, gw = k["bwd"](all_gather_rows(x, group), y, w, all_gather_rows(g, group), tau,
-                     want_x=False, want_w=True)
+    if src_counts is None:
+        src_counts = shard_counts(y.shape[1], y.device, group)
+    if row_counts is None:
+        row_counts = shard_counts(x.shape[1], x.device, group)
+    gx, _ = k["bwd"](x, all_gather_rows(y, group, src_counts), all_gather_rows(w, group, src_counts),
+                     g, tau, want_x=True, want_w=False)
+    _, gw = k["bwd"](all_gather_rows(x, group, row_counts), y, w,
+                     all_gather_rows(g, group, row_counts), tau, want_x=False, want_w=True)
     return gx, gw
 
 
-__all__ = ["all_gather_rows", "sharded_sum_fwd", "sharded_lse_fwd", "sharded_sum_bwd"]
+__all__ = ["shard_counts", "all_gather_rows", "sharded_sum_fwd", "sharded_lse_fwd",
+           "sharded_sum_bwd"]
