@@ -20,12 +20,19 @@
  *     g    [B, M, C]   float32 upstream gradient (backward only)
  *
  * Supported shapes and types:
- *     GS_F32           : 1 <= D <= 8 (CUDA-core path), any C >= 1
+ *     GS_F32           : 1 <= D <= 8 (CUDA-core path), any C >= 1;
+ *                        9 <= D <= 128 (tensor-core path at fp32 accuracy:
+ *                        every operand split into tf32 hi + lo, three tf32
+ *                        MMAs per product) for the sums, their gradients,
+ *                        the diffusion operator and the log-sum-exp.
  *     GS_F16 / GS_BF16 : 1 <= D <= 128 (tensor-core path), any C >= 1.
  *                        Arithmetic: x.y on the tensor cores with fp32
  *                        accumulation, kernel values rounded to fp16 for the
  *                        second product, weights converted to fp16 (for bf16
  *                        weights this is exact for |w| in [2^-14, 65504]).
+ *                        The log-sum-exp runs on the tf32 tensor-core path
+ *                        (fp16 / bf16 values are exact in tf32).
+ *     The log-sum-exp backward and the k-nearest reduction: GS_F32, D <= 8.
  *   Anything else returns GS_ERR_UNSUPPORTED; there is no CPU fallback.
  *
  * Ownership and synchronisation: the caller owns every buffer, allocates the
@@ -105,7 +112,9 @@ gs_status gauss_sum_fwd(const void *x, const void *y, const void *w, float *out,
  * computed with a shift so that rows whose every kernel value underflows fp32
  * still get a finite result.  Requires w > 0 (not checked: a non-positive
  * weight gives NaN or -inf, as log does).  N == 0 writes -inf.
- * Supported for GS_F32 with 1 <= D <= 8.
+ * Supported for 1 <= D <= 128 in every dtype: GS_F32 with D <= 8 on the
+ * CUDA-core path (power-of-two weight shifts), the rest on the tf32
+ * tensor-core path (a running maximum per row).
  */
 gs_status gauss_lse_fwd(const void *x, const void *y, const void *w, float *out, int64_t B,
                         int64_t M, int64_t N, int64_t D, int64_t C, float tau, gs_dtype dt,

@@ -51,7 +51,7 @@ gs_status check_dims(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, int64
     if (D > kSdMaxD && (op == GS_OP_LSE_BWD || op == GS_OP_KNN)) return GS_ERR_UNSUPPORTED;
   } else {
     if (D > kTcMaxD) return GS_ERR_UNSUPPORTED;
-    if (op == GS_OP_LSE || op == GS_OP_LSE_BWD) return GS_ERR_UNSUPPORTED;
+    if (op == GS_OP_LSE_BWD) return GS_ERR_UNSUPPORTED;   // (the forward runs on the tf32 path)
   }
   return GS_OK;
 }
@@ -238,7 +238,8 @@ gs_status run_pass(const Pass& p, const PassLayout& L, float* out, uint8_t* ws, 
     F32Args a{};
     a.x = p.rows_pts;
     a.y = p.cols_pts;
-    a.w = static_cast<const float*>(p.w);
+    a.w = p.w;
+    a.dt = GS_F32;
     a.values = static_cast<TcValues>(p.vmode);
     a.C = p.C;
     a.CV = p.CV;
@@ -381,10 +382,12 @@ struct LseF32Layout {
   size_t off_zc, off_xpack, off_rnorm, off_ypack, off_qw, off_m, off_l, total;
 };
 
-LseF32Layout lse_f32_layout(int64_t B, int64_t M, int64_t N, int64_t D, int64_t C, int sm) {
+LseF32Layout lse_f32_layout(int64_t B, int64_t M, int64_t N, int64_t D, int64_t C, gs_dtype dt,
+                            int sm) {
   LseF32Layout L{};
-  L.plan = f32_plan(B, M, N, D, sm);
-  const size_t rowb = size_t(2) * L.plan.Kp * 4;
+  // fp16 / bf16 values are exact in tf32: unsplit rows, one MMA per K step
+  L.plan = f32_plan(B, M, N, D, sm, dt == GS_F32);
+  const size_t rowb = size_t(L.plan.split ? 2 : 1) * L.plan.Kp * 4;
   const size_t Nq = (N + 127) / 128 * 128;
   size_t off = 0;
   L.off_zc = off;
@@ -532,7 +535,7 @@ size_t gs_workspace_bytes(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, 
   }
   if (op == GS_OP_LSE) {
     if (M == 0 || N == 0) return 0;
-    if (D > kSdMaxD) return lse_f32_layout(B, M, N, D, C, sm).total;
+    if (dt != GS_F32 || D > kSdMaxD) return lse_f32_layout(B, M, N, D, C, dt, sm).total;
     const SdPlan sp = sd_plan(B, M, N, static_cast<int>(D), C, sm);
     return align_up(size_t(2) * sp.splits * B * M * C * 4);
   }
@@ -583,9 +586,9 @@ gs_status gauss_lse_fwd(const void* x, const void* y, const void* w, float* out,
     return GS_OK;
   }
   const int sm = sm_count();
-  if (D > kSdMaxD) {
-    // fp32 tensor-core path: running-maximum (m, l) per split, then the finalize
-    const LseF32Layout L = lse_f32_layout(B, M, N, D, C, sm);
+  if (dt != GS_F32 || D > kSdMaxD) {
+    // tensor-core (tf32) path: running-maximum (m, l) per split, then the finalize
+    const LseF32Layout L = lse_f32_layout(B, M, N, D, C, dt, sm);
     if (ws_bytes < L.total) return GS_ERR_WORKSPACE;
     GS_TRY(check_ptr(ws, 1));
     uint8_t* w8 = static_cast<uint8_t*>(ws);
@@ -593,7 +596,8 @@ gs_status gauss_lse_fwd(const void* x, const void* y, const void* w, float* out,
     F32Args a{};
     a.x = x;
     a.y = y;
-    a.w = static_cast<const float*>(w);
+    a.w = w;
+    a.dt = dt;
     a.values = kValuesW;
     a.C = static_cast<int>(C);
     a.CV = static_cast<int>(C);
@@ -629,6 +633,7 @@ gs_status gauss_lse_fwd(const void* x, const void* y, const void* w, float* out,
     f.D = static_cast<int>(D);
     f.C = static_cast<int>(C);
     f.scale = coord_scale(tau);
+    f.no_fallback = 1;
     GS_CUDA(launch_lse_finalize(f, s));
     return GS_OK;
   }

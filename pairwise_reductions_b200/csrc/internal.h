@@ -83,6 +83,9 @@ struct LseFinalizeArgs {
   int64_t B, M, N;
   int D, C;
   float scale;
+  // the tensor-core path shifts by the running maximum (l >= 1): no recompute,
+  // and x, y, w may not be fp32
+  int no_fallback;
 };
 cudaError_t launch_lse_finalize(const LseFinalizeArgs& a, cudaStream_t s);
 
@@ -175,20 +178,22 @@ bool make_tmap_3d(CUtensorMap* m, CUtensorMapDataType dt, void* base, uint64_t d
 // ------------------------------------------------------------- fp32 tensor-core path
 // fp32 inputs with kSdMaxD < D <= kTcMaxD: split-tf32 MMAs (tc_f32_sm100.cu).
 struct F32Plan {
+  bool split;          // fp32 inputs: rows [hi | lo]; fp16 / bf16 (exact tf32): [hi] only
   int Kp;              // D rounded up to 8: floats per half of a packed row [hi | lo]
-  int atoms;           // 128-byte atoms per packed row (2 Kp floats)
+  int atoms;           // 128-byte atoms per packed row (2 Kp floats, or Kp)
   int max_chunk;       // channels per pass (64, or 32 for the widest rows)
   int splits;
   int64_t cols_per_split;   // multiple of 128
 };
-F32Plan f32_plan(int64_t B, int64_t M, int64_t N, int64_t D, int sm_count);
+F32Plan f32_plan(int64_t B, int64_t M, int64_t N, int64_t D, int sm_count, bool split = true);
 int f32_chunk_pad(int cw);            // 16, 32 or 64
 int f32_tile_cols(int KA, int mode);  // columns per tile of an instantiation
 
 struct F32Args {
-  const void* x;       // rows side [B, M, D] float32
-  const void* y;       // column side [B, N, D] float32
-  const float* w;      // values source [B, N, C] float32
+  const void* x;       // rows side [B, M, D], dtype dt
+  const void* y;       // column side [B, N, D], dtype dt
+  const void* w;       // values source [B, N, C], dtype dt
+  gs_dtype dt;         // fp32 (split operands); fp16 / bf16 (log-sum-exp only)
   TcValues values;     // value mode (values.cuh; its own centre x[b, 0])
   int C, CV;
   float* out;          // [S?][B][M][CV]; log-sum-exp: the shifts m (log2 units)
@@ -201,7 +206,7 @@ struct F32Args {
   F32Plan plan;
   // workspace pieces
   float* zc;           // [B, D] centre of each batch (the mean of its column points)
-  float* xpack;        // [B, M, 2 Kp]
+  float* xpack;        // [B, M, 2 Kp] (or [B, M, Kp] unsplit)
   float* rnorm;        // [B, M]
   float* ypack;        // [B, N, 2 Kp]
   float* qw;           // [B, Nq, 4], Nq = N rounded up to 128: -c |y'|^2 (-inf past N)

@@ -388,7 +388,7 @@ __global__ void lse_finalize_kernel(const LseFinalizeArgs a) {
       const float contrib = (mk == -INFINITY) ? 0.f : lk * ex2(mk - m);
       const float l = warp_sum(contrib);
       float res;
-      if (!(l < kTiny) || a.D > kSdMaxD) {
+      if (!(l < kTiny) || a.D > kSdMaxD || a.no_fallback) {
         // (the tensor-core path for D > 8 shifts by the running maximum, so
         // its l is at least 1 whenever any term is nonzero)
         res = (m + log2f(l)) * kLn2;

@@ -36,6 +36,7 @@
 #include <cuda.h>
 
 #include <cmath>
+#include <type_traits>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -67,6 +68,7 @@ struct F32KParams {
   int atoms;            // 128-byte atoms of a packed row actually loaded (<= KA)
   int Bsz;              // batch count (the lo half of v sits at batch index B + b)
   int bn;               // tile width the TMA boxes were made for
+  int split;            // 1: rows [hi | lo]; 0: rows are exact tf32 (fp16 / bf16 inputs), hi only
   float two_c;
 };
 
@@ -164,7 +166,9 @@ __device__ __forceinline__ void exp_warps_sync() { asm volatile("bar.sync 1, 256
 // t_ij + log2 w_j as a running maximum m and a sum l of 2^(t - m), updated per
 // 32-column chunk (the maximum of the chunk first, then its shifted sum), so
 // that no value under- or overflows.
-template <int KA, int MODE, bool LSE>
+// SPLIT: rows [hi | lo] and three products per K step (fp32 inputs), or exact
+// tf32 rows (fp16 / bf16 inputs) and the large product alone.
+template <int KA, int MODE, bool LSE, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_f32_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                   const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmV,
@@ -175,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int CP = Cfg::CP;
   constexpr int NST = Cfg::NST;
   constexpr int BN = Cfg::BN;
-  if (p.bn != BN) {   // boxes sized for another tile: touch nothing, report
+  if (p.bn != BN || p.split != (SPLIT ? 1 : 0)) {   // boxes made for another instantiation
     if (threadIdx.x == 0) atomicOr(&g_device_error_f32, 2);
     return;
   }
@@ -299,19 +303,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_ss_tf32(d, kdesc(sX, kAtom, ka), bdesc, idS, acc);
           }
         };
+        // (exact tf32 operands, SPLIT false: the large products alone)
         if constexpr (REG) {
           for (int ks = 0; ks < p.ksteps; ++ks) {
-            const uint64_t bh = kdesc(sy, BN * 128, ks), bl = kdesc(sy, BN * 128, ks + ks_lo);
-            mma(ds, ks + ks_lo, bh, ks > 0 ? 1u : 0u);
-            mma(ds, ks, bl, 1u);
+            const uint64_t bh = kdesc(sy, BN * 128, ks);
+            if constexpr (SPLIT) {
+              mma(ds, ks + ks_lo, bh, ks > 0 ? 1u : 0u);
+              mma(ds, ks, kdesc(sy, BN * 128, ks + ks_lo), 1u);
+            }
             mma(db, ks, bh, ks > 0 ? 1u : 0u);
           }
         } else {
-          for (int ks = 0; ks < p.ksteps; ++ks) {
-            mma(db, ks + ks_lo, kdesc(sy, BN * 128, ks), ks > 0 ? 1u : 0u);
-            mma(db, ks, kdesc(sy, BN * 128, ks + ks_lo), 1u);
+          if constexpr (SPLIT) {
+            for (int ks = 0; ks < p.ksteps; ++ks) {
+              mma(db, ks + ks_lo, kdesc(sy, BN * 128, ks), ks > 0 ? 1u : 0u);
+              mma(db, ks, kdesc(sy, BN * 128, ks + ks_lo), 1u);
+            }
           }
-          for (int ks = 0; ks < p.ksteps; ++ks) mma(db, ks, kdesc(sy, BN * 128, ks), 1u);
+          for (int ks = 0; ks < p.ksteps; ++ks)
+            mma(db, ks, kdesc(sy, BN * 128, ks), (SPLIT || ks > 0) ? 1u : 0u);
         }
       };
       auto issue_O = [&](int h, int st, bool acc_prev) {
@@ -387,13 +397,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (Cfg::XT) {
       if (h == 0) {
         // this thread's packed row (zeros past M) into its TMEM lane
-        const int rowf = 2 * p.ksteps * 8;
+        const int rowf = (SPLIT ? 2 : 1) * p.ksteps * 8;
         const float4* src = reinterpret_cast<const float4*>(p.xpack + (b * p.M + i) * rowf);
-        for (int c = 0; c < rowf / 16; ++c) {
+        for (int c = 0; c < (rowf + 15) / 16; ++c) {   // (rowf is a multiple of 8)
           uint32_t v[16];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const float4 f = valid ? src[c * 4 + u] : make_float4(0.f, 0.f, 0.f, 0.f);
+            const bool in = valid && c * 16 + 4 * u < rowf;
+            const float4 f = in ? src[c * 4 + u] : make_float4(0.f, 0.f, 0.f, 0.f);
             v[4 * u + 0] = __float_as_uint(f.x);
             v[4 * u + 1] = __float_as_uint(f.y);
             v[4 * u + 2] = __float_as_uint(f.z);
@@ -428,7 +439,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tSs = tmem + lane_base + Cfg::col_ss(h);
         uint32_t cb[32], cs[32];
         tmem_ld32(tS, cb);
-        tmem_ld32(tSs, cs);
+        if constexpr (SPLIT) {
+          tmem_ld32(tSs, cs);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) cs[e] = 0u;   // no small products
+        }
         tmem_wait_ld();
         reg_fence32(cb);
         reg_fence32(cs);
@@ -441,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             cur[e] = fmaf(__uint_as_float(cb[e]) + __uint_as_float(cs[e]), two_c, r);
           if (ch + 1 < NCH) {
             tmem_ld32(tS + (ch + 1) * 32, cb);
-            tmem_ld32(tSs + (ch + 1) * 32, cs);
+            if constexpr (SPLIT) tmem_ld32(tSs + (ch + 1) * 32, cs);
           } else {
             tc_fence_before();
             mbar_arrive(bar_f(h));
@@ -639,12 +655,14 @@ __global__ void column_mean_kernel(const float* __restrict__ y, float* __restric
 // Packed operand rows [hi (K') | lo (K')] of the centred points v' = v - z,
 // z = zc[b, :], and the norm term -c |v'|^2: for the row side into
 // norm[b * R + r]; for the column side into norm[(b * Rpad + r) * 4] (lanes
-// 1-3 zeroed) with -inf for the padding columns r >= R.  One warp per row,
-// lanes along the features (coalesced reads and writes).
-__global__ void pack_rows_f32_kernel(const float* __restrict__ src, const float* __restrict__ zc,
+// 1-3 zeroed) with -inf for the padding columns r >= R.  Exact tf32 inputs
+// (fp16 / bf16, zc == nullptr, split == 0): v itself, rows [hi (K')] only.
+// One warp per row, lanes along the features (coalesced reads and writes).
+template <typename T>
+__global__ void pack_rows_f32_kernel(const T* __restrict__ src, const float* __restrict__ zc,
                                      float* __restrict__ dst, float* __restrict__ norm, int64_t B,
                                      int64_t R, int64_t Rpad, int D, int Kp, float c,
-                                     int norm_stride) {
+                                     int norm_stride, int split) {
   const int lane = threadIdx.x & 31;
   const int64_t total = B * Rpad;
   const int64_t wstride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -659,16 +677,16 @@ __global__ void pack_rows_f32_kernel(const float* __restrict__ src, const float*
       }
       continue;
     }
-    const float* v = src + (b * R + rr) * D;
-    const float* z = zc + b * D;
-    float* out = dst + (b * R + rr) * (2 * static_cast<int64_t>(Kp));
+    const T* v = src + (b * R + rr) * D;
+    const float* z = zc ? zc + b * D : nullptr;
+    float* out = dst + (b * R + rr) * ((split ? 2 : 1) * static_cast<int64_t>(Kp));
     float sq = 0.f;
     for (int k = lane; k < Kp; k += 32) {
-      const float d = (k < D) ? v[k] - z[k] : 0.f;
+      const float d = (k < D) ? vf(v[k]) - (z ? z[k] : 0.f) : 0.f;
       sq = fmaf(d, d, sq);
       const float hi = tf32_round(d);
       out[k] = hi;
-      out[Kp + k] = tf32_round(d - hi);
+      if (split) out[Kp + k] = tf32_round(d - hi);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
@@ -682,8 +700,9 @@ __global__ void pack_rows_f32_kernel(const float* __restrict__ src, const float*
 // Register-path values: channels [c0, c0 + cw) (cw <= 3) of the pass's values
 // (values.cuh) into lanes 1.. of qw[b, j, :]; for the log-sum-exp, their
 // base-2 logarithms.
-__global__ void pack_values_qw_kernel(const float* __restrict__ w, const float* __restrict__ y,
-                                      const float* __restrict__ rows, float* __restrict__ qw,
+template <typename TW, typename TY>
+__global__ void pack_values_qw_kernel(const TW* __restrict__ w, const TY* __restrict__ y,
+                                      const TY* __restrict__ rows, float* __restrict__ qw,
                                       int64_t B, int64_t N, int64_t Nq, int64_t Mrows, int C, int D,
                                       int c0, int cw, int log2_values) {
   const int64_t total = B * N;
@@ -731,10 +750,10 @@ struct TileMaps {
   CUtensorMap x, y, q, v;
 };
 
-template <int KA, int MODE, bool LSE = false>
+template <int KA, int MODE, bool LSE = false, bool SPLIT = true>
 cudaError_t launch_kernel(const TileMaps& m, const F32KParams& kp, dim3 grid, cudaStream_t s) {
   using Cfg = F32Cfg<KA, MODE>;
-  auto fn = tc_f32_kernel<KA, MODE, LSE>;
+  auto fn = tc_f32_kernel<KA, MODE, LSE, SPLIT>;
   static bool attr_done = false;   // idempotent; a benign race at worst repeats the call
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
@@ -748,7 +767,10 @@ cudaError_t launch_kernel(const TileMaps& m, const F32KParams& kp, dim3 grid, cu
 template <int KA>
 cudaError_t launch_mode(int mode, bool lse, const TileMaps& m, const F32KParams& kp, dim3 grid,
                         cudaStream_t s) {
-  if (lse) return launch_kernel<KA, 1, true>(m, kp, grid, s);   // one channel per pass
+  if (lse)   // one channel per pass
+    return kp.split ? launch_kernel<KA, 1, true, true>(m, kp, grid, s)
+                    : launch_kernel<KA, 1, true, false>(m, kp, grid, s);
+  if (!kp.split) return cudaErrorInvalidValue;   // unsplit rows: log-sum-exp only
   switch (mode) {
     case 1: return launch_kernel<KA, 1>(m, kp, grid, s);
     case 3: return launch_kernel<KA, 3>(m, kp, grid, s);
@@ -780,10 +802,11 @@ int tile_cols_ka(int mode) {
 
 }  // namespace
 
-F32Plan f32_plan(int64_t B, int64_t M, int64_t N, int64_t D, int sm_count) {
+F32Plan f32_plan(int64_t B, int64_t M, int64_t N, int64_t D, int sm_count, bool split) {
   F32Plan p{};
+  p.split = split;
   p.Kp = static_cast<int>((D + 7) / 8 * 8);
-  p.atoms = (2 * p.Kp + 31) / 32;
+  p.atoms = ((split ? 2 : 1) * p.Kp + 31) / 32;
   p.max_chunk = ka_for(p.atoms) >= 8 ? 32 : 64;
   // a split is a whole number of 128-column blocks (every tile width divides
   // it, so no tile straddles two splits)
@@ -821,27 +844,56 @@ int f32_tile_cols(int KA, int mode) {
   }
 }
 
+// Packed rows of x and y (and, for fp32, the column centre first).
+template <typename T>
+void pack_operands_f32(const F32Args& a, int64_t Nq, float c, cudaStream_t s) {
+  const T* x = static_cast<const T*>(a.x);
+  const T* y = static_cast<const T*>(a.y);
+  const int split = a.plan.split ? 1 : 0;
+  const float* zc = nullptr;
+  if constexpr (std::is_same<T, float>::value) {
+    if (split) {
+      column_mean_kernel<<<dim3(static_cast<unsigned>(a.B), static_cast<unsigned>((a.D + 31) / 32)),
+                           256, 0, s>>>(y, a.zc, a.N, a.D);
+      zc = a.zc;
+    }
+  }
+  // one warp per row, 8 rows per 256-thread block
+  pack_rows_f32_kernel<T><<<grid_for(a.B * a.M, 8), 256, 0, s>>>(x, zc, a.xpack, a.rnorm, a.B, a.M,
+                                                                a.M, a.D, a.plan.Kp, c, 1, split);
+  pack_rows_f32_kernel<T><<<grid_for(a.B * Nq, 8), 256, 0, s>>>(y, zc, a.ypack, a.qw, a.B, a.N, Nq,
+                                                               a.D, a.plan.Kp, c, 4, split);
+}
+
+template <typename T>
+void pack_qw_values(const F32Args& a, int64_t Nq, int c0, int cw, cudaStream_t s) {
+  const T* x = static_cast<const T*>(a.x);
+  const T* y = static_cast<const T*>(a.y);
+  pack_values_qw_kernel<T, T><<<grid_for(a.B * a.N, 256), 256, 0, s>>>(
+      static_cast<const T*>(a.w), y, x, a.qw, a.B, a.N, Nq, a.M, a.C, a.D, c0, cw, a.lse ? 1 : 0);
+}
+
 cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
   if (a.B == 0 || a.M == 0) return cudaSuccess;
   const int Kp = a.plan.Kp;
   const float c = 0.5f * a.tau * kLog2e;
   const int64_t Nq = (a.N + 127) / 128 * 128;
-  const float* x = static_cast<const float*>(a.x);
-  const float* y = static_cast<const float*>(a.y);
-  column_mean_kernel<<<dim3(static_cast<unsigned>(a.B), static_cast<unsigned>((a.D + 31) / 32)),
-                       256, 0, s>>>(y, a.zc, a.N, a.D);
-  // one warp per row, 8 rows per 256-thread block
-  pack_rows_f32_kernel<<<grid_for(a.B * a.M, 8), 256, 0, s>>>(x, a.zc, a.xpack, a.rnorm, a.B, a.M,
-                                                             a.M, a.D, Kp, c, 1);
-  pack_rows_f32_kernel<<<grid_for(a.B * Nq, 8), 256, 0, s>>>(y, a.zc, a.ypack, a.qw, a.B, a.N, Nq,
-                                                            a.D, Kp, c, 4);
+  // register values for at most 3 channels per pass; the log-sum-exp one
+  // channel per pass; fp16 / bf16 inputs (exact tf32) take the register path only
+  const bool reg = a.lse || a.CV <= 3;
+  if (a.dt != GS_F32 && (!reg || a.plan.split)) return cudaErrorInvalidValue;
+  if (a.dt == GS_F32)
+    pack_operands_f32<float>(a, Nq, c, s);
+  else if (a.dt == GS_F16)
+    pack_operands_f32<__half>(a, Nq, c, s);
+  else
+    pack_operands_f32<__nv_bfloat16>(a, Nq, c, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // register values for at most 3 channels per pass; the log-sum-exp one
-  // channel per pass
-  const bool reg = a.lse || a.CV <= 3;
+  const float* x = static_cast<const float*>(a.x);   // fp32 only below (tensor-core values)
+  const float* y = static_cast<const float*>(a.y);
   TileMaps m;
-  const uint64_t rowf = 2ull * Kp;
+  const uint64_t rowf = (a.plan.split ? 2ull : 1ull) * Kp;
   if (!make_tmap_3d(&m.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.xpack, rowf, a.M, a.B, rowf * 4,
                     a.M * rowf * 4, 32, kBM))
     return cudaErrorInvalidValue;
@@ -854,8 +906,12 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
     const int cw = (a.CV - c0) < chunk ? (a.CV - c0) : chunk;
     const int mode = reg ? (cw == 1 ? 1 : 3) : f32_chunk_pad(cw);
     if (reg) {
-      pack_values_qw_kernel<<<grid_for(a.B * a.N, 256), 256, 0, s>>>(
-          a.w, y, x, a.qw, a.B, a.N, Nq, a.M, a.C, a.D, c0, cw, a.lse ? 1 : 0);
+      if (a.dt == GS_F32)
+        pack_qw_values<float>(a, Nq, c0, cw, s);
+      else if (a.dt == GS_F16)
+        pack_qw_values<__half>(a, Nq, c0, cw, s);
+      else
+        pack_qw_values<__nv_bfloat16>(a, Nq, c0, cw, s);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }
@@ -872,7 +928,7 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
       const int CP = mode;
       const int64_t total = a.B * CP * a.N;
       pack_values_f32_split_kernel<<<grid_for(total, 256), 256, 0, s>>>(
-          a.w, y, x, a.vt, a.B, a.N, Nst, a.M, a.C, a.D, a.CV, c0, CP);
+          static_cast<const float*>(a.w), y, x, a.vt, a.B, a.N, Nst, a.M, a.C, a.D, a.CV, c0, CP);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
       if (!make_tmap_3d(&m.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.vt, a.N, CP, 2 * a.B, Nst * 4ull,
@@ -895,6 +951,7 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
     kp.atoms = a.plan.atoms;
     kp.Bsz = static_cast<int>(a.B);
     kp.bn = BN;
+    kp.split = a.plan.split ? 1 : 0;
     kp.two_c = a.tau * kLog2e;
     switch (KA) {
       case 1: e = launch_mode<1>(mode, a.lse, m, kp, grid, s); break;

@@ -67,8 +67,13 @@ def test_invalid_arguments_are_rejected_before_any_launch(fn):
     assert _fwd(fn, B=70000) == 2
 
 
-def test_lse_has_no_half_precision_path():
-    assert _fwd("gauss_lse_fwd", dt=1, D=32) == 2
+def test_lse_in_half_precision_runs_on_the_tf32_path():
+    # fp16 / bf16 log-sum-exp (exact tf32 operands) asks for its workspace; its
+    # backward has no half-precision path
+    assert _fwd("gauss_lse_fwd", dt=1, D=32) == 4
+    assert _fwd("gauss_lse_fwd", dt=2, D=3) == 4
+    with pytest.raises(ValueError):
+        gs.workspace_bytes(gs.GS_OP_LSE_BWD, 1, 10, 10, 3, 1, gs.GS_F16)
 
 
 def test_fp32_wide_features_route_to_the_tensor_core_path():

@@ -185,6 +185,23 @@ def test_lse_f32_tensor_core_shapes(shape, tau):
     assert rel_l2(np.exp(out), np.exp(ref)) <= TOL["f32"]
 
 
+@pytest.mark.parametrize("dtype,shape,tau", [("f16", (1, 300, 700, 3, 1), 30.0),
+                                             ("bf16", (2, 200, 500, 32, 2), 1.0),
+                                             ("f16", (1, 130, 1000, 100, 1), 1.0),
+                                             ("f16", (1, 257, 900, 128, 3), 2.0)])
+def test_lse_half_precision_shapes(dtype, shape, tau):
+    """fp16 / bf16 log-sum-exp: exact tf32 operands on the tensor-core path."""
+    B, M, N, D, C = shape
+    inp = synth.make_inputs(3, seed=43, B=B, M=M, N=N, D=D, C=C, dtype=dtype)
+    inp["x"] = (inp["x"].double() / D ** 0.5).to(inp["x"].dtype)
+    inp["y"] = (inp["y"].double() / D ** 0.5).to(inp["y"].dtype)
+    d = dev(inp)
+    out = gs().gauss_lse_fwd(d["x"], d["y"], d["w"], tau).cpu().numpy()
+    ref = oracle.gauss_lse(f64(inp, "x"), f64(inp, "y"), f64(inp, "w"), tau)
+    assert rel_l2(out, ref) <= TOL[dtype], rel_l2(out, ref)
+    assert rel_l2(np.exp(out), np.exp(ref)) <= TOL[dtype]
+
+
 def test_lse_f32_tensor_core_rows_far_from_every_point():
     """Rows whose every kernel value underflows fp32 (exp(-tau/2 d^2) ~ e^-5000):
     the running maximum keeps the log-sum-exp finite and exact."""
