@@ -32,7 +32,8 @@
  *                        weights this is exact for |w| in [2^-14, 65504]).
  *                        The log-sum-exp runs on the tf32 tensor-core path
  *                        (fp16 / bf16 values are exact in tf32).
- *     The log-sum-exp backward and the k-nearest reduction: GS_F32, D <= 8.
+ *     The log-sum-exp backward: GS_F32, 1 <= D <= 128.  The k-nearest
+ *     reduction: GS_F32, D <= 8.
  *   Anything else returns GS_ERR_UNSUPPORTED; there is no CPU fallback.
  *
  * Ownership and synchronisation: the caller owns every buffer, allocates the

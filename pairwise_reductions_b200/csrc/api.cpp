@@ -48,7 +48,7 @@ gs_status check_dims(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, int64
   if (dt == GS_F32) {
     // D > 8: the split-tf32 tensor-core path, for the Gauss-sum passes only
     if (D > kTcMaxD) return GS_ERR_UNSUPPORTED;
-    if (D > kSdMaxD && (op == GS_OP_LSE_BWD || op == GS_OP_KNN)) return GS_ERR_UNSUPPORTED;
+    if (D > kSdMaxD && op == GS_OP_KNN) return GS_ERR_UNSUPPORTED;
   } else {
     if (D > kTcMaxD) return GS_ERR_UNSUPPORTED;
     if (op == GS_OP_LSE_BWD) return GS_ERR_UNSUPPORTED;   // (the forward runs on the tf32 path)
@@ -241,6 +241,16 @@ gs_status run_pass(const Pass& p, const PassLayout& L, float* out, uint8_t* ws, 
     a.w = p.w;
     a.dt = GS_F32;
     a.values = static_cast<TcValues>(p.vmode);
+    a.src_ld = p.src_ld;
+    if (p.shift_mode == 1 || p.shift_mode == 2) {
+      a.shift_mode = p.shift_mode;
+      a.shift_src = p.shift_src;
+      a.shift_ld = p.shift_ld;
+      a.shift_c = p.shift_c;
+      a.shift_scale = p.shift_scale;
+    } else if (p.shift_mode != 0) {
+      return GS_ERR_UNSUPPORTED;   // squared-distance modes: CUDA-core path only
+    }
     a.C = p.C;
     a.CV = p.CV;
     a.out = dst;
@@ -414,6 +424,7 @@ LseF32Layout lse_f32_layout(int64_t B, int64_t M, int64_t N, int64_t D, int64_t 
 // the per-row shift and the squared-distance factor (dL/dtau), and rows y /
 // columns x with values [g_c, g_c (x - z)] and a per-column shift (dL/dw, dL/dy).
 struct LseBwdLayout {
+  bool tau_in_x;
   Pass px, pt, py;
   PassLayout lx, lt, ly;
   size_t off_ox, off_ot, off_oy, off_tau, total;
@@ -424,9 +435,12 @@ LseBwdLayout lse_bwd_layout(const void* x, const void* y, const void* w, const f
                             float tau, int sm) {
   LseBwdLayout L{};
   const float kNegLog2e = -1.4426950408889634f;
+  // D > 8 (tf32 tensor-core passes): the dL/dtau sums ride as a third value
+  // part of the x pass instead of a squared-distance pass
+  L.tau_in_x = pass_path(GS_F32, static_cast<int>(D)) != kPathSmallD;
   L.px = fwd_pass(x, y, w, B, M, N, D, 1, tau, GS_F32);
-  L.px.vmode = 1;
-  L.px.CV = value_channels(1, 1, static_cast<int>(D));
+  L.px.vmode = L.tau_in_x ? 2 : 1;
+  L.px.CV = value_channels(L.px.vmode, 1, static_cast<int>(D));
   L.px.src_ld = C;
   L.px.shift_mode = 1;
   L.px.shift_src = lse;
@@ -447,7 +461,7 @@ LseBwdLayout lse_bwd_layout(const void* x, const void* y, const void* w, const f
   L.py.shift_ld = C;
   L.py.shift_scale = kNegLog2e;
   L.lx = pass_layout(L.px, sm);
-  L.lt = pass_layout(L.pt, sm);
+  if (!L.tau_in_x) L.lt = pass_layout(L.pt, sm);
   L.ly = pass_layout(L.py, sm);
   size_t scratch = L.lx.total;
   if (L.lt.total > scratch) scratch = L.lt.total;
@@ -792,15 +806,16 @@ gs_status gauss_lse_bwd(const void* x, const void* y, const void* w, const float
       L.px.w = wf + c;
       L.px.shift_c = c;
       GS_TRY(run_pass(L.px, L.lx, ox, wsb, s));
-      if (grad_tau) {
+      if (grad_tau && !L.tau_in_x) {
         L.pt.w = wf + c;
         L.pt.shift_c = c;
         GS_TRY(run_pass(L.pt, L.lt, ot, wsb, s));
       }
-      GS_CUDA(launch_lse_x_tau_epilogue(static_cast<const float*>(x), g, ox, grad_tau ? ot : nullptr,
+      GS_CUDA(launch_lse_x_tau_epilogue(static_cast<const float*>(x), g, ox,
+                                        (grad_tau && !L.tau_in_x) ? ot : nullptr,
                                         grad_x, grad_tau ? tau_rows : nullptr, B, M,
                                         static_cast<int>(D), static_cast<int>(C), c, tau,
-                                        static_cast<float>(1.0 / cfac), acc, s));
+                                        static_cast<float>(1.0 / cfac), acc, s, L.px.CV));
     }
     if (grad_y || grad_w) {
       L.py.w = g + c;

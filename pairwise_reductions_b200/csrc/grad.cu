@@ -155,13 +155,16 @@ __global__ void sum_rows_kernel(const float* __restrict__ v, int64_t n, float* _
 // every p_ij of the row, so dividing by A cancels it:
 //   dL/dx_ik   += -tau g_ic ((x_ik - z_k) - B_k / A)
 //   dL/dtau(i) += -1/2 g_ic (T / A) / (tau/2 log2 e)
+// o rows have ocv channels; with ot == nullptr (ocv = 2 + D) the rows carry a
+// third part (values mode 2):
+// Q = sum_j p |y_j - z|^2, and sum_j p |x_i - y_j|^2 = Q - 2 (x_i - z).B + |x_i - z|^2 A.
 __global__ void lse_x_tau_epilogue_kernel(const float* __restrict__ x, const float* __restrict__ g,
                                           const float* __restrict__ o, const float* __restrict__ ot,
                                           float* __restrict__ gx, float* __restrict__ tau_rows,
                                           int64_t B, int64_t M, int D, int C, int c, float tau,
-                                          float inv_cfac, int accumulate) {
+                                          float inv_cfac, int accumulate, int ocv) {
   const int64_t rows = B * M;
-  const int CV = 1 + D;
+  const int CV = ocv;
   for (int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; r < rows;
        r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t b = r / M;
@@ -177,7 +180,19 @@ __global__ void lse_x_tau_epilogue_kernel(const float* __restrict__ x, const flo
       }
     }
     if (tau_rows) {
-      const float v = -0.5f * gic * ot[r] * inv_a * inv_cfac;
+      float dist;   // sum_j p |x_i - y_j|^2
+      if (ot) {
+        dist = ot[r] * inv_cfac;
+      } else {
+        float xb = 0.f, xx = 0.f;
+        for (int k = 0; k < D; ++k) {
+          const float d = xi[k] - z[k];
+          xb = fmaf(d, oi[1 + k], xb);
+          xx = fmaf(d, d, xx);
+        }
+        dist = oi[1 + D] - 2.f * xb + xx * oi[0];
+      }
+      const float v = -0.5f * gic * dist * inv_a;
       tau_rows[r] = accumulate ? tau_rows[r] + v : v;
     }
   }
@@ -302,9 +317,9 @@ cudaError_t launch_grad_y_epilogue(const void* y, const void* w, gs_dtype dt, co
 cudaError_t launch_lse_x_tau_epilogue(const float* x, const float* g, const float* o,
                                       const float* ot, float* grad_x, float* tau_rows, int64_t B,
                                       int64_t M, int D, int C, int c, float tau, float inv_cfac,
-                                      bool accumulate, cudaStream_t s) {
+                                      bool accumulate, cudaStream_t s, int ocv) {
   lse_x_tau_epilogue_kernel<<<grid_for(B * M, 256), 256, 0, s>>>(
-      x, g, o, ot, grad_x, tau_rows, B, M, D, C, c, tau, inv_cfac, accumulate ? 1 : 0);
+      x, g, o, ot, grad_x, tau_rows, B, M, D, C, c, tau, inv_cfac, accumulate ? 1 : 0, ocv);
   return cudaGetLastError();
 }
 

@@ -99,11 +99,12 @@ cudaError_t launch_pack_values_f32(const void* src, int64_t src_ld, const void* 
 // holds [sum_j p, sum_j p (y - z)] and o_y [B, N, 1 + D] holds
 // [sum_i g p / w, sum_i g p (x - z) / w]; with `accumulate` the results add to
 // the outputs of the previous channels.
-// ot [B, M] holds sum_j p |x^ - y^|^2 (NULL when tau_rows is NULL)
+// ot [B, M] holds sum_j p |x^ - y^|^2; when it is NULL (and tau_rows is not),
+// o has 2 + D channels per row, the last sum_j p |y - z|^2 (values mode 2)
 cudaError_t launch_lse_x_tau_epilogue(const float* x, const float* g, const float* o,
                                       const float* ot, float* grad_x, float* tau_rows, int64_t B,
                                       int64_t M, int D, int C, int c, float tau, float inv_cfac,
-                                      bool accumulate, cudaStream_t s);
+                                      bool accumulate, cudaStream_t s, int ocv);
 cudaError_t launch_lse_grad_y_epilogue(const float* y, const float* w, const float* o,
                                        float* grad_y, float* grad_w, int64_t B, int64_t N, int D,
                                        int C, int c, float tau, bool accumulate, cudaStream_t s);
@@ -196,6 +197,14 @@ struct F32Args {
   gs_dtype dt;         // fp32 (split operands); fp16 / bf16 (log-sum-exp only)
   TcValues values;     // value mode (values.cuh; its own centre x[b, 0])
   int C, CV;
+  int64_t src_ld;      // row stride of the value source (C when it is a whole array)
+  // optional exponent shift (log2 units) added to the row norms (shift_mode 1)
+  // or to the column norms (2): shift_scale * shift_src[(b * n + p) * shift_ld + shift_c]
+  int shift_mode;
+  const float* shift_src;
+  int64_t shift_ld;
+  int shift_c;
+  float shift_scale;
   float* out;          // [S?][B][M][CV]; log-sum-exp: the shifts m (log2 units)
   float* out_l;        // log-sum-exp only: the scaled sums l, same layout
   bool lse;            // log-sum-exp of w K per channel (w > 0) instead of the sum

@@ -704,13 +704,13 @@ template <typename TW, typename TY>
 __global__ void pack_values_qw_kernel(const TW* __restrict__ w, const TY* __restrict__ y,
                                       const TY* __restrict__ rows, float* __restrict__ qw,
                                       int64_t B, int64_t N, int64_t Nq, int64_t Mrows, int C, int D,
-                                      int c0, int cw, int log2_values) {
+                                      int c0, int cw, int log2_values, int64_t src_ld) {
   const int64_t total = B * N;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t b = e / N, j = e % N;
     for (int ch = 0; ch < cw; ++ch) {
-      const float v = value_at(w, y, rows, b, e, Mrows, D, C, c0 + ch, C);
+      const float v = value_at(w, y, rows, b, e, Mrows, D, C, c0 + ch, src_ld);
       qw[(b * Nq + j) * 4 + 1 + ch] = log2_values ? lg2(v) : v;
     }
   }
@@ -723,7 +723,7 @@ __global__ void pack_values_f32_split_kernel(const float* __restrict__ w,
                                              const float* __restrict__ rows,
                                              float* __restrict__ vt, int64_t B, int64_t N,
                                              int64_t Nst, int64_t Mrows, int C, int D, int CV,
-                                             int c0, int CP) {
+                                             int c0, int CP, int64_t src_ld) {
   const int64_t total = B * CP * N;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -732,10 +732,22 @@ __global__ void pack_values_f32_split_kernel(const float* __restrict__ w,
     const int cc = static_cast<int>(bc % CP);
     const int64_t b = bc / CP;
     const int ch = c0 + cc;
-    const float v = (ch < CV) ? value_at(w, y, rows, b, b * N + j, Mrows, D, C, ch, C) : 0.f;
+    const float v = (ch < CV) ? value_at(w, y, rows, b, b * N + j, Mrows, D, C, ch, src_ld) : 0.f;
     const float hi = tf32_round(v);
     vt[(b * CP + cc) * Nst + j] = hi;
     vt[((B + b) * CP + cc) * Nst + j] = tf32_round(v - hi);
+  }
+}
+
+// Exponent shift of a pass (log2 units): rows -- norm[b * R + r] -- or columns
+// -- norm[(b * Rpad + r) * 4], r < R -- gain scale * src[(b * R + r) * ld + c].
+__global__ void add_shift_kernel(float* __restrict__ norm, int stride, const float* __restrict__ src,
+                                 int64_t ld, int c, float scale, int64_t B, int64_t R, int64_t Rpad) {
+  const int64_t total = B * R;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = e / R, r = e % R;
+    norm[(b * Rpad + r) * stride] += scale * src[e * ld + c];
   }
 }
 
@@ -870,7 +882,8 @@ void pack_qw_values(const F32Args& a, int64_t Nq, int c0, int cw, cudaStream_t s
   const T* x = static_cast<const T*>(a.x);
   const T* y = static_cast<const T*>(a.y);
   pack_values_qw_kernel<T, T><<<grid_for(a.B * a.N, 256), 256, 0, s>>>(
-      static_cast<const T*>(a.w), y, x, a.qw, a.B, a.N, Nq, a.M, a.C, a.D, c0, cw, a.lse ? 1 : 0);
+      static_cast<const T*>(a.w), y, x, a.qw, a.B, a.N, Nq, a.M, a.C, a.D, c0, cw, a.lse ? 1 : 0,
+      a.src_ld > 0 ? a.src_ld : a.C);
 }
 
 cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
@@ -888,6 +901,14 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
     pack_operands_f32<__half>(a, Nq, c, s);
   else
     pack_operands_f32<__nv_bfloat16>(a, Nq, c, s);
+  if (a.shift_mode == 1)
+    add_shift_kernel<<<grid_for(a.B * a.M, 256), 256, 0, s>>>(a.rnorm, 1, a.shift_src, a.shift_ld,
+                                                             a.shift_c, a.shift_scale, a.B, a.M, a.M);
+  else if (a.shift_mode == 2)
+    add_shift_kernel<<<grid_for(a.B * a.N, 256), 256, 0, s>>>(a.qw, 4, a.shift_src, a.shift_ld,
+                                                             a.shift_c, a.shift_scale, a.B, a.N, Nq);
+  else if (a.shift_mode != 0)
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const float* x = static_cast<const float*>(a.x);   // fp32 only below (tensor-core values)
@@ -928,7 +949,8 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
       const int CP = mode;
       const int64_t total = a.B * CP * a.N;
       pack_values_f32_split_kernel<<<grid_for(total, 256), 256, 0, s>>>(
-          static_cast<const float*>(a.w), y, x, a.vt, a.B, a.N, Nst, a.M, a.C, a.D, a.CV, c0, CP);
+          static_cast<const float*>(a.w), y, x, a.vt, a.B, a.N, Nst, a.M, a.C, a.D, a.CV, c0, CP,
+          a.src_ld > 0 ? a.src_ld : a.C);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
       if (!make_tmap_3d(&m.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.vt, a.N, CP, 2 * a.B, Nst * 4ull,

@@ -383,10 +383,17 @@ def test_vjp_d32_c1_full_size_sampled():
 
 # ------------------------------------------------------------------ log-sum-exp backward
 @pytest.mark.parametrize("shape,shift", [((1, 300, 500, 3, 1), 0.0), ((2, 200, 300, 2, 3), 0.0),
-                                         ((1, 150, 400, 8, 2), 0.0), ((1, 256, 700, 3, 1), 30.0)])
+                                         ((1, 150, 400, 8, 2), 0.0), ((1, 256, 700, 3, 1), 30.0),
+                                         ((1, 200, 500, 16, 1), 0.0), ((2, 150, 300, 32, 2), 0.0),
+                                         ((1, 180, 400, 24, 1), 30.0)])
 def test_lse_bwd_every_gradient(shape, shift):
+    """D > 8 runs the tf32 tensor-core passes (coordinates scaled by sqrt(3/D) so that
+    the clouds have the spread of the D = 3 ones)."""
     B, M, N, D, C = shape
     inp = synth.make_inputs(3, seed=17, B=B, M=M, N=N, D=D, C=C, with_g=True, tau=20.0)
+    if D > 8:
+        for k in ("x", "y"):
+            inp[k] = (inp[k].double() * (3.0 / D) ** 0.5).float()
     if shift:
         for k in ("x", "y"):
             inp[k] = inp[k] + shift
