@@ -172,8 +172,9 @@ gs_status gauss_sum_vjp(const void *x, const void *y, const void *w, const float
  *
  * lse [B, M, C] float32 is the forward's output for the same inputs.  The
  * shift -lse is folded into every kernel exponent, so the passes sum p
- * directly (no overflow, no separate normalisation).  GS_F32, 1 <= D <= 8,
- * w > 0; any output may be NULL.  Workspace: gs_workspace_bytes(GS_OP_LSE_BWD, ...).
+ * directly (no overflow, no separate normalisation).  GS_F32, 1 <= D <= 128
+ * (D > 8: tf32 tensor-core passes), w > 0; any output may be NULL.  Workspace:
+ * gs_workspace_bytes(GS_OP_LSE_BWD, ...).
  */
 gs_status gauss_lse_bwd(const void *x, const void *y, const void *w, const float *lse,
                         const float *g, float *grad_x, float *grad_y, float *grad_w,
