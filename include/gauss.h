@@ -32,8 +32,8 @@
  *                        weights this is exact for |w| in [2^-14, 65504]).
  *                        The log-sum-exp runs on the tf32 tensor-core path
  *                        (fp16 / bf16 values are exact in tf32).
- *     The log-sum-exp backward: GS_F32, 1 <= D <= 128.  The k-nearest
- *     reduction: GS_F32, D <= 8.
+ *     The log-sum-exp backward and the k-nearest reduction: GS_F32,
+ *     1 <= D <= 128.
  *   Anything else returns GS_ERR_UNSUPPORTED; there is no CPU fallback.
  *
  * Ownership and synchronisation: the caller owns every buffer, allocates the
@@ -193,7 +193,7 @@ gs_status gauss_lse_bwd(const void *x, const void *y, const void *w, const float
  * d = fma(e_k, e_k, d) for k = 1 .. D-1 (round to nearest), and every
  * comparison is made on those fp32 values.
  *     out_sqdist [B, M, K] float32, out_index [B, M, K] int64.
- * GS_F32, 1 <= D <= 8, 1 <= K <= 32.  Workspace:
+ * GS_F32, 1 <= D <= 128, 1 <= K <= 32.  Workspace:
  * gs_workspace_bytes(GS_OP_KNN, B, M, N, D, K, GS_F32).
  */
 gs_status gauss_knn(const void *x, const void *y, float *out_sqdist, int64_t *out_index, int64_t B,

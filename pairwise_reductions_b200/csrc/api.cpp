@@ -48,7 +48,6 @@ gs_status check_dims(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, int64
   if (dt == GS_F32) {
     // D > 8: the split-tf32 tensor-core path, for the Gauss-sum passes only
     if (D > kTcMaxD) return GS_ERR_UNSUPPORTED;
-    if (D > kSdMaxD && op == GS_OP_KNN) return GS_ERR_UNSUPPORTED;
   } else {
     if (D > kTcMaxD) return GS_ERR_UNSUPPORTED;
     if (op == GS_OP_LSE_BWD) return GS_ERR_UNSUPPORTED;   // (the forward runs on the tf32 path)
@@ -537,7 +536,7 @@ size_t gs_workspace_bytes(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, 
     if (dt != GS_F32 || C < 1 || C > kKnnMaxK || check_dims(GS_OP_KNN, B, M, N, D, 1, dt) != GS_OK)
       return kBad;
     if (B == 0 || M == 0 || N == 0) return 0;
-    const KnnPlan kp = knn_plan(B, M, N, static_cast<int>(C), sm_count());
+    const KnnPlan kp = knn_plan(B, M, N, D, static_cast<int>(C), sm_count());
     return align_up(size_t(kp.splits) * B * M * C * 8);
   }
   if (check_dims(op, B, M, N, D, C, dt) != GS_OK) return kBad;
@@ -847,7 +846,7 @@ gs_status gauss_knn(const void* x, const void* y, float* out_sqdist, int64_t* ou
     GS_CUDA(cudaMemsetAsync(out_index, 0xff, size_t(B) * M * K * sizeof(int64_t), s));
     return GS_OK;
   }
-  const KnnPlan kp = knn_plan(B, M, N, static_cast<int>(K), sm_count());
+  const KnnPlan kp = knn_plan(B, M, N, D, static_cast<int>(K), sm_count());
   const size_t need = align_up(size_t(kp.splits) * B * M * K * 8);
   if (ws_bytes < need) return GS_ERR_WORKSPACE;
   GS_TRY(check_ptr(ws, 1));

@@ -234,7 +234,7 @@ struct KnnPlan {
   int splits;
   int64_t cols_per_split;
 };
-KnnPlan knn_plan(int64_t B, int64_t M, int64_t N, int K, int sm_count);
+KnnPlan knn_plan(int64_t B, int64_t M, int64_t N, int64_t D, int K, int sm_count);
 struct KnnArgs {
   const float* x;
   const float* y;

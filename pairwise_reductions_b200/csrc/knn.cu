@@ -1,5 +1,5 @@
 // knn.cu -- the k-nearest reduction (min / argKmin) on the CUDA-core path
-// (fp32, 1 <= D <= 8, 1 <= K <= 32).
+// (fp32, 1 <= D <= 128, 1 <= K <= 32).
 //
 // For each row i: the K smallest squared distances |x_i - y_j|^2 over j,
 // ascending, with their indices, equal distances ordered by the lower index
@@ -16,6 +16,11 @@
 // memory; within one thread the indices arrive in increasing order, so a
 // strict "<" against the current K-th distance keeps the lower index on ties.
 // Column splits are merged afterwards, ties again by the lower index.
+// D > 8: the rows' coordinates no longer fit in registers, so a tile of TJ
+// points is staged 8 dimensions at a time and every (row, point) pair keeps
+// its partial distance in a register across the chunks -- the same fp32
+// operations in the same order (fma(e_k, e_k, d) for ascending k, starting
+// from fma(e_0, e_0, +0) = e_0 e_0), so the decisions are unchanged.
 #include <cmath>
 
 #include "internal.h"
@@ -140,6 +145,94 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+constexpr int kDC = 8;   // dimensions per staged chunk (wide kernel)
+
+template <int K, int TJ>
+__global__ void __launch_bounds__(kThreads)
+    knn_wide_kernel(const float* __restrict__ x, const float* __restrict__ y, float* __restrict__ od,
+                    int* __restrict__ oi, int64_t M, int64_t N, int D, int64_t cols_per_split,
+                    int64_t split_stride, int Kout) {
+  // negated coordinates of TJ points x 8 dimensions, each duplicated for the
+  // packed (two-row) arithmetic
+  __shared__ __align__(16) float tile[TJ][2 * kDC];
+  const int tid = threadIdx.x;
+  const int64_t b = blockIdx.z;
+  const int split = blockIdx.y;
+  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * (2 * kThreads) + tid;
+  const int64_t i1 = i0 + kThreads;
+  const int64_t jbeg = static_cast<int64_t>(split) * cols_per_split;
+  const int64_t jend = min(N, jbeg + cols_per_split);
+  const float* __restrict__ x0 = x + (b * M + i0) * D;
+  const float* __restrict__ x1 = x + (b * M + i1) * D;
+  const float* __restrict__ yb = y + b * N * D;
+  float bd[2][K];
+  int bj[2][K];
+#pragma unroll
+  for (int r = 0; r < 2; ++r)
+#pragma unroll
+    for (int p = 0; p < K; ++p) {
+      bd[r][p] = INFINITY;
+      bj[r][p] = -1;
+    }
+  for (int64_t j0 = jbeg; j0 < jend; j0 += TJ) {
+    uint64_t d[TJ];
+#pragma unroll
+    for (int jj = 0; jj < TJ; ++jj) d[jj] = 0ull;   // +0: fma(e_0, e_0, +0) = e_0 e_0
+    for (int k0 = 0; k0 < D; k0 += kDC) {
+      __syncthreads();   // the previous chunk has been read
+      for (int idx = tid; idx < TJ * kDC; idx += kThreads) {
+        const int jj = idx / kDC, kk = idx % kDC;
+        const int64_t j = j0 + jj;
+        const int k = k0 + kk;
+        const float v = (j < jend && k < D) ? -yb[j * D + k] : 0.f;
+        tile[jj][2 * kk] = v;
+        tile[jj][2 * kk + 1] = v;
+      }
+      __syncthreads();
+      // dimensions past D are 0 on both sides: fma(0, 0, d) = d exactly
+      uint64_t xk[kDC];
+#pragma unroll
+      for (int kk = 0; kk < kDC; ++kk) {
+        const int k = k0 + kk;
+        xk[kk] = pk2((i0 < M && k < D) ? x0[k] : 0.f, (i1 < M && k < D) ? x1[k] : 0.f);
+      }
+      const ulonglong2* t2 = reinterpret_cast<const ulonglong2*>(&tile[0][0]);
+#pragma unroll
+      for (int jj = 0; jj < TJ; ++jj) {
+#pragma unroll
+        for (int v = 0; v < kDC / 2; ++v) {
+          const ulonglong2 u = t2[jj * (kDC / 2) + v];
+          uint64_t e = add2(xk[2 * v], u.x);
+          d[jj] = fma2(e, e, d[jj]);
+          e = add2(xk[2 * v + 1], u.y);
+          d[jj] = fma2(e, e, d[jj]);
+        }
+      }
+    }
+#pragma unroll
+    for (int jj = 0; jj < TJ; ++jj) {
+      const int64_t j = j0 + jj;
+      if (j >= jend) break;
+      float d0, d1;
+      upk2(d[jj], d0, d1);
+      if (d0 < bd[0][K - 1]) insert<K>(bd[0], bj[0], d0, static_cast<int>(j));
+      if (d1 < bd[1][K - 1]) insert<K>(bd[1], bj[1], d1, static_cast<int>(j));
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int64_t i = r ? i1 : i0;
+    if (i >= M) continue;
+    const int64_t base = split * split_stride + (b * M + i) * Kout;
+#pragma unroll
+    for (int p = 0; p < K; ++p) {
+      if (p >= Kout) break;
+      od[base + p] = bd[r][p];
+      oi[base + p] = bj[r][p];
+    }
+  }
+}
+
 // Merge the sorted per-split lists of each row (ties by the lower index) and
 // write the final distances and 64-bit indices.
 __global__ void knn_merge_kernel(const float* __restrict__ pd, const int* __restrict__ pi,
@@ -188,6 +281,26 @@ cudaError_t launch_t(const KnnArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+template <int K>
+cudaError_t launch_wide_t(const KnnArgs& a, cudaStream_t s) {
+  constexpr int TJ = K >= 16 ? 16 : 32;
+  const int64_t tiles = (a.M + 2 * kThreads - 1) / (2 * kThreads);
+  const dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(a.splits),
+                  static_cast<unsigned>(a.B));
+  knn_wide_kernel<K, TJ><<<grid, kThreads, 0, s>>>(a.x, a.y, a.part_d, a.part_i, a.M, a.N, a.D,
+                                                   a.cols_per_split, a.split_stride, a.K);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wide(const KnnArgs& a, cudaStream_t s) {
+  if (a.K <= 1) return launch_wide_t<1>(a, s);
+  if (a.K <= 2) return launch_wide_t<2>(a, s);
+  if (a.K <= 4) return launch_wide_t<4>(a, s);
+  if (a.K <= 8) return launch_wide_t<8>(a, s);
+  if (a.K <= 16) return launch_wide_t<16>(a, s);
+  return launch_wide_t<32>(a, s);
+}
+
 template <int D>
 cudaError_t launch_k(const KnnArgs& a, cudaStream_t s) {
   if (a.K <= 1) return launch_t<D, 1>(a, s);
@@ -207,9 +320,10 @@ int grid_for(int64_t n, int threads) {
 
 }  // namespace
 
-KnnPlan knn_plan(int64_t B, int64_t M, int64_t N, int K, int sm_count) {
+KnnPlan knn_plan(int64_t B, int64_t M, int64_t N, int64_t D, int K, int sm_count) {
   KnnPlan p{};
-  const int R = knn_rows(K <= 1 ? 1 : (K <= 2 ? 2 : (K <= 4 ? 4 : (K <= 8 ? 8 : (K <= 16 ? 16 : 32)))));
+  const int R = D > 8 ? 2
+                      : knn_rows(K <= 1 ? 1 : (K <= 2 ? 2 : (K <= 4 ? 4 : (K <= 8 ? 8 : (K <= 16 ? 16 : 32)))));
   const int64_t U = B * ((M + kThreads * R - 1) / (kThreads * R));
   int64_t smax = N / 512;
   if (smax > 32) smax = 32;
@@ -243,7 +357,10 @@ cudaError_t launch_knn(const KnnArgs& a, cudaStream_t s) {
     case 6: e = launch_k<6>(a, s); break;
     case 7: e = launch_k<7>(a, s); break;
     case 8: e = launch_k<8>(a, s); break;
-    default: return cudaErrorInvalidValue;
+    default:
+      if (a.D > 128) return cudaErrorInvalidValue;
+      e = launch_wide(a, s);
+      break;
   }
   if (e != cudaSuccess) return e;
   const int64_t rows = a.B * a.M;

@@ -77,14 +77,14 @@ def test_lse_in_half_precision_runs_on_the_tf32_path():
 
 
 def test_fp32_wide_features_route_to_the_tensor_core_path():
-    # fp32 with D > 8 (split-tf32 tensor cores): sums, the log-sum-exp and its
-    # backward are supported (they ask for their workspace); kNN stays on the
-    # small-D path
+    # fp32 with D > 8: sums, the log-sum-exp and its backward (split-tf32 tensor
+    # cores) and kNN (chunked CUDA-core kernel) ask for their workspace
     assert _fwd("gauss_lse_fwd", D=9) == 4
     assert _fwd("gauss_sum_fwd", D=9) == 4
     lib = gs.library()
     i64 = ctypes.c_void_p(0x100000)
-    assert lib.gauss_knn(FAKE, FAKE, FAKE, i64, 1, 10, 10, 9, 1, 0, NULL, 0, NULL) == 2
+    assert lib.gauss_knn(FAKE, FAKE, FAKE, i64, 1, 10, 10, 9, 1, 0, NULL, 0, NULL) == 4
+    assert lib.gauss_knn(FAKE, FAKE, FAKE, i64, 1, 10, 10, 129, 1, 0, NULL, 0, NULL) == 2
 
 
 def test_empty_problems_are_no_ops_without_pointers():
@@ -112,8 +112,9 @@ def test_workspace_query():
         ws(gs.GS_OP_SUM, 1, 10, 10, 129, 1, gs.GS_F32)
     assert ws(gs.GS_OP_LSE, 1, 1000, 1000, 9, 1, gs.GS_F32) >= 2 * 1000 * 2 * 16 * 4
     assert ws(gs.GS_OP_LSE_BWD, 1, 1000, 1000, 9, 1, gs.GS_F32) > 0
+    assert ws(gs.GS_OP_KNN, 1, 10, 10, 9, 1, gs.GS_F32) > 0
     with pytest.raises(ValueError):
-        ws(gs.GS_OP_KNN, 1, 10, 10, 9, 1, gs.GS_F32)
+        ws(gs.GS_OP_KNN, 1, 10, 10, 129, 1, gs.GS_F32)
     with pytest.raises(ValueError):
         ws(7, 1, 10, 10, 3, 1, gs.GS_F32)
 

@@ -427,7 +427,8 @@ def test_lse_bwd_rows_far_from_every_point():
 # ------------------------------------------------------------------ k-nearest reduction
 @pytest.mark.parametrize("shape", [(1, 1000, 3000, 3, 1), (2, 777, 1301, 3, 5), (1, 300, 5000, 8, 32),
                                    (1, 513, 257, 2, 16), (1, 50, 10, 3, 16), (3, 129, 4097, 1, 8),
-                                   (1, 2049, 20000, 3, 4)])
+                                   (1, 2049, 20000, 3, 4), (1, 300, 1000, 9, 5), (2, 257, 700, 16, 32),
+                                   (1, 400, 1500, 33, 1), (1, 129, 300, 100, 16), (1, 200, 999, 128, 8)])
 def test_knn_bit_exact(shape):
     """Indices bit-exact, distances bit-exact: both sides decide in fp32 with the
     same order of operations, ties by the lower index."""
@@ -440,12 +441,14 @@ def test_knn_bit_exact(shape):
     assert np.array_equal(od.cpu().numpy(), rd), "distances differ"
 
 
-def test_knn_duplicates_and_quantised_grid():
-    """Many exact ties: duplicated sources and points on a coarse grid."""
+@pytest.mark.parametrize("D", [3, 12, 40])
+def test_knn_duplicates_and_quantised_grid(D):
+    """Many exact ties: duplicated sources and points on a coarse grid (D > 8:
+    the chunked kernel)."""
     g = torch.Generator().manual_seed(20)
-    y = torch.randint(0, 4, (1, 3000, 3), generator=g).float() * 0.5
+    y = torch.randint(0, 4, (1, 3000, D), generator=g).float() * 0.5
     y = torch.cat([y, y[:, :500]], dim=1)                 # exact duplicates at higher indices
-    x = torch.randint(0, 4, (1, 700, 3), generator=g).float() * 0.5 + 0.25
+    x = torch.randint(0, 4, (1, 700, D), generator=g).float() * 0.5 + 0.25
     od, oi = gs().gauss_knn(x.cuda(), y.cuda(), 12)
     rd, ri = oracle.knn(x.numpy(), y.numpy(), 12, f32=True)
     assert np.array_equal(oi.cpu().numpy(), ri)
