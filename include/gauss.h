@@ -122,6 +122,38 @@ gs_status gauss_lse_fwd(const void *x, const void *y, const void *w, float *out,
                         void *ws, size_t ws_bytes, gs_stream_t stream);
 
 /*
+ * Forward sum that also keeps what the x-gradient needs, for a forward pass
+ * followed by a backward pass on the same inputs.  The gradient formula of
+ * gauss_sum_bwd splits as
+ *
+ *     grad_x[b,i,k] = -tau * sum_c g[b,i,c] ((x_ik - z_k) s0[b,i,c] - s1[b,i,c,k])
+ *     s0[b,i,c]   = sum_j K_ij w[b,j,c]                 (= out[b,i,c])
+ *     s1[b,i,c,k] = sum_j K_ij w[b,j,c] (y_jk - z_k),   z = x[b,0,:]
+ *
+ * and neither s0 nor s1 depends on the upstream gradient g, so one fused pass
+ * computes them with the forward result.  `saved` [B, M, C * (1 + D)] float32
+ * receives [s0 (C) | s1 (C x D, channel c's D values together)] per row;
+ * `out` [B, M, C] receives s0.  The pages keep no such sums (they recompute
+ * every reduction from scratch): this is a reuse of the same reductions, no
+ * approximation.  Workspace: gs_workspace_bytes(GS_OP_SUM_BWD, ...) is enough.
+ */
+gs_status gauss_sum_fwd_saved(const void *x, const void *y, const void *w, float *out,
+                              float *saved, int64_t B, int64_t M, int64_t N, int64_t D,
+                              int64_t C, float tau, gs_dtype dt, void *ws, size_t ws_bytes,
+                              gs_stream_t stream);
+
+/*
+ * The backward of gauss_sum_bwd from the sums gauss_sum_fwd_saved kept for the
+ * same x, y, w, tau: grad_x from `saved` and g (a per-row epilogue, no pair
+ * work) and grad_w by one fused pass (rows y, columns x, values g).  Either
+ * output may be NULL.  Workspace: gs_workspace_bytes(GS_OP_SUM_BWD, ...).
+ */
+gs_status gauss_sum_bwd_saved(const void *x, const void *y, const void *w, const float *g,
+                              const float *saved, float *grad_x, float *grad_w, int64_t B,
+                              int64_t M, int64_t N, int64_t D, int64_t C, float tau, gs_dtype dt,
+                              void *ws, size_t ws_bytes, gs_stream_t stream);
+
+/*
  * Gradient of L = sum_{b,i,c} g[b,i,c] * out[b,i,c] for the Gaussian kernel sum
  * ("Kernel matrix reduction", Variants: gradients through the same fused
  * reduction; the torch.autograd.grad example of the LazyTensor API):

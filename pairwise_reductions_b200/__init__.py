@@ -40,6 +40,10 @@ SIGNATURES = {
                                      _f, ctypes.c_int, _vp, _sz, _vp]),
     "gauss_sum_vjp": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                      _i64, _f, ctypes.c_int, _vp, _sz, _vp]),
+    "gauss_sum_fwd_saved": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64,
+                                           _f, ctypes.c_int, _vp, _sz, _vp]),
+    "gauss_sum_bwd_saved": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                           _i64, _i64, _f, ctypes.c_int, _vp, _sz, _vp]),
     "gauss_lse_bwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
                                      _i64, _i64, _f, ctypes.c_int, _vp, _sz, _vp]),
     "gauss_knn": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, ctypes.c_int, _vp,
@@ -66,7 +70,7 @@ class GaussError(RuntimeError):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m pairwise_reductions_b200.build` (needs nvcc)")
+                          "`python pairwise_reductions_b200/build.py` (needs nvcc)")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in SIGNATURES.items():
         f = getattr(lib, name)
@@ -192,6 +196,45 @@ def gauss_sum_bwd(x, y, w, g, tau, want_x=True, want_w=True, workspace=None, str
     return gx, gw
 
 
+def gauss_sum_fwd_saved(x, y, w, tau, out=None, saved=None, workspace=None, stream=None):
+    """The forward sum plus the sums its x-gradient needs (one fused pass):
+    returns (out [B, M, C], saved [B, M, C (1 + D)]) for gauss_sum_bwd_saved."""
+    x, y, w = _as3(x, "x"), _as3(y, "y"), _as3(w, "w")
+    B, M, N, D, C = _dims(x, y, w)
+    if out is None:
+        out = torch.empty((B, M, C), dtype=torch.float32, device=x.device)
+    if saved is None:
+        saved = torch.empty((B, M, C * (1 + D)), dtype=torch.float32, device=x.device)
+    nbytes = workspace_bytes(GS_OP_SUM_BWD, B, M, N, D, C, x.dtype)
+    ws = _workspace(nbytes, x.device, workspace)
+    st = _lib.gauss_sum_fwd_saved(_ptr(x), _ptr(y), _ptr(w), _ptr(out), _ptr(saved), B, M, N, D, C,
+                                  float(tau), _DT[x.dtype], _ptr(ws),
+                                  nbytes if ws is not None else 0, _stream(stream))
+    _check("gauss_sum_fwd_saved", st)
+    return out, saved
+
+
+def gauss_sum_bwd_saved(x, y, w, g, saved, tau, want_x=True, want_w=True, workspace=None,
+                        stream=None):
+    """gauss_sum_bwd from the sums gauss_sum_fwd_saved kept: (grad_x, grad_w)."""
+    x, y, w, g = _as3(x, "x"), _as3(y, "y"), _as3(w, "w"), _as3(g, "g")
+    B, M, N, D, C = _dims(x, y, w)
+    if g.shape != (B, M, C) or g.dtype != torch.float32:
+        raise ValueError(f"g must be float32 of shape {(B, M, C)}")
+    if saved.shape != (B, M, C * (1 + D)) or saved.dtype != torch.float32:
+        raise ValueError(f"saved must be float32 of shape {(B, M, C * (1 + D))}")
+    gx = torch.empty((B, M, D), dtype=torch.float32, device=x.device) if want_x else None
+    gw = torch.empty((B, N, C), dtype=torch.float32, device=x.device) if want_w else None
+    nbytes = workspace_bytes(GS_OP_SUM_BWD, B, M, N, D, C, x.dtype)
+    ws = _workspace(nbytes, x.device, workspace)
+    st = _lib.gauss_sum_bwd_saved(_ptr(x), _ptr(y), _ptr(w), _ptr(g), _ptr(saved),
+                                  _ptr(gx) if want_x else None, _ptr(gw) if want_w else None,
+                                  B, M, N, D, C, float(tau), _DT[x.dtype], _ptr(ws),
+                                  nbytes if ws is not None else 0, _stream(stream))
+    _check("gauss_sum_bwd_saved", st)
+    return gx, gw
+
+
 def gauss_sum_vjp(x, y, w, g, tau, want=("x", "y", "w", "tau"), workspace=None, stream=None):
     """Every first-order gradient of sum(g * gauss_sum_fwd(x, y, w, tau)):
     returns a dict with the requested keys among x, y, w, tau."""
@@ -300,6 +343,7 @@ def last_device_error(stream=None):
     return int(_lib.gs_last_device_error(_stream(stream)))
 
 
-__all__ = ["gauss_sum_fwd", "gauss_sum_fwd_noalloc", "gauss_lse_fwd", "gauss_sum_bwd", "gauss_sum_vjp", "gauss_lse_bwd", "gauss_knn", "gauss_diffusion_scales", "gauss_diffusion_apply", "workspace_bytes",
+__all__ = ["gauss_sum_fwd", "gauss_sum_fwd_noalloc", "gauss_lse_fwd", "gauss_sum_bwd",
+           "gauss_sum_fwd_saved", "gauss_sum_bwd_saved", "gauss_sum_vjp", "gauss_lse_bwd", "gauss_knn", "gauss_diffusion_scales", "gauss_diffusion_apply", "workspace_bytes",
            "last_device_error", "library", "status_string", "GaussError", "SIGNATURES",
            "LIB_PATH"]

@@ -765,6 +765,78 @@ gs_status gauss_sum_bwd(const void* x, const void* y, const void* w, const float
                        ws_bytes, stream);
 }
 
+gs_status gauss_sum_fwd_saved(const void* x, const void* y, const void* w, float* out,
+                              float* saved, int64_t B, int64_t M, int64_t N, int64_t D, int64_t C,
+                              float tau, gs_dtype dt, void* ws, size_t ws_bytes,
+                              gs_stream_t stream) {
+  GS_TRY(check_dims(GS_OP_SUM_BWD, B, M, N, D, C, dt));
+  GS_TRY(check_tau(tau));
+  GS_TRY(check_ptr(x, B * M * D));
+  GS_TRY(check_ptr(y, B * N * D));
+  GS_TRY(check_ptr(w, B * N * C));
+  GS_TRY(check_ptr(out, B * M * C));
+  const int CV = value_channels(1, static_cast<int>(C), static_cast<int>(D));
+  GS_TRY(check_ptr(saved, B * M * CV));
+  if (B == 0 || M == 0) return GS_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (N == 0) {
+    GS_CUDA(cudaMemsetAsync(out, 0, size_t(B) * M * C * 4, s));
+    GS_CUDA(cudaMemsetAsync(saved, 0, size_t(B) * M * CV * 4, s));
+    return GS_OK;
+  }
+  // the x-gradient pass: values [w, w (y - z)]; its first C channels are the sum
+  Pass px = fwd_pass(x, y, w, B, M, N, D, C, tau, dt);
+  px.vmode = 1;
+  px.CV = CV;
+  const PassLayout lx = pass_layout(px, sm_count());
+  if (lx.total > 0) {
+    if (ws_bytes < lx.total) return GS_ERR_WORKSPACE;
+    GS_TRY(check_ptr(ws, 1));
+  }
+  GS_TRY(run_pass(px, lx, saved, static_cast<uint8_t*>(ws), s));
+  GS_CUDA(cudaMemcpy2DAsync(out, size_t(C) * 4, saved, size_t(CV) * 4, size_t(C) * 4,
+                            size_t(B) * M, cudaMemcpyDeviceToDevice, s));
+  return GS_OK;
+}
+
+gs_status gauss_sum_bwd_saved(const void* x, const void* y, const void* w, const float* g,
+                              const float* saved, float* grad_x, float* grad_w, int64_t B,
+                              int64_t M, int64_t N, int64_t D, int64_t C, float tau, gs_dtype dt,
+                              void* ws, size_t ws_bytes, gs_stream_t stream) {
+  GS_TRY(check_dims(GS_OP_SUM_BWD, B, M, N, D, C, dt));
+  GS_TRY(check_tau(tau));
+  GS_TRY(check_ptr(x, B * M * D));
+  GS_TRY(check_ptr(y, B * N * D));
+  GS_TRY(check_ptr(w, B * N * C));
+  GS_TRY(check_ptr(g, B * M * C));
+  const int CV = value_channels(1, static_cast<int>(C), static_cast<int>(D));
+  GS_TRY(check_ptr(saved, B * M * CV));
+  if (grad_x) GS_TRY(check_ptr(grad_x, B * M * D));
+  if (grad_w) GS_TRY(check_ptr(grad_w, B * N * C));
+  if (!grad_x && !grad_w) return GS_OK;
+  if (B == 0) return GS_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (M == 0 || N == 0) {   // every kernel sum is empty: all gradients vanish
+    if (grad_x && M > 0) GS_CUDA(cudaMemsetAsync(grad_x, 0, size_t(B) * M * D * 4, s));
+    if (grad_w && N > 0) GS_CUDA(cudaMemsetAsync(grad_w, 0, size_t(B) * N * C * 4, s));
+    return GS_OK;
+  }
+  if (grad_w) {   // rows y, columns x, values g: dL/dw directly
+    Pass py = fwd_pass(y, x, g, B, N, M, D, C, tau, dt);
+    py.w_is_f32 = true;
+    const PassLayout ly = pass_layout(py, sm_count());
+    if (ly.total > 0) {
+      if (ws_bytes < ly.total) return GS_ERR_WORKSPACE;
+      GS_TRY(check_ptr(ws, 1));
+    }
+    GS_TRY(run_pass(py, ly, grad_w, static_cast<uint8_t*>(ws), s));
+  }
+  if (grad_x)
+    GS_CUDA(launch_grad_x_epilogue(x, dt, g, saved, grad_x, nullptr, B, M, static_cast<int>(D),
+                                   static_cast<int>(C), CV, tau, s));
+  return GS_OK;
+}
+
 gs_status gauss_lse_bwd(const void* x, const void* y, const void* w, const float* lse,
                         const float* g, float* grad_x, float* grad_y, float* grad_w,
                         float* grad_tau, int64_t B, int64_t M, int64_t N, int64_t D, int64_t C,

@@ -333,6 +333,36 @@ def test_tensor_core_path_is_deterministic_under_repetition(C):
     assert rel_l2(ref.cpu().numpy()[:, ::7], ro) <= TOL["f16"]
 
 
+# ------------------------------------------------------------------ forward that keeps the x-gradient sums
+@pytest.mark.parametrize("dtype,shape", [("f32", (1, 400, 600, 3, 1)), ("f32", (2, 300, 500, 2, 3)),
+                                         ("f16", (1, 300, 500, 32, 1)), ("bf16", (2, 257, 300, 16, 2)),
+                                         ("f32", (1, 250, 400, 32, 2))])
+def test_fwd_saved_then_bwd_saved(dtype, shape):
+    """gauss_sum_fwd_saved + gauss_sum_bwd_saved against the oracle (and against
+    the separate forward and backward entry points)."""
+    B, M, N, D, C = shape
+    wid = 1 if (dtype == "f32" and D <= 8) else 5
+    inp = synth.make_inputs(wid, seed=21, B=B, M=M, N=N, D=D, C=C, dtype=dtype, with_g=True)
+    d = dev(inp)
+    m = gs()
+    out, saved = m.gauss_sum_fwd_saved(d["x"], d["y"], d["w"], inp["tau"])
+    assert saved.shape == (B, M, C * (1 + D))
+    gx, gw = m.gauss_sum_bwd_saved(d["x"], d["y"], d["w"], d["g"], saved, inp["tau"])
+    x, y, w, g = (f64(inp, k) for k in "xywg")
+    ref = oracle.gauss_sum(x, y, w, inp["tau"])
+    rgx, rgw = oracle.gauss_sum_bwd(x, y, w, g, inp["tau"])
+    tol = TOL[dtype]
+    assert rel_l2(out.cpu().numpy(), ref) <= tol, rel_l2(out.cpu().numpy(), ref)
+    assert rel_l2(gx.cpu().numpy(), rgx) <= tol, rel_l2(gx.cpu().numpy(), rgx)
+    assert rel_l2(gw.cpu().numpy(), rgw) <= tol, rel_l2(gw.cpu().numpy(), rgw)
+    # the same grad_w pass as gauss_sum_bwd, bit for bit; grad_x from the same sums
+    bx, bw = m.gauss_sum_bwd(d["x"], d["y"], d["w"], d["g"], inp["tau"])
+    assert torch.equal(bw, gw)
+    assert torch.equal(bx, gx)
+    only_w = m.gauss_sum_bwd_saved(d["x"], d["y"], d["w"], d["g"], saved, inp["tau"], want_x=False)
+    assert only_w[0] is None and torch.equal(only_w[1], gw)
+
+
 # ------------------------------------------------------------------ full gradient
 @pytest.mark.parametrize("dtype,shape,shift", [
     ("f32", (1, 400, 600, 3, 1), 0.0), ("f32", (2, 300, 500, 2, 3), 0.0), ("f32", (1, 250, 350, 8, 2), 0.0),
