@@ -266,6 +266,22 @@ def test_empty_inputs():
     assert torch.equal(m.gauss_sum_fwd(xh, yh, wh, 1.0), torch.zeros(2, 5, 4, device="cuda"))
     gx, gw = m.gauss_sum_bwd(xh, yh, wh, torch.randn(2, 5, 4, device="cuda"), 1.0)
     assert torch.equal(gx, torch.zeros_like(gx)) and gw.shape == (2, 0, 4)
+    # the forward that keeps the gradient sums, and the backward from them
+    out, saved = m.gauss_sum_fwd_saved(xh, yh, wh, 1.0)
+    assert torch.equal(out, torch.zeros(2, 5, 4, device="cuda"))
+    assert torch.equal(saved, torch.zeros(2, 5, 4 * 33, device="cuda"))
+    gx, gw = m.gauss_sum_bwd_saved(xh, yh, wh, torch.randn(2, 5, 4, device="cuda"), saved, 1.0)
+    assert torch.equal(gx, torch.zeros_like(gx)) and gw.shape == (2, 0, 4)
+    # log-sum-exp on the tf32 paths (fp16, and fp32 with D > 8)
+    assert torch.isneginf(m.gauss_lse_fwd(xh, yh, wh, 1.0)).all()
+    xw, yw, ww0 = torch.randn(1, 6, 20, device="cuda"), torch.empty(1, 0, 20, device="cuda"), \
+        torch.empty(1, 0, 1, device="cuda")
+    assert torch.isneginf(m.gauss_lse_fwd(xw, yw, ww0, 1.0)).all()
+    assert torch.equal(m.gauss_sum_fwd(xw, yw, ww0, 1.0), torch.zeros(1, 6, 1, device="cuda"))
+    # k-nearest at D > 8 with fewer sources than K: +inf distances and index -1 pad
+    od, oi = m.gauss_knn(xw, torch.randn(1, 3, 20, device="cuda"), 5)
+    assert torch.isinf(od[..., 3:]).all() and (oi[..., 3:] == -1).all()
+    assert (oi[..., :3] >= 0).all()
 
 
 def test_coincident_points_give_the_weight_sum():
