@@ -32,8 +32,9 @@
  *                        weights this is exact for |w| in [2^-14, 65504]).
  *                        The log-sum-exp runs on the tf32 tensor-core path
  *                        (fp16 / bf16 values are exact in tf32).
- *     The log-sum-exp backward and the k-nearest reduction: GS_F32,
- *     1 <= D <= 128.
+ *     The log-sum-exp backward and the k-nearest reduction: every dtype,
+ *     1 <= D <= 128 (fp16 / bf16 inputs are widened, exactly, to fp32 copies
+ *     in the workspace and take the fp32 implementation).
  *   Anything else returns GS_ERR_UNSUPPORTED; there is no CPU fallback.
  *
  * Ownership and synchronisation: the caller owns every buffer, allocates the
@@ -204,8 +205,9 @@ gs_status gauss_sum_vjp(const void *x, const void *y, const void *w, const float
  *
  * lse [B, M, C] float32 is the forward's output for the same inputs.  The
  * shift -lse is folded into every kernel exponent, so the passes sum p
- * directly (no overflow, no separate normalisation).  GS_F32, 1 <= D <= 128
- * (D > 8: tf32 tensor-core passes), w > 0; any output may be NULL.  Workspace:
+ * directly (no overflow, no separate normalisation).  1 <= D <= 128 (fp32:
+ * D > 8 on tf32 tensor-core passes; fp16 / bf16: exact fp32 copies first),
+ * w > 0; any output may be NULL.  Workspace:
  * gs_workspace_bytes(GS_OP_LSE_BWD, ...).
  */
 gs_status gauss_lse_bwd(const void *x, const void *y, const void *w, const float *lse,
@@ -225,7 +227,8 @@ gs_status gauss_lse_bwd(const void *x, const void *y, const void *w, const float
  * d = fma(e_k, e_k, d) for k = 1 .. D-1 (round to nearest), and every
  * comparison is made on those fp32 values.
  *     out_sqdist [B, M, K] float32, out_index [B, M, K] int64.
- * GS_F32, 1 <= D <= 128, 1 <= K <= 32.  Workspace:
+ * 1 <= D <= 128, 1 <= K <= 32; fp16 / bf16 inputs are widened (exactly) to
+ * fp32 copies in the workspace.  Workspace:
  * gs_workspace_bytes(GS_OP_KNN, B, M, N, D, K, GS_F32).
  */
 gs_status gauss_knn(const void *x, const void *y, float *out_sqdist, int64_t *out_index, int64_t B,

@@ -258,8 +258,8 @@ def gauss_sum_vjp(x, y, w, g, tau, want=("x", "y", "w", "tau"), workspace=None, 
 
 
 def gauss_lse_bwd(x, y, w, lse, g, tau, want=("x", "y", "w", "tau"), workspace=None, stream=None):
-    """Every first-order gradient of sum(g * lse) with lse = gauss_lse_fwd(x, y, w, tau)
-    (float32 inputs); returns a dict with the requested keys among x, y, w, tau."""
+    """Every first-order gradient of sum(g * lse) with lse = gauss_lse_fwd(x, y, w, tau);
+    returns a dict with the requested keys among x, y, w, tau."""
     x, y, w, lse, g = (_as3(t, n) for t, n in ((x, "x"), (y, "y"), (w, "w"), (lse, "lse"), (g, "g")))
     B, M, N, D, C = _dims(x, y, w)
     for t, n in ((lse, "lse"), (g, "g")):
@@ -282,7 +282,7 @@ def gauss_lse_bwd(x, y, w, lse, g, tau, want=("x", "y", "w", "tau"), workspace=N
 
 def gauss_knn(x, y, K, workspace=None, stream=None):
     """K smallest squared distances per row (ascending, ties by the lower index)
-    and their int64 indices; float32 inputs."""
+    and their int64 indices, decided in fp32 (fp16 / bf16 inputs exactly widened)."""
     x, y = _as3(x, "x"), _as3(y, "y")
     B, M, D = x.shape
     N = y.shape[1]

@@ -50,7 +50,6 @@ gs_status check_dims(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, int64
     if (D > kTcMaxD) return GS_ERR_UNSUPPORTED;
   } else {
     if (D > kTcMaxD) return GS_ERR_UNSUPPORTED;
-    if (op == GS_OP_LSE_BWD) return GS_ERR_UNSUPPORTED;   // (the forward runs on the tf32 path)
   }
   return GS_OK;
 }
@@ -384,6 +383,15 @@ VjpLayout vjp_layout(const void* x, const void* y, const void* w, const float* g
   return L;
 }
 
+// fp16 / bf16 inputs of the k-nearest reduction and of the log-sum-exp
+// backward are widened (exactly) to fp32 copies at the front of the workspace;
+// the fp32 implementation then runs on them.
+size_t widened_bytes(gs_dtype dt, int64_t B, int64_t M, int64_t N, int64_t D, int64_t Cw) {
+  if (dt == GS_F32) return 0;
+  return align_up(size_t(B) * M * D * 4) + align_up(size_t(B) * N * D * 4) +
+         align_up(size_t(B) * N * Cw * 4);
+}
+
 // Log-sum-exp forward on the fp32 tensor-core path (D > 8): packed operands,
 // the column norms / log-weights, and the per-split (m, l) partials.
 struct LseF32Layout {
@@ -533,11 +541,11 @@ size_t gs_workspace_bytes(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, 
   }
   if (op == GS_OP_KNN) {
     // C carries K for this op
-    if (dt != GS_F32 || C < 1 || C > kKnnMaxK || check_dims(GS_OP_KNN, B, M, N, D, 1, dt) != GS_OK)
+    if (C < 1 || C > kKnnMaxK || check_dims(GS_OP_KNN, B, M, N, D, 1, dt) != GS_OK)
       return kBad;
     if (B == 0 || M == 0 || N == 0) return 0;
     const KnnPlan kp = knn_plan(B, M, N, D, static_cast<int>(C), sm_count());
-    return align_up(size_t(kp.splits) * B * M * C * 8);
+    return widened_bytes(dt, B, M, N, D, 0) + align_up(size_t(kp.splits) * B * M * C * 8);
   }
   if (check_dims(op, B, M, N, D, C, dt) != GS_OK) return kBad;
   if (B == 0) return 0;
@@ -553,9 +561,9 @@ size_t gs_workspace_bytes(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, 
     return align_up(size_t(2) * sp.splits * B * M * C * 4);
   }
   if (op == GS_OP_LSE_BWD) {
-    if (dt != GS_F32) return kBad;
     if (M == 0 || N == 0) return 0;
-    return lse_bwd_layout(nullptr, nullptr, nullptr, nullptr, nullptr, B, M, N, D, C, 1.f, sm).total;
+    return widened_bytes(dt, B, M, N, D, C) +
+           lse_bwd_layout(nullptr, nullptr, nullptr, nullptr, nullptr, B, M, N, D, C, 1.f, sm).total;
   }
   if (M == 0 || N == 0) return 0;
   return vjp_layout(nullptr, nullptr, nullptr, nullptr, B, M, N, D, C, 1.f, dt, sm, true, true, true,
@@ -853,6 +861,22 @@ gs_status gauss_lse_bwd(const void* x, const void* y, const void* w, const float
   if (grad_w) GS_TRY(check_ptr(grad_w, B * N * C));
   if (!grad_x && !grad_y && !grad_w && !grad_tau) return GS_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dt != GS_F32 && B > 0 && M > 0 && N > 0) {
+    // exact fp32 copies of x, y, w, then the fp32 backward on them
+    const size_t pre = widened_bytes(dt, B, M, N, D, C);
+    if (ws_bytes < pre) return GS_ERR_WORKSPACE;
+    GS_TRY(check_ptr(ws, 1));
+    uint8_t* w8 = static_cast<uint8_t*>(ws);
+    float* wx = reinterpret_cast<float*>(w8);
+    float* wy = reinterpret_cast<float*>(w8 + align_up(size_t(B) * M * D * 4));
+    float* ww = reinterpret_cast<float*>(w8 + align_up(size_t(B) * M * D * 4) +
+                                         align_up(size_t(B) * N * D * 4));
+    GS_CUDA(launch_widen_to_f32(x, dt, wx, B * M * D, s));
+    GS_CUDA(launch_widen_to_f32(y, dt, wy, B * N * D, s));
+    GS_CUDA(launch_widen_to_f32(w, dt, ww, B * N * C, s));
+    return gauss_lse_bwd(wx, wy, ww, lse, g, grad_x, grad_y, grad_w, grad_tau, B, M, N, D, C, tau,
+                         GS_F32, w8 + pre, ws_bytes - pre, stream);
+  }
   if (grad_tau) GS_CUDA(cudaMemsetAsync(grad_tau, 0, sizeof(float), s));
   if (B == 0) return GS_OK;
   if (M == 0 || N == 0) {   // no terms: every gradient vanishes
@@ -906,7 +930,7 @@ gs_status gauss_knn(const void* x, const void* y, float* out_sqdist, int64_t* ou
                     size_t ws_bytes, gs_stream_t stream) {
   GS_TRY(check_dims(GS_OP_KNN, B, M, N, D, 1, dt));
   if (K < 1) return GS_ERR_INVALID_ARG;
-  if (dt != GS_F32 || K > kKnnMaxK) return GS_ERR_UNSUPPORTED;
+  if (K > kKnnMaxK) return GS_ERR_UNSUPPORTED;
   GS_TRY(check_ptr(x, B * M * D));
   GS_TRY(check_ptr(y, B * N * D));
   GS_TRY(check_ptr(out_sqdist, B * M * K));
@@ -919,14 +943,26 @@ gs_status gauss_knn(const void* x, const void* y, float* out_sqdist, int64_t* ou
     return GS_OK;
   }
   const KnnPlan kp = knn_plan(B, M, N, D, static_cast<int>(K), sm_count());
-  const size_t need = align_up(size_t(kp.splits) * B * M * K * 8);
+  const size_t pre = widened_bytes(dt, B, M, N, D, 0);
+  const size_t need = pre + align_up(size_t(kp.splits) * B * M * K * 8);
   if (ws_bytes < need) return GS_ERR_WORKSPACE;
   GS_TRY(check_ptr(ws, 1));
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  const float* xf = static_cast<const float*>(x);
+  const float* yf = static_cast<const float*>(y);
+  if (dt != GS_F32) {   // exact fp32 copies: the decisions are those of fp32 on the same values
+    float* wx = reinterpret_cast<float*>(w8);
+    float* wy = reinterpret_cast<float*>(w8 + align_up(size_t(B) * M * D * 4));
+    GS_CUDA(launch_widen_to_f32(x, dt, wx, B * M * D, s));
+    GS_CUDA(launch_widen_to_f32(y, dt, wy, B * N * D, s));
+    xf = wx;
+    yf = wy;
+  }
   KnnArgs a{};
-  a.x = static_cast<const float*>(x);
-  a.y = static_cast<const float*>(y);
-  a.part_d = static_cast<float*>(ws);
-  a.part_i = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + size_t(kp.splits) * B * M * K * 4);
+  a.x = xf;
+  a.y = yf;
+  a.part_d = reinterpret_cast<float*>(w8 + pre);
+  a.part_i = reinterpret_cast<int*>(w8 + pre + size_t(kp.splits) * B * M * K * 4);
   a.out_d = out_sqdist;
   a.out_i = out_index;
   a.B = B;

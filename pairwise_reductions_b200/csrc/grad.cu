@@ -346,6 +346,26 @@ cudaError_t launch_diffusion_elementwise(int op, const float* a, const float* b,
   return cudaGetLastError();
 }
 
+template <typename T>
+__global__ void widen_kernel(const T* __restrict__ src, float* __restrict__ dst, int64_t n) {
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    dst[e] = tf(src[e]);
+}
+
+cudaError_t launch_widen_to_f32(const void* src, gs_dtype dt, float* dst, int64_t n,
+                                cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int blocks = grid_for(n, 256);
+  if (dt == GS_F16)
+    widen_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<const __half*>(src), dst, n);
+  else if (dt == GS_BF16)
+    widen_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(src), dst, n);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
 cudaError_t launch_sum_rows(const float* v, int64_t n, float* out, cudaStream_t s) {
   sum_rows_kernel<<<1, 1024, 0, s>>>(v, n, out);
   return cudaGetLastError();

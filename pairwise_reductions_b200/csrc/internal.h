@@ -126,6 +126,9 @@ cudaError_t launch_weighted_rows(const float* g, const float* o, float* tau_rows
 // op 3 o1[e] = a[e / C] * b[e].
 cudaError_t launch_diffusion_elementwise(int op, const float* a, const float* b, float* o1,
                                          float* o2, int64_t n, int C, float alpha, cudaStream_t s);
+// dst[0 .. n) = the fp16 / bf16 values of src as float32 (exact).
+cudaError_t launch_widen_to_f32(const void* src, gs_dtype dt, float* dst, int64_t n,
+                                cudaStream_t s);
 // out[0] = sum of v[0 .. n) in a fixed order (double accumulation).
 cudaError_t launch_sum_rows(const float* v, int64_t n, float* out, cudaStream_t s);
 

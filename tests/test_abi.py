@@ -67,13 +67,17 @@ def test_invalid_arguments_are_rejected_before_any_launch(fn):
     assert _fwd(fn, B=70000) == 2
 
 
-def test_lse_in_half_precision_runs_on_the_tf32_path():
-    # fp16 / bf16 log-sum-exp (exact tf32 operands) asks for its workspace; its
-    # backward has no half-precision path
+def test_every_entry_point_takes_half_precision():
+    # fp16 / bf16: the log-sum-exp (exact tf32 operands) asks for its workspace;
+    # its backward and kNN widen the inputs to fp32 copies in the workspace
     assert _fwd("gauss_lse_fwd", dt=1, D=32) == 4
     assert _fwd("gauss_lse_fwd", dt=2, D=3) == 4
-    with pytest.raises(ValueError):
-        gs.workspace_bytes(gs.GS_OP_LSE_BWD, 1, 10, 10, 3, 1, gs.GS_F16)
+    ws = gs.workspace_bytes
+    f32 = ws(gs.GS_OP_LSE_BWD, 1, 100, 200, 3, 2, gs.GS_F32)
+    f16 = ws(gs.GS_OP_LSE_BWD, 1, 100, 200, 3, 2, gs.GS_F16)
+    assert f16 >= f32 + (100 * 3 + 200 * 3 + 200 * 2) * 4     # plus the widened copies
+    assert ws(gs.GS_OP_KNN, 1, 100, 200, 3, 4, gs.GS_BF16) >= \
+        ws(gs.GS_OP_KNN, 1, 100, 200, 3, 4, gs.GS_F32) + (100 * 3 + 200 * 3) * 4
 
 
 def test_fp32_wide_features_route_to_the_tensor_core_path():

@@ -454,6 +454,25 @@ def test_lse_bwd_every_gradient(shape, shift):
     assert et <= TOL["f32"], ("tau", et, float(got["tau"].item()), rgt)
 
 
+@pytest.mark.parametrize("dtype,shape", [("f16", (1, 300, 500, 3, 1)), ("bf16", (2, 150, 300, 32, 2))])
+def test_lse_bwd_half_precision(dtype, shape):
+    """fp16 / bf16: the backward runs on exact fp32 copies of the inputs."""
+    B, M, N, D, C = shape
+    inp = synth.make_inputs(3, seed=27, B=B, M=M, N=N, D=D, C=C, with_g=True, tau=20.0, dtype=dtype)
+    if D > 8:
+        for k in ("x", "y"):
+            inp[k] = (inp[k].double() * (3.0 / D) ** 0.5).to(inp[k].dtype)
+    d = dev(inp)
+    lse = gs().gauss_lse_fwd(d["x"], d["y"], d["w"], inp["tau"])
+    got = gs().gauss_lse_bwd(d["x"], d["y"], d["w"], lse, d["g"], inp["tau"])
+    rgx, rgy, rgw, rgt = oracle.gauss_lse_bwd(*(f64(inp, k) for k in "xywg"), inp["tau"])
+    for name, ref in (("x", rgx), ("y", rgy), ("w", rgw)):
+        e = rel_l2(got[name].cpu().numpy(), ref)
+        assert e <= TOL[dtype], (name, e)
+    et = abs(float(got["tau"].item()) - rgt) / max(abs(rgt), 1e-30)
+    assert et <= TOL[dtype], ("tau", et)
+
+
 def test_lse_bwd_rows_far_from_every_point():
     """Rows whose kernel values all underflow fp32: the -lse shift in the
     exponent keeps the normalised weights exact."""
@@ -483,6 +502,19 @@ def test_knn_bit_exact(shape):
     d = dev(inp)
     od, oi = gs().gauss_knn(d["x"], d["y"], K)
     rd, ri = oracle.knn(inp["x"].numpy(), inp["y"].numpy(), K, f32=True)
+    assert np.array_equal(oi.cpu().numpy(), ri), "indices differ"
+    assert np.array_equal(od.cpu().numpy(), rd), "distances differ"
+
+
+@pytest.mark.parametrize("dtype,shape", [("f16", (1, 700, 2000, 3, 8)), ("bf16", (2, 300, 900, 16, 5)),
+                                         ("f16", (1, 257, 600, 64, 32))])
+def test_knn_half_precision_bit_exact(dtype, shape):
+    """fp16 / bf16 inputs: decided in fp32 on their exact fp32 values."""
+    B, M, N, D, K = shape
+    inp = synth.make_inputs(1, seed=25, B=B, M=M, N=N, D=D, C=1, dtype=dtype)
+    d = dev(inp)
+    od, oi = gs().gauss_knn(d["x"], d["y"], K)
+    rd, ri = oracle.knn(inp["x"].float().numpy(), inp["y"].float().numpy(), K, f32=True)
     assert np.array_equal(oi.cpu().numpy(), ri), "indices differ"
     assert np.array_equal(od.cpu().numpy(), rd), "distances differ"
 
