@@ -21,16 +21,26 @@
 // with S from the split MMAs; P is split into tf32 hi/lo again for P.v.
 //
 // CTA = one 128-row tile, 10 warps:
-//   warp 0      TMA producer: x' tile once, then a ring of (y' tile, v tile) stages
+//   warp 0      TMA producer: the x' rows once (unless they sit in TMEM), then a
+//               ring of stages: y' tile, a 16-byte record per column {q_j, values
+//               or log2 values}, and for tensor-core values the split v^T tile
 //   warp 1      TMEM owner + single-thread MMA issuer
 //   warps 2-5   exp warpgroup 0: column tiles 0, 2, 4, ...
 //   warps 6-9   exp warpgroup 1: column tiles 1, 3, 5, ...
 // Both warpgroups hold the same rows (TMEM lanes), so each keeps its own
-// accumulator O_h and warpgroup 0 adds O_0 + O_1 at the end.  Per column tile
+// partial result and warpgroup 0 combines the two at the end.  Per column tile
 // t of warpgroup h:
-//   S_h  = x'.y'(t)^T                 3 tf32 MMAs per K step (smem x smem -> TMEM)
-//   P_h  = ex2(fma(S_h, 2c, r) + q)   tcgen05.ld -> MUFU -> hi/lo -> tcgen05.st
-//   O_h += P_h . v(t)                 3 tf32 MMAs per K step (A = P from TMEM)
+//   S_h  = x'.y'(t)^T                 3 tf32 MMAs per K step (A from shared
+//                                     memory, or from TMEM when it has room)
+//   P_h  = ex2(fma(S_h, 2c, r) + q)   tcgen05.ld -> MUFU
+// then either (register values, <= 3 channels, and the log-sum-exp)
+//   row sums += P_h . v in registers, exact fp32 FMAs (or a running maximum and
+//   shifted sum for the log-sum-exp)
+// or (tensor-core values, 4 .. 64 channels per pass)
+//   P_h -> tf32 hi/lo -> tcgen05.st;  O_h += P_h . v(t), 3 tf32 MMAs per K step
+//   (A = P from TMEM).
+// fp16 / bf16 inputs (log-sum-exp) are exact in tf32: unsplit rows, one MMA
+// per K step (template SPLIT = false).
 // Every mbarrier wait is bounded (2 s); on expiry the kernel raises its device
 // error word, lets the other warps leave, frees TMEM and returns.
 #include <cuda.h>
