@@ -152,7 +152,7 @@ PassLayout pass_layout(const Pass& p, int sm) {
       off = align_up(off + size_t(L.f32.splits) * p.B * p.R * p.CV * 4);
     }
   } else if (!L.tc) {
-    L.sd = sd_plan(p.B, p.R, p.N, p.D, p.CV, sm);
+    L.sd = sd_plan(p.B, p.R, p.N, p.D, p.CV, sm, 256);
     if (p.vmode != 0) {
       L.off_vals = off;
       off = align_up(off + size_t(p.B) * p.N * p.CV * 4);
@@ -557,7 +557,7 @@ size_t gs_workspace_bytes(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, 
   if (op == GS_OP_LSE) {
     if (M == 0 || N == 0) return 0;
     if (dt != GS_F32 || D > kSdMaxD) return lse_f32_layout(B, M, N, D, C, dt, sm).total;
-    const SdPlan sp = sd_plan(B, M, N, static_cast<int>(D), C, sm);
+    const SdPlan sp = sd_plan(B, M, N, static_cast<int>(D), C, sm, 32);
     return align_up(size_t(2) * sp.splits * B * M * C * 4);
   }
   if (op == GS_OP_LSE_BWD) {
@@ -658,7 +658,7 @@ gs_status gauss_lse_fwd(const void* x, const void* y, const void* w, float* out,
     GS_CUDA(launch_lse_finalize(f, s));
     return GS_OK;
   }
-  const SdPlan sp = sd_plan(B, M, N, static_cast<int>(D), C, sm);
+  const SdPlan sp = sd_plan(B, M, N, static_cast<int>(D), C, sm, 32);
   const size_t need = align_up(size_t(2) * sp.splits * B * M * C * 4);
   if (ws_bytes < need) return GS_ERR_WORKSPACE;
   GS_TRY(check_ptr(ws, 1));

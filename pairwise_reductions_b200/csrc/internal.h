@@ -35,7 +35,8 @@ struct SdPlan {
 };
 
 // Choose rows per CTA and the j-split for the small-D kernel.
-SdPlan sd_plan(int64_t B, int64_t M, int64_t N, int D, int64_t C, int sm_count);
+// max_splits: 32 for the log-sum-exp (its finalize merges the splits in one warp)
+SdPlan sd_plan(int64_t B, int64_t M, int64_t N, int D, int64_t C, int sm_count, int max_splits);
 
 struct SdArgs {
   const float* x;

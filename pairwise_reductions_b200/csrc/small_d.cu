@@ -218,8 +218,11 @@ __global__ void __launch_bounds__(kSdThreads, sd_min_blocks(D, CP, SHIFT))
       for (int c = 0; c < CP; ++c) tacc[q][c] = 0ull;
 
     const ulonglong2* t2 = reinterpret_cast<const ulonglong2*>(tile);
+    // staged points past jend carry zero weight: a short last tile stops at
+    // its own width (rounded up to the unroll pair) instead of the full tile
+    const int nj = static_cast<int>(min(static_cast<int64_t>(kTileJ), jend - j0) + 1) & ~1;
 #pragma unroll 2
-    for (int jj = 0; jj < kTileJ; ++jj) {
+    for (int jj = 0; jj < nj; ++jj) {
       uint64_t pk[PK / 2];
 #pragma unroll
       for (int v = 0; v < PK / 4; ++v) {
@@ -467,31 +470,39 @@ int grid_for(int64_t n, int threads) {
 
 }  // namespace
 
-SdPlan sd_plan(int64_t B, int64_t M, int64_t N, int D, int64_t C, int sm_count) {
+SdPlan sd_plan(int64_t B, int64_t M, int64_t N, int D, int64_t C, int sm_count, int max_splits) {
   SdPlan p{};
   const int cw = static_cast<int>(C < kSdMaxChunk ? C : kSdMaxChunk);
   const int R = sd_rows_per_thread(D, sd_chunk_pad(cw));
   p.rows_per_cta = kSdThreads * R;
   const int64_t U = B * ((M + p.rows_per_cta - 1) / p.rows_per_cta);
-  int64_t smax = N / 256;
-  if (smax > 32) smax = 32;
+  // candidates: at least 128 columns a split, at most max_splits, and split
+  // partials of at most 2^25 floats
+  int64_t smax = N / 128;
+  if (smax > max_splits) smax = max_splits;
+  const int64_t part_cap = (int64_t(1) << 25) / (B * M * C > 0 ? B * M * C : 1);
+  if (smax > part_cap) smax = part_cap;
   if (smax < 1) smax = 1;
-  // cost ~ CTAs per SM (at least 12 resident-CTA equivalents, to keep the MUFU
-  // pipe fed: measured on B200 at 100k points, a floor of 4 left 10% and 8
-  // left 2.5% on the table) x columns per CTA
-  const int64_t k_sat = 12;
+  // Cost of S splits, fit to B200 timings of the D = 3 kernel from 10^4 to
+  // 10^6 points: the U x S CTAs run in W = U S / (SMs x 8 resident) waves; a
+  // partial last wave costs at least half a wave (with fewer than about four
+  // CTAs on an SM its MUFU pipe idles); every CTA pays about 16 columns of
+  // fixed work; a tenth of one CTA's columns goes to the ragged end.
   int best = 1;
   double best_cost = 1e300;
+  const double wave = static_cast<double>(sm_count) * 8.0;
   for (int64_t S = 1; S <= smax; ++S) {
-    int64_t per_sm = (U * S + sm_count - 1) / sm_count;
-    if (per_sm < k_sat) per_sm = k_sat;
-    const double cost = static_cast<double>(per_sm) * static_cast<double>((N + S - 1) / S + 64);
+    const double W = static_cast<double>(U * S) / wave;
+    const double full = std::floor(W), frac = W - full;
+    const double phases = (full == 0.0) ? std::fmax(W, 0.5)
+                                        : full + (frac > 1e-9 ? std::fmax(frac, 0.5) : 0.0);
+    const double cols = static_cast<double>((N + S - 1) / S);
+    const double cost = phases * (cols + 16.0) + 0.1 * cols;
     if (cost < best_cost * 0.999) {
       best_cost = cost;
       best = static_cast<int>(S);
     }
   }
-  p.splits = best;
   p.cols_per_split = (N + best - 1) / best;
   // keep every split non-empty
   if (p.cols_per_split < 1) p.cols_per_split = 1;
