@@ -61,6 +61,7 @@ struct TcKParams {
   int64_t cols_per_split;
   float two_c;
   float out_scale;
+  int s_ksteps;         // K steps of 16 holding the D + 2 nonzero packed columns
 };
 
 template <int KP, int CP>
@@ -232,10 +233,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idS = idesc_f16(DTFMT, kBM, kBN);
       const uint32_t idO = idesc_f16(0, kBM, CP);
+      const int s_ksteps = p.s_ksteps;
       auto issue_S = [&](int h, int st) {
         const uint8_t* sy = sStage + st * Cfg::STAGE;
 #pragma unroll
         for (int ks = 0; ks < KP / 16; ++ks) {
+          if (ks >= s_ksteps) break;   // the packed columns past D + 2 are zero
           const int kc = ks >> 2, kw = ks & 3;
           const uint64_t ad = desc_k_sw128(smem_u32(sX + (h * Cfg::KC + kc) * Cfg::ATOM) + kw * 32);
           const uint64_t bd = desc_k_sw128(smem_u32(sy + kc * Cfg::ATOM) + kw * 32);
@@ -339,41 +342,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      // double-buffered TMEM loads: chunk ch + 1 is in flight while chunk ch
-      // is exponentiated and its fp16 P written back
-      uint32_t va[32], vb[32];
+      // TMEM loads run up to three chunks of 32 columns deep: chunks 0 and 1
+      // first, chunk 2 while chunk 0 is exponentiated, chunk 3 while chunk 1
+      // is.  After chunk 1 the whole S tile is in registers and its columns
+      // are released, so the next S MMA has the second half of this tile's
+      // exponentials to complete in.
+      static_assert(kBN == 128, "four 32-column chunks per tile");
+      uint32_t va[32], vb[32], vc[32];
+      uint32_t pk[16];
       tmem_ld32(tS, va);
+      tmem_ld32(tS + 32, vb);
       tmem_wait_ld();
       reg_fence32(va);
-#pragma unroll
-      for (int ch = 0; ch < kBN / 32; ++ch) {
-        uint32_t(&cur)[32] = (ch & 1) ? vb : va;
-        uint32_t(&nxt)[32] = (ch & 1) ? va : vb;
-        if (ch + 1 < kBN / 32) tmem_ld32(tS + (ch + 1) * 32, nxt);
-        uint32_t pk[16];
-        exp_chunk(cur, two_c2, r2, pk);
-        if (Cfg::P_SEPARATE && ch == 0 && t > 0) {
-          // a warp that runs ahead must not overwrite its rows of P(t-1) before
-          // the P MMA of tile t-1 has read them (waited for as late as possible)
-          ok = __all_sync(0xffffffffu, wait_bar(bar_q(h), (t - 1) & 1, abort_flag));
-          if (!ok) {
-            tmem_wait_ld();   // the next chunk's load may still be in flight
-            break;
-          }
-          tc_fence_after();
+      reg_fence32(vb);
+      tmem_ld32(tS + 64, vc);
+      exp_chunk(va, two_c2, r2, pk);
+      if (Cfg::P_SEPARATE && t > 0) {
+        // a warp that runs ahead must not overwrite its rows of P(t-1) before
+        // the P MMA of tile t-1 has read them (waited for as late as possible)
+        ok = __all_sync(0xffffffffu, wait_bar(bar_q(h), (t - 1) & 1, abort_flag));
+        if (!ok) {
+          tmem_wait_ld();   // chunk 2's load may still be in flight
+          break;
         }
-        tmem_st16(tP + ch * 16, pk);
-        if (ch + 1 < kBN / 32) {
-          tmem_wait_ld();
-          reg_fence32(nxt);
-          if (ch + 2 == kBN / 32) {
-            // the whole S tile is in registers: its TMEM columns may be reused
-            tc_fence_before();
-            mbar_arrive(bar_f(h));
-          }
-        }
+        tc_fence_after();
       }
-      if (!ok) break;
+      tmem_st16(tP, pk);
+      tmem_ld32(tS + 96, va);
+      exp_chunk(vb, two_c2, r2, pk);
+      tmem_st16(tP + 16, pk);
+      tmem_wait_ld();
+      reg_fence32(vc);
+      reg_fence32(va);
+      tc_fence_before();
+      mbar_arrive(bar_f(h));
+      exp_chunk(vc, two_c2, r2, pk);
+      tmem_st16(tP + 32, pk);
+      exp_chunk(va, two_c2, r2, pk);
+      tmem_st16(tP + 48, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p(h));
@@ -698,6 +704,7 @@ cudaError_t launch_tc_sum(const TcArgs& a, cudaStream_t s) {
     kp.cols_per_split = a.plan.cols_per_split;
     kp.two_c = a.tau * kLog2e;
     kp.out_scale = exp2f(-kPShift);
+    kp.s_ksteps = static_cast<int>((a.D + 2 + 15) / 16);
     if (KP == 64)
       e = bf ? launch_cp<64, 1>(CP, tx, ty, tv, kp, grid, s) : launch_cp<64, 0>(CP, tx, ty, tv, kp, grid, s);
     else if (KP == 128)
