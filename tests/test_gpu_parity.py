@@ -105,6 +105,8 @@ HALF_SHAPES = [
     (1, 1, 1, 32, 1), (1, 1, 300, 32, 1), (2, 300, 1000, 32, 32), (1, 257, 129, 16, 33),
     (1, 200, 700, 5, 1), (1, 100, 300, 100, 16), (2, 130, 260, 48, 130), (1, 511, 640, 62, 64),
     (1, 70, 1200, 63, 3), (1, 129, 257, 126, 96), (1, 300, 700, 127, 1), (2, 257, 390, 128, 50),
+    # D + 2 at and just past a multiple of 16 (the similarity MMA's K steps)
+    (1, 300, 500, 14, 2), (1, 260, 530, 30, 4), (1, 200, 400, 31, 1), (1, 150, 300, 46, 1),
 ]
 # fp32 with D > 8: the split-tf32 tensor-core path (every packed-row width, one
 # and two value passes, single and several column tiles per warpgroup)
