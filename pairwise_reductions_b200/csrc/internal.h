@@ -222,7 +222,7 @@ struct F32Args {
   float* xpack;        // [B, M, 2 Kp] (or [B, M, Kp] unsplit)
   float* rnorm;        // [B, M]
   float* ypack;        // [B, N, 2 Kp]
-  float* qw;           // [B, Nq, 4], Nq = N rounded up to 128: -c |y'|^2 (-inf past N)
+  float* qw;           // [B, 4, Nq] lane by lane, Nq = N rounded up to 128: lane 0 -c |y'|^2 (-inf past N)
                        // and up to 3 value channels
   float* vt;           // [2 B, CP, Nst] (hi, lo), Nst = N rounded up to 4
 };

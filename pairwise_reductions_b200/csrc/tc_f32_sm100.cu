@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int a = 0; a < p.atoms; ++a)
           tma_load_3d(smem_u32(sy + a * BN * 128), &tmY, bar_full(st), a * 32, j0,
                       static_cast<int>(b));
-        tma_load_3d(smem_u32(sq), &tmQ, bar_full(st), 0, j0, static_cast<int>(b));
+        tma_load_3d(smem_u32(sq), &tmQ, bar_full(st), j0, 0, static_cast<int>(b));
         if constexpr (!REG) {
           for (int hl = 0; hl < 2; ++hl)
             for (int a = 0; a < BN / 32; ++a)
@@ -402,6 +402,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tPh = tmem + lane_base + Cfg::col_phi(h);
     const uint32_t tPl = tmem + lane_base + Cfg::col_plo(h);
     const float two_c = p.two_c;
+    const uint64_t two_c2 = pk2(two_c, two_c);
+    const uint64_t r2 = pk2(r, r);
     float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f;   // register values: running row sums (l for LSE)
     float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY;   // LSE: running maxima
     if constexpr (Cfg::XT) {
@@ -439,7 +441,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const uint32_t tS = tmem + lane_base + Cfg::col_s(h);
-      const float4* qw = reinterpret_cast<const float4*>(sStage + st * Cfg::STAGE + Cfg::Y_BYTES);
+      // the column records, lane by lane: q_j at qrec[j], value c at qrec[(1 + c) BN + j]
+      const float* qrec = reinterpret_cast<const float*>(sStage + st * Cfg::STAGE + Cfg::Y_BYTES);
       if constexpr (REG) {
         // S = Sbig + Ssmall, 32 columns at a time: the loads of chunk ch + 1
         // are in flight while chunk ch is exponentiated; once the last chunk
@@ -458,55 +461,78 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         reg_fence32(cb);
         reg_fence32(cs);
-        float p0 = 0.f, p1 = 0.f, p2 = 0.f;
+        // P.v partial sums of this tile, even and odd columns packed
+        uint64_t s0 = 0ull, s1 = 0ull, s2 = 0ull;
 #pragma unroll
         for (int ch = 0; ch < NCH; ++ch) {
-          float cur[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            cur[e] = fmaf(__uint_as_float(cb[e]) + __uint_as_float(cs[e]), two_c, r);
-          if (ch + 1 < NCH) {
-            tmem_ld32(tS + (ch + 1) * 32, cb);
-            if constexpr (SPLIT) tmem_ld32(tSs + (ch + 1) * 32, cs);
-          } else {
-            tc_fence_before();
-            mbar_arrive(bar_f(h));
-          }
           if constexpr (!LSE) {
+            // t = (Sbig + Ssmall) 2c + r + q_j, two columns per packed operation
+            uint64_t cur2[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int j = ch * 32 + e;
-              if constexpr (MODE == 1) {
-                // (norm, value): the first half of the column's 16 bytes
-                const float2 q = reinterpret_cast<const float2*>(qw)[2 * j];
-                p0 = fmaf(ex2(cur[e] + q.x), q.y, p0);
-              } else {
-                const float4 q = qw[j];
-                const float pe = ex2(cur[e] + q.x);
-                p0 = fmaf(pe, q.y, p0);
-                p1 = fmaf(pe, q.z, p1);
-                p2 = fmaf(pe, q.w, p2);
+            for (int e = 0; e < 16; ++e) {
+              uint64_t sv2 = pk2(__uint_as_float(cb[2 * e]), __uint_as_float(cb[2 * e + 1]));
+              if constexpr (SPLIT)
+                sv2 = add2(sv2, pk2(__uint_as_float(cs[2 * e]), __uint_as_float(cs[2 * e + 1])));
+              cur2[e] = fma2(sv2, two_c2, r2);
+            }
+            if (ch + 1 < NCH) {
+              tmem_ld32(tS + (ch + 1) * 32, cb);
+              if constexpr (SPLIT) tmem_ld32(tSs + (ch + 1) * 32, cs);
+            } else {
+              tc_fence_before();
+              mbar_arrive(bar_f(h));
+            }
+#pragma unroll
+            for (int e4 = 0; e4 < 8; ++e4) {
+              const int j = ch * 32 + 4 * e4;
+              const float4 qv = *reinterpret_cast<const float4*>(qrec + j);
+              const float4 w0 = *reinterpret_cast<const float4*>(qrec + BN + j);
+              float4 w1, w2;
+              if constexpr (MODE == 3) {
+                w1 = *reinterpret_cast<const float4*>(qrec + 2 * BN + j);
+                w2 = *reinterpret_cast<const float4*>(qrec + 3 * BN + j);
+              }
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                float t0, t1;
+                upk2(add2(cur2[2 * e4 + hh], hh ? pk2(qv.z, qv.w) : pk2(qv.x, qv.y)), t0, t1);
+                const uint64_t pe = pk2(ex2(t0), ex2(t1));
+                s0 = fma2(pe, hh ? pk2(w0.z, w0.w) : pk2(w0.x, w0.y), s0);
+                if constexpr (MODE == 3) {
+                  s1 = fma2(pe, hh ? pk2(w1.z, w1.w) : pk2(w1.x, w1.y), s1);
+                  s2 = fma2(pe, hh ? pk2(w2.z, w2.w) : pk2(w2.x, w2.y), s2);
+                }
               }
             }
           } else {
-            // lanes 1.. of qw hold log2 w: u = t + log2 w per channel
+            float cur[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              cur[e] = fmaf(__uint_as_float(cb[e]) + __uint_as_float(cs[e]), two_c, r);
+            if (ch + 1 < NCH) {
+              tmem_ld32(tS + (ch + 1) * 32, cb);
+              if constexpr (SPLIT) tmem_ld32(tSs + (ch + 1) * 32, cs);
+            } else {
+              tc_fence_before();
+              mbar_arrive(bar_f(h));
+            }
+            // lanes 1.. of the records hold log2 w: u = t + log2 w per channel
             auto lse_channel = [&](int lanec, float& m, float& l) {
+              const float* lw = qrec + lanec * BN + ch * 32;
               float cm = -INFINITY;
 #pragma unroll
-              for (int e = 0; e < 32; ++e)
-                cm = fmaxf(cm, cur[e] + reinterpret_cast<const float*>(qw + ch * 32 + e)[lanec]);
+              for (int e = 0; e < 32; ++e) cm = fmaxf(cm, cur[e] + lw[e]);
               const float mn = fmaxf(m, cm);
               if (mn != -INFINITY) {
                 float cs = 0.f;
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                  cs += ex2(cur[e] + reinterpret_cast<const float*>(qw + ch * 32 + e)[lanec] - mn);
+                for (int e = 0; e < 32; ++e) cs += ex2(cur[e] + lw[e] - mn);
                 l = fmaf(l, ex2(m - mn), cs);   // m = -inf: l = 0 and ex2(-inf) = 0
                 m = mn;
               }
             };
 #pragma unroll
-            for (int e = 0; e < 32; ++e) cur[e] += qw[ch * 32 + e].x;
+            for (int e = 0; e < 32; ++e) cur[e] += qrec[ch * 32 + e];
             lse_channel(1, mx0, acc0);
             if constexpr (MODE > 1) {
               lse_channel(2, mx1, acc1);
@@ -520,9 +546,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if constexpr (!LSE) {   // (log-sum-exp: the running (m, l) are mx*, acc*)
-          acc0 += p0;
-          acc1 += p1;
-          acc2 += p2;
+          float lo, hi;
+          upk2(s0, lo, hi);
+          acc0 += lo + hi;
+          if constexpr (MODE == 3) {
+            upk2(s1, lo, hi);
+            acc1 += lo + hi;
+            upk2(s2, lo, hi);
+            acc2 += lo + hi;
+          }
         }
         mbar_arrive(bar_empty(st));
       } else {
@@ -543,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const int c = half * 16 + e;
-              const float pe = ex2(fmaf(__uint_as_float(sv[ch][c]), two_c, r) + qw[ch * 32 + c].x);
+              const float pe = ex2(fmaf(__uint_as_float(sv[ch][c]), two_c, r) + qrec[ch * 32 + c]);
               const float ph = tf32_trunc(pe);
               hi[e] = __float_as_uint(ph);
               lo[e] = __float_as_uint(pe - ph);
@@ -664,26 +696,28 @@ __global__ void column_mean_kernel(const float* __restrict__ y, float* __restric
 
 // Packed operand rows [hi (K') | lo (K')] of the centred points v' = v - z,
 // z = zc[b, :], and the norm term -c |v'|^2: for the row side into
-// norm[b * R + r]; for the column side into norm[(b * Rpad + r) * 4] (lanes
-// 1-3 zeroed) with -inf for the padding columns r >= R.  Exact tf32 inputs
+// norm[b * R + r]; for the column side (records) into lane 0 of the column's
+// record, norm[4 b Rpad + r] (lanes 1-3, Rpad floats apart, zeroed), with -inf
+// for the padding columns r >= R.  Exact tf32 inputs
 // (fp16 / bf16, zc == nullptr, split == 0): v itself, rows [hi (K')] only.
 // One warp per row, lanes along the features (coalesced reads and writes).
 template <typename T>
 __global__ void pack_rows_f32_kernel(const T* __restrict__ src, const float* __restrict__ zc,
                                      float* __restrict__ dst, float* __restrict__ norm, int64_t B,
                                      int64_t R, int64_t Rpad, int D, int Kp, float c,
-                                     int norm_stride, int split) {
+                                     int records, int split) {
   const int lane = threadIdx.x & 31;
   const int64_t total = B * Rpad;
   const int64_t wstride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
        e < total; e += wstride) {
     const int64_t b = e / Rpad, rr = e % Rpad;
-    float* nrm = norm + e * norm_stride;
+    // records: lane l of column rr at norm[(4 b + l) Rpad + rr]; rows: norm[e]
+    float* nrm = records ? norm + 4 * b * Rpad + rr : norm + e;
     if (rr >= R) {
       if (lane == 0) {
         nrm[0] = -INFINITY;   // padding columns: kernel value 0
-        if (norm_stride == 4) nrm[1] = nrm[2] = nrm[3] = 0.f;
+        if (records) nrm[Rpad] = nrm[2 * Rpad] = nrm[3 * Rpad] = 0.f;
       }
       continue;
     }
@@ -702,13 +736,13 @@ __global__ void pack_rows_f32_kernel(const T* __restrict__ src, const float* __r
     for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
     if (lane == 0) {
       nrm[0] = -c * sq;
-      if (norm_stride == 4) nrm[1] = nrm[2] = nrm[3] = 0.f;
+      if (records) nrm[Rpad] = nrm[2 * Rpad] = nrm[3 * Rpad] = 0.f;
     }
   }
 }
 
 // Register-path values: channels [c0, c0 + cw) (cw <= 3) of the pass's values
-// (values.cuh) into lanes 1.. of qw[b, j, :]; for the log-sum-exp, their
+// (values.cuh) into lanes 1.. of the records (qw[(4 b + l) Nq + j]); for the log-sum-exp, their
 // base-2 logarithms.
 template <typename TW, typename TY>
 __global__ void pack_values_qw_kernel(const TW* __restrict__ w, const TY* __restrict__ y,
@@ -721,7 +755,7 @@ __global__ void pack_values_qw_kernel(const TW* __restrict__ w, const TY* __rest
     const int64_t b = e / N, j = e % N;
     for (int ch = 0; ch < cw; ++ch) {
       const float v = value_at(w, y, rows, b, e, Mrows, D, C, c0 + ch, src_ld);
-      qw[(b * Nq + j) * 4 + 1 + ch] = log2_values ? lg2(v) : v;
+      qw[(4 * b + 1 + ch) * Nq + j] = log2_values ? lg2(v) : v;
     }
   }
 }
@@ -750,14 +784,14 @@ __global__ void pack_values_f32_split_kernel(const float* __restrict__ w,
 }
 
 // Exponent shift of a pass (log2 units): rows -- norm[b * R + r] -- or columns
-// -- norm[(b * Rpad + r) * 4], r < R -- gain scale * src[(b * R + r) * ld + c].
-__global__ void add_shift_kernel(float* __restrict__ norm, int stride, const float* __restrict__ src,
-                                 int64_t ld, int c, float scale, int64_t B, int64_t R, int64_t Rpad) {
+// -- the records' lane 0, norm[4 b Nq + r], r < R -- gain scale * src[(b * R + r) * ld + c].
+__global__ void add_shift_kernel(float* __restrict__ norm, int64_t bstride, const float* __restrict__ src,
+                                 int64_t ld, int c, float scale, int64_t B, int64_t R) {
   const int64_t total = B * R;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t b = e / R, r = e % R;
-    norm[(b * Rpad + r) * stride] += scale * src[e * ld + c];
+    norm[b * bstride + r] += scale * src[e * ld + c];
   }
 }
 
@@ -882,9 +916,9 @@ void pack_operands_f32(const F32Args& a, int64_t Nq, float c, cudaStream_t s) {
   }
   // one warp per row, 8 rows per 256-thread block
   pack_rows_f32_kernel<T><<<grid_for(a.B * a.M, 8), 256, 0, s>>>(x, zc, a.xpack, a.rnorm, a.B, a.M,
-                                                                a.M, a.D, a.plan.Kp, c, 1, split);
+                                                                a.M, a.D, a.plan.Kp, c, 0, split);
   pack_rows_f32_kernel<T><<<grid_for(a.B * Nq, 8), 256, 0, s>>>(y, zc, a.ypack, a.qw, a.B, a.N, Nq,
-                                                               a.D, a.plan.Kp, c, 4, split);
+                                                               a.D, a.plan.Kp, c, 1, split);
 }
 
 template <typename T>
@@ -912,11 +946,11 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
   else
     pack_operands_f32<__nv_bfloat16>(a, Nq, c, s);
   if (a.shift_mode == 1)
-    add_shift_kernel<<<grid_for(a.B * a.M, 256), 256, 0, s>>>(a.rnorm, 1, a.shift_src, a.shift_ld,
-                                                             a.shift_c, a.shift_scale, a.B, a.M, a.M);
+    add_shift_kernel<<<grid_for(a.B * a.M, 256), 256, 0, s>>>(a.rnorm, a.M, a.shift_src, a.shift_ld,
+                                                             a.shift_c, a.shift_scale, a.B, a.M);
   else if (a.shift_mode == 2)
-    add_shift_kernel<<<grid_for(a.B * a.N, 256), 256, 0, s>>>(a.qw, 4, a.shift_src, a.shift_ld,
-                                                             a.shift_c, a.shift_scale, a.B, a.N, Nq);
+    add_shift_kernel<<<grid_for(a.B * a.N, 256), 256, 0, s>>>(a.qw, 4 * Nq, a.shift_src, a.shift_ld,
+                                                             a.shift_c, a.shift_scale, a.B, a.N);
   else if (a.shift_mode != 0)
     return cudaErrorInvalidValue;
   cudaError_t e = cudaGetLastError();
@@ -950,8 +984,8 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
     if (BN != 32 && BN != 64 && BN != 128) return cudaErrorInvalidValue;
     if (!make_tmap_3d(&m.y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.ypack, rowf, a.N, a.B, rowf * 4,
                       a.N * rowf * 4, 32, BN) ||
-        !make_tmap_3d(&m.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.qw, 4, Nq, a.B, 16, Nq * 16ull, 4,
-                      BN, false))
+        !make_tmap_3d(&m.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.qw, Nq, 4, a.B, Nq * 4ull,
+                      Nq * 16ull, BN, 4, false))
       return cudaErrorInvalidValue;
     if (reg) {
       m.v = m.q;   // unused
