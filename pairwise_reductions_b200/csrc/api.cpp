@@ -135,8 +135,8 @@ PassLayout pass_layout(const Pass& p, int sm) {
         f32_chunk_pad(p.CV < L.f32.max_chunk ? p.CV : L.f32.max_chunk));
     const size_t Nst = (p.N + 3) / 4 * 4;
     const size_t Nq = (p.N + 127) / 128 * 128;
-    L.off_zc = off;
-    off = align_up(off + size_t(p.B) * p.D * 4);
+    L.off_zc = off;   // column centres [B, D], then one max word per batch
+    off = align_up(off + size_t(p.B) * (p.D + 1) * 4);
     L.off_xpack = off;
     off = align_up(off + size_t(p.B) * p.R * rowb);
     L.off_rnorm = off;
@@ -407,8 +407,8 @@ LseF32Layout lse_f32_layout(int64_t B, int64_t M, int64_t N, int64_t D, int64_t 
   const size_t rowb = size_t(L.plan.split ? 2 : 1) * L.plan.Kp * 4;
   const size_t Nq = (N + 127) / 128 * 128;
   size_t off = 0;
-  L.off_zc = off;
-  off = align_up(off + size_t(B) * D * 4);
+  L.off_zc = off;   // column centres [B, D], then one max word per batch
+  off = align_up(off + size_t(B) * (D + 1) * 4);
   L.off_xpack = off;
   off = align_up(off + size_t(B) * M * rowb);
   L.off_rnorm = off;

@@ -1,14 +1,16 @@
 // tc_f32_sm100.cu -- tensor-core Gaussian kernel sum for fp32 inputs with
-// 9 <= D <= 128 on sm_100a, at fp32 accuracy: split-tf32 products on tcgen05.
+// 9 <= D <= 128 on sm_100a, at fp32 accuracy: split products on tcgen05.
 //
-// Each fp32 operand v is split into v = hi + lo with hi = v rounded to tf32
-// (the 19 bits the kind::tf32 MMA reads) and lo = v - hi, itself rounded to
-// tf32.  A product a b is then taken as a_lo b_hi + a_hi b_lo + a_hi b_hi: the
-// dropped a_lo b_lo is ~2^-22 of a b, so three tf32 MMAs give close to fp32
+// Each fp32 operand v is split into v = hi + lo, two values of 11 significant
+// bits each, and a product a b is taken as a_lo b_hi + a_hi b_lo + a_hi b_hi:
+// the dropped a_lo b_lo is ~2^-22 of a b, so three MMAs give close to fp32
 // products with fp32 accumulation.  This is the "memory-efficient" fp32 runs'
 // arithmetic of "Fast Gauss Sums via Flash Attention" (Figures 4 and 5), done
-// with B200's tensor cores: both products of the method -- the similarity
-// tile x.y^T and the value product P.v -- are split this way.
+// with B200's tensor cores.  The similarity tile x.y^T splits into fp16 parts
+// (kind::f16, 16 per K step: half the MMAs of tf32 parts, which carry the same
+// 11 bits), the coordinates scaled by a power of two per batch so that fp16's
+// range holds them (split_exp); the value product P.v splits P and v into tf32
+// hi/lo parts (kind::tf32).
 //
 // The exponent.  With c = tau/2 * log2 e and the points centred at z, the mean
 // of a strided sample of the batch's column points (x' = x - z, y' = y - z:
@@ -22,16 +24,17 @@
 //
 // CTA = one 128-row tile, 10 warps:
 //   warp 0      TMA producer: the x' rows once (unless they sit in TMEM), then a
-//               ring of stages: y' tile, a 16-byte record per column {q_j, values
-//               or log2 values}, and for tensor-core values the split v^T tile
+//               ring of stages: y' tile, the column records lane by lane (q_j,
+//               then values or log2 values), and for tensor-core values the
+//               split v^T tile
 //   warp 1      TMEM owner + single-thread MMA issuer
 //   warps 2-5   exp warpgroup 0: column tiles 0, 2, 4, ...
 //   warps 6-9   exp warpgroup 1: column tiles 1, 3, 5, ...
 // Both warpgroups hold the same rows (TMEM lanes), so each keeps its own
 // partial result and warpgroup 0 combines the two at the end.  Per column tile
 // t of warpgroup h:
-//   S_h  = x'.y'(t)^T                 3 tf32 MMAs per K step (A from shared
-//                                     memory, or from TMEM when it has room)
+//   S_h  = x'.y'(t)^T                 3 fp16 MMAs per K step of 16 (A from
+//                                     shared memory, or from TMEM when it has room)
 //   P_h  = ex2(fma(S_h, 2c, r) + q)   tcgen05.ld -> MUFU
 // then either (register values, <= 3 channels, and the log-sum-exp)
 //   row sums += P_h . v in registers, exact fp32 FMAs (or a running maximum and
@@ -39,8 +42,8 @@
 // or (tensor-core values, 4 .. 64 channels per pass)
 //   P_h -> tf32 hi/lo -> tcgen05.st;  O_h += P_h . v(t), 3 tf32 MMAs per K step
 //   (A = P from TMEM).
-// fp16 / bf16 inputs (log-sum-exp) are exact in tf32: unsplit rows, one MMA
-// per K step (template SPLIT = false).
+// fp16 / bf16 inputs (log-sum-exp) are exact in tf32: unsplit tf32 rows, one
+// MMA per K step of 8 (template SPLIT = false).
 // Every mbarrier wait is bounded (2 s); on expiry the kernel raises its device
 // error word, lets the other warps leave, frees TMEM and returns.
 #include <cuda.h>
@@ -74,12 +77,13 @@ struct F32KParams {
   int64_t ldo;
   int c0, cw;
   int64_t cols_per_split;
-  int ksteps;           // K' / 8: tf32 K steps of the hi (and of the lo) half
+  int ksteps;           // 32-byte K steps of the hi (and of the lo) half: K'/16 fp16, K'/8 tf32
   int atoms;            // 128-byte atoms of a packed row actually loaded (<= KA)
   int Bsz;              // batch count (the lo half of v sits at batch index B + b)
   int bn;               // tile width the TMA boxes were made for
-  int split;            // 1: rows [hi | lo]; 0: rows are exact tf32 (fp16 / bf16 inputs), hi only
+  int split;            // 1: fp16 rows [hi | lo]; 0: rows are exact tf32 (fp16 / bf16 inputs), hi only
   float two_c;
+  const int* amax;      // split rows: per batch, the bits of max |v'| (sets the power-of-two scale)
 };
 
 // KA: 128-byte atoms per packed row [hi K' | lo K'] the operands may hold.
@@ -169,6 +173,20 @@ __device__ __forceinline__ float tf32_round(float v) {
   return __uint_as_float((__float_as_uint(v) + 0x1000u) & 0xFFFFE000u);
 }
 
+// Split rows hold v' 2^e in fp16 hi + lo parts, e per batch from the bits of
+// max |v'| over its x' and y' rows: the largest scaled value lies in
+// [2^14, 2^15), clear of fp16's overflow, and the lo parts keep their 11 bits
+// down to values 2^-14 (below that their absolute error stays under 2^-25,
+// i.e. 2^-39 of the largest).  e is clamped to [-40, 60]; S from scaled rows
+// is 2^(2e) S, undone in the exponent's constant.
+__device__ __forceinline__ int split_exp(int amax_bits) {
+  if (amax_bits <= 0) return 0;   // all points at the centre
+  const int e = 14 - (((amax_bits >> 23) & 0xff) - 127);
+  return e < -40 ? -40 : (e > 60 ? 60 : e);
+}
+// 2^k for an integer -126 <= k <= 127, exactly.
+__device__ __forceinline__ float pow2_int(int k) { return __int_as_float((k + 127) << 23); }
+
 // Named barrier of the two exp warpgroups (warps 2-9).
 __device__ __forceinline__ void exp_warps_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
@@ -186,6 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using Cfg = F32Cfg<KA, MODE>;
   constexpr bool REG = Cfg::REG;
   static_assert(REG || !LSE, "log-sum-exp runs on the register path");
+  constexpr int kAtomElems = SPLIT ? 64 : 32;   // packed-row elements per 128-byte atom
   constexpr int CP = Cfg::CP;
   constexpr int NST = Cfg::NST;
   constexpr int BN = Cfg::BN;
@@ -259,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmX);
         mbar_arrive_expect_tx(bar_x, p.atoms * kAtom);
         for (int a = 0; a < p.atoms; ++a)
-          tma_load_3d(smem_u32(sX + a * kAtom), &tmX, bar_x, a * 32, static_cast<int>(row0),
+          tma_load_3d(smem_u32(sX + a * kAtom), &tmX, bar_x, a * kAtomElems, static_cast<int>(row0),
                       static_cast<int>(b));
       }
       const uint32_t stage_tx = p.atoms * BN * 128 + BN * 16 + Cfg::V_BYTES;
@@ -272,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int j0 = static_cast<int>(jbeg + static_cast<int64_t>(t) * BN);
         mbar_arrive_expect_tx(bar_full(st), stage_tx);
         for (int a = 0; a < p.atoms; ++a)
-          tma_load_3d(smem_u32(sy + a * BN * 128), &tmY, bar_full(st), a * 32, j0,
+          tma_load_3d(smem_u32(sy + a * BN * 128), &tmY, bar_full(st), a * kAtomElems, j0,
                       static_cast<int>(b));
         tma_load_3d(smem_u32(sq), &tmQ, bar_full(st), j0, 0, static_cast<int>(b));
         if constexpr (!REG) {
@@ -287,7 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idS = idesc_f16(2, kBM, BN);
+      // split rows: fp16 hi / lo parts (kind::f16, 16 per K step); unsplit: tf32
+      const uint32_t idS = idesc_f16(SPLIT ? 0 : 2, kBM, BN);
       const uint32_t idO = idesc_f16(2, kBM, CP);
       const int ks_lo = p.ksteps;
       // K step ks (8 floats = 32 bytes) of a packed row block whose atoms are
@@ -308,9 +328,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ds = REG ? tmem + Cfg::col_ss(h) : db;
         auto mma = [&](uint32_t d, int ka, uint64_t bdesc, uint32_t acc) {
           if constexpr (Cfg::XT) {
-            mma_ts_tf32(d, tmem + Cfg::COL_X + ka * 8, bdesc, idS, acc);
+            if constexpr (SPLIT)
+              mma_ts(d, tmem + Cfg::COL_X + ka * 8, bdesc, idS, acc);
+            else
+              mma_ts_tf32(d, tmem + Cfg::COL_X + ka * 8, bdesc, idS, acc);
           } else {
-            mma_ss_tf32(d, kdesc(sX, kAtom, ka), bdesc, idS, acc);
+            if constexpr (SPLIT)
+              mma_ss(d, kdesc(sX, kAtom, ka), bdesc, idS, acc);
+            else
+              mma_ss_tf32(d, kdesc(sX, kAtom, ka), bdesc, idS, acc);
           }
         };
         // (exact tf32 operands, SPLIT false: the large products alone)
@@ -401,7 +427,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tPh = tmem + lane_base + Cfg::col_phi(h);
     const uint32_t tPl = tmem + lane_base + Cfg::col_plo(h);
-    const float two_c = p.two_c;
+    // the exponent's constant, with the split rows' scale 2^(2e) undone
+    const float two_c =
+        SPLIT ? p.two_c * pow2_int(-split_exp(p.amax[b])) * pow2_int(-split_exp(p.amax[b])) : p.two_c;
     const uint64_t two_c2 = pk2(two_c, two_c);
     const uint64_t r2 = pk2(r, r);
     float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f;   // register values: running row sums (l for LSE)
@@ -694,8 +722,35 @@ __global__ void column_mean_kernel(const float* __restrict__ y, float* __restric
   }
 }
 
-// Packed operand rows [hi (K') | lo (K')] of the centred points v' = v - z,
-// z = zc[b, :], and the norm term -c |v'|^2: for the row side into
+// Per batch, the bits of max |v_k - z_k| over the rows of x and y (non-negative
+// floats order like their bit patterns): the split rows' scale.  Grid
+// (B, blocks); amax zeroed before.
+__global__ void centred_maxabs_kernel(const float* __restrict__ x, const float* __restrict__ y,
+                                      const float* __restrict__ zc, int* __restrict__ amax,
+                                      int64_t M, int64_t N, int D) {
+  const int64_t b = blockIdx.x;
+  const int64_t nx = M * D, total = (M + N) * D;
+  float m = 0.f;
+  for (int64_t e = blockIdx.y * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.y) * blockDim.x) {
+    const int k = static_cast<int>(e % D);
+    const float v = e < nx ? x[b * nx + e] : y[b * N * D + (e - nx)];
+    m = fmaxf(m, fabsf(v - zc[b * D + k]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ float wm[32];
+  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) m = fmaxf(m, wm[w]);
+    atomicMax(amax + b, __float_as_int(m));
+  }
+}
+
+// Packed operand rows of the centred points v' = v - z, z = zc[b, :]: fp16
+// [hi (K') | lo (K')] of v' 2^e (split_exp), and the norm term -c |v'|^2 from
+// v' itself in fp32: for the row side into
 // norm[b * R + r]; for the column side (records) into lane 0 of the column's
 // record, norm[4 b Rpad + r] (lanes 1-3, Rpad floats apart, zeroed), with -inf
 // for the padding columns r >= R.  Exact tf32 inputs
@@ -705,7 +760,7 @@ template <typename T>
 __global__ void pack_rows_f32_kernel(const T* __restrict__ src, const float* __restrict__ zc,
                                      float* __restrict__ dst, float* __restrict__ norm, int64_t B,
                                      int64_t R, int64_t Rpad, int D, int Kp, float c,
-                                     int records, int split) {
+                                     int records, int split, const int* __restrict__ amax) {
   const int lane = threadIdx.x & 31;
   const int64_t total = B * Rpad;
   const int64_t wstride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -723,14 +778,27 @@ __global__ void pack_rows_f32_kernel(const T* __restrict__ src, const float* __r
     }
     const T* v = src + (b * R + rr) * D;
     const float* z = zc ? zc + b * D : nullptr;
-    float* out = dst + (b * R + rr) * ((split ? 2 : 1) * static_cast<int64_t>(Kp));
     float sq = 0.f;
-    for (int k = lane; k < Kp; k += 32) {
-      const float d = (k < D) ? vf(v[k]) - (z ? z[k] : 0.f) : 0.f;
-      sq = fmaf(d, d, sq);
-      const float hi = tf32_round(d);
-      out[k] = hi;
-      if (split) out[Kp + k] = tf32_round(d - hi);
+    if (split) {
+      // fp16 [hi (K') | lo (K')] of v' 2^e: v' 2^e is exact, hi its nearest
+      // fp16, lo the nearest fp16 of the (exact) remainder
+      const float sc = pow2_int(split_exp(amax[b]));
+      __half* out = reinterpret_cast<__half*>(dst) + (b * R + rr) * (2 * static_cast<int64_t>(Kp));
+      for (int k = lane; k < Kp; k += 32) {
+        const float d = (k < D) ? vf(v[k]) - z[k] : 0.f;
+        sq = fmaf(d, d, sq);
+        const float u = d * sc;
+        const __half hi = __float2half_rn(u);
+        out[k] = hi;
+        out[Kp + k] = __float2half_rn(u - __half2float(hi));
+      }
+    } else {
+      float* out = dst + (b * R + rr) * static_cast<int64_t>(Kp);
+      for (int k = lane; k < Kp; k += 32) {
+        const float d = (k < D) ? vf(v[k]) - (z ? z[k] : 0.f) : 0.f;
+        sq = fmaf(d, d, sq);
+        out[k] = tf32_round(d);
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
@@ -861,8 +929,10 @@ int tile_cols_ka(int mode) {
 F32Plan f32_plan(int64_t B, int64_t M, int64_t N, int64_t D, int sm_count, bool split) {
   F32Plan p{};
   p.split = split;
-  p.Kp = static_cast<int>((D + 7) / 8 * 8);
-  p.atoms = ((split ? 2 : 1) * p.Kp + 31) / 32;
+  // split: fp16 [hi | lo] rows, K' = D rounded up to 16 (kind::f16 K steps);
+  // unsplit: tf32 [hi] rows, K' = D rounded up to 8
+  p.Kp = static_cast<int>(split ? (D + 15) / 16 * 16 : (D + 7) / 8 * 8);
+  p.atoms = split ? (2 * p.Kp + 63) / 64 : (p.Kp + 31) / 32;
   p.max_chunk = ka_for(p.atoms) >= 8 ? 32 : 64;
   // a split is a whole number of 128-column blocks (every tile width divides
   // it, so no tile straddles two splits)
@@ -901,24 +971,37 @@ int f32_tile_cols(int KA, int mode) {
 }
 
 // Packed rows of x and y (and, for fp32, the column centre first).
+// The per-batch max words sit right after the column centres (the workspace
+// layouts reserve B (D + 1) floats there).
+int* f32_amax(const F32Args& a) { return reinterpret_cast<int*>(a.zc + a.B * a.D); }
+
 template <typename T>
 void pack_operands_f32(const F32Args& a, int64_t Nq, float c, cudaStream_t s) {
   const T* x = static_cast<const T*>(a.x);
   const T* y = static_cast<const T*>(a.y);
   const int split = a.plan.split ? 1 : 0;
   const float* zc = nullptr;
+  int* amax = nullptr;
   if constexpr (std::is_same<T, float>::value) {
     if (split) {
       column_mean_kernel<<<dim3(static_cast<unsigned>(a.B), static_cast<unsigned>((a.D + 31) / 32)),
                            256, 0, s>>>(y, a.zc, a.N, a.D);
       zc = a.zc;
+      amax = f32_amax(a);
+      cudaMemsetAsync(amax, 0, static_cast<size_t>(a.B) * sizeof(int), s);
+      int64_t blocks = ((a.M + a.N) * a.D + 255) / 256;
+      const int64_t cap = (148 * 8 + a.B - 1) / a.B;
+      if (blocks > cap) blocks = cap;
+      if (blocks > 65535) blocks = 65535;
+      centred_maxabs_kernel<<<dim3(static_cast<unsigned>(a.B), static_cast<unsigned>(blocks)), 256, 0,
+                              s>>>(x, y, a.zc, amax, a.M, a.N, a.D);
     }
   }
   // one warp per row, 8 rows per 256-thread block
   pack_rows_f32_kernel<T><<<grid_for(a.B * a.M, 8), 256, 0, s>>>(x, zc, a.xpack, a.rnorm, a.B, a.M,
-                                                                a.M, a.D, a.plan.Kp, c, 0, split);
+                                                                a.M, a.D, a.plan.Kp, c, 0, split, amax);
   pack_rows_f32_kernel<T><<<grid_for(a.B * Nq, 8), 256, 0, s>>>(y, zc, a.ypack, a.qw, a.B, a.N, Nq,
-                                                               a.D, a.plan.Kp, c, 1, split);
+                                                               a.D, a.plan.Kp, c, 1, split, amax);
 }
 
 template <typename T>
@@ -958,9 +1041,13 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
   const float* x = static_cast<const float*>(a.x);   // fp32 only below (tensor-core values)
   const float* y = static_cast<const float*>(a.y);
   TileMaps m;
-  const uint64_t rowf = (a.plan.split ? 2ull : 1ull) * Kp;
-  if (!make_tmap_3d(&m.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.xpack, rowf, a.M, a.B, rowf * 4,
-                    a.M * rowf * 4, 32, kBM))
+  // split rows: fp16 [hi | lo], 64 per 128-byte atom; unsplit: tf32 [hi], 32 per atom
+  const bool sp = a.plan.split;
+  const CUtensorMapDataType rdt = sp ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const uint64_t rowe = (sp ? 2ull : 1ull) * Kp;   // elements per packed row
+  const uint64_t rowb = rowe * (sp ? 2ull : 4ull);  // bytes per packed row
+  const int atom_e = sp ? 64 : 32;
+  if (!make_tmap_3d(&m.x, rdt, a.xpack, rowe, a.M, a.B, rowb, a.M * rowb, atom_e, kBM))
     return cudaErrorInvalidValue;
   const int KA = ka_for(a.plan.atoms);
   const int64_t Nst = (a.N + 3) / 4 * 4;
@@ -982,8 +1069,7 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
     }
     const int BN = f32_tile_cols(KA, mode);
     if (BN != 32 && BN != 64 && BN != 128) return cudaErrorInvalidValue;
-    if (!make_tmap_3d(&m.y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.ypack, rowf, a.N, a.B, rowf * 4,
-                      a.N * rowf * 4, 32, BN) ||
+    if (!make_tmap_3d(&m.y, rdt, a.ypack, rowe, a.N, a.B, rowb, a.N * rowb, atom_e, BN) ||
         !make_tmap_3d(&m.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.qw, Nq, 4, a.B, Nq * 4ull,
                       Nq * 16ull, BN, 4, false))
       return cudaErrorInvalidValue;
@@ -1013,12 +1099,13 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
     kp.c0 = c0;
     kp.cw = cw;
     kp.cols_per_split = a.plan.cols_per_split;
-    kp.ksteps = Kp / 8;
+    kp.ksteps = sp ? Kp / 16 : Kp / 8;
     kp.atoms = a.plan.atoms;
     kp.Bsz = static_cast<int>(a.B);
     kp.bn = BN;
     kp.split = a.plan.split ? 1 : 0;
     kp.two_c = a.tau * kLog2e;
+    kp.amax = sp ? f32_amax(a) : nullptr;
     switch (KA) {
       case 1: e = launch_mode<1>(mode, a.lse, m, kp, grid, s); break;
       case 2: e = launch_mode<2>(mode, a.lse, m, kp, grid, s); break;
