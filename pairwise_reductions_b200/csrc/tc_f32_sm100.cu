@@ -724,26 +724,31 @@ __global__ void column_mean_kernel(const float* __restrict__ y, float* __restric
 
 // Per batch, the bits of max |v_k - z_k| over the rows of x and y (non-negative
 // floats order like their bit patterns): the split rows' scale.  Grid
-// (B, blocks); amax zeroed before.
+// (B, blocks) of 256 threads, one warp per row, lanes along the features (the
+// centre in registers, D <= 128); amax zeroed before.
 __global__ void centred_maxabs_kernel(const float* __restrict__ x, const float* __restrict__ y,
                                       const float* __restrict__ zc, int* __restrict__ amax,
                                       int64_t M, int64_t N, int D) {
   const int64_t b = blockIdx.x;
-  const int64_t nx = M * D, total = (M + N) * D;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float z[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) z[u] = (lane + 32 * u < D) ? zc[b * D + lane + 32 * u] : 0.f;
   float m = 0.f;
-  for (int64_t e = blockIdx.y * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
-       e += static_cast<int64_t>(gridDim.y) * blockDim.x) {
-    const int k = static_cast<int>(e % D);
-    const float v = e < nx ? x[b * nx + e] : y[b * N * D + (e - nx)];
-    m = fmaxf(m, fabsf(v - zc[b * D + k]));
+  for (int64_t r = static_cast<int64_t>(blockIdx.y) * 8 + warp; r < M + N;
+       r += static_cast<int64_t>(gridDim.y) * 8) {
+    const float* v = r < M ? x + (b * M + r) * D : y + (b * N + (r - M)) * D;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (lane + 32 * u < D) m = fmaxf(m, fabsf(v[lane + 32 * u] - z[u]));
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  __shared__ float wm[32];
-  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+  __shared__ float wm[8];
+  if (lane == 0) wm[warp] = m;
   __syncthreads();
   if (threadIdx.x == 0) {
-    for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) m = fmaxf(m, wm[w]);
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, wm[w]);
     atomicMax(amax + b, __float_as_int(m));
   }
 }
@@ -989,8 +994,8 @@ void pack_operands_f32(const F32Args& a, int64_t Nq, float c, cudaStream_t s) {
       zc = a.zc;
       amax = f32_amax(a);
       cudaMemsetAsync(amax, 0, static_cast<size_t>(a.B) * sizeof(int), s);
-      int64_t blocks = ((a.M + a.N) * a.D + 255) / 256;
-      const int64_t cap = (148 * 8 + a.B - 1) / a.B;
+      int64_t blocks = (a.M + a.N + 7) / 8;   // 8 rows (warps) per block and pass
+      const int64_t cap = (148 * 16 + a.B - 1) / a.B;
       if (blocks > cap) blocks = cap;
       if (blocks > 65535) blocks = 65535;
       centred_maxabs_kernel<<<dim3(static_cast<unsigned>(a.B), static_cast<unsigned>(blocks)), 256, 0,

@@ -161,6 +161,34 @@ def test_f32_tensor_core_shifted_clouds_and_sharp_kernels(shift, tau):
     assert rel_l2(out, ref) <= TOL["f32"], rel_l2(out, ref)
 
 
+@pytest.mark.parametrize("scale", [1e-5, 1e-2, 1e3, 1e6])
+@pytest.mark.parametrize("D,C", [(32, 1), (32, 5), (100, 2)])
+def test_f32_tensor_core_coordinate_scales(scale, D, C):
+    """Coordinates s times larger with tau / s^2: the same kernel matrix.  The
+    similarity tile's fp16 parts are scaled by a power of two per batch, so
+    neither tiny nor huge coordinates leave fp16's range.  Batch 1's cloud is
+    1000 times smaller than batch 0's (one scale per batch)."""
+    inp = synth.make_inputs(4, seed=37, B=2, M=260, N=700, D=D, C=C, dtype="f32")
+    for k in ("x", "y"):
+        v = inp[k].double() * scale
+        v[1] *= 1e-3
+        inp[k] = v.float()
+    tau = 1.0 / scale ** 2
+    d = dev(inp)
+    x, y, w = (f64(inp, k) for k in "xyw")
+    out = gs().gauss_sum_fwd(d["x"], d["y"], d["w"], tau).cpu().numpy()
+    ref = oracle.gauss_sum(x, y, w, tau)
+    # batch 1 with its own tau (a 1000 times smaller cloud)
+    out1 = gs().gauss_sum_fwd(d["x"][1:], d["y"][1:], d["w"][1:], tau * 1e6).cpu().numpy()
+    ref1 = oracle.gauss_sum(x[1:], y[1:], w[1:], tau * 1e6)
+    assert rel_l2(out[0], ref[0]) <= TOL["f32"], rel_l2(out[0], ref[0])
+    assert rel_l2(out1, ref1) <= TOL["f32"], rel_l2(out1, ref1)
+    wpos = inp["w"][:1].abs() + 0.1   # positive weights, float32, for both sides
+    lse = gs().gauss_lse_fwd(d["x"][:1], d["y"][:1], wpos.cuda(), tau).cpu().numpy()
+    lref = oracle.gauss_lse(x[:1], y[:1], synth.as_f64(wpos), tau)
+    assert rel_l2(lse, lref) <= TOL["f32"], rel_l2(lse, lref)
+
+
 @pytest.mark.parametrize("shape", [(1, 700, 900, 3, 1), (2, 300, 1100, 2, 3), (1, 64, 5000, 8, 9)])
 def test_lse_f32_shapes(shape):
     B, M, N, D, C = shape
