@@ -135,8 +135,8 @@ PassLayout pass_layout(const Pass& p, int sm) {
         f32_chunk_pad(p.CV < L.f32.max_chunk ? p.CV : L.f32.max_chunk));
     const size_t Nst = (p.N + 3) / 4 * 4;
     const size_t Nq = (p.N + 127) / 128 * 128;
-    L.off_zc = off;   // column centres [B, D], then one max word per batch
-    off = align_up(off + size_t(p.B) * (p.D + 1) * 4);
+    L.off_zc = off;   // column centres [B, D], one max word per batch, 64 per value chunk
+    off = align_up(off + size_t(p.B) * (p.D + 1 + 64) * 4);
     L.off_xpack = off;
     off = align_up(off + size_t(p.B) * p.R * rowb);
     L.off_rnorm = off;

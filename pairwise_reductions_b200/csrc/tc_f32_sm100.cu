@@ -9,8 +9,8 @@
 // with B200's tensor cores.  The similarity tile x.y^T splits into fp16 parts
 // (kind::f16, 16 per K step: half the MMAs of tf32 parts, which carry the same
 // 11 bits), the coordinates scaled by a power of two per batch so that fp16's
-// range holds them (split_exp); the value product P.v splits P and v into tf32
-// hi/lo parts (kind::tf32).
+// range holds them (split_exp); the value product P.v on the tensor cores
+// splits P 2^14 and v 2^e (e per batch and channel) into fp16 parts as well.
 //
 // The exponent.  With c = tau/2 * log2 e and the points centred at z, the mean
 // of a strided sample of the batch's column points (x' = x - z, y' = y - z:
@@ -40,8 +40,8 @@
 //   row sums += P_h . v in registers, exact fp32 FMAs (or a running maximum and
 //   shifted sum for the log-sum-exp)
 // or (tensor-core values, 4 .. 64 channels per pass)
-//   P_h -> tf32 hi/lo -> tcgen05.st;  O_h += P_h . v(t), 3 tf32 MMAs per K step
-//   (A = P from TMEM).
+//   P_h 2^14 -> fp16 hi/lo -> tcgen05.st;  O_h += P_h . v(t), 3 fp16 MMAs per
+//   K step of 16 (A = P from TMEM); the scales are undone on output.
 // fp16 / bf16 inputs (log-sum-exp) are exact in tf32: unsplit tf32 rows, one
 // MMA per K step of 8 (template SPLIT = false).
 // Every mbarrier wait is bounded (2 s); on expiry the kernel raises its device
@@ -84,6 +84,7 @@ struct F32KParams {
   int split;            // 1: fp16 rows [hi | lo]; 0: rows are exact tf32 (fp16 / bf16 inputs), hi only
   float two_c;
   const int* amax;      // split rows: per batch, the bits of max |v'| (sets the power-of-two scale)
+  const int* vmax;      // tensor-core values: per (batch, channel of the chunk), the bits of max |v|
 };
 
 // KA: 128-byte atoms per packed row [hi K' | lo K'] the operands may hold.
@@ -96,15 +97,17 @@ struct F32Cfg {
   static constexpr int CP = REG ? 16 : MODE;
   static constexpr int CPA = (CP + 31) / 32 * 32;
   static constexpr int qw_bytes(int bn) { return bn * 16 <= 1024 ? 1024 : bn * 16; }
-  static constexpr int v_bytes(int bn) { return REG ? 0 : 2 * (bn / 32) * CP * 128; }
+  // v^T in fp16 [hi | lo] parts: 64 columns per 128-byte atom row
+  static constexpr int va(int bn) { return bn < 64 ? 1 : bn / 64; }
+  static constexpr int v_bytes(int bn) { return REG ? 0 : 2 * va(bn) * CP * 128; }
   static constexpr int stage_bytes(int bn) { return KA * bn * 128 + qw_bytes(bn) + v_bytes(bn); }
   static constexpr int BUDGET = 214 * 1024;
   // TMEM columns of the accumulators.  Register values: the large and the
   // small products of S in separate accumulators for each warpgroup (two
   // independent MMA chains; the small ones never round against the large
   // sum).  Tensor-core values: one S (small products first, then the large
-  // ones), P hi/lo and O per warpgroup.
-  static constexpr int tmem_acc(int bn) { return REG ? 4 * bn : 6 * bn + 2 * CPA; }
+  // ones), P hi/lo (fp16 pairs: bn / 2 columns each) and O per warpgroup.
+  static constexpr int tmem_acc(int bn) { return REG ? 4 * bn : 4 * bn + 2 * CPA; }
   // The x' rows (2 K' <= 32 KA columns) sit in TMEM as the A operand of the
   // similarity MMAs when the accumulators leave room, else in shared memory.
   static constexpr bool xt(int bn) { return tmem_acc(bn) + 32 * KA <= 512; }
@@ -122,7 +125,8 @@ struct F32Cfg {
   static constexpr int X_BYTES = x_bytes(BN);
   static constexpr int QW_BYTES = qw_bytes(BN);
   static constexpr int Y_BYTES = KA * BN * 128;
-  static constexpr int V_ATOM = CP * 128;               // CP rows x 32 columns
+  static constexpr int V_ATOM = CP * 128;               // CP rows x 64 fp16 columns
+  static constexpr int VA = va(BN);                     // v^T atoms per part and stage
   static constexpr int V_BYTES = v_bytes(BN);
   static constexpr int STAGE = stage_bytes(BN);
   static constexpr int NST_FIT = (BUDGET - X_BYTES) / STAGE;
@@ -136,9 +140,9 @@ struct F32Cfg {
   // Tensor-core values: S0 | S1 | Phi0 | Phi1 | Plo0 | Plo1 | O0 | O1 | x'.
   __host__ __device__ static constexpr uint32_t col_s(int h) { return h * BN; }
   __host__ __device__ static constexpr uint32_t col_ss(int h) { return 2 * BN + h * BN; }
-  __host__ __device__ static constexpr uint32_t col_phi(int h) { return 2 * BN + BN * h; }
-  __host__ __device__ static constexpr uint32_t col_plo(int h) { return 4 * BN + BN * h; }
-  __host__ __device__ static constexpr uint32_t col_o(int h) { return 6 * BN + CPA * h; }
+  __host__ __device__ static constexpr uint32_t col_phi(int h) { return 2 * BN + (BN / 2) * h; }
+  __host__ __device__ static constexpr uint32_t col_plo(int h) { return 3 * BN + (BN / 2) * h; }
+  __host__ __device__ static constexpr uint32_t col_o(int h) { return 4 * BN + CPA * h; }
   static constexpr uint32_t COL_X = tmem_acc(BN);
   static_assert(NST >= 2, "shared memory budget");
   static_assert(tmem_acc(BN) + (XT ? 32 * KA : 0) <= 512, "TMEM budget");
@@ -186,6 +190,9 @@ __device__ __forceinline__ int split_exp(int amax_bits) {
 }
 // 2^k for an integer -126 <= k <= 127, exactly.
 __device__ __forceinline__ float pow2_int(int k) { return __int_as_float((k + 127) << 23); }
+// Tensor-core values: P is multiplied by 2^14 before its fp16 split, which
+// keeps every P at or above 2^-28 in fp16's normal range.
+constexpr float kPScale = 16384.f;
 
 // Named barrier of the two exp warpgroups (warps 2-9).
 __device__ __forceinline__ void exp_warps_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
@@ -296,9 +303,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(smem_u32(sq), &tmQ, bar_full(st), j0, 0, static_cast<int>(b));
         if constexpr (!REG) {
           for (int hl = 0; hl < 2; ++hl)
-            for (int a = 0; a < BN / 32; ++a)
-              tma_load_3d(smem_u32(sv + (hl * (BN / 32) + a) * Cfg::V_ATOM), &tmV, bar_full(st),
-                          j0 + a * 32, 0, static_cast<int>(hl * p.Bsz + b));
+            for (int a = 0; a < Cfg::VA; ++a)
+              tma_load_3d(smem_u32(sv + (hl * Cfg::VA + a) * Cfg::V_ATOM), &tmV, bar_full(st),
+                          j0 + a * 64, 0, static_cast<int>(hl * p.Bsz + b));
         }
       }
     }
@@ -308,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // split rows: fp16 hi / lo parts (kind::f16, 16 per K step); unsplit: tf32
       const uint32_t idS = idesc_f16(SPLIT ? 0 : 2, kBM, BN);
-      const uint32_t idO = idesc_f16(2, kBM, CP);
+      const uint32_t idO = idesc_f16(0, kBM, CP);   // P.v: fp16 parts of P 2^14 and v 2^e
       const int ks_lo = p.ksteps;
       // K step ks (8 floats = 32 bytes) of a packed row block whose atoms are
       // atom_bytes apart
@@ -364,15 +371,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint8_t* sv = sStage + st * Cfg::STAGE + Cfg::Y_BYTES + Cfg::QW_BYTES;
         const uint32_t d = tmem + Cfg::col_o(h);
 #pragma unroll
-        for (int ks = 0; ks < BN / 8; ++ks) {
+        for (int ks = 0; ks < BN / 16; ++ks) {   // K steps of 16 columns
           const int a = ks >> 2, within = (ks & 3) * 32;
           const uint64_t bh = desc_k_sw128(smem_u32(sv + a * Cfg::V_ATOM) + within);
-          const uint64_t bl = desc_k_sw128(smem_u32(sv + ((BN / 32) + a) * Cfg::V_ATOM) + within);
+          const uint64_t bl = desc_k_sw128(smem_u32(sv + (Cfg::VA + a) * Cfg::V_ATOM) + within);
           const uint32_t phi = tmem + Cfg::col_phi(h) + ks * 8;
           const uint32_t plo = tmem + Cfg::col_plo(h) + ks * 8;
-          mma_ts_tf32(d, plo, bh, idO, (acc_prev || ks > 0) ? 1u : 0u);
-          mma_ts_tf32(d, phi, bl, idO, 1u);
-          mma_ts_tf32(d, phi, bh, idO, 1u);
+          mma_ts(d, plo, bh, idO, (acc_prev || ks > 0) ? 1u : 0u);
+          mma_ts(d, phi, bl, idO, 1u);
+          mma_ts(d, phi, bh, idO, 1u);
         }
       };
       bool ok = wait_bar(bar_x, 0, abort_flag);
@@ -597,28 +604,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar_f(h));
 #pragma unroll
         for (int ch = 0; ch < BN / 32; ++ch) {
+          // P 2^14 in fp16 hi + lo parts, two columns per 32-bit TMEM word:
+          // every P keeps an absolute error under 2^-39 (relative 2^-22 from
+          // P = 2^-3 up)
+          uint32_t hi[16], lo[16];
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t hi[16], lo[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int c = half * 16 + e;
-              const float pe = ex2(fmaf(__uint_as_float(sv[ch][c]), two_c, r) + qrec[ch * 32 + c]);
-              const float ph = tf32_trunc(pe);
-              hi[e] = __float_as_uint(ph);
-              lo[e] = __float_as_uint(pe - ph);
-            }
-            if (ch == 0 && half == 0 && k > 0) {
-              // P_h(previous tile) must have been read by its P.v MMAs
-              // (waited for as late as possible)
-              ok = __all_sync(0xffffffffu, wait_bar(bar_q(h), (k - 1) & 1, abort_flag));
-              if (!ok) break;
-              tc_fence_after();
-            }
-            tmem_st16(tPh + ch * 32 + half * 16, hi);
-            tmem_st16(tPl + ch * 32 + half * 16, lo);
+          for (int e = 0; e < 16; ++e) {
+            const int c = ch * 32 + 2 * e;
+            float t0, t1;
+            upk2(add2(fma2(pk2(__uint_as_float(sv[ch][2 * e]), __uint_as_float(sv[ch][2 * e + 1])),
+                           two_c2, r2),
+                      *reinterpret_cast<const uint64_t*>(qrec + c)),
+                 t0, t1);
+            const float u0 = ex2(t0) * kPScale, u1 = ex2(t1) * kPScale;
+            const __half2 h2 = __floats2half2_rn(u0, u1);
+            const float2 hf = __half22float2(h2);
+            const __half2 l2 = __floats2half2_rn(u0 - hf.x, u1 - hf.y);
+            hi[e] = *reinterpret_cast<const uint32_t*>(&h2);
+            lo[e] = *reinterpret_cast<const uint32_t*>(&l2);
           }
-          if (!ok) break;
+          if (ch == 0 && k > 0) {
+            // P_h(previous tile) must have been read by its P.v MMAs
+            // (waited for as late as possible)
+            ok = __all_sync(0xffffffffu, wait_bar(bar_q(h), (k - 1) & 1, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+          }
+          tmem_st16(tPh + ch * 16, hi);
+          tmem_st16(tPl + ch * 16, lo);
         }
         if (!ok) break;
         tmem_wait_st();
@@ -681,7 +694,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               float o = 0.f;
               if (T > 0) o = __uint_as_float(v0[q]);
               if (T > 1) o += __uint_as_float(v1[q]);   // O_1 holds tiles only when T > 1
-              if (c < p.cw) orow[c] = o;
+              // undo P's 2^14 and the channel's 2^e, exactly
+              if (c < p.cw) orow[c] = o * pow2_int(-14 - split_exp(p.vmax[b * CP + c]));
             }
           }
         }
@@ -833,14 +847,43 @@ __global__ void pack_values_qw_kernel(const TW* __restrict__ w, const TY* __rest
   }
 }
 
-// Split fp32 value matrix v^T: hi at [b][CP][Nst], lo at [B + b][CP][Nst], for
-// channels [c0, c0 + CP) of the pass's values (values.cuh); zeros past CV.
+// Per (batch, channel cc of the chunk [c0, c0 + CP)), the bits of max |v| over
+// the columns: the value parts' scale.  Grid (B CP, blocks) of 256 threads;
+// vmax zeroed before.
+__global__ void values_maxabs_kernel(const float* __restrict__ w, const float* __restrict__ y,
+                                     const float* __restrict__ rows, int* __restrict__ vmax,
+                                     int64_t N, int64_t Mrows, int C, int D, int CV, int c0, int CP,
+                                     int64_t src_ld) {
+  const int64_t bc = blockIdx.x;
+  const int cc = static_cast<int>(bc % CP);
+  const int64_t b = bc / CP;
+  const int ch = c0 + cc;
+  float m = 0.f;
+  if (ch < CV) {
+    for (int64_t j = blockIdx.y * static_cast<int64_t>(blockDim.x) + threadIdx.x; j < N;
+         j += static_cast<int64_t>(gridDim.y) * blockDim.x)
+      m = fmaxf(m, fabsf(value_at(w, y, rows, b, b * N + j, Mrows, D, C, ch, src_ld)));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ float wm[8];
+  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int v = 1; v < 8; ++v) m = fmaxf(m, wm[v]);
+    if (m > 0.f) atomicMax(vmax + bc, __float_as_int(m));
+  }
+}
+
+// Value matrix v^T in fp16 parts of v 2^e (e per batch and channel, from vmax):
+// hi at [b][CP][Nst], lo at [B + b][CP][Nst], for channels [c0, c0 + CP) of the
+// pass's values (values.cuh); zeros past CV.
 __global__ void pack_values_f32_split_kernel(const float* __restrict__ w,
                                              const float* __restrict__ y,
                                              const float* __restrict__ rows,
-                                             float* __restrict__ vt, int64_t B, int64_t N,
-                                             int64_t Nst, int64_t Mrows, int C, int D, int CV,
-                                             int c0, int CP, int64_t src_ld) {
+                                             __half* __restrict__ vt, const int* __restrict__ vmax,
+                                             int64_t B, int64_t N, int64_t Nst, int64_t Mrows, int C,
+                                             int D, int CV, int c0, int CP, int64_t src_ld) {
   const int64_t total = B * CP * N;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -850,9 +893,10 @@ __global__ void pack_values_f32_split_kernel(const float* __restrict__ w,
     const int64_t b = bc / CP;
     const int ch = c0 + cc;
     const float v = (ch < CV) ? value_at(w, y, rows, b, b * N + j, Mrows, D, C, ch, src_ld) : 0.f;
-    const float hi = tf32_round(v);
+    const float u = v * pow2_int(split_exp(vmax[b * CP + cc]));
+    const __half hi = __float2half_rn(u);
     vt[(b * CP + cc) * Nst + j] = hi;
-    vt[((B + b) * CP + cc) * Nst + j] = tf32_round(v - hi);
+    vt[((B + b) * CP + cc) * Nst + j] = __float2half_rn(u - __half2float(hi));
   }
 }
 
@@ -976,9 +1020,11 @@ int f32_tile_cols(int KA, int mode) {
 }
 
 // Packed rows of x and y (and, for fp32, the column centre first).
-// The per-batch max words sit right after the column centres (the workspace
-// layouts reserve B (D + 1) floats there).
+// The per-batch max words sit right after the column centres, then the
+// per-(batch, channel) max words of a tensor-core value chunk (the workspace
+// layouts reserve B (D + 1) floats, and B (D + 1 + 64) where chunks run).
 int* f32_amax(const F32Args& a) { return reinterpret_cast<int*>(a.zc + a.B * a.D); }
+int* f32_vmax(const F32Args& a) { return reinterpret_cast<int*>(a.zc + a.B * (a.D + 1)); }
 
 template <typename T>
 void pack_operands_f32(const F32Args& a, int64_t Nq, float c, cudaStream_t s) {
@@ -1055,7 +1101,7 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
   if (!make_tmap_3d(&m.x, rdt, a.xpack, rowe, a.M, a.B, rowb, a.M * rowb, atom_e, kBM))
     return cudaErrorInvalidValue;
   const int KA = ka_for(a.plan.atoms);
-  const int64_t Nst = (a.N + 3) / 4 * 4;
+  const int64_t Nst = (a.N + 7) / 8 * 8;   // fp16 rows of v^T: 16-byte multiples
   const dim3 grid(static_cast<unsigned>((a.M + kBM - 1) / kBM), static_cast<unsigned>(a.plan.splits),
                   static_cast<unsigned>(a.B));
   const int chunk = a.lse ? 1 : (reg ? 3 : a.plan.max_chunk);
@@ -1083,13 +1129,25 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
     } else {
       const int CP = mode;
       const int64_t total = a.B * CP * a.N;
+      int* vmax = f32_vmax(a);
+      e = cudaMemsetAsync(vmax, 0, static_cast<size_t>(a.B) * CP * sizeof(int), s);
+      if (e != cudaSuccess) return e;
+      {
+        int64_t nb = (a.N + 255) / 256;
+        const int64_t cap = (148 * 16 + a.B * CP - 1) / (a.B * CP);
+        if (nb > cap) nb = cap;
+        if (nb > 65535) nb = 65535;
+        values_maxabs_kernel<<<dim3(static_cast<unsigned>(a.B * CP), static_cast<unsigned>(nb)), 256, 0,
+                               s>>>(static_cast<const float*>(a.w), y, x, vmax, a.N, a.M, a.C, a.D,
+                                    a.CV, c0, CP, a.src_ld > 0 ? a.src_ld : a.C);
+      }
       pack_values_f32_split_kernel<<<grid_for(total, 256), 256, 0, s>>>(
-          static_cast<const float*>(a.w), y, x, a.vt, a.B, a.N, Nst, a.M, a.C, a.D, a.CV, c0, CP,
-          a.src_ld > 0 ? a.src_ld : a.C);
+          static_cast<const float*>(a.w), y, x, reinterpret_cast<__half*>(a.vt), vmax, a.B, a.N, Nst,
+          a.M, a.C, a.D, a.CV, c0, CP, a.src_ld > 0 ? a.src_ld : a.C);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
-      if (!make_tmap_3d(&m.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.vt, a.N, CP, 2 * a.B, Nst * 4ull,
-                        CP * Nst * 4ull, 32, CP))
+      if (!make_tmap_3d(&m.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.vt, a.N, CP, 2 * a.B, Nst * 2ull,
+                        CP * Nst * 2ull, 64, CP))
         return cudaErrorInvalidValue;
     }
     F32KParams kp{};
@@ -1111,6 +1169,7 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
     kp.split = a.plan.split ? 1 : 0;
     kp.two_c = a.tau * kLog2e;
     kp.amax = sp ? f32_amax(a) : nullptr;
+    kp.vmax = reg ? nullptr : f32_vmax(a);
     switch (KA) {
       case 1: e = launch_mode<1>(mode, a.lse, m, kp, grid, s); break;
       case 2: e = launch_mode<2>(mode, a.lse, m, kp, grid, s); break;
