@@ -189,6 +189,26 @@ def test_f32_tensor_core_coordinate_scales(scale, D, C):
     assert rel_l2(lse, lref) <= TOL["f32"], rel_l2(lse, lref)
 
 
+@pytest.mark.parametrize("tau", [1.0, 20.0])
+def test_f32_tensor_core_values_channel_scales(tau):
+    """Tensor-core values (4+ channels): channel c carries weights 10^(c - 10),
+    so one pass holds values from 1e-10 to 1e9; each channel's fp16 parts get
+    their own power-of-two scale.  Checked channel by channel; tau = 20 makes
+    most kernel values tiny (P 2^14 keeps them in fp16's normal range)."""
+    inp = synth.make_inputs(4, seed=41, B=2, M=200, N=900, D=32, C=20, dtype="f32")
+    wv = inp["w"].double() * torch.tensor([10.0 ** (c - 10) for c in range(20)], dtype=torch.float64)
+    inp["w"] = wv.float()
+    if tau > 1:
+        for k in ("x", "y"):
+            inp[k] = (inp[k].double() * 0.5).float()
+    d = dev(inp)
+    out = gs().gauss_sum_fwd(d["x"], d["y"], d["w"], tau).cpu().numpy()
+    ref = oracle.gauss_sum(f64(inp, "x"), f64(inp, "y"), f64(inp, "w"), tau)
+    for c in range(20):
+        e = rel_l2(out[..., c], ref[..., c])
+        assert e <= TOL["f32"], (c, e)
+
+
 @pytest.mark.parametrize("shape", [(1, 700, 900, 3, 1), (2, 300, 1100, 2, 3), (1, 64, 5000, 8, 9)])
 def test_lse_f32_shapes(shape):
     B, M, N, D, C = shape
