@@ -24,6 +24,8 @@
 //   P_h = ex2(fma(S_h, 2c, r))  (tcgen05.ld -> MUFU -> fp16 -> tcgen05.st)
 //   O_h += P_h . v(t)           (tcgen05.mma, A = P from TMEM, B = v^T smem)
 // The issue order S0(t+1) before O1(t) lets both exp warpgroups run at once.
+// One value channel (CP = 1): no P.v MMAs; the exp warps sum P w in registers
+// against an fp32 record per column that rides with the stage.
 // Every mbarrier wait is bounded (2 s); on expiry the kernel raises the device
 // error word, lets the other warps leave, frees TMEM and returns.
 #include <cuda.h>
@@ -70,8 +72,14 @@ struct TcCfg {
   static constexpr int ATOM = kBM * 128;        // one 128-row x 64-col block: 16 KB
   static constexpr int X_BYTES = kNT * KC * ATOM;
   static constexpr int Y_BYTES = KC * ATOM;
-  static constexpr int V_BYTES = 2 * CP * 128;  // two 64-column atoms of CP rows
+  // One value channel (CP == 1) is summed in registers from an fp32 record per
+  // column (512 bytes a tile, padded to keep the stages 1024-byte aligned);
+  // wider chunks go through the tensor cores from v^T, two 64-column atoms of
+  // CP rows.
+  static constexpr bool REG = CP == 1;
+  static constexpr int V_BYTES = REG ? 1024 : 2 * CP * 128;
   static constexpr int STAGE = Y_BYTES + V_BYTES;
+  static constexpr int TX = Y_BYTES + (REG ? kBN * 4 : V_BYTES);   // bytes a stage's TMA loads
   // 200 KB of operand stages; the three-atom rows (D > 126) may take 220 KB
   static constexpr int BUDGET = (KC > 2 ? 220 : 200) * 1024;
   static constexpr int NST_FIT = (BUDGET - X_BYTES) / STAGE;
@@ -93,7 +101,7 @@ struct TcCfg {
     return P_SEPARATE ? 384u + 64u * h : 128u * h;
   }
   static_assert(NST >= 2, "shared memory budget");
-  static_assert(CP % 16 == 0 && CP >= 16 && CP <= 128, "value chunk");
+  static_assert(CP == 1 || (CP % 16 == 0 && CP >= 16 && CP <= 128), "value chunk");
 };
 
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
@@ -177,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(bar_full(s), 1);
-      mbar_init(bar_empty(s), 1);
+      mbar_init(bar_empty(s), Cfg::REG ? 8 : 1);   // register values: the 8 exp warps release it
     }
     mbar_init(bar_x, 1);
     mbar_init(bar_s(0), 1);
@@ -218,13 +226,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* sy = sStage + st * Cfg::STAGE;
         uint8_t* sv = sy + Cfg::Y_BYTES;
         const int j0 = static_cast<int>(jbeg + static_cast<int64_t>(t) * kBN);
-        mbar_arrive_expect_tx(bar_full(st), Cfg::STAGE);
+        mbar_arrive_expect_tx(bar_full(st), Cfg::TX);
         for (int kc = 0; kc < Cfg::KC; ++kc)
           tma_load_3d(smem_u32(sy + kc * Cfg::ATOM), &tmY, bar_full(st), kc * 64, j0,
                       static_cast<int>(b));
-        for (int hh = 0; hh < 2; ++hh)
-          tma_load_3d(smem_u32(sv + hh * CP * 128), &tmV, bar_full(st), j0 + hh * 64, 0,
-                      static_cast<int>(b));
+        if constexpr (Cfg::REG) {
+          tma_load_3d(smem_u32(sv), &tmV, bar_full(st), j0, 0, static_cast<int>(b));
+        } else {
+          for (int hh = 0; hh < 2; ++hh)
+            tma_load_3d(smem_u32(sv + hh * CP * 128), &tmV, bar_full(st), j0 + hh * 64, 0,
+                        static_cast<int>(b));
+        }
       }
     }
     __syncwarp();
@@ -269,7 +281,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; ok && t < T; ++t) {
         const int st = t % NST;
         const int st1 = (t + 1) % NST;
-        if constexpr (Cfg::P_SEPARATE) {
+        if constexpr (Cfg::REG) {
+          // register values: only the similarity MMAs; S_h(t+1) once warpgroup h
+          // has read S_h(t) (the exp warps release the stages themselves)
+          if (t + 1 < T) {
+            if (!(ok = wait_bar(bar_f(0), t & 1, abort_flag))) break;
+            if (!(ok = wait_bar(bar_full(st1), ((t + 1) / NST) & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_S(0, st1);
+            mma_commit(bar_s(0));
+            if (!(ok = wait_bar(bar_f(1), t & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_S(1, st1);
+            mma_commit(bar_s(1));
+          }
+        } else if constexpr (Cfg::P_SEPARATE) {
           // S_h(t+1) may overwrite S_h as soon as warpgroup h has read S_h(t)
           // into registers: it then runs while the exponentials of tile t are
           // still being computed.
@@ -316,7 +342,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      mma_commit(bar_o);   // also the drain point for whatever was issued
+      // the drain point for whatever was issued (register values: every S MMA
+      // was waited for by the exp warps, and nothing waits on this barrier)
+      if constexpr (!Cfg::REG) mma_commit(bar_o);
     }
     __syncwarp();
   } else {
@@ -335,8 +363,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     const uint64_t two_c2 = pk2(two_c, two_c);
     const uint64_t r2 = pk2(r, r);
+    float row_sum = 0.f;   // register values: the row's sum over the tiles
     for (int t = 0; t < T; ++t) {
       ok = wait_bar(bar_s(h), t & 1, abort_flag);
+      // register values read the stage's records themselves: its loads landed
+      if (Cfg::REG && ok) ok = wait_bar(bar_full(t % NST), (t / NST) & 1, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
@@ -356,51 +387,98 @@ __global__ void __launch_bounds__(kThreads, 1)
       reg_fence32(va);
       reg_fence32(vb);
       tmem_ld32(tS + 64, vc);
-      exp_chunk(va, two_c2, r2, pk);
-      if (Cfg::P_SEPARATE && t > 0) {
-        // a warp that runs ahead must not overwrite its rows of P(t-1) before
-        // the P MMA of tile t-1 has read them (waited for as late as possible)
-        ok = __all_sync(0xffffffffu, wait_bar(bar_q(h), (t - 1) & 1, abort_flag));
-        if (!ok) {
-          tmem_wait_ld();   // chunk 2's load may still be in flight
-          break;
-        }
-        tc_fence_after();
-      }
-      tmem_st16(tP, pk);
-      tmem_ld32(tS + 96, va);
-      exp_chunk(vb, two_c2, r2, pk);
-      tmem_st16(tP + 16, pk);
-      tmem_wait_ld();
-      reg_fence32(vc);
-      reg_fence32(va);
-      tc_fence_before();
-      mbar_arrive(bar_f(h));
-      exp_chunk(vc, two_c2, r2, pk);
-      tmem_st16(tP + 32, pk);
-      exp_chunk(va, two_c2, r2, pk);
-      tmem_st16(tP + 48, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar_p(h));
-    }
-    if (ok) ok = wait_bar(bar_o, 0, abort_flag);
-    ok = __all_sync(0xffffffffu, ok);
-    tc_fence_after();
-    if (ok) {
-      float* orow = p.out + static_cast<int64_t>(blockIdx.y) * p.split_stride +
-                    (b * p.M + i) * p.ldo + p.c0;
+      if constexpr (Cfg::REG) {
+        // one value channel: P w summed in registers (fp32 P, exact products),
+        // two columns per packed operation, a partial per tile
+        const float* wr =
+            reinterpret_cast<const float*>(sStage + (t % NST) * Cfg::STAGE + Cfg::Y_BYTES);
+        uint64_t acc2 = 0ull;
+        auto reg_chunk = [&](const uint32_t(&v)[32], const float* w) {
 #pragma unroll
-      for (int ch = 0; ch < CP / 16; ++ch) {
-        uint32_t v[16];
-        tmem_ld16(tO + ch * 16, v);
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 w4 = *reinterpret_cast<const float4*>(w + 4 * e4);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              float t0, t1;
+              upk2(fma2(pk2(__uint_as_float(v[4 * e4 + 2 * hh]),
+                            __uint_as_float(v[4 * e4 + 2 * hh + 1])),
+                        two_c2, r2),
+                   t0, t1);
+              acc2 = fma2(pk2(ex2(t0), ex2(t1)), hh ? pk2(w4.z, w4.w) : pk2(w4.x, w4.y), acc2);
+            }
+          }
+        };
+        reg_chunk(va, wr);
+        tmem_ld32(tS + 96, va);
+        reg_chunk(vb, wr + 32);
         tmem_wait_ld();
-        reg_fence16(v);
-        if (valid) {
+        reg_fence32(vc);
+        reg_fence32(va);
+        tc_fence_before();
+        mbar_arrive(bar_f(h));
+        reg_chunk(vc, wr + 64);
+        reg_chunk(va, wr + 96);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_empty(t % NST));   // this warp is done with the records
+        float lo, hi;
+        upk2(acc2, lo, hi);
+        row_sum += lo + hi;
+      } else {
+        exp_chunk(va, two_c2, r2, pk);
+        if (Cfg::P_SEPARATE && t > 0) {
+          // a warp that runs ahead must not overwrite its rows of P(t-1) before
+          // the P MMA of tile t-1 has read them (waited for as late as possible)
+          ok = __all_sync(0xffffffffu, wait_bar(bar_q(h), (t - 1) & 1, abort_flag));
+          if (!ok) {
+            tmem_wait_ld();   // chunk 2's load may still be in flight
+            break;
+          }
+          tc_fence_after();
+        }
+        tmem_st16(tP, pk);
+        tmem_ld32(tS + 96, va);
+        exp_chunk(vb, two_c2, r2, pk);
+        tmem_st16(tP + 16, pk);
+        tmem_wait_ld();
+        reg_fence32(vc);
+        reg_fence32(va);
+        tc_fence_before();
+        mbar_arrive(bar_f(h));
+        exp_chunk(vc, two_c2, r2, pk);
+        tmem_st16(tP + 32, pk);
+        exp_chunk(va, two_c2, r2, pk);
+        tmem_st16(tP + 48, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_p(h));
+      }
+    }
+    if constexpr (Cfg::REG) {
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok && valid && !*abort_flag) {
+        float* orow = p.out + static_cast<int64_t>(blockIdx.y) * p.split_stride +
+                      (b * p.M + i) * p.ldo + p.c0;
+        orow[0] = (T > 0) ? row_sum * p.out_scale : 0.f;
+      }
+    } else {
+      if (ok) ok = wait_bar(bar_o, 0, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+      if (ok) {
+        float* orow = p.out + static_cast<int64_t>(blockIdx.y) * p.split_stride +
+                      (b * p.M + i) * p.ldo + p.c0;
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            const int c = ch * 16 + q;
-            if (c < p.cw) orow[c] = (T > 0) ? __uint_as_float(v[q]) * p.out_scale : 0.f;
+        for (int ch = 0; ch < CP / 16; ++ch) {
+          uint32_t v[16];
+          tmem_ld16(tO + ch * 16, v);
+          tmem_wait_ld();
+          reg_fence16(v);
+          if (valid) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const int c = ch * 16 + q;
+              if (c < p.cw) orow[c] = (T > 0) ? __uint_as_float(v[q]) * p.out_scale : 0.f;
+            }
           }
         }
       }
@@ -516,6 +594,20 @@ __global__ void pack_values_kernel(const TW* __restrict__ w, const TY* __restric
   }
 }
 
+// One value channel (CV == 1): its fp32 values rec [B, Nw] (zeros past N), the
+// per-column records the register-value kernel sums against.
+template <typename TW, typename TY>
+__global__ void pack_records_kernel(const TW* __restrict__ w, const TY* __restrict__ y,
+                                    const TY* __restrict__ rows, float* __restrict__ rec, int64_t B,
+                                    int64_t N, int64_t Nw, int64_t Mrows, int C, int D) {
+  const int64_t total = B * Nw;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = e / Nw, j = e % Nw;
+    rec[e] = (j < N) ? value_at(w, y, rows, b, b * N + j, Mrows, D, C, 0, C) : 0.f;
+  }
+}
+
 // ------------------------------------------------------------------ host side
 int grid_for(int64_t n, int threads) {
   int64_t b = (n + threads - 1) / threads;
@@ -542,6 +634,21 @@ cudaError_t pack_operands(const TcArgs& a, cudaStream_t s) {
   };
   launch_rows(a.x, a.xpack, a.rnorm, a.B * a.M, 1);
   launch_rows(a.y, a.ypack, nullptr, a.B * a.N, 0);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t pack_records(const TcArgs& a, int64_t Nw, cudaStream_t s) {
+  const int blocks = grid_for(a.B * Nw, 256);
+  const T* y = static_cast<const T*>(a.y);
+  const T* rows = static_cast<const T*>(a.x);
+  float* rec = static_cast<float*>(a.vt);
+  if (a.w_is_f32)
+    pack_records_kernel<float, T><<<blocks, 256, 0, s>>>(static_cast<const float*>(a.w), y, rows, rec,
+                                                         a.B, a.N, Nw, a.M, a.C, a.D);
+  else
+    pack_records_kernel<T, T><<<blocks, 256, 0, s>>>(static_cast<const T*>(a.w), y, rows, rec, a.B,
+                                                     a.N, Nw, a.M, a.C, a.D);
   return cudaGetLastError();
 }
 
@@ -583,12 +690,14 @@ cudaError_t launch_cp(int CP, const CUtensorMap& tx, const CUtensorMap& ty, cons
   if constexpr (KP > 128) {
     // three-atom rows: value chunks of at most 48 channels fit two stages
     switch (CP) {
+      case 1: return launch_kernel<KP, 1, DTFMT>(tx, ty, tv, kp, grid, s);
       case 16: return launch_kernel<KP, 16, DTFMT>(tx, ty, tv, kp, grid, s);
       case 32: return launch_kernel<KP, 32, DTFMT>(tx, ty, tv, kp, grid, s);
       default: return launch_kernel<KP, 48, DTFMT>(tx, ty, tv, kp, grid, s);
     }
   } else {
     switch (CP) {
+      case 1: return launch_kernel<KP, 1, DTFMT>(tx, ty, tv, kp, grid, s);
       case 16: return launch_kernel<KP, 16, DTFMT>(tx, ty, tv, kp, grid, s);
       case 32: return launch_kernel<KP, 32, DTFMT>(tx, ty, tv, kp, grid, s);
       case 48: return launch_kernel<KP, 48, DTFMT>(tx, ty, tv, kp, grid, s);
@@ -685,13 +794,24 @@ cudaError_t launch_tc_sum(const TcArgs& a, cudaStream_t s) {
   const int chunk = tc_max_chunk(KP);
   for (int c0 = 0; c0 < a.CV; c0 += chunk) {
     const int cw = (a.CV - c0) < chunk ? (a.CV - c0) : chunk;
-    const int CP = tc_chunk_pad(cw);
-    e = bf ? pack_values<__nv_bfloat16>(a, c0, CP, Nst, s) : pack_values<__half>(a, c0, CP, Nst, s);
-    if (e != cudaSuccess) return e;
+    // one value channel: fp32 records summed in registers (CP = 1)
+    const bool reg1 = a.CV == 1;
+    const int CP = reg1 ? 1 : tc_chunk_pad(cw);
     CUtensorMap tv;
-    if (!make_tmap_3d(&tv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.vt, a.N, CP, a.B, Nst * 2ull,
-                      CP * Nst * 2ull, 64, CP))
-      return cudaErrorInvalidValue;
+    if (reg1) {
+      const int64_t Nw = (a.N + 3) / 4 * 4;
+      e = bf ? pack_records<__nv_bfloat16>(a, Nw, s) : pack_records<__half>(a, Nw, s);
+      if (e != cudaSuccess) return e;
+      if (!make_tmap_3d(&tv, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.vt, Nw, 1, a.B, Nw * 4ull, Nw * 4ull,
+                        kBN, 1, false))
+        return cudaErrorInvalidValue;
+    } else {
+      e = bf ? pack_values<__nv_bfloat16>(a, c0, CP, Nst, s) : pack_values<__half>(a, c0, CP, Nst, s);
+      if (e != cudaSuccess) return e;
+      if (!make_tmap_3d(&tv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.vt, a.N, CP, a.B, Nst * 2ull,
+                        CP * Nst * 2ull, 64, CP))
+        return cudaErrorInvalidValue;
+    }
     TcKParams kp{};
     kp.rnorm = a.rnorm;
     kp.out = a.out;
