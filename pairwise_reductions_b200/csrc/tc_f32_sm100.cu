@@ -167,11 +167,6 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
-// v -> its tf32 part by truncation (the bits a kind::tf32 MMA reads); v - hi
-// is then exact in fp32.
-__device__ __forceinline__ float tf32_trunc(float v) {
-  return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
-}
 // Round to the nearest tf32 value, ties away from zero (finite inputs).
 __device__ __forceinline__ float tf32_round(float v) {
   return __uint_as_float((__float_as_uint(v) + 0x1000u) & 0xFFFFE000u);
