@@ -161,3 +161,28 @@ def test_binding_status_checks_are_well_formed():
         first = c.args[0]
         if isinstance(first, ast.Constant):
             assert first.value in declared, first.value
+
+
+@pytest.mark.parametrize("n", [1_000, 10_000, 100_000, 1_000_000])
+def test_split_counts_stay_within_the_combines(n):
+    # small-D fp32: the sum's workspace is its split partials [S, B, M, C]; the
+    # log-sum-exp's is (m, l) per split, and its finalize merges the splits
+    # within one warp, so S <= 32 there; the sum allows up to 256 splits and at
+    # most 2^25 partial floats
+    ws = gs.workspace_bytes
+    s_sum = ws(gs.GS_OP_SUM, 1, n, n, 3, 1, gs.GS_F32) // (4 * n)
+    s_lse = ws(gs.GS_OP_LSE, 1, n, n, 3, 1, gs.GS_F32) // (8 * n)
+    assert 1 <= s_lse <= 32, s_lse
+    assert s_sum <= 256 and s_sum * n <= (1 << 25) + 256, s_sum
+    # every split keeps at least 128 columns
+    assert s_sum <= max(1, n // 128)
+
+
+def test_autograd_wrappers_validate_tau_before_any_launch():
+    import torch
+    from pairwise_reductions_b200 import autograd
+    x = torch.zeros(4, 3)
+    with pytest.raises(ValueError):
+        autograd.gauss_sum(x, x, torch.zeros(4, 1), torch.ones(2))
+    with pytest.raises(ValueError):
+        autograd.gauss_lse(x, x, torch.ones(4, 1), torch.ones(3))
