@@ -23,6 +23,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import torch
@@ -56,6 +57,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-launch-count", action="store_true",
                     help="skip the profiler-based kernel count (use under ncu)")
+    ap.add_argument("--clock-log", default=None,
+                    help="CSV of the nvidia-smi clock samples (default: a file under the temp directory)")
     ap.add_argument("--sharded", action="store_true",
                     help="one problem of the workload's size split over the ranks by rows and "
                          "sources (strong scaling; the sources are all-gathered every step)")
@@ -375,8 +378,9 @@ def main():
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    clk = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
-                       if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/gs_clocks_{rank}.csv")
+    clk_path = (args.clock_log.replace(".csv", f"_rank{rank}.csv") if args.clock_log
+                else os.path.join(tempfile.gettempdir(), f"gs_clocks_{rank}.csv"))
+    clk = ClockSampler(local, clk_path)
     barrier(pg)
     torch.cuda.synchronize()
     with clk:
