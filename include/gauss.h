@@ -22,14 +22,18 @@
  * Supported shapes and types:
  *     GS_F32           : 1 <= D <= 8 (CUDA-core path), any C >= 1;
  *                        9 <= D <= 128 (tensor-core path at fp32 accuracy:
- *                        every operand split into tf32 hi + lo, three tf32
+ *                        every operand split into two fp16 parts of 11
+ *                        significant bits under power-of-two scales, three
  *                        MMAs per product) for the sums, their gradients,
  *                        the diffusion operator and the log-sum-exp.
  *     GS_F16 / GS_BF16 : 1 <= D <= 128 (tensor-core path), any C >= 1.
  *                        Arithmetic: x.y on the tensor cores with fp32
- *                        accumulation, kernel values rounded to fp16 for the
- *                        second product, weights converted to fp16 (for bf16
- *                        weights this is exact for |w| in [2^-14, 65504]).
+ *                        accumulation; with C > 1 (per pass of value
+ *                        channels) kernel values rounded to fp16 for the
+ *                        second product and weights converted to fp16 (for
+ *                        bf16 weights exact for |w| in [2^-14, 65504]); with
+ *                        one channel the products are summed in fp32 from the
+ *                        fp32 kernel value and the exact weight.
  *                        The log-sum-exp runs on the tf32 tensor-core path
  *                        (fp16 / bf16 values are exact in tf32).
  *     The log-sum-exp backward and the k-nearest reduction: every dtype,
@@ -115,8 +119,9 @@ gs_status gauss_sum_fwd(const void *x, const void *y, const void *w, float *out,
  * still get a finite result.  Requires w > 0 (not checked: a non-positive
  * weight gives NaN or -inf, as log does).  N == 0 writes -inf.
  * Supported for 1 <= D <= 128 in every dtype: GS_F32 with D <= 8 on the
- * CUDA-core path (power-of-two weight shifts), the rest on the tf32
- * tensor-core path (a running maximum per row).
+ * CUDA-core path (power-of-two weight shifts), the rest on the tensor-core
+ * path (split fp16 parts for fp32, tf32 for fp16 / bf16; a running maximum
+ * per row).
  */
 gs_status gauss_lse_fwd(const void *x, const void *y, const void *w, float *out, int64_t B,
                         int64_t M, int64_t N, int64_t D, int64_t C, float tau, gs_dtype dt,
@@ -206,7 +211,7 @@ gs_status gauss_sum_vjp(const void *x, const void *y, const void *w, const float
  * lse [B, M, C] float32 is the forward's output for the same inputs.  The
  * shift -lse is folded into every kernel exponent, so the passes sum p
  * directly (no overflow, no separate normalisation).  1 <= D <= 128 (fp32:
- * D > 8 on tf32 tensor-core passes; fp16 / bf16: exact fp32 copies first),
+ * D > 8 on split tensor-core passes; fp16 / bf16: exact fp32 copies first),
  * w > 0; any output may be NULL.  Workspace:
  * gs_workspace_bytes(GS_OP_LSE_BWD, ...).
  */
