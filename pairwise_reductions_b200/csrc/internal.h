@@ -183,9 +183,9 @@ bool make_tmap_3d(CUtensorMap* m, CUtensorMapDataType dt, void* base, uint64_t d
 // ------------------------------------------------------------- fp32 tensor-core path
 // fp32 inputs with kSdMaxD < D <= kTcMaxD: split-tf32 MMAs (tc_f32_sm100.cu).
 struct F32Plan {
-  bool split;          // fp32 inputs: fp16 rows [hi | lo]; fp16 / bf16 (exact tf32): tf32 [hi] only
-  int Kp;              // elements per half of a packed row: D rounded up to 16 (split) or 8
-  int atoms;           // 128-byte atoms per packed row (2 Kp halves, or Kp floats)
+  bool split;          // fp32 inputs: fp16 rows [hi | lo]; fp16 / bf16: the input values, unsplit
+  int Kp;              // 16-bit elements per half of a packed row: D rounded up to 16
+  int atoms;           // 128-byte atoms per packed row (2 Kp or Kp 16-bit values)
   int max_chunk;       // channels per pass (64, or 32 for the widest rows)
   int splits;
   int64_t cols_per_split;   // multiple of 128

@@ -20,7 +20,7 @@
 //     exp(-tau/2 |x_i - y_j|^2) = 2^(2c x'_i.y'_j + r_i + q_j),
 //     r_i = -c |x'_i|^2,  q_j = -c |y'_j|^2
 // (the norm factors of Algorithm 1 on the same page).  P_ij = ex2(fma(S, 2c, r_i) + q_j)
-// with S from the split MMAs; P is split into tf32 hi/lo again for P.v.
+// with S from the split MMAs; P is split into fp16 hi/lo parts again for P.v.
 //
 // CTA = one 128-row tile, 10 warps:
 //   warp 0      TMA producer: the x' rows once (unless they sit in TMEM), then a
@@ -42,8 +42,9 @@
 // or (tensor-core values, 4 .. 64 channels per pass)
 //   P_h 2^14 -> fp16 hi/lo -> tcgen05.st;  O_h += P_h . v(t), 3 fp16 MMAs per
 //   K step of 16 (A = P from TMEM); the scales are undone on output.
-// fp16 / bf16 inputs (log-sum-exp) are exact in tf32: unsplit tf32 rows, one
-// MMA per K step of 8 (template SPLIT = false).
+// fp16 / bf16 inputs (log-sum-exp) are exact in their own format: unsplit
+// rows of the input values, one kind::f16 MMA (fp16 or bf16 encoding) per K
+// step of 16 (template SPLIT = false).
 // Every mbarrier wait is bounded (2 s); on expiry the kernel raises its device
 // error word, lets the other warps leave, frees TMEM and returns.
 #include <cuda.h>
@@ -77,11 +78,12 @@ struct F32KParams {
   int64_t ldo;
   int c0, cw;
   int64_t cols_per_split;
-  int ksteps;           // 32-byte K steps of the hi (and of the lo) half: K'/16 fp16, K'/8 tf32
+  int ksteps;           // K'/16: 32-byte K steps of the hi (and of the lo) half
   int atoms;            // 128-byte atoms of a packed row actually loaded (<= KA)
   int Bsz;              // batch count (the lo half of v sits at batch index B + b)
   int bn;               // tile width the TMA boxes were made for
-  int split;            // 1: fp16 rows [hi | lo]; 0: rows are exact tf32 (fp16 / bf16 inputs), hi only
+  int split;            // 1: fp16 rows [hi | lo]; 0: rows are the fp16 / bf16 inputs themselves
+  int afmt;             // unsplit rows: 0 fp16, 1 bf16 (the MMA's operand encoding)
   float two_c;
   const int* amax;      // split rows: per batch, the bits of max |v'| (sets the power-of-two scale)
   const int* vmax;      // tensor-core values: per (batch, channel of the chunk), the bits of max |v|
@@ -115,8 +117,8 @@ struct F32Cfg {
   static constexpr bool fits(int bn) {
     return tmem_acc(bn) <= 512 && (BUDGET - x_bytes(bn)) / stage_bytes(bn) >= 2;
   }
-  // Column tile.  An M = 128 tf32 MMA takes about the same time for any N up
-  // to 128 (measured on B200: ~78 cycles at N = 32 .. 128), so the widest
+  // Column tile.  An M = 128 MMA takes about the same time for any N up to
+  // 128 (measured on B200: ~78 cycles at N = 32 .. 128 for tf32), so the widest
   // tile that fits is the cheapest per pair; three register channels use 32
   // columns (registers).
   static constexpr int BN =
@@ -167,10 +169,10 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
-// Round to the nearest tf32 value, ties away from zero (finite inputs).
-__device__ __forceinline__ float tf32_round(float v) {
-  return __uint_as_float((__float_as_uint(v) + 0x1000u) & 0xFFFFE000u);
-}
+// The 16 bits of an fp16 / bf16 value (unsplit rows; fp32 inputs never take them).
+__device__ __forceinline__ uint16_t raw16(__half v) { return __half_as_ushort(v); }
+__device__ __forceinline__ uint16_t raw16(__nv_bfloat16 v) { return __bfloat16_as_ushort(v); }
+__device__ __forceinline__ uint16_t raw16(float v) { return __half_as_ushort(__float2half_rn(v)); }
 
 // Split rows hold v' 2^e in fp16 hi + lo parts, e per batch from the bits of
 // max |v'| over its x' and y' rows: the largest scaled value lies in
@@ -196,8 +198,8 @@ __device__ __forceinline__ void exp_warps_sync() { asm volatile("bar.sync 1, 256
 // t_ij + log2 w_j as a running maximum m and a sum l of 2^(t - m), updated per
 // 32-column chunk (the maximum of the chunk first, then its shifted sum), so
 // that no value under- or overflows.
-// SPLIT: rows [hi | lo] and three products per K step (fp32 inputs), or exact
-// tf32 rows (fp16 / bf16 inputs) and the large product alone.
+// SPLIT: rows [hi | lo] and three products per K step (fp32 inputs), or the
+// exact fp16 / bf16 input rows and the large product alone.
 template <int KA, int MODE, bool LSE, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_f32_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
@@ -206,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using Cfg = F32Cfg<KA, MODE>;
   constexpr bool REG = Cfg::REG;
   static_assert(REG || !LSE, "log-sum-exp runs on the register path");
-  constexpr int kAtomElems = SPLIT ? 64 : 32;   // packed-row elements per 128-byte atom
+  constexpr int kAtomElems = 64;   // 16-bit packed-row elements per 128-byte atom
   constexpr int CP = Cfg::CP;
   constexpr int NST = Cfg::NST;
   constexpr int BN = Cfg::BN;
@@ -308,8 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      // split rows: fp16 hi / lo parts (kind::f16, 16 per K step); unsplit: tf32
-      const uint32_t idS = idesc_f16(SPLIT ? 0 : 2, kBM, BN);
+      // kind::f16, 16 per K step: fp16 hi / lo parts, or the unsplit fp16 / bf16 rows
+      const uint32_t idS = idesc_f16(SPLIT ? 0 : p.afmt, kBM, BN);
       const uint32_t idO = idesc_f16(0, kBM, CP);   // P.v: fp16 parts of P 2^14 and v 2^e
       const int ks_lo = p.ksteps;
       // K step ks (8 floats = 32 bytes) of a packed row block whose atoms are
@@ -329,19 +331,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t db = tmem + Cfg::col_s(h);
         const uint32_t ds = REG ? tmem + Cfg::col_ss(h) : db;
         auto mma = [&](uint32_t d, int ka, uint64_t bdesc, uint32_t acc) {
-          if constexpr (Cfg::XT) {
-            if constexpr (SPLIT)
-              mma_ts(d, tmem + Cfg::COL_X + ka * 8, bdesc, idS, acc);
-            else
-              mma_ts_tf32(d, tmem + Cfg::COL_X + ka * 8, bdesc, idS, acc);
-          } else {
-            if constexpr (SPLIT)
-              mma_ss(d, kdesc(sX, kAtom, ka), bdesc, idS, acc);
-            else
-              mma_ss_tf32(d, kdesc(sX, kAtom, ka), bdesc, idS, acc);
-          }
+          if constexpr (Cfg::XT)
+            mma_ts(d, tmem + Cfg::COL_X + ka * 8, bdesc, idS, acc);
+          else
+            mma_ss(d, kdesc(sX, kAtom, ka), bdesc, idS, acc);
         };
-        // (exact tf32 operands, SPLIT false: the large products alone)
+        // (exact 16-bit operands, SPLIT false: the large products alone)
         if constexpr (REG) {
           for (int ks = 0; ks < p.ksteps; ++ks) {
             const uint64_t bh = kdesc(sy, BN * 128, ks);
@@ -767,8 +762,8 @@ __global__ void centred_maxabs_kernel(const float* __restrict__ x, const float* 
 // v' itself in fp32: for the row side into
 // norm[b * R + r]; for the column side (records) into lane 0 of the column's
 // record, norm[4 b Rpad + r] (lanes 1-3, Rpad floats apart, zeroed), with -inf
-// for the padding columns r >= R.  Exact tf32 inputs
-// (fp16 / bf16, zc == nullptr, split == 0): v itself, rows [hi (K')] only.
+// for the padding columns r >= R.  fp16 / bf16 inputs (zc == nullptr,
+// split == 0): the input values themselves, rows [v (K')] only.
 // One warp per row, lanes along the features (coalesced reads and writes).
 template <typename T>
 __global__ void pack_rows_f32_kernel(const T* __restrict__ src, const float* __restrict__ zc,
@@ -807,11 +802,12 @@ __global__ void pack_rows_f32_kernel(const T* __restrict__ src, const float* __r
         out[Kp + k] = __float2half_rn(u - __half2float(hi));
       }
     } else {
-      float* out = dst + (b * R + rr) * static_cast<int64_t>(Kp);
+      // the fp16 / bf16 input values themselves (exact in the MMA's encoding)
+      uint16_t* out = reinterpret_cast<uint16_t*>(dst) + (b * R + rr) * static_cast<int64_t>(Kp);
       for (int k = lane; k < Kp; k += 32) {
-        const float d = (k < D) ? vf(v[k]) - (z ? z[k] : 0.f) : 0.f;
+        const float d = (k < D) ? vf(v[k]) : 0.f;
         sq = fmaf(d, d, sq);
-        out[k] = tf32_round(d);
+        out[k] = (k < D) ? raw16(v[k]) : static_cast<uint16_t>(0);
       }
     }
 #pragma unroll
@@ -973,10 +969,10 @@ int tile_cols_ka(int mode) {
 F32Plan f32_plan(int64_t B, int64_t M, int64_t N, int64_t D, int sm_count, bool split) {
   F32Plan p{};
   p.split = split;
-  // split: fp16 [hi | lo] rows, K' = D rounded up to 16 (kind::f16 K steps);
-  // unsplit: tf32 [hi] rows, K' = D rounded up to 8
-  p.Kp = static_cast<int>(split ? (D + 15) / 16 * 16 : (D + 7) / 8 * 8);
-  p.atoms = split ? (2 * p.Kp + 63) / 64 : (p.Kp + 31) / 32;
+  // 16-bit rows, K' = D rounded up to 16 (kind::f16 K steps): fp16 [hi | lo]
+  // (split) or the fp16 / bf16 input values (unsplit)
+  p.Kp = static_cast<int>((D + 15) / 16 * 16);
+  p.atoms = ((split ? 2 : 1) * p.Kp + 63) / 64;
   p.max_chunk = ka_for(p.atoms) >= 8 ? 32 : 64;
   // a split is a whole number of 128-column blocks (every tile width divides
   // it, so no tile straddles two splits)
@@ -1065,7 +1061,7 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
   const float c = 0.5f * a.tau * kLog2e;
   const int64_t Nq = (a.N + 127) / 128 * 128;
   // register values for at most 3 channels per pass; the log-sum-exp one
-  // channel per pass; fp16 / bf16 inputs (exact tf32) take the register path only
+  // channel per pass; fp16 / bf16 inputs (unsplit rows) take the register path only
   const bool reg = a.lse || a.CV <= 3;
   if (a.dt != GS_F32 && (!reg || a.plan.split)) return cudaErrorInvalidValue;
   if (a.dt == GS_F32)
@@ -1087,12 +1083,14 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
   const float* x = static_cast<const float*>(a.x);   // fp32 only below (tensor-core values)
   const float* y = static_cast<const float*>(a.y);
   TileMaps m;
-  // split rows: fp16 [hi | lo], 64 per 128-byte atom; unsplit: tf32 [hi], 32 per atom
+  // 16-bit packed rows, 64 per 128-byte atom: split fp16 [hi | lo], or the
+  // fp16 / bf16 inputs unsplit
   const bool sp = a.plan.split;
-  const CUtensorMapDataType rdt = sp ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const CUtensorMapDataType rdt = (!sp && a.dt == GS_BF16) ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   const uint64_t rowe = (sp ? 2ull : 1ull) * Kp;   // elements per packed row
-  const uint64_t rowb = rowe * (sp ? 2ull : 4ull);  // bytes per packed row
-  const int atom_e = sp ? 64 : 32;
+  const uint64_t rowb = rowe * 2ull;                // bytes per packed row
+  const int atom_e = 64;
   if (!make_tmap_3d(&m.x, rdt, a.xpack, rowe, a.M, a.B, rowb, a.M * rowb, atom_e, kBM))
     return cudaErrorInvalidValue;
   const int KA = ka_for(a.plan.atoms);
@@ -1157,7 +1155,8 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
     kp.c0 = c0;
     kp.cw = cw;
     kp.cols_per_split = a.plan.cols_per_split;
-    kp.ksteps = sp ? Kp / 16 : Kp / 8;
+    kp.ksteps = Kp / 16;
+    kp.afmt = a.dt == GS_BF16 ? 1 : 0;
     kp.atoms = a.plan.atoms;
     kp.Bsz = static_cast<int>(a.B);
     kp.bn = BN;

@@ -238,7 +238,9 @@ def test_lse_f32_tensor_core_shapes(shape, tau):
 @pytest.mark.parametrize("dtype,shape,tau", [("f16", (1, 300, 700, 3, 1), 30.0),
                                              ("bf16", (2, 200, 500, 32, 2), 1.0),
                                              ("f16", (1, 130, 1000, 100, 1), 1.0),
-                                             ("f16", (1, 257, 900, 128, 3), 2.0)])
+                                             ("f16", (1, 257, 900, 128, 3), 2.0),
+                                             ("bf16", (1, 190, 640, 17, 1), 4.0),
+                                             ("f16", (3, 100, 333, 16, 2), 1.0)])
 def test_lse_half_precision_shapes(dtype, shape, tau):
     """fp16 / bf16 log-sum-exp: exact tf32 operands on the tensor-core path."""
     B, M, N, D, C = shape
