@@ -200,11 +200,14 @@ def step_fn(gs, w, d, ws, outs):
     tau = d["tau"]
     ops = w.ops
 
-    def run():
+    def run(mid=None):
         if "sum" in ops and "bwd" in ops:
             # forward that keeps the x-gradient sums, then the backward from them
+            # (mid: an event recorded between the two, for the per-part times)
             gs.gauss_sum_fwd_saved(d["x"], d["y"], d["w"], tau, out=outs["sum"],
                                    saved=outs["saved"], workspace=ws)
+            if mid is not None:
+                mid.record()
             gs.gauss_sum_bwd_saved(d["x"], d["y"], d["w"], d["g"], outs["saved"], tau, workspace=ws)
         elif "sum" in ops:
             gs.gauss_sum_fwd(d["x"], d["y"], d["w"], tau, out=outs["sum"], workspace=ws)
@@ -378,6 +381,8 @@ def main():
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    two_part = (not args.sharded) and "sum" in w.ops and "bwd" in w.ops
+    mids = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)] if two_part else None
     clk_path = (args.clock_log.replace(".csv", f"_rank{rank}.csv") if args.clock_log
                 else os.path.join(tempfile.gettempdir(), f"gs_clocks_{rank}.csv"))
     clk = ClockSampler(local, clk_path)
@@ -388,12 +393,23 @@ def main():
         for k in range(args.steps):
             flush.fill_(float(k))
             starts[k].record(stream)
-            run()
+            if two_part:
+                run(mids[k])
+            else:
+                run()
             ends[k].record(stream)
         torch.cuda.synchronize()
         time.sleep(0.2)
     barrier(pg)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    parts = None
+    if two_part:
+        # forward (keeping the x-gradient sums) and backward, each against B M N pairs
+        f_ms = statistics.median(s.elapsed_time(m) for s, m in zip(starts, mids))
+        b_ms = statistics.median(m.elapsed_time(e) for m, e in zip(mids, ends))
+        parts = {"fwd_saved_ms": f_ms, "bwd_saved_ms": b_ms,
+                 "fwd_g_pairs_s": w.pairs / (f_ms * 1e-3) / 1e9,
+                 "bwd_g_pairs_s": w.pairs / (b_ms * 1e-3) / 1e9}
     total_ms = max_over_ranks(sum(step_ms), pg, dev)
     ms_per_step = total_ms / args.steps
     evals = pairs_per_step(w)   # one problem's pairs per step
@@ -507,6 +523,8 @@ def main():
                         "two streams: step k+1's copies overlap step k's pair work"},
                 "gpu_launches": (n_launch * args.steps) if n_launch is not None else None, "kernels": kernel_names,
                 "clocks": clocks}
+        if parts is not None:
+            line["parts"] = parts   # rank 0's medians
         print(json.dumps(line), flush=True)
     if pg is not None:
         pg.destroy_process_group()
