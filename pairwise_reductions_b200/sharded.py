@@ -9,13 +9,21 @@ The gradient adds one more exchange: dL/dx of the local rows needs (y, w) as
 above, while dL/dw and dL/dy of the local sources need every row and its
 upstream gradient, i.e. an all-gather of (x, g).
 
+The log-sum-exp backward shards the same way: dL/dx of the local rows (and
+their share of dL/dtau) against the gathered (y, w); dL/dy and dL/dw of the
+local sources against the gathered (x, g, lse) -- the backward takes the
+forward's lse of every row as an input, so a pass over a subset of the sources
+still normalises by the full sum --; the dL/dtau shares are summed over the
+ranks.
+
 The exchanges are `torch.distributed` collectives on the group's backend (NCCL
 over NVLink for CUDA tensors); the pair work runs in this library's kernels
-(`gauss_sum_fwd`, `gauss_lse_fwd`, `gauss_sum_bwd`).  Shards may differ in
-size; they are concatenated in rank order.
+(`gauss_sum_fwd`, `gauss_lse_fwd`, `gauss_sum_bwd`, `gauss_lse_bwd`).  Shards
+may differ in size; they are concatenated in rank order.  Every rank makes the
+same calls with the same `want`, so the collectives match.
 
-`kernels` replaces the three compute calls (same signatures); the default is
-the CUDA library.  `row_counts` / `src_counts` (every rank's number of rows /
+`kernels` replaces the compute calls (same signatures); the default is the
+CUDA library.  `row_counts` / `src_counts` (every rank's number of rows /
 sources, from `shard_counts`) spare each gather the exchange of the counts and
 its host synchronisation; without them the counts are exchanged every call.
 """
@@ -24,8 +32,9 @@ import torch.distributed as dist
 
 
 def _default_kernels():
-    from . import gauss_lse_fwd, gauss_sum_bwd, gauss_sum_fwd
-    return {"sum": gauss_sum_fwd, "lse": gauss_lse_fwd, "bwd": gauss_sum_bwd}
+    from . import gauss_lse_bwd, gauss_lse_fwd, gauss_sum_bwd, gauss_sum_fwd
+    return {"sum": gauss_sum_fwd, "lse": gauss_lse_fwd, "bwd": gauss_sum_bwd,
+            "lse_bwd": gauss_lse_bwd}
 
 
 def shard_counts(n_local, device, group=None):
@@ -95,5 +104,34 @@ def sharded_sum_bwd(x, y, w, g, tau, group=None, kernels=None, row_counts=None, 
     return gx, gw
 
 
+def sharded_lse_bwd(x, y, w, lse, g, tau, group=None, kernels=None, row_counts=None,
+                    src_counts=None, want=("x", "y", "w", "tau")):
+    """Gradients of L = <g, lse> with lse = the log-sum-exp over every rank's sources:
+    a dict with the requested keys -- x for this rank's rows, y and w for this rank's
+    sources, tau (summed over the ranks).  lse and g are this rank's rows."""
+    k = kernels or _default_kernels()
+    out = {}
+    row_side = tuple(n for n in ("x", "tau") if n in want)
+    src_side = tuple(n for n in ("y", "w") if n in want)
+    if row_side:
+        if src_counts is None:
+            src_counts = shard_counts(y.shape[1], y.device, group)
+        r = k["lse_bwd"](x, all_gather_rows(y, group, src_counts), all_gather_rows(w, group, src_counts),
+                         lse, g, tau, want=row_side)
+        out.update(r)
+    if src_side:
+        if row_counts is None:
+            row_counts = shard_counts(x.shape[1], x.device, group)
+        r = k["lse_bwd"](all_gather_rows(x, group, row_counts), y, w,
+                         all_gather_rows(lse, group, row_counts), all_gather_rows(g, group, row_counts),
+                         tau, want=src_side)
+        out.update(r)
+    if "tau" in out:
+        t = out["tau"].clone()
+        dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+        out["tau"] = t
+    return out
+
+
 __all__ = ["shard_counts", "all_gather_rows", "sharded_sum_fwd", "sharded_lse_fwd",
-           "sharded_sum_bwd"]
+           "sharded_sum_bwd", "sharded_lse_bwd"]

@@ -49,7 +49,26 @@ def _oracle_kernels():
         return (t(gx) if want_x else None), (t(gw) if want_w else None)
     return {"sum": lambda x, y, w, tau: t(oracle.gauss_sum(n(x), n(y), n(w), tau)),
             "lse": lambda x, y, w, tau: t(oracle.gauss_lse(n(x), n(y), n(w), tau)),
-            "bwd": bwd}
+            "bwd": bwd, "lse_bwd": _lse_bwd_given_lse}
+
+
+def _lse_bwd_given_lse(x, y, w, lse, g, tau, want=("x", "y", "w", "tau")):
+    """Gradients of <g, lse> for the given sources, normalised by the given lse
+    (dense float64 from the definition: p_ijc = w_jc K_ij exp(-lse_ic))."""
+    d2 = ((x[:, :, None, :] - y[:, None, :, :]) ** 2).sum(-1)            # [B, M, N]
+    K = torch.exp(-0.5 * tau * d2)
+    p = w[:, None, :, :] * K[..., None] * torch.exp(-lse)[:, :, None, :]  # [B, M, N, C]
+    gp = (g[:, :, None, :] * p).sum(-1)                                  # sum_c g_ic p_ijc
+    out = {}
+    if "x" in want:
+        out["x"] = -tau * (x * gp.sum(2)[..., None] - gp @ y)
+    if "y" in want:
+        out["y"] = tau * (gp.transpose(1, 2) @ x - y * gp.sum(1)[..., None])
+    if "w" in want:
+        out["w"] = ((g * torch.exp(-lse))[:, :, None, :] * K[..., None]).sum(1)
+    if "tau" in want:
+        out["tau"] = (-0.5 * gp * d2).sum().reshape(1)
+    return out
 
 
 def _worker(rank, world, port, q):
@@ -70,6 +89,8 @@ def _worker(rank, world, port, q):
         "lse": sharded.sharded_lse_fwd(xs, ys, ws, TAU, kernels=k),
     }
     out["gx"], out["gw"] = sharded.sharded_sum_bwd(xs, ys, ws, gs_, TAU, kernels=k)
+    lg = sharded.sharded_lse_bwd(xs, ys, ws, out["lse"], gs_, TAU, kernels=k)
+    out.update({"lse_g" + kk: v for kk, v in lg.items()})
     q.put((rank, {kk: v.numpy() for kk, v in out.items()}))
     dist.destroy_process_group()
 
@@ -91,6 +112,7 @@ def test_sharded_problem_matches_the_whole_problem_gloo():
     s = oracle.gauss_sum(x, y, w, TAU)
     lse = oracle.gauss_lse(x, y, w, TAU)
     gx, gw = oracle.gauss_sum_bwd(x, y, w, g, TAU)
+    lgx, lgy, lgw, lgt = oracle.gauss_lse_bwd(x, y, w, g, TAU)
     for rank in range(world):
         r0, s0 = sum(ROWS[:rank]), sum(SRCS[:rank])
         rows, srcs = slice(r0, r0 + ROWS[rank]), slice(s0, s0 + SRCS[rank])
@@ -100,6 +122,12 @@ def test_sharded_problem_matches_the_whole_problem_gloo():
         np.testing.assert_allclose(o["lse"], lse[:, rows], rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(o["gx"], gx[:, rows], rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(o["gw"], gw[:, srcs], rtol=1e-12, atol=1e-12)
+        # log-sum-exp backward: x of the local rows, y and w of the local sources,
+        # tau summed over the ranks
+        np.testing.assert_allclose(o["lse_gx"], lgx[:, rows], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(o["lse_gy"], lgy[:, srcs], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(o["lse_gw"], lgw[:, srcs], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(o["lse_gtau"], [lgt], rtol=1e-10)
 
 
 def _gpu_worker(port, q):
@@ -114,8 +142,12 @@ def _gpu_worker(port, q):
     b = m.gauss_sum_fwd(x, y, w, TAU)
     gx, gw = sharded.sharded_sum_bwd(x, y, w, g, TAU)
     rx, rw = m.gauss_sum_bwd(x, y, w, g, TAU)
+    lse = m.gauss_lse_fwd(x, y, w, TAU)
+    lg = sharded.sharded_lse_bwd(x, y, w, lse, g, TAU)
+    rl = m.gauss_lse_bwd(x, y, w, lse, g, TAU)
     torch.cuda.synchronize()
-    q.put(bool(torch.equal(a, b) and torch.equal(gx, rx) and torch.equal(gw, rw)))
+    lse_ok = all(torch.allclose(lg[k], rl[k], rtol=1e-6, atol=1e-7) for k in ("x", "y", "w", "tau"))
+    q.put(bool(torch.equal(a, b) and torch.equal(gx, rx) and torch.equal(gw, rw) and lse_ok))
     dist.destroy_process_group()
 
 
