@@ -18,7 +18,8 @@ ranks.
 
 The exchanges are `torch.distributed` collectives on the group's backend (NCCL
 over NVLink for CUDA tensors); the pair work runs in this library's kernels
-(`gauss_sum_fwd`, `gauss_lse_fwd`, `gauss_sum_bwd`, `gauss_lse_bwd`).  Shards
+(`gauss_sum_fwd`, `gauss_lse_fwd`, `gauss_sum_bwd`, `gauss_sum_vjp`,
+`gauss_lse_bwd`).  Shards
 may differ in size; they are concatenated in rank order.  Every rank makes the
 same calls with the same `want`, so the collectives match.
 
@@ -32,9 +33,9 @@ import torch.distributed as dist
 
 
 def _default_kernels():
-    from . import gauss_lse_bwd, gauss_lse_fwd, gauss_sum_bwd, gauss_sum_fwd
+    from . import gauss_lse_bwd, gauss_lse_fwd, gauss_sum_bwd, gauss_sum_fwd, gauss_sum_vjp
     return {"sum": gauss_sum_fwd, "lse": gauss_lse_fwd, "bwd": gauss_sum_bwd,
-            "lse_bwd": gauss_lse_bwd}
+            "lse_bwd": gauss_lse_bwd, "vjp": gauss_sum_vjp}
 
 
 def shard_counts(n_local, device, group=None):
@@ -104,6 +105,33 @@ def sharded_sum_bwd(x, y, w, g, tau, group=None, kernels=None, row_counts=None, 
     return gx, gw
 
 
+def sharded_sum_vjp(x, y, w, g, tau, group=None, kernels=None, row_counts=None, src_counts=None,
+                    want=("x", "y", "w", "tau")):
+    """Every first-order gradient of L = <g, sum> over the whole problem: a dict with
+    the requested keys -- x for this rank's rows (and its share of tau) against the
+    gathered (y, w); y and w for this rank's sources against the gathered (x, g);
+    tau summed over the ranks."""
+    k = kernels or _default_kernels()
+    out = {}
+    row_side = tuple(n for n in ("x", "tau") if n in want)
+    src_side = tuple(n for n in ("y", "w") if n in want)
+    if row_side:
+        if src_counts is None:
+            src_counts = shard_counts(y.shape[1], y.device, group)
+        out.update(k["vjp"](x, all_gather_rows(y, group, src_counts),
+                            all_gather_rows(w, group, src_counts), g, tau, want=row_side))
+    if src_side:
+        if row_counts is None:
+            row_counts = shard_counts(x.shape[1], x.device, group)
+        out.update(k["vjp"](all_gather_rows(x, group, row_counts), y, w,
+                            all_gather_rows(g, group, row_counts), tau, want=src_side))
+    if "tau" in out:
+        t = out["tau"].clone()
+        dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+        out["tau"] = t
+    return out
+
+
 def sharded_lse_bwd(x, y, w, lse, g, tau, group=None, kernels=None, row_counts=None,
                     src_counts=None, want=("x", "y", "w", "tau")):
     """Gradients of L = <g, lse> with lse = the log-sum-exp over every rank's sources:
@@ -134,4 +162,4 @@ def sharded_lse_bwd(x, y, w, lse, g, tau, group=None, kernels=None, row_counts=N
 
 
 __all__ = ["shard_counts", "all_gather_rows", "sharded_sum_fwd", "sharded_lse_fwd",
-           "sharded_sum_bwd", "sharded_lse_bwd"]
+           "sharded_sum_bwd", "sharded_sum_vjp", "sharded_lse_bwd"]

@@ -47,9 +47,15 @@ def _oracle_kernels():
     def bwd(x, y, w, g, tau, want_x=True, want_w=True):
         gx, gw = oracle.gauss_sum_bwd(n(x), n(y), n(w), n(g), tau)
         return (t(gx) if want_x else None), (t(gw) if want_w else None)
+
+    def vjp(x, y, w, g, tau, want=("x", "y", "w", "tau")):
+        gx, gw = oracle.gauss_sum_bwd(n(x), n(y), n(w), n(g), tau)
+        gy, gt = oracle.gauss_sum_vjp_y_tau(n(x), n(y), n(w), n(g), tau)
+        full = {"x": t(gx), "y": t(gy), "w": t(gw), "tau": torch.tensor([gt], dtype=torch.float64)}
+        return {kk: full[kk] for kk in want}
     return {"sum": lambda x, y, w, tau: t(oracle.gauss_sum(n(x), n(y), n(w), tau)),
             "lse": lambda x, y, w, tau: t(oracle.gauss_lse(n(x), n(y), n(w), tau)),
-            "bwd": bwd, "lse_bwd": _lse_bwd_given_lse}
+            "bwd": bwd, "lse_bwd": _lse_bwd_given_lse, "vjp": vjp}
 
 
 def _lse_bwd_given_lse(x, y, w, lse, g, tau, want=("x", "y", "w", "tau")):
@@ -90,6 +96,8 @@ def _worker(rank, world, port, q):
     }
     out["gx"], out["gw"] = sharded.sharded_sum_bwd(xs, ys, ws, gs_, TAU, kernels=k)
     lg = sharded.sharded_lse_bwd(xs, ys, ws, out["lse"], gs_, TAU, kernels=k)
+    vg = sharded.sharded_sum_vjp(xs, ys, ws, gs_, TAU, kernels=k)
+    out.update({"vjp_g" + kk: v for kk, v in vg.items()})
     out.update({"lse_g" + kk: v for kk, v in lg.items()})
     q.put((rank, {kk: v.numpy() for kk, v in out.items()}))
     dist.destroy_process_group()
@@ -113,6 +121,7 @@ def test_sharded_problem_matches_the_whole_problem_gloo():
     lse = oracle.gauss_lse(x, y, w, TAU)
     gx, gw = oracle.gauss_sum_bwd(x, y, w, g, TAU)
     lgx, lgy, lgw, lgt = oracle.gauss_lse_bwd(x, y, w, g, TAU)
+    vgy, vgt = oracle.gauss_sum_vjp_y_tau(x, y, w, g, TAU)
     for rank in range(world):
         r0, s0 = sum(ROWS[:rank]), sum(SRCS[:rank])
         rows, srcs = slice(r0, r0 + ROWS[rank]), slice(s0, s0 + SRCS[rank])
@@ -128,6 +137,11 @@ def test_sharded_problem_matches_the_whole_problem_gloo():
         np.testing.assert_allclose(o["lse_gy"], lgy[:, srcs], rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(o["lse_gw"], lgw[:, srcs], rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(o["lse_gtau"], [lgt], rtol=1e-10)
+        # every gradient of the sum: tau summed over the ranks
+        np.testing.assert_allclose(o["vjp_gx"], gx[:, rows], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(o["vjp_gy"], vgy[:, srcs], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(o["vjp_gw"], gw[:, srcs], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(o["vjp_gtau"], [vgt], rtol=1e-12)
 
 
 def _gpu_worker(port, q):
