@@ -186,3 +186,31 @@ def test_autograd_wrappers_validate_tau_before_any_launch():
         autograd.gauss_sum(x, x, torch.zeros(4, 1), torch.ones(2))
     with pytest.raises(ValueError):
         autograd.gauss_lse(x, x, torch.ones(4, 1), torch.ones(3))
+
+
+def test_binding_rejects_mismatched_tensors_before_any_call():
+    import torch
+    x = torch.zeros(2, 5, 3)
+    y = torch.zeros(2, 7, 3)
+    w = torch.zeros(2, 7, 1)
+    with pytest.raises(ValueError):           # batch sizes differ
+        gs.gauss_sum_fwd(x, torch.zeros(1, 7, 3), torch.zeros(1, 7, 1), 1.0)
+    with pytest.raises(ValueError):           # feature sizes differ
+        gs.gauss_sum_fwd(x, torch.zeros(2, 7, 4), w, 1.0)
+    with pytest.raises(ValueError):           # weights for another number of sources
+        gs.gauss_sum_fwd(x, y, torch.zeros(2, 6, 1), 1.0)
+    with pytest.raises(ValueError):           # mixed dtypes
+        gs.gauss_sum_fwd(x, y, w.double(), 1.0)
+    with pytest.raises(ValueError):           # not contiguous
+        gs.gauss_sum_fwd(torch.zeros(2, 3, 5).transpose(1, 2), y, w, 1.0)
+    with pytest.raises(ValueError):           # 1-D input
+        gs.gauss_sum_fwd(torch.zeros(5), y, w, 1.0)
+    g = torch.zeros(2, 5, 1)
+    with pytest.raises(ValueError):           # upstream gradient of the wrong shape
+        gs.gauss_sum_bwd(x, y, w, torch.zeros(2, 4, 1), 1.0)
+    with pytest.raises(ValueError):           # upstream gradient not float32
+        gs.gauss_sum_vjp(x, y, w, g.double(), 1.0)
+    with pytest.raises(ValueError):           # saved sums of the wrong width
+        gs.gauss_sum_bwd_saved(x, y, w, g, torch.zeros(2, 5, 3), 1.0)
+    with pytest.raises(ValueError):           # lse of the wrong shape
+        gs.gauss_lse_bwd(x, y, w, torch.zeros(2, 5, 2), g, 1.0)
