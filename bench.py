@@ -305,9 +305,12 @@ def reference_arm(args, w):
     if rank != 0:
         return
     inp = synth.make_inputs(w)
+    # the whole timed loop takes about --cpu-seconds: each step a row sample of at
+    # least 0.1 s of oracle work (~2e8 pairs on 16 cores), so even thousands of
+    # steps end within minutes
     per_step = args.cpu_seconds / max(args.steps, 1)
     import oracle
-    base, rows = oracle_sample(w, inp, max(per_step, 0.5))
+    base, rows = oracle_sample(w, inp, max(per_step, 0.1))
     x, y, wt = (synth.as_f64(inp[k]) for k in ("x", "y", "w"))
     g = synth.as_f64(inp["g"]) if "g" in inp else None
 
