@@ -4,9 +4,11 @@ roofline fraction of the dominant kernel and the CPU oracle as the baseline.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 One step is one pass of the whole hot path of the workload over its seeded
-synthetic inputs (already resident in HBM).  Default workload: ``d3_100k``
-(B=1, M=N=100,000, D=3, C=1, fp32, tau=1, x,y ~ N(0,1)^3, w ~ N(0,1) signed),
-the Gaussian product at 100k points of "Kernel matrix reduction" (Variants).
+synthetic inputs (already resident in HBM).  Default workload: ``d3_1m_lse``
+(B=1, M=N=1,000,000, D=3, C=1, fp32, tau=100, x,y ~ U[0,1)^3, w ~ U(0.5,1.5)):
+one step is the Gaussian kernel sum and its log-sum-exp over the same inputs,
+the largest single-GPU workload (the 1M-point Gaussian product of "Kernel
+matrix reduction", Variants, plus the log-sum-exp reduction of its Overview).
 Under torchrun (N > 1) every rank runs its own independent problem of that
 size (rank-specific query points, same sources): rows are independent, so
 there is no data-path collective, and throughput scales weakly; the time is
@@ -47,18 +49,24 @@ PUBLISHED = {  # context only: the pages' number for the same workload, another 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="d3_100k", choices=sorted(synth.BY_NAME))
+    ap.add_argument("--workload", default="d3_1m_lse", choices=sorted(synth.BY_NAME))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--e2e-single-steps", type=int, default=5,
+                    help="steps of the one-call-at-a-time end-to-end figure (one stream, no overlap)")
     ap.add_argument("--no-launch-count", action="store_true",
                     help="skip the profiler-based kernel count (use under ncu)")
     ap.add_argument("--clock-log", default=None,
                     help="CSV of the nvidia-smi clock samples (default: a file under the temp directory)")
+    ap.add_argument("--two-call", action="store_true",
+                    help="forward + backward workloads: time gauss_sum_fwd_saved then "
+                         "gauss_sum_bwd_saved (two sweeps, g not needed by the forward) instead "
+                         "of the one-call gauss_sum_fwd_bwd")
     ap.add_argument("--sharded", action="store_true",
                     help="one problem of the workload's size split over the ranks by rows and "
                          "sources (strong scaling; the sources are all-gathered every step)")
@@ -195,13 +203,17 @@ def shard_of(inp, rank, world):
     return out
 
 
-def step_fn(gs, w, d, ws, outs):
+def step_fn(gs, w, d, ws, outs, two_call=False):
     """Return a closure running one pass of the workload's hot path."""
     tau = d["tau"]
     ops = w.ops
 
     def run(mid=None):
-        if "sum" in ops and "bwd" in ops:
+        if "sum" in ops and "bwd" in ops and not two_call:
+            # forward and backward in one call (g given up front)
+            gs.gauss_sum_fwd_bwd(d["x"], d["y"], d["w"], d["g"], tau, out=outs["sum"],
+                                 grad_x=outs["gx"], grad_w=outs["gw"], workspace=ws)
+        elif "sum" in ops and "bwd" in ops:
             # forward that keeps the x-gradient sums, then the backward from them
             # (mid: an event recorded between the two, for the per-part times)
             gs.gauss_sum_fwd_saved(d["x"], d["y"], d["w"], tau, out=outs["sum"],
@@ -226,10 +238,20 @@ def pairs_per_step(w):
     return per * (("sum" in w.ops or "bwd" in w.ops) + ("lse" in w.ops))
 
 
-def kernel_evals_per_step(w):
-    """Kernel evaluations (exponentials) one step performs: one pass per sum or
-    log-sum-exp; the forward + backward step runs two (the forward that keeps the
-    x-gradient sums, and the grad_w pass)."""
+def fused_fwd_bwd(w):
+    """Whether gauss_sum_fwd_bwd evaluates each kernel value once for this
+    workload (fp16 / bf16, C = 1, D <= 47); else it runs two sweeps."""
+    return w.dtype != "f32" and w.C == 1 and w.D <= 47
+
+
+def kernel_evals_per_step(w, two_call=False):
+    """Kernel evaluations (exponentials) one step performs: one sweep per sum or
+    log-sum-exp; the forward + backward step runs one sweep in one call where it
+    fuses, else two (the forward that keeps the x-gradient sums, and the
+    grad_w pass)."""
+    if "sum" in w.ops and "bwd" in w.ops:
+        return w.pairs * (1 if (fused_fwd_bwd(w) and not two_call) else 2) + \
+            w.pairs * ("lse" in w.ops)
     return w.pairs * (("sum" in w.ops) + ("lse" in w.ops) + ("bwd" in w.ops))
 
 
@@ -363,15 +385,18 @@ def main():
     outs = {"sum": torch.empty(w.B, w.M, w.C, device=dev), "lse": torch.empty(w.B, w.M, w.C, device=dev)}
     if "bwd" in w.ops:
         outs["saved"] = torch.empty(w.B, w.M, w.C * (1 + w.D), device=dev)
+        outs["gx"] = torch.empty(w.B, w.M, w.D, device=dev)
+        outs["gw"] = torch.empty(w.B, w.N, w.C, device=dev)
     ws_bytes = max(gs.workspace_bytes(op, w.B, w.M, w.N, w.D, w.C, d["x"].dtype)
-                   for op, name in ((gs.GS_OP_SUM, "sum"), (gs.GS_OP_LSE, "lse"), (gs.GS_OP_SUM_BWD, "bwd"))
+                   for op, name in ((gs.GS_OP_SUM, "sum"), (gs.GS_OP_LSE, "lse"), (gs.GS_OP_SUM_BWD, "bwd"),
+                                    (gs.GS_OP_SUM_FWD_BWD, "bwd"))
                    if name in w.ops)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     counts = None
     if args.sharded:
         from pairwise_reductions_b200 import sharded
         counts = (sharded.shard_counts(d["x"].shape[1], dev), sharded.shard_counts(d["y"].shape[1], dev))
-    run = sharded_step_fn(w, d, counts) if args.sharded else step_fn(gs, w, d, ws, outs)
+    run = sharded_step_fn(w, d, counts) if args.sharded else step_fn(gs, w, d, ws, outs, args.two_call)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -384,7 +409,7 @@ def main():
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    two_part = (not args.sharded) and "sum" in w.ops and "bwd" in w.ops
+    two_part = (not args.sharded) and "sum" in w.ops and "bwd" in w.ops and args.two_call
     mids = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)] if two_part else None
     clk_path = (args.clock_log.replace(".csv", f"_rank{rank}.csv") if args.clock_log
                 else os.path.join(tempfile.gettempdir(), f"gs_clocks_{rank}.csv"))
@@ -416,7 +441,7 @@ def main():
     total_ms = max_over_ranks(sum(step_ms), pg, dev)
     ms_per_step = total_ms / args.steps
     evals = pairs_per_step(w)   # one problem's pairs per step
-    kevals = kernel_evals_per_step(w)
+    kevals = kernel_evals_per_step(w, args.two_call or args.sharded)
     jobs = 1 if args.sharded else world   # problems the whole job solves per step
     value = evals * jobs * args.steps / (total_ms * 1e-3) / 1e9
     if gs.last_device_error() != 0:
@@ -424,9 +449,16 @@ def main():
 
     # ---- end to end through the public API: pinned host inputs -> device -> result -> host
     hx = {k: inp[k].pin_memory() for k in ("x", "y", "w", "g") if k in inp}
-    hout = torch.empty(w.B, inp["x"].shape[1], w.C).pin_memory()
+    # the step's results read back: the sum (or the log-sum-exp), and for the
+    # one-call forward + backward step its two gradients too
+    res_keys = ["lse" if "lse" in w.ops and "sum" not in w.ops else "sum"]
+    if "bwd" in w.ops and not args.two_call and not args.sharded:
+        res_keys += ["gx", "gw"]
+    hres = {k: torch.empty(outs[k].shape).pin_memory() for k in res_keys[1:]}
+    hres[res_keys[0]] = torch.empty(w.B, inp["x"].shape[1], w.C).pin_memory()   # this rank's rows
+    hout = hres[res_keys[0]]
     h2d = sum(t.numel() * t.element_size() for t in hx.values())
-    d2h = hout.numel() * hout.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in hres.values())
     e_s = torch.cuda.Event(enable_timing=True)
     e_e = torch.cuda.Event(enable_timing=True)
 
@@ -438,8 +470,9 @@ def main():
             hout.copy_(dd["out_lse" if "lse" in w.ops and "sum" not in w.ops else "out_sum"],
                        non_blocking=True)
         else:
-            step_fn(gs, w, dd, ws, outs)()
-            hout.copy_(outs["lse" if "lse" in w.ops and "sum" not in w.ops else "sum"], non_blocking=True)
+            step_fn(gs, w, dd, ws, outs, args.two_call)()
+            for k in res_keys:
+                hres[k].copy_(outs[k], non_blocking=True)
 
     # Independent problems: two lanes, each with its own stream, device buffers,
     # workspace and pinned result buffer; step k runs on lane k % 2, so the
@@ -452,7 +485,7 @@ def main():
                   "d": {k: torch.empty_like(t, device=dev) for k, t in hx.items()},
                   "outs": {k: torch.empty_like(v) for k, v in outs.items()},
                   "ws": torch.empty_like(ws),
-                  "hout": torch.empty_like(hout).pin_memory()}
+                  "hres": {k: torch.empty_like(t).pin_memory() for k, t in hres.items()}}
             ln["d"]["tau"] = inp["tau"]
             lanes.append(ln)
 
@@ -460,9 +493,9 @@ def main():
         with torch.cuda.stream(ln["stream"]):
             for k, t in hx.items():
                 ln["d"][k].copy_(t, non_blocking=True)
-            step_fn(gs, w, ln["d"], ln["ws"], ln["outs"])()
-            ln["hout"].copy_(ln["outs"]["lse" if "lse" in w.ops and "sum" not in w.ops else "sum"],
-                             non_blocking=True)
+            step_fn(gs, w, ln["d"], ln["ws"], ln["outs"], args.two_call)()
+            for k in res_keys:
+                ln["hres"][k].copy_(ln["outs"][k], non_blocking=True)
 
     e2e_ms, e2e_value = None, None
     if args.e2e_steps > 0:
@@ -481,6 +514,26 @@ def main():
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e_s.elapsed_time(e_e), pg, dev) / args.e2e_steps
         e2e_value = evals * jobs / (e2e_ms * 1e-3) / 1e9
+    # One call at a time on one stream: copies in, the step, the result out,
+    # each step between its own start and end events (the latency one call sees).
+    single = None
+    if args.e2e_single_steps > 0 and not args.sharded:
+        ln = lanes[0]
+        e2e_lane_step(ln)
+        torch.cuda.synchronize()
+        barrier(pg)
+        one = []
+        for _ in range(args.e2e_single_steps):
+            a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(ln["stream"])
+            e2e_lane_step(ln)
+            z.record(ln["stream"])
+            ln["stream"].synchronize()
+            one.append(a.elapsed_time(z))
+        single_ms = max_over_ranks(statistics.median(one), pg, dev)
+        single = {"value": evals * jobs / (single_ms * 1e-3) / 1e9, "ms_per_step": single_ms,
+                  "steps": args.e2e_single_steps,
+                  "pipelining": "none: one stream, each call finished before the next starts"}
     clocks = clk.summary()
 
     if rank == 0:
@@ -523,7 +576,8 @@ def main():
                 "e2e": {"value": e2e_value, "unit": "G pairs/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                         "pipelining": "none (sharded)" if args.sharded else
-                        "two streams: step k+1's copies overlap step k's pair work"},
+                        "two streams: step k+1's copies overlap step k's pair work",
+                        "single_call": single},
                 "gpu_launches": (n_launch * args.steps) if n_launch is not None else None, "kernels": kernel_names,
                 "clocks": clocks}
         if parts is not None:

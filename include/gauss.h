@@ -76,7 +76,9 @@ typedef enum {
     GS_OP_SUM_BWD = 2,
     GS_OP_LSE_BWD = 3,
     GS_OP_KNN = 4,      /* gs_workspace_bytes: pass K as C */
-    GS_OP_DIFFUSION = 5 /* gs_workspace_bytes: M = N, C = columns of V (1 for the scales) */
+    GS_OP_DIFFUSION = 5, /* gs_workspace_bytes: M = N, C = columns of V (1 for the scales) */
+    GS_OP_SUM_FWD_BWD = 6,
+    GS_OP_DIFFUSION_BLOCK = 7
 } gs_op;
 
 typedef enum {
@@ -158,6 +160,28 @@ gs_status gauss_sum_bwd_saved(const void *x, const void *y, const void *w, const
                               const float *saved, float *grad_x, float *grad_w, int64_t B,
                               int64_t M, int64_t N, int64_t D, int64_t C, float tau, gs_dtype dt,
                               void *ws, size_t ws_bytes, gs_stream_t stream);
+
+/*
+ * Forward and backward in one call, for an upstream gradient g [B, M, C]
+ * (float32) known before the forward (a loss linear in the output, or a
+ * cotangent fixed in advance): out = gauss_sum_fwd(x, y, w) and, of
+ * L = sum g * out, grad_x [B, M, D] and grad_w [B, N, C] exactly as
+ * gauss_sum_bwd defines them ("Kernel matrix reduction", Variants: the
+ * gradient is the same fused reduction, its tiles recomputed).  With fp16 /
+ * bf16 inputs, C = 1 and D <= 47 every kernel value is computed once: one
+ * tensor-core sweep forms the forward sum, the x-gradient sums of
+ * gauss_sum_fwd_saved and the column sums grad_w = sum_i K_ij g_i together
+ * (g enters the tensor cores as fp16 hi + lo parts under a per-batch power of
+ * two, ~22 significant bits; grad_w is then a fixed-order sum of per-128-row-
+ * tile partials).  Otherwise the call runs gauss_sum_fwd_saved's pass and
+ * gauss_sum_bwd_saved's.  `out` must not be NULL; grad_x and grad_w may be
+ * NULL (without grad_w there is nothing to fuse).  Workspace:
+ * gs_workspace_bytes(GS_OP_SUM_FWD_BWD, ...); errors as gauss_sum_fwd.
+ */
+gs_status gauss_sum_fwd_bwd(const void *x, const void *y, const void *w, const float *g, float *out,
+                            float *grad_x, float *grad_w, int64_t B, int64_t M, int64_t N,
+                            int64_t D, int64_t C, float tau, gs_dtype dt, void *ws,
+                            size_t ws_bytes, gs_stream_t stream);
 
 /*
  * Gradient of L = sum_{b,i,c} g[b,i,c] * out[b,i,c] for the Gaussian kernel sum
@@ -258,6 +282,20 @@ gs_status gauss_knn(const void *x, const void *y, float *out_sqdist, int64_t *ou
  * gauss_sum_fwd).  Workspace: gs_workspace_bytes(GS_OP_DIFFUSION, B, N, N, D, C, dt)
  * with C = 1 for the scales.
  */
+/*
+ * The kernel application those passes are made of, between a block of rows and
+ * a set of columns of the point set:
+ *     out[b,i,c] = sum_j exp(-tau/2 |x_rows[b,i] - x_cols[b,j]|^2) v[b,j,c]
+ * x_rows [B, M, D] and x_cols [B, N, D] of dtype dt, v [B, N, C] and out
+ * [B, M, C] float32 whatever dt (the Gauss sum with float32 values).  With the
+ * rows of one rank and the columns of every rank it gives that rank's rows of
+ * q = K 1, of K q^-alpha and of K (s v): "FlashDiffusion" (section 3) runs its
+ * operator sharded over rows this way.  Workspace:
+ * gs_workspace_bytes(GS_OP_DIFFUSION_BLOCK, B, M, N, D, C, dt).
+ */
+gs_status gauss_diffusion_block(const void *x_rows, const void *x_cols, const float *v, float *out,
+                                int64_t B, int64_t M, int64_t N, int64_t D, int64_t C, float tau,
+                                gs_dtype dt, void *ws, size_t ws_bytes, gs_stream_t stream);
 gs_status gauss_diffusion_scales(const void *x, float *q_out, float *d_out, float *s_out,
                                  int64_t B, int64_t N, int64_t D, float tau, float alpha,
                                  gs_dtype dt, void *ws, size_t ws_bytes, gs_stream_t stream);

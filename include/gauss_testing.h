@@ -22,6 +22,36 @@ extern "C" {
  */
 gs_status gs_test_exp2_poly(const float *x, float *out, int64_t n, int degree, gs_stream_t stream);
 
+/*
+ * The limit of the tensor-core kernels' bounded mbarrier waits (default
+ * 2e9 ns) and a stall mode that makes those waits run out on purpose, so that
+ * the abort path can be tested without a fault:
+ *   stall 0  normal operation;
+ *   stall 1  the MMA-issuing thread issues nothing: the TMA producer fills its
+ *            stages and the exp warps wait for similarity tiles that never come;
+ *   stall 2  the exp warps skip their loops: the issuer's first MMAs run, then
+ *            it waits for exponentials that never come.
+ * A kernel whose wait runs out raises the device error word (read and cleared
+ * by gs_last_device_error, which then returns GS_ERR_TIMEOUT); its other warps
+ * leave their loops; the producer waits (bounded) for the loads it issued and
+ * the issuer for the MMAs it issued before TMEM is freed and the CTA exits.
+ * Outputs of a call made in a stall mode are unspecified.  limit_ns must lie in
+ * [1e3, 1e10] and stall in {0, 1, 2}, else GS_ERR_INVALID_ARG.  The setting is
+ * per process and per device (the current one), synchronous, and applies to
+ * launches made after it returns; restore (2000000000, 0) when done.
+ */
+gs_status gs_test_set_waits(uint64_t limit_ns, int stall);
+
+/*
+ * Synchronises `stream`, then reads and clears the raw device error word of the
+ * tensor-core kernels into *word: bit 0 (1) a bounded wait ran out; bit 1 (2)
+ * an fp32 kernel was launched with tensor-map boxes made for another
+ * instantiation (it returned at once); bit 2 (4) a wait for work already issued
+ * (the drain after an abort) ran out.  GS_ERR_INVALID_ARG for a NULL word,
+ * GS_ERR_CUDA if the synchronisation or the read fails.
+ */
+gs_status gs_test_read_error_word(int *word, gs_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,6 +24,7 @@ LIB_PATH = _build.LIB
 
 GS_F32, GS_F16, GS_BF16 = 0, 1, 2
 GS_OP_SUM, GS_OP_LSE, GS_OP_SUM_BWD, GS_OP_LSE_BWD, GS_OP_KNN, GS_OP_DIFFUSION = 0, 1, 2, 3, 4, 5
+GS_OP_SUM_FWD_BWD, GS_OP_DIFFUSION_BLOCK = 6, 7
 STATUS = {0: "GS_OK", 1: "GS_ERR_INVALID_ARG", 2: "GS_ERR_UNSUPPORTED", 3: "GS_ERR_ALIGNMENT",
           4: "GS_ERR_WORKSPACE", 5: "GS_ERR_TIMEOUT", 6: "GS_ERR_CUDA"}
 _DT = {torch.float32: GS_F32, torch.float16: GS_F16, torch.bfloat16: GS_BF16}
@@ -55,7 +56,13 @@ SIGNATURES = {
     "gs_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "gs_last_device_error": (ctypes.c_int, [_vp]),
     "gs_version": (ctypes.c_int, []),
+    "gauss_sum_fwd_bwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                                         _i64, _f, ctypes.c_int, _vp, _sz, _vp]),
+    "gauss_diffusion_block": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _f,
+                                             ctypes.c_int, _vp, _sz, _vp]),
     "gs_test_exp2_poly": (ctypes.c_int, [_vp, _vp, _i64, ctypes.c_int, _vp]),
+    "gs_test_set_waits": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_int]),
+    "gs_test_read_error_word": (ctypes.c_int, [_vp, _vp]),
     "gauss_sum_fwd_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _f,
                                              ctypes.c_int, _vp]),
 }
@@ -235,6 +242,33 @@ def gauss_sum_bwd_saved(x, y, w, g, saved, tau, want_x=True, want_w=True, worksp
     return gx, gw
 
 
+def gauss_sum_fwd_bwd(x, y, w, g, tau, want_x=True, want_w=True, out=None, grad_x=None,
+                      grad_w=None, workspace=None, stream=None):
+    """Forward sum and the gradients of sum(g * out) in one call, for an upstream
+    gradient g known in advance: returns (out, grad_x, grad_w) (None where not
+    wanted).  fp16 / bf16 with C = 1 and D <= 47 evaluates each kernel value once."""
+    x, y, w, g = _as3(x, "x"), _as3(y, "y"), _as3(w, "w"), _as3(g, "g")
+    B, M, N, D, C = _dims(x, y, w)
+    if g.shape != (B, M, C) or g.dtype != torch.float32:
+        raise ValueError(f"g must be float32 of shape {(B, M, C)}")
+    if out is None:
+        out = torch.empty((B, M, C), dtype=torch.float32, device=x.device)
+    if want_x and grad_x is None:
+        grad_x = torch.empty((B, M, D), dtype=torch.float32, device=x.device)
+    if want_w and grad_w is None:
+        grad_w = torch.empty((B, N, C), dtype=torch.float32, device=x.device)
+    gx = grad_x if want_x else None
+    gw = grad_w if want_w else None
+    nbytes = workspace_bytes(GS_OP_SUM_FWD_BWD, B, M, N, D, C, x.dtype)
+    ws = _workspace(nbytes, x.device, workspace)
+    st = _lib.gauss_sum_fwd_bwd(_ptr(x), _ptr(y), _ptr(w), _ptr(g), _ptr(out),
+                                _ptr(gx) if want_x else None, _ptr(gw) if want_w else None,
+                                B, M, N, D, C, float(tau), _DT[x.dtype], _ptr(ws),
+                                nbytes if ws is not None else 0, _stream(stream))
+    _check("gauss_sum_fwd_bwd", st)
+    return out, gx, gw
+
+
 def gauss_sum_vjp(x, y, w, g, tau, want=("x", "y", "w", "tau"), workspace=None, stream=None):
     """Every first-order gradient of sum(g * gauss_sum_fwd(x, y, w, tau)):
     returns a dict with the requested keys among x, y, w, tau."""
@@ -298,6 +332,26 @@ def gauss_knn(x, y, K, workspace=None, stream=None):
     return od, oi
 
 
+def gauss_diffusion_block(x_rows, x_cols, v, tau, out=None, workspace=None, stream=None):
+    """K(x_rows, x_cols) v with float32 values v [B, N, C] whatever the points' dtype."""
+    xr, xc, v = _as3(x_rows, "x_rows"), _as3(x_cols, "x_cols"), _as3(v, "v")
+    B, M, D = xr.shape
+    N, C = xc.shape[1], v.shape[2]
+    if (xc.shape[0] != B or xc.shape[2] != D or xc.dtype != xr.dtype or v.shape[:2] != (B, N)
+            or v.dtype != torch.float32):
+        raise ValueError(f"shape/dtype mismatch x_rows{tuple(xr.shape)} x_cols{tuple(xc.shape)} "
+                         f"v{tuple(v.shape)}")
+    if out is None:
+        out = torch.empty((B, M, C), dtype=torch.float32, device=xr.device)
+    nbytes = workspace_bytes(GS_OP_DIFFUSION_BLOCK, B, M, N, D, C, xr.dtype)
+    ws = _workspace(nbytes, xr.device, workspace)
+    st = _lib.gauss_diffusion_block(_ptr(xr), _ptr(xc), _ptr(v), _ptr(out), B, M, N, D, C, float(tau),
+                                    _DT[xr.dtype], _ptr(ws), nbytes if ws is not None else 0,
+                                    _stream(stream))
+    _check("gauss_diffusion_block", st)
+    return out
+
+
 def gauss_diffusion_scales(x, tau, alpha, workspace=None, stream=None):
     """(q, d, s) of the alpha-normalised diffusion operator over the point set x."""
     x = _as3(x, "x")
@@ -338,12 +392,28 @@ def test_exp2_poly(x, degree, stream=None):
     return out
 
 
+def test_set_waits(limit_ns, stall):
+    """Wait limit and stall mode of the tensor-core kernels (test hook, see
+    include/gauss_testing.h); restore with test_set_waits(2_000_000_000, 0)."""
+    _check("gs_test_set_waits", _lib.gs_test_set_waits(int(limit_ns), int(stall)))
+
+
+def test_read_error_word(stream=None):
+    """Synchronise, then read and clear the raw device error word (test hook,
+    see include/gauss_testing.h): bit 0 a wait ran out, bit 1 mismatched boxes,
+    bit 2 a drain wait ran out."""
+    word = ctypes.c_int(0)
+    _check("gs_test_read_error_word", _lib.gs_test_read_error_word(ctypes.byref(word),
+                                                                   _stream(stream)))
+    return word.value
+
+
 def last_device_error(stream=None):
     """Synchronise and read/clear the device error word (0 = none)."""
     return int(_lib.gs_last_device_error(_stream(stream)))
 
 
 __all__ = ["gauss_sum_fwd", "gauss_sum_fwd_noalloc", "gauss_lse_fwd", "gauss_sum_bwd",
-           "gauss_sum_fwd_saved", "gauss_sum_bwd_saved", "gauss_sum_vjp", "gauss_lse_bwd", "gauss_knn", "gauss_diffusion_scales", "gauss_diffusion_apply", "workspace_bytes",
+           "gauss_sum_fwd_saved", "gauss_sum_bwd_saved", "gauss_sum_fwd_bwd", "gauss_sum_vjp", "gauss_lse_bwd", "gauss_knn", "gauss_diffusion_block", "gauss_diffusion_scales", "gauss_diffusion_apply", "workspace_bytes",
            "last_device_error", "library", "status_string", "GaussError", "SIGNATURES",
            "LIB_PATH"]

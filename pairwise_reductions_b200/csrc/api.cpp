@@ -6,6 +6,7 @@
 #include <cstdint>
 #include <cstring>
 
+#include "gauss_testing.h"
 #include "internal.h"
 #include "values.cuh"
 
@@ -184,8 +185,21 @@ PassLayout pass_layout(const Pass& p, int sm) {
   return L;
 }
 
-// Run one pass into `out` ([B, R, CV] float32) using workspace `ws`.
-gs_status run_pass(const Pass& p, const PassLayout& L, float* out, uint8_t* ws, cudaStream_t s) {
+// The forward + backward sweep's extra outputs (tensor-core fp16/bf16 path).
+struct GwArgs {
+  const float* g;      // [B, R, g_ld], channel 0
+  int64_t g_ld;
+  uint32_t* gpack;     // [B, R]
+  float* gscale;       // [B]
+  float* gw_part;      // [ceil(R / 128), B, N]
+};
+
+// Run one pass into `out` ([B, R, CV] float32) using workspace `ws`; with
+// `gw`, the same sweep also writes the column sums sum_i K_ij g_i of every
+// 128-row tile (tensor-core fp16/bf16 path only).
+gs_status run_pass(const Pass& p, const PassLayout& L, float* out, uint8_t* ws, cudaStream_t s,
+                   const GwArgs* gw = nullptr) {
+  if (gw && L.path != kPathTcHalf) return GS_ERR_UNSUPPORTED;
   const int64_t total = p.B * p.R * p.CV;
   if (total == 0) return GS_OK;
   if (p.N == 0) {
@@ -292,6 +306,13 @@ gs_status run_pass(const Pass& p, const PassLayout& L, float* out, uint8_t* ws, 
   a.rnorm = reinterpret_cast<float*>(ws + L.off_rnorm);
   a.ypack = ws + L.off_ypack;
   a.vt = ws + L.off_vt;
+  if (gw) {
+    a.g = gw->g;
+    a.g_ld = gw->g_ld;
+    a.gpack = gw->gpack;
+    a.gscale = gw->gscale;
+    a.gw_part = gw->gw_part;
+  }
   GS_CUDA(launch_tc_sum(a, s));
   if (S > 1) GS_CUDA(launch_combine_sum(dst, S, total, out, s));
   return GS_OK;
@@ -314,6 +335,55 @@ Pass fwd_pass(const void* x, const void* y, const void* w, int64_t B, int64_t M,
   p.dt = dt;
   p.tau = tau;
   return p;
+}
+
+// Forward + backward in one call: the x-gradient pass (values [w, w (y - z)],
+// whose first C channels are the forward sum) into `saved`, and dL/dw either
+// from the same sweep (fp16 / bf16, C = 1, 1 + D <= 48: each kernel value
+// computed once) or from the separate pass rows y / columns x / values g.
+constexpr int kFusedMaxD = 47;
+
+struct FwdBwdLayout {
+  Pass px, py;
+  PassLayout lx, ly;
+  bool fused;
+  int CV;
+  int64_t RT;          // 128-row tiles of the fused sweep's dL/dw partials
+  size_t off_saved, off_gpack, off_gscale, off_gwpart, off_pass;
+  size_t total;
+};
+
+FwdBwdLayout fwd_bwd_layout(const void* x, const void* y, const void* w, const float* g, int64_t B,
+                            int64_t M, int64_t N, int64_t D, int64_t C, float tau, gs_dtype dt,
+                            int sm, bool want_w) {
+  FwdBwdLayout L{};
+  L.CV = value_channels(1, static_cast<int>(C), static_cast<int>(D));
+  L.px = fwd_pass(x, y, w, B, M, N, D, C, tau, dt);
+  L.px.vmode = 1;
+  L.px.CV = L.CV;
+  L.lx = pass_layout(L.px, sm);
+  L.fused = want_w && dt != GS_F32 && C == 1 && D <= kFusedMaxD;
+  L.RT = (M + 127) / 128;
+  size_t off = 0;
+  L.off_saved = off;
+  off = align_up(off + size_t(B) * M * L.CV * 4);
+  size_t pass = L.lx.total;
+  if (L.fused) {
+    L.off_gpack = off;
+    off = align_up(off + size_t(B) * M * 4);
+    L.off_gscale = off;
+    off = align_up(off + size_t(B) * 4);
+    L.off_gwpart = off;
+    off = align_up(off + size_t(L.RT) * B * N * 4);
+  } else if (want_w) {
+    L.py = fwd_pass(y, x, g, B, N, M, D, C, tau, dt);
+    L.py.w_is_f32 = true;
+    L.ly = pass_layout(L.py, sm);
+    if (L.ly.total > pass) pass = L.ly.total;
+  }
+  L.off_pass = off;
+  L.total = align_up(off + pass);
+  return L;
 }
 
 // Gradients = up to two passes (grad.cu): rows y / columns x with values
@@ -531,7 +601,8 @@ const char* gs_status_string(gs_status st) {
 size_t gs_workspace_bytes(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, int64_t C,
                           gs_dtype dt) {
   if (op != GS_OP_SUM && op != GS_OP_LSE && op != GS_OP_SUM_BWD && op != GS_OP_LSE_BWD &&
-      op != GS_OP_KNN && op != GS_OP_DIFFUSION)
+      op != GS_OP_KNN && op != GS_OP_DIFFUSION && op != GS_OP_SUM_FWD_BWD &&
+      op != GS_OP_DIFFUSION_BLOCK)
     return kBad;
   if (op == GS_OP_DIFFUSION) {
     // one point set: M = N; C = columns of the block V (1 for the scales)
@@ -559,6 +630,17 @@ size_t gs_workspace_bytes(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, 
     if (dt != GS_F32 || D > kSdMaxD) return lse_f32_layout(B, M, N, D, C, dt, sm).total;
     const SdPlan sp = sd_plan(B, M, N, static_cast<int>(D), C, sm, 32);
     return align_up(size_t(2) * sp.splits * B * M * C * 4);
+  }
+  if (op == GS_OP_DIFFUSION_BLOCK) {
+    if (M == 0 || N == 0) return 0;
+    Pass p = fwd_pass(nullptr, nullptr, nullptr, B, M, N, D, C, 1.f, dt);
+    p.w_is_f32 = true;
+    return pass_layout(p, sm).total;
+  }
+  if (op == GS_OP_SUM_FWD_BWD) {
+    if (M == 0 || N == 0) return 0;
+    return fwd_bwd_layout(nullptr, nullptr, nullptr, nullptr, B, M, N, D, C, 1.f, dt, sm, true)
+        .total;
   }
   if (op == GS_OP_LSE_BWD) {
     if (M == 0 || N == 0) return 0;
@@ -845,6 +927,54 @@ gs_status gauss_sum_bwd_saved(const void* x, const void* y, const void* w, const
   return GS_OK;
 }
 
+gs_status gauss_sum_fwd_bwd(const void* x, const void* y, const void* w, const float* g, float* out,
+                            float* grad_x, float* grad_w, int64_t B, int64_t M, int64_t N,
+                            int64_t D, int64_t C, float tau, gs_dtype dt, void* ws, size_t ws_bytes,
+                            gs_stream_t stream) {
+  GS_TRY(check_dims(GS_OP_SUM_FWD_BWD, B, M, N, D, C, dt));
+  GS_TRY(check_tau(tau));
+  GS_TRY(check_ptr(x, B * M * D));
+  GS_TRY(check_ptr(y, B * N * D));
+  GS_TRY(check_ptr(w, B * N * C));
+  GS_TRY(check_ptr(g, B * M * C));
+  GS_TRY(check_ptr(out, B * M * C));
+  if (grad_x) GS_TRY(check_ptr(grad_x, B * M * D));
+  if (grad_w) GS_TRY(check_ptr(grad_w, B * N * C));
+  if (B == 0) return GS_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (M == 0 || N == 0) {   // empty sums: out = 0 and every gradient vanishes
+    if (M > 0) GS_CUDA(cudaMemsetAsync(out, 0, size_t(B) * M * C * 4, s));
+    if (grad_x && M > 0) GS_CUDA(cudaMemsetAsync(grad_x, 0, size_t(B) * M * D * 4, s));
+    if (grad_w && N > 0) GS_CUDA(cudaMemsetAsync(grad_w, 0, size_t(B) * N * C * 4, s));
+    return GS_OK;
+  }
+  const FwdBwdLayout L =
+      fwd_bwd_layout(x, y, w, g, B, M, N, D, C, tau, dt, sm_count(), grad_w != nullptr);
+  if (ws_bytes < L.total) return GS_ERR_WORKSPACE;
+  GS_TRY(check_ptr(ws, 1));
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  float* saved = reinterpret_cast<float*>(wsb + L.off_saved);
+  if (L.fused) {
+    GwArgs ga{};
+    ga.g = g;
+    ga.g_ld = C;
+    ga.gpack = reinterpret_cast<uint32_t*>(wsb + L.off_gpack);
+    ga.gscale = reinterpret_cast<float*>(wsb + L.off_gscale);
+    ga.gw_part = reinterpret_cast<float*>(wsb + L.off_gwpart);
+    GS_TRY(run_pass(L.px, L.lx, saved, wsb + L.off_pass, s, &ga));
+    GS_CUDA(launch_combine_sum(ga.gw_part, static_cast<int>(L.RT), B * N, grad_w, s));
+  } else {
+    GS_TRY(run_pass(L.px, L.lx, saved, wsb + L.off_pass, s));
+    if (grad_w) GS_TRY(run_pass(L.py, L.ly, grad_w, wsb + L.off_pass, s));
+  }
+  GS_CUDA(cudaMemcpy2DAsync(out, size_t(C) * 4, saved, size_t(L.CV) * 4, size_t(C) * 4,
+                            size_t(B) * M, cudaMemcpyDeviceToDevice, s));
+  if (grad_x)
+    GS_CUDA(launch_grad_x_epilogue(x, dt, g, saved, grad_x, nullptr, B, M, static_cast<int>(D),
+                                   static_cast<int>(C), L.CV, tau, s));
+  return GS_OK;
+}
+
 gs_status gauss_lse_bwd(const void* x, const void* y, const void* w, const float* lse,
                         const float* g, float* grad_x, float* grad_y, float* grad_w,
                         float* grad_tau, int64_t B, int64_t M, int64_t N, int64_t D, int64_t C,
@@ -977,6 +1107,31 @@ gs_status gauss_knn(const void* x, const void* y, float* out_sqdist, int64_t* ou
   return GS_OK;
 }
 
+gs_status gauss_diffusion_block(const void* x_rows, const void* x_cols, const float* v, float* out,
+                                int64_t B, int64_t M, int64_t N, int64_t D, int64_t C, float tau,
+                                gs_dtype dt, void* ws, size_t ws_bytes, gs_stream_t stream) {
+  GS_TRY(check_dims(GS_OP_SUM, B, M, N, D, C, dt));
+  GS_TRY(check_tau(tau));
+  GS_TRY(check_ptr(x_rows, B * M * D));
+  GS_TRY(check_ptr(x_cols, B * N * D));
+  GS_TRY(check_ptr(v, B * N * C));
+  GS_TRY(check_ptr(out, B * M * C));
+  if (B == 0 || M == 0) return GS_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (N == 0) {
+    GS_CUDA(cudaMemsetAsync(out, 0, size_t(B) * M * C * 4, s));
+    return GS_OK;
+  }
+  Pass p = fwd_pass(x_rows, x_cols, v, B, M, N, D, C, tau, dt);
+  p.w_is_f32 = true;
+  const PassLayout L = pass_layout(p, sm_count());
+  if (L.total > 0) {
+    if (ws_bytes < L.total) return GS_ERR_WORKSPACE;
+    GS_TRY(check_ptr(ws, 1));
+  }
+  return run_pass(p, L, out, static_cast<uint8_t*>(ws), s);
+}
+
 gs_status gauss_diffusion_scales(const void* x, float* q_out, float* d_out, float* s_out,
                                  int64_t B, int64_t N, int64_t D, float tau, float alpha,
                                  gs_dtype dt, void* ws, size_t ws_bytes, gs_stream_t stream) {
@@ -1029,6 +1184,25 @@ gs_status gauss_diffusion_apply(const void* x, const float* s_scale, const float
   GS_TRY(run_pass(p, L.lp, out, wsb, s));                     // K (s V)
   GS_CUDA(launch_diffusion_elementwise(3, s_scale, out, out, nullptr, n, static_cast<int>(C), 0.f,
                                        s));                    // left scaling
+  return GS_OK;
+}
+
+gs_status gs_test_set_waits(uint64_t limit_ns, int stall) {
+  if (limit_ns < 1000 || limit_ns > 10000000000ull || stall < 0 || stall > 2)
+    return GS_ERR_INVALID_ARG;
+  if (set_test_waits(limit_ns, stall) != cudaSuccess) return GS_ERR_CUDA;
+  if (set_test_waits_f32(limit_ns, stall) != cudaSuccess) return GS_ERR_CUDA;
+  return GS_OK;
+}
+
+gs_status gs_test_read_error_word(int* word, gs_stream_t stream) {
+  if (!word) return GS_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return GS_ERR_CUDA;
+  int v = 0, v32 = 0;
+  if (read_and_clear_device_error(&v) != cudaSuccess) return GS_ERR_CUDA;
+  if (read_and_clear_device_error_f32(&v32) != cudaSuccess) return GS_ERR_CUDA;
+  *word = v | v32;
   return GS_OK;
 }
 

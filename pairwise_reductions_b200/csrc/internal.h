@@ -171,6 +171,12 @@ struct TcArgs {
   float* rnorm;        // [B, M]
   void* ypack;         // [B, N, KP]
   void* vt;            // [B, CP, Nst] f16
+  // forward + backward sweep (gw_part != nullptr): dL/dw column sums as well
+  const float* g;      // [B, M, g_ld] upstream gradient, channel 0
+  int64_t g_ld;
+  uint32_t* gpack;     // [B, M]
+  float* gscale;       // [B]
+  float* gw_part;      // [ceil(M / 128), B, N]
 };
 cudaError_t launch_tc_sum(const TcArgs& a, cudaStream_t s);
 
@@ -228,6 +234,7 @@ struct F32Args {
 };
 cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s);
 cudaError_t read_and_clear_device_error_f32(int* value);
+cudaError_t set_test_waits_f32(uint64_t limit_ns, int stall);
 
 // out[0 .. n) = value
 cudaError_t launch_fill(float* out, int64_t n, float value, cudaStream_t s);
@@ -256,5 +263,7 @@ cudaError_t launch_knn(const KnnArgs& a, cudaStream_t s);
 
 // Device error word (set by kernels whose waits time out).
 cudaError_t read_and_clear_device_error(int* value);
+// Test hook: the wait limit and stall mode of the tensor-core kernels.
+cudaError_t set_test_waits(uint64_t limit_ns, int stall);
 
 }  // namespace gs

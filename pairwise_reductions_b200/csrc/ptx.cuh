@@ -267,6 +267,12 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld2(uint32_t taddr, uint32_t (&v)[2]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];"
+               : "=r"(v[0]), "=r"(v[1])
+               : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -297,6 +303,29 @@ __device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
   d |= static_cast<uint64_t>(1u) << 46;                      // descriptor version (sm_100)
   d |= static_cast<uint64_t>(2u) << 61;                      // 128-byte swizzle
   return d;
+}
+
+// Shared-memory matrix descriptor for an MN-major operand in the 128-byte
+// swizzle layout: 8 K-rows of 128 B (64 two-byte elements along M or N) form a
+// 1024-byte atom; `lbo` is the byte distance between atoms along M/N, `sbo`
+// between groups of 8 K-rows.  The start must be 1024-byte aligned.
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+// Instruction-descriptor bit marking operand A as MN-major (read transposed).
+constexpr uint32_t kIdescAMajorMN = 1u << 15;
+
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (tensor-core operand reads) before it signals them with an mbarrier.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // Instruction descriptor with fp32 accumulation, both operands K-major.

@@ -59,12 +59,16 @@
 namespace gs {
 
 __device__ int g_device_error_f32;
+// The bounded waits' limit, and a stall mode that makes them run out on
+// purpose (0: off; 1: the MMA issuer issues nothing; 2: the exp warps do
+// nothing): test hooks, set by gs_test_set_waits.
+__device__ unsigned long long g_wait_limit_ns_f32 = 2000000000ull;
+__device__ int g_test_stall_f32;
 
 namespace {
 
 constexpr int kBM = 128;        // rows per CTA (one MMA tile)
 constexpr int kThreads = 320;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kAtom = kBM * 128;   // one 128-row x 32-float (128-byte) swizzle atom
 
@@ -152,7 +156,8 @@ struct F32Cfg {
   static_assert(SMEM_RAW <= 227 * 1024, "shared memory per CTA");
 };
 
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   uint32_t n = 0;
@@ -160,11 +165,24 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     if (mbar_try_wait(bar, parity)) return true;
     if ((++n & 63u) == 0u) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         atomicOr(&g_device_error_f32, 1);
         return false;
       }
+    }
+  }
+}
+
+// After an abort: wait for asynchronous work this CTA already started (a TMA
+// load's bytes, an MMA commit), bounded but not cut short by the abort flag.
+__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = global_timer_ns();
+  uint32_t n = 0;
+  while (!mbar_try_wait(bar, parity)) {
+    if ((++n & 63u) == 0u && global_timer_ns() - t0 > limit_ns) {
+      atomicOr(&g_device_error_f32, 4);
+      return;
     }
   }
 }
@@ -242,6 +260,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t jbeg = static_cast<int64_t>(blockIdx.y) * p.cols_per_split;
   const int64_t jend = min(p.N, jbeg + p.cols_per_split);
   const int T = (jend > jbeg) ? static_cast<int>((jend - jbeg + BN - 1) / BN) : 0;
+  const uint64_t wlim = g_wait_limit_ns_f32;
+  const int stall = g_test_stall_f32;
+  int issued = 0;   // producer lane: column tiles whose loads were issued
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
@@ -288,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t stage_tx = p.atoms * BN * 128 + BN * 16 + Cfg::V_BYTES;
       for (int t = 0; t < T; ++t) {
         const int st = t % NST;
-        if (t >= NST && !wait_bar(bar_empty(st), ((t / NST) - 1) & 1, abort_flag)) break;
+        if (t >= NST && !wait_bar(bar_empty(st), ((t / NST) - 1) & 1, abort_flag, wlim)) break;
         uint8_t* sy = sStage + st * Cfg::STAGE;
         uint8_t* sq = sy + Cfg::Y_BYTES;
         uint8_t* sv = sq + Cfg::QW_BYTES;
@@ -304,6 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_3d(smem_u32(sv + (hl * Cfg::VA + a) * Cfg::V_ATOM), &tmV, bar_full(st),
                           j0 + a * 64, 0, static_cast<int>(hl * p.Bsz + b));
         }
+        issued = t + 1;
       }
     }
     __syncwarp();
@@ -372,10 +394,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(d, phi, bh, idO, 1u);
         }
       };
-      bool ok = wait_bar(bar_x, 0, abort_flag);
+      bool ok = wait_bar(bar_x, 0, abort_flag, wlim) && stall != 1;
       tc_fence_after();
       for (int h = 0; ok && h < 2 && h < T; ++h) {
-        ok = wait_bar(bar_full(h), 0, abort_flag);
+        ok = wait_bar(bar_full(h), 0, abort_flag, wlim);
         if (ok) {
           tc_fence_after();
           issue_S(h, h);
@@ -387,8 +409,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // need the stage of tile t (three or more stages), else after it.
       constexpr bool kSFirst = REG || NST >= 3;
       auto next_S = [&](int h, int k, int t2) {
-        if (!wait_bar(bar_f(h), k & 1, abort_flag)) return false;
-        if (!wait_bar(bar_full(t2 % NST), (t2 / NST) & 1, abort_flag)) return false;
+        if (!wait_bar(bar_f(h), k & 1, abort_flag, wlim)) return false;
+        if (!wait_bar(bar_full(t2 % NST), (t2 / NST) & 1, abort_flag, wlim)) return false;
         tc_fence_after();
         issue_S(h, t2 % NST);
         mma_commit(bar_s(h));
@@ -401,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int t2 = t + 2;
           if (kSFirst && t2 < T && !(ok = next_S(h, k, t2))) break;
           if constexpr (!REG) {
-            if (!(ok = wait_bar(bar_p(h), k & 1, abort_flag))) break;
+            if (!(ok = wait_bar(bar_p(h), k & 1, abort_flag, wlim))) break;
             tc_fence_after();
             issue_O(h, t % NST, k > 0);
             mma_commit(bar_q(h));
@@ -455,11 +477,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     bool ok = true;
+    if (stall == 2) {   // test hook: wait on a barrier nobody arrives on, until the limit
+      wait_bar(bar_p(h), 0, abort_flag, wlim);
+      ok = false;
+    }
     int k = 0;
-    for (int t = h; t < T; t += 2, ++k) {
+    for (int t = h; ok && t < T; t += 2, ++k) {
       const int st = t % NST;
-      ok = wait_bar(bar_s(h), k & 1, abort_flag) &&
-           wait_bar(bar_full(st), (t / NST) & 1, abort_flag);   // norms and values landed
+      ok = wait_bar(bar_s(h), k & 1, abort_flag, wlim) &&
+           wait_bar(bar_full(st), (t / NST) & 1, abort_flag, wlim);   // norms and values landed
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
@@ -616,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ch == 0 && k > 0) {
             // P_h(previous tile) must have been read by its P.v MMAs
             // (waited for as late as possible)
-            ok = __all_sync(0xffffffffu, wait_bar(bar_q(h), (k - 1) & 1, abort_flag));
+            ok = __all_sync(0xffffffffu, wait_bar(bar_q(h), (k - 1) & 1, abort_flag, wlim));
             if (!ok) break;
             tc_fence_after();
           }
@@ -661,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     } else {
-      if (ok) ok = wait_bar(bar_o, 0, abort_flag);
+      if (ok) ok = wait_bar(bar_o, 0, abort_flag, wlim);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       if (ok && h == 0) {
@@ -693,6 +719,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  tc_fence_before();
+  __syncthreads();
+  // Every warp has left its loop.  The loads and MMAs already issued must land
+  // before the shared memory and TMEM they write are given up: after an abort
+  // some were never waited for (in a normal run these waits return at once).
+  if (warp == 0 && lane == 0) {
+    for (int t = issued > NST ? issued - NST : 0; t < issued; ++t)
+      drain_bar(bar_full(t % NST), (t / NST) & 1, wlim);
+    if constexpr (!Cfg::XT) drain_bar(bar_x, 0, wlim);
+  }
+  if (warp == 1 && lane == 0) drain_bar(bar_o, 0, wlim);
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -1174,6 +1211,13 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+cudaError_t set_test_waits_f32(uint64_t limit_ns, int stall) {
+  const unsigned long long l = limit_ns;
+  cudaError_t e = cudaMemcpyToSymbol(g_wait_limit_ns_f32, &l, sizeof(l));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_test_stall_f32, &stall, sizeof(int));
+  return e;
 }
 
 cudaError_t read_and_clear_device_error_f32(int* value) {

@@ -26,8 +26,16 @@
 // The issue order S0(t+1) before O1(t) lets both exp warpgroups run at once.
 // One value channel (CP = 1): no P.v MMAs; the exp warps sum P w in registers
 // against an fp32 record per column that rides with the stage.
+// Forward + backward in one sweep (GW): the exp warps also write P_h to shared
+// memory, and the issuer adds Gw_h = P_h^T . g_h (P_h read MN-major, i.e.
+// transposed, g_h the rows' upstream gradient as fp16 hi + lo parts), the
+// tile's column sums sum_i K_ij g_i, into TMEM; warpgroup h moves Gw_h to a
+// per-row-tile partial in global memory at its next tile.  Each kernel value
+// is then computed once for the forward sum, the x-gradient sums and dL/dw.
 // Every mbarrier wait is bounded (2 s); on expiry the kernel raises the device
-// error word, lets the other warps leave, frees TMEM and returns.
+// error word and the other warps leave their loops; before TMEM is freed and
+// the CTA exits, the producer waits for the loads it issued and the issuer for
+// the MMAs it issued (bounded, deaf to the abort), so nothing is in flight.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -42,6 +50,11 @@
 namespace gs {
 
 __device__ int g_device_error;
+// The bounded waits' limit, and a stall mode that makes them run out on
+// purpose (0: off; 1: the MMA issuer issues nothing; 2: the exp warps do
+// nothing): test hooks, set by gs_test_set_waits.
+__device__ unsigned long long g_wait_limit_ns = 2000000000ull;
+__device__ int g_test_stall;
 
 namespace {
 
@@ -50,7 +63,6 @@ constexpr int kBN = 128;   // columns per tile
 constexpr int kNT = 2;     // row tiles per CTA
 constexpr int kThreads = 320;
 constexpr float kPShift = 14.f;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct TcKParams {
@@ -64,9 +76,14 @@ struct TcKParams {
   float two_c;
   float out_scale;
   int s_ksteps;         // K steps of 16 holding the D + 2 nonzero packed columns
+  // forward + backward sweep only
+  const uint32_t* gpack;   // [B, M] the rows' upstream gradient: fp16 hi | lo << 16, scaled 2^e_b
+  const float* gscale;     // [B] 2^-e_b
+  float* gw_part;          // [RT, B, N] column sums of each 128-row tile
+  int64_t rt_count;        // RT = ceil(M / 128)
 };
 
-template <int KP, int CP>
+template <int KP, int CP, bool GW = false>
 struct TcCfg {
   static constexpr int KC = KP / 64;            // 128-byte swizzle atoms along K
   static constexpr int ATOM = kBM * 128;        // one 128-row x 64-col block: 16 KB
@@ -80,12 +97,19 @@ struct TcCfg {
   static constexpr int V_BYTES = REG ? 1024 : 2 * CP * 128;
   static constexpr int STAGE = Y_BYTES + V_BYTES;
   static constexpr int TX = Y_BYTES + (REG ? kBN * 4 : V_BYTES);   // bytes a stage's TMA loads
+  // Forward + backward sweep: P of both row tiles in shared memory as the
+  // MN-major operand of P^T . g (per tile: two 64-column atoms of 128 rows x
+  // 128 B, 32 KB), and g of both row tiles as its K-major B operand (16 rows
+  // x 128 K in two 64-element atoms, 4 KB).
+  static constexpr int P_TILE = kBM * kBN * 2;
+  static constexpr int G_TILE = 2 * 16 * 128;
+  static constexpr int PG_BYTES = GW ? kNT * (P_TILE + G_TILE) : 0;
   // 200 KB of operand stages; the three-atom rows (D > 126) may take 220 KB
-  static constexpr int BUDGET = (KC > 2 ? 220 : 200) * 1024;
+  static constexpr int BUDGET = (KC > 2 || GW ? 220 : 200) * 1024 - PG_BYTES;
   static constexpr int NST_FIT = (BUDGET - X_BYTES) / STAGE;
   static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
   static constexpr int NBARS = 2 * NST + 11;
-  static constexpr int SMEM_RAW = 1024 + X_BYTES + NST * STAGE + 8 * NBARS + 16;
+  static constexpr int SMEM_RAW = 1024 + X_BYTES + NST * STAGE + PG_BYTES + 8 * NBARS + 16;
   // at least ~120 KB so that a second CTA never lands on the SM and blocks on
   // the 512-column TMEM allocation
   static constexpr int SMEM = SMEM_RAW < 122880 ? 122880 : SMEM_RAW;
@@ -100,11 +124,16 @@ struct TcCfg {
   __host__ __device__ static constexpr uint32_t col_p(int h) {
     return P_SEPARATE ? 384u + 64u * h : 128u * h;
   }
+  // Gw_h: 16 columns after O_h's CP (the sweep needs CP <= 48)
+  __host__ __device__ static constexpr uint32_t col_g(int h) { return col_o(h) + 48u; }
+  static_assert(!GW || (P_SEPARATE && CP >= 16 && CP <= 48 && KC == 1), "forward + backward sweep");
+  static_assert(SMEM_RAW <= 227 * 1024, "shared memory per CTA");
   static_assert(NST >= 2, "shared memory budget");
   static_assert(CP == 1 || (CP % 16 == 0 && CP >= 16 && CP <= 128), "value chunk");
 };
 
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   uint32_t n = 0;
@@ -112,11 +141,24 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     if (mbar_try_wait(bar, parity)) return true;
     if ((++n & 63u) == 0u) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         atomicOr(&g_device_error, 1);
         return false;
       }
+    }
+  }
+}
+
+// After an abort: wait for asynchronous work this CTA already started (a TMA
+// load's bytes, an MMA commit), bounded but not cut short by the abort flag.
+__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = global_timer_ns();
+  uint32_t n = 0;
+  while (!mbar_try_wait(bar, parity)) {
+    if ((++n & 63u) == 0u && global_timer_ns() - t0 > limit_ns) {
+      atomicOr(&g_device_error, 4);
+      return;
     }
   }
 }
@@ -150,18 +192,20 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&v)[32], uint64_t two_
   }
 }
 
-template <int KP, int CP, int DTFMT>
+template <int KP, int CP, int DTFMT, bool GW>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gauss_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                     const __grid_constant__ CUtensorMap tmV, const TcKParams p) {
-  using Cfg = TcCfg<KP, CP>;
+  using Cfg = TcCfg<KP, CP, GW>;
   constexpr int NST = Cfg::NST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sX = smem;
   uint8_t* sStage = smem + Cfg::X_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + NST * Cfg::STAGE);
+  uint8_t* sP = sStage + NST * Cfg::STAGE;               // GW: P_0 | P_1 (1024-aligned)
+  uint8_t* sG = sP + kNT * Cfg::P_TILE;                   // GW: g_0 | g_1
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + NST * Cfg::STAGE + Cfg::PG_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -181,6 +225,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t jbeg = static_cast<int64_t>(blockIdx.y) * p.cols_per_split;
   const int64_t jend = min(p.N, jbeg + p.cols_per_split);
   const int T = (jend > jbeg) ? static_cast<int>((jend - jbeg + kBN - 1) / kBN) : 0;
+  const uint64_t wlim = g_wait_limit_ns;
+  const int stall = g_test_stall;
+  int issued = 0;   // producer lane: column tiles whose loads were issued
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
@@ -222,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       static_cast<int>(row0 + h * kBM), static_cast<int>(b));
       for (int t = 0; t < T; ++t) {
         const int st = t % NST;
-        if (t >= NST && !wait_bar(bar_empty(st), ((t / NST) - 1) & 1, abort_flag)) break;
+        if (t >= NST && !wait_bar(bar_empty(st), ((t / NST) - 1) & 1, abort_flag, wlim)) break;
         uint8_t* sy = sStage + st * Cfg::STAGE;
         uint8_t* sv = sy + Cfg::Y_BYTES;
         const int j0 = static_cast<int>(jbeg + static_cast<int64_t>(t) * kBN);
@@ -237,6 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(smem_u32(sv + hh * CP * 128), &tmV, bar_full(st), j0 + hh * 64, 0,
                         static_cast<int>(b));
         }
+        issued = t + 1;
       }
     }
     __syncwarp();
@@ -266,10 +314,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(tmem + Cfg::col_o(h), tmem + Cfg::col_p(h) + ks * 8, bd, idO,
                  (acc_prev || ks > 0) ? 1u : 0u);
         }
+        if constexpr (GW) {
+          // Gw_h = P_h^T . g_h: M = the tile's 128 columns, N = 16 (g hi, lo,
+          // zeros), K = the 128 rows, 16 per MMA (two 8-row groups of P_h)
+          const uint32_t idG = idesc_f16(0, kBM, 16) | kIdescAMajorMN;
+          const uint32_t pa = smem_u32(sP + h * Cfg::P_TILE);
+          const uint32_t ga = smem_u32(sG + h * Cfg::G_TILE);
+#pragma unroll
+          for (int ks = 0; ks < kBM / 16; ++ks) {
+            const uint64_t ad = desc_mn_sw128(pa + ks * 2048, 64 * 2 * kBM, 1024);
+            const uint64_t bd = desc_k_sw128(ga + (ks >> 2) * 2048 + (ks & 3) * 32);
+            mma_ss(tmem + Cfg::col_g(h), ad, bd, idG, ks > 0 ? 1u : 0u);
+          }
+        }
       };
-      bool ok = wait_bar(bar_x, 0, abort_flag);
+      bool ok = wait_bar(bar_x, 0, abort_flag, wlim) && stall != 1;
       if (ok && T > 0) {
-        ok = wait_bar(bar_full(0), 0, abort_flag);
+        ok = wait_bar(bar_full(0), 0, abort_flag, wlim);
         if (ok) {
           tc_fence_after();
           issue_S(0, 0);
@@ -285,12 +346,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           // register values: only the similarity MMAs; S_h(t+1) once warpgroup h
           // has read S_h(t) (the exp warps release the stages themselves)
           if (t + 1 < T) {
-            if (!(ok = wait_bar(bar_f(0), t & 1, abort_flag))) break;
-            if (!(ok = wait_bar(bar_full(st1), ((t + 1) / NST) & 1, abort_flag))) break;
+            if (!(ok = wait_bar(bar_f(0), t & 1, abort_flag, wlim))) break;
+            if (!(ok = wait_bar(bar_full(st1), ((t + 1) / NST) & 1, abort_flag, wlim))) break;
             tc_fence_after();
             issue_S(0, st1);
             mma_commit(bar_s(0));
-            if (!(ok = wait_bar(bar_f(1), t & 1, abort_flag))) break;
+            if (!(ok = wait_bar(bar_f(1), t & 1, abort_flag, wlim))) break;
             tc_fence_after();
             issue_S(1, st1);
             mma_commit(bar_s(1));
@@ -300,39 +361,39 @@ __global__ void __launch_bounds__(kThreads, 1)
           // into registers: it then runs while the exponentials of tile t are
           // still being computed.
           if (t + 1 < T) {
-            if (!(ok = wait_bar(bar_f(0), t & 1, abort_flag))) break;
-            if (!(ok = wait_bar(bar_full(st1), ((t + 1) / NST) & 1, abort_flag))) break;
+            if (!(ok = wait_bar(bar_f(0), t & 1, abort_flag, wlim))) break;
+            if (!(ok = wait_bar(bar_full(st1), ((t + 1) / NST) & 1, abort_flag, wlim))) break;
             tc_fence_after();
             issue_S(0, st1);
             mma_commit(bar_s(0));
           }
-          if (!(ok = wait_bar(bar_p(0), t & 1, abort_flag))) break;
+          if (!(ok = wait_bar(bar_p(0), t & 1, abort_flag, wlim))) break;
           tc_fence_after();
           issue_O(0, st, t > 0);
           mma_commit(bar_q(0));
           if (t + 1 < T) {
-            if (!(ok = wait_bar(bar_f(1), t & 1, abort_flag))) break;
+            if (!(ok = wait_bar(bar_f(1), t & 1, abort_flag, wlim))) break;
             tc_fence_after();
             issue_S(1, st1);
             mma_commit(bar_s(1));
           }
-          if (!(ok = wait_bar(bar_p(1), t & 1, abort_flag))) break;
+          if (!(ok = wait_bar(bar_p(1), t & 1, abort_flag, wlim))) break;
           tc_fence_after();
           issue_O(1, st, t > 0);
           mma_commit(bar_q(1));
           mma_commit(bar_empty(st));
         } else {
           // P lives in the S columns: the next S MMA must follow the P MMA
-          if (!(ok = wait_bar(bar_p(0), t & 1, abort_flag))) break;
+          if (!(ok = wait_bar(bar_p(0), t & 1, abort_flag, wlim))) break;
           tc_fence_after();
           issue_O(0, st, t > 0);
           if (t + 1 < T) {
-            if (!(ok = wait_bar(bar_full(st1), ((t + 1) / NST) & 1, abort_flag))) break;
+            if (!(ok = wait_bar(bar_full(st1), ((t + 1) / NST) & 1, abort_flag, wlim))) break;
             tc_fence_after();
             issue_S(0, st1);
             mma_commit(bar_s(0));
           }
-          if (!(ok = wait_bar(bar_p(1), t & 1, abort_flag))) break;
+          if (!(ok = wait_bar(bar_p(1), t & 1, abort_flag, wlim))) break;
           tc_fence_after();
           issue_O(1, st, t > 0);
           mma_commit(bar_empty(st));
@@ -342,9 +403,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // the drain point for whatever was issued (register values: every S MMA
-      // was waited for by the exp warps, and nothing waits on this barrier)
-      if constexpr (!Cfg::REG) mma_commit(bar_o);
+      // the drain point for whatever was issued (register values: the exp
+      // warps wait for every S MMA themselves; only an abort waits on it)
+      mma_commit(bar_o);
     }
     __syncwarp();
   } else {
@@ -364,10 +425,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t two_c2 = pk2(two_c, two_c);
     const uint64_t r2 = pk2(r, r);
     float row_sum = 0.f;   // register values: the row's sum over the tiles
-    for (int t = 0; t < T; ++t) {
-      ok = wait_bar(bar_s(h), t & 1, abort_flag);
+    // Forward + backward sweep.  TMEM lane `row` of Gw_h is column j0 + row of
+    // the tile; row tile rt of the matrix.
+    const int64_t rt = static_cast<int64_t>(blockIdx.x) * kNT + h;
+    uint8_t* const sPh = sP + h * Cfg::P_TILE;
+    if constexpr (GW) {
+      // this row's (g hi, g lo) as column `row` of g_h: rows 0 and 1 of the
+      // 16-row K-major operand, rows 2..15 zero
+      const uint32_t gv = valid ? p.gpack[b * p.M + i] : 0u;
+      uint8_t* gh = sG + h * Cfg::G_TILE + (row >> 6) * 2048;
+      const int kin = row & 63;
+#pragma unroll
+      for (int n = 0; n < 16; ++n) {
+        const uint16_t v = n == 0 ? static_cast<uint16_t>(gv & 0xffffu)
+                                  : (n == 1 ? static_cast<uint16_t>(gv >> 16) : uint16_t(0));
+        *reinterpret_cast<uint16_t*>(gh + n * 128 + ((((kin >> 3) ^ (n & 7)) << 4) | ((kin & 7) << 1))) = v;
+      }
+      fence_proxy_async_smem();
+    }
+    // P columns [32 c, 32 c + 32) of this row into P_h: row `row` of 8-row
+    // group row / 8, 64-column atom c / 2, 16-byte pieces swizzled by row % 8
+    auto store_p = [&](int c, const uint32_t(&pk)[16]) {
+      uint8_t* base = sPh + (c >> 1) * (64 * 2 * kBM) + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int piece = (((c & 1) << 2) + q) ^ (row & 7);
+        *reinterpret_cast<uint4*>(base + piece * 16) =
+            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+      }
+    };
+    // Gw_h of column tile tt (complete: its MMAs were waited for) to the
+    // row tile's partial; also completes any TMEM load still in flight
+    const float gsc = GW ? p.gscale[b] * p.out_scale : 0.f;
+    auto drain_gw = [&](int tt) {
+      uint32_t gq[2];
+      tmem_ld2(tmem + lane_base + Cfg::col_g(h), gq);
+      tmem_wait_ld();
+      asm volatile("" : "+r"(gq[0]), "+r"(gq[1]));
+      const int64_t j = jbeg + static_cast<int64_t>(tt) * kBN + row;
+      if (rt < p.rt_count && j < jend)
+        p.gw_part[(rt * gridDim.z + b) * p.N + j] =
+            (__uint_as_float(gq[0]) + __uint_as_float(gq[1])) * gsc;
+    };
+    if (stall == 2) {   // test hook: wait on a barrier nobody arrives on, until the limit
+      wait_bar(bar_p(h), 0, abort_flag, wlim);
+      ok = false;
+    }
+    for (int t = 0; ok && t < T; ++t) {
+      ok = wait_bar(bar_s(h), t & 1, abort_flag, wlim);
       // register values read the stage's records themselves: its loads landed
-      if (Cfg::REG && ok) ok = wait_bar(bar_full(t % NST), (t / NST) & 1, abort_flag);
+      if (Cfg::REG && ok) ok = wait_bar(bar_full(t % NST), (t / NST) & 1, abort_flag, wlim);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
@@ -428,17 +535,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (Cfg::P_SEPARATE && t > 0) {
           // a warp that runs ahead must not overwrite its rows of P(t-1) before
           // the P MMA of tile t-1 has read them (waited for as late as possible)
-          ok = __all_sync(0xffffffffu, wait_bar(bar_q(h), (t - 1) & 1, abort_flag));
+          ok = __all_sync(0xffffffffu, wait_bar(bar_q(h), (t - 1) & 1, abort_flag, wlim));
           if (!ok) {
             tmem_wait_ld();   // chunk 2's load may still be in flight
             break;
           }
           tc_fence_after();
+          if constexpr (GW) drain_gw(t - 1);
         }
         tmem_st16(tP, pk);
+        if constexpr (GW) store_p(0, pk);
         tmem_ld32(tS + 96, va);
         exp_chunk(vb, two_c2, r2, pk);
         tmem_st16(tP + 16, pk);
+        if constexpr (GW) store_p(1, pk);
         tmem_wait_ld();
         reg_fence32(vc);
         reg_fence32(va);
@@ -446,9 +556,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar_f(h));
         exp_chunk(vc, two_c2, r2, pk);
         tmem_st16(tP + 32, pk);
+        if constexpr (GW) store_p(2, pk);
         exp_chunk(va, two_c2, r2, pk);
         tmem_st16(tP + 48, pk);
+        if constexpr (GW) store_p(3, pk);
         tmem_wait_st();
+        if constexpr (GW) fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(bar_p(h));
       }
@@ -461,9 +574,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         orow[0] = (T > 0) ? row_sum * p.out_scale : 0.f;
       }
     } else {
-      if (ok) ok = wait_bar(bar_o, 0, abort_flag);
+      if (ok) ok = wait_bar(bar_o, 0, abort_flag, wlim);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
+      if constexpr (GW) {
+        if (ok && T > 0) drain_gw(T - 1);
+      }
       if (ok) {
         float* orow = p.out + static_cast<int64_t>(blockIdx.y) * p.split_stride +
                       (b * p.M + i) * p.ldo + p.c0;
@@ -485,6 +601,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  tc_fence_before();
+  __syncthreads();
+  // Every warp has left its loop.  The loads and MMAs already issued must land
+  // before the shared memory and TMEM they write are given up: after an abort
+  // some were never waited for (in a normal run these waits return at once).
+  if (warp == 0 && lane == 0) {
+    for (int t = issued > NST ? issued - NST : 0; t < issued; ++t)
+      drain_bar(bar_full(t % NST), (t / NST) & 1, wlim);
+    drain_bar(bar_x, 0, wlim);
+  }
+  if (warp == 1 && lane == 0) drain_bar(bar_o, 0, wlim);
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -608,6 +735,38 @@ __global__ void pack_records_kernel(const TW* __restrict__ w, const TY* __restri
   }
 }
 
+// The rows' upstream gradient g[b, :, 0] for the forward + backward sweep, as
+// fp16 hi + lo parts of g 2^e_b (e_b per batch puts the largest |g| in
+// [2^13, 2^14)): hi = fp16(g 2^e), lo = fp16(g 2^e - hi), ~22 significant bits
+// together.  gscale[b] = 2^-e_b.  One block per batch.
+__global__ void pack_g_kernel(const float* __restrict__ g, int64_t ldg, uint32_t* __restrict__ gpack,
+                              float* __restrict__ gscale, int64_t M) {
+  __shared__ float red[32];
+  const int64_t b = blockIdx.x;
+  const float* gb = g + b * M * ldg;
+  float mx = 0.f;
+  for (int64_t i = threadIdx.x; i < M; i += blockDim.x) mx = fmaxf(mx, fabsf(gb[i * ldg]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  mx = red[0];
+  for (int v = 1; v < static_cast<int>(blockDim.x >> 5); ++v) mx = fmaxf(mx, red[v]);
+  // e = 13 - floor(log2 max), from the exponent bits; within [-126, 126]
+  int e = 0;
+  if (mx > 0.f) e = 13 - (((__float_as_int(mx) >> 23) & 0xff) - 127);
+  e = e > 126 ? 126 : (e < -126 ? -126 : e);
+  const float sc = __int_as_float((e + 127) << 23);
+  for (int64_t i = threadIdx.x; i < M; i += blockDim.x) {
+    const float v = gb[i * ldg] * sc;
+    const __half hi = __float2half_rn(v);
+    const __half lo = __float2half_rn(v - __half2float(hi));
+    gpack[b * M + i] = static_cast<uint32_t>(__half_as_ushort(hi)) |
+                       (static_cast<uint32_t>(__half_as_ushort(lo)) << 16);
+  }
+  if (threadIdx.x == 0) gscale[b] = __int_as_float((127 - e) << 23);
+}
+
 // ------------------------------------------------------------------ host side
 int grid_for(int64_t n, int threads) {
   int64_t b = (n + threads - 1) / threads;
@@ -669,11 +828,11 @@ cudaError_t pack_values(const TcArgs& a, int c0, int CP, int64_t Nst, cudaStream
   return cudaGetLastError();
 }
 
-template <int KP, int CP, int DTFMT>
+template <int KP, int CP, int DTFMT, bool GW = false>
 cudaError_t launch_kernel(const CUtensorMap& tx, const CUtensorMap& ty, const CUtensorMap& tv,
                           const TcKParams& kp, dim3 grid, cudaStream_t s) {
-  using Cfg = TcCfg<KP, CP>;
-  auto fn = tc_gauss_kernel<KP, CP, DTFMT>;
+  using Cfg = TcCfg<KP, CP, GW>;
+  auto fn = tc_gauss_kernel<KP, CP, DTFMT, GW>;
   static bool attr_done = false;   // idempotent; a benign race at worst repeats the call
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
@@ -682,6 +841,19 @@ cudaError_t launch_kernel(const CUtensorMap& tx, const CUtensorMap& ty, const CU
   }
   fn<<<grid, kThreads, Cfg::SMEM, s>>>(tx, ty, tv, kp);
   return cudaGetLastError();
+}
+
+// The forward + backward sweep: 64-wide packed rows, one chunk of 16, 32 or 48
+// value channels.
+template <int DTFMT>
+cudaError_t launch_gw(int CP, const CUtensorMap& tx, const CUtensorMap& ty, const CUtensorMap& tv,
+                      const TcKParams& kp, dim3 grid, cudaStream_t s) {
+  switch (CP) {
+    case 16: return launch_kernel<64, 16, DTFMT, true>(tx, ty, tv, kp, grid, s);
+    case 32: return launch_kernel<64, 32, DTFMT, true>(tx, ty, tv, kp, grid, s);
+    case 48: return launch_kernel<64, 48, DTFMT, true>(tx, ty, tv, kp, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 template <int KP, int DTFMT>
@@ -792,6 +964,14 @@ cudaError_t launch_tc_sum(const TcArgs& a, cudaStream_t s) {
   const dim3 grid(static_cast<unsigned>((a.M + kNT * kBM - 1) / (kNT * kBM)),
                   static_cast<unsigned>(a.plan.splits), static_cast<unsigned>(a.B));
   const int chunk = tc_max_chunk(KP);
+  const bool gw = a.gw_part != nullptr;
+  if (gw) {
+    // one fused sweep: the values in a single chunk of at most 48 channels
+    if (KP != 64 || a.CV > 48 || a.CV < 2) return cudaErrorInvalidValue;
+    pack_g_kernel<<<static_cast<unsigned>(a.B), 1024, 0, s>>>(a.g, a.g_ld, a.gpack, a.gscale, a.M);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   for (int c0 = 0; c0 < a.CV; c0 += chunk) {
     const int cw = (a.CV - c0) < chunk ? (a.CV - c0) : chunk;
     // one value channel: fp32 records summed in registers (CP = 1)
@@ -825,6 +1005,15 @@ cudaError_t launch_tc_sum(const TcArgs& a, cudaStream_t s) {
     kp.two_c = a.tau * kLog2e;
     kp.out_scale = exp2f(-kPShift);
     kp.s_ksteps = static_cast<int>((a.D + 2 + 15) / 16);
+    if (gw) {
+      kp.gpack = a.gpack;
+      kp.gscale = a.gscale;
+      kp.gw_part = a.gw_part;
+      kp.rt_count = (a.M + kBM - 1) / kBM;
+      e = bf ? launch_gw<1>(CP, tx, ty, tv, kp, grid, s) : launch_gw<0>(CP, tx, ty, tv, kp, grid, s);
+      if (e != cudaSuccess) return e;
+      continue;
+    }
     if (KP == 64)
       e = bf ? launch_cp<64, 1>(CP, tx, ty, tv, kp, grid, s) : launch_cp<64, 0>(CP, tx, ty, tv, kp, grid, s);
     else if (KP == 128)
@@ -834,6 +1023,13 @@ cudaError_t launch_tc_sum(const TcArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+cudaError_t set_test_waits(uint64_t limit_ns, int stall) {
+  const unsigned long long l = limit_ns;
+  cudaError_t e = cudaMemcpyToSymbol(g_wait_limit_ns, &l, sizeof(l));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_test_stall, &stall, sizeof(int));
+  return e;
 }
 
 cudaError_t read_and_clear_device_error(int* value) {

@@ -16,6 +16,15 @@ forward's lse of every row as an input, so a pass over a subset of the sources
 still normalises by the full sum --; the dL/dtau shares are summed over the
 ranks.
 
+The diffusion operator of "FlashDiffusion" (§2.2: q = K 1, d = q^-alpha
+(K q^-alpha), s = q^-alpha d^-1/2, then diag(s) K diag(s) V) shards by rows of
+its one point set: every rank needs every point (one all-gather of x), then
+the q^-alpha of every point for its rows of d (a second all-gather), and for
+the operator the s V of every point (a third).  Each rank's rows of q, d, s and
+of the operator's output are its own; the pair work is
+`gauss_diffusion_block` (rows of this rank, columns of every rank, float32
+values), the per-point arithmetic between the passes is elementwise.
+
 The exchanges are `torch.distributed` collectives on the group's backend (NCCL
 over NVLink for CUDA tensors); the pair work runs in this library's kernels
 (`gauss_sum_fwd`, `gauss_lse_fwd`, `gauss_sum_bwd`, `gauss_sum_vjp`,
@@ -33,9 +42,10 @@ import torch.distributed as dist
 
 
 def _default_kernels():
-    from . import gauss_lse_bwd, gauss_lse_fwd, gauss_sum_bwd, gauss_sum_fwd, gauss_sum_vjp
+    from . import (gauss_diffusion_block, gauss_lse_bwd, gauss_lse_fwd, gauss_sum_bwd,
+                   gauss_sum_fwd, gauss_sum_vjp)
     return {"sum": gauss_sum_fwd, "lse": gauss_lse_fwd, "bwd": gauss_sum_bwd,
-            "lse_bwd": gauss_lse_bwd, "vjp": gauss_sum_vjp}
+            "lse_bwd": gauss_lse_bwd, "vjp": gauss_sum_vjp, "block": gauss_diffusion_block}
 
 
 def shard_counts(n_local, device, group=None):
@@ -161,5 +171,36 @@ def sharded_lse_bwd(x, y, w, lse, g, tau, group=None, kernels=None, row_counts=N
     return out
 
 
+def sharded_diffusion_scales(x, tau, alpha, group=None, kernels=None, counts=None):
+    """(q, d, s) of the alpha-normalised diffusion operator for this rank's points
+    x [B, N_r, D] of a point set sharded by rows: each [B, N_r] float32 (float64
+    when the compute is), over the kernel of every rank's points."""
+    k = kernels or _default_kernels()
+    if counts is None:
+        counts = shard_counts(x.shape[1], x.device, group)
+    xa = all_gather_rows(x, group, counts)
+    B = x.shape[0]
+    dt = torch.float64 if x.dtype == torch.float64 else torch.float32
+    ones = torch.ones((B, xa.shape[1], 1), dtype=dt, device=x.device)
+    q = k["block"](x, xa, ones, tau)[..., 0]
+    qa = q.pow(-alpha)
+    u = k["block"](x, xa, all_gather_rows(qa[..., None].contiguous(), group, counts), tau)[..., 0]
+    d = qa * u
+    s = qa * d.rsqrt()
+    return q, d, s
+
+
+def sharded_diffusion_apply(x, s, v, tau, group=None, kernels=None, counts=None):
+    """This rank's rows of diag(s) K diag(s) V over the whole point set: x [B, N_r, D],
+    s [B, N_r] and v [B, N_r, C] are this rank's points, scales and rows of V."""
+    k = kernels or _default_kernels()
+    if counts is None:
+        counts = shard_counts(x.shape[1], x.device, group)
+    xa = all_gather_rows(x, group, counts)
+    sv = all_gather_rows((s[..., None] * v).contiguous(), group, counts)
+    return s[..., None] * k["block"](x, xa, sv, tau)
+
+
 __all__ = ["shard_counts", "all_gather_rows", "sharded_sum_fwd", "sharded_lse_fwd",
-           "sharded_sum_bwd", "sharded_sum_vjp", "sharded_lse_bwd"]
+           "sharded_sum_bwd", "sharded_sum_vjp", "sharded_lse_bwd", "sharded_diffusion_scales",
+           "sharded_diffusion_apply"]

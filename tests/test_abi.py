@@ -119,8 +119,15 @@ def test_workspace_query():
     assert ws(gs.GS_OP_KNN, 1, 10, 10, 9, 1, gs.GS_F32) > 0
     with pytest.raises(ValueError):
         ws(gs.GS_OP_KNN, 1, 10, 10, 129, 1, gs.GS_F32)
+    # the forward + backward call: the x-pass sums, g's parts and the dL/dw
+    # partials of every 128-row tile on top of the pass scratch
+    fb = ws(gs.GS_OP_SUM_FWD_BWD, 4, 16384, 16384, 32, 1, gs.GS_F16)
+    assert fb >= 4 * 16384 * 33 * 4 + 4 * 16384 * 4 + 128 * 4 * 16384 * 4
+    assert ws(gs.GS_OP_SUM_FWD_BWD, 1, 1000, 1000, 3, 1, gs.GS_F32) >= 1000 * 4 * 4
+    assert ws(gs.GS_OP_DIFFUSION_BLOCK, 1, 500, 2000, 3, 2, gs.GS_F32) >= 0
+    assert ws(gs.GS_OP_DIFFUSION_BLOCK, 1, 500, 2000, 32, 2, gs.GS_F16) > 0
     with pytest.raises(ValueError):
-        ws(7, 1, 10, 10, 3, 1, gs.GS_F32)
+        ws(8, 1, 10, 10, 3, 1, gs.GS_F32)
 
 
 def test_bwd_argument_checks():
@@ -214,3 +221,12 @@ def test_binding_rejects_mismatched_tensors_before_any_call():
         gs.gauss_sum_bwd_saved(x, y, w, g, torch.zeros(2, 5, 3), 1.0)
     with pytest.raises(ValueError):           # lse of the wrong shape
         gs.gauss_lse_bwd(x, y, w, torch.zeros(2, 5, 2), g, 1.0)
+
+
+def test_testing_hooks_reject_bad_arguments_without_a_device_call():
+    lib = gs.library()
+    assert lib.gs_test_set_waits(999, 0) == 1
+    assert lib.gs_test_set_waits(10_000_000_001, 0) == 1
+    assert lib.gs_test_set_waits(1_000_000, 3) == 1
+    assert lib.gs_test_set_waits(1_000_000, -1) == 1
+    assert lib.gs_test_read_error_word(NULL, NULL) == 1

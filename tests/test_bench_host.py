@@ -31,10 +31,13 @@ def test_pairs_and_kernel_evaluations_per_step():
     # the sum and the log-sum-exp: two outputs, two passes
     assert bench.pairs_per_step(w["d3_1m_lse"]) == 2 * 10 ** 12
     assert bench.kernel_evals_per_step(w["d3_1m_lse"]) == 2 * 10 ** 12
-    # forward + backward: the pairs once (B M N / (t_fwd + t_bwd)), two passes of exponentials
+    # forward + backward: the pairs once; one sweep of exponentials in one call
+    # (fp16, C = 1, D = 32), two for the two-call path
     p = 4 * 16384 * 16384
     assert bench.pairs_per_step(w["d32_c1_bwd"]) == p
-    assert bench.kernel_evals_per_step(w["d32_c1_bwd"]) == 2 * p
+    assert bench.fused_fwd_bwd(w["d32_c1_bwd"])
+    assert bench.kernel_evals_per_step(w["d32_c1_bwd"]) == p
+    assert bench.kernel_evals_per_step(w["d32_c1_bwd"], two_call=True) == 2 * p
 
 
 def test_traffic_figure_only_while_the_kernel_source_is_unchanged(tmp_path, monkeypatch):

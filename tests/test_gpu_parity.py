@@ -12,6 +12,7 @@ import torch
 
 import oracle
 import synth
+from knn_check import knn_valid_under_exact_distances
 
 pytestmark = pytest.mark.gpu
 
@@ -93,6 +94,31 @@ def test_d32_c1_f16_fwd_bwd_sampled():
     rgx, rgw = oracle.gauss_sum_bwd(x, y, w, g, inp["tau"], rows=rows, wrows=wrows)
     assert rel_l2(gx[:, rows], rgx) <= TOL["f16"], rel_l2(gx[:, rows], rgx)
     assert rel_l2(gw[:, wrows], rgw) <= TOL["f16"], rel_l2(gw[:, wrows], rgw)
+
+
+def test_d32_c1_f16_saved_pair_full_size():
+    """The call pair the benchmark times for this workload (B=4, M=N=16384, D=32,
+    C=1, fp16): gauss_sum_fwd_saved then gauss_sum_bwd_saved, at full size and in
+    the same launch configuration, against the oracle on sampled rows and
+    sources; and bit for bit against the separate backward entry point, which
+    runs the same passes."""
+    inp = synth.make_inputs(5)
+    d = dev(inp)
+    m = gs()
+    out, saved = m.gauss_sum_fwd_saved(d["x"], d["y"], d["w"], inp["tau"])
+    gx, gw = m.gauss_sum_bwd_saved(d["x"], d["y"], d["w"], d["g"], saved, inp["tau"])
+    x, y, w, g = (f64(inp, k) for k in "xywg")
+    rows = synth.sample_rows(inp["M"], 512, seed=40).numpy()
+    wrows = synth.sample_rows(inp["N"], 512, seed=41).numpy()
+    ref = oracle.gauss_sum(x, y, w, inp["tau"], rows=rows)
+    o = out.cpu().numpy()
+    assert rel_l2(o[:, rows], ref) <= TOL["f16"], rel_l2(o[:, rows], ref)
+    rgx, rgw = oracle.gauss_sum_bwd(x, y, w, g, inp["tau"], rows=rows, wrows=wrows)
+    gxn, gwn = gx.cpu().numpy(), gw.cpu().numpy()
+    assert rel_l2(gxn[:, rows], rgx) <= TOL["f16"], rel_l2(gxn[:, rows], rgx)
+    assert rel_l2(gwn[:, wrows], rgw) <= TOL["f16"], rel_l2(gwn[:, wrows], rgw)
+    bx, bw = m.gauss_sum_bwd(d["x"], d["y"], d["w"], d["g"], inp["tau"])
+    assert torch.equal(bx, gx) and torch.equal(bw, gw)
 
 
 # ------------------------------------------------------------------ odd shapes, both paths
@@ -431,6 +457,123 @@ def test_fwd_saved_then_bwd_saved(dtype, shape):
     assert only_w[0] is None and torch.equal(only_w[1], gw)
 
 
+# ------------------------------------------------------------------ forward + backward in one call
+FWD_BWD_FUSED = [  # dtype, (B, M, N, D): fp16 / bf16, C = 1, D <= 47 -> one sweep
+    ("f16", (1, 300, 500, 32)), ("bf16", (2, 257, 700, 32)), ("f16", (1, 129, 1000, 1)),
+    ("f16", (2, 513, 300, 15)), ("bf16", (1, 1, 900, 16)), ("f16", (1, 700, 1, 31)),
+    ("f16", (1, 1000, 2100, 47)), ("bf16", (3, 260, 390, 46)), ("f16", (1, 2049, 1500, 5)),
+]
+FWD_BWD_OTHER = [  # dtype, (B, M, N, D, C): the two-pass path
+    ("f32", (1, 300, 500, 3, 1)), ("f32", (1, 250, 400, 32, 1)), ("f16", (1, 200, 300, 60, 1)),
+    ("f16", (2, 150, 250, 32, 2)), ("bf16", (1, 120, 333, 16, 3)),
+]
+
+
+def _fwd_bwd_check(inp, dtype, tol_w=None):
+    d = dev(inp)
+    m = gs()
+    out, gx, gw = m.gauss_sum_fwd_bwd(d["x"], d["y"], d["w"], d["g"], inp["tau"])
+    x, y, w, g = (f64(inp, k) for k in "xywg")
+    ref = oracle.gauss_sum(x, y, w, inp["tau"])
+    rgx, rgw = oracle.gauss_sum_bwd(x, y, w, g, inp["tau"])
+    tol = TOL[dtype]
+    assert rel_l2(out.cpu().numpy(), ref) <= tol, rel_l2(out.cpu().numpy(), ref)
+    assert rel_l2(gx.cpu().numpy(), rgx) <= tol, rel_l2(gx.cpu().numpy(), rgx)
+    assert rel_l2(gw.cpu().numpy(), rgw) <= (tol_w or tol), rel_l2(gw.cpu().numpy(), rgw)
+    return d, out, gx, gw
+
+
+@pytest.mark.parametrize("dtype,shape", FWD_BWD_FUSED, ids=[f"{d}-{s}" for d, s in FWD_BWD_FUSED])
+def test_fwd_bwd_fused_sweep(dtype, shape):
+    """gauss_sum_fwd_bwd on the one-sweep path against the oracle; its forward
+    sum and x-gradient are the same arithmetic as gauss_sum_fwd_saved +
+    gauss_sum_bwd_saved (bit for bit), its grad_w comes from P^T g in the same
+    sweep."""
+    B, M, N, D = shape
+    inp = synth.make_inputs(5, seed=61, B=B, M=M, N=N, D=D, C=1, dtype=dtype, with_g=True)
+    if M == 1:
+        # one row: its relative error is that of a single sum, which signed
+        # weights can make arbitrarily ill-conditioned; positive weights keep
+        # the case a test of the one-row tile rather than of cancellation
+        inp["w"] = (inp["w"].double().abs() + 0.25).to(inp["w"].dtype)
+    d, out, gx, gw = _fwd_bwd_check(inp, dtype)
+    m = gs()
+    so, saved = m.gauss_sum_fwd_saved(d["x"], d["y"], d["w"], inp["tau"])
+    sx, _ = m.gauss_sum_bwd_saved(d["x"], d["y"], d["w"], d["g"], saved, inp["tau"], want_w=False)
+    assert torch.equal(out, so) and torch.equal(gx, sx)
+    # deterministic: fixed-order partial sums, no atomics
+    o2, x2, w2 = m.gauss_sum_fwd_bwd(d["x"], d["y"], d["w"], d["g"], inp["tau"])
+    assert torch.equal(o2, out) and torch.equal(x2, gx) and torch.equal(w2, gw)
+
+
+@pytest.mark.parametrize("dtype,shape", FWD_BWD_OTHER, ids=[f"{d}-{s}" for d, s in FWD_BWD_OTHER])
+def test_fwd_bwd_two_pass_path(dtype, shape):
+    B, M, N, D, C = shape
+    wid = 1 if (dtype == "f32" and D <= 8) else 5
+    inp = synth.make_inputs(wid, seed=62, B=B, M=M, N=N, D=D, C=C, dtype=dtype, with_g=True)
+    _fwd_bwd_check(inp, dtype)
+
+
+@pytest.mark.parametrize("gscale", [1e-30, 1e-6, 1e6, 1e30])
+def test_fwd_bwd_upstream_gradient_scales(gscale):
+    """g far from unit scale: the per-batch power of two keeps its fp16 parts
+    in range (two batches 10^3 apart, one row of zeros)."""
+    inp = synth.make_inputs(5, seed=63, B=2, M=300, N=700, D=32, C=1, with_g=True)
+    g = inp["g"].double() * gscale
+    g[1] *= 1e3
+    g[0, 7] = 0.0
+    inp["g"] = g.float()
+    _fwd_bwd_check(inp, "f16")
+
+
+def test_fwd_bwd_edge_cases():
+    m = gs()
+    for (M, N) in ((0, 50), (40, 0), (1, 1)):
+        inp = synth.make_inputs(5, seed=64, B=2, M=M, N=N, D=32, C=1, with_g=True)
+        d = dev(inp)
+        out, gx, gw = m.gauss_sum_fwd_bwd(d["x"], d["y"], d["w"], d["g"], inp["tau"])
+        x, y, w, g = (f64(inp, k) for k in "xywg")
+        if M and N:
+            assert rel_l2(out.cpu().numpy(), oracle.gauss_sum(x, y, w, inp["tau"])) <= TOL["f16"]
+            rgx, rgw = oracle.gauss_sum_bwd(x, y, w, g, inp["tau"])
+            assert rel_l2(gx.cpu().numpy(), rgx) <= TOL["f16"]
+            assert rel_l2(gw.cpu().numpy(), rgw) <= TOL["f16"]
+        else:
+            assert not out.abs().sum() and not gx.abs().sum() and not gw.abs().sum()
+    # outputs left out
+    inp = synth.make_inputs(5, seed=65, B=1, M=300, N=400, D=32, C=1, with_g=True)
+    d = dev(inp)
+    ref_o, ref_x, ref_w = m.gauss_sum_fwd_bwd(d["x"], d["y"], d["w"], d["g"], inp["tau"])
+    o, gx, gw = m.gauss_sum_fwd_bwd(d["x"], d["y"], d["w"], d["g"], inp["tau"], want_w=False)
+    assert gw is None and torch.equal(o, ref_o) and torch.equal(gx, ref_x)
+    o, gx, gw = m.gauss_sum_fwd_bwd(d["x"], d["y"], d["w"], d["g"], inp["tau"], want_x=False)
+    assert gx is None and torch.equal(o, ref_o) and torch.equal(gw, ref_w)
+
+
+def test_d32_c1_f16_fwd_bwd_one_call_full_size():
+    """The forward + backward workload (B=4, M=N=16384, D=32, C=1, fp16) through
+    gauss_sum_fwd_bwd, the call the benchmark times for it, against the oracle
+    on sampled rows and sources, and against the two-call path."""
+    inp = synth.make_inputs(5)
+    d = dev(inp)
+    m = gs()
+    out, gx, gw = m.gauss_sum_fwd_bwd(d["x"], d["y"], d["w"], d["g"], inp["tau"])
+    x, y, w, g = (f64(inp, k) for k in "xywg")
+    rows = synth.sample_rows(inp["M"], 512, seed=66).numpy()
+    wrows = synth.sample_rows(inp["N"], 512, seed=67).numpy()
+    ref = oracle.gauss_sum(x, y, w, inp["tau"], rows=rows)
+    rgx, rgw = oracle.gauss_sum_bwd(x, y, w, g, inp["tau"], rows=rows, wrows=wrows)
+    o, gxn, gwn = out.cpu().numpy(), gx.cpu().numpy(), gw.cpu().numpy()
+    assert rel_l2(o[:, rows], ref) <= TOL["f16"], rel_l2(o[:, rows], ref)
+    assert rel_l2(gxn[:, rows], rgx) <= TOL["f16"], rel_l2(gxn[:, rows], rgx)
+    assert rel_l2(gwn[:, wrows], rgw) <= TOL["f16"], rel_l2(gwn[:, wrows], rgw)
+    so, saved = m.gauss_sum_fwd_saved(d["x"], d["y"], d["w"], inp["tau"])
+    sx, sw = m.gauss_sum_bwd_saved(d["x"], d["y"], d["w"], d["g"], saved, inp["tau"])
+    assert torch.equal(out, so) and torch.equal(gx, sx)
+    # grad_w: fp16 P (this sweep) against fp32 P (the separate pass), whole arrays
+    assert rel_l2(gwn, sw.cpu().numpy()) <= TOL["f16"]
+
+
 # ------------------------------------------------------------------ full gradient
 @pytest.mark.parametrize("dtype,shape,shift", [
     ("f32", (1, 400, 600, 3, 1), 0.0), ("f32", (2, 300, 500, 2, 3), 0.0), ("f32", (1, 250, 350, 8, 2), 0.0),
@@ -556,6 +699,7 @@ def test_knn_bit_exact(shape):
     rd, ri = oracle.knn(inp["x"].numpy(), inp["y"].numpy(), K, f32=True)
     assert np.array_equal(oi.cpu().numpy(), ri), "indices differ"
     assert np.array_equal(od.cpu().numpy(), rd), "distances differ"
+    knn_valid_under_exact_distances(inp["x"].numpy(), inp["y"].numpy(), od.cpu(), oi.cpu(), K)
 
 
 @pytest.mark.parametrize("dtype,shape", [("f16", (1, 700, 2000, 3, 8)), ("bf16", (2, 300, 900, 16, 5)),
@@ -569,6 +713,8 @@ def test_knn_half_precision_bit_exact(dtype, shape):
     rd, ri = oracle.knn(inp["x"].float().numpy(), inp["y"].float().numpy(), K, f32=True)
     assert np.array_equal(oi.cpu().numpy(), ri), "indices differ"
     assert np.array_equal(od.cpu().numpy(), rd), "distances differ"
+    knn_valid_under_exact_distances(inp["x"].float().numpy(), inp["y"].float().numpy(), od.cpu(),
+                                    oi.cpu(), K)
 
 
 @pytest.mark.parametrize("D", [3, 12, 40])
@@ -583,6 +729,7 @@ def test_knn_duplicates_and_quantised_grid(D):
     rd, ri = oracle.knn(x.numpy(), y.numpy(), 12, f32=True)
     assert np.array_equal(oi.cpu().numpy(), ri)
     assert np.array_equal(od.cpu().numpy(), rd)
+    knn_valid_under_exact_distances(x.numpy(), y.numpy(), od.cpu(), oi.cpu(), 12)
 
 
 # ------------------------------------------------------------------ diffusion operator
@@ -606,3 +753,17 @@ def test_diffusion_scales_and_apply(dtype, shape, alpha):
     # sqrt(d) is the operator's fixed point
     fp = gs().gauss_diffusion_apply(x, s, dd.sqrt()[..., None].contiguous(), tau)
     assert rel_l2(fp.cpu().numpy(), dd.sqrt()[..., None].cpu().numpy()) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype,shape", [("f32", (1, 700, 2000, 3, 2)), ("f32", (2, 300, 900, 40, 3)),
+                                         ("f16", (1, 500, 1300, 32, 1)), ("bf16", (2, 257, 640, 16, 4))])
+def test_diffusion_block_rows_against_other_columns(dtype, shape):
+    """K(x_rows, x_cols) v with float32 values: a rank's rows against every
+    rank's points, the pair work of the row-sharded diffusion operator."""
+    B, M, N, D, C = shape
+    small = dtype == "f32" and D <= 8
+    inp = synth.make_inputs(1 if small else 4, seed=71, B=B, M=M, N=N, D=D, C=C, dtype=dtype)
+    v = torch.rand(B, N, C, generator=torch.Generator().manual_seed(72)) + 0.5
+    out = gs().gauss_diffusion_block(inp["x"].cuda(), inp["y"].cuda(), v.cuda(), 2.0)
+    ref = oracle.gauss_sum(f64(inp, "x"), f64(inp, "y"), v.double().numpy(), 2.0)
+    assert rel_l2(out.cpu().numpy(), ref) <= TOL[dtype], rel_l2(out.cpu().numpy(), ref)

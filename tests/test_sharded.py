@@ -22,6 +22,14 @@ ROWS = (37, 21)
 SRCS = (15, 40)
 
 
+ALPHA = 0.5
+
+
+def _diffusion_v():
+    g = torch.Generator().manual_seed(78)
+    return torch.randn(2, sum(SRCS), 3, generator=g, dtype=torch.float64)
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
@@ -55,7 +63,8 @@ def _oracle_kernels():
         return {kk: full[kk] for kk in want}
     return {"sum": lambda x, y, w, tau: t(oracle.gauss_sum(n(x), n(y), n(w), tau)),
             "lse": lambda x, y, w, tau: t(oracle.gauss_lse(n(x), n(y), n(w), tau)),
-            "bwd": bwd, "lse_bwd": _lse_bwd_given_lse, "vjp": vjp}
+            "bwd": bwd, "lse_bwd": _lse_bwd_given_lse, "vjp": vjp,
+            "block": lambda xr, xc, v, tau: t(oracle.gauss_sum(n(xr), n(xc), n(v), tau))}
 
 
 def _lse_bwd_given_lse(x, y, w, lse, g, tau, want=("x", "y", "w", "tau")):
@@ -99,6 +108,11 @@ def _worker(rank, world, port, q):
     vg = sharded.sharded_sum_vjp(xs, ys, ws, gs_, TAU, kernels=k)
     out.update({"vjp_g" + kk: v for kk, v in vg.items()})
     out.update({"lse_g" + kk: v for kk, v in lg.items()})
+    # the diffusion operator over the point set y, sharded by its rows (the sources)
+    dv = _diffusion_v()
+    vs = dv[:, s0:s0 + SRCS[rank]].contiguous()
+    out["dq"], out["dd"], out["ds"] = sharded.sharded_diffusion_scales(ys, TAU, ALPHA, kernels=k)
+    out["dapply"] = sharded.sharded_diffusion_apply(ys, out["ds"], vs, TAU, kernels=k)
     q.put((rank, {kk: v.numpy() for kk, v in out.items()}))
     dist.destroy_process_group()
 
@@ -122,6 +136,8 @@ def test_sharded_problem_matches_the_whole_problem_gloo():
     gx, gw = oracle.gauss_sum_bwd(x, y, w, g, TAU)
     lgx, lgy, lgw, lgt = oracle.gauss_lse_bwd(x, y, w, g, TAU)
     vgy, vgt = oracle.gauss_sum_vjp_y_tau(x, y, w, g, TAU)
+    dq, dd, ds = oracle.diffusion_scales(y, TAU, ALPHA)
+    dap = oracle.diffusion_apply(y, ds, _diffusion_v().numpy(), TAU)
     for rank in range(world):
         r0, s0 = sum(ROWS[:rank]), sum(SRCS[:rank])
         rows, srcs = slice(r0, r0 + ROWS[rank]), slice(s0, s0 + SRCS[rank])
@@ -142,6 +158,11 @@ def test_sharded_problem_matches_the_whole_problem_gloo():
         np.testing.assert_allclose(o["vjp_gy"], vgy[:, srcs], rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(o["vjp_gw"], gw[:, srcs], rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(o["vjp_gtau"], [vgt], rtol=1e-12)
+        # diffusion operator: this rank's rows of q, d, s and of diag(s) K diag(s) V
+        np.testing.assert_allclose(o["dq"], dq[:, srcs], rtol=1e-12)
+        np.testing.assert_allclose(o["dd"], dd[:, srcs], rtol=1e-12)
+        np.testing.assert_allclose(o["ds"], ds[:, srcs], rtol=1e-12)
+        np.testing.assert_allclose(o["dapply"], dap[:, srcs], rtol=1e-11, atol=1e-14)
 
 
 def _gpu_worker(port, q):
@@ -159,9 +180,18 @@ def _gpu_worker(port, q):
     lse = m.gauss_lse_fwd(x, y, w, TAU)
     lg = sharded.sharded_lse_bwd(x, y, w, lse, g, TAU)
     rl = m.gauss_lse_bwd(x, y, w, lse, g, TAU)
+    # diffusion operator of the point set y: one rank against the single-GPU entry points
+    dq, dd, ds = sharded.sharded_diffusion_scales(y, TAU, 0.5)
+    rq, rd, rs = m.gauss_diffusion_scales(y, TAU, 0.5)
+    v = torch.rand(y.shape[0], y.shape[1], 2, device="cuda")
+    da = sharded.sharded_diffusion_apply(y, ds, v, TAU)
+    ra = m.gauss_diffusion_apply(y, rs, v, TAU)
     torch.cuda.synchronize()
     lse_ok = all(torch.allclose(lg[k], rl[k], rtol=1e-6, atol=1e-7) for k in ("x", "y", "w", "tau"))
-    q.put(bool(torch.equal(a, b) and torch.equal(gx, rx) and torch.equal(gw, rw) and lse_ok))
+    diff_ok = (torch.equal(dq, rq) and all(torch.allclose(p_, r_, rtol=1e-6)
+                                           for p_, r_ in ((dd, rd), (ds, rs), (da, ra))))
+    q.put(bool(torch.equal(a, b) and torch.equal(gx, rx) and torch.equal(gw, rw) and lse_ok
+               and diff_ok))
     dist.destroy_process_group()
 
 
