@@ -63,6 +63,9 @@ def parse():
                     help="skip the profiler-based kernel count (use under ncu)")
     ap.add_argument("--clock-log", default=None,
                     help="CSV of the nvidia-smi clock samples (default: a file under the temp directory)")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch each timed step from the host instead of replaying it from a "
+                         "CUDA graph captured after the warm-up")
     ap.add_argument("--two-call", action="store_true",
                     help="forward + backward workloads: time gauss_sum_fwd_saved then "
                          "gauss_sum_bwd_saved (two sweeps, g not needed by the forward) instead "
@@ -406,10 +409,29 @@ def main():
     n_launch, kernel_names = (None, []) if args.no_launch_count else launches_per_step(gs, run)
     if gs.last_device_error() != 0:
         raise SystemExit("device error word set during warm-up")
+    two_part = (not args.sharded) and "sum" in w.ops and "bwd" in w.ops and args.two_call
+    # The timed steps replay one step captured in a CUDA graph: the same kernels
+    # on the same buffers, without the host's launch gaps between them (which
+    # matter at tens of microseconds a step).
+    graph, graph_note = None, "host launches"
+    if not args.no_graph and not args.sharded and not two_part:
+        try:
+            g = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream(device=dev)
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                run()
+            torch.cuda.current_stream().wait_stream(side)
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g):
+                run()
+            torch.cuda.synchronize()
+            graph, graph_note = g, "one step captured in a CUDA graph, replayed each timed step"
+        except Exception as exc:   # capture unsupported here: time host launches
+            graph, graph_note = None, f"host launches (graph capture failed: {type(exc).__name__})"
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    two_part = (not args.sharded) and "sum" in w.ops and "bwd" in w.ops and args.two_call
     mids = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)] if two_part else None
     clk_path = (args.clock_log.replace(".csv", f"_rank{rank}.csv") if args.clock_log
                 else os.path.join(tempfile.gettempdir(), f"gs_clocks_{rank}.csv"))
@@ -423,6 +445,8 @@ def main():
             starts[k].record(stream)
             if two_part:
                 run(mids[k])
+            elif graph is not None:
+                graph.replay()
             else:
                 run()
             ends[k].record(stream)
@@ -569,6 +593,7 @@ def main():
                            "tau": w.tau, "ops": list(w.ops), "pairs_per_step": evals,
                            "kernel_evaluations_per_step": kevals,
                            "l2": "flushed by a 256 MiB write between timed steps",
+                           "launch": graph_note,
                            "parallelism": (f"one problem sharded over {world} rank(s): rows and "
                                            f"sources split, sources all-gathered each step")
                            if args.sharded else f"independent problems, {world} rank(s)"},
@@ -583,6 +608,7 @@ def main():
         if parts is not None:
             line["parts"] = parts   # rank 0's medians
         print(json.dumps(line), flush=True)
+    graph = None   # released before the process group
     if pg is not None:
         pg.destroy_process_group()
 

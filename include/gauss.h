@@ -310,8 +310,10 @@ gs_status gauss_diffusion_apply(const void *x, const float *s, const float *v, f
  * a latency-critical loop that must not block in the CUDA allocator, a process
  * under a hard memory cap).  Same arguments, results and kernels as
  * gauss_sum_fwd, without ws / ws_bytes: the scratch comes from a fixed 32 MiB
- * device array inside the library, held by every GPU on which it has been used
- * until the process exits.  Calls whose scratch need (gs_workspace_bytes of
+ * device array inside the library, held per device context until the process
+ * exits: on every device context the process creates when CUDA loads modules
+ * eagerly (CUDA_MODULE_LOADING=EAGER), and only on devices where this call has
+ * been made under lazy loading (the default).  Calls whose scratch need (gs_workspace_bytes of
  * GS_OP_SUM) exceeds 32 MiB return GS_ERR_WORKSPACE.  All calls on a device
  * share the array: calls that overlap on the GPU race (order them on one
  * stream).  The array keeps the last call's contents; nothing in it needs to

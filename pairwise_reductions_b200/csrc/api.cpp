@@ -46,12 +46,8 @@ gs_status check_dims(gs_op op, int64_t B, int64_t M, int64_t N, int64_t D, int64
   const double big = 9.0e18;
   if (double(B) * double(M > N ? M : N) * double((D > C ? D : C) + 1) * double(D + 2) > big)
     return GS_ERR_UNSUPPORTED;
-  if (dt == GS_F32) {
-    // D > 8: the split-tf32 tensor-core path, for the Gauss-sum passes only
-    if (D > kTcMaxD) return GS_ERR_UNSUPPORTED;
-  } else {
-    if (D > kTcMaxD) return GS_ERR_UNSUPPORTED;
-  }
+  // every dtype: the CUDA-core path up to D = 8 (fp32), the tensor-core paths up to 128
+  if (D > kTcMaxD) return GS_ERR_UNSUPPORTED;
   return GS_OK;
 }
 
@@ -191,7 +187,9 @@ struct GwArgs {
   int64_t g_ld;
   uint32_t* gpack;     // [B, R]
   float* gscale;       // [B]
+  float* gtmax;        // [B, ceil(R / 128)]
   float* gw_part;      // [ceil(R / 128), B, N]
+  bool keep_splits;    // leave the pass's split partials uncombined (the caller reads them)
 };
 
 // Run one pass into `out` ([B, R, CV] float32) using workspace `ws`; with
@@ -311,10 +309,11 @@ gs_status run_pass(const Pass& p, const PassLayout& L, float* out, uint8_t* ws, 
     a.g_ld = gw->g_ld;
     a.gpack = gw->gpack;
     a.gscale = gw->gscale;
+    a.gtmax = gw->gtmax;
     a.gw_part = gw->gw_part;
   }
   GS_CUDA(launch_tc_sum(a, s));
-  if (S > 1) GS_CUDA(launch_combine_sum(dst, S, total, out, s));
+  if (S > 1 && !(gw && gw->keep_splits)) GS_CUDA(launch_combine_sum(dst, S, total, out, s));
   return GS_OK;
 }
 
@@ -349,7 +348,7 @@ struct FwdBwdLayout {
   bool fused;
   int CV;
   int64_t RT;          // 128-row tiles of the fused sweep's dL/dw partials
-  size_t off_saved, off_gpack, off_gscale, off_gwpart, off_pass;
+  size_t off_saved, off_gpack, off_gscale, off_gtmax, off_gwpart, off_pass;
   size_t total;
 };
 
@@ -373,6 +372,8 @@ FwdBwdLayout fwd_bwd_layout(const void* x, const void* y, const void* w, const f
     off = align_up(off + size_t(B) * M * 4);
     L.off_gscale = off;
     off = align_up(off + size_t(B) * 4);
+    L.off_gtmax = off;
+    off = align_up(off + size_t(B) * L.RT * 4);
     L.off_gwpart = off;
     off = align_up(off + size_t(L.RT) * B * N * 4);
   } else if (want_w) {
@@ -921,7 +922,10 @@ gs_status gauss_sum_bwd_saved(const void* x, const void* y, const void* w, const
     }
     GS_TRY(run_pass(py, ly, grad_w, static_cast<uint8_t*>(ws), s));
   }
-  if (grad_x)
+  if (grad_x && C == 1)   // one row per warp; the same arithmetic as the general epilogue
+    GS_CUDA(launch_fwd_bwd_epilogue(x, dt, g, saved, 1, 0, nullptr, grad_x, B, M,
+                                    static_cast<int>(D), CV, tau, s));
+  else if (grad_x)
     GS_CUDA(launch_grad_x_epilogue(x, dt, g, saved, grad_x, nullptr, B, M, static_cast<int>(D),
                                    static_cast<int>(C), CV, tau, s));
   return GS_OK;
@@ -955,17 +959,31 @@ gs_status gauss_sum_fwd_bwd(const void* x, const void* y, const void* w, const f
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   float* saved = reinterpret_cast<float*>(wsb + L.off_saved);
   if (L.fused) {
+    // one sweep; the x-side sums stay as the sweep's split partials, which the
+    // epilogue adds in the combine's fixed order while it forms out and grad_x
     GwArgs ga{};
     ga.g = g;
     ga.g_ld = C;
     ga.gpack = reinterpret_cast<uint32_t*>(wsb + L.off_gpack);
     ga.gscale = reinterpret_cast<float*>(wsb + L.off_gscale);
+    ga.gtmax = reinterpret_cast<float*>(wsb + L.off_gtmax);
     ga.gw_part = reinterpret_cast<float*>(wsb + L.off_gwpart);
+    ga.keep_splits = true;
     GS_TRY(run_pass(L.px, L.lx, saved, wsb + L.off_pass, s, &ga));
+    const int S = L.lx.tcp.splits;
+    const float* part = S > 1 ? reinterpret_cast<const float*>(wsb + L.off_pass + L.lx.off_part)
+                              : saved;
     GS_CUDA(launch_combine_sum(ga.gw_part, static_cast<int>(L.RT), B * N, grad_w, s));
-  } else {
-    GS_TRY(run_pass(L.px, L.lx, saved, wsb + L.off_pass, s));
-    if (grad_w) GS_TRY(run_pass(L.py, L.ly, grad_w, wsb + L.off_pass, s));
+    GS_CUDA(launch_fwd_bwd_epilogue(x, dt, g, part, S, B * M * L.CV, out, grad_x, B, M,
+                                    static_cast<int>(D), L.CV, tau, s));
+    return GS_OK;
+  }
+  GS_TRY(run_pass(L.px, L.lx, saved, wsb + L.off_pass, s));
+  if (grad_w) GS_TRY(run_pass(L.py, L.ly, grad_w, wsb + L.off_pass, s));
+  if (C == 1) {
+    GS_CUDA(launch_fwd_bwd_epilogue(x, dt, g, saved, 1, 0, out, grad_x, B, M, static_cast<int>(D),
+                                    L.CV, tau, s));
+    return GS_OK;
   }
   GS_CUDA(cudaMemcpy2DAsync(out, size_t(C) * 4, saved, size_t(L.CV) * 4, size_t(C) * 4,
                             size_t(B) * M, cudaMemcpyDeviceToDevice, s));

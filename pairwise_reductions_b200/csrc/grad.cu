@@ -20,6 +20,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "combine.cuh"
 #include "internal.h"
 #include "values.cuh"
 
@@ -91,6 +92,42 @@ __global__ void grad_x_epilogue_kernel(const T* __restrict__ x, const float* __r
       for (int c = 0; c < C; ++c)
         tau_acc = fmaf(gi[c], fmaf(xx, oi[c], oi[C * (1 + D) + c]), tau_acc);
       tau_rows[r] = -0.5f * tau_acc;
+    }
+  }
+}
+
+// Forward + backward, one value channel (C = 1): the forward sum (unless `out`
+// is null) and dL/dx straight from the x pass's split partials part[k][b, i, :] (k < splits,
+// `stride` apart), summed in the fixed order of combine.cuh -- the same values
+// the combine kernel would have written, so the results equal those of the
+// combine followed by grad_x_epilogue_kernel bit for bit:
+//     s = sum_k part[k][b,i,:],  out[b,i] = s[0],
+//     dL/dx[b,i,k] = -tau g_i ((x_ik - z_k) s[0] - s[1 + k]).
+// One warp per row; lanes over the D dimensions (coalesced reads of x, of each
+// split's sums and of the gradient row).
+template <typename T>
+__global__ void fwd_bwd_epilogue_kernel(const T* __restrict__ x, const float* __restrict__ g,
+                                        const float* __restrict__ part, int splits,
+                                        int64_t stride, float* __restrict__ out,
+                                        float* __restrict__ gx, int64_t B, int64_t M, int D,
+                                        int CV, float tau) {
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = B * M;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
+       r < rows; r += warps) {
+    const int64_t b = r / M;
+    const float* o = part + r * CV;
+    const float s0 = split_sum(o, splits, stride);
+    if (lane == 0 && out) out[r] = s0;
+    if (!gx) continue;
+    const float gi = g[r];
+    const T* xi = x + r * D;
+    const T* z = x + b * M * D;
+    for (int k = lane; k < D; k += 32) {
+      const float xk = tf(xi[k]) - tf(z[k]);
+      const float t = gi * fmaf(xk, s0, -split_sum(o + 1 + k, splits, stride));
+      gx[r * D + k] = -tau * t;
     }
   }
 }
@@ -269,6 +306,31 @@ cudaError_t launch_pack_values_f32(const void* src, int64_t src_ld, const void* 
   const int blocks = grid_for(n, 256);
   pack_values_f32_kernel<float, float><<<blocks, 256, 0, s>>>(
       as<float>(src), src_ld, as<float>(cols), as<float>(rows), v, B, N, Mrows, D, C, mode);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_bwd_epilogue(const void* x, gs_dtype dt, const float* g, const float* part,
+                                    int splits, int64_t stride, float* out, float* grad_x,
+                                    int64_t B, int64_t M, int D, int CV, float tau,
+                                    cudaStream_t s) {
+  int64_t blocks = (B * M + 7) / 8;   // 8 warps a block, one row each
+  if (blocks > 148 * 64) blocks = 148 * 64;
+  if (blocks < 1) blocks = 1;
+  const unsigned nb = static_cast<unsigned>(blocks);
+  switch (dt) {
+    case GS_F32:
+      fwd_bwd_epilogue_kernel<float><<<nb, 256, 0, s>>>(as<float>(x), g, part, splits, stride, out,
+                                                        grad_x, B, M, D, CV, tau);
+      break;
+    case GS_F16:
+      fwd_bwd_epilogue_kernel<__half><<<nb, 256, 0, s>>>(as<__half>(x), g, part, splits, stride, out,
+                                                         grad_x, B, M, D, CV, tau);
+      break;
+    default:
+      fwd_bwd_epilogue_kernel<__nv_bfloat16><<<nb, 256, 0, s>>>(
+          as<__nv_bfloat16>(x), g, part, splits, stride, out, grad_x, B, M, D, CV, tau);
+      break;
+  }
   return cudaGetLastError();
 }
 

@@ -115,6 +115,11 @@ cudaError_t launch_lse_grad_y_epilogue(const float* y, const float* w, const flo
 cudaError_t launch_grad_x_epilogue(const void* x, gs_dtype dt, const float* g, const float* o,
                                    float* grad_x, float* tau_rows, int64_t B, int64_t M, int D,
                                    int C, int CV, float tau, cudaStream_t s);
+// Forward + backward (C = 1): out and grad_x from the x pass's `splits` partials.
+cudaError_t launch_fwd_bwd_epilogue(const void* x, gs_dtype dt, const float* g, const float* part,
+                                    int splits, int64_t stride, float* out, float* grad_x,
+                                    int64_t B, int64_t M, int D, int CV, float tau,
+                                    cudaStream_t s);
 cudaError_t launch_grad_y_epilogue(const void* y, const void* w, gs_dtype dt, const float* o,
                                    float* grad_y, float* grad_w, int64_t B, int64_t N, int D,
                                    int C, int CV, float tau, cudaStream_t s);
@@ -174,8 +179,9 @@ struct TcArgs {
   // forward + backward sweep (gw_part != nullptr): dL/dw column sums as well
   const float* g;      // [B, M, g_ld] upstream gradient, channel 0
   int64_t g_ld;
-  uint32_t* gpack;     // [B, M]
-  float* gscale;       // [B]
+  uint32_t* gpack;     // [B, M] packed parts of g
+  float* gscale;       // [B] their scales
+  float* gtmax;        // [B, ceil(M / 128)] largest |g| of each 128-row tile
   float* gw_part;      // [ceil(M / 128), B, N]
 };
 cudaError_t launch_tc_sum(const TcArgs& a, cudaStream_t s);

@@ -9,8 +9,12 @@
 // from a fixed array compiled into this library instead of a caller buffer.
 //
 // Costs and limits:
-//   * every GPU that loads the library holds kScratchBytes (32 MiB) of device
-//     memory for this array until the process exits;
+//   * the array is part of this file's own module (the library is built
+//     without relocatable device code, so each source file is one module):
+//     kScratchBytes (32 MiB) of device memory per device context, held until
+//     the process exits -- on every context the process creates when modules
+//     load eagerly (CUDA_MODULE_LOADING=EAGER), and under lazy loading (the
+//     default) only on devices where this entry point has been called;
 //   * a call whose scratch need exceeds 32 MiB is rejected with
 //     GS_ERR_WORKSPACE (use gauss_sum_fwd with a caller workspace instead);
 //   * all calls on a device share the one array, so calls that overlap on the
@@ -42,13 +46,18 @@ void* g_scratch_ptr[kMaxDevices] = {};
 // Device address of the scratch array on the current device (set up once per device).
 gs_status scratch_for_current_device(void** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GS_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();   // leave no error behind for the next, unrelated call to report
+    return GS_ERR_CUDA;
+  }
   if (dev < 0 || dev >= kMaxDevices) return GS_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
   if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
       return GS_ERR_CUDA;
+    }
     g_scratch_ptr[dev] = p;
   }
   *out = g_scratch_ptr[dev];

@@ -31,6 +31,7 @@
 #include <cmath>
 
 #include "../../include/gauss_testing.h"
+#include "combine.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -345,13 +346,28 @@ cudaError_t launch_d(const SdArgs& a, cudaStream_t s) {
 }
 
 // ------------------------------------------------------------------ combine
-__global__ void combine_sum_kernel(const float* __restrict__ part, int splits, int64_t total,
-                                   float* __restrict__ out) {
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    float s = 0.f;
-    for (int k = 0; k < splits; ++k) s += part[k * total + e];
-    out[e] = s;
+// out[e] = sum_k part[k * total + e] in the fixed order of combine.cuh.  A block
+// takes 32 consecutive elements with one warp per lane of that order: warp l
+// sums splits l, l + 8, ... in turn (reading 128 contiguous bytes of a split
+// at a time), then the 8 lane sums are added in lane order.  Eight short
+// chains instead of one long one keep the loads of many splits in flight.
+__global__ void __launch_bounds__(32 * kCombineLanes)
+    combine_sum_kernel(const float* __restrict__ part, int splits, int64_t total,
+                       float* __restrict__ out) {
+  __shared__ float red[kCombineLanes][33];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int64_t e0 = blockIdx.x * 32ll; e0 < total; e0 += gridDim.x * 32ll) {
+    const int64_t e = e0 + tx;
+    const float s = (e < total) ? split_lane_sum(part + e, ty, splits, total) : 0.f;
+    red[ty][tx] = s;
+    __syncthreads();
+    if (ty == 0 && e < total) {
+      float t = red[0][tx];
+#pragma unroll
+      for (int v = 1; v < kCombineLanes; ++v) t += red[v][tx];
+      out[e] = t;
+    }
+    __syncthreads();
   }
 }
 
@@ -516,7 +532,7 @@ cudaError_t launch_small_d_lse(const SdArgs& a, cudaStream_t s) { return launch_
 
 cudaError_t launch_combine_sum(const float* part, int splits, int64_t total, float* out,
                                cudaStream_t s) {
-  combine_sum_kernel<<<grid_for(total, 256), 256, 0, s>>>(part, splits, total, out);
+  combine_sum_kernel<<<grid_for(total, 32), 32 * kCombineLanes, 0, s>>>(part, splits, total, out);
   return cudaGetLastError();
 }
 

@@ -703,21 +703,24 @@ __global__ void pack_rows_kernel(const T* __restrict__ src, T* __restrict__ dst,
 // Transposed fp16 value matrix v^T [B, CP, Nst] for channels [c0, c0 + CP) of
 // the pass's value matrix (values.cuh; columns = the y side of this pass,
 // centre = its first row point).  Channels past CV are written as zeros.
+// One thread per column (b, j), all CP channels: consecutive threads take
+// consecutive j, so each channel's store is coalesced, and the column's point
+// and weights are read once.
 template <typename TW, typename TY>
 __global__ void pack_values_kernel(const TW* __restrict__ w, const TY* __restrict__ y,
                                    const TY* __restrict__ rows, __half* __restrict__ vt, int64_t B,
                                    int64_t N, int64_t Nst, int64_t Mrows, int C, int D, int CV,
                                    int c0, int CP) {
-  const int64_t total = B * CP * N;
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t j = e % N;
-    const int64_t bc = e / N;
-    const int cc = static_cast<int>(bc % CP);
-    const int64_t b = bc / CP;
-    const int ch = c0 + cc;
-    const float v = (ch < CV) ? value_at(w, y, rows, b, b * N + j, Mrows, D, C, ch, C) : 0.f;
-    vt[(b * CP + cc) * Nst + j] = __float2half_rn(v);
+  const int64_t total = B * N;
+  for (int64_t bj = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; bj < total;
+       bj += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = bj / N, j = bj - b * N;
+    __half* dst = vt + b * CP * Nst + j;
+    for (int cc = 0; cc < CP; ++cc) {
+      const int ch = c0 + cc;
+      const float v = (ch < CV) ? value_at(w, y, rows, b, bj, Mrows, D, C, ch, C) : 0.f;
+      dst[cc * Nst] = __float2half_rn(v);
+    }
   }
 }
 
@@ -736,35 +739,51 @@ __global__ void pack_records_kernel(const TW* __restrict__ w, const TY* __restri
 }
 
 // The rows' upstream gradient g[b, :, 0] for the forward + backward sweep, as
-// fp16 hi + lo parts of g 2^e_b (e_b per batch puts the largest |g| in
-// [2^13, 2^14)): hi = fp16(g 2^e), lo = fp16(g 2^e - hi), ~22 significant bits
-// together.  gscale[b] = 2^-e_b.  One block per batch.
-__global__ void pack_g_kernel(const float* __restrict__ g, int64_t ldg, uint32_t* __restrict__ gpack,
-                              float* __restrict__ gscale, int64_t M) {
-  __shared__ float red[32];
-  const int64_t b = blockIdx.x;
-  const float* gb = g + b * M * ldg;
-  float mx = 0.f;
-  for (int64_t i = threadIdx.x; i < M; i += blockDim.x) mx = fmaxf(mx, fabsf(gb[i * ldg]));
+// fp16 hi + lo parts of g 2^e_b (~22 significant bits together), e_b per batch
+// putting the batch's largest |g 2^e_b| in [2^13, 2^14): hi = fp16(g 2^e),
+// lo = fp16(g 2^e - hi), gpack = hi | lo << 16, gscale[b] = 2^-e_b.  Two
+// launches over (128-row tile, batch) blocks: the tiles' largest |g|, then
+// each block reduces its batch's tile maxima and packs its tile.
+__global__ void __launch_bounds__(128) g_tile_max_kernel(const float* __restrict__ g, int64_t ldg,
+                                                         float* __restrict__ tmax, int64_t M,
+                                                         int64_t RT) {
+  __shared__ float red[4];
+  const int64_t rt = blockIdx.x, b = blockIdx.y;
+  const int64_t i = rt * 128 + threadIdx.x;
+  float mx = i < M ? fabsf(g[(b * M + i) * ldg]) : 0.f;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
   __syncthreads();
-  mx = red[0];
-  for (int v = 1; v < static_cast<int>(blockDim.x >> 5); ++v) mx = fmaxf(mx, red[v]);
-  // e = 13 - floor(log2 max), from the exponent bits; within [-126, 126]
-  int e = 0;
+  if (threadIdx.x == 0) tmax[b * RT + rt] = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+}
+
+__global__ void __launch_bounds__(128) pack_g_kernel(const float* __restrict__ g, int64_t ldg,
+                                                     const float* __restrict__ tmax,
+                                                     uint32_t* __restrict__ gpack,
+                                                     float* __restrict__ gscale, int64_t M,
+                                                     int64_t RT) {
+  __shared__ float red[4];
+  const int64_t rt = blockIdx.x, b = blockIdx.y;
+  float mx = 0.f;
+  for (int64_t t = threadIdx.x; t < RT; t += 128) mx = fmaxf(mx, tmax[b * RT + t]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  int e = 0;   // from the exponent bits; within [-126, 126]
   if (mx > 0.f) e = 13 - (((__float_as_int(mx) >> 23) & 0xff) - 127);
   e = e > 126 ? 126 : (e < -126 ? -126 : e);
-  const float sc = __int_as_float((e + 127) << 23);
-  for (int64_t i = threadIdx.x; i < M; i += blockDim.x) {
-    const float v = gb[i * ldg] * sc;
+  const int64_t i = rt * 128 + threadIdx.x;
+  if (i < M) {
+    const float v = g[(b * M + i) * ldg] * __int_as_float((e + 127) << 23);
     const __half hi = __float2half_rn(v);
     const __half lo = __float2half_rn(v - __half2float(hi));
     gpack[b * M + i] = static_cast<uint32_t>(__half_as_ushort(hi)) |
                        (static_cast<uint32_t>(__half_as_ushort(lo)) << 16);
   }
-  if (threadIdx.x == 0) gscale[b] = __int_as_float((127 - e) << 23);
+  if (rt == 0 && threadIdx.x == 0) gscale[b] = __int_as_float((127 - e) << 23);
 }
 
 // ------------------------------------------------------------------ host side
@@ -813,16 +832,15 @@ cudaError_t pack_records(const TcArgs& a, int64_t Nw, cudaStream_t s) {
 
 template <typename T>
 cudaError_t pack_values(const TcArgs& a, int c0, int CP, int64_t Nst, cudaStream_t s) {
-  const int64_t total = a.B * CP * a.N;
-  const int blocks = grid_for(total, 256);
+  const int blocks = grid_for(a.B * a.N, 128);
   const T* y = static_cast<const T*>(a.y);
   const T* rows = static_cast<const T*>(a.x);
   if (a.w_is_f32)
-    pack_values_kernel<float, T><<<blocks, 256, 0, s>>>(static_cast<const float*>(a.w), y, rows,
+    pack_values_kernel<float, T><<<blocks, 128, 0, s>>>(static_cast<const float*>(a.w), y, rows,
                                                         static_cast<__half*>(a.vt), a.B, a.N, Nst,
                                                         a.M, a.C, a.D, a.CV, c0, CP);
   else
-    pack_values_kernel<T, T><<<blocks, 256, 0, s>>>(static_cast<const T*>(a.w), y, rows,
+    pack_values_kernel<T, T><<<blocks, 128, 0, s>>>(static_cast<const T*>(a.w), y, rows,
                                                     static_cast<__half*>(a.vt), a.B, a.N, Nst, a.M,
                                                     a.C, a.D, a.CV, c0, CP);
   return cudaGetLastError();
@@ -967,8 +985,12 @@ cudaError_t launch_tc_sum(const TcArgs& a, cudaStream_t s) {
   const bool gw = a.gw_part != nullptr;
   if (gw) {
     // one fused sweep: the values in a single chunk of at most 48 channels
-    if (KP != 64 || a.CV > 48 || a.CV < 2) return cudaErrorInvalidValue;
-    pack_g_kernel<<<static_cast<unsigned>(a.B), 1024, 0, s>>>(a.g, a.g_ld, a.gpack, a.gscale, a.M);
+    const int64_t RT = (a.M + kBM - 1) / kBM;
+    if (KP != 64 || a.CV > 48 || a.CV < 2 || a.B > 65535 || RT > 0x7fffffff)
+      return cudaErrorInvalidValue;
+    const dim3 gg(static_cast<unsigned>(RT), static_cast<unsigned>(a.B));
+    g_tile_max_kernel<<<gg, 128, 0, s>>>(a.g, a.g_ld, a.gtmax, a.M, RT);
+    pack_g_kernel<<<gg, 128, 0, s>>>(a.g, a.g_ld, a.gtmax, a.gpack, a.gscale, a.M, RT);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
