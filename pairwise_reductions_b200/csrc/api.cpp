@@ -149,7 +149,9 @@ PassLayout pass_layout(const Pass& p, int sm) {
       off = align_up(off + size_t(L.f32.splits) * p.B * p.R * p.CV * 4);
     }
   } else if (!L.tc) {
-    L.sd = sd_plan(p.B, p.R, p.N, p.D, p.CV, sm, 256);
+    L.sd = sd_plan(p.B, p.R, p.N, p.D, p.CV, sm, 256,
+                   p.CV == 1 && p.D <= 3 &&
+                       (p.shift_mode == 0 || p.shift_mode == 2 || p.shift_mode == 3));
     if (p.vmode != 0) {
       L.off_vals = off;
       off = align_up(off + size_t(p.B) * p.N * p.CV * 4);

@@ -32,11 +32,15 @@ struct SdPlan {
   int rows_per_cta;    // kSdThreads * rows per thread
   int splits;          // j-splits (partials combined afterwards when > 1)
   int64_t cols_per_split;
+  int threads;         // threads per CTA: kSdThreads, or twice that (same rows per CTA)
 };
 
 // Choose rows per CTA and the j-split for the small-D kernel.
-// max_splits: 32 for the log-sum-exp (its finalize merges the splits in one warp)
-SdPlan sd_plan(int64_t B, int64_t M, int64_t N, int D, int64_t C, int sm_count, int max_splits);
+// max_splits: 32 for the log-sum-exp (its finalize merges the splits in one warp).
+// wide_ok: the 256-thread sum kernel may run this pass (one channel, D <= 3,
+// exponent modes 0, 2 and 3).
+SdPlan sd_plan(int64_t B, int64_t M, int64_t N, int D, int64_t C, int sm_count, int max_splits,
+               bool wide_ok = false);
 
 struct SdArgs {
   const float* x;

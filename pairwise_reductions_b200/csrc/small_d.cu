@@ -39,7 +39,6 @@ namespace gs {
 namespace {
 
 constexpr int kTileJ = 256;
-constexpr int kPer = kTileJ / kSdThreads;   // points each thread stages per tile
 constexpr float kLn2 = 0.69314718055994530942f;
 
 template <int D, int CP, int SHIFT = 0>
@@ -80,15 +79,25 @@ __host__ __device__ constexpr int sd_min_blocks(int D, int CP, int SHIFT) {
   return (CP == 1 && D <= 3 && SHIFT != 1 && SHIFT != 4) ? 8 : 1;
 }
 
-template <int D, int CP, bool LSE, int SHIFT>
-__global__ void __launch_bounds__(kSdThreads, sd_min_blocks(D, CP, SHIFT))
+// NT threads per CTA, the same kSdThreads * sd_rows_per_thread rows per CTA:
+// NT = 256 halves the rows of each thread and doubles the warps.  A grid of
+// one partial wave (too few CTAs to fill every SM with 128-thread CTAs) has
+// few warps per SM to hide the latency of the pair loop; measured at
+// M = N = 10^4 (730 CTAs of 128 threads): 16 warps per SM, MUFU busy 73% of
+// the active cycles.  (Register bound as for NT = 128: 64 a thread.)
+template <int D, int CP, bool LSE, int SHIFT, int NT>
+__global__ void __launch_bounds__(NT, sd_min_blocks(D, CP, SHIFT) * kSdThreads / NT)
     sd_kernel(const SdArgs a) {
-  constexpr int R = sd_rows_per_thread(D, CP);
+  constexpr int R = sd_rows_per_thread(D, CP) * kSdThreads / NT;
+  constexpr int kPer = kTileJ / NT;   // points each thread stages per tile
+  // a programmatic dependent (the split combine) may be scheduled as soon as
+  // every block of this grid has started; it waits for this grid to complete
+  asm volatile("griddepcontrol.launch_dependents;");
   constexpr int RP = R / 2;                     // row pairs per thread
   constexpr int NPOLY = poly_pairs<D, CP, R>();
   constexpr int PK = PackShape<D, CP, SHIFT>::PK;
   static_assert(!(LSE && SHIFT), "shifts apply to the sum kernel");
-  constexpr int NW = kSdThreads / 32;
+  constexpr int NW = NT / 32;
   static_assert(R % 2 == 0, "rows are processed in pairs");
   __shared__ __align__(16) float tile[kTileJ * PK];
   __shared__ float red[NW][CP];
@@ -97,7 +106,7 @@ __global__ void __launch_bounds__(kSdThreads, sd_min_blocks(D, CP, SHIFT))
   const int lane = tid & 31, warp = tid >> 5;
   const int64_t b = blockIdx.z;
   const int split = blockIdx.y;
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * (kSdThreads * R);
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * (NT * R);
   const int64_t jbeg = static_cast<int64_t>(split) * a.plan.cols_per_split;
   const int64_t jend = min(a.N, jbeg + a.plan.cols_per_split);
   const float* __restrict__ yb = a.y + b * a.N * D;
@@ -107,8 +116,8 @@ __global__ void __launch_bounds__(kSdThreads, sd_min_blocks(D, CP, SHIFT))
   uint64_t xs[RP][D];
 #pragma unroll
   for (int q = 0; q < RP; ++q) {
-    const int64_t i0 = row0 + tid + (2 * q) * kSdThreads;
-    const int64_t i1 = i0 + kSdThreads;
+    const int64_t i0 = row0 + tid + (2 * q) * NT;
+    const int64_t i1 = i0 + NT;
 #pragma unroll
     for (int k = 0; k < D; ++k) {
       const float v0 = (i0 < a.M) ? a.x[(b * a.M + i0) * D + k] * a.scale : 0.f;
@@ -120,8 +129,8 @@ __global__ void __launch_bounds__(kSdThreads, sd_min_blocks(D, CP, SHIFT))
 #pragma unroll
   for (int q = 0; q < RP; ++q) {
     if constexpr (SHIFT == 1 || SHIFT == 4) {
-      const int64_t i0 = row0 + tid + (2 * q) * kSdThreads;
-      const int64_t i1 = i0 + kSdThreads;
+      const int64_t i0 = row0 + tid + (2 * q) * NT;
+      const int64_t i1 = i0 + NT;
       const float s0 = (i0 < a.M) ? a.shift_scale * a.shift_src[(b * a.M + i0) * a.shift_ld + a.shift_c] : 0.f;
       const float s1 = (i1 < a.M) ? a.shift_scale * a.shift_src[(b * a.M + i1) * a.shift_ld + a.shift_c] : 0.f;
       rho[q] = pk2(s0, s1);
@@ -143,7 +152,7 @@ __global__ void __launch_bounds__(kSdThreads, sd_min_blocks(D, CP, SHIFT))
     float sy[kPer][D], sv[kPer][CP], sk[kPer];
 #pragma unroll
     for (int q = 0; q < kPer; ++q) {
-      const int64_t j = j0 + tid + q * kSdThreads;
+      const int64_t j = j0 + tid + q * NT;
       const bool ok = j < jend;
       if constexpr (SHIFT == 2)
         sk[q] = ok ? a.shift_scale * a.shift_src[(b * a.N + j) * a.shift_ld + a.shift_c] : 0.f;
@@ -191,7 +200,7 @@ __global__ void __launch_bounds__(kSdThreads, sd_min_blocks(D, CP, SHIFT))
     }
 #pragma unroll
     for (int q = 0; q < kPer; ++q) {
-      float* p = tile + (tid + q * kSdThreads) * PK;
+      float* p = tile + (tid + q * NT) * PK;
 #pragma unroll
       for (int k = 0; k < D; ++k) {
         p[2 * k] = sy[q][k];
@@ -280,7 +289,7 @@ __global__ void __launch_bounds__(kSdThreads, sd_min_blocks(D, CP, SHIFT))
   for (int q = 0; q < RP; ++q) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int64_t i = row0 + tid + (2 * q + h) * kSdThreads;
+      const int64_t i = row0 + tid + (2 * q + h) * NT;
       if (i >= a.M) continue;
       const int64_t base = split * a.split_stride + (b * a.M + i) * a.ldo + a.c0;
 #pragma unroll
@@ -306,15 +315,27 @@ cudaError_t launch_t(const SdArgs& a, cudaStream_t s) {
   const int64_t tiles = (a.M + kSdThreads * R - 1) / (kSdThreads * R);
   dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(a.plan.splits),
             static_cast<unsigned>(a.B));
+  constexpr bool kWide = !LSE && sd_min_blocks(D, CP, 0) == 8;   // NT = 256 instantiated
   if constexpr (LSE) {
-    sd_kernel<D, CP, true, 0><<<grid, kSdThreads, 0, s>>>(a);
+    sd_kernel<D, CP, true, 0, kSdThreads><<<grid, kSdThreads, 0, s>>>(a);
   } else {
+    if constexpr (kWide) {
+      if (a.plan.threads == 2 * kSdThreads && (a.shift_mode == 0 || a.shift_mode == 2 ||
+                                               a.shift_mode == 3)) {
+        switch (a.shift_mode) {
+          case 2: sd_kernel<D, CP, false, 2, 2 * kSdThreads><<<grid, 2 * kSdThreads, 0, s>>>(a); break;
+          case 3: sd_kernel<D, CP, false, 3, 2 * kSdThreads><<<grid, 2 * kSdThreads, 0, s>>>(a); break;
+          default: sd_kernel<D, CP, false, 0, 2 * kSdThreads><<<grid, 2 * kSdThreads, 0, s>>>(a); break;
+        }
+        return cudaGetLastError();
+      }
+    }
     switch (a.shift_mode) {
-      case 1: sd_kernel<D, CP, false, 1><<<grid, kSdThreads, 0, s>>>(a); break;
-      case 2: sd_kernel<D, CP, false, 2><<<grid, kSdThreads, 0, s>>>(a); break;
-      case 3: sd_kernel<D, CP, false, 3><<<grid, kSdThreads, 0, s>>>(a); break;
-      case 4: sd_kernel<D, CP, false, 4><<<grid, kSdThreads, 0, s>>>(a); break;
-      default: sd_kernel<D, CP, false, 0><<<grid, kSdThreads, 0, s>>>(a); break;
+      case 1: sd_kernel<D, CP, false, 1, kSdThreads><<<grid, kSdThreads, 0, s>>>(a); break;
+      case 2: sd_kernel<D, CP, false, 2, kSdThreads><<<grid, kSdThreads, 0, s>>>(a); break;
+      case 3: sd_kernel<D, CP, false, 3, kSdThreads><<<grid, kSdThreads, 0, s>>>(a); break;
+      case 4: sd_kernel<D, CP, false, 4, kSdThreads><<<grid, kSdThreads, 0, s>>>(a); break;
+      default: sd_kernel<D, CP, false, 0, kSdThreads><<<grid, kSdThreads, 0, s>>>(a); break;
     }
   }
   return cudaGetLastError();
@@ -348,13 +369,17 @@ cudaError_t launch_d(const SdArgs& a, cudaStream_t s) {
 // ------------------------------------------------------------------ combine
 // out[e] = sum_k part[k * total + e] in the fixed order of combine.cuh.  A block
 // takes 32 consecutive elements with one warp per lane of that order: warp l
-// sums splits l, l + 8, ... in turn (reading 128 contiguous bytes of a split
-// at a time), then the 8 lane sums are added in lane order.  Eight short
-// chains instead of one long one keep the loads of many splits in flight.
+// sums splits l, l + kCombineLanes, ... in turn (reading 128 contiguous bytes
+// of a split at a time, four splits' loads in flight at once), then the lane
+// sums are added in lane order.
+// Launched as a programmatic dependent of the pass that wrote the partials:
+// its blocks may start while that kernel drains, and griddepcontrol.wait holds
+// them until it has completed and its stores are visible.
 __global__ void __launch_bounds__(32 * kCombineLanes)
     combine_sum_kernel(const float* __restrict__ part, int splits, int64_t total,
                        float* __restrict__ out) {
   __shared__ float red[kCombineLanes][33];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   for (int64_t e0 = blockIdx.x * 32ll; e0 < total; e0 += gridDim.x * 32ll) {
     const int64_t e = e0 + tx;
@@ -486,8 +511,10 @@ int grid_for(int64_t n, int threads) {
 
 }  // namespace
 
-SdPlan sd_plan(int64_t B, int64_t M, int64_t N, int D, int64_t C, int sm_count, int max_splits) {
+SdPlan sd_plan(int64_t B, int64_t M, int64_t N, int D, int64_t C, int sm_count, int max_splits,
+               bool wide_ok) {
   SdPlan p{};
+  p.threads = kSdThreads;
   const int cw = static_cast<int>(C < kSdMaxChunk ? C : kSdMaxChunk);
   const int R = sd_rows_per_thread(D, sd_chunk_pad(cw));
   p.rows_per_cta = kSdThreads * R;
@@ -519,6 +546,17 @@ SdPlan sd_plan(int64_t B, int64_t M, int64_t N, int D, int64_t C, int sm_count, 
       best = static_cast<int>(S);
     }
   }
+  // One partial wave of 128-thread CTAs leaves too few warps per SM to keep
+  // MUFU busy: 256-thread CTAs (4 resident per SM at 64 registers), and the
+  // split count that fills one wave of them.
+  if (wide_ok && static_cast<double>(U * best) < wave) {
+    int64_t s2 = static_cast<int64_t>(sm_count) * 4 / U;
+    if (s2 > smax) s2 = smax;
+    if (s2 >= 1) {
+      best = static_cast<int>(s2);
+      p.threads = 2 * kSdThreads;
+    }
+  }
   p.cols_per_split = (N + best - 1) / best;
   // keep every split non-empty
   if (p.cols_per_split < 1) p.cols_per_split = 1;
@@ -532,8 +570,16 @@ cudaError_t launch_small_d_lse(const SdArgs& a, cudaStream_t s) { return launch_
 
 cudaError_t launch_combine_sum(const float* part, int splits, int64_t total, float* out,
                                cudaStream_t s) {
-  combine_sum_kernel<<<grid_for(total, 32), 32 * kCombineLanes, 0, s>>>(part, splits, total, out);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid_for(total, 32)));
+  cfg.blockDim = dim3(32 * kCombineLanes);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_sum_kernel, part, splits, total, out);
 }
 
 cudaError_t launch_lse_finalize(const LseFinalizeArgs& a, cudaStream_t s) {

@@ -133,6 +133,8 @@ HALF_SHAPES = [
     (1, 70, 1200, 63, 3), (1, 129, 257, 126, 96), (1, 300, 700, 127, 1), (2, 257, 390, 128, 50),
     # D + 2 at and just past a multiple of 16 (the similarity MMA's K steps)
     (1, 300, 500, 14, 2), (1, 260, 530, 30, 4), (1, 200, 400, 31, 1), (1, 150, 300, 46, 1),
+    # one and two column tiles with several channels (the three-buffer S ring's edges)
+    (1, 300, 100, 32, 8), (2, 130, 128, 20, 40), (1, 257, 250, 62, 64),
 ]
 # fp32 with D > 8: the split-tf32 tensor-core path (every packed-row width, one
 # and two value passes, single and several column tiles per warpgroup)
