@@ -13,21 +13,14 @@ namespace gs {
 
 constexpr int kCombineLanes = 8;
 
-// Lane l's sum (sequential, starting from 0), its loads issued four at a time.
+// Lane l's sum (sequential, starting from 0).  A plain loop: the compiler
+// keeps several of its loads in flight with few registers (measured faster
+// than explicit batches of four or eight loads, whose extra registers cost
+// resident warps).
 __device__ __forceinline__ float split_lane_sum(const float* __restrict__ p, int lane_l, int splits,
                                                 int64_t stride) {
   float s = 0.f;
-  for (int k0 = lane_l; k0 < splits; k0 += 4 * kCombineLanes) {
-    float v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int k = k0 + u * kCombineLanes;
-      v[u] = k < splits ? p[k * stride] : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (k0 + u * kCombineLanes < splits) s += v[u];
-  }
+  for (int k = lane_l; k < splits; k += kCombineLanes) s += p[k * stride];
   return s;
 }
 

@@ -103,32 +103,78 @@ __global__ void grad_x_epilogue_kernel(const T* __restrict__ x, const float* __r
 // combine followed by grad_x_epilogue_kernel bit for bit:
 //     s = sum_k part[k][b,i,:],  out[b,i] = s[0],
 //     dL/dx[b,i,k] = -tau g_i ((x_ik - z_k) s[0] - s[1 + k]).
-// One warp per row; lanes over the D dimensions (coalesced reads of x, of each
-// split's sums and of the gradient row).
+// A block takes `tile_rows` consecutive rows at a time.  Their C V sums in each
+// split slice are one contiguous run of floats: the block copies every slice's
+// run into shared memory with coalesced loads, eight independent loads in
+// flight per thread, then sums each element over the splits there in the fixed
+// order (the same split_sum, on shared memory), and computes dL/dx with a warp
+// per row.
+constexpr int kEpiMaxRows = 32;
+constexpr int kEpiThreads = 256;
+constexpr int kEpiSmemFloats = 12 * 1024;   // 48 KB: splits + 1 runs of tile_rows * CV floats
+
 template <typename T>
-__global__ void fwd_bwd_epilogue_kernel(const T* __restrict__ x, const float* __restrict__ g,
-                                        const float* __restrict__ part, int splits,
-                                        int64_t stride, float* __restrict__ out,
-                                        float* __restrict__ gx, int64_t B, int64_t M, int D,
-                                        int CV, float tau) {
-  const int lane = threadIdx.x & 31;
+__global__ void __launch_bounds__(kEpiThreads)
+    fwd_bwd_epilogue_kernel(const T* __restrict__ x, const float* __restrict__ g,
+                            const float* __restrict__ part, int splits, int64_t stride,
+                            float* __restrict__ out, float* __restrict__ gx, int64_t B, int64_t M,
+                            int D, int CV, float tau, int tile_rows) {
+  extern __shared__ float sm[];   // [splits][tile_rows * CV] copies, then [tile_rows * CV] sums
+  __shared__ int64_t zoff[kEpiMaxRows];
+  const int tid = threadIdx.x;
   const int64_t rows = B * M;
-  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
-       r < rows; r += warps) {
-    const int64_t b = r / M;
-    const float* o = part + r * CV;
-    const float s0 = split_sum(o, splits, stride);
-    if (lane == 0 && out) out[r] = s0;
-    if (!gx) continue;
-    const float gi = g[r];
-    const T* xi = x + r * D;
-    const T* z = x + b * M * D;
-    for (int k = lane; k < D; k += 32) {
-      const float xk = tf(xi[k]) - tf(z[k]);
-      const float t = gi * fmaf(xk, s0, -split_sum(o + 1 + k, splits, stride));
-      gx[r * D + k] = -tau * t;
+  for (int64_t r0 = blockIdx.x * static_cast<int64_t>(tile_rows); r0 < rows;
+       r0 += static_cast<int64_t>(gridDim.x) * tile_rows) {
+    const int nr = static_cast<int>(min(static_cast<int64_t>(tile_rows), rows - r0));
+    const int ne = nr * CV;
+    const int n = splits * ne;
+    const float* base = part + r0 * CV;
+    // thread tid copies elements tid, tid + 256, ... of the concatenated runs:
+    // (l, e) = split and offset of the next one, src = split l's run
+    int l = tid / ne, e = tid - l * ne;
+    const float* src = base + l * stride;
+    constexpr int kPer = 8;
+    for (int i0 = tid; i0 < n; i0 += kPer * kEpiThreads) {
+      float v[kPer];
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        v[u] = (i0 + u * kEpiThreads < n) ? src[e] : 0.f;
+        e += kEpiThreads;
+        while (e >= ne) {
+          e -= ne;
+          src += stride;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int idx = i0 + u * kEpiThreads;
+        if (idx < n) sm[idx] = v[u];
+      }
     }
+    if (tid < nr) zoff[tid] = ((r0 + tid) / M) * M * D;   // the batch's first row point
+    __syncthreads();
+    float* sums = sm + n;
+    for (int e2 = tid; e2 < ne; e2 += kEpiThreads) sums[e2] = split_sum(sm + e2, splits, ne);
+    __syncthreads();
+    if (out)
+      for (int i = tid; i < nr; i += kEpiThreads) out[r0 + i] = sums[i * CV];
+    if (gx) {
+      // a warp per row, lanes over the dimensions
+      const int warp = tid >> 5, lane = tid & 31;
+      for (int i = warp; i < nr; i += kEpiThreads / 32) {
+        const int64_t r = r0 + i;
+        const float gi = g[r], s0 = sums[i * CV];
+        const T* xr = x + r * D;
+        const T* zr = x + zoff[i];
+        float* gr = gx + r * D;
+        for (int k = lane; k < D; k += 32) {
+          const float xk = tf(xr[k]) - tf(zr[k]);
+          const float t = gi * fmaf(xk, s0, -sums[i * CV + 1 + k]);
+          gr[k] = -tau * t;
+        }
+      }
+    }
+    __syncthreads();
   }
 }
 
@@ -313,22 +359,27 @@ cudaError_t launch_fwd_bwd_epilogue(const void* x, gs_dtype dt, const float* g, 
                                     int splits, int64_t stride, float* out, float* grad_x,
                                     int64_t B, int64_t M, int D, int CV, float tau,
                                     cudaStream_t s) {
-  int64_t blocks = (B * M + 7) / 8;   // 8 warps a block, one row each
+  // rows a tile: as many as the (splits + 1) runs of CV floats leave room for
+  const int64_t fit = kEpiSmemFloats / (static_cast<int64_t>(splits + 1) * CV);
+  if (fit < 1) return cudaErrorInvalidValue;   // splits and CV are bounded far below this
+  const int tile_rows = static_cast<int>(fit < kEpiMaxRows ? fit : kEpiMaxRows);
+  int64_t blocks = (B * M + tile_rows - 1) / tile_rows;
   if (blocks > 148 * 64) blocks = 148 * 64;
   if (blocks < 1) blocks = 1;
   const unsigned nb = static_cast<unsigned>(blocks);
+  const size_t smem = sizeof(float) * static_cast<size_t>(splits + 1) * tile_rows * CV;
   switch (dt) {
     case GS_F32:
-      fwd_bwd_epilogue_kernel<float><<<nb, 256, 0, s>>>(as<float>(x), g, part, splits, stride, out,
-                                                        grad_x, B, M, D, CV, tau);
+      fwd_bwd_epilogue_kernel<float><<<nb, kEpiThreads, smem, s>>>(
+          as<float>(x), g, part, splits, stride, out, grad_x, B, M, D, CV, tau, tile_rows);
       break;
     case GS_F16:
-      fwd_bwd_epilogue_kernel<__half><<<nb, 256, 0, s>>>(as<__half>(x), g, part, splits, stride, out,
-                                                         grad_x, B, M, D, CV, tau);
+      fwd_bwd_epilogue_kernel<__half><<<nb, kEpiThreads, smem, s>>>(
+          as<__half>(x), g, part, splits, stride, out, grad_x, B, M, D, CV, tau, tile_rows);
       break;
     default:
-      fwd_bwd_epilogue_kernel<__nv_bfloat16><<<nb, 256, 0, s>>>(
-          as<__nv_bfloat16>(x), g, part, splits, stride, out, grad_x, B, M, D, CV, tau);
+      fwd_bwd_epilogue_kernel<__nv_bfloat16><<<nb, kEpiThreads, smem, s>>>(
+          as<__nv_bfloat16>(x), g, part, splits, stride, out, grad_x, B, M, D, CV, tau, tile_rows);
       break;
   }
   return cudaGetLastError();

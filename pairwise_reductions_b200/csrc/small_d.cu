@@ -370,8 +370,7 @@ cudaError_t launch_d(const SdArgs& a, cudaStream_t s) {
 // out[e] = sum_k part[k * total + e] in the fixed order of combine.cuh.  A block
 // takes 32 consecutive elements with one warp per lane of that order: warp l
 // sums splits l, l + kCombineLanes, ... in turn (reading 128 contiguous bytes
-// of a split at a time, four splits' loads in flight at once), then the lane
-// sums are added in lane order.
+// of a split at a time), then the lane sums are added in lane order.
 // Launched as a programmatic dependent of the pass that wrote the partials:
 // its blocks may start while that kernel drains, and griddepcontrol.wait holds
 // them until it has completed and its stores are visible.

@@ -644,15 +644,23 @@ __device__ __forceinline__ uint16_t bits16(__nv_bfloat16 v) { return __bfloat16_
 
 // Packed operand rows.  Row side (is_x): [x, 1, 1, 0 ...] and
 // rnorm = -c |x|^2 + shift.  Column side: [y, h, l, 0 ...] with h + l = -|y|^2/2.
-// A group of 8 consecutive threads builds one row, KP/8 elements each, written
-// as 8-element (16-byte) pieces: thread `part` owns pieces part, part + 8, ...
+// Both sides in one launch: blocks below `blocks_x` pack the rows, the rest the
+// columns.  A group of 8 consecutive threads builds one row, KP/8 elements
+// each, written as 8-element (16-byte) pieces: thread `part` owns pieces part,
+// part + 8, ...
 template <typename T, int KP>
-__global__ void pack_rows_kernel(const T* __restrict__ src, T* __restrict__ dst,
-                                 float* __restrict__ rnorm, int64_t rows, int D, float c,
-                                 float shift, int is_x) {
+__global__ void pack_rows_kernel(const T* __restrict__ src_x, T* __restrict__ dst_x,
+                                 float* __restrict__ rnorm, int64_t rows_x,
+                                 const T* __restrict__ src_y, T* __restrict__ dst_y,
+                                 int64_t rows_y, int64_t blocks_x, int D, float c, float shift) {
   constexpr int G = 8;          // threads per row
   constexpr int NPC = KP / 64;  // pieces per thread (1, 2 or 3)
-  const int64_t gt = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const bool is_x = blockIdx.x < blocks_x;
+  const T* __restrict__ src = is_x ? src_x : src_y;
+  T* __restrict__ dst = is_x ? dst_x : dst_y;
+  const int64_t rows = is_x ? rows_x : rows_y;
+  const int64_t blk = is_x ? static_cast<int64_t>(blockIdx.x) : blockIdx.x - blocks_x;
+  const int64_t gt = blk * blockDim.x + threadIdx.x;
   const int64_t row = gt / G;
   const int part = static_cast<int>(gt % G);
   const bool live = row < rows;
@@ -703,20 +711,25 @@ __global__ void pack_rows_kernel(const T* __restrict__ src, T* __restrict__ dst,
 // Transposed fp16 value matrix v^T [B, CP, Nst] for channels [c0, c0 + CP) of
 // the pass's value matrix (values.cuh; columns = the y side of this pass,
 // centre = its first row point).  Channels past CV are written as zeros.
-// One thread per column (b, j), all CP channels: consecutive threads take
-// consecutive j, so each channel's store is coalesced, and the column's point
-// and weights are read once.
+// One thread per column (b, j) and group of kPackGroup channels (blockIdx.y):
+// consecutive threads take consecutive j, so each channel's store is
+// coalesced, and a thread reads its column's point and weights once for the
+// channels of its group.
+constexpr int kPackGroup = 16;
+
 template <typename TW, typename TY>
 __global__ void pack_values_kernel(const TW* __restrict__ w, const TY* __restrict__ y,
                                    const TY* __restrict__ rows, __half* __restrict__ vt, int64_t B,
                                    int64_t N, int64_t Nst, int64_t Mrows, int C, int D, int CV,
                                    int c0, int CP) {
   const int64_t total = B * N;
+  const int g0 = blockIdx.y * kPackGroup;
+  const int g1 = min(CP, g0 + kPackGroup);
   for (int64_t bj = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; bj < total;
        bj += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t b = bj / N, j = bj - b * N;
     __half* dst = vt + b * CP * Nst + j;
-    for (int cc = 0; cc < CP; ++cc) {
+    for (int cc = g0; cc < g1; ++cc) {
       const int ch = c0 + cc;
       const float v = (ch < CV) ? value_at(w, y, rows, b, bj, Mrows, D, C, ch, C) : 0.f;
       dst[cc * Nst] = __float2half_rn(v);
@@ -798,20 +811,23 @@ template <typename T>
 cudaError_t pack_operands(const TcArgs& a, cudaStream_t s) {
   const float c = 0.5f * a.tau * kLog2e;
   const int KP = a.plan.KP;
-  auto launch_rows = [&](const void* src, void* dst, float* rn, int64_t rows, int is_x) {
-    const int64_t threads_total = rows * 8;
-    const int blocks = static_cast<int>((threads_total + 255) / 256);
-    const T* sp = static_cast<const T*>(src);
-    T* dp = static_cast<T*>(dst);
-    if (KP == 64)
-      pack_rows_kernel<T, 64><<<blocks, 256, 0, s>>>(sp, dp, rn, rows, a.D, c, kPShift, is_x);
-    else if (KP == 128)
-      pack_rows_kernel<T, 128><<<blocks, 256, 0, s>>>(sp, dp, rn, rows, a.D, c, kPShift, is_x);
-    else
-      pack_rows_kernel<T, 192><<<blocks, 256, 0, s>>>(sp, dp, rn, rows, a.D, c, kPShift, is_x);
-  };
-  launch_rows(a.x, a.xpack, a.rnorm, a.B * a.M, 1);
-  launch_rows(a.y, a.ypack, nullptr, a.B * a.N, 0);
+  const int64_t rows_x = a.B * a.M, rows_y = a.B * a.N;
+  const int64_t blocks_x = (rows_x * 8 + 255) / 256, blocks_y = (rows_y * 8 + 255) / 256;
+  if (blocks_x + blocks_y > 0x7fffffff) return cudaErrorInvalidValue;
+  const unsigned blocks = static_cast<unsigned>(blocks_x + blocks_y);
+  const T* xs = static_cast<const T*>(a.x);
+  const T* ys = static_cast<const T*>(a.y);
+  T* xd = static_cast<T*>(a.xpack);
+  T* yd = static_cast<T*>(a.ypack);
+  if (KP == 64)
+    pack_rows_kernel<T, 64><<<blocks, 256, 0, s>>>(xs, xd, a.rnorm, rows_x, ys, yd, rows_y, blocks_x,
+                                                   a.D, c, kPShift);
+  else if (KP == 128)
+    pack_rows_kernel<T, 128><<<blocks, 256, 0, s>>>(xs, xd, a.rnorm, rows_x, ys, yd, rows_y, blocks_x,
+                                                    a.D, c, kPShift);
+  else
+    pack_rows_kernel<T, 192><<<blocks, 256, 0, s>>>(xs, xd, a.rnorm, rows_x, ys, yd, rows_y, blocks_x,
+                                                    a.D, c, kPShift);
   return cudaGetLastError();
 }
 
@@ -832,7 +848,7 @@ cudaError_t pack_records(const TcArgs& a, int64_t Nw, cudaStream_t s) {
 
 template <typename T>
 cudaError_t pack_values(const TcArgs& a, int c0, int CP, int64_t Nst, cudaStream_t s) {
-  const int blocks = grid_for(a.B * a.N, 128);
+  const dim3 blocks(grid_for(a.B * a.N, 128), (CP + kPackGroup - 1) / kPackGroup);
   const T* y = static_cast<const T*>(a.y);
   const T* rows = static_cast<const T*>(a.x);
   if (a.w_is_f32)
