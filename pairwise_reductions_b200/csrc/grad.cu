@@ -121,6 +121,8 @@ __global__ void __launch_bounds__(kEpiThreads)
                             int D, int CV, float tau, int tile_rows) {
   extern __shared__ float sm[];   // [splits][tile_rows * CV] copies, then [tile_rows * CV] sums
   __shared__ int64_t zoff[kEpiMaxRows];
+  // a programmatic dependent of the kernel before it: wait for its results
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int tid = threadIdx.x;
   const int64_t rows = B * M;
   for (int64_t r0 = blockIdx.x * static_cast<int64_t>(tile_rows); r0 < rows;
@@ -368,21 +370,27 @@ cudaError_t launch_fwd_bwd_epilogue(const void* x, gs_dtype dt, const float* g, 
   if (blocks < 1) blocks = 1;
   const unsigned nb = static_cast<unsigned>(blocks);
   const size_t smem = sizeof(float) * static_cast<size_t>(splits + 1) * tile_rows * CV;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(nb);
+  cfg.blockDim = dim3(kEpiThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   switch (dt) {
     case GS_F32:
-      fwd_bwd_epilogue_kernel<float><<<nb, kEpiThreads, smem, s>>>(
-          as<float>(x), g, part, splits, stride, out, grad_x, B, M, D, CV, tau, tile_rows);
-      break;
+      return cudaLaunchKernelEx(&cfg, fwd_bwd_epilogue_kernel<float>, as<float>(x), g, part, splits,
+                                stride, out, grad_x, B, M, D, CV, tau, tile_rows);
     case GS_F16:
-      fwd_bwd_epilogue_kernel<__half><<<nb, kEpiThreads, smem, s>>>(
-          as<__half>(x), g, part, splits, stride, out, grad_x, B, M, D, CV, tau, tile_rows);
-      break;
+      return cudaLaunchKernelEx(&cfg, fwd_bwd_epilogue_kernel<__half>, as<__half>(x), g, part,
+                                splits, stride, out, grad_x, B, M, D, CV, tau, tile_rows);
     default:
-      fwd_bwd_epilogue_kernel<__nv_bfloat16><<<nb, kEpiThreads, smem, s>>>(
-          as<__nv_bfloat16>(x), g, part, splits, stride, out, grad_x, B, M, D, CV, tau, tile_rows);
-      break;
+      return cudaLaunchKernelEx(&cfg, fwd_bwd_epilogue_kernel<__nv_bfloat16>, as<__nv_bfloat16>(x),
+                                g, part, splits, stride, out, grad_x, B, M, D, CV, tau, tile_rows);
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_grad_x_epilogue(const void* x, gs_dtype dt, const float* g, const float* o,

@@ -379,6 +379,7 @@ __global__ void __launch_bounds__(32 * kCombineLanes)
                        float* __restrict__ out) {
   __shared__ float red[kCombineLanes][33];
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   for (int64_t e0 = blockIdx.x * 32ll; e0 < total; e0 += gridDim.x * 32ll) {
     const int64_t e = e0 + tx;

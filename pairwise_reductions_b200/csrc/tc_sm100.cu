@@ -255,6 +255,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Launched as a programmatic dependent of the packing kernel: the set-up
+  // above overlaps its tail; the packed operands are read only after it has
+  // completed.  The next kernel (the split combine) may be scheduled now.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -722,6 +727,7 @@ __global__ void pack_values_kernel(const TW* __restrict__ w, const TY* __restric
                                    const TY* __restrict__ rows, __half* __restrict__ vt, int64_t B,
                                    int64_t N, int64_t Nst, int64_t Mrows, int C, int D, int CV,
                                    int c0, int CP) {
+  asm volatile("griddepcontrol.launch_dependents;");   // the sweep may set up meanwhile
   const int64_t total = B * N;
   const int g0 = blockIdx.y * kPackGroup;
   const int g1 = min(CP, g0 + kPackGroup);
@@ -743,6 +749,7 @@ template <typename TW, typename TY>
 __global__ void pack_records_kernel(const TW* __restrict__ w, const TY* __restrict__ y,
                                     const TY* __restrict__ rows, float* __restrict__ rec, int64_t B,
                                     int64_t N, int64_t Nw, int64_t Mrows, int C, int D) {
+  asm volatile("griddepcontrol.launch_dependents;");   // the sweep may set up meanwhile
   const int64_t total = B * Nw;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -873,8 +880,17 @@ cudaError_t launch_kernel(const CUtensorMap& tx, const CUtensorMap& ty, const CU
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  fn<<<grid, kThreads, Cfg::SMEM, s>>>(tx, ty, tv, kp);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Cfg::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fn, tx, ty, tv, kp);
 }
 
 // The forward + backward sweep: 64-wide packed rows, one chunk of 16, 32 or 48
