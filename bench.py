@@ -314,9 +314,16 @@ def oracle_sample(w, inp, seconds, seed=1234):
             oracle.gauss_sum_bwd(x, y, wt, g, w.tau, rows=rows, wrows=rows % w.N)
         return time.perf_counter() - t0
 
+    # size the sample in two probes: 16 rows carry the start-up costs, so a
+    # second probe of about a tenth of the target corrects the per-row time
     probe = synth.sample_rows(w.M, 16, seed).numpy()
     t = max(run(probe), 1e-3)
-    n = int(min(w.M, max(16, 16 * seconds / t)))
+    n1 = int(min(w.M, max(16, 16 * 0.1 * seconds / t)))
+    if n1 > 16:
+        t1 = max(run(synth.sample_rows(w.M, n1, seed).numpy()), 1e-3)
+        n = int(min(w.M, max(16, n1 * seconds / t1)))
+    else:
+        n = int(min(w.M, max(16, 16 * seconds / t)))
     rows = synth.sample_rows(w.M, n, seed).numpy()
     dt = run(rows)
     pairs = w.B * n * w.N * (("sum" in w.ops or "bwd" in w.ops) + ("lse" in w.ops))

@@ -112,8 +112,10 @@ struct F32Cfg {
   // small products of S in separate accumulators for each warpgroup (two
   // independent MMA chains; the small ones never round against the large
   // sum).  Tensor-core values: one S (small products first, then the large
-  // ones), P hi/lo (fp16 pairs: bn / 2 columns each) and O per warpgroup.
-  static constexpr int tmem_acc(int bn) { return REG ? 4 * bn : 4 * bn + 2 * CPA; }
+  // ones), P hi/lo (fp16 pairs: bn / 2 columns each) and O per warpgroup, O as
+  // two halves of CP columns: O_big (P_hi v_hi + P_lo v_hi) and O_small
+  // (P_hi v_lo), added in the epilogue.
+  static constexpr int tmem_acc(int bn) { return REG ? 4 * bn : 4 * bn + 4 * CPA; }
   // The x' rows (2 K' <= 32 KA columns) sit in TMEM as the A operand of the
   // similarity MMAs when the accumulators leave room, else in shared memory.
   static constexpr bool xt(int bn) { return tmem_acc(bn) + 32 * KA <= 512; }
@@ -143,16 +145,20 @@ struct F32Cfg {
   // at least ~120 KB: one CTA per SM, so the 512-column TMEM allocation never waits
   static constexpr int SMEM = SMEM_RAW < 122880 ? 122880 : SMEM_RAW;
   // TMEM columns.  Register values: Sbig0 | Sbig1 | Ssmall0 | Ssmall1 | x'.
-  // Tensor-core values: S0 | S1 | Phi0 | Phi1 | Plo0 | Plo1 | O0 | O1 | x'.
+  // Tensor-core values: S0 | S1 | Phi0 | Phi1 | Plo0 | Plo1 | O0 | O1 | x', O_h as
+  // [O_big (CP) | O_small (CP)] in 2 CPA columns.
   __host__ __device__ static constexpr uint32_t col_s(int h) { return h * BN; }
   __host__ __device__ static constexpr uint32_t col_ss(int h) { return 2 * BN + h * BN; }
   __host__ __device__ static constexpr uint32_t col_phi(int h) { return 2 * BN + (BN / 2) * h; }
   __host__ __device__ static constexpr uint32_t col_plo(int h) { return 3 * BN + (BN / 2) * h; }
-  __host__ __device__ static constexpr uint32_t col_o(int h) { return 4 * BN + CPA * h; }
+  __host__ __device__ static constexpr uint32_t col_o(int h) { return 4 * BN + 2 * CPA * h; }
   static constexpr uint32_t COL_X = tmem_acc(BN);
   static_assert(NST >= 2, "shared memory budget");
   static_assert(tmem_acc(BN) + (XT ? 32 * KA : 0) <= 512, "TMEM budget");
   static_assert(REG || (CP % 16 == 0 && CP >= 16 && CP <= 64), "value chunk");
+  // P_hi [v_hi ; v_lo] reads the hi and lo value atoms as one operand of 2 CP
+  // rows: they must be adjacent, one atom each (tiles of at most 64 columns)
+  static_assert(REG || VA == 1, "value atoms of a stage");
   static_assert(SMEM_RAW <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -379,19 +385,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma(db, ks, kdesc(sy, BN * 128, ks), (SPLIT || ks > 0) ? 1u : 0u);
         }
       };
+      // O_h += P_hi [v_hi ; v_lo] (one MMA of N = 2 CP: O_big and O_small at
+      // once, as cheap as one of N = CP) and P_lo v_hi into O_big: two MMAs a
+      // K step where three products of N = CP were three.
+      const uint32_t idO2 = idesc_f16(0, kBM, 2 * CP);
       auto issue_O = [&](int h, int st, bool acc_prev) {
         const uint8_t* sv = sStage + st * Cfg::STAGE + Cfg::Y_BYTES + Cfg::QW_BYTES;
         const uint32_t d = tmem + Cfg::col_o(h);
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks) {   // K steps of 16 columns
-          const int a = ks >> 2, within = (ks & 3) * 32;
-          const uint64_t bh = desc_k_sw128(smem_u32(sv + a * Cfg::V_ATOM) + within);
-          const uint64_t bl = desc_k_sw128(smem_u32(sv + (Cfg::VA + a) * Cfg::V_ATOM) + within);
+          const int within = ks * 32;
+          // rows 0 .. CP-1 the hi atom, CP .. 2 CP-1 the lo atom right after it
+          const uint64_t bhl = desc_k_sw128(smem_u32(sv) + within);
           const uint32_t phi = tmem + Cfg::col_phi(h) + ks * 8;
           const uint32_t plo = tmem + Cfg::col_plo(h) + ks * 8;
-          mma_ts(d, plo, bh, idO, (acc_prev || ks > 0) ? 1u : 0u);
-          mma_ts(d, phi, bl, idO, 1u);
-          mma_ts(d, phi, bh, idO, 1u);
+          mma_ts(d, phi, bhl, idO2, (acc_prev || ks > 0) ? 1u : 0u);
+          mma_ts(d, plo, bhl, idO, 1u);
         }
       };
       bool ok = wait_bar(bar_x, 0, abort_flag, wlim) && stall != 1;
@@ -697,21 +706,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                       (b * p.M + i) * p.ldo + p.c0;
 #pragma unroll
         for (int ch = 0; ch < CP / 16; ++ch) {
-          uint32_t v0[16], v1[16];
-          tmem_ld16(tO0 + ch * 16, v0);
-          tmem_ld16(tO1 + ch * 16, v1);
+          // O_h = O_big + O_small of each warpgroup, then O_0 + O_1
+          float o[16];
+          uint32_t vb[16], vs[16];
+          tmem_ld16(tO0 + ch * 16, vb);
+          tmem_ld16(tO0 + CP + ch * 16, vs);
           tmem_wait_ld();
-          reg_fence16(v0);
-          reg_fence16(v1);
+          reg_fence16(vb);
+          reg_fence16(vs);
+#pragma unroll
+          for (int q = 0; q < 16; ++q)
+            o[q] = T > 0 ? __uint_as_float(vb[q]) + __uint_as_float(vs[q]) : 0.f;
+          tmem_ld16(tO1 + ch * 16, vb);
+          tmem_ld16(tO1 + CP + ch * 16, vs);
+          tmem_wait_ld();
+          reg_fence16(vb);
+          reg_fence16(vs);
           if (valid) {
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
               const int c = ch * 16 + q;
-              float o = 0.f;
-              if (T > 0) o = __uint_as_float(v0[q]);
-              if (T > 1) o += __uint_as_float(v1[q]);   // O_1 holds tiles only when T > 1
+              // O_1 holds tiles only when T > 1
+              if (T > 1) o[q] += __uint_as_float(vb[q]) + __uint_as_float(vs[q]);
               // undo P's 2^14 and the channel's 2^e, exactly
-              if (c < p.cw) orow[c] = o * pow2_int(-14 - split_exp(p.vmax[b * CP + c]));
+              if (c < p.cw) orow[c] = o[q] * pow2_int(-14 - split_exp(p.vmax[b * CP + c]));
             }
           }
         }
@@ -765,23 +783,28 @@ __global__ void column_mean_kernel(const float* __restrict__ y, float* __restric
 
 // Per batch, the bits of max |v_k - z_k| over the rows of x and y (non-negative
 // floats order like their bit patterns): the split rows' scale.  Grid
-// (B, blocks) of 256 threads, one warp per row, lanes along the features (the
-// centre in registers, D <= 128); amax zeroed before.
+// (B, blocks) of 256 threads; a group of `grp` lanes (a power of two, 4
+// features a lane, D <= 128) reads one row, so a warp reads 32 / grp rows at
+// once; amax zeroed before.
 __global__ void centred_maxabs_kernel(const float* __restrict__ x, const float* __restrict__ y,
                                       const float* __restrict__ zc, int* __restrict__ amax,
-                                      int64_t M, int64_t N, int D) {
+                                      int64_t M, int64_t N, int D, int grp) {
   const int64_t b = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int rpw = 32 / grp, lig = lane & (grp - 1), sub = lane / grp;
+  const int k0 = 4 * lig;
   float z[4];
 #pragma unroll
-  for (int u = 0; u < 4; ++u) z[u] = (lane + 32 * u < D) ? zc[b * D + lane + 32 * u] : 0.f;
+  for (int u = 0; u < 4; ++u) z[u] = (k0 + u < D) ? zc[b * D + k0 + u] : 0.f;
   float m = 0.f;
-  for (int64_t r = static_cast<int64_t>(blockIdx.y) * 8 + warp; r < M + N;
-       r += static_cast<int64_t>(gridDim.y) * 8) {
+  for (int64_t r0 = (static_cast<int64_t>(blockIdx.y) * 8 + warp) * rpw; r0 < M + N;
+       r0 += static_cast<int64_t>(gridDim.y) * 8 * rpw) {
+    const int64_t r = r0 + sub;
+    if (r >= M + N) continue;
     const float* v = r < M ? x + (b * M + r) * D : y + (b * N + (r - M)) * D;
 #pragma unroll
     for (int u = 0; u < 4; ++u)
-      if (lane + 32 * u < D) m = fmaxf(m, fabsf(v[lane + 32 * u] - z[u]));
+      if (k0 + u < D) m = fmaxf(m, fabsf(v[k0 + u] - z[u]));
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -801,20 +824,86 @@ __global__ void centred_maxabs_kernel(const float* __restrict__ x, const float* 
 // record, norm[4 b Rpad + r] (lanes 1-3, Rpad floats apart, zeroed), with -inf
 // for the padding columns r >= R.  fp16 / bf16 inputs (zc == nullptr,
 // split == 0): the input values themselves, rows [v (K')] only.
-// One warp per row, lanes along the features (coalesced reads and writes).
+struct PackSide {
+  const void* src;
+  float* dst;
+  float* norm;
+  int64_t R, Rpad;
+  int records;
+};
+
+// Both sides in one launch: blockIdx.z = 0 the rows, 1 the columns; blockIdx.y
+// = the batch (its centre and scale read once per block).  Split rows: a group
+// of `grp` lanes (a power of two, 4 features a lane) builds one row, so a warp
+// builds 32 / grp rows at once; unsplit rows (fp16 / bf16 inputs): one warp per
+// row, lanes along the features.
 template <typename T>
-__global__ void pack_rows_f32_kernel(const T* __restrict__ src, const float* __restrict__ zc,
-                                     float* __restrict__ dst, float* __restrict__ norm, int64_t B,
-                                     int64_t R, int64_t Rpad, int D, int Kp, float c,
-                                     int records, int split, const int* __restrict__ amax) {
+__global__ void pack_rows_f32_kernel(PackSide rows_side, PackSide cols_side,
+                                     const float* __restrict__ zc, int D, int Kp, float c,
+                                     int split, const int* __restrict__ amax, int grp) {
+  const PackSide& ps = blockIdx.z == 0 ? rows_side : cols_side;
+  const T* __restrict__ src = static_cast<const T*>(ps.src);
+  const int64_t R = ps.R, Rpad = ps.Rpad;
+  const int records = ps.records;
   const int lane = threadIdx.x & 31;
-  const int64_t total = B * Rpad;
-  const int64_t wstride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
-       e < total; e += wstride) {
-    const int64_t b = e / Rpad, rr = e % Rpad;
-    // records: lane l of column rr at norm[(4 b + l) Rpad + rr]; rows: norm[e]
-    float* nrm = records ? norm + 4 * b * Rpad + rr : norm + e;
+  const int64_t b = blockIdx.y;
+  const float* z = zc ? zc + b * D : nullptr;
+  const int64_t gw = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  // records: lane l of column rr at norm[(4 b + l) Rpad + rr]; rows: norm[b Rpad + rr]
+  auto norm_at = [&](int64_t rr) { return records ? ps.norm + 4 * b * Rpad + rr : ps.norm + b * Rpad + rr; };
+  if (split) {
+    // fp16 [hi (K') | lo (K')] of v' 2^e: v' 2^e is exact, hi its nearest fp16,
+    // lo the nearest fp16 of the (exact) remainder
+    const float sc = pow2_int(split_exp(amax[b]));
+    const int rpw = 32 / grp, lig = lane & (grp - 1), sub = lane / grp;
+    const int k0 = 4 * lig;
+    for (int64_t r0 = gw * rpw; r0 < Rpad; r0 += nw * rpw) {
+      const int64_t rr = r0 + sub;
+      const bool row = rr < R;
+      const T* v = src + (b * R + (row ? rr : 0)) * D;
+      float d[4], sq = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int k = k0 + u;
+        d[u] = (row && k < D) ? vf(v[k]) - z[k] : 0.f;
+        sq = fmaf(d[u], d[u], sq);
+      }
+      for (int o = grp / 2; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      if (rr >= Rpad) continue;
+      float* nrm = norm_at(rr);
+      if (!row) {
+        if (lig == 0) {
+          nrm[0] = -INFINITY;   // padding columns: kernel value 0
+          if (records) nrm[Rpad] = nrm[2 * Rpad] = nrm[3 * Rpad] = 0.f;
+        }
+        continue;
+      }
+      if (k0 < Kp) {
+        __half hi[4], lo[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float x = d[u] * sc;
+          hi[u] = __float2half_rn(x);
+          lo[u] = __float2half_rn(x - __half2float(hi[u]));
+        }
+        __half* out = reinterpret_cast<__half*>(ps.dst) + (b * R + rr) * (2 * static_cast<int64_t>(Kp)) + k0;
+        *reinterpret_cast<uint2*>(out) = make_uint2(
+            static_cast<uint32_t>(__half_as_ushort(hi[0])) | (static_cast<uint32_t>(__half_as_ushort(hi[1])) << 16),
+            static_cast<uint32_t>(__half_as_ushort(hi[2])) | (static_cast<uint32_t>(__half_as_ushort(hi[3])) << 16));
+        *reinterpret_cast<uint2*>(out + Kp) = make_uint2(
+            static_cast<uint32_t>(__half_as_ushort(lo[0])) | (static_cast<uint32_t>(__half_as_ushort(lo[1])) << 16),
+            static_cast<uint32_t>(__half_as_ushort(lo[2])) | (static_cast<uint32_t>(__half_as_ushort(lo[3])) << 16));
+      }
+      if (lig == 0) {
+        nrm[0] = -c * sq;
+        if (records) nrm[Rpad] = nrm[2 * Rpad] = nrm[3 * Rpad] = 0.f;
+      }
+    }
+    return;
+  }
+  for (int64_t rr = gw; rr < Rpad; rr += nw) {
+    float* nrm = norm_at(rr);
     if (rr >= R) {
       if (lane == 0) {
         nrm[0] = -INFINITY;   // padding columns: kernel value 0
@@ -823,29 +912,13 @@ __global__ void pack_rows_f32_kernel(const T* __restrict__ src, const float* __r
       continue;
     }
     const T* v = src + (b * R + rr) * D;
-    const float* z = zc ? zc + b * D : nullptr;
     float sq = 0.f;
-    if (split) {
-      // fp16 [hi (K') | lo (K')] of v' 2^e: v' 2^e is exact, hi its nearest
-      // fp16, lo the nearest fp16 of the (exact) remainder
-      const float sc = pow2_int(split_exp(amax[b]));
-      __half* out = reinterpret_cast<__half*>(dst) + (b * R + rr) * (2 * static_cast<int64_t>(Kp));
-      for (int k = lane; k < Kp; k += 32) {
-        const float d = (k < D) ? vf(v[k]) - z[k] : 0.f;
-        sq = fmaf(d, d, sq);
-        const float u = d * sc;
-        const __half hi = __float2half_rn(u);
-        out[k] = hi;
-        out[Kp + k] = __float2half_rn(u - __half2float(hi));
-      }
-    } else {
-      // the fp16 / bf16 input values themselves (exact in the MMA's encoding)
-      uint16_t* out = reinterpret_cast<uint16_t*>(dst) + (b * R + rr) * static_cast<int64_t>(Kp);
-      for (int k = lane; k < Kp; k += 32) {
-        const float d = (k < D) ? vf(v[k]) : 0.f;
-        sq = fmaf(d, d, sq);
-        out[k] = (k < D) ? raw16(v[k]) : static_cast<uint16_t>(0);
-      }
+    // the fp16 / bf16 input values themselves (exact in the MMA's encoding)
+    uint16_t* out = reinterpret_cast<uint16_t*>(ps.dst) + (b * R + rr) * static_cast<int64_t>(Kp);
+    for (int k = lane; k < Kp; k += 32) {
+      const float d = (k < D) ? vf(v[k]) : 0.f;
+      sq = fmaf(d, d, sq);
+      out[k] = (k < D) ? raw16(v[k]) : static_cast<uint16_t>(0);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
@@ -1068,19 +1141,29 @@ void pack_operands_f32(const F32Args& a, int64_t Nq, float c, cudaStream_t s) {
       zc = a.zc;
       amax = f32_amax(a);
       cudaMemsetAsync(amax, 0, static_cast<size_t>(a.B) * sizeof(int), s);
-      int64_t blocks = (a.M + a.N + 7) / 8;   // 8 rows (warps) per block and pass
+      int grp = 4;   // lanes per row: the power of two covering D / 4 features' lanes
+      while (grp * 4 < a.D) grp *= 2;
+      const int64_t per_block = 8 * (32 / grp);   // rows per block and pass
+      int64_t blocks = (a.M + a.N + per_block - 1) / per_block;
       const int64_t cap = (148 * 16 + a.B - 1) / a.B;
       if (blocks > cap) blocks = cap;
       if (blocks > 65535) blocks = 65535;
       centred_maxabs_kernel<<<dim3(static_cast<unsigned>(a.B), static_cast<unsigned>(blocks)), 256, 0,
-                              s>>>(x, y, a.zc, amax, a.M, a.N, a.D);
+                              s>>>(x, y, a.zc, amax, a.M, a.N, a.D, grp);
     }
   }
-  // one warp per row, 8 rows per 256-thread block
-  pack_rows_f32_kernel<T><<<grid_for(a.B * a.M, 8), 256, 0, s>>>(x, zc, a.xpack, a.rnorm, a.B, a.M,
-                                                                a.M, a.D, a.plan.Kp, c, 0, split, amax);
-  pack_rows_f32_kernel<T><<<grid_for(a.B * Nq, 8), 256, 0, s>>>(y, zc, a.ypack, a.qw, a.B, a.N, Nq,
-                                                               a.D, a.plan.Kp, c, 1, split, amax);
+  // one warp per row, 8 rows per 256-thread block; about 148 x 32 blocks in all
+  const PackSide rs{x, a.xpack, a.rnorm, a.M, a.M, 0};
+  const PackSide cs{y, a.ypack, a.qw, a.N, Nq, 1};
+  const int64_t rmax = a.M > Nq ? a.M : Nq;
+  int64_t bx = (rmax + 7) / 8;
+  const int64_t cap = (148 * 16 + a.B - 1) / a.B;
+  if (bx > cap) bx = cap;
+  if (bx < 1) bx = 1;
+  int grp = 4;   // lanes per split row: the power of two covering Kp / 4 features' lanes
+  while (grp * 4 < a.plan.Kp) grp *= 2;
+  pack_rows_f32_kernel<T><<<dim3(static_cast<unsigned>(bx), static_cast<unsigned>(a.B), 2), 256, 0, s>>>(
+      rs, cs, zc, a.D, a.plan.Kp, c, split, amax, grp);
 }
 
 template <typename T>
