@@ -319,6 +319,15 @@ __device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr, uint32_t lbo, 
   return d;
 }
 
+// The descriptor of an operand `bytes` (a multiple of 16) past the one `d`
+// describes: only the 14-bit start-address field (address / 16) changes, and a
+// shared-memory address below 256 KB never carries out of it.  One add, where
+// building a descriptor from its address takes a chain of shifts and masks on
+// the single thread that issues the MMAs.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t d, uint32_t bytes) {
+  return d + static_cast<uint64_t>(bytes >> 4);
+}
+
 // Instruction-descriptor bit marking operand A as MN-major (read transposed).
 constexpr uint32_t kIdescAMajorMN = 1u << 15;
 

@@ -343,10 +343,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idO = idesc_f16(0, kBM, CP);   // P.v: fp16 parts of P 2^14 and v 2^e
       const int ks_lo = p.ksteps;
       // K step ks (8 floats = 32 bytes) of a packed row block whose atoms are
-      // atom_bytes apart
-      auto kdesc = [](const uint8_t* base, int atom_bytes, int ks) {
+      // atom_bytes apart, from the descriptor of the block's start: the
+      // descriptors of the operand regions are built once, and each operand's is
+      // one add away (the issuing thread's time goes to MMAs, not to masks)
+      const uint64_t dX = desc_k_sw128(smem_u32(sX));
+      const uint64_t dStage = desc_k_sw128(smem_u32(sStage));
+      auto kdesc = [](uint64_t dbase, int atom_bytes, int ks) {
         const int off = ks * 32;
-        return desc_k_sw128(smem_u32(base + (off >> 7) * atom_bytes) + (off & 127));
+        return desc_advance(dbase, static_cast<uint32_t>((off >> 7) * atom_bytes + (off & 127)));
       };
       // S = x'.y'^T for warpgroup h.  Register values: the small products
       // (lo.hi, hi.lo) into Ssmall_h and the large ones into Sbig_h, K step
@@ -355,14 +359,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // small, then the large ones -- each addition is rounded against the
       // magnitude of what it adds to.
       auto issue_S = [&](int h, int st) {
-        const uint8_t* sy = sStage + st * Cfg::STAGE;
+        const uint64_t sy = desc_advance(dStage, static_cast<uint32_t>(st * Cfg::STAGE));
         const uint32_t db = tmem + Cfg::col_s(h);
         const uint32_t ds = REG ? tmem + Cfg::col_ss(h) : db;
         auto mma = [&](uint32_t d, int ka, uint64_t bdesc, uint32_t acc) {
           if constexpr (Cfg::XT)
             mma_ts(d, tmem + Cfg::COL_X + ka * 8, bdesc, idS, acc);
           else
-            mma_ss(d, kdesc(sX, kAtom, ka), bdesc, idS, acc);
+            mma_ss(d, kdesc(dX, kAtom, ka), bdesc, idS, acc);
         };
         // (exact 16-bit operands, SPLIT false: the large products alone)
         if constexpr (REG) {
@@ -387,16 +391,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // O_h += P_hi [v_hi ; v_lo] (one MMA of N = 2 CP: O_big and O_small at
       // once, as cheap as one of N = CP) and P_lo v_hi into O_big: two MMAs a
-      // K step where three products of N = CP were three.
+      // K step where the three products of N = CP took three.
       const uint32_t idO2 = idesc_f16(0, kBM, 2 * CP);
       auto issue_O = [&](int h, int st, bool acc_prev) {
-        const uint8_t* sv = sStage + st * Cfg::STAGE + Cfg::Y_BYTES + Cfg::QW_BYTES;
+        const uint64_t sv = desc_advance(
+            dStage, static_cast<uint32_t>(st * Cfg::STAGE + Cfg::Y_BYTES + Cfg::QW_BYTES));
         const uint32_t d = tmem + Cfg::col_o(h);
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks) {   // K steps of 16 columns
           const int within = ks * 32;
           // rows 0 .. CP-1 the hi atom, CP .. 2 CP-1 the lo atom right after it
-          const uint64_t bhl = desc_k_sw128(smem_u32(sv) + within);
+          const uint64_t bhl = desc_advance(sv, static_cast<uint32_t>(within));
           const uint32_t phi = tmem + Cfg::col_phi(h) + ks * 8;
           const uint32_t plo = tmem + Cfg::col_plo(h) + ks * 8;
           mma_ts(d, phi, bhl, idO2, (acc_prev || ks > 0) ? 1u : 0u);
