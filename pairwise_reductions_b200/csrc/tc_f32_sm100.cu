@@ -341,7 +341,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // kind::f16, 16 per K step: fp16 hi / lo parts, or the unsplit fp16 / bf16 rows
       const uint32_t idS = idesc_f16(SPLIT ? 0 : p.afmt, kBM, BN);
       const uint32_t idO = idesc_f16(0, kBM, CP);   // P.v: fp16 parts of P 2^14 and v 2^e
-      const int ks_lo = p.ksteps;
+      const int ks_lo = p.ksteps;   // the lo half of a split row starts K' columns on
+      const int ksteps = p.ksteps;
       // K step ks (8 floats = 32 bytes) of a packed row block whose atoms are
       // atom_bytes apart, from the descriptor of the block's start: the
       // descriptors of the operand regions are built once, and each operand's is
@@ -368,25 +369,48 @@ __global__ void __launch_bounds__(kThreads, 1)
           else
             mma_ss(d, kdesc(dX, kAtom, ka), bdesc, idS, acc);
         };
-        // (exact 16-bit operands, SPLIT false: the large products alone)
-        if constexpr (REG) {
-          for (int ks = 0; ks < p.ksteps; ++ks) {
-            const uint64_t bh = kdesc(sy, BN * 128, ks);
+        // (exact 16-bit operands, SPLIT false: the large products alone).  The K
+        // step count is a template constant of each branch of the switch below:
+        // fully unrolled, the address arithmetic of every MMA is laid out ahead of
+        // the MMAs instead of between them on the one issuing thread (measured: a
+        // run-time loop here cost about twice the MMAs themselves)
+        auto steps = [&](auto kn) {
+          constexpr int KN = decltype(kn)::value;
+          if constexpr (REG) {
+#pragma unroll
+            for (int ks = 0; ks < KN; ++ks) {
+              const uint64_t bh = kdesc(sy, BN * 128, ks);
+              if constexpr (SPLIT) {
+                mma(ds, ks + ks_lo, bh, ks > 0 ? 1u : 0u);
+                mma(ds, ks, kdesc(sy, BN * 128, ks + ks_lo), 1u);
+              }
+              mma(db, ks, bh, ks > 0 ? 1u : 0u);
+            }
+          } else {
             if constexpr (SPLIT) {
-              mma(ds, ks + ks_lo, bh, ks > 0 ? 1u : 0u);
-              mma(ds, ks, kdesc(sy, BN * 128, ks + ks_lo), 1u);
+#pragma unroll
+              for (int ks = 0; ks < KN; ++ks) {
+                mma(db, ks + ks_lo, kdesc(sy, BN * 128, ks), ks > 0 ? 1u : 0u);
+                mma(db, ks, kdesc(sy, BN * 128, ks + ks_lo), 1u);
+              }
             }
-            mma(db, ks, bh, ks > 0 ? 1u : 0u);
+#pragma unroll
+            for (int ks = 0; ks < KN; ++ks)
+              mma(db, ks, kdesc(sy, BN * 128, ks), (SPLIT || ks > 0) ? 1u : 0u);
           }
-        } else {
-          if constexpr (SPLIT) {
-            for (int ks = 0; ks < p.ksteps; ++ks) {
-              mma(db, ks + ks_lo, kdesc(sy, BN * 128, ks), ks > 0 ? 1u : 0u);
-              mma(db, ks, kdesc(sy, BN * 128, ks + ks_lo), 1u);
-            }
-          }
-          for (int ks = 0; ks < p.ksteps; ++ks)
-            mma(db, ks, kdesc(sy, BN * 128, ks), (SPLIT || ks > 0) ? 1u : 0u);
+        };
+        // K steps a packed row can hold: split rows [hi K' | lo K'] fill 2 K' <= 64 KA
+        // columns, unsplit rows K' <= 64 KA
+        constexpr int KSMAX = SPLIT ? 2 * KA : 4 * KA;
+        switch (ksteps) {
+          case 1: steps(std::integral_constant<int, 1>{}); break;
+          case 2: if constexpr (KSMAX >= 2) steps(std::integral_constant<int, 2>{}); break;
+          case 3: if constexpr (KSMAX >= 3) steps(std::integral_constant<int, 3>{}); break;
+          case 4: if constexpr (KSMAX >= 4) steps(std::integral_constant<int, 4>{}); break;
+          case 5: if constexpr (KSMAX >= 5) steps(std::integral_constant<int, 5>{}); break;
+          case 6: if constexpr (KSMAX >= 6) steps(std::integral_constant<int, 6>{}); break;
+          case 7: if constexpr (KSMAX >= 7) steps(std::integral_constant<int, 7>{}); break;
+          default: if constexpr (KSMAX >= 8) steps(std::integral_constant<int, 8>{}); break;
         }
       };
       // O_h += P_hi [v_hi ; v_lo] (one MMA of N = 2 CP: O_big and O_small at
