@@ -197,7 +197,7 @@ bool make_tmap_3d(CUtensorMap* m, CUtensorMapDataType dt, void* base, uint64_t d
                   uint32_t box1, bool swizzle128 = true);
 
 // ------------------------------------------------------------- fp32 tensor-core path
-// fp32 inputs with kSdMaxD < D <= kTcMaxD: split-tf32 MMAs (tc_f32_sm100.cu).
+// fp32 inputs with kSdMaxD < D <= kTcMaxD: MMAs on split fp16 parts (tc_f32_sm100.cu).
 struct F32Plan {
   bool split;          // fp32 inputs: fp16 rows [hi | lo]; fp16 / bf16: the input values, unsplit
   int Kp;              // 16-bit elements per half of a packed row: D rounded up to 16

@@ -106,27 +106,37 @@ struct F32Cfg {
   // v^T in fp16 [hi | lo] parts: 64 columns per 128-byte atom row
   static constexpr int va(int bn) { return bn < 64 ? 1 : bn / 64; }
   static constexpr int v_bytes(int bn) { return REG ? 0 : 2 * va(bn) * CP * 128; }
-  static constexpr int stage_bytes(int bn) { return KA * bn * 128 + qw_bytes(bn) + v_bytes(bn); }
+  // Register values with wide rows (4+ atoms: two or three stages fit): the
+  // column records sit in a ring of their own, so that a y' stage is free once
+  // the similarity MMAs have read it, while the exp warps still read the
+  // tile's records (b64_d128_f32 +9..16%).  Narrower rows keep four stages of
+  // [y' | records], freed by the exp warps (the ring measured 0.9% slower there).
+  // Tensor-core values: one stage holds y', the records and v^T, freed by the
+  // P.v MMAs.
+  static constexpr int NR = (REG && KA >= 4) ? 4 : 0;
+  static constexpr int stage_bytes(int bn) {
+    return KA * bn * 128 + (NR > 0 ? 0 : qw_bytes(bn)) + v_bytes(bn);
+  }
+  static constexpr int rec_bytes(int bn) { return NR * qw_bytes(bn); }
   static constexpr int BUDGET = 214 * 1024;
-  // TMEM columns of the accumulators.  Register values: the large and the
-  // small products of S in separate accumulators for each warpgroup (two
-  // independent MMA chains; the small ones never round against the large
-  // sum).  Tensor-core values: one S (small products first, then the large
-  // ones), P hi/lo (fp16 pairs: bn / 2 columns each) and O per warpgroup, O as
+  // TMEM columns of the accumulators: one S per warpgroup (every small
+  // product first, while the sum is small, then the large ones: each addition
+  // is rounded against the magnitude of what it adds to); tensor-core values
+  // add P hi/lo (fp16 pairs: bn / 2 columns each) and O per warpgroup, O as
   // two halves of CP columns: O_big (P_hi v_hi + P_lo v_hi) and O_small
   // (P_hi v_lo), added in the epilogue.
-  static constexpr int tmem_acc(int bn) { return REG ? 4 * bn : 4 * bn + 4 * CPA; }
+  static constexpr int tmem_acc(int bn) { return REG ? 2 * bn : 4 * bn + 4 * CPA; }
   // The x' rows (2 K' <= 32 KA columns) sit in TMEM as the A operand of the
   // similarity MMAs when the accumulators leave room, else in shared memory.
   static constexpr bool xt(int bn) { return tmem_acc(bn) + 32 * KA <= 512; }
   static constexpr int x_bytes(int bn) { return xt(bn) ? 0 : KA * kAtom; }
   static constexpr bool fits(int bn) {
-    return tmem_acc(bn) <= 512 && (BUDGET - x_bytes(bn)) / stage_bytes(bn) >= 2;
+    return tmem_acc(bn) <= 512 && (BUDGET - x_bytes(bn) - rec_bytes(bn)) / stage_bytes(bn) >= 2;
   }
-  // Column tile.  An M = 128 MMA takes about the same time for any N up to
-  // 128 (measured on B200: ~78 cycles at N = 32 .. 128 for tf32), so the widest
-  // tile that fits is the cheapest per pair; three register channels use 32
-  // columns (registers).
+  // Column tile.  An M = 128, K = 16 MMA costs much the same at N = 32 and 64
+  // and a third more at 128 (measured on B200: 47, 49 and 65 issue cycles), so
+  // the widest tile that fits is the cheapest per pair; three register channels
+  // use 32 columns (registers).
   static constexpr int BN =
       MODE == 3 ? 32 : ((MODE == 1 && fits(128)) ? 128 : (fits(64) ? 64 : 32));
   static constexpr bool XT = xt(BN);
@@ -137,18 +147,19 @@ struct F32Cfg {
   static constexpr int VA = va(BN);                     // v^T atoms per part and stage
   static constexpr int V_BYTES = v_bytes(BN);
   static constexpr int STAGE = stage_bytes(BN);
-  static constexpr int NST_FIT = (BUDGET - X_BYTES) / STAGE;
+  static constexpr int REC_BYTES = rec_bytes(BN);
+  static constexpr int NST_FIT = (BUDGET - X_BYTES - REC_BYTES) / STAGE;
   static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
-  static constexpr int NBARS = 2 * NST + 10;
+  static constexpr int NBARS = 2 * NST + 10 + 2 * NR;
   static constexpr int RED_BYTES = kBM * 32;            // warpgroup 1 partial sums (m, l)
-  static constexpr int SMEM_RAW = 1024 + X_BYTES + NST * STAGE + 8 * NBARS + 16 + RED_BYTES;
+  static constexpr int SMEM_RAW =
+      1024 + X_BYTES + NST * STAGE + REC_BYTES + 8 * NBARS + 16 + RED_BYTES;
   // at least ~120 KB: one CTA per SM, so the 512-column TMEM allocation never waits
   static constexpr int SMEM = SMEM_RAW < 122880 ? 122880 : SMEM_RAW;
-  // TMEM columns.  Register values: Sbig0 | Sbig1 | Ssmall0 | Ssmall1 | x'.
+  // TMEM columns.  Register values: S0 | S1 | x'.
   // Tensor-core values: S0 | S1 | Phi0 | Phi1 | Plo0 | Plo1 | O0 | O1 | x', O_h as
   // [O_big (CP) | O_small (CP)] in 2 CPA columns.
   __host__ __device__ static constexpr uint32_t col_s(int h) { return h * BN; }
-  __host__ __device__ static constexpr uint32_t col_ss(int h) { return 2 * BN + h * BN; }
   __host__ __device__ static constexpr uint32_t col_phi(int h) { return 2 * BN + (BN / 2) * h; }
   __host__ __device__ static constexpr uint32_t col_plo(int h) { return 3 * BN + (BN / 2) * h; }
   __host__ __device__ static constexpr uint32_t col_o(int h) { return 4 * BN + 2 * CPA * h; }
@@ -245,7 +256,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sX = smem;
   uint8_t* sStage = smem + Cfg::X_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + NST * Cfg::STAGE);
+  uint8_t* sRec = sStage + NST * Cfg::STAGE;   // register values: the records ring
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sRec + Cfg::REC_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float4* red = reinterpret_cast<float4*>(tmem_slot + 4);   // 16-byte aligned
@@ -259,6 +271,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_p = [&](int h) { return bar0 + 8u * (2 * NST + 5 + h); };   // P_h written
   auto bar_q = [&](int h) { return bar0 + 8u * (2 * NST + 7 + h); };   // P_h consumed
   const uint32_t bar_o = bar0 + 8u * (2 * NST + 9);
+  constexpr int NR = Cfg::NR;
+  constexpr bool RSEP = NR > 0;          // the records in a ring of their own
+  constexpr int NRM = RSEP ? NR : 1;     // (slot arithmetic)
+  auto bar_rfull = [&](int r) { return bar0 + 8u * (2 * NST + 10 + r); };        // records landed
+  auto bar_rempty = [&](int r) { return bar0 + 8u * (2 * NST + 10 + NR + r); };  // records read
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t b = blockIdx.z;
@@ -273,9 +290,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(bar_full(s), 1);
-      // a stage is released by the P.v MMAs (tensor-core values) or by the
-      // 128 exp threads that read its norms and values (register values)
-      mbar_init(bar_empty(s), REG ? 4 * 32 : 1);
+      // a stage is released by the MMAs that read it last (the similarity with
+      // a records ring, P.v with tensor-core values), else by the 128 exp
+      // threads that read its records
+      mbar_init(bar_empty(s), (REG && !RSEP) ? 4 * 32 : 1);
+    }
+    // a records slot: loaded with its tile's y', released by the 128 exp
+    // threads of the warpgroup that summed the tile
+    for (int r = 0; r < NR; ++r) {
+      mbar_init(bar_rfull(r), 1);
+      mbar_init(bar_rempty(r), 4 * 32);
     }
     // x' ready: the TMA load (shared memory), or the 128 threads of exp
     // warpgroup 0 that copy the rows into TMEM
@@ -312,19 +336,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(smem_u32(sX + a * kAtom), &tmX, bar_x, a * kAtomElems, static_cast<int>(row0),
                       static_cast<int>(b));
       }
-      const uint32_t stage_tx = p.atoms * BN * 128 + BN * 16 + Cfg::V_BYTES;
+      const uint32_t stage_tx = p.atoms * BN * 128 + (RSEP ? 0 : BN * 16) + Cfg::V_BYTES;
       for (int t = 0; t < T; ++t) {
         const int st = t % NST;
+        const int rs = RSEP ? t % NRM : 0;
+        // both slots of tile t free before either load: "issued" then counts the
+        // tiles whose loads (all of them) are in flight
         if (t >= NST && !wait_bar(bar_empty(st), ((t / NST) - 1) & 1, abort_flag, wlim)) break;
+        if (RSEP && t >= NR && !wait_bar(bar_rempty(rs), ((t / NRM) - 1) & 1, abort_flag, wlim))
+          break;
         uint8_t* sy = sStage + st * Cfg::STAGE;
-        uint8_t* sq = sy + Cfg::Y_BYTES;
+        uint8_t* sq = RSEP ? sRec + rs * Cfg::QW_BYTES : sy + Cfg::Y_BYTES;
         uint8_t* sv = sq + Cfg::QW_BYTES;
         const int j0 = static_cast<int>(jbeg + static_cast<int64_t>(t) * BN);
         mbar_arrive_expect_tx(bar_full(st), stage_tx);
         for (int a = 0; a < p.atoms; ++a)
           tma_load_3d(smem_u32(sy + a * BN * 128), &tmY, bar_full(st), a * kAtomElems, j0,
                       static_cast<int>(b));
-        tma_load_3d(smem_u32(sq), &tmQ, bar_full(st), j0, 0, static_cast<int>(b));
+        const uint32_t bar_q_in = RSEP ? bar_rfull(rs) : bar_full(st);
+        if constexpr (RSEP) mbar_arrive_expect_tx(bar_q_in, BN * 16);
+        tma_load_3d(smem_u32(sq), &tmQ, bar_q_in, j0, 0, static_cast<int>(b));
         if constexpr (!REG) {
           for (int hl = 0; hl < 2; ++hl)
             for (int a = 0; a < Cfg::VA; ++a)
@@ -353,16 +384,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int off = ks * 32;
         return desc_advance(dbase, static_cast<uint32_t>((off >> 7) * atom_bytes + (off & 127)));
       };
-      // S = x'.y'^T for warpgroup h.  Register values: the small products
-      // (lo.hi, hi.lo) into Ssmall_h and the large ones into Sbig_h, K step
-      // by K step (two independent chains).  Tensor-core values: one
-      // accumulator, every small product of every K step first, while it is
-      // small, then the large ones -- each addition is rounded against the
-      // magnitude of what it adds to.
+      // S = x'.y'^T for warpgroup h, one accumulator: every small product
+      // (lo.hi, hi.lo) of every K step first, while the sum is small, then the
+      // large ones -- each addition is rounded against the magnitude of what it
+      // adds to.  (On B200 a chain of kind::f16 MMAs into one accumulator issues
+      // as fast as independent ones, so a second accumulator would buy nothing.)
       auto issue_S = [&](int h, int st) {
         const uint64_t sy = desc_advance(dStage, static_cast<uint32_t>(st * Cfg::STAGE));
         const uint32_t db = tmem + Cfg::col_s(h);
-        const uint32_t ds = REG ? tmem + Cfg::col_ss(h) : db;
         auto mma = [&](uint32_t d, int ka, uint64_t bdesc, uint32_t acc) {
           if constexpr (Cfg::XT)
             mma_ts(d, tmem + Cfg::COL_X + ka * 8, bdesc, idS, acc);
@@ -376,28 +405,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         // run-time loop here cost about twice the MMAs themselves)
         auto steps = [&](auto kn) {
           constexpr int KN = decltype(kn)::value;
-          if constexpr (REG) {
+          if constexpr (SPLIT) {
 #pragma unroll
             for (int ks = 0; ks < KN; ++ks) {
-              const uint64_t bh = kdesc(sy, BN * 128, ks);
-              if constexpr (SPLIT) {
-                mma(ds, ks + ks_lo, bh, ks > 0 ? 1u : 0u);
-                mma(ds, ks, kdesc(sy, BN * 128, ks + ks_lo), 1u);
-              }
-              mma(db, ks, bh, ks > 0 ? 1u : 0u);
+              mma(db, ks + ks_lo, kdesc(sy, BN * 128, ks), ks > 0 ? 1u : 0u);
+              mma(db, ks, kdesc(sy, BN * 128, ks + ks_lo), 1u);
             }
-          } else {
-            if constexpr (SPLIT) {
-#pragma unroll
-              for (int ks = 0; ks < KN; ++ks) {
-                mma(db, ks + ks_lo, kdesc(sy, BN * 128, ks), ks > 0 ? 1u : 0u);
-                mma(db, ks, kdesc(sy, BN * 128, ks + ks_lo), 1u);
-              }
-            }
-#pragma unroll
-            for (int ks = 0; ks < KN; ++ks)
-              mma(db, ks, kdesc(sy, BN * 128, ks), (SPLIT || ks > 0) ? 1u : 0u);
           }
+#pragma unroll
+          for (int ks = 0; ks < KN; ++ks)
+            mma(db, ks, kdesc(sy, BN * 128, ks), (SPLIT || ks > 0) ? 1u : 0u);
         };
         // K steps a packed row can hold: split rows [hi K' | lo K'] fill 2 K' <= 64 KA
         // columns, unsplit rows K' <= 64 KA
@@ -440,6 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           issue_S(h, h);
           mma_commit(bar_s(h));
+          if constexpr (RSEP) mma_commit(bar_empty(h % NST));
         }
       }
       // S_h(t + 2) may overwrite S_h once warpgroup h has read S_h(t).  With
@@ -452,6 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         issue_S(h, t2 % NST);
         mma_commit(bar_s(h));
+        if constexpr (RSEP) mma_commit(bar_empty(t2 % NST));
         return true;
       };
       for (int k = 0; ok && 2 * k < T; ++k) {
@@ -522,8 +541,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int k = 0;
     for (int t = h; ok && t < T; t += 2, ++k) {
       const int st = t % NST;
-      ok = wait_bar(bar_s(h), k & 1, abort_flag, wlim) &&
-           wait_bar(bar_full(st), (t / NST) & 1, abort_flag, wlim);   // norms and values landed
+      ok = wait_bar(bar_s(h), k & 1, abort_flag, wlim) &&   // norms and values landed
+           (RSEP ? wait_bar(bar_rfull(t % NRM), (t / NRM) & 1, abort_flag, wlim)
+                : wait_bar(bar_full(st), (t / NST) & 1, abort_flag, wlim));
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
@@ -531,42 +551,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tS = tmem + lane_base + Cfg::col_s(h);
       // the column records, lane by lane: q_j at qrec[j], value c at qrec[(1 + c) BN + j]
-      const float* qrec = reinterpret_cast<const float*>(sStage + st * Cfg::STAGE + Cfg::Y_BYTES);
+      const float* qrec = reinterpret_cast<const float*>(
+          RSEP ? sRec + (t % NRM) * Cfg::QW_BYTES : sStage + st * Cfg::STAGE + Cfg::Y_BYTES);
       if constexpr (REG) {
-        // S = Sbig + Ssmall, 32 columns at a time: the loads of chunk ch + 1
-        // are in flight while chunk ch is exponentiated; once the last chunk
-        // is in registers the TMEM columns may be reused.  P.v in registers,
-        // a partial sum per tile (two-level accumulation).
+        // S, 32 columns at a time: the loads of chunk ch + 1 are in flight
+        // while chunk ch is exponentiated; once the last chunk is in registers
+        // the TMEM columns may be reused.  P.v in registers, a partial sum per
+        // tile (two-level accumulation).
         constexpr int NCH = BN / 32;
-        const uint32_t tSs = tmem + lane_base + Cfg::col_ss(h);
-        uint32_t cb[32], cs[32];
+        uint32_t cb[32];
         tmem_ld32(tS, cb);
-        if constexpr (SPLIT) {
-          tmem_ld32(tSs, cs);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) cs[e] = 0u;   // no small products
-        }
         tmem_wait_ld();
         reg_fence32(cb);
-        reg_fence32(cs);
         // P.v partial sums of this tile, even and odd columns packed
         uint64_t s0 = 0ull, s1 = 0ull, s2 = 0ull;
 #pragma unroll
         for (int ch = 0; ch < NCH; ++ch) {
           if constexpr (!LSE) {
-            // t = (Sbig + Ssmall) 2c + r + q_j, two columns per packed operation
+            // t = S 2c + r + q_j, two columns per packed operation
             uint64_t cur2[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              uint64_t sv2 = pk2(__uint_as_float(cb[2 * e]), __uint_as_float(cb[2 * e + 1]));
-              if constexpr (SPLIT)
-                sv2 = add2(sv2, pk2(__uint_as_float(cs[2 * e]), __uint_as_float(cs[2 * e + 1])));
-              cur2[e] = fma2(sv2, two_c2, r2);
-            }
+            for (int e = 0; e < 16; ++e)
+              cur2[e] = fma2(pk2(__uint_as_float(cb[2 * e]), __uint_as_float(cb[2 * e + 1])), two_c2, r2);
             if (ch + 1 < NCH) {
               tmem_ld32(tS + (ch + 1) * 32, cb);
-              if constexpr (SPLIT) tmem_ld32(tSs + (ch + 1) * 32, cs);
             } else {
               tc_fence_before();
               mbar_arrive(bar_f(h));
@@ -597,10 +605,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             float cur[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              cur[e] = fmaf(__uint_as_float(cb[e]) + __uint_as_float(cs[e]), two_c, r);
+              cur[e] = fmaf(__uint_as_float(cb[e]), two_c, r);
             if (ch + 1 < NCH) {
               tmem_ld32(tS + (ch + 1) * 32, cb);
-              if constexpr (SPLIT) tmem_ld32(tSs + (ch + 1) * 32, cs);
             } else {
               tc_fence_before();
               mbar_arrive(bar_f(h));
@@ -631,7 +638,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ch + 1 < NCH) {
             tmem_wait_ld();
             reg_fence32(cb);
-            reg_fence32(cs);
           }
         }
         if constexpr (!LSE) {   // (log-sum-exp: the running (m, l) are mx*, acc*)
@@ -645,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc2 += lo + hi;
           }
         }
-        mbar_arrive(bar_empty(st));
+        mbar_arrive(RSEP ? bar_rempty(t % NRM) : bar_empty(st));
       } else {
         // the whole S tile into registers; then its TMEM columns may be reused
         uint32_t sv[BN / 32][32];
@@ -774,6 +780,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     for (int t = issued > NST ? issued - NST : 0; t < issued; ++t)
       drain_bar(bar_full(t % NST), (t / NST) & 1, wlim);
+    if constexpr (RSEP)
+      for (int t = issued > NR ? issued - NR : 0; t < issued; ++t)
+        drain_bar(bar_rfull(t % NRM), (t / NRM) & 1, wlim);
     if constexpr (!Cfg::XT) drain_bar(bar_x, 0, wlim);
   }
   if (warp == 1 && lane == 0) drain_bar(bar_o, 0, wlim);

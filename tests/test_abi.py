@@ -68,7 +68,7 @@ def test_invalid_arguments_are_rejected_before_any_launch(fn):
 
 
 def test_every_entry_point_takes_half_precision():
-    # fp16 / bf16: the log-sum-exp (exact tf32 operands) asks for its workspace;
+    # fp16 / bf16: the log-sum-exp (unsplit tensor-core operands) asks for its workspace;
     # its backward and kNN widen the inputs to fp32 copies in the workspace
     assert _fwd("gauss_lse_fwd", dt=1, D=32) == 4
     assert _fwd("gauss_lse_fwd", dt=2, D=3) == 4
@@ -81,7 +81,7 @@ def test_every_entry_point_takes_half_precision():
 
 
 def test_fp32_wide_features_route_to_the_tensor_core_path():
-    # fp32 with D > 8: sums, the log-sum-exp and its backward (split-tf32 tensor
+    # fp32 with D > 8: sums, the log-sum-exp and its backward (split-fp16 tensor
     # cores) and kNN (chunked CUDA-core kernel) ask for their workspace
     assert _fwd("gauss_lse_fwd", D=9) == 4
     assert _fwd("gauss_sum_fwd", D=9) == 4

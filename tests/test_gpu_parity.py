@@ -136,7 +136,7 @@ HALF_SHAPES = [
     # one and two column tiles with several channels (the three-buffer S ring's edges)
     (1, 300, 100, 32, 8), (2, 130, 128, 20, 40), (1, 257, 250, 62, 64),
 ]
-# fp32 with D > 8: the split-tf32 tensor-core path (every packed-row width, one
+# fp32 with D > 8: the split-fp16 tensor-core path (every packed-row width, one
 # and two value passes, single and several column tiles per warpgroup)
 F32_TC_SHAPES = [
     (1, 1, 1, 9, 1), (1, 1, 300, 12, 1), (1, 300, 700, 9, 1), (1, 257, 1000, 16, 3),
@@ -251,7 +251,7 @@ def test_lse_f32_shapes(shape):
 @pytest.mark.parametrize("shape,tau", [((1, 300, 700, 16, 1), 1.0), ((2, 200, 500, 32, 2), 1.0),
                                        ((1, 130, 1000, 100, 1), 1.0), ((1, 257, 900, 24, 3), 30.0)])
 def test_lse_f32_tensor_core_shapes(shape, tau):
-    """fp32 with D > 8: the log-sum-exp on the split-tf32 path (running maximum)."""
+    """fp32 with D > 8: the log-sum-exp on the split-fp16 path (running maximum)."""
     B, M, N, D, C = shape
     inp = synth.make_inputs(3, seed=41, B=B, M=M, N=N, D=D, C=C)
     inp["x"] = (inp["x"].double() / D ** 0.5).float()   # unit-scale clouds in D dimensions
@@ -270,7 +270,7 @@ def test_lse_f32_tensor_core_shapes(shape, tau):
                                              ("bf16", (1, 190, 640, 17, 1), 4.0),
                                              ("f16", (3, 100, 333, 16, 2), 1.0)])
 def test_lse_half_precision_shapes(dtype, shape, tau):
-    """fp16 / bf16 log-sum-exp: exact tf32 operands on the tensor-core path."""
+    """fp16 / bf16 log-sum-exp: the input values, unsplit, on the tensor-core path."""
     B, M, N, D, C = shape
     inp = synth.make_inputs(3, seed=43, B=B, M=M, N=N, D=D, C=C, dtype=dtype)
     inp["x"] = (inp["x"].double() / D ** 0.5).to(inp["x"].dtype)
@@ -352,7 +352,7 @@ def test_empty_inputs():
     assert torch.equal(saved, torch.zeros(2, 5, 4 * 33, device="cuda"))
     gx, gw = m.gauss_sum_bwd_saved(xh, yh, wh, torch.randn(2, 5, 4, device="cuda"), saved, 1.0)
     assert torch.equal(gx, torch.zeros_like(gx)) and gw.shape == (2, 0, 4)
-    # log-sum-exp on the tf32 paths (fp16, and fp32 with D > 8)
+    # log-sum-exp on the tensor-core paths (fp16, and fp32 with D > 8)
     assert torch.isneginf(m.gauss_lse_fwd(xh, yh, wh, 1.0)).all()
     xw, yw, ww0 = torch.randn(1, 6, 20, device="cuda"), torch.empty(1, 0, 20, device="cuda"), \
         torch.empty(1, 0, 1, device="cuda")
@@ -630,7 +630,7 @@ def test_vjp_d32_c1_full_size_sampled():
                                          ((1, 200, 500, 16, 1), 0.0), ((2, 150, 300, 32, 2), 0.0),
                                          ((1, 180, 400, 24, 1), 30.0)])
 def test_lse_bwd_every_gradient(shape, shift):
-    """D > 8 runs the tf32 tensor-core passes (coordinates scaled by sqrt(3/D) so that
+    """D > 8 runs the tensor-core passes (coordinates scaled by sqrt(3/D) so that
     the clouds have the spread of the D = 3 ones)."""
     B, M, N, D, C = shape
     inp = synth.make_inputs(3, seed=17, B=B, M=M, N=N, D=D, C=C, with_g=True, tau=20.0)
