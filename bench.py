@@ -258,6 +258,27 @@ def kernel_evals_per_step(w, two_call=False):
     return w.pairs * (("sum" in w.ops) + ("lse" in w.ops) + ("bwd" in w.ops))
 
 
+def tensor_flops_per_step(w):
+    """Tensor-core FLOPs (2 per multiply-add) one step needs by the method's own
+    arithmetic, or 0 where the pair work runs on the CUDA cores (fp32, D <= 8) or
+    the step mixes passes (the backward workloads report the MUFU bound).
+    fp32 inputs, D > 8: each value product is three fp16-part products, so the
+    similarity costs 3 * 2D a pair, and P.v with values on the tensor cores (more
+    than three channels) 3 * 2C a pair.  fp16 / bf16: the similarity on rows
+    augmented by the two norm terms, 2 (D + 2) a pair, and P.v 2C a pair for more
+    than one channel (one channel is summed in registers); their log-sum-exp
+    takes the unsplit rows, 2D a pair."""
+    if "bwd" in w.ops or (w.dtype == "f32" and w.D <= 8):
+        return 0
+    if w.dtype == "f32":
+        sum_pp = 6 * w.D + (6 * w.C if w.C > 3 else 0)
+        lse_pp = 6 * w.D
+    else:
+        sum_pp = 2 * (w.D + 2) + (2 * w.C if w.C > 1 else 0)
+        lse_pp = 2 * w.D
+    return w.pairs * (sum_pp * ("sum" in w.ops) + lse_pp * ("lse" in w.ops))
+
+
 def launches_per_step(gs, run):
     """Kernels one step launches, counted by the CUDA profiler (names prove they are ours)."""
     from torch.profiler import ProfilerActivity, profile
@@ -586,6 +607,21 @@ def main():
                 "peak_basis": f"16 ex2/clk/SM x {sms} SMs x {sm_max:.0f} MHz (max SM clock)"}
         if clocks.get("sm_mhz"):
             roof["frac_at_measured_clock"] = achieved / (EX2_PER_CLK_PER_SM * sms * clocks["sm_mhz"] * 1e-3)
+        # The binding resource: the tensor pipe where the step's MMA FLOPs need more time
+        # at the measured dense bf16 / fp16 rate than its exponentials at the MUFU rate.
+        tf = tensor_flops_per_step(w) * jobs / world
+        t_peak = peaks.get("bf16_tflops")
+        if tf and t_peak and tf / (t_peak * 1e12) > kevals * jobs / world / (peak * 1e9):
+            t_ach = tf / (ms_per_step * 1e-3) / 1e12
+            roof = {"bound": "tensor",
+                    "kernel": f"{dom}: fp16 MMAs, {tf / (kevals * jobs / world):.0f} FLOP per pair",
+                    "achieved": t_ach, "peak": t_peak, "unit": "TFLOP/s", "frac": t_ach / t_peak,
+                    "traffic": traffic,
+                    "peak_basis": "measured cuBLAS bf16 GEMM, burst (fp16 has the same rate)",
+                    "frac_of_sustained": t_ach / peaks["bf16_tflops_sustained"]
+                    if peaks.get("bf16_tflops_sustained") else None,
+                    "alu": {"achieved": achieved, "peak": peak, "unit": "G kernel evaluations/s",
+                            "frac": achieved / peak}}
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             cpu, _ = oracle_sample(w, inp, args.cpu_seconds)

@@ -1,6 +1,6 @@
 """bench.py's host-side bookkeeping, on the CPU: which kernel does each
-workload's pair work, how pairs and kernel evaluations are counted per step,
-and when the committed ncu traffic figure may be reported."""
+workload's pair work, how pairs, kernel evaluations and tensor-core FLOPs are
+counted per step, and when the committed ncu traffic figure may be reported."""
 import hashlib
 import os
 import shutil
@@ -38,6 +38,21 @@ def test_pairs_and_kernel_evaluations_per_step():
     assert bench.fused_fwd_bwd(w["d32_c1_bwd"])
     assert bench.kernel_evals_per_step(w["d32_c1_bwd"]) == p
     assert bench.kernel_evals_per_step(w["d32_c1_bwd"], two_call=True) == 2 * p
+
+
+def test_tensor_flops_per_step():
+    w = synth.BY_NAME
+    per = lambda n: bench.tensor_flops_per_step(w[n]) / w[n].pairs
+    # CUDA-core path (fp32, D <= 8) and the mixed-pass backward: no tensor roofline
+    assert per("d3_100k") == per("d3_1m_lse") == per("d32_c1_bwd") == 0
+    # fp32, D > 8: three fp16-part products per value product (one register
+    # channel: the similarity alone; 32 channels: P.v on the tensor cores too)
+    assert per("b64_d32_f32") == 3 * 2 * 32
+    assert per("b64_d128_f32") == 3 * 2 * 128
+    assert per("d32_c32_f32") == 3 * 2 * 32 + 3 * 2 * 32
+    # fp16: rows augmented by the two norm terms; one channel summed in registers
+    assert per("b64_d32_f16") == 2 * (32 + 2)
+    assert per("d32_c32") == 2 * (32 + 2) + 2 * 32
 
 
 def test_traffic_figure_only_while_the_kernel_source_is_unchanged(tmp_path, monkeypatch):
