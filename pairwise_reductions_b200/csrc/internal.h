@@ -202,7 +202,7 @@ struct F32Plan {
   bool split;          // fp32 inputs: fp16 rows [hi | lo]; fp16 / bf16: the input values, unsplit
   int Kp;              // 16-bit elements per half of a packed row: D rounded up to 16
   int atoms;           // 128-byte atoms per packed row (2 Kp or Kp 16-bit values)
-  int max_chunk;       // channels per pass (64, or 32 for the widest rows)
+  int max_chunk;       // channels per pass (64)
   int splits;
   int64_t cols_per_split;   // multiple of 128
 };

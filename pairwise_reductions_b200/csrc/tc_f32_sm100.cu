@@ -118,6 +118,9 @@ struct F32Cfg {
     return KA * bn * 128 + (NR > 0 ? 0 : qw_bytes(bn)) + v_bytes(bn);
   }
   static constexpr int rec_bytes(int bn) { return NR * qw_bytes(bn); }
+  // tensor-core values: each warpgroup's running fp32 sums of its drained O
+  // groups, [warpgroup][channel][row] (a thread's own row: conflict-free)
+  static constexpr int ORUN_BYTES = REG ? 0 : 2 * kBM * CP * 4;
   static constexpr int BUDGET = 214 * 1024;
   // TMEM columns of the accumulators: one S per warpgroup (every small
   // product first, while the sum is small, then the large ones: each addition
@@ -131,7 +134,8 @@ struct F32Cfg {
   static constexpr bool xt(int bn) { return tmem_acc(bn) + 32 * KA <= 512; }
   static constexpr int x_bytes(int bn) { return xt(bn) ? 0 : KA * kAtom; }
   static constexpr bool fits(int bn) {
-    return tmem_acc(bn) <= 512 && (BUDGET - x_bytes(bn) - rec_bytes(bn)) / stage_bytes(bn) >= 2;
+    return tmem_acc(bn) <= 512 &&
+           (BUDGET - x_bytes(bn) - rec_bytes(bn) - ORUN_BYTES) / stage_bytes(bn) >= 2;
   }
   // Column tile.  An M = 128, K = 16 MMA costs much the same at N = 32 and 64
   // and a third more at 128 (measured on B200: 47, 49 and 65 issue cycles), so
@@ -148,12 +152,12 @@ struct F32Cfg {
   static constexpr int V_BYTES = v_bytes(BN);
   static constexpr int STAGE = stage_bytes(BN);
   static constexpr int REC_BYTES = rec_bytes(BN);
-  static constexpr int NST_FIT = (BUDGET - X_BYTES - REC_BYTES) / STAGE;
+  static constexpr int NST_FIT = (BUDGET - X_BYTES - REC_BYTES - ORUN_BYTES) / STAGE;
   static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
   static constexpr int NBARS = 2 * NST + 10 + 2 * NR;
   static constexpr int RED_BYTES = kBM * 32;            // warpgroup 1 partial sums (m, l)
   static constexpr int SMEM_RAW =
-      1024 + X_BYTES + NST * STAGE + REC_BYTES + 8 * NBARS + 16 + RED_BYTES;
+      1024 + X_BYTES + NST * STAGE + REC_BYTES + ORUN_BYTES + 8 * NBARS + 16 + RED_BYTES;
   // at least ~120 KB: one CTA per SM, so the 512-column TMEM allocation never waits
   static constexpr int SMEM = SMEM_RAW < 122880 ? 122880 : SMEM_RAW;
   // TMEM columns.  Register values: S0 | S1 | x'.
@@ -225,6 +229,12 @@ __device__ __forceinline__ float pow2_int(int k) { return __int_as_float((k + 12
 // Tensor-core values: P is multiplied by 2^14 before its fp16 split, which
 // keeps every P at or above 2^-28 in fp16's normal range.
 constexpr float kPScale = 16384.f;
+// Tensor-core values: column tiles a warpgroup's O accumulator sums before the
+// exp warps add it into fp32 registers and the P.v MMAs start it afresh.  The
+// tensor core rounds each MMA's addition into its fp32 accumulator, and over the
+// ~2000 additions of a 65536-column split that drift reached 7.6e-5 of the sum
+// (B = 4, N = 65536, 32 channels); 16 tiles (64 additions) keep it near 2e-6.
+constexpr int kOGroup = 16;
 
 // Named barrier of the two exp warpgroups (warps 2-9).
 __device__ __forceinline__ void exp_warps_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
@@ -257,7 +267,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sX = smem;
   uint8_t* sStage = smem + Cfg::X_BYTES;
   uint8_t* sRec = sStage + NST * Cfg::STAGE;   // register values: the records ring
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sRec + Cfg::REC_BYTES);
+  float* sOrun = reinterpret_cast<float*>(sRec + Cfg::REC_BYTES);   // tensor-core values
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sRec + Cfg::REC_BYTES + Cfg::ORUN_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float4* red = reinterpret_cast<float4*>(tmem_slot + 4);   // 16-byte aligned
@@ -482,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (!REG) {
             if (!(ok = wait_bar(bar_p(h), k & 1, abort_flag, wlim))) break;
             tc_fence_after();
-            issue_O(h, t % NST, k > 0);
+            issue_O(h, t % NST, k % kOGroup != 0);
             mma_commit(bar_q(h));
             mma_commit(bar_empty(t % NST));
             if (!kSFirst && t2 < T && !(ok = next_S(h, k, t2))) break;
@@ -539,8 +550,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = false;
     }
     int k = 0;
+    // tensor-core values: this warpgroup's O summed over the drained tile groups,
+    // this thread's row of it in shared memory (channel c at orun[c * kBM])
+    float* orun = sOrun + h * CP * kBM + row;
+    if constexpr (!REG) {
+#pragma unroll 4
+      for (int c = 0; c < CP; ++c) orun[c * kBM] = 0.f;
+    }
+    const uint32_t tOh = tmem + lane_base + Cfg::col_o(h);
+    // O_h (big + small) added into orun, 16 channels at a time
+    auto add_o = [&]() {
+#pragma unroll 1
+      for (int ch = 0; ch < (REG ? 0 : CP / 16); ++ch) {
+        uint32_t vb[16], vs[16];
+        tmem_ld16(tOh + ch * 16, vb);
+        tmem_ld16(tOh + CP + ch * 16, vs);
+        tmem_wait_ld();
+        reg_fence16(vb);
+        reg_fence16(vs);
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          orun[(ch * 16 + q) * kBM] += __uint_as_float(vb[q]) + __uint_as_float(vs[q]);
+      }
+    };
     for (int t = h; ok && t < T; t += 2, ++k) {
       const int st = t % NST;
+      if constexpr (!REG) {
+        if (k > 0 && k % kOGroup == 0) {
+          // O_h has summed kOGroup tiles: once their P.v MMAs are done, into the
+          // registers; tile k's P.v MMAs then start O_h afresh
+          ok = __all_sync(0xffffffffu, wait_bar(bar_q(h), (k - 1) & 1, abort_flag, wlim));
+          if (!ok) break;
+          tc_fence_after();
+          add_o();
+        }
+      }
       ok = wait_bar(bar_s(h), k & 1, abort_flag, wlim) &&   // norms and values landed
            (RSEP ? wait_bar(bar_rfull(t % NRM), (t / NRM) & 1, abort_flag, wlim)
                 : wait_bar(bar_full(st), (t / NST) & 1, abort_flag, wlim));
@@ -734,40 +778,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) ok = wait_bar(bar_o, 0, abort_flag, wlim);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
-      if (ok && h == 0) {
-        const uint32_t tO0 = tmem + lane_base + Cfg::col_o(0);
-        const uint32_t tO1 = tmem + lane_base + Cfg::col_o(1);
+      // Each warpgroup's total: the drained groups plus the open one still in O_h
+      // (none when the warpgroup had no tile); then warpgroup 0 adds warpgroup 1's
+      // (both warpgroups reach the barrier)
+      const int kh = (T - h + 1) / 2;   // column tiles of warpgroup h
+      if (ok && kh > 0) add_o();
+      exp_warps_sync();
+      if (ok && h == 0 && valid) {
         float* orow = p.out + static_cast<int64_t>(blockIdx.y) * p.split_stride +
                       (b * p.M + i) * p.ldo + p.c0;
-#pragma unroll
-        for (int ch = 0; ch < CP / 16; ++ch) {
-          // O_h = O_big + O_small of each warpgroup, then O_0 + O_1
-          float o[16];
-          uint32_t vb[16], vs[16];
-          tmem_ld16(tO0 + ch * 16, vb);
-          tmem_ld16(tO0 + CP + ch * 16, vs);
-          tmem_wait_ld();
-          reg_fence16(vb);
-          reg_fence16(vs);
-#pragma unroll
-          for (int q = 0; q < 16; ++q)
-            o[q] = T > 0 ? __uint_as_float(vb[q]) + __uint_as_float(vs[q]) : 0.f;
-          tmem_ld16(tO1 + ch * 16, vb);
-          tmem_ld16(tO1 + CP + ch * 16, vs);
-          tmem_wait_ld();
-          reg_fence16(vb);
-          reg_fence16(vs);
-          if (valid) {
-#pragma unroll
-            for (int q = 0; q < 16; ++q) {
-              const int c = ch * 16 + q;
-              // O_1 holds tiles only when T > 1
-              if (T > 1) o[q] += __uint_as_float(vb[q]) + __uint_as_float(vs[q]);
-              // undo P's 2^14 and the channel's 2^e, exactly
-              if (c < p.cw) orow[c] = o[q] * pow2_int(-14 - split_exp(p.vmax[b * CP + c]));
-            }
-          }
-        }
+        const float* orun1 = sOrun + CP * kBM + row;
+        for (int c = 0; c < p.cw; ++c)   // undo P's 2^14 and the channel's 2^e, exactly
+          orow[c] = (orun[c * kBM] + orun1[c * kBM]) *
+                    pow2_int(-14 - split_exp(p.vmax[b * CP + c]));
       }
     }
   }
@@ -1088,14 +1111,13 @@ cudaError_t launch_mode(int mode, bool lse, const TileMaps& m, const F32KParams&
     case 3: return launch_kernel<KA, 3>(m, kp, grid, s);
     case 16: return launch_kernel<KA, 16>(m, kp, grid, s);
     case 32: return launch_kernel<KA, 32>(m, kp, grid, s);
-    default:
-      if constexpr (KA < 8) return launch_kernel<KA, 64>(m, kp, grid, s);
-      return cudaErrorInvalidValue;
+    default: return launch_kernel<KA, 64>(m, kp, grid, s);
   }
 }
 
 // Shared-memory atoms the kernel is compiled for, covering `atoms`.
-int ka_for(int atoms) { return atoms <= 1 ? 1 : (atoms <= 2 ? 2 : (atoms <= 4 ? 4 : (atoms <= 6 ? 6 : 8))); }
+// (D <= 128: a split row [hi K' | lo K'] holds at most four 128-byte atoms)
+int ka_for(int atoms) { return atoms <= 1 ? 1 : (atoms <= 2 ? 2 : 4); }
 
 // Tile width of instantiation (KA, mode): the host sizes the TMA boxes with it.
 template <int KA>
@@ -1105,9 +1127,7 @@ int tile_cols_ka(int mode) {
     case 3: return F32Cfg<KA, 3>::BN;
     case 16: return F32Cfg<KA, 16>::BN;
     case 32: return F32Cfg<KA, 32>::BN;
-    default:
-      if constexpr (KA < 8) return F32Cfg<KA, 64>::BN;
-      return 0;
+    default: return F32Cfg<KA, 64>::BN;
   }
 }
 
@@ -1121,7 +1141,7 @@ F32Plan f32_plan(int64_t B, int64_t M, int64_t N, int64_t D, int sm_count, bool 
   // (split) or the fp16 / bf16 input values (unsplit)
   p.Kp = static_cast<int>((D + 15) / 16 * 16);
   p.atoms = ((split ? 2 : 1) * p.Kp + 63) / 64;
-  p.max_chunk = ka_for(p.atoms) >= 8 ? 32 : 64;
+  p.max_chunk = 64;
   // a split is a whole number of 128-column blocks (every tile width divides
   // it, so no tile straddles two splits)
   const int64_t U = B * ((M + kBM - 1) / kBM);
@@ -1152,9 +1172,7 @@ int f32_tile_cols(int KA, int mode) {
   switch (KA) {
     case 1: return tile_cols_ka<1>(mode);
     case 2: return tile_cols_ka<2>(mode);
-    case 4: return tile_cols_ka<4>(mode);
-    case 6: return tile_cols_ka<6>(mode);
-    default: return tile_cols_ka<8>(mode);
+    default: return tile_cols_ka<4>(mode);
   }
 }
 
@@ -1325,9 +1343,7 @@ cudaError_t launch_tc_f32_sum(const F32Args& a, cudaStream_t s) {
     switch (KA) {
       case 1: e = launch_mode<1>(mode, a.lse, m, kp, grid, s); break;
       case 2: e = launch_mode<2>(mode, a.lse, m, kp, grid, s); break;
-      case 4: e = launch_mode<4>(mode, a.lse, m, kp, grid, s); break;
-      case 6: e = launch_mode<6>(mode, a.lse, m, kp, grid, s); break;
-      default: e = launch_mode<8>(mode, a.lse, m, kp, grid, s); break;
+      default: e = launch_mode<4>(mode, a.lse, m, kp, grid, s); break;
     }
     if (e != cudaSuccess) return e;
   }

@@ -96,6 +96,25 @@ def test_d32_c1_f16_fwd_bwd_sampled():
     assert rel_l2(gw[:, wrows], rgw) <= TOL["f16"], rel_l2(gw[:, wrows], rgw)
 
 
+@pytest.mark.parametrize("name,nrows", [("b64_d32_f16", 24), ("b64_d32_f32", 24),
+                                        ("b64_d128_f32", 16), ("d32_c32_f32", 96)])
+def test_bench_workload_full_size_sampled(name, nrows):
+    """The other workloads bench.py times (the points of "Fast Gauss Sums via Flash
+    Attention", Figures 3-5: B = 64 batches of 16384 x 16384 at D = 32 and 128,
+    fp16 and fp32; B = 4 of 65536 x 65536 with 32 channels, fp32), at full size in
+    the launch configuration the benchmark uses, against the oracle on sampled rows
+    of every batch."""
+    w = synth.BY_NAME[name]
+    inp = synth.make_inputs(w)
+    d = dev(inp)
+    out = gs().gauss_sum_fwd(d["x"], d["y"], d["w"], inp["tau"]).cpu().numpy()
+    del d
+    rows = synth.sample_rows(inp["M"], nrows, seed=12).numpy()
+    ref = oracle.gauss_sum(f64(inp, "x"), f64(inp, "y"), f64(inp, "w"), inp["tau"], rows=rows)
+    tol = TOL["f32"] if w.dtype == "f32" else TOL["f16"]
+    assert rel_l2(out[:, rows], ref) <= tol, rel_l2(out[:, rows], ref)
+
+
 def test_d32_c1_f16_saved_pair_full_size():
     """The call pair the benchmark times for this workload (B=4, M=N=16384, D=32,
     C=1, fp16): gauss_sum_fwd_saved then gauss_sum_bwd_saved, at full size and in
