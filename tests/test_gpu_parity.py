@@ -117,10 +117,10 @@ def test_bench_workload_full_size_sampled(name, nrows):
 
 def test_d32_c1_f16_saved_pair_full_size():
     """The call pair the benchmark times for this workload (B=4, M=N=16384, D=32,
-    C=1, fp16): gauss_sum_fwd_saved then gauss_sum_bwd_saved, at full size and in
-    the same launch configuration, against the oracle on sampled rows and
-    sources; and bit for bit against the separate backward entry point, which
-    runs the same passes."""
+    C=1, fp16): gauss_sum_fwd_saved then gauss_sum_bwd_saved (`--two-call`), at
+    full size and in the same launch configuration, against the oracle on
+    sampled rows and sources; bit for bit against the separate backward entry
+    point, which runs the same passes; and the one-sweep gauss_sum_fwd_bwd."""
     inp = synth.make_inputs(5)
     d = dev(inp)
     m = gs()
@@ -138,6 +138,13 @@ def test_d32_c1_f16_saved_pair_full_size():
     assert rel_l2(gwn[:, wrows], rgw) <= TOL["f16"], rel_l2(gwn[:, wrows], rgw)
     bx, bw = m.gauss_sum_bwd(d["x"], d["y"], d["w"], d["g"], inp["tau"])
     assert torch.equal(bx, gx) and torch.equal(bw, gw)
+    # the one-sweep call the benchmark times by default for this workload: the
+    # sum and grad_x bit for bit those of the saved pair, grad_w (P^T g from the
+    # same sweep) against the oracle on the sampled sources
+    fo, fx, fw = m.gauss_sum_fwd_bwd(d["x"], d["y"], d["w"], d["g"], inp["tau"])
+    assert torch.equal(fo, out) and torch.equal(fx, gx)
+    fwn = fw.cpu().numpy()
+    assert rel_l2(fwn[:, wrows], rgw) <= TOL["f16"], rel_l2(fwn[:, wrows], rgw)
 
 
 # ------------------------------------------------------------------ odd shapes, both paths
