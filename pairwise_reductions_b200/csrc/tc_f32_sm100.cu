@@ -22,19 +22,20 @@
 // (the norm factors of Algorithm 1 on the same page).  P_ij = ex2(fma(S, 2c, r_i) + q_j)
 // with S from the split MMAs; P is split into fp16 hi/lo parts again for P.v.
 //
-// CTA = one 128-row tile, 10 warps:
+// CTA = one 128-row tile, 2 + 4 NWG warps:
 //   warp 0      TMA producer: the x' rows once (unless they sit in TMEM), then a
 //               ring of stages: y' tile, the column records lane by lane (q_j,
 //               then values or log2 values), and for tensor-core values the
 //               split v^T tile
 //   warp 1      TMEM owner + single-thread MMA issuer
-//   warps 2-5   exp warpgroup 0: column tiles 0, 2, 4, ...
-//   warps 6-9   exp warpgroup 1: column tiles 1, 3, 5, ...
-// Both warpgroups hold the same rows (TMEM lanes), so each keeps its own
-// partial result and warpgroup 0 combines the two at the end.  Per column tile
+//   warps 2..   NWG exp warpgroups (three with register values, two with
+//               tensor-core values); warpgroup h takes column tiles h, h + NWG, ...
+// The warpgroups hold the same rows (TMEM lanes), so each keeps its own
+// partial result and warpgroup 0 combines them at the end.  Per column tile
 // t of warpgroup h:
-//   S_h  = x'.y'(t)^T                 3 fp16 MMAs per K step of 16 (A from
-//                                     shared memory, or from TMEM when it has room)
+//   S_h  = x'.y'(t)^T                 3 fp16 MMAs per K step of 16 into one
+//                                     accumulator (A from TMEM when it has room,
+//                                     else from shared memory)
 //   P_h  = ex2(fma(S_h, 2c, r) + q)   tcgen05.ld -> MUFU
 // then either (register values, <= 3 channels, and the log-sum-exp)
 //   row sums += P_h . v in registers, exact fp32 FMAs (or a running maximum and
@@ -68,7 +69,6 @@ __device__ int g_test_stall_f32;
 namespace {
 
 constexpr int kBM = 128;        // rows per CTA (one MMA tile)
-constexpr int kThreads = 320;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kAtom = kBM * 128;   // one 128-row x 32-float (128-byte) swizzle atom
 
@@ -100,6 +100,12 @@ struct F32KParams {
 template <int KA, int MODE>
 struct F32Cfg {
   static constexpr bool REG = MODE <= 3;
+  // exp warpgroups, each taking every NWG-th column tile of the CTA's rows.
+  // Register values: three (S of all three fits TMEM, and a third warp per
+  // sub-partition hides more of the exponent chain's latency); tensor-core
+  // values: two (S, P and O per warpgroup).  Plus a producer and an MMA warp.
+  static constexpr int NWG = REG ? 3 : 2;
+  static constexpr int THREADS = 64 + 128 * NWG;
   static constexpr int CP = REG ? 16 : MODE;
   static constexpr int CPA = (CP + 31) / 32 * 32;
   static constexpr int qw_bytes(int bn) { return bn * 16 <= 1024 ? 1024 : bn * 16; }
@@ -128,7 +134,7 @@ struct F32Cfg {
   // add P hi/lo (fp16 pairs: bn / 2 columns each) and O per warpgroup, O as
   // two halves of CP columns: O_big (P_hi v_hi + P_lo v_hi) and O_small
   // (P_hi v_lo), added in the epilogue.
-  static constexpr int tmem_acc(int bn) { return REG ? 2 * bn : 4 * bn + 4 * CPA; }
+  static constexpr int tmem_acc(int bn) { return REG ? NWG * bn : 4 * bn + 4 * CPA; }
   // The x' rows (2 K' <= 32 KA columns) sit in TMEM as the A operand of the
   // similarity MMAs when the accumulators leave room, else in shared memory.
   static constexpr bool xt(int bn) { return tmem_acc(bn) + 32 * KA <= 512; }
@@ -154,8 +160,8 @@ struct F32Cfg {
   static constexpr int REC_BYTES = rec_bytes(BN);
   static constexpr int NST_FIT = (BUDGET - X_BYTES - REC_BYTES - ORUN_BYTES) / STAGE;
   static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
-  static constexpr int NBARS = 2 * NST + 10 + 2 * NR;
-  static constexpr int RED_BYTES = kBM * 32;            // warpgroup 1 partial sums (m, l)
+  static constexpr int NBARS = 2 * NST + 2 + 4 * NWG + 2 * NR;
+  static constexpr int RED_BYTES = (NWG - 1) * kBM * 32;   // warpgroups 1.. partial sums (m, l)
   static constexpr int SMEM_RAW =
       1024 + X_BYTES + NST * STAGE + REC_BYTES + ORUN_BYTES + 8 * NBARS + 16 + RED_BYTES;
   // at least ~120 KB: one CTA per SM, so the 512-column TMEM allocation never waits
@@ -237,7 +243,10 @@ constexpr float kPScale = 16384.f;
 constexpr int kOGroup = 16;
 
 // Named barrier of the two exp warpgroups (warps 2-9).
-__device__ __forceinline__ void exp_warps_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// every exp warp of the CTA (nthreads = 128 per warpgroup)
+__device__ __forceinline__ void exp_warps_sync(int nthreads) {
+  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
 
 // LSE (register values, one channel): per row, the log-sum-exp of
 // t_ij + log2 w_j as a running maximum m and a sum l of 2^(t - m), updated per
@@ -246,7 +255,7 @@ __device__ __forceinline__ void exp_warps_sync() { asm volatile("bar.sync 1, 256
 // SPLIT: rows [hi | lo] and three products per K step (fp32 inputs), or the
 // exact fp16 / bf16 input rows and the large product alone.
 template <int KA, int MODE, bool LSE, bool SPLIT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(F32Cfg<KA, MODE>::THREADS, 1)
     tc_f32_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                   const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmV,
                   const F32KParams p) {
@@ -277,16 +286,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_full = [&](int s) { return bar0 + 8u * s; };
   auto bar_empty = [&](int s) { return bar0 + 8u * (NST + s); };
   const uint32_t bar_x = bar0 + 8u * (2 * NST);
-  auto bar_s = [&](int h) { return bar0 + 8u * (2 * NST + 1 + h); };   // S_h ready
-  auto bar_f = [&](int h) { return bar0 + 8u * (2 * NST + 3 + h); };   // S_h read out
-  auto bar_p = [&](int h) { return bar0 + 8u * (2 * NST + 5 + h); };   // P_h written
-  auto bar_q = [&](int h) { return bar0 + 8u * (2 * NST + 7 + h); };   // P_h consumed
-  const uint32_t bar_o = bar0 + 8u * (2 * NST + 9);
+  constexpr int NWG = Cfg::NWG;
+  auto bar_s = [&](int h) { return bar0 + 8u * (2 * NST + 1 + h); };             // S_h ready
+  auto bar_f = [&](int h) { return bar0 + 8u * (2 * NST + 1 + NWG + h); };       // S_h read out
+  auto bar_p = [&](int h) { return bar0 + 8u * (2 * NST + 1 + 2 * NWG + h); };   // P_h written
+  auto bar_q = [&](int h) { return bar0 + 8u * (2 * NST + 1 + 3 * NWG + h); };   // P_h consumed
+  const uint32_t bar_o = bar0 + 8u * (2 * NST + 1 + 4 * NWG);
   constexpr int NR = Cfg::NR;
   constexpr bool RSEP = NR > 0;          // the records in a ring of their own
   constexpr int NRM = RSEP ? NR : 1;     // (slot arithmetic)
-  auto bar_rfull = [&](int r) { return bar0 + 8u * (2 * NST + 10 + r); };        // records landed
-  auto bar_rempty = [&](int r) { return bar0 + 8u * (2 * NST + 10 + NR + r); };  // records read
+  auto bar_rfull = [&](int r) { return bar0 + 8u * (2 * NST + 2 + 4 * NWG + r); };        // landed
+  auto bar_rempty = [&](int r) { return bar0 + 8u * (2 * NST + 2 + 4 * NWG + NR + r); };  // read
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t b = blockIdx.z;
@@ -315,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // x' ready: the TMA load (shared memory), or the 128 threads of exp
     // warpgroup 0 that copy the rows into TMEM
     mbar_init(bar_x, Cfg::XT ? 4 * 32 : 1);
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < NWG; ++h) {
       mbar_init(bar_s(h), 1);
       mbar_init(bar_f(h), 4 * 32);
       mbar_init(bar_p(h), 4 * 32);
@@ -462,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       bool ok = wait_bar(bar_x, 0, abort_flag, wlim) && stall != 1;
       tc_fence_after();
-      for (int h = 0; ok && h < 2 && h < T; ++h) {
+      for (int h = 0; ok && h < NWG && h < T; ++h) {
         ok = wait_bar(bar_full(h), 0, abort_flag, wlim);
         if (ok) {
           tc_fence_after();
@@ -471,9 +481,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (RSEP) mma_commit(bar_empty(h % NST));
         }
       }
-      // S_h(t + 2) may overwrite S_h once warpgroup h has read S_h(t).  With
-      // tensor-core values it goes ahead of O_h(t) when tile t + 2 does not
-      // need the stage of tile t (three or more stages), else after it.
+      // S_h(t + NWG) may overwrite S_h once warpgroup h has read S_h(t).  With
+      // tensor-core values (two warpgroups) it goes ahead of O_h(t) when tile
+      // t + 2 does not need the stage of tile t (three or more stages), else
+      // after it.
       constexpr bool kSFirst = REG || NST >= 3;
       auto next_S = [&](int h, int k, int t2) {
         if (!wait_bar(bar_f(h), k & 1, abort_flag, wlim)) return false;
@@ -484,11 +495,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (RSEP) mma_commit(bar_empty(t2 % NST));
         return true;
       };
-      for (int k = 0; ok && 2 * k < T; ++k) {
-        for (int h = 0; h < 2; ++h) {
-          const int t = 2 * k + h;
+      for (int k = 0; ok && NWG * k < T; ++k) {
+        for (int h = 0; h < NWG; ++h) {
+          const int t = NWG * k + h;
           if (t >= T) break;
-          const int t2 = t + 2;
+          const int t2 = t + NWG;
           if (kSFirst && t2 < T && !(ok = next_S(h, k, t2))) break;
           if constexpr (!REG) {
             if (!(ok = wait_bar(bar_p(h), k & 1, abort_flag, wlim))) break;
@@ -573,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           orun[(ch * 16 + q) * kBM] += __uint_as_float(vb[q]) + __uint_as_float(vs[q]);
       }
     };
-    for (int t = h; ok && t < T; t += 2, ++k) {
+    for (int t = h; ok && t < T; t += NWG, ++k) {
       const int st = t % NST;
       if constexpr (!REG) {
         if (k > 0 && k % kOGroup == 0) {
@@ -744,34 +755,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if constexpr (REG) {
-      // warpgroup 1 hands its row sums (or its (m, l)) to warpgroup 0; both
-      // reach this barrier
-      if (h == 1) {
-        red[2 * row] = make_float4(acc0, acc1, acc2, 0.f);
-        red[2 * row + 1] = make_float4(mx0, mx1, mx2, 0.f);
+      // warpgroups 1.. hand their row sums (or their (m, l)) to warpgroup 0,
+      // which adds them in warpgroup order; every exp warp reaches the barrier
+      if (h > 0) {
+        red[2 * ((h - 1) * kBM + row)] = make_float4(acc0, acc1, acc2, 0.f);
+        red[2 * ((h - 1) * kBM + row) + 1] = make_float4(mx0, mx1, mx2, 0.f);
       }
-      exp_warps_sync();
+      exp_warps_sync(NWG * 128);
       if (h == 0 && valid && ok && !*abort_flag) {
-        const float4 o = red[2 * row];
         const int64_t at = static_cast<int64_t>(blockIdx.y) * p.split_stride +
                            (b * p.M + i) * p.ldo + p.c0;
+#pragma unroll
+        for (int g = 1; g < NWG; ++g) {
+          const float4 o = red[2 * ((g - 1) * kBM + row)];
+          if constexpr (!LSE) {
+            acc0 += o.x;
+            acc1 += o.y;
+            acc2 += o.z;
+          } else {
+            const float4 om = red[2 * ((g - 1) * kBM + row) + 1];
+            // (m, l) merged with (m1, l1): the larger shift, both sums rescaled to it
+            auto merge = [&](float& m0, float& l0, float m1, float l1) {
+              const float m = fmaxf(m0, m1);
+              float l = 0.f;
+              if (m != -INFINITY) l = l0 * ex2(m0 - m) + l1 * ex2(m1 - m);
+              m0 = m;
+              l0 = l;
+            };
+            merge(mx0, acc0, om.x, o.x);
+            merge(mx1, acc1, om.y, o.y);
+            merge(mx2, acc2, om.z, o.z);
+          }
+        }
         if constexpr (!LSE) {
           float* orow = p.out + at;
-          orow[0] = acc0 + o.x;
-          if (p.cw > 1) orow[1] = acc1 + o.y;
-          if (p.cw > 2) orow[2] = acc2 + o.z;
+          orow[0] = acc0;
+          if (p.cw > 1) orow[1] = acc1;
+          if (p.cw > 2) orow[2] = acc2;
         } else {
-          const float4 om = red[2 * row + 1];
-          auto merge = [&](int c, float m0, float l0, float m1, float l1) {
-            const float m = fmaxf(m0, m1);
-            float l = 0.f;
-            if (m != -INFINITY) l = l0 * ex2(m0 - m) + l1 * ex2(m1 - m);
-            p.out[at + c] = m;
-            p.out_l[at + c] = l;
-          };
-          merge(0, mx0, acc0, om.x, o.x);
-          if (p.cw > 1) merge(1, mx1, acc1, om.y, o.y);
-          if (p.cw > 2) merge(2, mx2, acc2, om.z, o.z);
+          p.out[at] = mx0;
+          p.out_l[at] = acc0;
+          if (p.cw > 1) { p.out[at + 1] = mx1; p.out_l[at + 1] = acc1; }
+          if (p.cw > 2) { p.out[at + 2] = mx2; p.out_l[at + 2] = acc2; }
         }
       }
     } else {
@@ -781,9 +806,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Each warpgroup's total: the drained groups plus the open one still in O_h
       // (none when the warpgroup had no tile); then warpgroup 0 adds warpgroup 1's
       // (both warpgroups reach the barrier)
-      const int kh = (T - h + 1) / 2;   // column tiles of warpgroup h
+      const int kh = T > h ? (T - h + NWG - 1) / NWG : 0;   // column tiles of warpgroup h
       if (ok && kh > 0) add_o();
-      exp_warps_sync();
+      exp_warps_sync(NWG * 128);
       if (ok && h == 0 && valid) {
         float* orow = p.out + static_cast<int64_t>(blockIdx.y) * p.split_stride +
                       (b * p.M + i) * p.ldo + p.c0;
@@ -1095,7 +1120,7 @@ cudaError_t launch_kernel(const TileMaps& m, const F32KParams& kp, dim3 grid, cu
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  fn<<<grid, kThreads, Cfg::SMEM, s>>>(m.x, m.y, m.q, m.v, kp);
+  fn<<<grid, Cfg::THREADS, Cfg::SMEM, s>>>(m.x, m.y, m.q, m.v, kp);
   return cudaGetLastError();
 }
 
