@@ -112,14 +112,12 @@ struct F32Cfg {
   // v^T in fp16 [hi | lo] parts: 64 columns per 128-byte atom row
   static constexpr int va(int bn) { return bn < 64 ? 1 : bn / 64; }
   static constexpr int v_bytes(int bn) { return REG ? 0 : 2 * va(bn) * CP * 128; }
-  // Register values with wide rows (4+ atoms: two or three stages fit): the
-  // column records sit in a ring of their own, so that a y' stage is free once
-  // the similarity MMAs have read it, while the exp warps still read the
-  // tile's records (b64_d128_f32 +9..16%).  Narrower rows keep four stages of
-  // [y' | records], freed by the exp warps (the ring measured 0.9% slower there).
-  // Tensor-core values: one stage holds y', the records and v^T, freed by the
-  // P.v MMAs.
-  static constexpr int NR = (REG && KA >= 4) ? 4 : 0;
+  // Register values: the column records sit in a ring of their own (two slots
+  // per exp warpgroup), so that a y' stage is free once the similarity MMAs
+  // have read it, while the exp warps still read the tile's records
+  // (b64_d128_f32 +9..16% at two stages).  Tensor-core values: one stage holds
+  // y', the records and v^T, freed by the P.v MMAs.
+  static constexpr int NR = REG ? 2 * NWG : 0;
   static constexpr int stage_bytes(int bn) {
     return KA * bn * 128 + (NR > 0 ? 0 : qw_bytes(bn)) + v_bytes(bn);
   }
@@ -293,7 +291,7 @@ __global__ void __launch_bounds__(F32Cfg<KA, MODE>::THREADS, 1)
   auto bar_q = [&](int h) { return bar0 + 8u * (2 * NST + 1 + 3 * NWG + h); };   // P_h consumed
   const uint32_t bar_o = bar0 + 8u * (2 * NST + 1 + 4 * NWG);
   constexpr int NR = Cfg::NR;
-  constexpr bool RSEP = NR > 0;          // the records in a ring of their own
+  constexpr bool RSEP = NR > 0;          // the records in a ring of their own (register values)
   constexpr int NRM = RSEP ? NR : 1;     // (slot arithmetic)
   auto bar_rfull = [&](int r) { return bar0 + 8u * (2 * NST + 2 + 4 * NWG + r); };        // landed
   auto bar_rempty = [&](int r) { return bar0 + 8u * (2 * NST + 2 + 4 * NWG + NR + r); };  // read
@@ -311,10 +309,9 @@ __global__ void __launch_bounds__(F32Cfg<KA, MODE>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(bar_full(s), 1);
-      // a stage is released by the MMAs that read it last (the similarity with
-      // a records ring, P.v with tensor-core values), else by the 128 exp
-      // threads that read its records
-      mbar_init(bar_empty(s), (REG && !RSEP) ? 4 * 32 : 1);
+      // a stage is released by the MMAs that read it last: the similarity
+      // (register values) or P.v (tensor-core values)
+      mbar_init(bar_empty(s), 1);
     }
     // a records slot: loaded with its tile's y', released by the 128 exp
     // threads of the warpgroup that summed the tile
@@ -706,7 +703,7 @@ __global__ void __launch_bounds__(F32Cfg<KA, MODE>::THREADS, 1)
             acc2 += lo + hi;
           }
         }
-        mbar_arrive(RSEP ? bar_rempty(t % NRM) : bar_empty(st));
+        mbar_arrive(bar_rempty(t % NRM));   // this thread is done with the records
       } else {
         // the whole S tile into registers; then its TMEM columns may be reused
         uint32_t sv[BN / 32][32];
