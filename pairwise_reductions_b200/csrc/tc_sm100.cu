@@ -60,8 +60,7 @@ namespace {
 
 constexpr int kBM = 128;   // rows per MMA tile
 constexpr int kBN = 128;   // columns per tile
-constexpr int kNT = 2;     // row tiles per CTA
-constexpr int kThreads = 320;
+constexpr int kNT = 2;     // row tiles per CTA (three for one register-summed channel: TcCfg::NT)
 constexpr float kPShift = 14.f;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -87,7 +86,13 @@ template <int KP, int CP, bool GW = false>
 struct TcCfg {
   static constexpr int KC = KP / 64;            // 128-byte swizzle atoms along K
   static constexpr int ATOM = kBM * 128;        // one 128-row x 64-col block: 16 KB
-  static constexpr int X_BYTES = kNT * KC * ATOM;
+  // Row tiles per CTA, one exp warpgroup each.  One register-summed value
+  // channel with rows of at most two atoms: three (S of three tiles fits TMEM,
+  // each y tile serves 384 rows, and a third warp per sub-partition hides more
+  // of the exponent chain's latency); else two.
+  static constexpr int NT = (CP == 1 && KC <= 2) ? 3 : kNT;
+  static constexpr int THREADS = 64 + 128 * NT;
+  static constexpr int X_BYTES = NT * KC * ATOM;
   static constexpr int Y_BYTES = KC * ATOM;
   // One value channel (CP == 1) is summed in registers from an fp32 record per
   // column (512 bytes a tile, padded to keep the stages 1024-byte aligned);
@@ -103,12 +108,12 @@ struct TcCfg {
   // x 128 K in two 64-element atoms, 4 KB).
   static constexpr int P_TILE = kBM * kBN * 2;
   static constexpr int G_TILE = 2 * 16 * 128;
-  static constexpr int PG_BYTES = GW ? kNT * (P_TILE + G_TILE) : 0;
+  static constexpr int PG_BYTES = GW ? NT * (P_TILE + G_TILE) : 0;
   // 200 KB of operand stages; the three-atom rows (D > 126) may take 220 KB
   static constexpr int BUDGET = (KC > 2 || GW ? 220 : 200) * 1024 - PG_BYTES;
   static constexpr int NST_FIT = (BUDGET - X_BYTES) / STAGE;
   static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
-  static constexpr int NBARS = 2 * NST + 11;
+  static constexpr int NBARS = 2 * NST + 2 + 4 * NT;
   static constexpr int SMEM_RAW = 1024 + X_BYTES + NST * STAGE + PG_BYTES + 8 * NBARS + 16;
   // at least ~120 KB so that a second CTA never lands on the SM and blocks on
   // the 512-column TMEM allocation
@@ -129,6 +134,7 @@ struct TcCfg {
   static_assert(!GW || (P_SEPARATE && CP >= 16 && CP <= 48 && KC == 1), "forward + backward sweep");
   static_assert(SMEM_RAW <= 227 * 1024, "shared memory per CTA");
   static_assert(NST >= 2, "shared memory budget");
+  static_assert(NT == kNT || (CP == 1 && !GW), "three row tiles: register values only (TMEM holds S only)");
   static_assert(CP == 1 || (CP % 16 == 0 && CP >= 16 && CP <= 128), "value chunk");
 };
 
@@ -193,7 +199,7 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&v)[32], uint64_t two_
 }
 
 template <int KP, int CP, int DTFMT, bool GW>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(TcCfg<KP, CP, GW>::THREADS, 1)
     tc_gauss_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                     const __grid_constant__ CUtensorMap tmV, const TcKParams p) {
   using Cfg = TcCfg<KP, CP, GW>;
@@ -204,7 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sX = smem;
   uint8_t* sStage = smem + Cfg::X_BYTES;
   uint8_t* sP = sStage + NST * Cfg::STAGE;               // GW: P_0 | P_1 (1024-aligned)
-  uint8_t* sG = sP + kNT * Cfg::P_TILE;                   // GW: g_0 | g_1
+  constexpr int NT = Cfg::NT;
+  uint8_t* sG = sP + NT * Cfg::P_TILE;                    // GW: g_0 | g_1
   uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + NST * Cfg::STAGE + Cfg::PG_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -213,15 +220,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_full = [&](int s) { return bar0 + 8u * s; };
   auto bar_empty = [&](int s) { return bar0 + 8u * (NST + s); };
   const uint32_t bar_x = bar0 + 8u * (2 * NST);
-  auto bar_s = [&](int h) { return bar0 + 8u * (2 * NST + 1 + h); };   // S tile h ready
-  auto bar_p = [&](int h) { return bar0 + 8u * (2 * NST + 3 + h); };   // P tile h written
-  const uint32_t bar_o = bar0 + 8u * (2 * NST + 5);
-  auto bar_f = [&](int h) { return bar0 + 8u * (2 * NST + 7 + h); };   // S tile h read out
-  auto bar_q = [&](int h) { return bar0 + 8u * (2 * NST + 9 + h); };   // P tile h consumed
+  auto bar_s = [&](int h) { return bar0 + 8u * (2 * NST + 1 + h); };            // S tile h ready
+  auto bar_p = [&](int h) { return bar0 + 8u * (2 * NST + 1 + NT + h); };       // P tile h written
+  auto bar_f = [&](int h) { return bar0 + 8u * (2 * NST + 1 + 2 * NT + h); };   // S tile h read out
+  auto bar_q = [&](int h) { return bar0 + 8u * (2 * NST + 1 + 3 * NT + h); };   // P tile h consumed
+  const uint32_t bar_o = bar0 + 8u * (2 * NST + 1 + 4 * NT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t b = blockIdx.z;
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * (kNT * kBM);
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * (NT * kBM);
   const int64_t jbeg = static_cast<int64_t>(blockIdx.y) * p.cols_per_split;
   const int64_t jend = min(p.N, jbeg + p.cols_per_split);
   const int T = (jend > jbeg) ? static_cast<int>((jend - jbeg + kBN - 1) / kBN) : 0;
@@ -232,18 +239,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(bar_full(s), 1);
-      mbar_init(bar_empty(s), Cfg::REG ? 8 : 1);   // register values: the 8 exp warps release it
+      mbar_init(bar_empty(s), Cfg::REG ? 4 * NT : 1);   // register values: the exp warps release it
     }
     mbar_init(bar_x, 1);
-    mbar_init(bar_s(0), 1);
-    mbar_init(bar_s(1), 1);
-    mbar_init(bar_p(0), 4 * 32);
-    mbar_init(bar_p(1), 4 * 32);
+    for (int h = 0; h < NT; ++h) {
+      mbar_init(bar_s(h), 1);
+      mbar_init(bar_p(h), 4 * 32);
+      mbar_init(bar_f(h), 4 * 32);
+      mbar_init(bar_q(h), 1);
+    }
     mbar_init(bar_o, 1);
-    mbar_init(bar_f(0), 4 * 32);
-    mbar_init(bar_f(1), 4 * 32);
-    mbar_init(bar_q(0), 1);
-    mbar_init(bar_q(1), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -268,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmY);
       tma_prefetch_desc(&tmV);
       mbar_arrive_expect_tx(bar_x, Cfg::X_BYTES);
-      for (int h = 0; h < kNT; ++h)
+      for (int h = 0; h < NT; ++h)
         for (int kc = 0; kc < Cfg::KC; ++kc)
           tma_load_3d(smem_u32(sX + (h * Cfg::KC + kc) * Cfg::ATOM), &tmX, bar_x, kc * 64,
                       static_cast<int>(row0 + h * kBM), static_cast<int>(b));
@@ -338,10 +343,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = wait_bar(bar_full(0), 0, abort_flag, wlim);
         if (ok) {
           tc_fence_after();
-          issue_S(0, 0);
-          mma_commit(bar_s(0));
-          issue_S(1, 0);
-          mma_commit(bar_s(1));
+          for (int h = 0; h < NT; ++h) {
+            issue_S(h, 0);
+            mma_commit(bar_s(h));
+          }
         }
       }
       for (int t = 0; ok && t < T; ++t) {
@@ -351,15 +356,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           // register values: only the similarity MMAs; S_h(t+1) once warpgroup h
           // has read S_h(t) (the exp warps release the stages themselves)
           if (t + 1 < T) {
-            if (!(ok = wait_bar(bar_f(0), t & 1, abort_flag, wlim))) break;
             if (!(ok = wait_bar(bar_full(st1), ((t + 1) / NST) & 1, abort_flag, wlim))) break;
-            tc_fence_after();
-            issue_S(0, st1);
-            mma_commit(bar_s(0));
-            if (!(ok = wait_bar(bar_f(1), t & 1, abort_flag, wlim))) break;
-            tc_fence_after();
-            issue_S(1, st1);
-            mma_commit(bar_s(1));
+            for (int h = 0; ok && h < NT; ++h) {
+              if (!(ok = wait_bar(bar_f(h), t & 1, abort_flag, wlim))) break;
+              tc_fence_after();
+              issue_S(h, st1);
+              mma_commit(bar_s(h));
+            }
+            if (!ok) break;
           }
         } else if constexpr (Cfg::P_SEPARATE) {
           // S_h(t+1) may overwrite S_h as soon as warpgroup h has read S_h(t)
@@ -432,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float row_sum = 0.f;   // register values: the row's sum over the tiles
     // Forward + backward sweep.  TMEM lane `row` of Gw_h is column j0 + row of
     // the tile; row tile rt of the matrix.
-    const int64_t rt = static_cast<int64_t>(blockIdx.x) * kNT + h;
+    const int64_t rt = static_cast<int64_t>(blockIdx.x) * NT + h;
     uint8_t* const sPh = sP + h * Cfg::P_TILE;
     if constexpr (GW) {
       // this row's (g hi, g lo) as column `row` of g_h: rows 0 and 1 of the
@@ -881,8 +885,9 @@ cudaError_t launch_kernel(const CUtensorMap& tx, const CUtensorMap& ty, const CU
     attr_done = true;
   }
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(kThreads);
+  // row blocks of Cfg::NT row tiles
+  cfg.gridDim = dim3(static_cast<unsigned>((kp.M + Cfg::NT * kBM - 1) / (Cfg::NT * kBM)), grid.y, grid.z);
+  cfg.blockDim = dim3(Cfg::THREADS);
   cfg.dynamicSmemBytes = Cfg::SMEM;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -1011,6 +1016,7 @@ cudaError_t launch_tc_sum(const TcArgs& a, cudaStream_t s) {
       !make_tmap_3d(&ty, tdt, a.ypack, KP, a.N, a.B, KP * 2ull, a.N * KP * 2ull, 64, kBN))
     return cudaErrorInvalidValue;
   const int64_t Nst = (a.N + 7) / 8 * 8;
+  // (launch_kernel sets the row-block count from the instantiation's row tiles per CTA)
   const dim3 grid(static_cast<unsigned>((a.M + kNT * kBM - 1) / (kNT * kBM)),
                   static_cast<unsigned>(a.plan.splits), static_cast<unsigned>(a.B));
   const int chunk = tc_max_chunk(KP);
