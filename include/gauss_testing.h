@@ -52,6 +52,33 @@ gs_status gs_test_set_waits(uint64_t limit_ns, int stall);
  */
 gs_status gs_test_read_error_word(int *word, gs_stream_t stream);
 
+/*
+ * Measurement probe: the MUFU ex2 rate of an SM.  Launches `blocks` CTAs of
+ * 1024 threads, one per SM (each holds 120 KB of shared memory); every thread
+ * runs 8 independent chains v <- 2^(-v/2) for `iters` steps (8 * iters ex2 a
+ * thread), and cycles[b] receives the SM cycles of CTA b's loop, so that
+ * 1024 * 8 * iters / cycles[b] is the SM's ex2 results per clock.  cycles: device
+ * array of `blocks` int64; sink: device array of blocks * 1024 floats (keeps the
+ * results live).  blocks in [1, 4096], iters in [1, 2^20], else
+ * GS_ERR_INVALID_ARG (checked before anything is launched).  Asynchronous on
+ * `stream`.
+ */
+gs_status gs_test_ex2_probe(long long *cycles, float *sink, int blocks, int iters, gs_stream_t stream);
+
+/*
+ * Measurement probe: the cost of back-to-back tcgen05.mma instructions issued by
+ * one thread.  Launches `blocks` CTAs of 128 threads, one per SM; in each, one
+ * thread issues n_mma MMAs of M = 128, N = n_cols, K = 16 (kind::f16, zero
+ * operands in shared memory, one TMEM accumulator), commits them and waits
+ * (bounded: 2 s) for their completion; cycles[b] = the SM cycles from the first
+ * issue to the completion (-1, and *status |= 1, if the wait ran out).  cycles:
+ * device array of `blocks` int64; status: device int, zeroed by the caller.
+ * blocks in [1, 4096], n_mma in [1, 65536], n_cols in {32, 64, 128, 256}, else
+ * GS_ERR_INVALID_ARG (checked before anything is launched).  Asynchronous.
+ */
+gs_status gs_test_mma_probe(long long *cycles, int *status, int blocks, int n_mma, int n_cols,
+                            gs_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -63,6 +63,8 @@ SIGNATURES = {
     "gs_test_exp2_poly": (ctypes.c_int, [_vp, _vp, _i64, ctypes.c_int, _vp]),
     "gs_test_set_waits": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_int]),
     "gs_test_read_error_word": (ctypes.c_int, [_vp, _vp]),
+    "gs_test_ex2_probe": (ctypes.c_int, [_vp, _vp, ctypes.c_int, ctypes.c_int, _vp]),
+    "gs_test_mma_probe": (ctypes.c_int, [_vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp]),
     "gauss_sum_fwd_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _f,
                                              ctypes.c_int, _vp]),
 }
@@ -406,6 +408,28 @@ def test_read_error_word(stream=None):
     _check("gs_test_read_error_word", _lib.gs_test_read_error_word(ctypes.byref(word),
                                                                    _stream(stream)))
     return word.value
+
+
+def test_ex2_probe(blocks, iters, stream=None):
+    """SM cycles of each CTA of the MUFU ex2 rate probe (test hook, see
+    include/gauss_testing.h): CTA b evaluated 1024 * 8 * iters exponentials."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cycles = torch.zeros(int(blocks), dtype=torch.int64, device=dev)
+    sink = torch.empty(int(blocks) * 1024, dtype=torch.float32, device=dev)
+    _check("gs_test_ex2_probe", _lib.gs_test_ex2_probe(_ptr(cycles), _ptr(sink), int(blocks),
+                                                       int(iters), _stream(stream)))
+    return cycles
+
+
+def test_mma_probe(blocks, n_mma, n_cols, stream=None):
+    """SM cycles of each CTA of the tcgen05.mma issue probe (test hook, see
+    include/gauss_testing.h), and the status word (0: every wait completed)."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cycles = torch.zeros(int(blocks), dtype=torch.int64, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    _check("gs_test_mma_probe", _lib.gs_test_mma_probe(_ptr(cycles), _ptr(status), int(blocks),
+                                                       int(n_mma), int(n_cols), _stream(stream)))
+    return cycles, status
 
 
 def last_device_error(stream=None):

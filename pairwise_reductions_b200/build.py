@@ -18,7 +18,7 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libgauss_b200.so")
 SOURCES = ["api.cpp", "small_d.cu", "tc_sm100.cu", "tc_f32_sm100.cu", "grad.cu", "knn.cu",
-           "noalloc.cu"]
+           "noalloc.cu", "probes.cu"]
 HEADERS = ["internal.h", "ptx.cuh", "exp2_poly.cuh", "values.cuh", "combine.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -230,3 +230,10 @@ def test_testing_hooks_reject_bad_arguments_without_a_device_call():
     assert lib.gs_test_set_waits(1_000_000, 3) == 1
     assert lib.gs_test_set_waits(1_000_000, -1) == 1
     assert lib.gs_test_read_error_word(NULL, NULL) == 1
+    # the measurement probes check their arguments before anything is launched
+    assert lib.gs_test_ex2_probe(NULL, NULL, 1, 1, NULL) == 1
+    assert lib.gs_test_ex2_probe(FAKE, FAKE, 0, 1, NULL) == 1
+    assert lib.gs_test_ex2_probe(FAKE, FAKE, 1, 0, NULL) == 1
+    assert lib.gs_test_mma_probe(FAKE, FAKE, 1, 64, 48, NULL) == 1
+    assert lib.gs_test_mma_probe(FAKE, FAKE, 1, 0, 64, NULL) == 1
+    assert lib.gs_test_mma_probe(NULL, FAKE, 1, 64, 64, NULL) == 1
