@@ -128,11 +128,11 @@ struct F32Cfg {
   static constexpr int BUDGET = 214 * 1024;
   // TMEM columns of the accumulators: one S per warpgroup (every small
   // product first, while the sum is small, then the large ones: each addition
-  // is rounded against the magnitude of what it adds to); tensor-core values
-  // add P hi/lo (fp16 pairs: bn / 2 columns each) and O per warpgroup, O as
-  // two halves of CP columns: O_big (P_hi v_hi + P_lo v_hi) and O_small
-  // (P_hi v_lo), added in the epilogue.
-  static constexpr int tmem_acc(int bn) { return REG ? NWG * bn : 4 * bn + 4 * CPA; }
+  // is rounded against the magnitude of what it adds to); with tensor-core
+  // values P (fp16 hi/lo pairs) is written over its own S columns, and each
+  // warpgroup has an O of two halves of CP columns: O_big (P_hi v_hi + P_lo
+  // v_hi) and O_small (P_hi v_lo), added in the epilogue.
+  static constexpr int tmem_acc(int bn) { return REG ? NWG * bn : 2 * bn + 4 * CPA; }
   // The x' rows (2 K' <= 32 KA columns) sit in TMEM as the A operand of the
   // similarity MMAs when the accumulators leave room, else in shared memory.
   static constexpr bool xt(int bn) { return tmem_acc(bn) + 32 * KA <= 512; }
@@ -141,12 +141,11 @@ struct F32Cfg {
     return tmem_acc(bn) <= 512 &&
            (BUDGET - x_bytes(bn) - rec_bytes(bn) - ORUN_BYTES) / stage_bytes(bn) >= 2;
   }
-  // Column tile.  An M = 128, K = 16 MMA costs much the same at N = 32 and 64
-  // and a third more at 128 (measured on B200: 47, 49 and 65 issue cycles), so
-  // the widest tile that fits is the cheapest per pair; three register channels
-  // use 32 columns (registers).
-  static constexpr int BN =
-      MODE == 3 ? 32 : ((MODE == 1 && fits(128)) ? 128 : (fits(64) ? 64 : 32));
+  // Column tile.  An M = 128, K = 16 MMA costs the same at N = 32 and 64 and a
+  // sixth more at 128 (measured on B200: 55.6, 55.6 and 64.9 cycles), and a
+  // tile's commits are paid once, so the widest tile that fits is the cheapest
+  // per pair; three register channels use 32 columns (registers).
+  static constexpr int BN = MODE == 3 ? 32 : (fits(128) ? 128 : (fits(64) ? 64 : 32));
   static constexpr bool XT = xt(BN);
   static constexpr int X_BYTES = x_bytes(BN);
   static constexpr int QW_BYTES = qw_bytes(BN);
@@ -164,20 +163,23 @@ struct F32Cfg {
       1024 + X_BYTES + NST * STAGE + REC_BYTES + ORUN_BYTES + 8 * NBARS + 16 + RED_BYTES;
   // at least ~120 KB: one CTA per SM, so the 512-column TMEM allocation never waits
   static constexpr int SMEM = SMEM_RAW < 122880 ? 122880 : SMEM_RAW;
-  // TMEM columns.  Register values: S0 | S1 | x'.
-  // Tensor-core values: S0 | S1 | Phi0 | Phi1 | Plo0 | Plo1 | O0 | O1 | x', O_h as
-  // [O_big (CP) | O_small (CP)] in 2 CPA columns.
+  // TMEM columns.  Register values: S0 | S1 | S2 | x'.  Tensor-core values:
+  // S0 | S1 | O0 | O1 | x', O_h as [O_big (CP) | O_small (CP)] in 2 CPA columns;
+  // P_h over S_h: the 32-column chunk c of S holds, once read, the fp16 pairs of
+  // its P_hi in columns [32 c, 32 c + 16) and of its P_lo in [32 c + 16, 32 c + 32).
   __host__ __device__ static constexpr uint32_t col_s(int h) { return h * BN; }
-  __host__ __device__ static constexpr uint32_t col_phi(int h) { return 2 * BN + (BN / 2) * h; }
-  __host__ __device__ static constexpr uint32_t col_plo(int h) { return 3 * BN + (BN / 2) * h; }
-  __host__ __device__ static constexpr uint32_t col_o(int h) { return 4 * BN + 2 * CPA * h; }
+  // P_hi of K step ks (16 S columns; its P_lo 16 columns on)
+  __host__ __device__ static constexpr uint32_t col_p(int h, int ks) {
+    return h * BN + (ks >> 1) * 32 + (ks & 1) * 8;
+  }
+  __host__ __device__ static constexpr uint32_t col_o(int h) { return 2 * BN + 2 * CPA * h; }
   static constexpr uint32_t COL_X = tmem_acc(BN);
   static_assert(NST >= 2, "shared memory budget");
   static_assert(tmem_acc(BN) + (XT ? 32 * KA : 0) <= 512, "TMEM budget");
   static_assert(REG || (CP % 16 == 0 && CP >= 16 && CP <= 64), "value chunk");
-  // P_hi [v_hi ; v_lo] reads the hi and lo value atoms as one operand of 2 CP
-  // rows: they must be adjacent, one atom each (tiles of at most 64 columns)
-  static_assert(REG || VA == 1, "value atoms of a stage");
+  // P_hi [v_hi ; v_lo] reads the hi and lo value atoms of 64 columns as one
+  // operand of 2 CP rows: a stage keeps them adjacent, atom a's hi then lo
+  static_assert(REG || (VA >= 1 && BN == 64 * VA), "value atoms of a stage");
   static_assert(SMEM_RAW <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -377,7 +379,7 @@ __global__ void __launch_bounds__(F32Cfg<KA, MODE>::THREADS, 1)
         if constexpr (!REG) {
           for (int hl = 0; hl < 2; ++hl)
             for (int a = 0; a < Cfg::VA; ++a)
-              tma_load_3d(smem_u32(sv + (hl * Cfg::VA + a) * Cfg::V_ATOM), &tmV, bar_full(st),
+              tma_load_3d(smem_u32(sv + (2 * a + hl) * Cfg::V_ATOM), &tmV, bar_full(st),
                           j0 + a * 64, 0, static_cast<int>(hl * p.Bsz + b));
         }
         issued = t + 1;
@@ -458,11 +460,12 @@ __global__ void __launch_bounds__(F32Cfg<KA, MODE>::THREADS, 1)
         const uint32_t d = tmem + Cfg::col_o(h);
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks) {   // K steps of 16 columns
-          const int within = ks * 32;
-          // rows 0 .. CP-1 the hi atom, CP .. 2 CP-1 the lo atom right after it
-          const uint64_t bhl = desc_advance(sv, static_cast<uint32_t>(within));
-          const uint32_t phi = tmem + Cfg::col_phi(h) + ks * 8;
-          const uint32_t plo = tmem + Cfg::col_plo(h) + ks * 8;
+          // atom ks / 4: rows 0 .. CP-1 the hi atom, CP .. 2 CP-1 the lo atom
+          // right after it; 32 bytes a K step within the atom
+          const uint64_t bhl = desc_advance(
+              sv, static_cast<uint32_t>((ks >> 2) * 2 * Cfg::V_ATOM + (ks & 3) * 32));
+          const uint32_t phi = tmem + Cfg::col_p(h, ks);
+          const uint32_t plo = phi + 16;
           mma_ts(d, phi, bhl, idO2, (acc_prev || ks > 0) ? 1u : 0u);
           mma_ts(d, plo, bhl, idO, 1u);
         }
@@ -478,13 +481,13 @@ __global__ void __launch_bounds__(F32Cfg<KA, MODE>::THREADS, 1)
           if constexpr (RSEP) mma_commit(bar_empty(h % NST));
         }
       }
-      // S_h(t + NWG) may overwrite S_h once warpgroup h has read S_h(t).  With
-      // tensor-core values (two warpgroups) it goes ahead of O_h(t) when tile
-      // t + 2 does not need the stage of tile t (three or more stages), else
-      // after it.
-      constexpr bool kSFirst = REG || NST >= 3;
+      // Register values: S_h(t + NWG) may overwrite S_h once warpgroup h has
+      // read S_h(t).  Tensor-core values: P_h(t) lives in S_h's columns, so
+      // S_h(t + 2) follows O_h(t), the MMA that reads it (the tensor core runs
+      // one thread's MMAs in order).
+      constexpr bool kSFirst = REG;
       auto next_S = [&](int h, int k, int t2) {
-        if (!wait_bar(bar_f(h), k & 1, abort_flag, wlim)) return false;
+        if (REG && !wait_bar(bar_f(h), k & 1, abort_flag, wlim)) return false;
         if (!wait_bar(bar_full(t2 % NST), (t2 / NST) & 1, abort_flag, wlim)) return false;
         tc_fence_after();
         issue_S(h, t2 % NST);
@@ -520,8 +523,6 @@ __global__ void __launch_bounds__(F32Cfg<KA, MODE>::THREADS, 1)
     const bool valid = i < p.M;
     const float r = valid ? p.rnorm[b * p.M + i] : 0.f;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tPh = tmem + lane_base + Cfg::col_phi(h);
-    const uint32_t tPl = tmem + lane_base + Cfg::col_plo(h);
     // the exponent's constant, with the split rows' scale 2^(2e) undone
     const float two_c =
         SPLIT ? p.two_c * pow2_int(-split_exp(p.amax[b])) * pow2_int(-split_exp(p.amax[b])) : p.two_c;
@@ -705,17 +706,15 @@ __global__ void __launch_bounds__(F32Cfg<KA, MODE>::THREADS, 1)
         }
         mbar_arrive(bar_rempty(t % NRM));   // this thread is done with the records
       } else {
-        // the whole S tile into registers; then its TMEM columns may be reused
-        uint32_t sv[BN / 32][32];
-#pragma unroll
-        for (int ch = 0; ch < BN / 32; ++ch) tmem_ld32(tS + ch * 32, sv[ch]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int ch = 0; ch < BN / 32; ++ch) reg_fence32(sv[ch]);
-        tc_fence_before();
-        mbar_arrive(bar_f(h));
+        // S chunk by chunk, 32 columns: each chunk's P goes over the chunk's
+        // own S columns once they are read.  (S_h(t) was written after O_h(t-2)
+        // had read P_h(t-2) from these columns: the MMAs run in order.)
 #pragma unroll
         for (int ch = 0; ch < BN / 32; ++ch) {
+          uint32_t sv[32];
+          tmem_ld32(tS + ch * 32, sv);
+          tmem_wait_ld();
+          reg_fence32(sv);
           // P 2^14 in fp16 hi + lo parts, two columns per 32-bit TMEM word:
           // every P keeps an absolute error under 2^-39 (relative 2^-22 from
           // P = 2^-3 up)
@@ -724,7 +723,7 @@ __global__ void __launch_bounds__(F32Cfg<KA, MODE>::THREADS, 1)
           for (int e = 0; e < 16; ++e) {
             const int c = ch * 32 + 2 * e;
             float t0, t1;
-            upk2(add2(fma2(pk2(__uint_as_float(sv[ch][2 * e]), __uint_as_float(sv[ch][2 * e + 1])),
+            upk2(add2(fma2(pk2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
                            two_c2, r2),
                       *reinterpret_cast<const uint64_t*>(qrec + c)),
                  t0, t1);
@@ -735,17 +734,9 @@ __global__ void __launch_bounds__(F32Cfg<KA, MODE>::THREADS, 1)
             hi[e] = *reinterpret_cast<const uint32_t*>(&h2);
             lo[e] = *reinterpret_cast<const uint32_t*>(&l2);
           }
-          if (ch == 0 && k > 0) {
-            // P_h(previous tile) must have been read by its P.v MMAs
-            // (waited for as late as possible)
-            ok = __all_sync(0xffffffffu, wait_bar(bar_q(h), (k - 1) & 1, abort_flag, wlim));
-            if (!ok) break;
-            tc_fence_after();
-          }
-          tmem_st16(tPh + ch * 16, hi);
-          tmem_st16(tPl + ch * 16, lo);
+          tmem_st16(tS + ch * 32, hi);
+          tmem_st16(tS + ch * 32 + 16, lo);
         }
-        if (!ok) break;
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar_p(h));
