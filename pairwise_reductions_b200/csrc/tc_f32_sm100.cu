@@ -290,7 +290,8 @@ __global__ void __launch_bounds__(F32Cfg<KA, MODE>::THREADS, 1)
   auto bar_s = [&](int h) { return bar0 + 8u * (2 * NST + 1 + h); };             // S_h ready
   auto bar_f = [&](int h) { return bar0 + 8u * (2 * NST + 1 + NWG + h); };       // S_h read out
   auto bar_p = [&](int h) { return bar0 + 8u * (2 * NST + 1 + 2 * NWG + h); };   // P_h written
-  auto bar_q = [&](int h) { return bar0 + 8u * (2 * NST + 1 + 3 * NWG + h); };   // P_h consumed
+  // O_h complete after the last tile of a group of kOGroup (tensor-core values)
+  auto bar_q = [&](int h) { return bar0 + 8u * (2 * NST + 1 + 3 * NWG + h); };
   const uint32_t bar_o = bar0 + 8u * (2 * NST + 1 + 4 * NWG);
   constexpr int NR = Cfg::NR;
   constexpr bool RSEP = NR > 0;          // the records in a ring of their own (register values)
@@ -505,7 +506,7 @@ __global__ void __launch_bounds__(F32Cfg<KA, MODE>::THREADS, 1)
             if (!(ok = wait_bar(bar_p(h), k & 1, abort_flag, wlim))) break;
             tc_fence_after();
             issue_O(h, t % NST, k % kOGroup != 0);
-            mma_commit(bar_q(h));
+            if ((k + 1) % kOGroup == 0) mma_commit(bar_q(h));   // (the group's drain waits on it)
             mma_commit(bar_empty(t % NST));
             if (!kSFirst && t2 < T && !(ok = next_S(h, k, t2))) break;
           }
@@ -587,8 +588,9 @@ __global__ void __launch_bounds__(F32Cfg<KA, MODE>::THREADS, 1)
       if constexpr (!REG) {
         if (k > 0 && k % kOGroup == 0) {
           // O_h has summed kOGroup tiles: once their P.v MMAs are done, into the
-          // registers; tile k's P.v MMAs then start O_h afresh
-          ok = __all_sync(0xffffffffu, wait_bar(bar_q(h), (k - 1) & 1, abort_flag, wlim));
+          // fp32 sums in shared memory; tile k's P.v MMAs then start O_h afresh
+          ok = __all_sync(0xffffffffu,
+                          wait_bar(bar_q(h), ((k / kOGroup) - 1) & 1, abort_flag, wlim));
           if (!ok) break;
           tc_fence_after();
           add_o();
