@@ -242,8 +242,8 @@ constexpr float kPScale = 16384.f;
 // (B = 4, N = 65536, 32 channels); 16 tiles (64 additions) keep it near 2e-6.
 constexpr int kOGroup = 16;
 
-// Named barrier of the two exp warpgroups (warps 2-9).
-// every exp warp of the CTA (nthreads = 128 per warpgroup)
+// Named barrier of every exp warp of the CTA (warps 2.., nthreads = 128 per
+// exp warpgroup).
 __device__ __forceinline__ void exp_warps_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }

@@ -14,11 +14,12 @@
 // is one FFMA and one MUFU ex2; the +14 (undone on output) keeps P in the
 // normal fp16 range down to kernel values of 2^-28.
 //
-// CTA = 256 rows (two 128-row MMA tiles) x one column split, 10 warps:
+// CTA = 256 rows (two 128-row MMA tiles) x one column split, 10 warps (one
+// register-summed channel: 384 rows, three row tiles, 14 warps):
 //   warp 0      TMA producer: x~ tiles once, then a ring of (y~, v^T) stages
 //   warp 1      TMEM owner + single-thread MMA issuer
 //   warps 2-5   exp warpgroup of row tile 0 (TMEM lane quarters 2,3,0,1)
-//   warps 6-9   exp warpgroup of row tile 1
+//   warps 6-9   exp warpgroup of row tile 1 (warps 10-13: row tile 2)
 // Per 128-column tile t and row tile h:
 //   S_h = x~_h . y~(t)^T        (tcgen05.mma, smem x smem -> TMEM fp32)
 //   P_h = ex2(fma(S_h, 2c, r))  (tcgen05.ld -> MUFU -> fp16 -> tcgen05.st)
